@@ -1,0 +1,415 @@
+"""CPU oracle for the AutoRound tuning step, INT4 packing and the W4A16 matmul.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
+the CUDA library and imports nothing from it; the two meet only through the
+seeded inputs of ``synth``.
+
+It is plain and slow on purpose: each function takes the method's steps in the
+order and notation of the pages, with numpy doing element-wise IEEE operations
+and fp64 matrix products.  Sources (page title, then section):
+
+* [AR] "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
+  Architectural Optimizations of AutoRound" (English write-up of the talk).
+  §2 "Minimal Example" (the [0.1, 0.2, 0.15, 8.0] vector), §3 "Optimization
+  Variables" table (v, min, max; shapes, ranges, initial values), §3
+  "Algorithm Flow" (steps 2-5), §3 "SignSGD" update rule, §3 "Minimal
+  State-Evolution Example" (3.3 rounds up once v passes 0.2), §4 "Minimal
+  State Evolution" table (w = 0.37, scale 0.05, zero 8).
+* [QC] "量化：从 Scale 到 W4A8 的完整坐标", §1.2 (symmetric mapping
+  q = clip(round(x/s)), x̂ = s·q; asymmetric adds a zero-point).
+* [IA] "Intel AutoRound 高级量化" (hotdry blog), section on the sign-gradient
+  mechanism: rounding is treated as the identity in the backward pass (STE).
+
+Readings where the pages are silent or disagree (all stated once more in
+the design doc):
+
+* The group range always contains 0: mx = max(0, max W), mn = min(0, min W).
+  [AR] §2 needs this: "no clipping" on [0.1, 0.2, 0.15, 8.0] gives scale 8/15.
+* Rounding is half away from zero ([AR] §2: 0.1/0.04 = 2.5 must become 3 to
+  give 0.12).
+* Clip bounds are multiplicative: hi = alpha·mx, lo = beta·mn with
+  alpha, beta in [0.5, 1], init 1 ([AR] §3 table gives min/max per group
+  initialised to the group's range; the parameterisation is the task's).
+* q = clamp(round(W/s + V) + zp, 0, 2^b - 1), zp = round(-lo/s),
+  s = (hi - lo)/(2^b - 1), guarded below at 1e-8.
+* STE: both roundings have derivative 1; clamp passes the gradient where
+  0 <= round(W/s+V)+zp <= 2^b-1 (inclusive).
+* Loss = mean squared error over all M·N outputs; dL/dŶ = 2R/(M·N).
+* Update p <- clamp(p - lr·sign(dp)) with sign(0) = 0 (descent; the page's
+  formula prints the step without its minus sign).
+* Precision points shared with the GPU path: X, W are bf16; the QDQ runs in
+  fp32 (it decides integer codes, so both sides decide in the kernel's
+  precision); Ŵ is rounded to bf16; products accumulate in fp64 here (fp32 on
+  the GPU) and are rounded to fp32; G is rounded to bf16.
+* Symmetric mode: s = max(hi, -lo)/(2^(b-1) - 1), zp = 2^(b-1) fixed, codes in
+  [0, 2^b - 1]; ds flows to whichever of hi, -lo is larger (ties to hi).
+* INT4 layout: row-major [N][K/8] uint32, element k at bits 4·(k mod 8);
+  scale and zero as fp16 (round to nearest even).  The pages give no layout.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+f32 = np.float32
+f64 = np.float64
+
+S_GUARD = 1e-8  # lower bound on the scale; never reached by the workloads
+
+
+# ----------------------------------------------------------------------------
+# rounding helpers (IEEE definitions written out)
+# ----------------------------------------------------------------------------
+
+def bf16_rne(x) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even); returns float32.
+
+    bfloat16 keeps the top 16 bits of the float32 encoding.  Round to nearest
+    even adds 0x7FFF plus the lowest kept bit before truncating.  NaN stays NaN.
+    """
+    x = np.asarray(x, dtype=f32)
+    b = x.view(np.uint32).astype(np.uint64)
+    keep_lsb = (b >> 16) & 1
+    r = ((b + 0x7FFF + keep_lsb) >> 16).astype(np.uint32) << np.uint32(16)
+    out = r.view(f32).reshape(x.shape)
+    return np.where(np.isnan(x), x, out).astype(f32)
+
+
+def round_half_away(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest integer, halves away from zero, in the array's own dtype.
+
+    r = trunc(x); x - r is exact, so the half test decides exactly.
+    """
+    x = np.asarray(x)
+    r = np.trunc(x)
+    frac = x - r
+    step = np.where(np.abs(frac) >= x.dtype.type(0.5), np.sign(x), x.dtype.type(0))
+    return (r + step).astype(x.dtype)
+
+
+def round_identity(x: np.ndarray) -> np.ndarray:
+    """'Rounding' that does nothing: the smooth surrogate used to check STE gradients by finite differences."""
+    return np.asarray(x)
+
+
+def sign0(x: np.ndarray) -> np.ndarray:
+    """sign with sign(0) = 0 and sign(NaN) = 0."""
+    s = np.sign(x)
+    return np.where(np.isnan(s), 0, s).astype(x.dtype)
+
+
+# ----------------------------------------------------------------------------
+# the quantizer ([AR] §2, §3 table, §4 table; [QC] §1.2)
+# ----------------------------------------------------------------------------
+
+def group_range(W: np.ndarray, g: int):
+    """Per-group range including zero: mx = max(0, max_k W), mn = min(0, min_k W).
+
+    ``W`` is [N][K]; groups are ``g`` consecutive entries along K.
+    """
+    N, K = W.shape
+    assert K % g == 0
+    Wg = W.reshape(N, K // g, g)
+    mx = np.maximum(Wg.max(axis=-1), 0).astype(W.dtype)
+    mn = np.minimum(Wg.min(axis=-1), 0).astype(W.dtype)
+    return mx, mn
+
+
+def qparams(mx, mn, alpha, beta, bits: int, symmetric: bool = False, dtype=f32, rnd=round_half_away):
+    """Scale and zero-point of each group from the learnable clip factors.
+
+    Asymmetric: hi = alpha·mx, lo = beta·mn, s = (hi - lo)/(2^b - 1),
+    zp = round(-lo/s).  Symmetric: s = max(hi, -lo)/(2^(b-1) - 1), zp = 2^(b-1).
+    Returns (hi, lo, s, zp, guarded).
+    """
+    T = dtype
+    mx, mn, alpha, beta = (np.asarray(a, dtype=T) for a in (mx, mn, alpha, beta))
+    hi = (alpha * mx).astype(T)
+    lo = (beta * mn).astype(T)
+    if not symmetric:
+        Q = T(2 ** bits - 1)
+        s = ((hi - lo) / Q).astype(T)
+    else:
+        Qs = T(2 ** (bits - 1) - 1)
+        s = (np.maximum(hi, -lo) / Qs).astype(T)
+    guarded = s < T(S_GUARD)
+    s = np.where(guarded, T(S_GUARD), s).astype(T)
+    if not symmetric:
+        zp = rnd((-lo / s).astype(T)).astype(T)
+    else:
+        zp = np.full_like(s, T(2 ** (bits - 1)))
+    return hi, lo, s, zp, guarded
+
+
+def quantize(W, V, s, zp, bits: int, dtype=f32, rnd=round_half_away):
+    """Codes and dequantized weights for given per-element offsets and per-group (s, zp).
+
+    q = clamp(round(W/s + V) + zp, 0, 2^b - 1);  Ŵ = s·(q - zp).
+    ``W, V`` are [N][K]; ``s, zp`` are [N][G].  Returns dict with the
+    intermediate ``wq = W/s``, the unclamped integer ``t``, the in-range mask
+    ``m``, the codes ``q`` and ``What`` (not yet rounded to bf16).
+    """
+    T = dtype
+    N, K = W.shape
+    G = s.shape[1]
+    g = K // G
+    Wg = np.asarray(W, T).reshape(N, G, g)
+    Vg = np.asarray(V, T).reshape(N, G, g)
+    s3 = np.asarray(s, T)[:, :, None]
+    z3 = np.asarray(zp, T)[:, :, None]
+    Q = T(2 ** bits - 1)
+    wq = (Wg / s3).astype(T)
+    u = (wq + Vg).astype(T)
+    r = rnd(u).astype(T)
+    t = (r + z3).astype(T)
+    m = (t >= 0) & (t <= Q)
+    q = np.clip(t, T(0), Q).astype(T)
+    what = (s3 * (q - z3)).astype(T)
+    return {
+        "wq": wq.reshape(N, K),
+        "t": t.reshape(N, K),
+        "m": m.reshape(N, K),
+        "q": q.reshape(N, K),
+        "What": what.reshape(N, K),
+    }
+
+
+def qdq(W, V, alpha, beta, bits: int, group_size: int, symmetric: bool = False, dtype=f32, rnd=round_half_away):
+    """The fake-quant (QDQ) forward of one weight matrix ([AR] §4 'QDQ / Fake Quantization').
+
+    Returns every per-group and per-element quantity the backward needs, plus
+    ``What_bf16`` (Ŵ rounded to bf16, the operand of the tuning GEMMs; only in
+    the fp32 instantiation).
+    """
+    T = dtype
+    W = np.asarray(W, T)
+    mx, mn = group_range(W, group_size)
+    hi, lo, s, zp, guarded = qparams(mx, mn, alpha, beta, bits, symmetric, T, rnd)
+    qd = quantize(W, V, s, zp, bits, T, rnd)
+    out = dict(qd)
+    out.update(mx=mx, mn=mn, hi=hi, lo=lo, s=s, zp=zp, guarded=guarded)
+    if T is f32:
+        out["What_bf16"] = bf16_rne(qd["What"])
+    return out
+
+
+# ----------------------------------------------------------------------------
+# forward, loss and gradients ([AR] §3 'Algorithm Flow' steps 2-4)
+# ----------------------------------------------------------------------------
+
+def reference_forward(Xb, Wb) -> np.ndarray:
+    """Y = X·Wᵀ with the original (bf16) weights, fp64 accumulation, rounded to fp32."""
+    return (np.asarray(Xb, f64) @ np.asarray(Wb, f64).T).astype(f32)
+
+
+def forward_loss(Xb, What_b, Y, count: int, *, round_g_bf16: bool = True, dtype=f32):
+    """QDQ forward and MSE: Ŷ = X·Ŵᵀ, R = Ŷ - Y, L = ΣR²/count, G = dL/dŶ = 2R/count.
+
+    ``count`` is M·N of the whole layer (a row subset passes the full count).
+    In the fp32 instantiation Ŷ and R are fp32 and G is rounded to bf16, the
+    rounding points the GPU path shares; the fp64 instantiation keeps fp64.
+    """
+    if dtype is f32:
+        Yhat = (np.asarray(Xb, f64) @ np.asarray(What_b, f64).T).astype(f32)
+        R = (Yhat - np.asarray(Y, f32)).astype(f32)
+        gscale = f32(2.0 / float(count))
+        G = (R * gscale).astype(f32)
+        if round_g_bf16:
+            G = bf16_rne(G)
+        L = float(np.sum(R.astype(f64) ** 2) / count)
+        return {"Yhat": Yhat, "R": R, "G": G, "loss": L}
+    Yhat = np.asarray(Xb, f64) @ np.asarray(What_b, f64).T
+    R = Yhat - np.asarray(Y, f64)
+    G = 2.0 * R / float(count)
+    L = float(np.sum(R ** 2) / count)
+    return {"Yhat": Yhat, "R": R, "G": G, "loss": L}
+
+
+def weight_grad(G, Xb, dtype=f32) -> np.ndarray:
+    """dL/dŴ = Gᵀ·X (reduction over the M tokens), fp64 accumulation."""
+    d = np.asarray(G, f64).T @ np.asarray(Xb, f64)
+    return d.astype(f32) if dtype is f32 else d
+
+
+def ste_fold(gW, W, st, bits: int, symmetric: bool = False):
+    """Straight-through backward of the QDQ, per element into dV and per group into dalpha, dbeta.
+
+    Reverse mode over the forward of ``qdq`` with d round(x)/dx := 1 ([IA],
+    [AR] §3 'SignSGD') and d clamp/dt := m (1 inside [0, 2^b-1]):
+
+        dV     = g·s·m
+        c      = g·((q - zp) - m·W/s - (1-m)·lo/s)        (= g·dŴ/ds)
+        dhi    = Σ_group c / Q
+        dlo    = -Σ_group c / Q + Σ_group g·(1-m)
+        dalpha = mx·dhi,   dbeta = mn·dlo
+
+    (symmetric: c = g·((q - zp) - m·W/s); ds goes to the larger of hi, -lo).
+    When the scale guard is active s does not depend on hi, lo and c := 0.
+    Evaluated in fp64 from the forward's values; returned as fp64.
+    """
+    N, K = gW.shape
+    G = st["s"].shape[1]
+    g = K // G
+    gw = np.asarray(gW, f64).reshape(N, G, g)
+    Wd = np.asarray(W, f64).reshape(N, G, g)
+    s = np.asarray(st["s"], f64)[:, :, None]
+    zp = np.asarray(st["zp"], f64)[:, :, None]
+    lo = np.asarray(st["lo"], f64)[:, :, None]
+    q = np.asarray(st["q"], f64).reshape(N, G, g)
+    m = np.asarray(st["m"], f64).reshape(N, G, g)
+    dV = gw * s * m
+    if not symmetric:
+        Q = float(2 ** bits - 1)
+        c = gw * ((q - zp) - m * Wd / s - (1.0 - m) * lo / s)
+        c = np.where(st["guarded"][:, :, None], 0.0, c)
+        csum = c.sum(axis=-1)
+        dhi = csum / Q
+        dlo = -csum / Q + (gw * (1.0 - m)).sum(axis=-1)
+    else:
+        Qs = float(2 ** (bits - 1) - 1)
+        c = gw * ((q - zp) - m * Wd / s)
+        c = np.where(st["guarded"][:, :, None], 0.0, c)
+        dsum = c.sum(axis=-1) / Qs
+        hi = np.asarray(st["hi"], f64)
+        lo2 = np.asarray(st["lo"], f64)
+        take_hi = hi >= -lo2
+        dhi = np.where(take_hi, dsum, 0.0)
+        dlo = np.where(take_hi, 0.0, -dsum)
+    dalpha = np.asarray(st["mx"], f64) * dhi
+    dbeta = np.asarray(st["mn"], f64) * dlo
+    return dV.reshape(N, K), dalpha, dbeta
+
+
+def signsgd(p, d, lr: float, lo: float, hi: float) -> np.ndarray:
+    """SignSGD step and clamp ([AR] §3 'SignSGD'): p <- clamp(p - lr·sign(d), lo, hi), in fp32.
+
+    Each step moves by exactly ±lr (one fp32 subtraction), or not at all when
+    the gradient is zero.
+    """
+    p = np.asarray(p, f32)
+    step = (f32(lr) * sign0(np.asarray(d, f64)).astype(f32)).astype(f32)
+    return np.clip((p - step).astype(f32), f32(lo), f32(hi)).astype(f32)
+
+
+# ----------------------------------------------------------------------------
+# one tuning step of a single linear layer ([AR] §3 'Algorithm Flow' 3-5)
+# ----------------------------------------------------------------------------
+
+class QConfig:
+    """Quantizer and optimiser settings: bits, group size, symmetric flag, learning rate and bounds."""
+
+    def __init__(self, bits=4, group_size=128, symmetric=False, lr=0.005,
+                 v_min=-0.5, v_max=0.5, clip_min=0.5, clip_max=1.0):
+        self.bits, self.group_size, self.symmetric, self.lr = bits, group_size, bool(symmetric), lr
+        self.v_min, self.v_max, self.clip_min, self.clip_max = v_min, v_max, clip_min, clip_max
+
+
+def tune_step_linear(Wb, Xb, Y, V, alpha, beta, cfg: QConfig, count: int | None = None):
+    """One SignSGD step on one linear layer.
+
+    Wb [N][K] and Xb [M][K] are bf16 values held in float32; Y [M][N] is the
+    reference output; V, alpha, beta are the current state (not modified).
+    ``count`` is the loss normaliser M·N_total (defaults to this layer's M·N);
+    pass the full layer's count when ``Wb`` holds only a subset of rows, which
+    then gives exactly those rows of the full result.
+
+    Returns (loss, (V', alpha', beta'), grads dict, qdq dict).
+    """
+    M = Xb.shape[0]
+    N = Wb.shape[0]
+    count = M * N if count is None else count
+    st = qdq(Wb, V, alpha, beta, cfg.bits, cfg.group_size, cfg.symmetric)
+    fw = forward_loss(Xb, st["What_bf16"], Y, count)
+    gW = weight_grad(fw["G"], Xb)
+    dV, da, db = ste_fold(gW, Wb, st, cfg.bits, cfg.symmetric)
+    V1 = signsgd(V, dV, cfg.lr, cfg.v_min, cfg.v_max)
+    a1 = signsgd(alpha, da, cfg.lr, cfg.clip_min, cfg.clip_max)
+    b1 = signsgd(beta, db, cfg.lr, cfg.clip_min, cfg.clip_max)
+    grads = {"gW": gW, "dV": dV.astype(f32), "dalpha": da.astype(f32), "dbeta": db.astype(f32), "G": fw["G"]}
+    return fw["loss"], (V1, a1, b1), grads, st
+
+
+def eval_loss_linear(Wb, Xb, Y, V, alpha, beta, cfg: QConfig, count: int | None = None) -> float:
+    """Reconstruction MSE of the current state (QDQ forward only)."""
+    M, N = Xb.shape[0], Wb.shape[0]
+    count = M * N if count is None else count
+    st = qdq(Wb, V, alpha, beta, cfg.bits, cfg.group_size, cfg.symmetric)
+    return forward_loss(Xb, st["What_bf16"], Y, count)["loss"]
+
+
+def tune_linear(Wb, Xb, V, alpha, beta, cfg: QConfig, steps: int, Y=None, count: int | None = None):
+    """Run ``steps`` SignSGD steps; returns (losses per step, final state, final MSE)."""
+    if Y is None:
+        Y = reference_forward(Xb, Wb)
+    losses = []
+    for _ in range(steps):
+        L, (V, alpha, beta), _, _ = tune_step_linear(Wb, Xb, Y, V, alpha, beta, cfg, count)
+        losses.append(L)
+    final = eval_loss_linear(Wb, Xb, Y, V, alpha, beta, cfg, count)
+    return np.array(losses), (V, alpha, beta), final
+
+
+# ----------------------------------------------------------------------------
+# smooth surrogate for finite-difference checks of the STE chain rule
+# ----------------------------------------------------------------------------
+
+def smooth_loss_linear(W, X, Y, V, alpha, beta, bits, group_size, symmetric=False):
+    """fp64 loss with every rounding replaced by the identity (no bf16, no round).
+
+    With the roundings gone the STE gradients are the exact gradients of this
+    function (away from the clamp kinks), which finite differences can check.
+    """
+    st = qdq(W, V, alpha, beta, bits, group_size, symmetric, dtype=f64, rnd=round_identity)
+    fw = forward_loss(X, st["What"], Y, X.shape[0] * W.shape[0], dtype=f64)
+    return fw["loss"], st, fw
+
+
+def smooth_grads_linear(W, X, Y, V, alpha, beta, bits, group_size, symmetric=False):
+    """Analytic (STE-fold) gradients of ``smooth_loss_linear``."""
+    L, st, fw = smooth_loss_linear(W, X, Y, V, alpha, beta, bits, group_size, symmetric)
+    gW = weight_grad(fw["G"], X, dtype=f64)
+    return L, ste_fold(gW, W, st, bits, symmetric)
+
+
+# ----------------------------------------------------------------------------
+# INT4 export and the W4A16 matmul ([AR] §4 'Real INT4 Kernel')
+# ----------------------------------------------------------------------------
+
+def pack_int4(q: np.ndarray, s: np.ndarray, zp: np.ndarray):
+    """Pack 4-bit codes and per-group metadata.
+
+    words[n][j] = Σ_{i<8} q[n][8j+i] · 16^i  (uint32);  scale = fp16(s), zero = fp16(zp),
+    both round to nearest even (zp is an integer ≤ 15, exact).  Returns the
+    words and the fp16 bit patterns of scale and zero.
+    """
+    N, K = q.shape
+    assert K % 8 == 0
+    qi = np.asarray(q).astype(np.uint32).reshape(N, K // 8, 8)
+    assert qi.max(initial=0) <= 15
+    shifts = (4 * np.arange(8, dtype=np.uint32))[None, None, :]
+    words = np.bitwise_or.reduce(qi << shifts, axis=-1).astype(np.uint32)
+    scale16 = np.asarray(s, f32).astype(np.float16).view(np.uint16)
+    zero16 = np.asarray(zp, f32).astype(np.float16).view(np.uint16)
+    return words, scale16, zero16
+
+
+def unpack_int4(words: np.ndarray, K: int) -> np.ndarray:
+    """Inverse of the code layout of ``pack_int4``."""
+    N = words.shape[0]
+    shifts = (4 * np.arange(8, dtype=np.uint32))[None, None, :]
+    q = (words[:, :, None] >> shifts) & np.uint32(0xF)
+    return q.reshape(N, K).astype(np.uint8)
+
+
+def w4a16_matmul(A, words, scale16, zero16, group_size: int) -> np.ndarray:
+    """out[t][n] = Σ_k A[t][k]·(q[n][k] - zero[n][k/g])·scale[n][k/g], fp64 (returned as fp64).
+
+    ``A`` holds bf16 values as float32; scale and zero are fp16 bit patterns.
+    """
+    N = words.shape[0]
+    K = words.shape[1] * 8
+    q = unpack_int4(words, K).astype(f64)
+    s = scale16.view(np.float16).astype(f64)
+    z = zero16.view(np.float16).astype(f64)
+    deq = (q.reshape(N, K // group_size, group_size) - z[:, :, None]) * s[:, :, None]
+    return np.asarray(A, f64) @ deq.reshape(N, K).T

@@ -1,0 +1,450 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself.
+
+Each test checks the oracle against something other than its own formulas:
+the worked examples the AutoRound pages print (fixtures in tests/golden/, each
+with its citation), library routines (torch's bf16 cast, libm's roundf,
+Python's IEEE half packing), brute force over all rounding choices, naive
+loops, finite differences and closed forms.  A dropped term, a wrong sign or a
+transposed operand in the oracle fails at least one of them.
+"""
+import ctypes
+import ctypes.util
+import itertools
+import json
+import os
+import struct
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import autoround_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------
+# rounding primitives against library routines
+# ----------------------------------------------------------------------------
+
+def test_bf16_rne_matches_torch_cast():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(10.0) ** rng.integers(-30, 30, 20000).astype(np.float32),
+        # exact ties between two bf16 neighbours, both parities
+        (np.arange(0x3F800000, 0x3F800000 + 4096, dtype=np.uint32) * 0 + np.uint32(0x3F808000)).view(np.float32)[:1],
+        np.array([0x3F818000, 0x3F808000, 0xBF818000, 0x7F7FFFFF, 0x00000001, 0x80000000], np.uint32).view(np.float32),
+        np.array([np.inf, -np.inf, 0.0, 1.0, -2.5], np.float32),
+    ])
+    ref = torch.from_numpy(x.copy()).to(torch.bfloat16).to(torch.float32).numpy()
+    got = O.bf16_rne(x)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    assert np.isnan(O.bf16_rne(np.array([np.nan], np.float32)))[0]
+
+
+def test_round_half_away_matches_libm_roundf():
+    libm = ctypes.CDLL(ctypes.util.find_library("m"))
+    libm.roundf.restype = ctypes.c_float
+    libm.roundf.argtypes = [ctypes.c_float]
+    rng = np.random.default_rng(2)
+    vals = np.concatenate([
+        rng.uniform(-40, 40, 3000).astype(np.float32),
+        (rng.integers(-40, 40, 500) + 0.5).astype(np.float32),
+        np.array([0.49999997, -0.49999997, 0.5, -0.5, 2.5, -2.5, 8388607.5, 1e-30, -0.0], np.float32),
+    ])
+    got = O.round_half_away(vals)
+    ref = np.array([libm.roundf(float(v)) for v in vals], np.float32)
+    assert np.array_equal(got, ref)
+    # fp64 instantiation: the largest double below 0.5 must not round up
+    assert O.round_half_away(np.array([0.49999999999999994, 2.5, -3.5]))[0] == 0.0
+    assert list(O.round_half_away(np.array([0.49999999999999994, 2.5, -3.5]))[1:]) == [3.0, -4.0]
+
+
+# ----------------------------------------------------------------------------
+# worked examples printed on the pages
+# ----------------------------------------------------------------------------
+
+def test_minimal_example_no_clip_and_clip():
+    gd = golden("minimal_example_clip.json")
+    W = np.array([gd["weights"]])
+    V = np.zeros_like(W)
+    one = np.ones((1, 1))
+    # Strategy A: no clipping, scale = 8/15, everything but the outlier collapses to 0.
+    for T in (np.float64, np.float32):
+        st = O.qdq(W.astype(T), V.astype(T), one, one, gd["bits"], 4, dtype=T)
+        assert st["s"][0, 0] == pytest.approx(gd["strategy_A_no_clip"]["scale"], rel=1e-6)
+        assert np.allclose(st["What"][0], gd["strategy_A_no_clip"]["dequant"], atol=1e-6)
+        assert st["zp"][0, 0] == 0
+    # Strategy B: clip the upper bound to 0.6 (alpha = 0.6/8), scale 0.04.
+    alpha = np.full((1, 1), gd["strategy_B_clip_0_6"]["upper_clip"] / max(gd["weights"]))
+    st = O.qdq(W, V, alpha, one, gd["bits"], 4, dtype=np.float64)
+    assert st["s"][0, 0] == pytest.approx(gd["strategy_B_clip_0_6"]["scale"], rel=1e-12)
+    assert np.allclose(st["What"][0], gd["strategy_B_clip_0_6"]["dequant"], atol=1e-12)
+    assert 8.0 - st["What"][0, 3] == pytest.approx(gd["strategy_B_clip_0_6"]["clip_error_of_outlier"], abs=1e-12)
+    # the same in fp32: the tie 2.5 is lost to the rounding of 0.6f/15 (recorded in the fixture)
+    st32 = O.qdq(W.astype(np.float32), V.astype(np.float32), alpha.astype(np.float32), one, 4, 4, dtype=np.float32)
+    assert np.allclose(st32["What"][0], [0.08, 0.20, 0.16, 0.6], atol=1e-6)
+
+
+def test_state_evolution_w037():
+    gd = golden("state_evolution_w037.json")
+    for T in (np.float64, np.float32):
+        r = O.quantize(np.array([[gd["w"]]], T), np.zeros((1, 1), T), np.array([[gd["scale"]]], T),
+                       np.array([[gd["zero"]]], T), gd["bits"], dtype=T)
+        assert r["q"][0, 0] == gd["quantized"]
+        assert r["What"][0, 0] == pytest.approx(gd["dequantized"], abs=1e-6)
+        assert gd["w"] - r["What"][0, 0] == pytest.approx(gd["error"], abs=1e-6)
+        assert bool(r["m"][0, 0])  # round(7.4) + 8 = 15 is the top code, still in range
+
+
+def test_state_evolution_offset_flip():
+    gd = golden("state_evolution_v.json")
+    s = np.ones((1, 1))
+    z = np.zeros((1, 1))
+    w = np.array([[gd["w"]]])
+    for v, code in [(0.0, gd["v0_code"]), (gd["flip_point_v"] - 0.01, gd["v0_code"]),
+                    (gd["flip_point_v"] + 0.01, gd["rounded_up_code"]), (gd["v_range"][1], gd["rounded_up_code"])]:
+        r = O.quantize(w, np.array([[v]]), s, z, 8, dtype=np.float64)
+        assert r["q"][0, 0] == code
+    assert abs(O.quantize(w, np.array([[0.3]]), s, z, 8, dtype=np.float64)["What"][0, 0] - gd["w"]) == pytest.approx(gd["rounded_up_error"])
+
+
+def test_clip_error_panel():
+    gd = golden("clip_error_panel.json")
+    s = np.array([[gd["clip"] / 15.0]])
+    r = O.quantize(np.array([[gd["value"]]]), np.zeros((1, 1)), s, np.zeros((1, 1)), 4, dtype=np.float64)
+    assert r["What"][0, 0] == pytest.approx(gd["clipped_to"], abs=1e-12)
+    assert not r["m"][0, 0]
+    assert gd["value"] - r["What"][0, 0] == pytest.approx(gd["error"], abs=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# invariants and brute force
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("symmetric", [False, True])
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_rtn_is_nearest_grid_point(bits, symmetric):
+    """V = 0, alpha = beta = 1: every weight maps to its nearest grid point (brute force over all codes)."""
+    rng = np.random.default_rng(bits + 10 * symmetric)
+    W = rng.standard_normal((6, 64)) * 0.02
+    g = 16
+    st = O.qdq(W, np.zeros_like(W), np.ones((6, 4)), np.ones((6, 4)), bits, g, symmetric, dtype=np.float64)
+    Q = 2 ** bits - 1
+    s = np.repeat(st["s"], g, axis=1)
+    zp = np.repeat(st["zp"], g, axis=1)
+    grid = s[..., None] * (np.arange(Q + 1)[None, None, :] - zp[..., None])
+    best = np.abs(grid - W[..., None]).min(axis=-1)
+    assert np.allclose(np.abs(st["What"] - W), best, atol=1e-15)
+    if not symmetric:
+        # the range covers the whole group: no element is clipped
+        assert st["m"].all()
+        assert (np.abs(st["What"] - W) <= s / 2 + 1e-15).all()
+
+
+def test_offsets_move_codes_by_at_most_one():
+    rng = np.random.default_rng(3)
+    W = rng.standard_normal((8, 128)) * 0.02
+    a = np.ones((8, 1))
+    st0 = O.qdq(W, np.zeros_like(W), a, a, 4, 128, dtype=np.float64)
+    V = rng.uniform(-0.5, 0.5, W.shape)
+    st1 = O.qdq(W, V, a, a, 4, 128, dtype=np.float64)
+    assert np.abs(st1["q"] - st0["q"]).max() <= 1
+    assert np.array_equal(st0["s"], st1["s"])
+
+
+def test_grid_weights_reconstruct_exactly():
+    """Weights already on the grid: Ŵ = W, the residual, G and every gradient vanish."""
+    rng = np.random.default_rng(4)
+    N, K, M, g = 4, 32, 8, 16
+    codes = rng.integers(0, 16, (N, K)).astype(np.float64)
+    codes[:, 0::g] = 0
+    codes[:, 1::g] = 15
+    zp = 5.0
+    s = 0.25
+    W = s * (codes - zp)  # group range [-1.25, 2.5] contains 0; exact in binary
+    X = rng.standard_normal((M, K))
+    Y = X @ W.T
+    a = np.ones((N, K // g))
+    st = O.qdq(W, np.zeros_like(W), a, a, 4, g, dtype=np.float64)
+    assert np.array_equal(st["What"], W)
+    fw = O.forward_loss(X, st["What"], Y, M * N, dtype=np.float64)
+    assert fw["loss"] == 0.0 and not fw["G"].any()
+    dV, da, db = O.ste_fold(O.weight_grad(fw["G"], X, dtype=np.float64), W, st, 4)
+    assert not dV.any() and not da.any() and not db.any()
+
+
+def _direct_loss(X, Y, What):
+    """Σ (X·Ŵᵀ - Y)² / (M·N) by explicit loops."""
+    M, K = X.shape
+    N = What.shape[0]
+    tot = 0.0
+    for i in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += X[i, k] * What[n, k]
+            tot += (acc - Y[i, n]) ** 2
+    return tot / (M * N)
+
+
+def test_bruteforce_all_rounding_choices_on_an_8_weight_group():
+    """All 2^8 up/down choices ([AR] §2: the search space grows as 2^N).
+
+    The oracle, driven through V = ±0.49, must reproduce the loss of every
+    choice computed directly, and the best choice must beat round-to-nearest.
+    """
+    rng = np.random.default_rng(5)
+    g = 8
+    s_true = 0.1
+    # fractional parts of W/s kept in [0.1, 0.9] so that ±0.49 selects floor/ceil cleanly
+    base = rng.integers(-6, 6, g) + rng.uniform(0.1, 0.9, g)
+    W = (base * s_true)[None, :]
+    W[0, 0] = 7.4 * s_true  # fixes the range
+    W[0, 1] = -7.3 * s_true
+    M = 12
+    X = rng.standard_normal((M, g))
+    Y = X @ W.T
+    one = np.ones((1, 1))
+    st0 = O.qdq(W, np.zeros_like(W), one, one, 4, g, dtype=np.float64)
+    s = st0["s"][0, 0]
+    zp = st0["zp"][0, 0]
+    wq = W[0] / s
+    fl, ce = np.floor(wq), np.ceil(wq)
+    assert ((wq - fl > 0.02) & (ce - wq > 0.02)).all()
+    losses = {}
+    for bits in itertools.product([0, 1], repeat=g):
+        up = np.array(bits, bool)
+        V = np.where(up, 0.49, -0.49)[None, :]
+        st = O.qdq(W, V, one, one, 4, g, dtype=np.float64)
+        t = np.where(up, ce, fl) + zp
+        assert np.array_equal(st["t"][0], t)
+        direct = s * (np.clip(t, 0, 15) - zp)
+        assert np.allclose(st["What"][0], direct, rtol=0, atol=1e-15)
+        Lo = O.forward_loss(X, st["What"], Y, M, dtype=np.float64)["loss"]
+        Ld = _direct_loss(X, Y, direct[None, :])
+        assert Lo == pytest.approx(Ld, rel=1e-12, abs=1e-18)
+        losses[bits] = Lo
+    L_rtn = O.forward_loss(X, st0["What"], Y, M, dtype=np.float64)["loss"]
+    assert min(losses.values()) <= L_rtn
+
+
+def test_gemms_and_loss_against_loops():
+    rng = np.random.default_rng(6)
+    M, N, K = 3, 2, 8
+    X = rng.standard_normal((M, K))
+    What = rng.standard_normal((N, K))
+    Y = rng.standard_normal((M, N))
+    fw = O.forward_loss(X, What, Y, M * N, dtype=np.float64)
+    assert fw["loss"] == pytest.approx(_direct_loss(X, Y, What), rel=1e-12)
+    for i in range(M):
+        for n in range(N):
+            yh = sum(X[i, k] * What[n, k] for k in range(K))
+            assert fw["G"][i, n] == pytest.approx(2 * (yh - Y[i, n]) / (M * N), rel=1e-12)
+    gW = O.weight_grad(fw["G"], X, dtype=np.float64)
+    for n in range(N):
+        for k in range(K):
+            assert gW[n, k] == pytest.approx(sum(fw["G"][i, n] * X[i, k] for i in range(M)), rel=1e-12, abs=1e-15)
+    Y2 = O.reference_forward(X, What)
+    assert np.allclose(Y2, np.array([[sum(X[i, k] * What[n, k] for k in range(K)) for n in range(N)] for i in range(M)]), rtol=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# STE gradients against finite differences of the smooth surrogate
+# ----------------------------------------------------------------------------
+
+def _fd_case(symmetric, seed=7):
+    rng = np.random.default_rng(seed)
+    N, K, M, g = 3, 32, 10, 16
+    W = rng.standard_normal((N, K)) * 0.05
+    W[1, :g] = np.abs(W[1, :g])  # a group with mn = 0: dbeta must vanish there
+    W[2, g:] = -np.abs(W[2, g:])  # a group with mx = 0: dalpha must vanish there
+    X = rng.standard_normal((M, K))
+    Y = X @ W.T
+    V = rng.uniform(-0.45, 0.45, (N, K))
+    alpha = rng.uniform(0.55, 0.95, (N, K // g))
+    beta = rng.uniform(0.55, 0.95, (N, K // g))
+    return W, X, Y, V, alpha, beta, g
+
+
+@pytest.mark.parametrize("symmetric", [False, True])
+def test_ste_gradients_match_finite_differences(symmetric):
+    W, X, Y, V, alpha, beta, g = _fd_case(symmetric)
+    bits = 3
+    L, (dV, da, db) = O.smooth_grads_linear(W, X, Y, V, alpha, beta, bits, g, symmetric)
+    st = O.smooth_loss_linear(W, X, Y, V, alpha, beta, bits, g, symmetric)[1]
+    assert 0 < st["m"].mean() < 1, "case must contain clamped and unclamped weights"
+    h = 1e-7
+
+    def f(V_, a_, b_):
+        return O.smooth_loss_linear(W, X, Y, V_, a_, b_, bits, g, symmetric)[0]
+
+    for (n, k) in [(0, 0), (0, 5), (1, 17), (2, 31), (1, 3), (2, 9)]:
+        Vp, Vm = V.copy(), V.copy()
+        Vp[n, k] += h
+        Vm[n, k] -= h
+        fd = (f(Vp, alpha, beta) - f(Vm, alpha, beta)) / (2 * h)
+        assert dV[n, k] == pytest.approx(fd, rel=1e-5, abs=1e-12)
+    for n in range(W.shape[0]):
+        for j in range(alpha.shape[1]):
+            ap, am = alpha.copy(), alpha.copy()
+            ap[n, j] += h
+            am[n, j] -= h
+            fd = (f(V, ap, beta) - f(V, am, beta)) / (2 * h)
+            assert da[n, j] == pytest.approx(fd, rel=1e-5, abs=1e-12)
+            bp, bm = beta.copy(), beta.copy()
+            bp[n, j] += h
+            bm[n, j] -= h
+            fd = (f(V, alpha, bp) - f(V, alpha, bm)) / (2 * h)
+            assert db[n, j] == pytest.approx(fd, rel=1e-5, abs=1e-12)
+    # closed-form zeros: no lower range -> no beta gradient; no upper range -> no alpha gradient
+    assert db[1, 0] == 0.0
+    assert da[2, 1] == 0.0
+    assert (dV[~st["m"]] == 0).all()
+
+
+def test_scale_guard_on_an_all_zero_group():
+    W = np.zeros((1, 8))
+    W[0, 4:] = [0.1, -0.2, 0.3, 0.05]
+    st = O.qdq(W, np.zeros_like(W), np.ones((1, 2)), np.ones((1, 2)), 4, 4, dtype=np.float64)
+    assert st["guarded"][0, 0] and not st["guarded"][0, 1]
+    assert st["s"][0, 0] == O.S_GUARD and st["zp"][0, 0] == 0
+    assert not st["What"][0, :4].any()
+    gW = np.ones((1, 8))
+    dV, da, db = O.ste_fold(gW, W, st, 4)
+    assert da[0, 0] == 0.0 and db[0, 0] == 0.0
+
+
+# ----------------------------------------------------------------------------
+# SignSGD update: exact closed forms
+# ----------------------------------------------------------------------------
+
+def test_signsgd_exact_steps_and_clamp():
+    lr = 0.005
+    p = np.zeros(4, np.float32)
+    d = np.array([1e-12, -3.0, 0.0, np.nan], np.float32)
+    p1 = O.signsgd(p, d, lr, -0.5, 0.5)
+    assert p1.tolist() == [np.float32(-lr), np.float32(lr), 0.0, 0.0]
+    # 150 steps against a positive gradient: fp32 walk of -lr steps, then pinned at the bound
+    q = np.zeros(1, np.float32)
+    walk = np.float32(0.0)
+    for i in range(150):
+        q = O.signsgd(q, np.array([1.0], np.float32), lr, -0.5, 0.5)
+        walk = max(np.float32(walk - np.float32(lr)), np.float32(-0.5))
+        assert q[0] == walk
+    assert q[0] == np.float32(-0.5)
+    # clip factors live in [0.5, 1]: from 1 a negative gradient cannot push above 1
+    a = O.signsgd(np.ones(1, np.float32), np.array([-1.0]), lr, 0.5, 1.0)
+    assert a[0] == 1.0
+
+
+# ----------------------------------------------------------------------------
+# INT4 packing and the W4A16 matmul
+# ----------------------------------------------------------------------------
+
+def test_pack_int4_layout_and_fp16_metadata():
+    rng = np.random.default_rng(8)
+    N, K, g = 3, 64, 32
+    q = rng.integers(0, 16, (N, K))
+    s = rng.uniform(1e-4, 0.2, (N, K // g)).astype(np.float32)
+    s[0, 0] = 0.1
+    s[0, 1] = 1.0 / 3.0
+    s[1, 0] = 6.0e-8  # fp16 subnormal range
+    zp = rng.integers(0, 16, (N, K // g)).astype(np.float32)
+    words, s16, z16 = O.pack_int4(q, s, zp)
+    for n in range(N):
+        for j in range(K // 8):
+            w = 0
+            for i in range(8):
+                w |= int(q[n, 8 * j + i]) << (4 * i)
+            assert int(words[n, j]) == w
+    assert np.array_equal(O.unpack_int4(words, K), q.astype(np.uint8))
+    for n in range(N):
+        for j in range(K // g):
+            assert int(s16[n, j]) == struct.unpack("<H", struct.pack("<e", float(s[n, j])))[0]
+            assert int(z16[n, j]) == struct.unpack("<H", struct.pack("<e", float(zp[n, j])))[0]
+    assert int(s16[0, 0]) == 0x2E66 and int(s16[0, 1]) == 0x3555
+
+
+def test_w4a16_matmul_against_loops():
+    rng = np.random.default_rng(9)
+    T, N, K, g = 2, 3, 32, 16
+    q = rng.integers(0, 16, (N, K))
+    s = rng.uniform(0.01, 0.1, (N, K // g)).astype(np.float32)
+    zp = rng.integers(0, 16, (N, K // g)).astype(np.float32)
+    words, s16, z16 = O.pack_int4(q, s, zp)
+    A = O.bf16_rne(rng.standard_normal((T, K)).astype(np.float32))
+    out = O.w4a16_matmul(A, words, s16, z16, g)
+    for t in range(T):
+        for n in range(N):
+            ref = 0.0
+            for k in range(K):
+                sc = struct.unpack("<e", struct.pack("<H", int(s16[n, k // g])))[0]
+                ref += float(A[t, k]) * (int(q[n, k]) - float(zp[n, k // g])) * sc
+            assert out[t, n] == pytest.approx(ref, rel=1e-12, abs=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# structure the GPU parity tests rely on
+# ----------------------------------------------------------------------------
+
+def test_row_subset_is_exact():
+    """Rows of a single linear are independent: a row subset with the full loss count reproduces those rows."""
+    import synth
+
+    d = synth.make_linear(64, 256, 48, seed=3, x_outlier_channels=2)
+    Wb = synth.bf16_bits_to_f32(d["W"])
+    Xb = synth.bf16_bits_to_f32(d["X"])
+    Y = O.reference_forward(Xb, Wb)
+    V, a, b = synth.make_state(64, 256, 128, seed=3, spread=True)
+    cfg = O.QConfig()
+    L, (V1, a1, b1), gr, _ = O.tune_step_linear(Wb, Xb, Y, V, a, b, cfg)
+    rows = np.array([3, 17, 40, 63])
+    Ls, (Vs, as_, bs), grs, _ = O.tune_step_linear(Wb[rows], Xb, Y[:, rows], V[rows], a[rows], b[rows], cfg, count=48 * 64)
+    assert np.array_equal(Vs, V1[rows]) and np.array_equal(as_, a1[rows]) and np.array_equal(bs, b1[rows])
+    assert np.array_equal(grs["dV"], gr["dV"][rows])
+    assert np.array_equal(grs["G"], gr["G"][:, rows])
+
+
+def test_small_workload_tuning_lowers_the_loss():
+    """The 256x256 fp32 workload: 10 SignSGD steps end below the round-to-nearest loss."""
+    import synth
+
+    wl = synth.WORKLOADS["linear_256"]
+    d = synth.make_linear(wl.n_out, wl.n_in, wl.m_tokens, seed=wl.seed, dtype="f32", x_outlier_channels=0)
+    Wb, Xb = O.bf16_rne(d["W"]), O.bf16_rne(d["X"])
+    V, a, b = synth.make_state(wl.n_out, wl.n_in, wl.group_size)
+    cfg = O.QConfig(bits=wl.bits, group_size=wl.group_size, lr=wl.lr)
+    losses, _, final = O.tune_linear(Wb, Xb, V, a, b, cfg, wl.steps)
+    assert final < losses[0]
+
+
+def test_fp32_instantiation_agrees_with_fp64():
+    """The fp32 path (the GPU's rounding points) stays within bf16 precision of the fp64 path.
+
+    The fp64 path is pinned by loops and finite differences above; this ties the
+    fp32 loss, G and folded gradients to it (a wrong scale or a dropped factor
+    in the fp32 path fails here).
+    """
+    rng = np.random.default_rng(11)
+    N, K, M, g = 16, 128, 64, 32
+    W = O.bf16_rne((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
+    X = O.bf16_rne(rng.standard_normal((M, K)).astype(np.float32))
+    V = rng.uniform(-0.5, 0.5, (N, K)).astype(np.float32)
+    a = rng.uniform(0.5, 1, (N, K // g)).astype(np.float32)
+    b = rng.uniform(0.5, 1, (N, K // g)).astype(np.float32)
+    Y = O.reference_forward(X, W)
+    cfg = O.QConfig(bits=4, group_size=g)
+    L32, _, gr, st = O.tune_step_linear(W, X, Y, V, a, b, cfg)
+    fw64 = O.forward_loss(X, st["What_bf16"], Y, M * N, dtype=np.float64)
+    assert L32 == pytest.approx(fw64["loss"], rel=1e-5)
+    assert np.allclose(gr["G"], fw64["G"], rtol=2 ** -8, atol=0)
+    gW64 = O.weight_grad(fw64["G"], X, dtype=np.float64)
+    dV64, da64, db64 = O.ste_fold(gW64, W, st, 4)
+    rel = lambda x, y: np.linalg.norm(x - y) / np.linalg.norm(y)
+    assert rel(gr["dV"], dV64) < 5e-3 and rel(gr["dalpha"], da64) < 5e-3 and rel(gr["dbeta"], db64) < 5e-3
