@@ -1,0 +1,215 @@
+/*
+ * autoround.h — C ABI of libautoround.so: the AutoRound weight-quantization
+ * tuning step, INT4 export and the W4A16 matmul on one NVIDIA B200 (sm_100a).
+ *
+ * Sources cited below (page title, then section):
+ *  [AR] "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
+ *       Architectural Optimizations of AutoRound" — §2 "Minimal Example",
+ *       §3 "Optimization Variables" table, §3 "Algorithm Flow", §3 "SignSGD",
+ *       §4 "QDQ Fake Quantization vs. Real Inference" (comparison table and
+ *       "Minimal State Evolution" table), §8 preset-mode table.
+ *  [QC] "量化：从 Scale 到 W4A8 的完整坐标" — §1.2 basic integer mapping.
+ *  [IA] "Intel AutoRound 高级量化" (hotdry blog) — sign-gradient mechanism
+ *       (STE), production parameter advice (int4 g128 lr 0.005; int8 g256 lr 0.002).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device unless
+ *    stated otherwise, row-major, densely packed, 16-byte aligned.
+ *  - bf16 / fp16 tensors are passed as uint16_t bit patterns.
+ *  - The caller owns every buffer.  The library never allocates or frees
+ *    device memory; scratch comes from the caller's workspace.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream).  The
+ *    return value covers host-side validation and kernel launch only.
+ *    Device-side problems (non-finite inputs or gradients, a pipeline wait that
+ *    timed out) set a sticky status word read by ar_get_device_status().
+ *  - No silent fallback: an unsupported combination returns
+ *    AR_ERR_UNSUPPORTED and launches nothing.
+ *  - On any error return nothing has been launched and ar_last_error() holds
+ *    a one-line reason.
+ */
+#ifndef AUTOROUND_H_
+#define AUTOROUND_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AR_API __attribute__((visibility("default")))
+#else
+#define AR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ar_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  AR_OK = 0,
+  AR_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape */
+  AR_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  AR_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  AR_ERR_NONFINITE = 4,   /* device status: NaN/Inf seen in an input or gradient */
+  AR_ERR_TIMEOUT = 5,     /* device status: a pipeline wait gave up */
+  AR_ERR_WORKSPACE = 6    /* workspace missing or smaller than required */
+} ar_status;
+
+/* Quantizer and optimiser settings ([AR] §3 table and §8 presets; [IA]).
+ *  bits        2..8 (ar_pack_int4 and ar_w4a16_gemm: 4 only)
+ *  group_size  weights per group along in_features (K); must divide K.
+ *              ar_qdq: 8, 16, ..., 1024 (power of two);
+ *              ar_tune_step: 32, 64, 128 or 256.
+ *  symmetric   0: asymmetric (s = (hi-lo)/(2^b-1), zp = round(-lo/s));
+ *              1: symmetric  (s = max(hi,-lo)/(2^(b-1)-1), zp = 2^(b-1)).
+ *  lr          SignSGD step ([AR] §3 "SignSGD"; 5e-3 in all presets).
+ *  iters       default step count for drivers; ar_tune_step takes n_steps.
+ *  v_min/v_max bounds of the rounding offsets V ([AR] §3 table: -0.5, 0.5).
+ *  clip_min/clip_max bounds of the clip factors alpha, beta (0.5, 1.0).     */
+typedef struct {
+  int bits;
+  int group_size;
+  int symmetric;
+  float lr;
+  int iters;
+  float v_min, v_max;
+  float clip_min, clip_max;
+} ar_qconfig;
+
+/* Fills *cfg with the defaults: 4 bits, group 128, asymmetric, lr 5e-3,
+ * 200 iterations, V in [-0.5, 0.5], alpha/beta in [0.5, 1]. */
+AR_API void ar_qconfig_default(ar_qconfig* cfg);
+
+/* One quantized linear layer of a block.
+ *  W      bf16 [N][K], original weights (read only)
+ *  V      fp32 [N][K], rounding offsets (in/out for ar_tune_step)
+ *  alpha  fp32 [N][K/group_size], multiplier of the group maximum (in/out)
+ *  beta   fp32 [N][K/group_size], multiplier of the group minimum (in/out) */
+typedef struct {
+  const uint16_t* W;
+  float* V;
+  float* alpha;
+  float* beta;
+  int64_t N; /* out_features */
+  int64_t K; /* in_features */
+} ar_layer;
+
+/* Optional gradient outputs of the LAST step of an ar_tune_step call (any
+ * pointer may be NULL).  Same shapes as V, alpha, beta of each layer. */
+typedef struct {
+  float* dV;
+  float* dalpha;
+  float* dbeta;
+} ar_grads;
+
+typedef enum {
+  AR_BLOCK_LINEAR = 0 /* one linear layer: Y = X W^T (n_layers = 1) */
+} ar_block_kind;
+
+/* ------------------------------------------------------------------------ */
+
+/* fp32 -> bf16 (round to nearest even) of n values: src fp32 [n], dst bf16 [n].
+ * Marshalling for fp32 workloads: the tuning path runs on bf16 X and W
+ * ([AR] §3 "Algorithm Flow" step 2: the reference uses the BF16 weights). */
+AR_API ar_status ar_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, ar_stream_t stream);
+
+/* Fake-quant (QDQ) forward of one weight matrix ([AR] §4 comparison table,
+ * "QDQ" column; [AR] §2 "Minimal Example"; [QC] §1.2):
+ *   mx = max(0, max_group W),  mn = min(0, min_group W)
+ *   hi = alpha*mx, lo = beta*mn, s = (hi-lo)/(2^b-1) (>= 1e-8), zp = round(-lo/s)
+ *   q  = clamp(round(W/s + V) + zp, 0, 2^b-1),  W_hat = s*(q - zp)
+ * All arithmetic in fp32 IEEE operations (no contraction), round() is half
+ * away from zero.
+ * Inputs:  W bf16 [N][K]; V fp32 [N][K]; alpha, beta fp32 [N][K/g].
+ * Outputs (each may be NULL, at least one non-NULL):
+ *   W_hat bf16 [N][K] (round to nearest even); codes uint8 [N][K];
+ *   scale fp32 [N][K/g]; zero fp32 [N][K/g] (integer valued).
+ * Errors: AR_ERR_INVALID_ARG (shape, alignment, K % g), AR_ERR_UNSUPPORTED
+ * (bits or group_size outside the ranges above). */
+AR_API ar_status ar_qdq(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N, int64_t K,
+                 const ar_qconfig* cfg, uint16_t* W_hat, uint8_t* codes, float* scale, float* zero,
+                 ar_stream_t stream);
+
+/* Reference forward of one linear layer with its original weights ([AR] §3
+ * "Algorithm Flow" step 2): Y fp32 [M][N] = X bf16 [M][K] x W bf16 [N][K]^T,
+ * fp32 accumulation on the tensor cores.  Needs N % 8 == 0, K % 8 == 0.
+ * No workspace. */
+AR_API ar_status ar_linear_forward(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K, float* Y,
+                            ar_stream_t stream);
+
+/* Bytes of workspace ar_tune_step needs for this block, M tokens and
+ * n_steps steps (0 on invalid input; see ar_last_error()). */
+AR_API size_t ar_tune_step_workspace(int block_kind, const ar_layer* layers, int n_layers, int64_t M,
+                              const ar_qconfig* cfg, int n_steps);
+
+/* n_steps SignSGD tuning steps of one block ([AR] §3 "Algorithm Flow" steps
+ * 3-5, "SignSGD"; [IA] STE):
+ *   QDQ forward -> Y_hat = X W_hat^T -> R = Y_hat - Y, loss = sum R^2/(M N),
+ *   G = bf16(2R/(M N)) -> dW_hat = G^T X -> straight-through fold:
+ *     dV = g s m,  c = g((q-zp) - m W/s - (1-m) lo/s),
+ *     dalpha = mx sum_group(c)/Q,  dbeta = mn (-sum_group(c)/Q + sum_group g(1-m))
+ *   (m = 1 where 0 <= round(W/s+V)+zp <= Q) -> p <- clamp(p - lr sign(dp)).
+ * X: bf16 [M][K] calibration activations (all M rows are used every step).
+ * Y: fp32 [M][N], the reference output of ar_linear_forward (required).
+ * layers[0].V/alpha/beta are updated in place after every step.
+ * loss_per_step: device fp32 [max(n_steps,1)]; entry i is the loss of the
+ *   state before update i.  n_steps = 0 evaluates the loss of the current
+ *   state into loss_per_step[0] and updates nothing.
+ * grads: NULL, or gradient outputs of the last step.
+ * workspace: device buffer of at least ar_tune_step_workspace() bytes.
+ * Supported: AR_BLOCK_LINEAR with n_layers = 1; bits 2..8; group_size 32,
+ * 64, 128, 256; N % 8 == 0; K % 256 == 0 is NOT required (K % g == 0 is).
+ * Errors: AR_ERR_INVALID_ARG, AR_ERR_UNSUPPORTED, AR_ERR_WORKSPACE. */
+AR_API ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_layers, const uint16_t* X, int64_t M,
+                       const float* Y, const ar_qconfig* cfg, int n_steps, float* loss_per_step,
+                       const ar_grads* grads, void* workspace, size_t workspace_bytes, ar_stream_t stream);
+
+/* Export the tuned codes as INT4 ([AR] §4 comparison table, "Real INT4
+ * Kernel" column: weights stored as 4-bit integers with per-group metadata).
+ * Recomputes the codes exactly as ar_qdq does, then writes
+ *   packed  uint32 [N][K/8]: element k at bits 4*(k mod 8) of word k/8
+ *   scale   fp16  [N][K/g]: fp16(s), round to nearest even
+ *   zero    fp16  [N][K/g]: fp16(zp) (exact: integer <= 15)
+ * Needs cfg->bits == 4, asymmetric or symmetric, K % 8 == 0. */
+AR_API ar_status ar_pack_int4(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                       int64_t K, const ar_qconfig* cfg, uint32_t* packed, uint16_t* scale_f16,
+                       uint16_t* zero_f16, ar_stream_t stream);
+
+/* W4A16 matmul ([AR] §4: dequantization fused into the kernel):
+ *   out[t][n] = sum_k A[t][k] (q[n][k] - zero[n][k/g]) scale[n][k/g]
+ * A bf16 [T][K]; packed/scale/zero as written by ar_pack_int4; out bf16 [T][N]
+ * (round to nearest even of the fp32 accumulation).
+ * Supported: 1 <= T <= 16, group_size 32..1024 (power of two) dividing K,
+ * K % 32 == 0.  Larger T returns AR_ERR_UNSUPPORTED. */
+AR_API ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, const uint16_t* scale_f16,
+                        const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, uint16_t* out,
+                        ar_stream_t stream);
+
+/* Plain tensor-core GEMM, fp32 out: D[M][N] = sum_k A(m,k) B(n,k).
+ * A is [M][K] (a_mn_major = 0) or [K][M] (a_mn_major = 1); B is [N][K]
+ * (b_mn_major = 0) or [K][N] (b_mn_major = 1); all bf16.  The same
+ * tcgen05 mainloop as the tuning step, exposed for testing the operand
+ * layouts.  Needs N % 8 == 0, K % 8 == 0 and, when A is MN-major, M % 8 == 0. */
+AR_API ar_status ar_gemm_bf16(const uint16_t* A, int a_mn_major, const uint16_t* B, int b_mn_major, float* D, int64_t M,
+                       int64_t N, int64_t K, ar_stream_t stream);
+
+/* Synchronizes `stream`, then returns and clears the sticky device status:
+ * AR_OK, AR_ERR_NONFINITE or AR_ERR_TIMEOUT (timeout wins if both are set),
+ * or AR_ERR_CUDA if the synchronization itself failed. */
+AR_API ar_status ar_get_device_status(ar_stream_t stream);
+
+/* One line describing the last error of this host thread ("" if none). */
+AR_API const char* ar_last_error(void);
+
+/* Names of the kernels the last successful call of this host thread launched,
+ * separated by ';' (tracing: shows which kernel variant ran). */
+AR_API const char* ar_last_kernels(void);
+
+/* Library version string. */
+AR_API const char* ar_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AUTOROUND_H_ */

@@ -1,0 +1,198 @@
+"""Python binding of libautoround.so: AutoRound tuning step, INT4 export, W4A16 matmul on B200.
+
+Argument marshalling only.  Every function below has the name of the C entry
+point it calls (``include/autoround.h``); tensors are ``torch`` CUDA tensors
+(bf16 tensors as ``torch.bfloat16``, fp16 bit patterns as ``torch.float16``),
+streams default to the current torch stream.  There is no CPU path: importing
+works without a GPU, but every call needs the built library and a CUDA device
+and raises :class:`ARError` otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "ARError", "QConfig", "Layer", "Grads", "lib", "library_path",
+    "ar_qconfig_default", "ar_f32_to_bf16", "ar_qdq", "ar_linear_forward", "ar_tune_step_workspace",
+    "ar_tune_step", "ar_pack_int4", "ar_w4a16_gemm", "ar_gemm_bf16", "ar_get_device_status",
+    "ar_last_error", "ar_last_kernels", "ar_version", "AR_BLOCK_LINEAR",
+]
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
+
+AR_OK, AR_ERR_INVALID_ARG, AR_ERR_UNSUPPORTED, AR_ERR_CUDA, AR_ERR_NONFINITE, AR_ERR_TIMEOUT, AR_ERR_WORKSPACE = range(7)
+_STATUS_NAMES = ["AR_OK", "AR_ERR_INVALID_ARG", "AR_ERR_UNSUPPORTED", "AR_ERR_CUDA", "AR_ERR_NONFINITE",
+                 "AR_ERR_TIMEOUT", "AR_ERR_WORKSPACE"]
+AR_BLOCK_LINEAR = 0
+
+
+class ARError(RuntimeError):
+    """A non-zero ``ar_status`` from the library, with its ``ar_last_error()`` text."""
+
+    def __init__(self, status: int, message: str):
+        name = _STATUS_NAMES[status] if 0 <= status < len(_STATUS_NAMES) else str(status)
+        super().__init__(f"{name}: {message}")
+        self.status = status
+
+
+class QConfig(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("symmetric", ctypes.c_int),
+                ("lr", ctypes.c_float), ("iters", ctypes.c_int), ("v_min", ctypes.c_float),
+                ("v_max", ctypes.c_float), ("clip_min", ctypes.c_float), ("clip_max", ctypes.c_float)]
+
+
+class Layer(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("V", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [("dV", ctypes.c_void_p), ("dalpha", ctypes.c_void_p), ("dbeta", ctypes.c_void_p)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+
+_SIGNATURES = {
+    "ar_qconfig_default": (None, [ctypes.POINTER(QConfig)]),
+    "ar_f32_to_bf16": (_INT, [_P, _P, _I64, _P]),
+    "ar_qdq": (_INT, [_P, _P, _P, _P, _I64, _I64, ctypes.POINTER(QConfig), _P, _P, _P, _P, _P]),
+    "ar_linear_forward": (_INT, [_P, _I64, _P, _I64, _I64, _P, _P]),
+    "ar_tune_step_workspace": (ctypes.c_size_t, [_INT, ctypes.POINTER(Layer), _INT, _I64, ctypes.POINTER(QConfig), _INT]),
+    "ar_tune_step": (_INT, [_INT, ctypes.POINTER(Layer), _INT, _P, _I64, _P, ctypes.POINTER(QConfig), _INT, _P,
+                            ctypes.POINTER(Grads), _P, ctypes.c_size_t, _P]),
+    "ar_pack_int4": (_INT, [_P, _P, _P, _P, _I64, _I64, ctypes.POINTER(QConfig), _P, _P, _P, _P]),
+    "ar_w4a16_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _P, _P]),
+    "ar_gemm_bf16": (_INT, [_P, _INT, _P, _INT, _P, _I64, _I64, _I64, _P]),
+    "ar_get_device_status": (_INT, [_P]),
+    "ar_last_error": (ctypes.c_char_p, []),
+    "ar_last_kernels": (ctypes.c_char_p, []),
+    "ar_version": (ctypes.c_char_p, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libautoround.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise ARError(AR_ERR_UNSUPPORTED, f"{library_path} is not built; run "
+                          "`python -m post_weight_quantization_autoround_b200.build`")
+        L = ctypes.CDLL(library_path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ARError(AR_ERR_INVALID_ARG, "tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ARError(AR_ERR_INVALID_ARG, "tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _check(status: int):
+    if status != AR_OK:
+        raise ARError(status, lib().ar_last_error().decode())
+
+
+def ar_last_error() -> str:
+    return lib().ar_last_error().decode()
+
+
+def ar_last_kernels() -> str:
+    return lib().ar_last_kernels().decode()
+
+
+def ar_version() -> str:
+    return lib().ar_version().decode()
+
+
+def ar_qconfig_default(**overrides) -> QConfig:
+    cfg = QConfig()
+    lib().ar_qconfig_default(ctypes.byref(cfg))
+    for k, v in overrides.items():
+        setattr(cfg, k, v)
+    return cfg
+
+
+def ar_f32_to_bf16(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    _check(lib().ar_f32_to_bf16(_ptr(src), _ptr(dst), src.numel(), _stream(stream)))
+
+
+def ar_qdq(W, V, alpha, beta, cfg: QConfig, W_hat=None, codes=None, scale=None, zero=None, stream=None) -> None:
+    N, K = W.shape
+    _check(lib().ar_qdq(_ptr(W), _ptr(V), _ptr(alpha), _ptr(beta), N, K, ctypes.byref(cfg), _ptr(W_hat),
+                        _ptr(codes), _ptr(scale), _ptr(zero), _stream(stream)))
+
+
+def ar_linear_forward(X, W, Y, stream=None) -> None:
+    M, K = X.shape
+    N = W.shape[0]
+    _check(lib().ar_linear_forward(_ptr(X), M, _ptr(W), N, K, _ptr(Y), _stream(stream)))
+
+
+def _layer(W, V, alpha, beta) -> Layer:
+    N, K = W.shape
+    return Layer(_ptr(W), _ptr(V), _ptr(alpha), _ptr(beta), N, K)
+
+
+def ar_tune_step_workspace(W, V, alpha, beta, M: int, cfg: QConfig, n_steps: int,
+                           block_kind: int = AR_BLOCK_LINEAR) -> int:
+    layer = _layer(W, V, alpha, beta)
+    n = lib().ar_tune_step_workspace(block_kind, ctypes.byref(layer), 1, M, ctypes.byref(cfg), n_steps)
+    if n == 0:
+        raise ARError(AR_ERR_INVALID_ARG, ar_last_error())
+    return int(n)
+
+
+def ar_tune_step(W, V, alpha, beta, X, Y, cfg: QConfig, n_steps: int, loss, workspace,
+                 dV=None, dalpha=None, dbeta=None, stream=None, block_kind: int = AR_BLOCK_LINEAR) -> None:
+    """Run ``n_steps`` tuning steps; V, alpha, beta are updated in place, losses go to ``loss``."""
+    layer = _layer(W, V, alpha, beta)
+    grads = Grads(_ptr(dV), _ptr(dalpha), _ptr(dbeta))
+    gp = ctypes.byref(grads) if (dV is not None or dalpha is not None or dbeta is not None) else None
+    _check(lib().ar_tune_step(block_kind, ctypes.byref(layer), 1, _ptr(X), X.shape[0], _ptr(Y), ctypes.byref(cfg),
+                              n_steps, _ptr(loss), gp, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)))
+
+
+def ar_pack_int4(W, V, alpha, beta, cfg: QConfig, packed, scale16, zero16, stream=None) -> None:
+    N, K = W.shape
+    _check(lib().ar_pack_int4(_ptr(W), _ptr(V), _ptr(alpha), _ptr(beta), N, K, ctypes.byref(cfg), _ptr(packed),
+                              _ptr(scale16), _ptr(zero16), _stream(stream)))
+
+
+def ar_w4a16_gemm(A, packed, scale16, zero16, group_size: int, out, stream=None) -> None:
+    T, K = A.shape
+    N = packed.shape[0]
+    _check(lib().ar_w4a16_gemm(_ptr(A), T, _ptr(packed), _ptr(scale16), _ptr(zero16), N, K, group_size, _ptr(out),
+                               _stream(stream)))
+
+
+def ar_gemm_bf16(A, a_mn_major: bool, B, b_mn_major: bool, D, M: int, N: int, K: int, stream=None) -> None:
+    _check(lib().ar_gemm_bf16(_ptr(A), int(a_mn_major), _ptr(B), int(b_mn_major), _ptr(D), M, N, K,
+                              _stream(stream)))
+
+
+def ar_get_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the sticky device status code."""
+    return int(lib().ar_get_device_status(_stream(stream)))

@@ -1,0 +1,355 @@
+// C ABI of libautoround.so (declared in include/autoround.h): argument
+// validation, workspace layout and the launch sequence of each entry point.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "../../include/autoround.h"
+#include "ar_internal.h"
+
+namespace ar {
+
+namespace {
+thread_local std::string t_error;
+thread_local std::string t_kernels;
+thread_local std::string t_kernels_last;
+
+ar_status fail(ar_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_error = buf;
+  return code;
+}
+
+ar_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(AR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+void begin_call() {
+  t_error.clear();
+  t_kernels.clear();
+}
+
+ar_status end_call() {
+  t_kernels_last = t_kernels;
+  return AR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+ar_status check_cfg(const ar_qconfig* cfg) {
+  if (!cfg) return fail(AR_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->bits < 2 || cfg->bits > 8) return fail(AR_ERR_UNSUPPORTED, "bits=%d outside 2..8", cfg->bits);
+  if (cfg->symmetric != 0 && cfg->symmetric != 1) return fail(AR_ERR_INVALID_ARG, "symmetric must be 0 or 1");
+  if (!(cfg->lr >= 0.0f) || !(cfg->lr < 1e30f)) return fail(AR_ERR_INVALID_ARG, "lr must be finite and >= 0");
+  if (!(cfg->v_min <= cfg->v_max) || !(cfg->clip_min <= cfg->clip_max))
+    return fail(AR_ERR_INVALID_ARG, "bounds must satisfy min <= max");
+  return AR_OK;
+}
+
+// Layout of the tuning workspace for one linear layer.
+struct LinearWs {
+  size_t what, g, s, zp, mx, mn, partial, total;
+  int partials_per_step;
+};
+
+LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int g, int n_steps) {
+  LinearWs w{};
+  const int64_t groups = N * (K / g);
+  size_t off = 0;
+  w.what = off;
+  off = align_up(off + static_cast<size_t>(N * K) * 2, 256);
+  w.g = off;
+  off = align_up(off + static_cast<size_t>(M * N) * 2, 256);
+  w.s = off;
+  off = align_up(off + static_cast<size_t>(groups) * 4, 256);
+  w.zp = off;
+  off = align_up(off + static_cast<size_t>(groups) * 4, 256);
+  w.mx = off;
+  off = align_up(off + static_cast<size_t>(groups) * 4, 256);
+  w.mn = off;
+  off = align_up(off + static_cast<size_t>(groups) * 4, 256);
+  w.partials_per_step = resid_partials(static_cast<int>(M), static_cast<int>(N));
+  w.partial = off;
+  off = align_up(off + static_cast<size_t>(w.partials_per_step) * (n_steps > 0 ? n_steps : 1) * 8, 256);
+  w.total = off;
+  return w;
+}
+
+ar_status check_linear(const ar_layer* layers, int n_layers, int64_t M, const ar_qconfig* cfg, bool for_tune) {
+  ar_status st = check_cfg(cfg);
+  if (st != AR_OK) return st;
+  if (!layers || n_layers != 1) return fail(AR_ERR_UNSUPPORTED, "AR_BLOCK_LINEAR needs exactly one layer");
+  const ar_layer& L = layers[0];
+  if (L.N <= 0 || L.K <= 0 || M <= 0) return fail(AR_ERR_INVALID_ARG, "sizes must be positive (M=%lld N=%lld K=%lld)",
+                                                  (long long)M, (long long)L.N, (long long)L.K);
+  const int g = cfg->group_size;
+  if (for_tune && g != 32 && g != 64 && g != 128 && g != 256)
+    return fail(AR_ERR_UNSUPPORTED, "ar_tune_step supports group_size 32, 64, 128, 256 (got %d)", g);
+  if (L.K % g != 0) return fail(AR_ERR_INVALID_ARG, "K=%lld is not a multiple of group_size=%d", (long long)L.K, g);
+  if (L.N % 8 != 0) return fail(AR_ERR_INVALID_ARG, "N=%lld must be a multiple of 8", (long long)L.N);
+  if (M > INT32_MAX || L.N > INT32_MAX || L.K > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  if (!L.W || !L.V || !L.alpha || !L.beta) return fail(AR_ERR_INVALID_ARG, "layer pointer is NULL");
+  if (!aligned16(L.W) || !aligned16(L.V) || !aligned16(L.alpha) || !aligned16(L.beta))
+    return fail(AR_ERR_INVALID_ARG, "layer pointers must be 16-byte aligned");
+  return AR_OK;
+}
+
+}  // namespace
+
+void trace_kernel(const char* name) {
+  if (!t_kernels.empty()) t_kernels += ";";
+  t_kernels += name;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = v > 0 ? v : 1;
+  }
+  return cache[dev];
+}
+
+}  // namespace ar
+
+using namespace ar;
+
+extern "C" {
+
+void ar_qconfig_default(ar_qconfig* cfg) {
+  if (!cfg) return;
+  cfg->bits = 4;
+  cfg->group_size = 128;
+  cfg->symmetric = 0;
+  cfg->lr = 0.005f;
+  cfg->iters = 200;
+  cfg->v_min = -0.5f;
+  cfg->v_max = 0.5f;
+  cfg->clip_min = 0.5f;
+  cfg->clip_max = 1.0f;
+}
+
+ar_status ar_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, ar_stream_t stream) {
+  begin_call();
+  if (n < 0) return fail(AR_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return end_call();
+  if (!src || !dst) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(src) || !aligned16(dst)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaError_t e = launch_f32_to_bf16(src, dst, n, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "f32_to_bf16 launch");
+  return end_call();
+}
+
+ar_status ar_qdq(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N, int64_t K,
+                 const ar_qconfig* cfg, uint16_t* W_hat, uint8_t* codes, float* scale, float* zero,
+                 ar_stream_t stream) {
+  begin_call();
+  ar_status st = check_cfg(cfg);
+  if (st != AR_OK) return st;
+  const int g = cfg->group_size;
+  if (!pow2(g) || g < 8 || g > 1024) return fail(AR_ERR_UNSUPPORTED, "group_size %d: ar_qdq needs a power of two in 8..1024", g);
+  if (N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "N, K must be positive");
+  if (K % g != 0) return fail(AR_ERR_INVALID_ARG, "K=%lld is not a multiple of group_size=%d", (long long)K, g);
+  if (!W || !V || !alpha || !beta) return fail(AR_ERR_INVALID_ARG, "NULL input pointer");
+  if (!W_hat && !codes && !scale && !zero) return fail(AR_ERR_INVALID_ARG, "no output requested");
+  const void* ptrs[] = {W, V, alpha, beta, W_hat, codes, scale, zero};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaError_t e = launch_qdq(W, V, alpha, beta, N, K, g, cfg->bits, cfg->symmetric, W_hat, codes, scale, zero,
+                             nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+  return end_call();
+}
+
+ar_status ar_linear_forward(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K, float* Y,
+                            ar_stream_t stream) {
+  begin_call();
+  if (M <= 0 || N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "sizes must be positive");
+  if (N % 8 != 0 || K % 8 != 0) return fail(AR_ERR_INVALID_ARG, "N and K must be multiples of 8");
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  if (!X || !W || !Y) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(X) || !aligned16(W) || !aligned16(Y)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaError_t e = launch_gemm_store(X, W, Y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                                    reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reference forward launch");
+  return end_call();
+}
+
+size_t ar_tune_step_workspace(int block_kind, const ar_layer* layers, int n_layers, int64_t M, const ar_qconfig* cfg,
+                              int n_steps) {
+  begin_call();
+  if (block_kind != AR_BLOCK_LINEAR) {
+    fail(AR_ERR_UNSUPPORTED, "block_kind %d not supported", block_kind);
+    return 0;
+  }
+  if (n_steps < 0) {
+    fail(AR_ERR_INVALID_ARG, "n_steps must be >= 0");
+    return 0;
+  }
+  if (check_cfg(cfg) != AR_OK) return 0;
+  if (!layers || n_layers != 1 || layers[0].N <= 0 || layers[0].K <= 0 || M <= 0 || cfg->group_size <= 0 ||
+      layers[0].K % cfg->group_size != 0) {
+    fail(AR_ERR_INVALID_ARG, "invalid layer shapes");
+    return 0;
+  }
+  return linear_ws(M, layers[0].N, layers[0].K, cfg->group_size, n_steps).total;
+}
+
+ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_layers, const uint16_t* X, int64_t M,
+                       const float* Y, const ar_qconfig* cfg, int n_steps, float* loss_per_step, const ar_grads* grads,
+                       void* workspace, size_t workspace_bytes, ar_stream_t stream) {
+  begin_call();
+  if (block_kind != AR_BLOCK_LINEAR) return fail(AR_ERR_UNSUPPORTED, "block_kind %d not supported", block_kind);
+  ar_status st = check_linear(layers, n_layers, M, cfg, true);
+  if (st != AR_OK) return st;
+  if (n_steps < 0) return fail(AR_ERR_INVALID_ARG, "n_steps must be >= 0");
+  if (!X || !Y || !loss_per_step) return fail(AR_ERR_INVALID_ARG, "X, Y and loss_per_step are required");
+  if (!aligned16(X) || !aligned16(Y)) return fail(AR_ERR_INVALID_ARG, "X and Y must be 16-byte aligned");
+  const ar_layer& L = layers[0];
+  const LinearWs w = linear_ws(M, L.N, L.K, cfg->group_size, n_steps);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (grads) {
+    const void* gp[] = {grads->dV, grads->dalpha, grads->dbeta};
+    for (const void* p : gp)
+      if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "gradient outputs must be 16-byte aligned");
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* W_hat = reinterpret_cast<uint16_t*>(ws + w.what);
+  uint16_t* G = reinterpret_cast<uint16_t*>(ws + w.g);
+  float* sc = reinterpret_cast<float*>(ws + w.s);
+  float* zp = reinterpret_cast<float*>(ws + w.zp);
+  float* mx = reinterpret_cast<float*>(ws + w.mx);
+  float* mn = reinterpret_cast<float*>(ws + w.mn);
+  double* partial = reinterpret_cast<double*>(ws + w.partial);
+  const int Mi = static_cast<int>(M), Ni = static_cast<int>(L.N), Ki = static_cast<int>(L.K);
+  const float gscale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(L.N)));
+  const int steps = n_steps > 0 ? n_steps : 1;
+  cudaError_t e;
+  for (int step = 0; step < steps; ++step) {
+    e = launch_qdq(L.W, L.V, L.alpha, L.beta, L.N, L.K, cfg->group_size, cfg->bits, cfg->symmetric, W_hat, nullptr,
+                   sc, zp, mx, mn, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+    e = launch_gemm_resid(X, W_hat, Y, G, gscale, partial + static_cast<size_t>(step) * w.partials_per_step, Mi, Ni,
+                          Ki, s);
+    if (e != cudaSuccess) return cuda_fail(e, "forward GEMM launch");
+    if (n_steps == 0) break;
+    FoldArgs fa{};
+    fa.W = L.W;
+    fa.V = L.V;
+    fa.alpha = L.alpha;
+    fa.beta = L.beta;
+    fa.s = sc;
+    fa.zp = zp;
+    fa.mx = mx;
+    fa.mn = mn;
+    const bool last = step == steps - 1;
+    fa.dV_out = (last && grads) ? grads->dV : nullptr;
+    fa.da_out = (last && grads) ? grads->dalpha : nullptr;
+    fa.db_out = (last && grads) ? grads->dbeta : nullptr;
+    fa.group_size = cfg->group_size;
+    fa.bits = cfg->bits;
+    fa.symmetric = cfg->symmetric;
+    fa.lr = cfg->lr;
+    fa.v_min = cfg->v_min;
+    fa.v_max = cfg->v_max;
+    fa.c_min = cfg->clip_min;
+    fa.c_max = cfg->clip_max;
+    e = launch_gemm_fold(G, X, fa, Mi, Ni, Ki, s);
+    if (e != cudaSuccess) return cuda_fail(e, "weight-gradient GEMM launch");
+  }
+  e = launch_loss_reduce(partial, w.partials_per_step, steps, 1.0 / (static_cast<double>(M) * static_cast<double>(L.N)),
+                         loss_per_step, s);
+  if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
+  return end_call();
+}
+
+ar_status ar_pack_int4(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N, int64_t K,
+                       const ar_qconfig* cfg, uint32_t* packed, uint16_t* scale_f16, uint16_t* zero_f16,
+                       ar_stream_t stream) {
+  begin_call();
+  ar_status st = check_cfg(cfg);
+  if (st != AR_OK) return st;
+  if (cfg->bits != 4) return fail(AR_ERR_UNSUPPORTED, "ar_pack_int4 needs bits == 4 (got %d)", cfg->bits);
+  const int g = cfg->group_size;
+  if (!pow2(g) || g < 8 || g > 1024) return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 8..1024", g);
+  if (N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "N, K must be positive");
+  if (K % g != 0 || K % 8 != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and of 8");
+  const void* ptrs[] = {W, V, alpha, beta, packed, scale_f16, zero_f16};
+  for (const void* p : ptrs) {
+    if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  cudaError_t e = launch_pack_int4(W, V, alpha, beta, N, K, g, cfg->symmetric, packed, scale_f16, zero_f16,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return end_call();
+}
+
+ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, const uint16_t* scale_f16,
+                        const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, uint16_t* out,
+                        ar_stream_t stream) {
+  begin_call();
+  if (T < 1 || N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "T, N, K must be positive");
+  if (T > 16) return fail(AR_ERR_UNSUPPORTED, "T=%lld: this build supports 1 <= T <= 16", (long long)T);
+  if (!pow2(group_size) || group_size < 32 || group_size > 1024)
+    return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 32..1024", group_size);
+  if (K % group_size != 0 || K % 32 != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and 32");
+  if (N > INT32_MAX || K > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  const void* ptrs[] = {A, packed, scale_f16, zero_f16, out};
+  for (const void* p : ptrs) {
+    if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  cudaError_t e = launch_w4a16(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N),
+                               static_cast<int>(K), group_size, out, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16 launch");
+  return end_call();
+}
+
+ar_status ar_gemm_bf16(const uint16_t* A, int a_mn_major, const uint16_t* B, int b_mn_major, float* D, int64_t M,
+                       int64_t N, int64_t K, ar_stream_t stream) {
+  begin_call();
+  if (M <= 0 || N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "sizes must be positive");
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  if (N % 8 != 0 || K % 8 != 0 || (a_mn_major && M % 8 != 0))
+    return fail(AR_ERR_INVALID_ARG, "row strides must be multiples of 16 bytes");
+  if (!A || !B || !D) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaError_t e = launch_gemm_plain(A, a_mn_major != 0, B, b_mn_major != 0, D, static_cast<int>(M),
+                                    static_cast<int>(N), static_cast<int>(K), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return end_call();
+}
+
+ar_status ar_get_device_status(ar_stream_t stream) {
+  unsigned int v = 0;
+  cudaError_t e = read_and_clear_status(&v, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(AR_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  if (v & kStatusTimeout) return fail(AR_ERR_TIMEOUT, "a pipeline wait timed out on the device");
+  if (v & kStatusNonFinite) return fail(AR_ERR_NONFINITE, "non-finite value seen on the device");
+  return AR_OK;
+}
+
+const char* ar_last_error(void) { return t_error.c_str(); }
+
+const char* ar_last_kernels(void) { return t_kernels_last.c_str(); }
+
+const char* ar_version(void) { return "autoround-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,559 @@
+// Tensor-core GEMMs of the AutoRound tuning step on sm_100a (tcgen05 + TMEM + TMA).
+//
+// The step ([AR] §3 "Algorithm Flow", steps 2-5) has two dense contractions
+// per linear layer: the QDQ forward Y_hat = X W_hat^T and the weight gradient
+// dW_hat = G^T X.  Both run in one persistent, warp-specialised kernel
+// template; what differs is operand major-ness and the fused epilogue:
+//
+//   EPI_STORE  D (fp32) = A B^T                          (reference forward, tests)
+//   EPI_RESID  R = A B^T - Y; G = bf16(R * 2/(MN)); per-tile sum R^2
+//              (MSE loss and its gradient, [AR] §3 step 4)
+//   EPI_FOLD   straight-through fold of dW_hat into dV (per element) and
+//              dalpha/dbeta (per group), then the SignSGD step and clamp
+//              ([AR] §3 "SignSGD"; STE as in [IA])
+//
+// ([AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
+// Architectural Optimizations of AutoRound"; [IA] = "Intel AutoRound 高级量化".)
+//
+// Block: 192 threads.  Warp 0 lane 0 issues TMA loads into a 4-stage ring
+// (128x64 A tile, 256x64 B tile, 128-byte swizzle); warp 1 allocates 512 TMEM
+// columns (two 128x256 fp32 accumulators) and lane 0 issues
+// tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16); warps 2-5 drain
+// an accumulator with tcgen05.ld (warp w reads TMEM lanes 32*(w%4)..+31, i.e.
+// one output row per thread) while the MMA warp fills the other one.  The
+// grid is persistent: one CTA per SM, tiles strided by gridDim.x with the
+// N index fastest so that concurrently running CTAs share the A panel.
+//
+// Operands: A is [M][K] (K-major) or [K][M] (MN-major); B is [N][K] or [K][N].
+// The weight-gradient GEMM reads G [tokens][N_w] and X [tokens][K_w] directly
+// as MN-major operands, so no transpose is ever materialised.
+//
+// Every mbarrier wait is bounded (ar_device.cuh): on a timeout the kernel
+// raises a block abort flag and the sticky device status, all roles leave
+// their loops, in-flight TMA copies and MMAs are drained, TMEM is freed.
+#include "ar_internal.h"
+
+namespace ar {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int kThreads = 192;
+constexpr int kAStage = BM * BK * 2;  // 16 KiB
+constexpr int kBStage = BN * BK * 2;  // 32 KiB
+constexpr int kTmemCols = 2 * BN;     // double-buffered accumulator
+constexpr int kSmemBytes = STAGES * (kAStage + kBStage) + 1024 + 256;
+
+enum { EPI_STORE = 0, EPI_RESID = 1, EPI_FOLD = 2 };
+
+struct Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Ctl) <= 256, "control block too large");
+
+struct Params {
+  int M, N, K;  // D is M x N, reduction over K
+  int tiles_m, tiles_n, num_kb;
+  float* D;          // EPI_STORE
+  const float* Y;    // EPI_RESID
+  uint16_t* G;
+  float gscale;
+  double* partial;
+  FoldArgs fold;     // EPI_FOLD
+};
+
+// Byte offsets of the MN-major canonical layout: the leading-dimension offset
+// steps between 64-element (128 B) chunks of the contiguous dimension, which
+// are 8 KiB apart (one 64-row TMA box each); the stride-dimension offset steps
+// between 8-row groups along K, 1 KiB apart.
+constexpr uint32_t kMnLbo = 8192;
+constexpr uint32_t kMnSbo = 1024;
+
+template <bool MN>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t stage_base, int kstep) {
+  if (MN) {
+    // K-step of 16 rows = two 8-row core groups = 2 KiB further.
+    return sdesc_sw128(stage_base + kstep * 2048, kMnLbo, kMnSbo);
+  } else {
+    // K-major: a K-step of 16 bf16 is 32 bytes inside the 128-byte swizzle atom.
+    return sdesc_sw128(stage_base + kstep * 32, 16, 1024);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// epilogues: one thread = one output row, 32 columns per TMEM load
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void epi_store(const Params& p, uint32_t taddr, int row, int col_base) {
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    const int col0 = col_base + c * 32;
+    if (row >= p.M || col0 >= p.N) continue;
+    float* d = p.D + static_cast<size_t>(row) * p.N + col0;
+    if (col0 + 32 <= p.N) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<float4*>(d + 4 * i) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+      for (int i = 0; i < 32 && col0 + i < p.N; ++i) d[i] = v[i];
+    }
+  }
+}
+
+__device__ __forceinline__ double epi_resid(const Params& p, uint32_t taddr, int row, int col_base) {
+  double acc = 0.0;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    const int col0 = col_base + c * 32;
+    if (row >= p.M || col0 >= p.N) continue;
+    const float* y = p.Y + static_cast<size_t>(row) * p.N + col0;
+    uint16_t* g = p.G + static_cast<size_t>(row) * p.N + col0;
+    float part = 0.0f;
+    if (col0 + 32 <= p.N) {
+      uint32_t gp[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 yv = *reinterpret_cast<const float4*>(y + 4 * i);
+        const float r0 = __fsub_rn(v[4 * i + 0], yv.x);
+        const float r1 = __fsub_rn(v[4 * i + 1], yv.y);
+        const float r2 = __fsub_rn(v[4 * i + 2], yv.z);
+        const float r3 = __fsub_rn(v[4 * i + 3], yv.w);
+        part += r0 * r0 + r1 * r1 + r2 * r2 + r3 * r3;
+        gp[2 * i] = pack_bf16x2(__fmul_rn(r0, p.gscale), __fmul_rn(r1, p.gscale));
+        gp[2 * i + 1] = pack_bf16x2(__fmul_rn(r2, p.gscale), __fmul_rn(r3, p.gscale));
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4*>(g + 8 * i) = make_uint4(gp[4 * i], gp[4 * i + 1], gp[4 * i + 2], gp[4 * i + 3]);
+    } else {
+      for (int i = 0; i < 32 && col0 + i < p.N; ++i) {
+        const float r = __fsub_rn(v[i], y[i]);
+        part += r * r;
+        __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(r, p.gscale));
+        g[i] = *reinterpret_cast<uint16_t*>(&h);
+      }
+    }
+    acc += static_cast<double>(part);
+  }
+  return acc;
+}
+
+__device__ __forceinline__ float sign_step(float p, float d, float lr, float lo, float hi) {
+  float r = p;
+  if (d > 0.0f) r = __fsub_rn(p, lr);
+  else if (d < 0.0f) r = __fadd_rn(p, lr);
+  return fminf(fmaxf(r, lo), hi);
+}
+
+// Straight-through fold + SignSGD.  GEMM rows are weight rows n (M = N_w),
+// GEMM columns are weight columns k (N = K_w).  A group of g >= 32 columns
+// spans g/32 consecutive TMEM loads of this thread, so its sums are local.
+__device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n, int col_base) {
+  const FoldArgs& f = p.fold;
+  const int g = f.group_size;
+  const int cpg = g >> 5;
+  const int groups_per_row = p.N / g;
+  const float Q = static_cast<float>((1 << f.bits) - 1);
+  const float Qs = static_cast<float>((1 << (f.bits - 1)) - 1);
+  bool bad = false;
+  float s = 1.f, zp = 0.f, lo_s = 0.f, mx = 0.f, mn = 0.f, al = 1.f, be = 1.f, csum = 0.f, osum = 0.f;
+  bool guarded = false, take_hi = true;
+  size_t gidx = 0;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float gw[32];
+    tmem_ld32(taddr + c * 32, gw);
+    const int col0 = col_base + c * 32;
+    if (n >= p.M || col0 >= p.N) continue;
+    if ((c % cpg) == 0) {
+      gidx = static_cast<size_t>(n) * groups_per_row + col0 / g;
+      s = f.s[gidx];
+      zp = f.zp[gidx];
+      mx = f.mx[gidx];
+      mn = f.mn[gidx];
+      al = f.alpha[gidx];
+      be = f.beta[gidx];
+      const float hi = __fmul_rn(al, mx);
+      const float lo = __fmul_rn(be, mn);
+      const float s_raw = f.symmetric ? __fdiv_rn(fmaxf(hi, -lo), Qs) : __fdiv_rn(__fsub_rn(hi, lo), Q);
+      guarded = s_raw < kScaleGuard;
+      take_hi = hi >= -lo;
+      lo_s = __fdiv_rn(lo, s);
+      csum = 0.f;
+      osum = 0.f;
+    }
+    const size_t e = static_cast<size_t>(n) * p.N + col0;
+    const uint16_t* wp = f.W + e;
+    float* vp = f.V + e;
+    uint32_t wr[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 t = *reinterpret_cast<const uint4*>(wp + 8 * i);
+      wr[4 * i] = t.x;
+      wr[4 * i + 1] = t.y;
+      wr[4 * i + 2] = t.z;
+      wr[4 * i + 3] = t.w;
+    }
+    float vv[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 t = *reinterpret_cast<const float4*>(vp + 4 * i);
+      vv[4 * i] = t.x;
+      vv[4 * i + 1] = t.y;
+      vv[4 * i + 2] = t.z;
+      vv[4 * i + 3] = t.w;
+    }
+    float dv[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float w = (i & 1) ? bf16_hi(wr[i >> 1]) : bf16_lo(wr[i >> 1]);
+      const float wq = __fdiv_rn(w, s);
+      const float t = __fadd_rn(roundf(__fadd_rn(wq, vv[i])), zp);
+      const bool in = (t >= 0.0f) && (t <= Q);
+      const float qz = __fsub_rn(fminf(fmaxf(t, 0.0f), Q), zp);
+      const float gi = gw[i];
+      bad |= !isfinite(gi);
+      dv[i] = in ? __fmul_rn(gi, s) : 0.0f;
+      float ci;
+      if (f.symmetric) ci = __fmul_rn(gi, in ? __fsub_rn(qz, wq) : qz);
+      else ci = __fmul_rn(gi, __fsub_rn(qz, in ? wq : lo_s));
+      csum = __fadd_rn(csum, ci);
+      if (!in) osum = __fadd_rn(osum, gi);
+      vv[i] = sign_step(vv[i], dv[i], f.lr, f.v_min, f.v_max);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<float4*>(vp + 4 * i) = make_float4(vv[4 * i], vv[4 * i + 1], vv[4 * i + 2], vv[4 * i + 3]);
+    if (f.dV_out) {
+      float* dp = f.dV_out + e;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<float4*>(dp + 4 * i) = make_float4(dv[4 * i], dv[4 * i + 1], dv[4 * i + 2], dv[4 * i + 3]);
+    }
+    if ((c % cpg) == cpg - 1) {
+      if (guarded) csum = 0.0f;
+      float dhi, dlo;
+      if (f.symmetric) {
+        const float ds = __fdiv_rn(csum, Qs);
+        dhi = take_hi ? ds : 0.0f;
+        dlo = take_hi ? 0.0f : -ds;
+      } else {
+        const float cq = __fdiv_rn(csum, Q);
+        dhi = cq;
+        dlo = __fsub_rn(osum, cq);
+      }
+      const float da = __fmul_rn(mx, dhi);
+      const float db = __fmul_rn(mn, dlo);
+      bad |= !isfinite(da) || !isfinite(db);
+      f.alpha[gidx] = sign_step(al, da, f.lr, f.c_min, f.c_max);
+      f.beta[gidx] = sign_step(be, db, f.lr, f.c_min, f.c_max);
+      if (f.da_out) f.da_out[gidx] = da;
+      if (f.db_out) f.db_out[gidx] = db;
+    }
+  }
+  return bad;
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+template <bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smA = base;
+  uint8_t* smB = base + STAGES * kAStage;
+  Ctl* ctl = reinterpret_cast<Ctl*>(smB + STAGES * kBStage);
+  volatile int* abort_flag = &ctl->abort_flag;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_tiles = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&ctl->tmem_full[a], 1);
+      mbar_init(&ctl->tmem_empty[a], 4);
+    }
+    mbar_init(&ctl->mma_done, 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        const int tm = t / p.tiles_n;
+        const int tn = t - tm * p.tiles_n;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl->full[stage], kAStage + kBStage);
+          uint8_t* a_dst = smA + stage * kAStage;
+          uint8_t* b_dst = smB + stage * kBStage;
+          if (A_MN) {
+#pragma unroll
+            for (int i = 0; i < BM / 64; ++i) tma_load_2d(a_dst + i * 8192, &tmA, &ctl->full[stage], tm * BM + 64 * i, kb * BK);
+          } else {
+            tma_load_2d(a_dst, &tmA, &ctl->full[stage], kb * BK, tm * BM);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i) tma_load_2d(b_dst + i * 8192, &tmB, &ctl->full[stage], tn * BN + 64 * i, kb * BK);
+          } else {
+            tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, tn * BN);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: every issued copy must have landed before the CTA may exit.
+      const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+      for (uint32_t i = first; i < issued; ++i) mbar_wait_drain(&ctl->full[i % STAGES], (i / STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        if (!mbar_wait(&ctl->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&ctl->full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smA + stage * kAStage);
+          const uint32_t b_base = smem_u32(smB + stage * kBStage);
+#pragma unroll
+          for (int j = 0; j < BK / 16; ++j) {
+            umma_bf16(d, operand_desc<A_MN>(a_base, j), operand_desc<B_MN>(b_base, j), idesc,
+                      (kb | j) != 0 ? 1u : 0u);
+          }
+          umma_commit(&ctl->empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&ctl->tmem_full[acc]);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // All issued MMAs must be complete before TMEM is released.
+      umma_commit(&ctl->mma_done);
+      mbar_wait_drain(&ctl->mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    uint32_t acc = 0, acc_phase = 0;
+    double loss_acc = 0.0;
+    bool bad = false;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const bool got = mbar_wait(&ctl->tmem_full[acc], acc_phase, abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
+      tc_fence_after();
+      const int tm = t / p.tiles_n;
+      const int tn = t - tm * p.tiles_n;
+      const int row = tm * BM + quarter * 32 + lane;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+      if (EPI == EPI_STORE) {
+        epi_store(p, taddr, row, tn * BN);
+      } else if (EPI == EPI_RESID) {
+        double part = epi_resid(p, taddr, row, tn * BN);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
+        if (lane == 0) p.partial[static_cast<size_t>(t) * 4 + quarter] = part;
+        (void)loss_acc;
+      } else {
+        bad |= epi_fold(p, taddr, row, tn * BN);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->tmem_empty[acc]);
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (bad) raise_status(kStatusNonFinite);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 matrix [rows][cols] (cols contiguous), box of box_rows x 64 columns, 128-byte swizzle.
+cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t stream, const char* name) {
+  CUtensorMap tmA, tmB;
+  // A: K-major [M][K] with 128-row boxes, or MN-major [K][M] with 64-row boxes.
+  cudaError_t e = A_MN ? make_tmap(&tmA, A, p.K, p.M, 64) : make_tmap(&tmA, A, p.M, p.K, BM);
+  if (e != cudaSuccess) return e;
+  e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64) : make_tmap(&tmB, B, p.N, p.K, BN);
+  if (e != cudaSuccess) return e;
+  p.tiles_m = (p.M + BM - 1) / BM;
+  p.tiles_n = (p.N + BN - 1) / BN;
+  p.num_kb = (p.K + BK - 1) / BK;
+  auto kern = umma_gemm_kernel<A_MN, B_MN, EPI>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+  trace_kernel(name);
+  return cudaGetLastError();
+}
+
+// One block per step; the partial sums of a step are added in a fixed order.
+__global__ void loss_reduce_kernel(const double* __restrict__ partial, int n, double inv_count,
+                                   float* __restrict__ loss) {
+  __shared__ double sh[256];
+  partial += static_cast<size_t>(blockIdx.x) * n;
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < n; i += 256) acc += partial[i];
+  sh[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) sh[threadIdx.x] += sh[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) loss[blockIdx.x] = static_cast<float>(sh[0] * inv_count);
+}
+
+}  // namespace
+
+int resid_partials(int M, int N) { return ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * 4; }
+
+cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,
+                              cudaStream_t stream) {
+  Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.D = Y;
+  return run<false, false, EPI_STORE>(X, W, p, stream, "umma_gemm<K,K,store>");
+}
+
+cudaError_t launch_gemm_resid(const uint16_t* X, const uint16_t* W_hat, const float* Y, uint16_t* G, float gscale,
+                              double* loss_partial, int M, int N, int K, cudaStream_t stream) {
+  Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.Y = Y;
+  p.G = G;
+  p.gscale = gscale;
+  p.partial = loss_partial;
+  return run<false, false, EPI_RESID>(X, W_hat, p, stream, "umma_gemm<K,K,resid>");
+}
+
+cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArgs& fa, int M, int N, int K,
+                             cudaStream_t stream) {
+  // dW_hat[N_w][K_w] = G[tokens][N_w]^T X[tokens][K_w]: GEMM M = N_w, N = K_w, reduction = tokens.
+  Params p{};
+  p.M = N;
+  p.N = K;
+  p.K = M;
+  p.fold = fa;
+  return run<true, true, EPI_FOLD>(G, X, p, stream, "umma_gemm<MN,MN,fold>");
+}
+
+cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, bool b_mn, float* D, int M, int N,
+                              int K, cudaStream_t stream) {
+  Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.D = D;
+  if (!a_mn && !b_mn) return run<false, false, EPI_STORE>(A, B, p, stream, "umma_gemm<K,K,store>");
+  if (!a_mn && b_mn) return run<false, true, EPI_STORE>(A, B, p, stream, "umma_gemm<K,MN,store>");
+  if (a_mn && !b_mn) return run<true, false, EPI_STORE>(A, B, p, stream, "umma_gemm<MN,K,store>");
+  return run<true, true, EPI_STORE>(A, B, p, stream, "umma_gemm<MN,MN,store>");
+}
+
+cudaError_t launch_loss_reduce(const double* partials, int n, int steps, double inv_count, float* loss,
+                               cudaStream_t stream) {
+  loss_reduce_kernel<<<steps, 256, 0, stream>>>(partials, n, inv_count, loss);
+  trace_kernel("loss_reduce_kernel");
+  return cudaGetLastError();
+}
+
+}  // namespace ar

@@ -1,0 +1,78 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ar_device.cuh"
+
+namespace ar {
+
+constexpr float kScaleGuard = 1e-8f;  // lower bound on a group's scale
+
+// Records the name of a kernel launched by the current API call (tracing).
+void trace_kernel(const char* name);
+
+int num_sms();
+
+cudaError_t launch_qdq(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                       int64_t K, int group_size, int bits, int symmetric, uint16_t* W_hat, uint8_t* codes,
+                       float* scale, float* zero, float* mx, float* mn, cudaStream_t stream);
+
+cudaError_t launch_pack_int4(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                             int64_t K, int group_size, int symmetric, uint32_t* packed, uint16_t* scale16,
+                             uint16_t* zero16, cudaStream_t stream);
+
+cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t stream);
+
+// ---- tensor-core GEMMs (ar_gemm.cu) ----
+struct FoldArgs {
+  const uint16_t* W;  // bf16 [N][K] original weights
+  float* V;           // fp32 [N][K], updated in place
+  float* alpha;       // fp32 [N][G], updated in place
+  float* beta;        // fp32 [N][G], updated in place
+  const float* s;     // fp32 [N][G] from the QDQ of this step
+  const float* zp;
+  const float* mx;
+  const float* mn;
+  float* dV_out;      // optional gradient outputs
+  float* da_out;
+  float* db_out;
+  int group_size, bits, symmetric;
+  float lr, v_min, v_max, c_min, c_max;
+};
+
+// Y[M][N] fp32 = X[M][K] * W[N][K]^T (both K-major bf16).
+cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,
+                              cudaStream_t stream);
+
+// Forward of the tuning step with the residual epilogue:
+//   R = X W_hat^T - Y, G = bf16(R * gscale), partial[tile*4+warp] = sum R^2 (fp64).
+cudaError_t launch_gemm_resid(const uint16_t* X, const uint16_t* W_hat, const float* Y, uint16_t* G, float gscale,
+                              double* loss_partial, int M, int N, int K, cudaStream_t stream);
+int resid_partials(int M, int N);
+
+// Backward of the tuning step: dW_hat = G^T X (reduction over the M tokens),
+// folded through the straight-through estimator and applied as a SignSGD step.
+cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArgs& fa, int M, int N, int K,
+                             cudaStream_t stream);
+
+// Plain D[M][N] fp32 = op(A) op(B)^T, with A given K-major ([M][K]) or
+// MN-major ([K][M]) and B given K-major ([N][K]) or MN-major ([K][N]).
+cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, bool b_mn, float* D, int M, int N,
+                              int K, cudaStream_t stream);
+
+// Fixed-order reduction of the loss partials, `n` per step for `steps` steps:
+// loss[i] = sum(partials[i*n .. i*n+n)) * inv_count.
+cudaError_t launch_loss_reduce(const double* partials, int n, int steps, double inv_count, float* loss,
+                               cudaStream_t stream);
+
+// Synchronizes `stream`, copies the sticky device status to *out and clears it.
+cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t stream);
+
+// ---- W4A16 (ar_w4a16.cu) ----
+cudaError_t launch_w4a16(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                         const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream);
+
+}  // namespace ar

@@ -1,0 +1,127 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared
+entry point, and rejects invalid arguments before any device work.
+
+No call here reaches a kernel: every argument set below fails host-side
+validation, so these run without a GPU (pointers are fake, never touched).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import post_weight_quantization_autoround_b200 as ar
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "autoround.h")
+
+pytestmark = pytest.mark.skipif(not os.path.exists(ar.library_path), reason="libautoround.so not built")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^AR_API\s+[\w\s\*]+?\b(ar_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_four_hot_path_entry_points():
+    syms = declared_symbols()
+    for name in ["ar_qdq", "ar_tune_step", "ar_pack_int4", "ar_w4a16_gemm"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(ar.library_path)
+    missing = [s for s in declared_symbols() if not hasattr(L, s)]
+    assert not missing, missing
+    # the binding wraps every exported entry point under the same name
+    for s in declared_symbols():
+        assert hasattr(ar, s), s
+
+
+def test_defaults_follow_the_pages():
+    cfg = ar.ar_qconfig_default()
+    assert (cfg.bits, cfg.group_size, cfg.symmetric, cfg.iters) == (4, 128, 0, 200)
+    assert cfg.lr == pytest.approx(0.005)
+    assert (cfg.v_min, cfg.v_max, cfg.clip_min, cfg.clip_max) == (-0.5, 0.5, 0.5, 1.0)
+    assert "sm_100a" in ar.ar_version()
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced
+
+
+def qdq_raw(cfg, N=8, K=128, W=FAKE, V=FAKE, a=FAKE, b=FAKE, out=FAKE):
+    return ar.lib().ar_qdq(W, V, a, b, N, K, ctypes.byref(cfg), out, None, None, None, None)
+
+
+@pytest.mark.parametrize("bits", [1, 9, 0])
+def test_qdq_rejects_unsupported_bits(bits):
+    assert qdq_raw(ar.ar_qconfig_default(bits=bits)) == ar.AR_ERR_UNSUPPORTED
+    assert "bits" in ar.ar_last_error()
+
+
+def test_qdq_rejects_bad_shapes_and_pointers():
+    cfg = ar.ar_qconfig_default()
+    assert qdq_raw(cfg, K=100) == ar.AR_ERR_INVALID_ARG  # K % g != 0
+    assert qdq_raw(cfg, N=0) == ar.AR_ERR_INVALID_ARG
+    assert qdq_raw(cfg, W=FAKE + 2) == ar.AR_ERR_INVALID_ARG  # misaligned
+    assert qdq_raw(cfg, V=None) == ar.AR_ERR_INVALID_ARG
+    assert qdq_raw(cfg, out=None) == ar.AR_ERR_INVALID_ARG  # nothing requested
+    assert qdq_raw(ar.ar_qconfig_default(group_size=96), K=192) == ar.AR_ERR_UNSUPPORTED
+    assert qdq_raw(ar.ar_qconfig_default(symmetric=2)) == ar.AR_ERR_INVALID_ARG
+    assert qdq_raw(ar.ar_qconfig_default(lr=float("nan"))) == ar.AR_ERR_INVALID_ARG
+    assert qdq_raw(ar.ar_qconfig_default(v_min=1.0, v_max=0.0)) == ar.AR_ERR_INVALID_ARG
+
+
+def _tune_raw(cfg, N=256, K=256, M=32, ws_bytes=1 << 40, X=FAKE, Y=FAKE, loss=FAKE, n_steps=1, ws=0x100000):
+    layer = ar.Layer(FAKE, FAKE, FAKE, FAKE, N, K)
+    return ar.lib().ar_tune_step(0, ctypes.byref(layer), 1, X, M, Y, ctypes.byref(cfg), n_steps, loss, None, ws,
+                                 ws_bytes, None)
+
+
+def test_tune_step_validation():
+    cfg = ar.ar_qconfig_default()
+    assert _tune_raw(ar.ar_qconfig_default(group_size=16)) == ar.AR_ERR_UNSUPPORTED
+    assert _tune_raw(ar.ar_qconfig_default(group_size=512), K=1024) == ar.AR_ERR_UNSUPPORTED
+    assert _tune_raw(cfg, N=100) == ar.AR_ERR_INVALID_ARG  # N % 8
+    assert _tune_raw(cfg, K=200) == ar.AR_ERR_INVALID_ARG  # K % g
+    assert _tune_raw(cfg, Y=None) == ar.AR_ERR_INVALID_ARG
+    assert _tune_raw(cfg, n_steps=-1) == ar.AR_ERR_INVALID_ARG
+    assert _tune_raw(cfg, ws_bytes=16) == ar.AR_ERR_WORKSPACE
+    assert _tune_raw(cfg, ws=0x100010) == ar.AR_ERR_INVALID_ARG  # workspace alignment
+    layer = ar.Layer(FAKE, FAKE, FAKE, FAKE, 256, 256)
+    bad_kind = ar.lib().ar_tune_step(7, ctypes.byref(layer), 1, FAKE, 32, FAKE, ctypes.byref(cfg), 1, FAKE, None,
+                                     0x100000, 1 << 40, None)
+    assert bad_kind == ar.AR_ERR_UNSUPPORTED
+
+
+def test_workspace_size_grows_with_steps_and_tokens():
+    cfg = ar.ar_qconfig_default()
+    layer = ar.Layer(FAKE, FAKE, FAKE, FAKE, 4096, 4096)
+    f = ar.lib().ar_tune_step_workspace
+    w1 = f(0, ctypes.byref(layer), 1, 16384, ctypes.byref(cfg), 1)
+    w200 = f(0, ctypes.byref(layer), 1, 16384, ctypes.byref(cfg), 200)
+    w_small = f(0, ctypes.byref(layer), 1, 2048, ctypes.byref(cfg), 1)
+    # W_hat (N K bf16) + G (M N bf16) + four per-group arrays + loss partials
+    assert w1 >= 4096 * 4096 * 2 + 16384 * 4096 * 2 + 4 * 4096 * 32 * 4
+    assert w200 > w1 > w_small > 0
+    assert f(5, ctypes.byref(layer), 1, 16384, ctypes.byref(cfg), 1) == 0
+
+
+def test_pack_and_w4a16_validation():
+    cfg3 = ar.ar_qconfig_default(bits=3)
+    assert ar.lib().ar_pack_int4(FAKE, FAKE, FAKE, FAKE, 8, 128, ctypes.byref(cfg3), FAKE, FAKE, FAKE, None) == \
+        ar.AR_ERR_UNSUPPORTED
+    w4 = ar.lib().ar_w4a16_gemm
+    assert w4(FAKE, 17, FAKE, FAKE, FAKE, 64, 256, 128, FAKE, None) == ar.AR_ERR_UNSUPPORTED
+    assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 16, FAKE, None) == ar.AR_ERR_UNSUPPORTED
+    assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 200, 128, FAKE, None) == ar.AR_ERR_INVALID_ARG
+    assert w4(FAKE, 0, FAKE, FAKE, FAKE, 64, 256, 128, FAKE, None) == ar.AR_ERR_INVALID_ARG
+    assert ar.lib().ar_linear_forward(FAKE, 32, FAKE, 100, 256, FAKE, None) == ar.AR_ERR_INVALID_ARG
+    assert ar.lib().ar_gemm_bf16(FAKE, 1, FAKE, 0, FAKE, 12, 64, 64, None) == ar.AR_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+
+    with pytest.raises(ar.ARError):
+        ar.ar_f32_to_bf16(torch.zeros(8), torch.zeros(8, dtype=torch.bfloat16))
