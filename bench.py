@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""AutoRound tuning-step benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one SignSGD tuning step of a Llama-7B-shaped 4096x4096 linear layer
+on 8 samples x 2048 tokens (16384 tokens), W4 asymmetric, group 128, lr 5e-3:
+QDQ -> forward GEMM with the MSE residual epilogue -> weight-gradient GEMM with
+the straight-through fold and SignSGD update fused in.  Inputs are seeded
+synthetic tensors (weights ~N(0, 0.02) with 0.1 % outliers x20, activations
+~N(0, 1) with 8 outlier channels x50) standing in for trained weights and
+calibration text.
+
+Prints ONE JSON line (rank 0).  ``value`` is tuning steps/s of the whole job
+(N ranks each tune their own independent layer: weak scaling, no collective on
+the data path).  Extra keys: ``roofline`` (dominant kernel vs the measured bf16
+peak), ``cpu_baseline`` (the CPU oracle on a bounded row sample), ``e2e``
+(the same metric through the host-buffer API with copies inside the timed
+region), ``gpu_launches``, ``clocks``, ``kernels`` (per-kernel device time)
+and ``w4a16`` (the INT4 decode matmul on the 8192x28672 down projection).
+
+``--impl reference`` times the CPU oracle itself on the host cores (rank 0
+only), on row samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "AutoRound tuning steps/s per layer (TFLOP/s, % bf16 roofline); W4A16 GEMV % HBM BW"
+WORKLOAD = "linear_4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SAMPLE_ROWS_CPU = 128
+SAMPLE_ROWS_REF = 128
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(wl, n_gpus):
+    return {
+        "workload": f"{wl.name}: {wl.n_out}x{wl.n_in} bf16 linear, {wl.m_tokens} tokens (8x2048), "
+                    f"W{wl.bits} asym g{wl.group_size}, lr {wl.lr}, one SignSGD step per iteration",
+        "n_out": wl.n_out, "n_in": wl.n_in, "tokens": wl.m_tokens, "bits": wl.bits, "group_size": wl.group_size,
+        "lr": wl.lr, "layers": n_gpus, "parallelism": f"{n_gpus} independent layers, one per GPU",
+        "l2": "inputs larger than L2: X 134 MB and Y 268 MB per layer exceed the 126 MB L2; no flush needed",
+    }
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._handle = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report what is missing
+            self.error = str(e)
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._handle is not None:
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._handle is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self._handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "no NVML")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# traffic of the dominant kernel from the committed ncu summary
+# ----------------------------------------------------------------------------
+
+KERNEL_SOURCES = ["post_weight_quantization_autoround_b200/csrc/ar_gemm.cu",
+                  "post_weight_quantization_autoround_b200/csrc/ar_device.cuh"]
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_tag: str):
+    """dram bytes per launch recorded in profiles/, or None if missing or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}_{WORKLOAD}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_b = re.search(r"dram_bytes_per_launch\s*=\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"source_hash\s*=\s*([0-9a-f]+)", text)
+    if not m_b or not m_h or m_h.group(1) != gemm_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (rank 0, N = 1) and the reference arm
+# ----------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max(i.get("num_threads", 1) for i in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleSample:
+    """The oracle's tuning step on ``rows`` of the layer's output rows (rows are independent)."""
+
+    def __init__(self, wl, d, rows):
+        from oracle import autoround_oracle as O
+
+        self.O = O
+        self.wl = wl
+        idx = np.arange(rows)
+        self.W = synth.bf16_bits_to_f32(d["W"][idx])
+        self.X = synth.bf16_bits_to_f32(d["X"])
+        self.Y = O.reference_forward(self.X, self.W)
+        self.V, self.a, self.b = synth.make_state(rows, wl.n_in, wl.group_size)
+        self.cfg = O.QConfig(bits=wl.bits, group_size=wl.group_size, lr=wl.lr)
+        self.count = wl.m_tokens * wl.n_out
+        self.scale = wl.n_out / rows  # sample -> whole layer
+
+    def step(self):
+        _, (self.V, self.a, self.b), _, _ = self.O.tune_step_linear(self.W, self.X, self.Y, self.V, self.a, self.b,
+                                                                    self.cfg, count=self.count)
+
+
+def cpu_baseline(wl, d, budget_s=12.0):
+    s = OracleSample(wl, d, SAMPLE_ROWS_CPU)
+    s.step()  # warm
+    n, t0 = 0, time.perf_counter()
+    while True:
+        s.step()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    per_layer_step = el / n * s.scale
+    return {"value": 1.0 / per_layer_step, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} oracle steps on {SAMPLE_ROWS_CPU} of {wl.n_out} output rows (rows are independent), "
+                      f"{el:.1f} s, scaled x{s.scale:g} to the full layer"}
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    d = synth.make_linear(wl.n_out, wl.n_in, wl.m_tokens, seed=wl.seed)
+    s = OracleSample(wl, d, SAMPLE_ROWS_REF)
+    for _ in range(args.warmup):
+        s.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s.step()
+    el = time.perf_counter() - t0
+    value = args.steps / (el * s.scale)
+    sample = (f"each step: the oracle's SignSGD step on {SAMPLE_ROWS_REF} of {wl.n_out} output rows "
+              f"(exact, rows are independent), time scaled x{s.scale:g} to the full layer")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, 1),
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def to_dev_bf16(bits, torch):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def w4a16_bench(ar, torch, peaks, reps=20):
+    wl = synth.WORKLOADS["down_8192_28672"]
+    N, K, g = wl.n_out, wl.n_in, wl.group_size
+    d = synth.make_linear(N, K, 1, seed=wl.seed, x_outlier_channels=0)
+    Wd = to_dev_bf16(d["W"], torch)
+    V = torch.zeros((N, K), dtype=torch.float32, device="cuda")
+    a = torch.ones((N, K // g), dtype=torch.float32, device="cuda")
+    b = torch.ones((N, K // g), dtype=torch.float32, device="cuda")
+    cfg = ar.ar_qconfig_default(bits=4, group_size=g)
+    packed = torch.empty((N, K // 8), dtype=torch.int32, device="cuda")
+    s16 = torch.empty((N, K // g), dtype=torch.float16, device="cuda")
+    z16 = torch.empty((N, K // g), dtype=torch.float16, device="cuda")
+    ar.ar_pack_int4(Wd, V, a, b, cfg, packed, s16, z16)
+    del Wd, V
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    out = {}
+    for T in (1, 4, 16):
+        A = to_dev_bf16(synth.make_activations(T, K, seed=T), torch)
+        y = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            ar.ar_w4a16_gemm(A, packed, s16, z16, g, y)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in ev:
+            flush.zero_()  # evict the 117 MB of packed weights from L2
+            e0.record()
+            ar.ar_w4a16_gemm(A, packed, s16, z16, g, y)
+            e1.record()
+        torch.cuda.synchronize()
+        ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+        nbytes = packed.numel() * 4 + s16.numel() * 2 + z16.numel() * 2 + A.numel() * 2 + y.numel() * 2
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[f"T{T}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                        "algorithmic_bytes": nbytes, "kernel": ar.ar_last_kernels()}
+    out["shape"] = f"{N}x{K} int4 g{g}, fp16 scale/zero, bf16 activations; L2 flushed before each launch"
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-w4a16", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.WORKLOADS[WORKLOAD]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    import torch.distributed as dist
+
+    import post_weight_quantization_autoround_b200 as ar
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    peaks, peaks_src = load_peaks()
+
+    # --- inputs: each rank tunes its own independent layer (seed = rank)
+    d = synth.make_linear(wl.n_out, wl.n_in, wl.m_tokens, seed=wl.seed + rank)
+    cfg = ar.ar_qconfig_default(bits=wl.bits, group_size=wl.group_size, lr=wl.lr)
+    W = to_dev_bf16(d["W"], torch)
+    X = to_dev_bf16(d["X"], torch)
+    N, K, M, g = wl.n_out, wl.n_in, wl.m_tokens, wl.group_size
+    V = torch.zeros((N, K), dtype=torch.float32, device="cuda")
+    alpha = torch.ones((N, K // g), dtype=torch.float32, device="cuda")
+    beta = torch.ones((N, K // g), dtype=torch.float32, device="cuda")
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    ar.ar_linear_forward(X, W, Y)
+    ws = torch.empty(ar.ar_tune_step_workspace(W, V, alpha, beta, M, cfg, 1), dtype=torch.uint8, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+
+    def step():
+        ar.ar_tune_step(W, V, alpha, beta, X, Y, cfg, 1, loss, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ar.ar_get_device_status() != 0:
+        raise SystemExit(f"device status after warm-up: {ar.ar_last_error()}")
+
+    # --- timed region: exactly K steps, barrier + synchronize on both sides
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ar.ar_profile_start()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        prof = ar.ar_profile_stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = ar.ar_get_device_status()
+    final_loss = float(loss.item())
+
+    launches = sum(n for n, _ in prof.values())
+    kernels = {k: {"launches": n, "ms_total": t_ms, "us_per_launch": 1e3 * t_ms / max(n, 1),
+                   "share": t_ms / max(sum(x[1] for x in prof.values()), 1e-12)} for k, (n, t_ms) in prof.items()}
+    flops_gemm = 2.0 * M * N * K
+    flops_step = 2 * flops_gemm
+    steps_s_rank = args.steps / (ms * 1e-3)
+    value = world * args.steps / (ms * 1e-3)
+    gemm_names = [k for k in prof if k.startswith("umma_gemm")]
+    dom = max(gemm_names, key=lambda k: prof[k][1])
+    dom_us = kernels[dom]["us_per_launch"]
+    achieved = flops_gemm / (dom_us * 1e-6) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    tag = "fwd_gemm" if "resid" in dom else "wgrad_fold_gemm"
+    traffic = profiled_traffic(tag)
+    result = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; Llama-7B-shaped layer and calibration stand-ins)",
+        "config": workload_config(wl, world),
+        "tflops": flops_step * steps_s_rank / 1e12 * world,
+        "step_roofline_frac": (max(flops_step / (peak * 1e12), 0.0) * 1e3) / (ms / args.steps),
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
+                     "algorithmic_flops_per_launch": flops_gemm},
+        "gpu_launches": launches,
+        "kernels": kernels,
+        "clocks": clocks.summary(),
+        "device_status": status,
+        "final_loss": final_loss,
+    }
+
+    # --- end to end through the host-buffer API (pinned host tensors, copies timed)
+    if not args.no_e2e:
+        tuner = ar.LinearTuner(N, K, M, cfg, args.steps)
+        pin = lambda t: t.pin_memory()
+        Wh = pin(torch.from_numpy(d["W"].view(np.int16)).view(torch.bfloat16))
+        Xh = pin(torch.from_numpy(d["X"].view(np.int16)).view(torch.bfloat16))
+        Vh = pin(torch.zeros((N, K), dtype=torch.float32))
+        ah = pin(torch.ones((N, K // g), dtype=torch.float32))
+        bh = pin(torch.ones((N, K // g), dtype=torch.float32))
+        lh = pin(torch.empty(args.steps, dtype=torch.float32))
+        tuner.run_host(Wh, Xh, Vh.clone().pin_memory(), ah.clone().pin_memory(), bh.clone().pin_memory(), lh)
+        torch.cuda.synchronize()
+        Vw, aw, bw = Vh.clone().pin_memory(), ah.clone().pin_memory(), bh.clone().pin_memory()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        tuner.run_host(Wh, Xh, Vw, aw, bw, lh)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        result["e2e"] = {"value": world * args.steps / (e2e_ms * 1e-3), "unit": "steps/s",
+                         "h2d_bytes_per_step": tuner.h2d_bytes() / args.steps,
+                         "d2h_bytes_per_step": tuner.d2h_bytes() / args.steps,
+                         "job": f"per layer: copy W, X, V, alpha, beta in; reference forward; {args.steps} steps; "
+                                "copy V, alpha, beta and the losses out"}
+        del tuner
+
+    if rank == 0 and world == 1 and not args.no_w4a16:
+        result["w4a16"] = w4a16_bench(ar, torch, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, d)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -205,6 +205,15 @@ AR_API const char* ar_last_error(void);
  * separated by ';' (tracing: shows which kernel variant ran). */
 AR_API const char* ar_last_kernels(void);
 
+/* Device-time profiling.  Between ar_profile_start() and ar_profile_stop()
+ * every kernel launch of this library (any host thread) is bracketed by two
+ * CUDA events recorded on its launch stream.  ar_profile_stop() waits for
+ * those events and writes one line per kernel name into buf (NUL-terminated,
+ * truncated to buf_len):  "<kernel name> <launches> <total device ms>\n".
+ * Events come from a pool the library keeps; no device memory is allocated. */
+AR_API ar_status ar_profile_start(void);
+AR_API ar_status ar_profile_stop(char* buf, size_t buf_len);
+
 /* Library version string. */
 AR_API const char* ar_version(void);
 

@@ -19,7 +19,7 @@ __all__ = [
     "ARError", "QConfig", "Layer", "Grads", "lib", "library_path",
     "ar_qconfig_default", "ar_f32_to_bf16", "ar_qdq", "ar_linear_forward", "ar_tune_step_workspace",
     "ar_tune_step", "ar_pack_int4", "ar_w4a16_gemm", "ar_gemm_bf16", "ar_get_device_status",
-    "ar_last_error", "ar_last_kernels", "ar_version", "AR_BLOCK_LINEAR",
+    "ar_last_error", "ar_last_kernels", "ar_version", "ar_profile_start", "ar_profile_stop", "AR_BLOCK_LINEAR",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -74,6 +74,8 @@ _SIGNATURES = {
     "ar_last_error": (ctypes.c_char_p, []),
     "ar_last_kernels": (ctypes.c_char_p, []),
     "ar_version": (ctypes.c_char_p, []),
+    "ar_profile_start": (_INT, []),
+    "ar_profile_stop": (_INT, [ctypes.c_char_p, ctypes.c_size_t]),
 }
 
 
@@ -193,6 +195,61 @@ def ar_gemm_bf16(A, a_mn_major: bool, B, b_mn_major: bool, D, M: int, N: int, K:
                               _stream(stream)))
 
 
+def ar_profile_start() -> None:
+    _check(lib().ar_profile_start())
+
+
+def ar_profile_stop() -> dict:
+    """Stop device-time profiling; returns {kernel name: (launches, total ms)}."""
+    buf = ctypes.create_string_buffer(1 << 16)
+    _check(lib().ar_profile_stop(buf, len(buf)))
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, n, ms = line.rsplit(" ", 2)
+        out[name] = (int(n), float(ms))
+    return out
+
+
 def ar_get_device_status(stream=None) -> int:
     """Synchronise and return (and clear) the sticky device status code."""
     return int(lib().ar_get_device_status(_stream(stream)))
+
+
+class LinearTuner:
+    """Device buffers for tuning one linear layer from host memory (the end-to-end path).
+
+    ``run_host`` copies W, X and the state (V, alpha, beta) from pinned host
+    tensors to the device, computes the reference output, runs ``n_steps``
+    tuning steps and copies the tuned state and the per-step losses back into
+    the host tensors.  Device memory is allocated once here, so repeated runs
+    allocate nothing.
+    """
+
+    def __init__(self, N: int, K: int, M: int, cfg: QConfig, n_steps: int, device=None):
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        g = cfg.group_size
+        self.cfg, self.n_steps = cfg, n_steps
+        self.W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        self.X = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.V = torch.empty((N, K), dtype=torch.float32, device=dev)
+        self.alpha = torch.empty((N, K // g), dtype=torch.float32, device=dev)
+        self.beta = torch.empty((N, K // g), dtype=torch.float32, device=dev)
+        self.Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        self.loss = torch.empty(max(n_steps, 1), dtype=torch.float32, device=dev)
+        nbytes = ar_tune_step_workspace(self.W, self.V, self.alpha, self.beta, M, cfg, n_steps)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def h2d_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.W, self.X, self.V, self.alpha, self.beta))
+
+    def d2h_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.V, self.alpha, self.beta, self.loss))
+
+    def run_host(self, W, X, V, alpha, beta, loss, stream=None) -> None:
+        for dst, src in ((self.W, W), (self.X, X), (self.V, V), (self.alpha, alpha), (self.beta, beta)):
+            dst.copy_(src, non_blocking=True)
+        ar_linear_forward(self.X, self.W, self.Y, stream=stream)
+        ar_tune_step(self.W, self.V, self.alpha, self.beta, self.X, self.Y, self.cfg, self.n_steps, self.loss,
+                     self.workspace, stream=stream)
+        for dst, src in ((V, self.V), (alpha, self.alpha), (beta, self.beta), (loss, self.loss)):
+            dst.copy_(src, non_blocking=True)

@@ -4,7 +4,11 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+#include <map>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/autoround.h"
 #include "ar_internal.h"
@@ -108,6 +112,51 @@ ar_status check_linear(const ar_layer* layers, int n_layers, int64_t M, const ar
 void trace_kernel(const char* name) {
   if (!t_kernels.empty()) t_kernels += ";";
   t_kernels += name;
+}
+
+// ---- device-time profiler: events around every launch while enabled ----
+namespace {
+struct ProfRecord {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mu;
+std::vector<ProfRecord> g_prof_records;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  cudaEvent_t e = nullptr;
+  if (!g_event_pool.empty()) {
+    e = g_event_pool.back();
+    g_event_pool.pop_back();
+  } else if (cudaEventCreate(&e) != cudaSuccess) {
+    e = nullptr;
+  }
+  return e;
+}
+}  // namespace
+
+LaunchScope::LaunchScope(cudaStream_t stream, const char* name) : stream_(stream), name_(name), start_(nullptr) {
+  if (g_prof_on.load(std::memory_order_relaxed)) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    start_ = take_event();
+    if (start_) cudaEventRecord(start_, stream_);
+  }
+}
+
+LaunchScope::~LaunchScope() {
+  trace_kernel(name_);
+  if (start_) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t stop = take_event();
+    if (stop) {
+      cudaEventRecord(stop, stream_);
+      g_prof_records.push_back({name_, start_, stop});
+    } else {
+      g_event_pool.push_back(start_);
+    }
+  }
 }
 
 int num_sms() {
@@ -344,6 +393,51 @@ ar_status ar_get_device_status(ar_stream_t stream) {
   if (v & kStatusTimeout) return fail(AR_ERR_TIMEOUT, "a pipeline wait timed out on the device");
   if (v & kStatusNonFinite) return fail(AR_ERR_NONFINITE, "non-finite value seen on the device");
   return AR_OK;
+}
+
+ar_status ar_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (const ProfRecord& r : g_prof_records) {
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_prof_records.clear();
+  g_prof_on.store(true);
+  return AR_OK;
+}
+
+ar_status ar_profile_stop(char* buf, size_t buf_len) {
+  g_prof_on.store(false);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  std::map<std::string, std::pair<long, double>> agg;
+  ar_status st = AR_OK;
+  for (const ProfRecord& r : g_prof_records) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.stop);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.start, r.stop);
+    if (e != cudaSuccess) {
+      st = fail(AR_ERR_CUDA, "profile events: %s", cudaGetErrorString(e));
+      continue;
+    }
+    auto& a = agg[r.name];
+    a.first += 1;
+    a.second += ms;
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_prof_records.clear();
+  std::string out;
+  char line[256];
+  for (const auto& kv : agg) {
+    snprintf(line, sizeof(line), "%s %ld %.6f\n", kv.first.c_str(), kv.second.first, kv.second.second);
+    out += line;
+  }
+  if (buf && buf_len > 0) {
+    const size_t n = out.size() < buf_len - 1 ? out.size() : buf_len - 1;
+    memcpy(buf, out.data(), n);
+    buf[n] = 0;
+  }
+  return st;
 }
 
 const char* ar_last_error(void) { return t_error.c_str(); }

@@ -477,8 +477,10 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
-  trace_kernel(name);
+  {
+    LaunchScope scope(stream, name);
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+  }
   return cudaGetLastError();
 }
 
@@ -551,8 +553,10 @@ cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, b
 
 cudaError_t launch_loss_reduce(const double* partials, int n, int steps, double inv_count, float* loss,
                                cudaStream_t stream) {
-  loss_reduce_kernel<<<steps, 256, 0, stream>>>(partials, n, inv_count, loss);
-  trace_kernel("loss_reduce_kernel");
+  {
+    LaunchScope scope(stream, "loss_reduce_kernel");
+    loss_reduce_kernel<<<steps, 256, 0, stream>>>(partials, n, inv_count, loss);
+  }
   return cudaGetLastError();
 }
 

@@ -14,6 +14,22 @@ constexpr float kScaleGuard = 1e-8f;  // lower bound on a group's scale
 // Records the name of a kernel launched by the current API call (tracing).
 void trace_kernel(const char* name);
 
+// Wraps one kernel launch: traces its name and, while device profiling is on
+// (ar_profile_start), records CUDA events around it on the launch stream.
+// `name` must be a string literal.
+class LaunchScope {
+ public:
+  LaunchScope(cudaStream_t stream, const char* name);
+  ~LaunchScope();
+  LaunchScope(const LaunchScope&) = delete;
+  LaunchScope& operator=(const LaunchScope&) = delete;
+
+ private:
+  cudaStream_t stream_;
+  const char* name_;
+  cudaEvent_t start_;
+};
+
 int num_sms();
 
 cudaError_t launch_qdq(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,

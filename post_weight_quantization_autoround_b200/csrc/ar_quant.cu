@@ -226,9 +226,9 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ src, uint16_t* __re
   case (TPG_ * 8 * CH_): {                                                                                      \
     const int64_t threads = n_groups * TPG_;                                                                    \
     const int blocks = static_cast<int>((threads + 255) / 256);                                                 \
+    LaunchScope scope(stream, "qdq_kernel<g=" #TPG_ "x8x" #CH_ ">");                                           \
     qdq_kernel<TPG_, CH_><<<blocks, 256, 0, stream>>>(W, V, alpha, beta, n_groups, groups_per_row, bits,      \
                                                       symmetric, W_hat, codes, scale, zero, mx, mn);           \
-    trace_kernel("qdq_kernel<g=" #TPG_ "x8x" #CH_ ">");                                                        \
     break;                                                                                                      \
   }
 
@@ -257,10 +257,10 @@ cudaError_t launch_qdq(const uint16_t* W, const float* V, const float* alpha, co
   case (TPG_ * 8 * CH_): {                                                                                      \
     const int64_t threads = n_groups * TPG_;                                                                    \
     const int blocks = static_cast<int>((threads + 255) / 256);                                                 \
+    LaunchScope scope(stream, "pack_int4_kernel<g=" #TPG_ "x8x" #CH_ ">");                                     \
     pack_int4_kernel<TPG_, CH_><<<blocks, 256, 0, stream>>>(W, V, alpha, beta, n_groups, symmetric, packed,   \
                                                             reinterpret_cast<__half*>(scale16),                \
                                                             reinterpret_cast<__half*>(zero16));                \
-    trace_kernel("pack_int4_kernel<g=" #TPG_ "x8x" #CH_ ">");                                                  \
     break;                                                                                                      \
   }
 
@@ -289,8 +289,10 @@ cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaS
   int blocks = static_cast<int>((vec + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  f32_to_bf16_kernel<<<blocks, 256, 0, stream>>>(src, dst, n);
-  trace_kernel("f32_to_bf16_kernel");
+  {
+    LaunchScope scope(stream, "f32_to_bf16_kernel");
+    f32_to_bf16_kernel<<<blocks, 256, 0, stream>>>(src, dst, n);
+  }
   return cudaGetLastError();
 }
 

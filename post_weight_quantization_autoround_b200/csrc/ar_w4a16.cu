@@ -96,8 +96,10 @@ cudaError_t launch_w4a16(const uint16_t* A, int T, const uint32_t* packed, const
   const __half* s16 = reinterpret_cast<const __half*>(scale16);
   const __half* z16 = reinterpret_cast<const __half*>(zero16);
 #define AR_W4_CASE(TT)                                                                                 \
-  w4a16_kernel<TT><<<blocks, 256, 0, stream>>>(A, packed, s16, z16, N, K, group_shift, T, out);       \
-  trace_kernel("w4a16_kernel<T=" #TT ">");
+  {                                                                                                    \
+    LaunchScope scope(stream, "w4a16_kernel<T=" #TT ">");                                              \
+    w4a16_kernel<TT><<<blocks, 256, 0, stream>>>(A, packed, s16, z16, N, K, group_shift, T, out);     \
+  }
   if (T <= 1) {
     AR_W4_CASE(1)
   } else if (T <= 2) {
