@@ -164,6 +164,33 @@ AR_API ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_laye
                        const float* Y, const ar_qconfig* cfg, int n_steps, float* loss_per_step,
                        const ar_grads* grads, void* workspace, size_t workspace_bytes, ar_stream_t stream);
 
+/* Fixed scratch size of ar_tune_step_noalloc, in bytes (16 MiB per GPU). */
+#define AR_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+
+/* ar_tune_step without a caller workspace.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory —
+ * a process whose GPU memory is owned by another allocator (for example a
+ * framework's caching allocator that has reserved it), or a latency-critical
+ * loop that cannot take the implicit device synchronisation of
+ * cudaMalloc/cudaFree.  It runs exactly the kernels of ar_tune_step, with
+ * the same arguments minus the workspace, and allocates nothing: its scratch
+ * is one file-scope device array of AR_NOALLOC_SCRATCH_BYTES that every GPU
+ * loading this library holds until the process exits.
+ *  - Problems whose ar_tune_step_workspace() exceeds AR_NOALLOC_SCRATCH_BYTES
+ *    return AR_ERR_WORKSPACE with the sizes in ar_last_error(); at 4-bit g128
+ *    this admits e.g. a 1024x1024 layer with 2048 tokens, not a 4096x4096
+ *    layer with 16384 tokens.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; nothing in it needs to start at zero (each step writes every
+ *    scratch byte it later reads).  Calls that overlap on the GPU (other
+ *    streams, other host threads) race on the array: serialise them. */
+AR_API ar_status ar_tune_step_noalloc(int block_kind, const ar_layer* layers, int n_layers, const uint16_t* X,
+                                      int64_t M, const float* Y, const ar_qconfig* cfg, int n_steps,
+                                      float* loss_per_step, const ar_grads* grads, ar_stream_t stream);
+
 /* Export the tuned codes as INT4 ([AR] §4 comparison table, "Real INT4
  * Kernel" column: weights stored as 4-bit integers with per-group metadata).
  * Recomputes the codes exactly as ar_qdq does, then writes

@@ -20,6 +20,7 @@ __all__ = [
     "ar_qconfig_default", "ar_f32_to_bf16", "ar_qdq", "ar_linear_forward", "ar_tune_step_workspace",
     "ar_tune_step", "ar_pack_int4", "ar_w4a16_gemm", "ar_gemm_bf16", "ar_get_device_status",
     "ar_last_error", "ar_last_kernels", "ar_version", "ar_profile_start", "ar_profile_stop", "AR_BLOCK_LINEAR",
+    "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -74,6 +75,8 @@ _SIGNATURES = {
     "ar_last_error": (ctypes.c_char_p, []),
     "ar_last_kernels": (ctypes.c_char_p, []),
     "ar_version": (ctypes.c_char_p, []),
+    "ar_tune_step_noalloc": (_INT, [_INT, ctypes.POINTER(Layer), _INT, _P, _I64, _P, ctypes.POINTER(QConfig), _INT,
+                                    _P, ctypes.POINTER(Grads), _P]),
     "ar_profile_start": (_INT, []),
     "ar_profile_stop": (_INT, [ctypes.c_char_p, ctypes.c_size_t]),
 }
@@ -175,6 +178,24 @@ def ar_tune_step(W, V, alpha, beta, X, Y, cfg: QConfig, n_steps: int, loss, work
     _check(lib().ar_tune_step(block_kind, ctypes.byref(layer), 1, _ptr(X), X.shape[0], _ptr(Y), ctypes.byref(cfg),
                               n_steps, _ptr(loss), gp, _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)))
+
+
+AR_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def ar_tune_step_noalloc(W, V, alpha, beta, X, Y, cfg: QConfig, n_steps: int, loss,
+                         dV=None, dalpha=None, dbeta=None, stream=None, block_kind: int = AR_BLOCK_LINEAR) -> None:
+    """``ar_tune_step`` without a workspace, for callers that cannot allocate device memory.
+
+    The scratch is a fixed device array of ``AR_NOALLOC_SCRATCH_BYTES`` inside
+    the library, shared by all calls on a device (serialise overlapping calls);
+    larger problems raise ``ARError`` (AR_ERR_WORKSPACE).
+    """
+    layer = _layer(W, V, alpha, beta)
+    grads = Grads(_ptr(dV), _ptr(dalpha), _ptr(dbeta))
+    gp = ctypes.byref(grads) if (dV is not None or dalpha is not None or dbeta is not None) else None
+    _check(lib().ar_tune_step_noalloc(block_kind, ctypes.byref(layer), 1, _ptr(X), X.shape[0], _ptr(Y),
+                                      ctypes.byref(cfg), n_steps, _ptr(loss), gp, _stream(stream)))
 
 
 def ar_pack_int4(W, V, alpha, beta, cfg: QConfig, packed, scale16, zero16, stream=None) -> None:

@@ -109,6 +109,8 @@ ar_status check_linear(const ar_layer* layers, int n_layers, int64_t M, const ar
 
 }  // namespace
 
+void set_last_error(const char* msg) { t_error = msg; }
+
 void trace_kernel(const char* name) {
   if (!t_kernels.empty()) t_kernels += ";";
   t_kernels += name;

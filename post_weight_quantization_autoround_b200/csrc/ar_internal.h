@@ -11,6 +11,9 @@ namespace ar {
 
 constexpr float kScaleGuard = 1e-8f;  // lower bound on a group's scale
 
+// Sets the text ar_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 // Records the name of a kernel launched by the current API call (tracing).
 void trace_kernel(const char* name);
 
