@@ -360,7 +360,7 @@ ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
   if (T > 16) return fail(AR_ERR_UNSUPPORTED, "T=%lld: this build supports 1 <= T <= 16", (long long)T);
   if (!pow2(group_size) || group_size < 32 || group_size > 1024)
     return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 32..1024", group_size);
-  if (K % group_size != 0 || K % 32 != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and 32");
+  if (K % group_size != 0 || K % 128 != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and 128");
   if (N > INT32_MAX || K > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
   const void* ptrs[] = {A, packed, scale_f16, zero_f16, out};
   for (const void* p : ptrs) {

@@ -45,6 +45,12 @@ cudaError_t launch_pack_int4(const uint16_t* W, const float* V, const float* alp
 
 cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t stream);
 
+// 2-D tensor map over a row-major [rows][cols] array (cols contiguous) with a
+// box of box_rows x box_cols elements; zero fill out of bounds.
+cudaError_t make_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, uint32_t elem_bytes, const void* ptr,
+                         uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows,
+                         CUtensorMapSwizzle swizzle);
+
 // ---- tensor-core GEMMs (ar_gemm.cu) ----
 struct FoldArgs {
   const uint16_t* W;  // bf16 [N][K] original weights

@@ -115,6 +115,7 @@ def test_pack_and_w4a16_validation():
     assert w4(FAKE, 17, FAKE, FAKE, FAKE, 64, 256, 128, FAKE, None) == ar.AR_ERR_UNSUPPORTED
     assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 16, FAKE, None) == ar.AR_ERR_UNSUPPORTED
     assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 200, 128, FAKE, None) == ar.AR_ERR_INVALID_ARG
+    assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 96, 32, FAKE, None) == ar.AR_ERR_INVALID_ARG  # K % 128
     assert w4(FAKE, 0, FAKE, FAKE, FAKE, 64, 256, 128, FAKE, None) == ar.AR_ERR_INVALID_ARG
     assert ar.lib().ar_linear_forward(FAKE, 32, FAKE, 100, 256, FAKE, None) == ar.AR_ERR_INVALID_ARG
     assert ar.lib().ar_gemm_bf16(FAKE, 1, FAKE, 0, FAKE, 12, 64, 64, None) == ar.AR_ERR_INVALID_ARG
