@@ -413,3 +413,124 @@ def w4a16_matmul(A, words, scale16, zero16, group_size: int) -> np.ndarray:
     z = zero16.view(np.float16).astype(f64)
     deq = (q.reshape(N, K // group_size, group_size) - z[:, :, None]) * s[:, :, None]
     return np.asarray(A, f64) @ deq.reshape(N, K).T
+
+
+# ----------------------------------------------------------------------------
+# SwiGLU MLP block tuned jointly ([AR] §3 "Why Block-Wise Optimization": the
+# error of downstream sub-layers back-propagates to upstream weights)
+# ----------------------------------------------------------------------------
+#
+# Block: Y = (silu(X Wgᵀ) ⊙ (X Wuᵀ)) Wdᵀ with silu(x) = x / (1 + e^{-x}).
+# Rounding points shared with the GPU path (fp32 instantiation): the gate and
+# up products a, b are rounded to bf16, h = bf16(silu(a) b), the down product
+# accumulates in fp32; in the backward G, dA = bf16(dH · b · silu'(a)) and
+# dB = bf16(dH · silu(a)) are the bf16 operands of the next products.
+
+def silu(x):
+    x = np.asarray(x, f64)
+    return x / (1.0 + np.exp(-x))
+
+
+def silu_grad(x):
+    """d/dx [x·σ(x)] = σ(x)·(1 + x·(1 − σ(x)))."""
+    x = np.asarray(x, f64)
+    s = 1.0 / (1.0 + np.exp(-x))
+    return s * (1.0 + x * (1.0 - s))
+
+
+def mlp_forward(Xb, Wg, Wu, Wd, dtype=f32):
+    """SwiGLU block forward with the given (bf16-valued) weights.
+
+    Returns a, b (the gate/up products), h and the block output y.
+    """
+    X = np.asarray(Xb, f64)
+    if dtype is f32:
+        a = bf16_rne((X @ np.asarray(Wg, f64).T).astype(f32))
+        b = bf16_rne((X @ np.asarray(Wu, f64).T).astype(f32))
+        h = bf16_rne((silu(a) * np.asarray(b, f64)).astype(f32))
+        y = (np.asarray(h, f64) @ np.asarray(Wd, f64).T).astype(f32)
+        return {"a": a, "b": b, "h": h, "y": y}
+    a = X @ np.asarray(Wg, f64).T
+    b = X @ np.asarray(Wu, f64).T
+    h = silu(a) * b
+    return {"a": a, "b": b, "h": h, "y": h @ np.asarray(Wd, f64).T}
+
+
+def mlp_backward(Xb, fw, G, Wd_hat, dtype=f32):
+    """Gradients of the block loss w.r.t. the three fake-quantized weights.
+
+    dŴd = Gᵀ h;  dH = G Ŵd;  dA = dH · b · silu'(a);  dB = dH · silu(a);
+    dŴg = dAᵀ X;  dŴu = dBᵀ X.
+    """
+    X = np.asarray(Xb, f64)
+    G64 = np.asarray(G, f64)
+    a = np.asarray(fw["a"], f64)
+    b = np.asarray(fw["b"], f64)
+    gWd = G64.T @ np.asarray(fw["h"], f64)
+    dH = G64 @ np.asarray(Wd_hat, f64)
+    if dtype is f32:
+        dH = dH.astype(f32).astype(f64)
+        dA = bf16_rne((dH * b * silu_grad(a)).astype(f32))
+        dB = bf16_rne((dH * silu(a)).astype(f32))
+        gWg = np.asarray(dA, f64).T @ X
+        gWu = np.asarray(dB, f64).T @ X
+        return gWg.astype(f32), gWu.astype(f32), gWd.astype(f32), {"dA": dA, "dB": dB, "dH": dH.astype(f32)}
+    dA = dH * b * silu_grad(a)
+    dB = dH * silu(a)
+    return dA.T @ X, dB.T @ X, gWd, {"dA": dA, "dB": dB, "dH": dH}
+
+
+def mlp_reference(Xb, Wg, Wu, Wd):
+    """Block output with the original bf16 weights ([AR] §3 'Algorithm Flow' step 2)."""
+    return mlp_forward(Xb, Wg, Wu, Wd)["y"]
+
+
+def tune_step_mlp(Ws, Xb, Y, states, cfg: QConfig):
+    """One joint SignSGD step on the three weights of the SwiGLU block.
+
+    ``Ws`` = (Wg, Wu, Wd) bf16 values in float32; ``states`` = three
+    (V, alpha, beta) tuples.  Returns (loss, new states, grads, qdq dicts).
+    """
+    sts = [qdq(W, *st, cfg.bits, cfg.group_size, cfg.symmetric) for W, st in zip(Ws, states)]
+    fw = mlp_forward(Xb, sts[0]["What_bf16"], sts[1]["What_bf16"], sts[2]["What_bf16"])
+    M, H = fw["y"].shape
+    count = M * H
+    R = (fw["y"] - np.asarray(Y, f32)).astype(f32)
+    loss = float(np.sum(R.astype(f64) ** 2) / count)
+    G = bf16_rne((R * f32(2.0 / float(count))).astype(f32))
+    gWg, gWu, gWd, extra = mlp_backward(Xb, fw, G, sts[2]["What_bf16"])
+    new_states, grads = [], []
+    for W, st, (V, a, b), gW in zip(Ws, sts, states, (gWg, gWu, gWd)):
+        dV, da, db = ste_fold(gW, W, st, cfg.bits, cfg.symmetric)
+        new_states.append((signsgd(V, dV, cfg.lr, cfg.v_min, cfg.v_max),
+                           signsgd(a, da, cfg.lr, cfg.clip_min, cfg.clip_max),
+                           signsgd(b, db, cfg.lr, cfg.clip_min, cfg.clip_max)))
+        grads.append({"gW": gW, "dV": dV.astype(f32), "dalpha": da.astype(f32), "dbeta": db.astype(f32)})
+    extra.update(G=G, fw=fw)
+    return loss, new_states, grads, sts, extra
+
+
+def eval_loss_mlp(Ws, Xb, Y, states, cfg: QConfig) -> float:
+    sts = [qdq(W, *st, cfg.bits, cfg.group_size, cfg.symmetric) for W, st in zip(Ws, states)]
+    y = mlp_forward(Xb, sts[0]["What_bf16"], sts[1]["What_bf16"], sts[2]["What_bf16"])["y"]
+    R = (y - np.asarray(Y, f32)).astype(f64)
+    return float(np.sum(R ** 2) / R.size)
+
+
+def smooth_grads_mlp(Ws, X, Y, states, bits, group_size, symmetric=False):
+    """fp64 block loss with all roundings replaced by the identity, and its STE-fold gradients."""
+    sts = [qdq(W, *st, bits, group_size, symmetric, dtype=f64, rnd=round_identity) for W, st in zip(Ws, states)]
+    fw = mlp_forward(X, sts[0]["What"], sts[1]["What"], sts[2]["What"], dtype=f64)
+    R = fw["y"] - np.asarray(Y, f64)
+    L = float(np.sum(R ** 2) / R.size)
+    G = 2.0 * R / R.size
+    gWg, gWu, gWd, _ = mlp_backward(X, fw, G, sts[2]["What"], dtype=f64)
+    grads = [ste_fold(gW, W, st, bits, symmetric) for W, st, gW in zip(Ws, sts, (gWg, gWu, gWd))]
+    return L, grads
+
+
+def smooth_loss_mlp(Ws, X, Y, states, bits, group_size, symmetric=False):
+    sts = [qdq(W, *st, bits, group_size, symmetric, dtype=f64, rnd=round_identity) for W, st in zip(Ws, states)]
+    fw = mlp_forward(X, sts[0]["What"], sts[1]["What"], sts[2]["What"], dtype=f64)
+    R = fw["y"] - np.asarray(Y, f64)
+    return float(np.sum(R ** 2) / R.size)

@@ -448,3 +448,89 @@ def test_fp32_instantiation_agrees_with_fp64():
     dV64, da64, db64 = O.ste_fold(gW64, W, st, 4)
     rel = lambda x, y: np.linalg.norm(x - y) / np.linalg.norm(y)
     assert rel(gr["dV"], dV64) < 5e-3 and rel(gr["dalpha"], da64) < 5e-3 and rel(gr["dbeta"], db64) < 5e-3
+
+
+# ----------------------------------------------------------------------------
+# SwiGLU MLP block
+# ----------------------------------------------------------------------------
+
+def test_silu_and_its_derivative():
+    x = np.linspace(-8, 8, 33)
+    assert np.allclose(O.silu(x), x / (1 + np.exp(-x)))
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    h = 1e-6
+    fd = (O.silu(x + h) - O.silu(x - h)) / (2 * h)
+    assert np.allclose(O.silu_grad(x), fd, rtol=1e-7, atol=1e-9)
+    assert O.silu_grad(np.array([0.0]))[0] == pytest.approx(0.5)
+
+
+def test_swiglu_forward_against_loops():
+    rng = np.random.default_rng(12)
+    M, H, F = 3, 4, 5
+    X = rng.standard_normal((M, H))
+    Wg, Wu, Wd = rng.standard_normal((F, H)), rng.standard_normal((F, H)), rng.standard_normal((H, F))
+    y = O.mlp_forward(X, Wg, Wu, Wd, dtype=np.float64)["y"]
+    for m in range(M):
+        for n in range(H):
+            acc = 0.0
+            for f in range(F):
+                a = sum(X[m, k] * Wg[f, k] for k in range(H))
+                b = sum(X[m, k] * Wu[f, k] for k in range(H))
+                acc += (a / (1 + np.exp(-a))) * b * Wd[n, f]
+            assert y[m, n] == pytest.approx(acc, rel=1e-12)
+
+
+def test_mlp_ste_gradients_match_finite_differences():
+    """Joint block gradients of all three weights (through SiLU and the gating product) vs finite differences."""
+    rng = np.random.default_rng(13)
+    M, H, F, g, bits = 6, 32, 48, 16, 3
+    Ws = [rng.standard_normal((F, H)) * 0.2, rng.standard_normal((F, H)) * 0.2, rng.standard_normal((H, F)) * 0.2]
+    X = rng.standard_normal((M, H))
+    Y = O.mlp_forward(X, *Ws, dtype=np.float64)["y"] + 0.01 * rng.standard_normal((M, H))
+    states = []
+    for W in Ws:
+        states.append((rng.uniform(-0.45, 0.45, W.shape), rng.uniform(0.55, 0.95, (W.shape[0], W.shape[1] // g)),
+                       rng.uniform(0.55, 0.95, (W.shape[0], W.shape[1] // g))))
+    L, grads = O.smooth_grads_mlp(Ws, X, Y, states, bits, g)
+    h = 1e-7
+
+    def f(sts):
+        return O.smooth_loss_mlp(Ws, X, Y, sts, bits, g)
+
+    for li in range(3):
+        dV, da, db = grads[li]
+        for (n, k) in [(0, 0), (1, 7), (2, 15), (3, 20)]:
+            sp = [tuple(x.copy() for x in st) for st in states]
+            sm = [tuple(x.copy() for x in st) for st in states]
+            sp[li][0][n, k] += h
+            sm[li][0][n, k] -= h
+            assert dV[n, k] == pytest.approx((f(sp) - f(sm)) / (2 * h), rel=1e-5, abs=1e-12)
+        for which, dref in ((1, da), (2, db)):
+            for (n, j) in [(0, 0), (2, 1), (5, 0)]:
+                sp = [tuple(x.copy() for x in st) for st in states]
+                sm = [tuple(x.copy() for x in st) for st in states]
+                sp[li][which][n, j] += h
+                sm[li][which][n, j] -= h
+                assert dref[n, j] == pytest.approx((f(sp) - f(sm)) / (2 * h), rel=1e-5, abs=1e-12)
+
+
+def test_mlp_fp32_instantiation_agrees_with_fp64():
+    rng = np.random.default_rng(14)
+    M, H, F, g = 32, 128, 96, 32
+    Ws = [O.bf16_rne((rng.standard_normal(s) * 0.05).astype(np.float32)) for s in ((F, H), (F, H), (H, F))]
+    X = O.bf16_rne(rng.standard_normal((M, H)).astype(np.float32))
+    Y = O.mlp_reference(X, *Ws)
+    states = [(rng.uniform(-0.5, 0.5, W.shape).astype(np.float32),
+               rng.uniform(0.5, 1, (W.shape[0], W.shape[1] // g)).astype(np.float32),
+               rng.uniform(0.5, 1, (W.shape[0], W.shape[1] // g)).astype(np.float32)) for W in Ws]
+    cfg = O.QConfig(bits=4, group_size=g)
+    L, _, grads, sts, extra = O.tune_step_mlp(Ws, X, Y, states, cfg)
+    # the same step with every rounding point kept in fp64
+    fw64 = O.mlp_forward(X, sts[0]["What_bf16"], sts[1]["What_bf16"], sts[2]["What_bf16"], dtype=np.float64)
+    R = fw64["y"] - np.asarray(Y, np.float64)
+    assert L == pytest.approx(np.mean(R ** 2), rel=2e-2)
+    gWg, gWu, gWd, _ = O.mlp_backward(X, fw64, 2 * R / R.size, sts[2]["What_bf16"], dtype=np.float64)
+    rel = lambda x, y: np.linalg.norm(x - y) / np.linalg.norm(y)
+    for gr, g64, W, st in zip(grads, (gWg, gWu, gWd), Ws, sts):
+        dV64, da64, db64 = O.ste_fold(g64, W, st, 4)
+        assert rel(gr["dV"], dV64) < 5e-2 and rel(gr["dalpha"], da64) < 5e-2
