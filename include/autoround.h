@@ -103,7 +103,9 @@ typedef struct {
 } ar_grads;
 
 typedef enum {
-  AR_BLOCK_LINEAR = 0 /* one linear layer: Y = X W^T (n_layers = 1) */
+  AR_BLOCK_LINEAR = 0,    /* one linear layer: Y = X W^T (n_layers = 1) */
+  AR_BLOCK_SWIGLU_MLP = 1 /* SwiGLU MLP: Y = (silu(X Wg^T) * (X Wu^T)) Wd^T; layers = {gate, up, down},
+                             gate/up [F][H], down [H][F] (n_layers = 3) */
 } ar_block_kind;
 
 /* ------------------------------------------------------------------------ */
@@ -137,6 +139,17 @@ AR_API ar_status ar_qdq(const uint16_t* W, const float* V, const float* alpha, c
 AR_API ar_status ar_linear_forward(const uint16_t* X, int64_t M, const uint16_t* W, int64_t N, int64_t K, float* Y,
                             ar_stream_t stream);
 
+/* Bytes of workspace ar_block_forward needs (0 on invalid input). */
+AR_API size_t ar_block_forward_workspace(int block_kind, const ar_layer* layers, int n_layers, int64_t M);
+
+/* Reference output of a block with its original weights ([AR] §3 "Algorithm
+ * Flow" step 2; for the SwiGLU block [AR] §3 "Why Block-Wise Optimization").
+ * AR_BLOCK_LINEAR: as ar_linear_forward.  AR_BLOCK_SWIGLU_MLP: a = bf16(X Wg^T),
+ * b = bf16(X Wu^T), h = bf16(silu(a) b) (workspace holds h, M x F bf16),
+ * Y fp32 [M][H] = h Wd^T.  Only layers[i].W are read. */
+AR_API ar_status ar_block_forward(int block_kind, const ar_layer* layers, int n_layers, const uint16_t* X, int64_t M,
+                                  float* Y, void* workspace, size_t workspace_bytes, ar_stream_t stream);
+
 /* Bytes of workspace ar_tune_step needs for this block, M tokens and
  * n_steps steps (0 on invalid input; see ar_last_error()). */
 AR_API size_t ar_tune_step_workspace(int block_kind, const ar_layer* layers, int n_layers, int64_t M,
@@ -155,10 +168,17 @@ AR_API size_t ar_tune_step_workspace(int block_kind, const ar_layer* layers, int
  * loss_per_step: device fp32 [max(n_steps,1)]; entry i is the loss of the
  *   state before update i.  n_steps = 0 evaluates the loss of the current
  *   state into loss_per_step[0] and updates nothing.
- * grads: NULL, or gradient outputs of the last step.
+ * grads: NULL, or an array of n_layers gradient outputs of the last step.
+ * AR_BLOCK_SWIGLU_MLP (n_layers = 3: gate, up, down) tunes the three weights
+ *   jointly against the block output ([AR] §3 "Why Block-Wise Optimization"):
+ *   h = bf16(silu(a) b) with a, b the bf16 gate/up products; G as above on the
+ *   block output (M x H); dWd = G^T h; dH = G Wd_hat; dA = bf16(dH b silu'(a)),
+ *   dB = bf16(dH silu(a)); dWg = dA^T X, dWu = dB^T X; each folded and
+ *   updated as above.  X [M][H] bf16, Y [M][H] fp32 from ar_block_forward.
  * workspace: device buffer of at least ar_tune_step_workspace() bytes.
- * Supported: AR_BLOCK_LINEAR with n_layers = 1; bits 2..8; group_size 32,
- * 64, 128, 256; N % 8 == 0; K % 256 == 0 is NOT required (K % g == 0 is).
+ * Supported: AR_BLOCK_LINEAR with n_layers = 1 and AR_BLOCK_SWIGLU_MLP with
+ * n_layers = 3; bits 2..8; group_size 32, 64, 128, 256 dividing every K;
+ * N % 8 == 0 (H, F % 8 == 0 for the MLP).
  * Errors: AR_ERR_INVALID_ARG, AR_ERR_UNSUPPORTED, AR_ERR_WORKSPACE. */
 AR_API ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_layers, const uint16_t* X, int64_t M,
                        const float* Y, const ar_qconfig* cfg, int n_steps, float* loss_per_step,

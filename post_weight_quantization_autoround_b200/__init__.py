@@ -20,7 +20,8 @@ __all__ = [
     "ar_qconfig_default", "ar_f32_to_bf16", "ar_qdq", "ar_linear_forward", "ar_tune_step_workspace",
     "ar_tune_step", "ar_pack_int4", "ar_w4a16_gemm", "ar_gemm_bf16", "ar_get_device_status",
     "ar_last_error", "ar_last_kernels", "ar_version", "ar_profile_start", "ar_profile_stop", "AR_BLOCK_LINEAR",
-    "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES",
+    "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES", "AR_BLOCK_SWIGLU_MLP", "ar_block_forward",
+    "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -29,6 +30,7 @@ AR_OK, AR_ERR_INVALID_ARG, AR_ERR_UNSUPPORTED, AR_ERR_CUDA, AR_ERR_NONFINITE, AR
 _STATUS_NAMES = ["AR_OK", "AR_ERR_INVALID_ARG", "AR_ERR_UNSUPPORTED", "AR_ERR_CUDA", "AR_ERR_NONFINITE",
                  "AR_ERR_TIMEOUT", "AR_ERR_WORKSPACE"]
 AR_BLOCK_LINEAR = 0
+AR_BLOCK_SWIGLU_MLP = 1
 
 
 class ARError(RuntimeError):
@@ -75,6 +77,8 @@ _SIGNATURES = {
     "ar_last_error": (ctypes.c_char_p, []),
     "ar_last_kernels": (ctypes.c_char_p, []),
     "ar_version": (ctypes.c_char_p, []),
+    "ar_block_forward_workspace": (ctypes.c_size_t, [_INT, ctypes.POINTER(Layer), _INT, _I64]),
+    "ar_block_forward": (_INT, [_INT, ctypes.POINTER(Layer), _INT, _P, _I64, _P, _P, ctypes.c_size_t, _P]),
     "ar_tune_step_noalloc": (_INT, [_INT, ctypes.POINTER(Layer), _INT, _P, _I64, _P, ctypes.POINTER(QConfig), _INT,
                                     _P, ctypes.POINTER(Grads), _P]),
     "ar_profile_start": (_INT, []),
@@ -177,6 +181,54 @@ def ar_tune_step(W, V, alpha, beta, X, Y, cfg: QConfig, n_steps: int, loss, work
     gp = ctypes.byref(grads) if (dV is not None or dalpha is not None or dbeta is not None) else None
     _check(lib().ar_tune_step(block_kind, ctypes.byref(layer), 1, _ptr(X), X.shape[0], _ptr(Y), ctypes.byref(cfg),
                               n_steps, _ptr(loss), gp, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)))
+
+
+def _layers(ws):
+    """ctypes array of Layer from a list of (W, V, alpha, beta) tuples (V/alpha/beta may be None)."""
+    arr = (Layer * len(ws))()
+    for i, (W, V, a, b) in enumerate(ws):
+        N, K = W.shape
+        arr[i] = Layer(_ptr(W), _ptr(V), _ptr(a), _ptr(b), N, K)
+    return arr
+
+
+def ar_block_forward_workspace(block_kind: int, weights, M: int) -> int:
+    arr = _layers([(W, None, None, None) for W in weights])
+    n = lib().ar_block_forward_workspace(block_kind, arr, len(weights), M)
+    if n == 0:
+        raise ARError(AR_ERR_INVALID_ARG, ar_last_error())
+    return int(n)
+
+
+def ar_block_forward(block_kind: int, weights, X, Y, workspace, stream=None) -> None:
+    """Reference output of a block with its original weights (list of W tensors)."""
+    arr = _layers([(W, None, None, None) for W in weights])
+    _check(lib().ar_block_forward(block_kind, arr, len(weights), _ptr(X), X.shape[0], _ptr(Y), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def ar_tune_block_workspace(block_kind: int, layers, M: int, cfg: QConfig, n_steps: int) -> int:
+    """``ar_tune_step_workspace`` for a block given as a list of (W, V, alpha, beta)."""
+    arr = _layers(layers)
+    n = lib().ar_tune_step_workspace(block_kind, arr, len(layers), M, ctypes.byref(cfg), n_steps)
+    if n == 0:
+        raise ARError(AR_ERR_INVALID_ARG, ar_last_error())
+    return int(n)
+
+
+def ar_tune_block(block_kind: int, layers, X, Y, cfg: QConfig, n_steps: int, loss, workspace, grads=None,
+                  stream=None) -> None:
+    """``ar_tune_step`` for a block given as a list of (W, V, alpha, beta); grads: list of (dV, dalpha, dbeta)."""
+    arr = _layers(layers)
+    gp = None
+    if grads is not None:
+        g = (Grads * len(layers))()
+        for i, (dv, da, db) in enumerate(grads):
+            g[i] = Grads(_ptr(dv), _ptr(da), _ptr(db))
+        gp = g
+    _check(lib().ar_tune_step(block_kind, arr, len(layers), _ptr(X), X.shape[0], _ptr(Y), ctypes.byref(cfg), n_steps,
+                              _ptr(loss), gp, _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)))
 
 

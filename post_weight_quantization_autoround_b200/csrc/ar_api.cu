@@ -107,6 +107,157 @@ ar_status check_linear(const ar_layer* layers, int n_layers, int64_t M, const ar
   return AR_OK;
 }
 
+
+// Layout of the tuning workspace for a SwiGLU block (gate, up: [F][H]; down: [H][F]).
+struct MlpWs {
+  size_t what[3], s[3], zp[3], mx[3], mn[3];
+  size_t a, b, h, da, db, g, partial, total;
+  int partials_per_step;
+};
+
+MlpWs mlp_ws(int64_t M, int64_t Hd, int64_t F, int g, int n_steps) {
+  MlpWs w{};
+  size_t off = 0;
+  const int64_t NK = F * Hd;
+  for (int i = 0; i < 3; ++i) {
+    w.what[i] = off;
+    off = align_up(off + static_cast<size_t>(NK) * 2, 256);
+  }
+  for (int i = 0; i < 3; ++i) {
+    const int64_t groups = NK / g;
+    size_t* dst[4] = {&w.s[i], &w.zp[i], &w.mx[i], &w.mn[i]};
+    for (size_t* d : dst) {
+      *d = off;
+      off = align_up(off + static_cast<size_t>(groups) * 4, 256);
+    }
+  }
+  size_t* acts[5] = {&w.a, &w.b, &w.h, &w.da, &w.db};
+  for (size_t* d : acts) {
+    *d = off;
+    off = align_up(off + static_cast<size_t>(M * F) * 2, 256);
+  }
+  w.g = off;
+  off = align_up(off + static_cast<size_t>(M * Hd) * 2, 256);
+  w.partials_per_step = resid_partials(static_cast<int>(M), static_cast<int>(Hd));
+  w.partial = off;
+  off = align_up(off + static_cast<size_t>(w.partials_per_step) * (n_steps > 0 ? n_steps : 1) * 8, 256);
+  w.total = off;
+  return w;
+}
+
+// gate [F][H], up [F][H], down [H][F]; returns H and F.
+ar_status check_mlp(const ar_layer* layers, int n_layers, int64_t M, const ar_qconfig* cfg, bool for_tune,
+                    int64_t* Hd, int64_t* F) {
+  if (!layers || n_layers != 3) return fail(AR_ERR_UNSUPPORTED, "AR_BLOCK_SWIGLU_MLP needs three layers (gate, up, down)");
+  const ar_layer &lg = layers[0], &lu = layers[1], &ld = layers[2];
+  if (lg.N <= 0 || lg.K <= 0 || M <= 0) return fail(AR_ERR_INVALID_ARG, "sizes must be positive");
+  if (lu.N != lg.N || lu.K != lg.K || ld.N != lg.K || ld.K != lg.N)
+    return fail(AR_ERR_INVALID_ARG, "SwiGLU shapes: gate and up [F][H], down [H][F]");
+  *F = lg.N;
+  *Hd = lg.K;
+  if (cfg) {
+    ar_status st = check_cfg(cfg);
+    if (st != AR_OK) return st;
+    const int g = cfg->group_size;
+    if (for_tune && g != 32 && g != 64 && g != 128 && g != 256)
+      return fail(AR_ERR_UNSUPPORTED, "ar_tune_step supports group_size 32, 64, 128, 256 (got %d)", g);
+    if (*Hd % g != 0 || *F % g != 0) return fail(AR_ERR_INVALID_ARG, "H and F must be multiples of group_size");
+  }
+  if (*Hd % 8 != 0 || *F % 8 != 0) return fail(AR_ERR_INVALID_ARG, "H and F must be multiples of 8");
+  if (M > INT32_MAX || *Hd > INT32_MAX || *F > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  for (int i = 0; i < 3; ++i) {
+    const ar_layer& L = layers[i];
+    if (!L.W || (for_tune && (!L.V || !L.alpha || !L.beta))) return fail(AR_ERR_INVALID_ARG, "layer pointer is NULL");
+    if (!aligned16(L.W) || (for_tune && (!aligned16(L.V) || !aligned16(L.alpha) || !aligned16(L.beta))))
+      return fail(AR_ERR_INVALID_ARG, "layer pointers must be 16-byte aligned");
+  }
+  return AR_OK;
+}
+
+FoldArgs fold_args(const ar_layer& L, const ar_qconfig* cfg, float* sc, float* zp, float* mx, float* mn,
+                   const ar_grads* gr) {
+  FoldArgs fa{};
+  fa.W = L.W;
+  fa.V = L.V;
+  fa.alpha = L.alpha;
+  fa.beta = L.beta;
+  fa.s = sc;
+  fa.zp = zp;
+  fa.mx = mx;
+  fa.mn = mn;
+  fa.dV_out = gr ? gr->dV : nullptr;
+  fa.da_out = gr ? gr->dalpha : nullptr;
+  fa.db_out = gr ? gr->dbeta : nullptr;
+  fa.group_size = cfg->group_size;
+  fa.bits = cfg->bits;
+  fa.symmetric = cfg->symmetric;
+  fa.lr = cfg->lr;
+  fa.v_min = cfg->v_min;
+  fa.v_max = cfg->v_max;
+  fa.c_min = cfg->clip_min;
+  fa.c_max = cfg->clip_max;
+  return fa;
+}
+
+ar_status tune_mlp(const ar_layer* L, const uint16_t* X, int64_t M, const float* Y, const ar_qconfig* cfg,
+                   int n_steps, float* loss_per_step, const ar_grads* grads, void* workspace,
+                   size_t workspace_bytes, cudaStream_t s) {
+  int64_t Hd = 0, F = 0;
+  ar_status st = check_mlp(L, 3, M, cfg, true, &Hd, &F);
+  if (st != AR_OK) return st;
+  const MlpWs w = mlp_ws(M, Hd, F, cfg->group_size, n_steps);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (grads) {
+    for (int i = 0; i < 3; ++i) {
+      const void* gp[] = {grads[i].dV, grads[i].dalpha, grads[i].dbeta};
+      for (const void* p : gp)
+        if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "gradient outputs must be 16-byte aligned");
+    }
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto bf = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
+  auto f32p = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  const int Mi = static_cast<int>(M), Hi = static_cast<int>(Hd), Fi = static_cast<int>(F);
+  const float gscale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(Hd)));
+  double* partial = reinterpret_cast<double*>(ws + w.partial);
+  const int steps = n_steps > 0 ? n_steps : 1;
+  cudaError_t e;
+  for (int step = 0; step < steps; ++step) {
+    for (int i = 0; i < 3; ++i) {
+      e = launch_qdq(L[i].W, L[i].V, L[i].alpha, L[i].beta, L[i].N, L[i].K, cfg->group_size, cfg->bits,
+                     cfg->symmetric, bf(w.what[i]), nullptr, f32p(w.s[i]), f32p(w.zp[i]), f32p(w.mx[i]),
+                     f32p(w.mn[i]), s);
+      if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+    }
+    e = launch_gemm_swiglu_fwd(X, bf(w.what[0]), bf(w.what[1]), bf(w.a), bf(w.b), bf(w.h), Mi, Fi, Hi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "SwiGLU forward GEMM launch");
+    e = launch_gemm_resid(bf(w.h), bf(w.what[2]), Y, bf(w.g), gscale,
+                          partial + static_cast<size_t>(step) * w.partials_per_step, Mi, Hi, Fi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "down-projection GEMM launch");
+    if (n_steps == 0) break;
+    const bool last = step == steps - 1;
+    FoldArgs fd = fold_args(L[2], cfg, f32p(w.s[2]), f32p(w.zp[2]), f32p(w.mx[2]), f32p(w.mn[2]),
+                            (last && grads) ? &grads[2] : nullptr);
+    e = launch_gemm_fold(bf(w.g), bf(w.h), fd, Mi, Hi, Fi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "down weight-gradient GEMM launch");
+    e = launch_gemm_swiglu_bwd(bf(w.g), bf(w.what[2]), bf(w.a), bf(w.b), bf(w.da), bf(w.db), Mi, Fi, Hi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "SwiGLU backward GEMM launch");
+    FoldArgs fg = fold_args(L[0], cfg, f32p(w.s[0]), f32p(w.zp[0]), f32p(w.mx[0]), f32p(w.mn[0]),
+                            (last && grads) ? &grads[0] : nullptr);
+    e = launch_gemm_fold(bf(w.da), X, fg, Mi, Fi, Hi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "gate weight-gradient GEMM launch");
+    FoldArgs fu = fold_args(L[1], cfg, f32p(w.s[1]), f32p(w.zp[1]), f32p(w.mx[1]), f32p(w.mn[1]),
+                            (last && grads) ? &grads[1] : nullptr);
+    e = launch_gemm_fold(bf(w.db), X, fu, Mi, Fi, Hi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "up weight-gradient GEMM launch");
+  }
+  e = launch_loss_reduce(partial, w.partials_per_step, steps,
+                         1.0 / (static_cast<double>(M) * static_cast<double>(Hd)), loss_per_step, s);
+  if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
+  return end_call();
+}
 }  // namespace
 
 void set_last_error(const char* msg) { t_error = msg; }
@@ -242,6 +393,15 @@ ar_status ar_linear_forward(const uint16_t* X, int64_t M, const uint16_t* W, int
 size_t ar_tune_step_workspace(int block_kind, const ar_layer* layers, int n_layers, int64_t M, const ar_qconfig* cfg,
                               int n_steps) {
   begin_call();
+  if (block_kind == AR_BLOCK_SWIGLU_MLP) {
+    int64_t Hd = 0, F = 0;
+    if (n_steps < 0 || check_cfg(cfg) != AR_OK || check_mlp(layers, n_layers, M, nullptr, false, &Hd, &F) != AR_OK ||
+        cfg->group_size <= 0 || Hd % cfg->group_size != 0 || F % cfg->group_size != 0) {
+      if (t_error.empty()) fail(AR_ERR_INVALID_ARG, "invalid SwiGLU block");
+      return 0;
+    }
+    return mlp_ws(M, Hd, F, cfg->group_size, n_steps).total;
+  }
   if (block_kind != AR_BLOCK_LINEAR) {
     fail(AR_ERR_UNSUPPORTED, "block_kind %d not supported", block_kind);
     return 0;
@@ -263,6 +423,13 @@ ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_layers, con
                        const float* Y, const ar_qconfig* cfg, int n_steps, float* loss_per_step, const ar_grads* grads,
                        void* workspace, size_t workspace_bytes, ar_stream_t stream) {
   begin_call();
+  if (block_kind == AR_BLOCK_SWIGLU_MLP) {
+    if (n_steps < 0) return fail(AR_ERR_INVALID_ARG, "n_steps must be >= 0");
+    if (!X || !Y || !loss_per_step) return fail(AR_ERR_INVALID_ARG, "X, Y and loss_per_step are required");
+    if (!aligned16(X) || !aligned16(Y)) return fail(AR_ERR_INVALID_ARG, "X and Y must be 16-byte aligned");
+    return tune_mlp(layers, X, M, Y, cfg, n_steps, loss_per_step, grads, workspace, workspace_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+  }
   if (block_kind != AR_BLOCK_LINEAR) return fail(AR_ERR_UNSUPPORTED, "block_kind %d not supported", block_kind);
   ar_status st = check_linear(layers, n_layers, M, cfg, true);
   if (st != AR_OK) return st;
@@ -327,6 +494,51 @@ ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_layers, con
   e = launch_loss_reduce(partial, w.partials_per_step, steps, 1.0 / (static_cast<double>(M) * static_cast<double>(L.N)),
                          loss_per_step, s);
   if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
+  return end_call();
+}
+
+size_t ar_block_forward_workspace(int block_kind, const ar_layer* layers, int n_layers, int64_t M) {
+  begin_call();
+  if (block_kind == AR_BLOCK_LINEAR) {
+    if (!layers || n_layers != 1) {
+      fail(AR_ERR_INVALID_ARG, "AR_BLOCK_LINEAR needs one layer");
+      return 0;
+    }
+    return 256;  // no scratch needed; a non-zero size keeps 0 for errors
+  }
+  if (block_kind != AR_BLOCK_SWIGLU_MLP) {
+    fail(AR_ERR_UNSUPPORTED, "block_kind %d not supported", block_kind);
+    return 0;
+  }
+  int64_t Hd = 0, F = 0;
+  if (check_mlp(layers, n_layers, M, nullptr, false, &Hd, &F) != AR_OK) return 0;
+  return align_up(static_cast<size_t>(M * F) * 2, 256);
+}
+
+ar_status ar_block_forward(int block_kind, const ar_layer* layers, int n_layers, const uint16_t* X, int64_t M,
+                           float* Y, void* workspace, size_t workspace_bytes, ar_stream_t stream) {
+  begin_call();
+  if (!X || !Y) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(X) || !aligned16(Y)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (block_kind == AR_BLOCK_LINEAR) {
+    if (!layers || n_layers != 1) return fail(AR_ERR_INVALID_ARG, "AR_BLOCK_LINEAR needs one layer");
+    return ar_linear_forward(X, M, layers[0].W, layers[0].N, layers[0].K, Y, stream);
+  }
+  if (block_kind != AR_BLOCK_SWIGLU_MLP) return fail(AR_ERR_UNSUPPORTED, "block_kind %d not supported", block_kind);
+  int64_t Hd = 0, F = 0;
+  ar_status st = check_mlp(layers, n_layers, M, nullptr, false, &Hd, &F);
+  if (st != AR_OK) return st;
+  const size_t need = align_up(static_cast<size_t>(M * F) * 2, 256);
+  if (!workspace || workspace_bytes < need)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  uint16_t* H = static_cast<uint16_t*>(workspace);
+  cudaError_t e = launch_gemm_swiglu_fwd(X, layers[0].W, layers[1].W, nullptr, nullptr, H, static_cast<int>(M),
+                                         static_cast<int>(F), static_cast<int>(Hd), s);
+  if (e != cudaSuccess) return cuda_fail(e, "SwiGLU forward GEMM launch");
+  e = launch_gemm_store(H, layers[2].W, Y, static_cast<int>(M), static_cast<int>(Hd), static_cast<int>(F), s);
+  if (e != cudaSuccess) return cuda_fail(e, "down-projection GEMM launch");
   return end_call();
 }
 

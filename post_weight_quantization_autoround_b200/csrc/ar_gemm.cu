@@ -11,6 +11,11 @@
 //   EPI_FOLD   straight-through fold of dW_hat into dV (per element) and
 //              dalpha/dbeta (per group), then the SignSGD step and clamp
 //              ([AR] §3 "SignSGD"; STE as in [IA])
+//   EPI_SWIGLU_FWD  gate and up products of a SwiGLU block in one 256-wide
+//              tile (128 gate rows + the same 128 up rows of B): a, b -> bf16,
+//              h = bf16(silu(a) b)  ([AR] §3 "Why Block-Wise Optimization")
+//   EPI_SWIGLU_BWD  dH = G W_down; SiLU backward: dA = bf16(dH b silu'(a)),
+//              dB = bf16(dH silu(a))
 //
 // ([AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
 // Architectural Optimizations of AutoRound"; [IA] = "Intel AutoRound 高级量化".)
@@ -46,7 +51,7 @@ constexpr int kBStage = BN * BK * 2;  // 32 KiB
 constexpr int kTmemCols = 2 * BN;     // double-buffered accumulator
 constexpr int kSmemBytes = STAGES * (kAStage + kBStage) + 1024 + 256;
 
-enum { EPI_STORE = 0, EPI_RESID = 1, EPI_FOLD = 2 };
+enum { EPI_STORE = 0, EPI_RESID = 1, EPI_FOLD = 2, EPI_SWIGLU_FWD = 3, EPI_SWIGLU_BWD = 4 };
 
 struct Ctl {
   uint64_t full[STAGES];
@@ -68,6 +73,11 @@ struct Params {
   float gscale;
   double* partial;
   FoldArgs fold;     // EPI_FOLD
+  uint16_t* act_a;   // EPI_SWIGLU_FWD outputs / EPI_SWIGLU_BWD inputs: a, b, h [M][N] bf16
+  uint16_t* act_b;
+  uint16_t* act_h;
+  uint16_t* grad_a;  // EPI_SWIGLU_BWD outputs: dA, dB [M][N] bf16
+  uint16_t* grad_b;
 };
 
 // Byte offsets of the MN-major canonical layout: the leading-dimension offset
@@ -265,13 +275,119 @@ __device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n,
   return bad;
 }
 
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ float sigmoidf(float x) { return __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-x))); }
+
+// SwiGLU forward: TMEM columns 0..127 hold the gate product a, 128..255 the
+// up product b of the same 128 outputs f.  Writes a, b, h = silu(a) b (bf16).
+__device__ __forceinline__ void epi_swiglu_fwd(const Params& p, uint32_t taddr, int row, int f_base) {
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    float va[32], vb[32];
+    tmem_ld32(taddr + c * 32, va);
+    tmem_ld32(taddr + 128 + c * 32, vb);
+    const int col0 = f_base + c * 32;
+    if (row >= p.M || col0 >= p.N) continue;
+    const size_t e = static_cast<size_t>(row) * p.N + col0;
+    uint32_t pa[16], pb[16], ph[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float a0 = bf16_round(va[i]), a1 = bf16_round(va[i + 1]);
+      const float b0 = bf16_round(vb[i]), b1 = bf16_round(vb[i + 1]);
+      pa[i / 2] = pack_bf16x2(a0, a1);
+      pb[i / 2] = pack_bf16x2(b0, b1);
+      ph[i / 2] = pack_bf16x2(__fmul_rn(__fmul_rn(a0, sigmoidf(a0)), b0), __fmul_rn(__fmul_rn(a1, sigmoidf(a1)), b1));
+    }
+    if (col0 + 32 <= p.N) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (p.act_a) *reinterpret_cast<uint4*>(p.act_a + e + 8 * i) = make_uint4(pa[4 * i], pa[4 * i + 1], pa[4 * i + 2], pa[4 * i + 3]);
+        if (p.act_b) *reinterpret_cast<uint4*>(p.act_b + e + 8 * i) = make_uint4(pb[4 * i], pb[4 * i + 1], pb[4 * i + 2], pb[4 * i + 3]);
+        *reinterpret_cast<uint4*>(p.act_h + e + 8 * i) = make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
+      }
+    } else {
+      for (int i = 0; i < 32 && col0 + i < p.N; ++i) {
+        const int sh = (i & 1) ? 16 : 0;
+        if (p.act_a) p.act_a[e + i] = static_cast<uint16_t>(pa[i / 2] >> sh);
+        if (p.act_b) p.act_b[e + i] = static_cast<uint16_t>(pb[i / 2] >> sh);
+        p.act_h[e + i] = static_cast<uint16_t>(ph[i / 2] >> sh);
+      }
+    }
+  }
+}
+
+// SiLU backward on dH (the accumulator): dA = dH b silu'(a), dB = dH silu(a).
+__device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, int row, int col_base) {
+  bool bad = false;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float dh[32];
+    tmem_ld32(taddr + c * 32, dh);
+    const int col0 = col_base + c * 32;
+    if (row >= p.M || col0 >= p.N) continue;
+    const size_t e = static_cast<size_t>(row) * p.N + col0;
+    const int n = col0 + 32 <= p.N ? 32 : p.N - col0;
+    uint32_t ra[16], rb[16];
+    if (n == 32) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 x = *reinterpret_cast<const uint4*>(p.act_a + e + 8 * i);
+        const uint4 y = *reinterpret_cast<const uint4*>(p.act_b + e + 8 * i);
+        ra[4 * i] = x.x; ra[4 * i + 1] = x.y; ra[4 * i + 2] = x.z; ra[4 * i + 3] = x.w;
+        rb[4 * i] = y.x; rb[4 * i + 1] = y.y; rb[4 * i + 2] = y.z; rb[4 * i + 3] = y.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        ra[i] = 0;
+        rb[i] = 0;
+      }
+      for (int i = 0; i < n; ++i) {
+        ra[i / 2] |= static_cast<uint32_t>(p.act_a[e + i]) << ((i & 1) ? 16 : 0);
+        rb[i / 2] |= static_cast<uint32_t>(p.act_b[e + i]) << ((i & 1) ? 16 : 0);
+      }
+    }
+    uint32_t ga[16], gb[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      float da[2], db[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float a = u ? bf16_hi(ra[i / 2]) : bf16_lo(ra[i / 2]);
+        const float b = u ? bf16_hi(rb[i / 2]) : bf16_lo(rb[i / 2]);
+        const float sg = sigmoidf(a);
+        const float ds = __fmul_rn(sg, __fadd_rn(1.0f, __fmul_rn(a, __fsub_rn(1.0f, sg))));
+        da[u] = __fmul_rn(__fmul_rn(dh[i + u], b), ds);
+        db[u] = __fmul_rn(dh[i + u], __fmul_rn(a, sg));
+        bad |= !isfinite(dh[i + u]);
+      }
+      ga[i / 2] = pack_bf16x2(da[0], da[1]);
+      gb[i / 2] = pack_bf16x2(db[0], db[1]);
+    }
+    if (n == 32) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        *reinterpret_cast<uint4*>(p.grad_a + e + 8 * i) = make_uint4(ga[4 * i], ga[4 * i + 1], ga[4 * i + 2], ga[4 * i + 3]);
+        *reinterpret_cast<uint4*>(p.grad_b + e + 8 * i) = make_uint4(gb[4 * i], gb[4 * i + 1], gb[4 * i + 2], gb[4 * i + 3]);
+      }
+    } else {
+      for (int i = 0; i < n; ++i) {
+        const int sh = (i & 1) ? 16 : 0;
+        p.grad_a[e + i] = static_cast<uint16_t>(ga[i / 2] >> sh);
+        p.grad_b[e + i] = static_cast<uint16_t>(gb[i / 2] >> sh);
+      }
+    }
+  }
+  return bad;
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const Params p) {
+                     const __grid_constant__ CUtensorMap tmB2, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smA = base;
@@ -298,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI == EPI_SWIGLU_FWD) tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
@@ -331,7 +448,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(a_dst, &tmA, &ctl->full[stage], kb * BK, tm * BM);
           }
-          if (B_MN) {
+          if (EPI == EPI_SWIGLU_FWD) {
+            // 128 gate rows then the same 128 up rows
+            tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, tn * (BN / 2));
+            tma_load_2d(b_dst + kBStage / 2, &tmB2, &ctl->full[stage], kb * BK, tn * (BN / 2));
+          } else if (B_MN) {
 #pragma unroll
             for (int i = 0; i < BN / 64; ++i) tma_load_2d(b_dst + i * 8192, &tmB, &ctl->full[stage], tn * BN + 64 * i, kb * BK);
           } else {
@@ -408,8 +529,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
         if (lane == 0) p.partial[static_cast<size_t>(t) * 4 + quarter] = part;
         (void)loss_acc;
-      } else {
+      } else if (EPI == EPI_FOLD) {
         bad |= epi_fold(p, taddr, row, tn * BN);
+      } else if (EPI == EPI_SWIGLU_FWD) {
+        epi_swiglu_fwd(p, taddr, row, tn * (BN / 2));
+      } else {
+        bad |= epi_swiglu_bwd(p, taddr, row, tn * BN);
       }
       tc_fence_before();
       __syncwarp();
@@ -438,15 +563,24 @@ cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t 
 }
 
 template <bool A_MN, bool B_MN, int EPI>
-cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t stream, const char* name) {
-  CUtensorMap tmA, tmB;
+cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t stream, const char* name,
+                const uint16_t* B2 = nullptr) {
+  CUtensorMap tmA, tmB, tmB2;
   // A: K-major [M][K] with 128-row boxes, or MN-major [K][M] with 64-row boxes.
   cudaError_t e = A_MN ? make_tmap(&tmA, A, p.K, p.M, 64) : make_tmap(&tmA, A, p.M, p.K, BM);
   if (e != cudaSuccess) return e;
-  e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64) : make_tmap(&tmB, B, p.N, p.K, BN);
+  if (EPI == EPI_SWIGLU_FWD) {
+    // gate and up weights [N][K], 128-row boxes each
+    e = make_tmap(&tmB, B, p.N, p.K, BN / 2);
+    if (e != cudaSuccess) return e;
+    e = make_tmap(&tmB2, B2, p.N, p.K, BN / 2);
+  } else {
+    e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64) : make_tmap(&tmB, B, p.N, p.K, BN);
+    tmB2 = tmB;
+  }
   if (e != cudaSuccess) return e;
   p.tiles_m = (p.M + BM - 1) / BM;
-  p.tiles_n = (p.N + BN - 1) / BN;
+  p.tiles_n = EPI == EPI_SWIGLU_FWD ? (p.N + BN / 2 - 1) / (BN / 2) : (p.N + BN - 1) / BN;
   p.num_kb = (p.K + BK - 1) / BK;
   auto kern = umma_gemm_kernel<A_MN, B_MN, EPI>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
@@ -455,7 +589,7 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
   const int grid = tiles < num_sms() ? tiles : num_sms();
   {
     LaunchScope scope(stream, name);
-    kern<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
+    kern<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmB2, p);
   }
   return cudaGetLastError();
 }
@@ -542,6 +676,33 @@ cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArg
   p.K = M;
   p.fold = fa;
   return run<true, true, EPI_FOLD>(G, X, p, stream, "umma_gemm<MN,MN,fold>");
+}
+
+cudaError_t launch_gemm_swiglu_fwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* Wu, uint16_t* A_out,
+                                   uint16_t* B_out, uint16_t* H_out, int M, int F, int Hd, cudaStream_t stream) {
+  Params p{};
+  p.M = M;
+  p.N = F;
+  p.K = Hd;
+  p.act_a = A_out;
+  p.act_b = B_out;
+  p.act_h = H_out;
+  return run<false, false, EPI_SWIGLU_FWD>(X, Wg, p, stream, "umma_gemm<K,K,swiglu_fwd>", Wu);
+}
+
+cudaError_t launch_gemm_swiglu_bwd(const uint16_t* G, const uint16_t* Wd_hat, const uint16_t* A_in,
+                                   const uint16_t* B_in, uint16_t* dA, uint16_t* dB, int M, int F, int Hd,
+                                   cudaStream_t stream) {
+  // dH[M][F] = G[M][Hd] W_down[Hd][F]: A = G (K-major over Hd), B = W_down as [K=Hd][N=F] (MN-major)
+  Params p{};
+  p.M = M;
+  p.N = F;
+  p.K = Hd;
+  p.act_a = const_cast<uint16_t*>(A_in);
+  p.act_b = const_cast<uint16_t*>(B_in);
+  p.grad_a = dA;
+  p.grad_b = dB;
+  return run<false, true, EPI_SWIGLU_BWD>(G, Wd_hat, p, stream, "umma_gemm<K,MN,swiglu_bwd>");
 }
 
 cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, bool b_mn, float* D, int M, int N,

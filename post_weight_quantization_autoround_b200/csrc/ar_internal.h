@@ -83,6 +83,16 @@ int resid_partials(int M, int N);
 cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArgs& fa, int M, int N, int K,
                              cudaStream_t stream);
 
+// SwiGLU forward of X[M][Hd] with gate/up weights [F][Hd]: a, b, h [M][F]
+// bf16 (a, b nullable).
+cudaError_t launch_gemm_swiglu_fwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* Wu, uint16_t* A_out,
+                                   uint16_t* B_out, uint16_t* H_out, int M, int F, int Hd, cudaStream_t stream);
+
+// dH = G[M][Hd] W_down[Hd][F] with the SiLU backward epilogue -> dA, dB [M][F] bf16.
+cudaError_t launch_gemm_swiglu_bwd(const uint16_t* G, const uint16_t* Wd_hat, const uint16_t* A_in,
+                                   const uint16_t* B_in, uint16_t* dA, uint16_t* dB, int M, int F, int Hd,
+                                   cudaStream_t stream);
+
 // Plain D[M][N] fp32 = op(A) op(B)^T, with A given K-major ([M][K]) or
 // MN-major ([K][M]) and B given K-major ([N][K]) or MN-major ([K][N]).
 cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, bool b_mn, float* D, int M, int N,
