@@ -278,6 +278,103 @@ def w4a16_bench(ar, torch, peaks, reps=20):
     return out
 
 
+# ----------------------------------------------------------------------------
+# multi-rank plumbing (independent layers per rank; timing only crosses ranks)
+# ----------------------------------------------------------------------------
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank tunes its own independent layer."""
+    return base_seed + rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Largest value over all ranks (the job's device time); identity without a process group."""
+    import torch
+
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, max_ms: float) -> float:
+    """Whole-job steps/s: every rank ran `steps` steps; the job took the slowest rank's time."""
+    return world * steps / (max_ms * 1e-3)
+
+
+def _time_call(torch, fn, warmup=1):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def other_workloads(ar, torch, peaks, steps=10):
+    """Tuning throughput on the remaining workloads (one call of ``steps`` steps each)."""
+    out = {}
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # SwiGLU MLP block, tuned jointly
+    wl = synth.WORKLOADS["mlp_4096_11008"]
+    M, Hd, F = wl.m_tokens, wl.n_in, wl.inter
+    d = synth.make_mlp(Hd, F, M, seed=wl.seed)
+    Ws = [to_dev_bf16(d[k], torch) for k in ("Wg", "Wu", "Wd")]
+    X = to_dev_bf16(d["X"], torch)
+    del d
+    g = wl.group_size
+    st = [(torch.zeros(W.shape, device="cuda"), torch.ones((W.shape[0], W.shape[1] // g), device="cuda"),
+           torch.ones((W.shape[0], W.shape[1] // g), device="cuda")) for W in Ws]
+    cfg = ar.ar_qconfig_default(bits=wl.bits, group_size=g, lr=wl.lr)
+    Y = torch.empty((M, Hd), device="cuda")
+    fws = torch.empty(ar.ar_block_forward_workspace(ar.AR_BLOCK_SWIGLU_MLP, Ws, M), dtype=torch.uint8, device="cuda")
+    ar.ar_block_forward(ar.AR_BLOCK_SWIGLU_MLP, Ws, X, Y, fws)
+    del fws
+    layers = [(W, *s) for W, s in zip(Ws, st)]
+    ws = torch.empty(ar.ar_tune_block_workspace(ar.AR_BLOCK_SWIGLU_MLP, layers, M, cfg, steps), dtype=torch.uint8,
+                     device="cuda")
+    loss = torch.empty(steps, device="cuda")
+    ms = _time_call(torch, lambda: ar.ar_tune_block(ar.AR_BLOCK_SWIGLU_MLP, layers, X, Y, cfg, steps, loss, ws))
+    flops = 14.0 * M * Hd * F
+    out[wl.name] = {"steps_per_s": steps / (ms * 1e-3), "ms_per_step": ms / steps,
+                    "tflops": flops * steps / (ms * 1e-3) / 1e12,
+                    "frac_sustained_bf16": flops * steps / (ms * 1e-3) / 1e12 / peak,
+                    "kernels": ar.ar_last_kernels().count(";") + 1, "steps": steps,
+                    "final_loss": float(loss[-1].item())}
+    del Ws, X, Y, st, layers, ws
+    torch.cuda.empty_cache()
+    # single linear layers: low-bit stress and the 70B-shaped down projection
+    for name in ("lowbit_b3g32", "lowbit_b2g32", "lowbit_b8g256", "down_8192_28672"):
+        wl = synth.WORKLOADS[name]
+        N, K, M, g = wl.n_out, wl.n_in, wl.m_tokens, wl.group_size
+        d = synth.make_linear(N, K, M, seed=wl.seed)
+        W, X = to_dev_bf16(d["W"], torch), to_dev_bf16(d["X"], torch)
+        del d
+        V = torch.zeros((N, K), device="cuda")
+        a = torch.ones((N, K // g), device="cuda")
+        b = torch.ones((N, K // g), device="cuda")
+        cfg = ar.ar_qconfig_default(bits=wl.bits, group_size=g, lr=wl.lr)
+        Y = torch.empty((M, N), device="cuda")
+        ar.ar_linear_forward(X, W, Y)
+        n = steps if name.startswith("down") else 5 * steps
+        ws = torch.empty(ar.ar_tune_step_workspace(W, V, a, b, M, cfg, n), dtype=torch.uint8, device="cuda")
+        loss = torch.empty(n, device="cuda")
+        ms = _time_call(torch, lambda: ar.ar_tune_step(W, V, a, b, X, Y, cfg, n, loss, ws))
+        flops = 4.0 * M * N * K
+        out[name] = {"steps_per_s": n / (ms * 1e-3), "ms_per_step": ms / n, "tflops": flops * n / (ms * 1e-3) / 1e12,
+                     "frac_sustained_bf16": flops * n / (ms * 1e-3) / 1e12 / peak, "steps": n,
+                     "final_loss": float(loss[-1].item())}
+        del W, X, V, a, b, Y, ws
+        torch.cuda.empty_cache()
+    if ar.ar_get_device_status() != 0:
+        out["device_status"] = ar.ar_last_error()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -287,6 +384,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w4a16", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads (MLP, low-bit, 70B down)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -311,8 +409,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     peaks, peaks_src = load_peaks()
 
-    # --- inputs: each rank tunes its own independent layer (seed = rank)
-    d = synth.make_linear(wl.n_out, wl.n_in, wl.m_tokens, seed=wl.seed + rank)
+    # --- inputs: each rank tunes its own independent layer
+    d = synth.make_linear(wl.n_out, wl.n_in, wl.m_tokens, seed=rank_seed(wl.seed, rank))
     cfg = ar.ar_qconfig_default(bits=wl.bits, group_size=wl.group_size, lr=wl.lr)
     W = to_dev_bf16(d["W"], torch)
     X = to_dev_bf16(d["X"], torch)
@@ -322,14 +420,15 @@ def main():
     beta = torch.ones((N, K // g), dtype=torch.float32, device="cuda")
     Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     ar.ar_linear_forward(X, W, Y)
-    ws = torch.empty(ar.ar_tune_step_workspace(W, V, alpha, beta, M, cfg, 1), dtype=torch.uint8, device="cuda")
-    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    n_max = max(args.steps, args.warmup)
+    ws = torch.empty(ar.ar_tune_step_workspace(W, V, alpha, beta, M, cfg, n_max), dtype=torch.uint8, device="cuda")
+    loss = torch.empty(n_max, dtype=torch.float32, device="cuda")
 
-    def step():
-        ar.ar_tune_step(W, V, alpha, beta, X, Y, cfg, 1, loss, ws)
+    def steps(n):
+        # one call runs n tuning steps (QDQ, forward GEMM, weight-gradient GEMM each)
+        ar.ar_tune_step(W, V, alpha, beta, X, Y, cfg, n, loss, ws)
 
-    for _ in range(args.warmup):
-        step()
+    steps(args.warmup)
     torch.cuda.synchronize()
     if ar.ar_get_device_status() != 0:
         raise SystemExit(f"device status after warm-up: {ar.ar_last_error()}")
@@ -343,20 +442,15 @@ def main():
         torch.cuda.synchronize()
         ar.ar_profile_start()
         e0.record(stream)
-        for _ in range(args.steps):
-            step()
+        steps(args.steps)
         e1.record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         prof = ar.ar_profile_stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, "cuda")
     status = ar.ar_get_device_status()
-    final_loss = float(loss.item())
+    final_loss = float(loss[args.steps - 1].item())
 
     launches = sum(n for n, _ in prof.values())
     kernels = {k: {"launches": n, "ms_total": t_ms, "us_per_launch": 1e3 * t_ms / max(n, 1),
@@ -364,7 +458,7 @@ def main():
     flops_gemm = 2.0 * M * N * K
     flops_step = 2 * flops_gemm
     steps_s_rank = args.steps / (ms * 1e-3)
-    value = world * args.steps / (ms * 1e-3)
+    value = job_throughput(world, args.steps, ms)
     gemm_names = [k for k in prof if k.startswith("umma_gemm")]
     dom = max(gemm_names, key=lambda k: prof[k][1])
     dom_us = kernels[dom]["us_per_launch"]
@@ -411,12 +505,8 @@ def main():
         tuner.run_host(Wh, Xh, Vw, aw, bw, lh)
         f1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = f0.elapsed_time(f1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        result["e2e"] = {"value": world * args.steps / (e2e_ms * 1e-3), "unit": "steps/s",
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1), dist if world > 1 else None, "cuda")
+        result["e2e"] = {"value": job_throughput(world, args.steps, e2e_ms), "unit": "steps/s",
                          "h2d_bytes_per_step": tuner.h2d_bytes() / args.steps,
                          "d2h_bytes_per_step": tuner.d2h_bytes() / args.steps,
                          "job": f"per layer: copy W, X, V, alpha, beta in; reference forward; {args.steps} steps; "
@@ -425,6 +515,10 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_w4a16:
         result["w4a16"] = w4a16_bench(ar, torch, peaks)
+    if rank == 0 and world == 1 and not args.no_extra:
+        del W, X, V, alpha, beta, Y, ws
+        torch.cuda.empty_cache()
+        result["workloads"] = other_workloads(ar, torch, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, d)
     if rank == 0:

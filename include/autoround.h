@@ -243,6 +243,14 @@ AR_API ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* pac
 AR_API ar_status ar_gemm_bf16(const uint16_t* A, int a_mn_major, const uint16_t* B, int b_mn_major, float* D, int64_t M,
                        int64_t N, int64_t K, ar_stream_t stream);
 
+/* Diagnostic of the failure path (the pages have no counterpart): one warp
+ * waits on a device barrier that nothing completes, with the same bounded-wait
+ * mechanism the pipelined kernels use but a limit of limit_ns (at most 1 s).
+ * The wait gives up, writes 1 to *gave_up (device int) and raises the sticky
+ * AR_ERR_TIMEOUT status; the kernel returns normally and the context stays
+ * usable.  No fault, trap or hang is involved. */
+AR_API ar_status ar_debug_wait_timeout(uint64_t limit_ns, int* gave_up, ar_stream_t stream);
+
 /* Synchronizes `stream`, then returns and clears the sticky device status:
  * AR_OK, AR_ERR_NONFINITE or AR_ERR_TIMEOUT (timeout wins if both are set),
  * or AR_ERR_CUDA if the synchronization itself failed. */

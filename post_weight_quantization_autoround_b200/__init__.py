@@ -21,7 +21,7 @@ __all__ = [
     "ar_tune_step", "ar_pack_int4", "ar_w4a16_gemm", "ar_gemm_bf16", "ar_get_device_status",
     "ar_last_error", "ar_last_kernels", "ar_version", "ar_profile_start", "ar_profile_stop", "AR_BLOCK_LINEAR",
     "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES", "AR_BLOCK_SWIGLU_MLP", "ar_block_forward",
-    "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace",
+    "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace", "ar_debug_wait_timeout",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -81,6 +81,7 @@ _SIGNATURES = {
     "ar_block_forward": (_INT, [_INT, ctypes.POINTER(Layer), _INT, _P, _I64, _P, _P, ctypes.c_size_t, _P]),
     "ar_tune_step_noalloc": (_INT, [_INT, ctypes.POINTER(Layer), _INT, _P, _I64, _P, ctypes.POINTER(QConfig), _INT,
                                     _P, ctypes.POINTER(Grads), _P]),
+    "ar_debug_wait_timeout": (_INT, [ctypes.c_uint64, _P, _P]),
     "ar_profile_start": (_INT, []),
     "ar_profile_stop": (_INT, [ctypes.c_char_p, ctypes.c_size_t]),
 }
@@ -281,6 +282,11 @@ def ar_profile_stop() -> dict:
         name, n, ms = line.rsplit(" ", 2)
         out[name] = (int(n), float(ms))
     return out
+
+
+def ar_debug_wait_timeout(limit_ns: int, gave_up, stream=None) -> None:
+    """Run the bounded-wait diagnostic: a wait on a barrier nothing completes gives up after limit_ns."""
+    _check(lib().ar_debug_wait_timeout(int(limit_ns), _ptr(gave_up), _stream(stream)))
 
 
 def ar_get_device_status(stream=None) -> int:

@@ -600,6 +600,15 @@ ar_status ar_gemm_bf16(const uint16_t* A, int a_mn_major, const uint16_t* B, int
   return end_call();
 }
 
+ar_status ar_debug_wait_timeout(uint64_t limit_ns, int* gave_up, ar_stream_t stream) {
+  begin_call();
+  if (!gave_up) return fail(AR_ERR_INVALID_ARG, "gave_up is NULL");
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return fail(AR_ERR_INVALID_ARG, "limit_ns must be in (0, 1e9]");
+  cudaError_t e = launch_wait_timeout(limit_ns, gave_up, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait-timeout launch");
+  return end_call();
+}
+
 ar_status ar_get_device_status(ar_stream_t stream) {
   unsigned int v = 0;
   cudaError_t e = read_and_clear_status(&v, reinterpret_cast<cudaStream_t>(stream));

@@ -20,12 +20,13 @@
 // ([AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
 // Architectural Optimizations of AutoRound"; [IA] = "Intel AutoRound 高级量化".)
 //
-// Block: 192 threads.  Warp 0 lane 0 issues TMA loads into a 4-stage ring
+// Block: 320 threads.  Warp 0 lane 0 issues TMA loads into a 4-stage ring
 // (128x64 A tile, 256x64 B tile, 128-byte swizzle); warp 1 allocates 512 TMEM
 // columns (two 128x256 fp32 accumulators) and lane 0 issues
-// tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16); warps 2-5 drain
-// an accumulator with tcgen05.ld (warp w reads TMEM lanes 32*(w%4)..+31, i.e.
-// one output row per thread) while the MMA warp fills the other one.  The
+// tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16); warps 2-9 drain
+// an accumulator with tcgen05.ld while the MMA warp fills the other one: warp
+// w reads TMEM lanes 32*(w%4)..+31 (one output row per thread) and one half
+// of the 256 columns, so two warps share each lane quarter.  The
 // grid is persistent: one CTA per SM, tiles strided by gridDim.x with the
 // N index fastest so that concurrently running CTAs share the A panel.
 //
@@ -45,11 +46,12 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;     // TMA warp, MMA warp, epilogue warps
 constexpr int kAStage = BM * BK * 2;  // 16 KiB
 constexpr int kBStage = BN * BK * 2;  // 32 KiB
 constexpr int kTmemCols = 2 * BN;     // double-buffered accumulator
-constexpr int kSmemBytes = STAGES * (kAStage + kBStage) + 1024 + 256;
+constexpr int kSmemBytes = STAGES * (kAStage + kBStage) + 1024 + 24576;
 
 enum { EPI_STORE = 0, EPI_RESID = 1, EPI_FOLD = 2, EPI_SWIGLU_FWD = 3, EPI_SWIGLU_BWD = 4 };
 
@@ -61,8 +63,15 @@ struct Ctl {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
+  float2 xch[4][2][32];  // fold epilogue: per lane quarter, the two halves' group sums
+  uint64_t xbar[4];      // and the mbarrier that orders their exchange
+  // split reduction (two CTAs of a cluster): rank 1 ships 32 rows x 16 columns
+  // of its accumulator per message into rank 0's slot of the same epilogue warp
+  uint64_t full_x[kEpiWarps];   // rank 0: message landed (32 remote arrivals)
+  uint64_t empty_x[kEpiWarps];  // rank 1: slot free again (one remote arrival per message)
+  float slot[kEpiWarps][32][20];  // 16 floats per lane, padded against bank conflicts
 };
-static_assert(sizeof(Ctl) <= 256, "control block too large");
+static_assert(sizeof(Ctl) <= 24576, "control block too large");
 
 struct Params {
   int M, N, K;  // D is M x N, reduction over K
@@ -101,9 +110,9 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t stage_base, int kstep)
 // ---------------------------------------------------------------------------
 // epilogues: one thread = one output row, 32 columns per TMEM load
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void epi_store(const Params& p, uint32_t taddr, int row, int col_base) {
+__device__ __forceinline__ void epi_store(const Params& p, uint32_t taddr, int row, int col_base, int c0, int c1) {
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = c0; c < c1; ++c) {
     float v[32];
     tmem_ld32(taddr + c * 32, v);
     const int col0 = col_base + c * 32;
@@ -119,10 +128,11 @@ __device__ __forceinline__ void epi_store(const Params& p, uint32_t taddr, int r
   }
 }
 
-__device__ __forceinline__ double epi_resid(const Params& p, uint32_t taddr, int row, int col_base) {
+__device__ __forceinline__ double epi_resid(const Params& p, uint32_t taddr, int row, int col_base, int c0,
+                                            int c1) {
   double acc = 0.0;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = c0; c < c1; ++c) {
     float v[32];
     tmem_ld32(taddr + c * 32, v);
     const int col0 = col_base + c * 32;
@@ -159,118 +169,229 @@ __device__ __forceinline__ double epi_resid(const Params& p, uint32_t taddr, int
   return acc;
 }
 
+// p - lr*sign(d), clamped; sign(0) = sign(NaN) = 0.  p - (-lr) is the same
+// IEEE result as p + lr.
 __device__ __forceinline__ float sign_step(float p, float d, float lr, float lo, float hi) {
-  float r = p;
-  if (d > 0.0f) r = __fsub_rn(p, lr);
-  else if (d < 0.0f) r = __fadd_rn(p, lr);
-  return fminf(fmaxf(r, lo), hi);
+  const float step = d > 0.0f ? lr : (d < 0.0f ? -lr : 0.0f);
+  return fminf(fmaxf(__fsub_rn(p, step), lo), hi);
 }
 
 // Straight-through fold + SignSGD.  GEMM rows are weight rows n (M = N_w),
-// GEMM columns are weight columns k (N = K_w).  A group of g >= 32 columns
-// spans g/32 consecutive TMEM loads of this thread, so its sums are local.
-__device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n, int col_base) {
-  const FoldArgs& f = p.fold;
-  const int g = f.group_size;
-  const int cpg = g >> 5;
-  const int groups_per_row = p.N / g;
+// GEMM columns are weight columns k (N = K_w).  Each epilogue warp owns 32
+// rows and half of the tile's 256 columns (chunks c0..c0+3 of 32).  Groups of
+// g <= 128 columns lie inside one half, so their sums stay in the thread; a
+// group of 256 spans both halves and the two warps of a lane quarter add
+// their partial sums through shared memory (fixed order: half 0 + half 1).
+//
+// All global loads of the tile (group parameters, W and V of the first chunk)
+// are issued before waiting for the accumulator, and each next chunk's W and
+// V are loaded while the current chunk is computed.
+struct FoldChunk {
+  uint4 w[4];   // 32 bf16 weights
+  float4 v[8];  // 32 rounding offsets
+};
+
+__device__ __forceinline__ void fold_load(const FoldArgs& f, size_t e, FoldChunk& ch) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ch.w[i] = *reinterpret_cast<const uint4*>(f.W + e + 8 * i);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ch.v[i] = *reinterpret_cast<const float4*>(f.V + e + 4 * i);
+}
+
+struct GroupParams {
+  float s, zp, lo_s, mx, mn, al, be;
+  bool guarded, take_hi;
+  size_t gidx;
+};
+
+__device__ __forceinline__ void group_load(const FoldArgs& f, size_t gidx, GroupParams& gp) {
+  gp.gidx = gidx;
+  gp.s = f.s[gidx];
+  gp.zp = f.zp[gidx];
+  gp.mx = f.mx[gidx];
+  gp.mn = f.mn[gidx];
+  gp.al = f.alpha[gidx];
+  gp.be = f.beta[gidx];
+}
+
+__device__ __forceinline__ void group_prepare(const FoldArgs& f, GroupParams& gp) {
   const float Q = static_cast<float>((1 << f.bits) - 1);
   const float Qs = static_cast<float>((1 << (f.bits - 1)) - 1);
+  const float hi = __fmul_rn(gp.al, gp.mx);
+  const float lo = __fmul_rn(gp.be, gp.mn);
+  const float s_raw = f.symmetric ? __fdiv_rn(fmaxf(hi, -lo), Qs) : __fdiv_rn(__fsub_rn(hi, lo), Q);
+  gp.guarded = s_raw < kScaleGuard;
+  gp.take_hi = hi >= -lo;
+  gp.lo_s = __fdiv_rn(lo, gp.s);
+}
+
+// Finishes a group: dalpha, dbeta from the (full) sums and the SignSGD step of alpha, beta.
+__device__ __forceinline__ bool group_finish(const FoldArgs& f, const GroupParams& gp, float csum, float osum,
+                                             bool write) {
+  const float Q = static_cast<float>((1 << f.bits) - 1);
+  const float Qs = static_cast<float>((1 << (f.bits - 1)) - 1);
+  if (gp.guarded) csum = 0.0f;
+  float dhi, dlo;
+  if (f.symmetric) {
+    const float ds = __fdiv_rn(csum, Qs);
+    dhi = gp.take_hi ? ds : 0.0f;
+    dlo = gp.take_hi ? 0.0f : -ds;
+  } else {
+    const float cq = __fdiv_rn(csum, Q);
+    dhi = cq;
+    dlo = __fsub_rn(osum, cq);
+  }
+  const bool sums_bad = !isfinite(csum) || !isfinite(osum);
+  const float da = __fmul_rn(gp.mx, dhi);
+  const float db = __fmul_rn(gp.mn, dlo);
+  if (write) {
+    f.alpha[gp.gidx] = sign_step(gp.al, da, f.lr, f.c_min, f.c_max);
+    f.beta[gp.gidx] = sign_step(gp.be, db, f.lr, f.c_min, f.c_max);
+    if (f.da_out) f.da_out[gp.gidx] = da;
+    if (f.db_out) f.db_out[gp.gidx] = db;
+  }
+  return sums_bad || !isfinite(da) || !isfinite(db);
+}
+
+// `wait_acc` waits for the accumulator (returns false on abort); `xch` is this
+// lane quarter's exchange slot [2 halves][32 lanes] of float2 in shared memory
+// and `xbar` its mbarrier (two arrivals per phase, two phases per exchange).
+// Rank 0 of a split pair receives the peer's partial accumulator: per message
+// 16 columns of this warp's 32 rows, added as own + peer.
+struct SplitRecv {
+  bool on;
+  const float* slot;      // this lane's 16 floats
+  uint64_t* full;         // local barrier the peer arrives on
+  uint32_t peer_empty;    // the peer's slot-free barrier (cluster address)
+  uint32_t* msg;          // messages received so far by this warp
+};
+
+template <class WaitAcc>
+__device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n, int col_base, int half,
+                                         float2* xch, uint64_t* xbar, volatile int* abort_flag, WaitAcc wait_acc,
+                                         bool* aborted, const SplitRecv& rx) {
+  const FoldArgs& f = p.fold;
+  const int g = f.group_size;
+  const int cpg = g >> 5;  // chunks per group: 1, 2, 4 or 8
+  const int groups_per_row = p.N / g;
+  const float Q = static_cast<float>((1 << f.bits) - 1);
+  const int c0 = 4 * half;
+  const bool row_ok = n < p.M;
   bool bad = false;
-  float s = 1.f, zp = 0.f, lo_s = 0.f, mx = 0.f, mn = 0.f, al = 1.f, be = 1.f, csum = 0.f, osum = 0.f;
-  bool guarded = false, take_hi = true;
-  size_t gidx = 0;
+
+  GroupParams gp{};
+  FoldChunk cur, nxt;
+  // prefetch before the accumulator is ready
+  if (row_ok && col_base + c0 * 32 < p.N) {
+    const int col = col_base + c0 * 32;
+    group_load(f, static_cast<size_t>(n) * groups_per_row + col / g, gp);
+    fold_load(f, static_cast<size_t>(n) * p.N + col, nxt);
+  }
+  if (!wait_acc()) {
+    *aborted = true;
+    return false;
+  }
+  float csum = 0.f, osum = 0.f;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
-    float gw[32];
-    tmem_ld32(taddr + c * 32, gw);
+  for (int c = c0; c < c0 + 4; ++c) {
     const int col0 = col_base + c * 32;
-    if (n >= p.M || col0 >= p.N) continue;
-    if ((c % cpg) == 0) {
-      gidx = static_cast<size_t>(n) * groups_per_row + col0 / g;
-      s = f.s[gidx];
-      zp = f.zp[gidx];
-      mx = f.mx[gidx];
-      mn = f.mn[gidx];
-      al = f.alpha[gidx];
-      be = f.beta[gidx];
-      const float hi = __fmul_rn(al, mx);
-      const float lo = __fmul_rn(be, mn);
-      const float s_raw = f.symmetric ? __fdiv_rn(fmaxf(hi, -lo), Qs) : __fdiv_rn(__fsub_rn(hi, lo), Q);
-      guarded = s_raw < kScaleGuard;
-      take_hi = hi >= -lo;
-      lo_s = __fdiv_rn(lo, s);
+    const bool ok = row_ok && col0 < p.N;
+    cur = nxt;
+    if (ok && c + 1 < c0 + 4 && col0 + 32 < p.N) fold_load(f, static_cast<size_t>(n) * p.N + col0 + 32, nxt);
+    if (ok && ((c % cpg) == 0 || c == c0)) {
+      if (c != c0) group_load(f, static_cast<size_t>(n) * groups_per_row + col0 / g, gp);
+      group_prepare(f, gp);
       csum = 0.f;
       osum = 0.f;
     }
     const size_t e = static_cast<size_t>(n) * p.N + col0;
-    const uint16_t* wp = f.W + e;
-    float* vp = f.V + e;
-    uint32_t wr[16];
+    // two messages of 16 columns (split pairs), each two sub-blocks of 8 weights:
+    // one 16-byte W word, two 16-byte V words and 8 accumulator columns
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 t = *reinterpret_cast<const uint4*>(wp + 8 * i);
-      wr[4 * i] = t.x;
-      wr[4 * i + 1] = t.y;
-      wr[4 * i + 2] = t.z;
-      wr[4 * i + 3] = t.w;
-    }
-    float vv[32];
+    for (int sc = 0; sc < 2; ++sc) {
+      float part[16];
+      if (rx.on) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(rx.full, *rx.msg & 1u, abort_flag))) {
+          *aborted = true;
+          return bad;
+        }
+        const float4* src = reinterpret_cast<const float4*>(rx.slot);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 t = *reinterpret_cast<const float4*>(vp + 4 * i);
-      vv[4 * i] = t.x;
-      vv[4 * i + 1] = t.y;
-      vv[4 * i + 2] = t.z;
-      vv[4 * i + 3] = t.w;
-    }
-    float dv[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float w = (i & 1) ? bf16_hi(wr[i >> 1]) : bf16_lo(wr[i >> 1]);
-      const float wq = __fdiv_rn(w, s);
-      const float t = __fadd_rn(roundf(__fadd_rn(wq, vv[i])), zp);
-      const bool in = (t >= 0.0f) && (t <= Q);
-      const float qz = __fsub_rn(fminf(fmaxf(t, 0.0f), Q), zp);
-      const float gi = gw[i];
-      bad |= !isfinite(gi);
-      dv[i] = in ? __fmul_rn(gi, s) : 0.0f;
-      float ci;
-      if (f.symmetric) ci = __fmul_rn(gi, in ? __fsub_rn(qz, wq) : qz);
-      else ci = __fmul_rn(gi, __fsub_rn(qz, in ? wq : lo_s));
-      csum = __fadd_rn(csum, ci);
-      if (!in) osum = __fadd_rn(osum, gi);
-      vv[i] = sign_step(vv[i], dv[i], f.lr, f.v_min, f.v_max);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      *reinterpret_cast<float4*>(vp + 4 * i) = make_float4(vv[4 * i], vv[4 * i + 1], vv[4 * i + 2], vv[4 * i + 3]);
-    if (f.dV_out) {
-      float* dp = f.dV_out + e;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        *reinterpret_cast<float4*>(dp + 4 * i) = make_float4(dv[4 * i], dv[4 * i + 1], dv[4 * i + 2], dv[4 * i + 3]);
-    }
-    if ((c % cpg) == cpg - 1) {
-      if (guarded) csum = 0.0f;
-      float dhi, dlo;
-      if (f.symmetric) {
-        const float ds = __fdiv_rn(csum, Qs);
-        dhi = take_hi ? ds : 0.0f;
-        dlo = take_hi ? 0.0f : -ds;
-      } else {
-        const float cq = __fdiv_rn(csum, Q);
-        dhi = cq;
-        dlo = __fsub_rn(osum, cq);
+        for (int i = 0; i < 4; ++i) {
+          const float4 v = src[i];
+          part[4 * i] = v.x;
+          part[4 * i + 1] = v.y;
+          part[4 * i + 2] = v.z;
+          part[4 * i + 3] = v.w;
+        }
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive_remote(rx.peer_empty);
+        ++*rx.msg;
       }
-      const float da = __fmul_rn(mx, dhi);
-      const float db = __fmul_rn(mn, dlo);
-      bad |= !isfinite(da) || !isfinite(db);
-      f.alpha[gidx] = sign_step(al, da, f.lr, f.c_min, f.c_max);
-      f.beta[gidx] = sign_step(be, db, f.lr, f.c_min, f.c_max);
-      if (f.da_out) f.da_out[gidx] = da;
-      if (f.db_out) f.db_out[gidx] = db;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int sb = 2 * sc + h2;
+        float gw[8];
+        tmem_ld8(taddr + c * 32 + 8 * sb, gw);
+        if (rx.on) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) gw[i] = __fadd_rn(gw[i], part[8 * h2 + i]);
+        }
+        if (!ok) continue;
+        const uint32_t wr[4] = {cur.w[sb].x, cur.w[sb].y, cur.w[sb].z, cur.w[sb].w};
+        float vv[8] = {cur.v[2 * sb].x, cur.v[2 * sb].y, cur.v[2 * sb].z, cur.v[2 * sb].w,
+                       cur.v[2 * sb + 1].x, cur.v[2 * sb + 1].y, cur.v[2 * sb + 1].z, cur.v[2 * sb + 1].w};
+        float dv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float w = (i & 1) ? bf16_hi(wr[i >> 1]) : bf16_lo(wr[i >> 1]);
+          const float wq = __fdiv_rn(w, gp.s);
+          const float t = __fadd_rn(roundf(__fadd_rn(wq, vv[i])), gp.zp);
+          const bool in = (t >= 0.0f) && (t <= Q);
+          const float qz = __fsub_rn(fminf(fmaxf(t, 0.0f), Q), gp.zp);
+          const float gi = gw[i];
+          dv[i] = in ? __fmul_rn(gi, gp.s) : 0.0f;
+          float ci;
+          if (f.symmetric) ci = __fmul_rn(gi, in ? __fsub_rn(qz, wq) : qz);
+          else ci = __fmul_rn(gi, __fsub_rn(qz, in ? wq : gp.lo_s));
+          // a NaN/Inf gradient reaches csum (or osum) and is reported at the group's end
+          csum = __fadd_rn(csum, ci);
+          osum = in ? osum : __fadd_rn(osum, gi);
+          vv[i] = sign_step(vv[i], dv[i], f.lr, f.v_min, f.v_max);
+        }
+        float* vp = f.V + e + 8 * sb;
+        *reinterpret_cast<float4*>(vp) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+        *reinterpret_cast<float4*>(vp + 4) = make_float4(vv[4], vv[5], vv[6], vv[7]);
+        if (f.dV_out) {
+          float* dp = f.dV_out + e + 8 * sb;
+          *reinterpret_cast<float4*>(dp) = make_float4(dv[0], dv[1], dv[2], dv[3]);
+          *reinterpret_cast<float4*>(dp + 4) = make_float4(dv[4], dv[5], dv[6], dv[7]);
+        }
+      }
     }
+    if (!ok) continue;
+    if (cpg <= 4 && (c % cpg) == cpg - 1) bad |= group_finish(f, gp, csum, osum, true);
+  }
+  if (cpg == 8) {
+    // a 256-wide group: add the two halves' sums (the same order in both warps);
+    // phase 0 publishes both halves, phase 1 frees the slot for the next tile
+    const int lane = threadIdx.x & 31;
+    xch[half * 32 + lane] = make_float2(csum, osum);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(xbar);
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(xbar, 0, abort_flag))) {
+      *aborted = true;
+      return bad;
+    }
+    const float2 a = xch[lane];
+    const float2 b = xch[32 + lane];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(xbar);
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(xbar, 1, abort_flag))) {
+      *aborted = true;
+      return bad;
+    }
+    if (row_ok && col_base < p.N) bad |= group_finish(f, gp, __fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), half == 0);
   }
   return bad;
 }
@@ -280,9 +401,10 @@ __device__ __forceinline__ float sigmoidf(float x) { return __fdiv_rn(1.0f, __fa
 
 // SwiGLU forward: TMEM columns 0..127 hold the gate product a, 128..255 the
 // up product b of the same 128 outputs f.  Writes a, b, h = silu(a) b (bf16).
-__device__ __forceinline__ void epi_swiglu_fwd(const Params& p, uint32_t taddr, int row, int f_base) {
+__device__ __forceinline__ void epi_swiglu_fwd(const Params& p, uint32_t taddr, int row, int f_base, int c0,
+                                               int c1) {
 #pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
+  for (int c = c0; c < c1; ++c) {
     float va[32], vb[32];
     tmem_ld32(taddr + c * 32, va);
     tmem_ld32(taddr + 128 + c * 32, vb);
@@ -317,10 +439,11 @@ __device__ __forceinline__ void epi_swiglu_fwd(const Params& p, uint32_t taddr, 
 }
 
 // SiLU backward on dH (the accumulator): dA = dH b silu'(a), dB = dH silu(a).
-__device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, int row, int col_base) {
+__device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, int row, int col_base, int c0,
+                                               int c1) {
   bool bad = false;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = c0; c < c1; ++c) {
     float dh[32];
     tmem_ld32(taddr + c * 32, dh);
     const int col0 = col_base + c * 32;
@@ -384,7 +507,9 @@ __device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, 
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <bool A_MN, bool B_MN, int EPI>
+// KSPLIT = 2 (weight-gradient GEMM only): the two CTAs of a cluster share each
+// tile, rank 0 reducing the first half of the k-blocks and rank 1 the second.
+template <bool A_MN, bool B_MN, int EPI, int KSPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmB2, const Params p) {
@@ -397,17 +522,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_tiles = p.tiles_m * p.tiles_n;
+  const int rank = KSPLIT == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int tile0 = KSPLIT == 2 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int tile_step = KSPLIT == 2 ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+  const int kb_begin = (KSPLIT == 2 && rank == 1) ? p.num_kb / 2 : 0;
+  const int kb_end = (KSPLIT == 2 && rank == 0) ? p.num_kb / 2 : p.num_kb;
 
   if (threadIdx.x == 0) {
+    for (int w = 0; w < kEpiWarps; ++w) {
+      mbar_init(&ctl->full_x[w], 32);
+      mbar_init(&ctl->empty_x[w], 1);
+    }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ctl->tmem_full[a], 1);
-      mbar_init(&ctl->tmem_empty[a], 4);
+      mbar_init(&ctl->tmem_empty[a], kEpiWarps);
     }
     mbar_init(&ctl->mma_done, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&ctl->xbar[q], 2);
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
@@ -423,6 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (KSPLIT == 2) cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == 0) {
@@ -431,10 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int t = tile0; ok && t < num_tiles; t += tile_step) {
         const int tm = t / p.tiles_n;
         const int tn = t - tm * p.tiles_n;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -475,11 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int t = tile0; ok && t < num_tiles; t += tile_step) {
         if (!mbar_wait(&ctl->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -490,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
             umma_bf16(d, operand_desc<A_MN>(a_base, j), operand_desc<B_MN>(b_base, j), idesc,
-                      (kb | j) != 0 ? 1u : 0u);
+                      (kb != kb_begin || j != 0) ? 1u : 0u);
           }
           umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) {
@@ -509,32 +645,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // warp -> TMEM lane quarter (warp % 4, hardware rule) and column half
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     uint32_t acc = 0, acc_phase = 0;
-    double loss_acc = 0.0;
     bool bad = false;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const bool got = mbar_wait(&ctl->tmem_full[acc], acc_phase, abort_flag);
-      if (!__all_sync(0xFFFFFFFFu, got)) break;
-      tc_fence_after();
+    const int ew = warp - 2;  // epilogue warp index 0..7
+    uint32_t msg = 0;
+    SplitRecv rx{};
+    if (KSPLIT == 2 && rank == 0) {
+      rx.on = true;
+      rx.slot = &ctl->slot[ew][lane][0];
+      rx.full = &ctl->full_x[ew];
+      rx.peer_empty = mapa_shared(smem_u32(&ctl->empty_x[ew]), 1);
+      rx.msg = &msg;
+    }
+    const uint32_t peer_slot = KSPLIT == 2 ? mapa_shared(smem_u32(&ctl->slot[ew][lane][0]), 0) : 0;
+    const uint32_t peer_full = KSPLIT == 2 ? mapa_shared(smem_u32(&ctl->full_x[ew]), 0) : 0;
+    for (int t = tile0; t < num_tiles; t += tile_step) {
       const int tm = t / p.tiles_n;
       const int tn = t - tm * p.tiles_n;
       const int row = tm * BM + quarter * 32 + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-      if (EPI == EPI_STORE) {
-        epi_store(p, taddr, row, tn * BN);
-      } else if (EPI == EPI_RESID) {
-        double part = epi_resid(p, taddr, row, tn * BN);
+      auto wait_acc = [&]() {
+        const bool got = mbar_wait(&ctl->tmem_full[acc], acc_phase, abort_flag);
+        if (!__all_sync(0xFFFFFFFFu, got)) return false;
+        tc_fence_after();
+        return true;
+      };
+      if (KSPLIT == 2 && rank == 1) {
+        // ship this warp's 32 rows x 128 columns to rank 0, 16 columns per message
+        if (!wait_acc()) break;
+        bool aborted = false;
+        for (int c = 4 * half; c < 4 * half + 4 && !aborted; ++c) {
+          float v[32];
+          tmem_ld32(taddr + c * 32, v);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
-        if (lane == 0) p.partial[static_cast<size_t>(t) * 4 + quarter] = part;
-        (void)loss_acc;
+          for (int sc = 0; sc < 2; ++sc) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&ctl->empty_x[ew], (msg & 1u) ^ 1u, abort_flag))) {
+              aborted = true;
+              break;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              st_cluster_v4(peer_slot + 16 * i, v[16 * sc + 4 * i], v[16 * sc + 4 * i + 1], v[16 * sc + 4 * i + 2],
+                            v[16 * sc + 4 * i + 3]);
+            mbar_arrive_remote(peer_full);
+            ++msg;
+          }
+        }
+        if (aborted) break;
       } else if (EPI == EPI_FOLD) {
-        bad |= epi_fold(p, taddr, row, tn * BN);
-      } else if (EPI == EPI_SWIGLU_FWD) {
-        epi_swiglu_fwd(p, taddr, row, tn * (BN / 2));
+        bool aborted = false;
+        bad |= epi_fold(p, taddr, row, tn * BN, half, &ctl->xch[quarter][0][0], &ctl->xbar[quarter], abort_flag,
+                        wait_acc, &aborted, rx);
+        if (aborted) break;
       } else {
-        bad |= epi_swiglu_bwd(p, taddr, row, tn * BN);
+        if (!wait_acc()) break;
+        if (EPI == EPI_STORE) {
+          epi_store(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
+        } else if (EPI == EPI_RESID) {
+          double part = epi_resid(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
+          if (lane == 0) p.partial[static_cast<size_t>(t) * kEpiWarps + half * 4 + quarter] = part;
+        } else if (EPI == EPI_SWIGLU_FWD) {
+          epi_swiglu_fwd(p, taddr, row, tn * (BN / 2), 2 * half, 2 * half + 2);
+        } else {
+          bad |= epi_swiglu_bwd(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -547,6 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (KSPLIT == 2) cluster_sync_all();  // the peer may still read or write this CTA's shared memory
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -562,7 +742,7 @@ cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t 
                       CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, int KSPLIT = 1>
 cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t stream, const char* name,
                 const uint16_t* B2 = nullptr) {
   CUtensorMap tmA, tmB, tmB2;
@@ -582,15 +762,38 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
   p.tiles_m = (p.M + BM - 1) / BM;
   p.tiles_n = EPI == EPI_SWIGLU_FWD ? (p.N + BN / 2 - 1) / (BN / 2) : (p.N + BN - 1) / BN;
   p.num_kb = (p.K + BK - 1) / BK;
-  auto kern = umma_gemm_kernel<A_MN, B_MN, EPI>;
+  auto kern = umma_gemm_kernel<A_MN, B_MN, EPI, KSPLIT>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
-  const int grid = tiles < num_sms() ? tiles : num_sms();
-  {
+  if (KSPLIT == 1) {
+    const int grid = tiles < num_sms() ? tiles : num_sms();
     LaunchScope scope(stream, name);
     kern<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmB2, p);
+    return cudaGetLastError();
   }
+  // pairs of CTAs: as many clusters as can be resident at once, at most one per tile
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int max_clusters = 0;
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+  cfg.gridDim = dim3(2 * clusters);
+  LaunchScope scope(stream, name);
+  e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmB2, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -642,7 +845,7 @@ cudaError_t make_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, uint32_t el
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-int resid_partials(int M, int N) { return ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * 4; }
+int resid_partials(int M, int N) { return ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * kEpiWarps; }
 
 cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,
                               cudaStream_t stream) {
@@ -675,6 +878,18 @@ cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArg
   p.N = K;
   p.K = M;
   p.fold = fa;
+  // Split the token reduction over CTA pairs when pairs fill the last wave
+  // better and each half of the reduction still outlasts the fold epilogue of
+  // a tile (~60 us, compute bound), i.e. from 32768 tokens on; below that the
+  // epilogue paces the pair and the unsplit kernel is faster (measured on
+  // 16384 tokens: 533 us split vs 511 us unsplit for a 4096 x 4096 layer).
+  const int tiles = ((N + BM - 1) / BM) * ((K + BN - 1) / BN);
+  const int sms = num_sms();
+  const double eff1 = static_cast<double>(tiles) / (((tiles + sms - 1) / sms) * sms);
+  const int pairs = sms / 2;
+  const double eff2 = static_cast<double>(tiles) / (((tiles + pairs - 1) / pairs) * pairs);
+  if (M >= 32768 && eff2 > eff1 + 0.02)
+    return run<true, true, EPI_FOLD, 2>(G, X, p, stream, "umma_gemm<MN,MN,fold,split2>");
   return run<true, true, EPI_FOLD>(G, X, p, stream, "umma_gemm<MN,MN,fold>");
 }
 

@@ -103,6 +103,9 @@ cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, b
 cudaError_t launch_loss_reduce(const double* partials, int n, int steps, double inv_count, float* loss,
                                cudaStream_t stream);
 
+// Diagnostic wait that is bound to time out (see ar_debug_wait_timeout).
+cudaError_t launch_wait_timeout(uint64_t limit_ns, int* gave_up, cudaStream_t stream);
+
 // Synchronizes `stream`, copies the sticky device status to *out and clears it.
 cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t stream);
 

@@ -30,6 +30,37 @@ cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t stream) {
   return cudaMemcpyToSymbol(g_status, &zero, sizeof(unsigned int));
 }
 
+// Diagnostic: one warp waits on an mbarrier that nothing arrives on, with a
+// limit of `limit_ns`; the bounded wait gives up, raises the timeout status
+// and the kernel returns normally.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, int* gave_up) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const uint32_t addr = smem_u32(&bar);
+  const uint64_t t0 = globaltimer_ns();
+  bool done = false;
+  while (!done) {
+    if (mbar_try_wait(addr, 0)) break;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      done = true;
+      if (threadIdx.x == 0) {
+        raise_status(kStatusTimeout);
+        *gave_up = 1;
+      }
+    }
+  }
+}
+
+cudaError_t launch_wait_timeout(uint64_t limit_ns, int* gave_up, cudaStream_t stream) {
+  LaunchScope scope(stream, "wait_timeout_kernel");
+  wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_ns, gave_up);
+  return cudaGetLastError();
+}
+
 struct QParams {
   float s, zp, lo, mx, mn;
   bool guarded;

@@ -121,6 +121,12 @@ def test_pack_and_w4a16_validation():
     assert ar.lib().ar_gemm_bf16(FAKE, 1, FAKE, 0, FAKE, 12, 64, 64, None) == ar.AR_ERR_INVALID_ARG
 
 
+def test_debug_wait_validation():
+    assert ar.lib().ar_debug_wait_timeout(0, FAKE, None) == ar.AR_ERR_INVALID_ARG
+    assert ar.lib().ar_debug_wait_timeout(2_000_000_000, FAKE, None) == ar.AR_ERR_INVALID_ARG
+    assert ar.lib().ar_debug_wait_timeout(1000, None, None) == ar.AR_ERR_INVALID_ARG
+
+
 def test_binding_refuses_host_tensors():
     import torch
 

@@ -401,3 +401,38 @@ def test_nonfinite_weight_raises_status(ar):
     ar.ar_qdq(bf16_dev(Wb), f32_dev(V), f32_dev(a), f32_dev(b), cfg, What)
     assert ar.ar_get_device_status() == ar.AR_ERR_NONFINITE
     assert ar.ar_get_device_status() == 0  # sticky until read, then cleared
+
+
+@pytest.mark.parametrize("g", [128, 256])
+def test_split_reduction_pairs_match_oracle(ar, g):
+    """32768 tokens over a 512x512 layer: the weight-gradient GEMM splits the token
+    reduction across CTA pairs (rank 1 ships its partial accumulator to rank 0).
+    Every output row is checked against the oracle."""
+    N, K, M = 512, 512, 32768
+    d = synth.make_linear(N, K, M, seed=31 + g)
+    V, a, b = synth.make_state(N, K, g, seed=4, spread=True)
+    cfg, ocfg = cfg_pair(ar, 4, g)
+    gl = GpuLinear(ar, d["W"], d["X"], V, a, b, cfg)
+    out = gl.step(1, grads=True)
+    assert "split2" in ar.ar_last_kernels()
+    Wf, Xf = synth.bf16_bits_to_f32(d["W"]), synth.bf16_bits_to_f32(d["X"])
+    L, (V1, a1, b1), gr, _ = O.tune_step_linear(Wf, Xf, O.reference_forward(Xf, Wf), V, a, b, ocfg)
+    assert out["loss"][0] == pytest.approx(L, rel=1e-4)
+    for k in ("dV", "dalpha", "dbeta"):
+        assert rel_l2(out[k], gr[k]) <= GRAD_RTOL, (k, rel_l2(out[k], gr[k]))
+    Vg, ag, bg = gl.state()
+    assert np.mean(Vg == V1) >= SIGN_AGREE and np.mean(ag == a1) >= 0.99 and np.mean(bg == b1) >= 0.99
+
+
+def test_bounded_wait_gives_up_and_reports_timeout(ar):
+    """A device wait on a barrier nothing completes ends after its limit with AR_ERR_TIMEOUT;
+    the context stays usable (a normal call follows)."""
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ar.ar_debug_wait_timeout(20_000_000, flag)  # 20 ms
+    assert ar.ar_get_device_status() == ar.AR_ERR_TIMEOUT
+    assert int(flag.item()) == 1
+    assert ar.ar_get_device_status() == 0
+    x = np.arange(8, dtype=np.float32)
+    out = torch.empty(8, dtype=torch.bfloat16, device="cuda")
+    ar.ar_f32_to_bf16(f32_dev(x), out)
+    assert out.float().cpu().numpy().tolist() == x.tolist()
