@@ -226,11 +226,15 @@ AR_API ar_status ar_pack_int4(const uint16_t* W, const float* V, const float* al
  *   out[t][n] = sum_k A[t][k] (q[n][k] - zero[n][k/g]) scale[n][k/g]
  * A bf16 [T][K]; packed/scale/zero as written by ar_pack_int4 (zero must hold
  * integers 0..15, as ar_pack_int4 writes them); out bf16 [T][N] (round to
- * nearest even of the fp32 accumulation).  (q - zero) is exact in bf16, each
- * 32-k slice's product is accumulated in fp32 on the tensor cores and scaled
- * by its group's scale in fp32.
- * Supported: 1 <= T <= 16, group_size 32..1024 (power of two) dividing K,
- * K % 128 == 0.  Larger T returns AR_ERR_UNSUPPORTED. */
+ * nearest even of the fp32 accumulation).  (q - zero) is exact in bf16; the
+ * products are accumulated in fp32 on the tensor cores, one group (or 32-k
+ * slice of a group) at a time, and scaled by the group's scale in fp32.
+ * T <= 16 runs a decode kernel (mma.sync fragments built in registers);
+ * larger T a tcgen05 GEMM that dequantizes each 128-row x 64-k tile of codes
+ * into shared memory.  Results are deterministic for a given T.
+ * Supported: 1 <= T < 2^31, group_size 32..1024 (power of two) dividing K,
+ * K % 128 == 0; anything else returns AR_ERR_UNSUPPORTED or
+ * AR_ERR_INVALID_ARG before any launch. */
 AR_API ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, const uint16_t* scale_f16,
                         const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, uint16_t* out,
                         ar_stream_t stream);

@@ -569,18 +569,19 @@ ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
                         ar_stream_t stream) {
   begin_call();
   if (T < 1 || N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "T, N, K must be positive");
-  if (T > 16) return fail(AR_ERR_UNSUPPORTED, "T=%lld: this build supports 1 <= T <= 16", (long long)T);
   if (!pow2(group_size) || group_size < 32 || group_size > 1024)
     return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 32..1024", group_size);
   if (K % group_size != 0 || K % 128 != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and 128");
-  if (N > INT32_MAX || K > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  if (N > INT32_MAX || K > INT32_MAX || T > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
   const void* ptrs[] = {A, packed, scale_f16, zero_f16, out};
   for (const void* p : ptrs) {
     if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   }
-  cudaError_t e = launch_w4a16(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N),
-                               static_cast<int>(K), group_size, out, reinterpret_cast<cudaStream_t>(stream));
+  // decode batches: CUDA-core dequant into mma.sync fragments; larger: tcgen05 dequant GEMM
+  auto launch = T <= 16 ? launch_w4a16 : launch_w4a16_tc;
+  cudaError_t e = launch(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N), static_cast<int>(K),
+                         group_size, out, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "w4a16 launch");
   return end_call();
 }

@@ -112,7 +112,8 @@ def test_pack_and_w4a16_validation():
     assert ar.lib().ar_pack_int4(FAKE, FAKE, FAKE, FAKE, 8, 128, ctypes.byref(cfg3), FAKE, FAKE, FAKE, None) == \
         ar.AR_ERR_UNSUPPORTED
     w4 = ar.lib().ar_w4a16_gemm
-    assert w4(FAKE, 17, FAKE, FAKE, FAKE, 64, 256, 128, FAKE, None) == ar.AR_ERR_UNSUPPORTED
+    assert w4(FAKE, 1 << 31, FAKE, FAKE, FAKE, 64, 256, 128, FAKE, None) == ar.AR_ERR_UNSUPPORTED
+    assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 4096, 2048, FAKE, None) == ar.AR_ERR_UNSUPPORTED
     assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 16, FAKE, None) == ar.AR_ERR_UNSUPPORTED
     assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 200, 128, FAKE, None) == ar.AR_ERR_INVALID_ARG
     assert w4(FAKE, 1, FAKE, FAKE, FAKE, 64, 96, 32, FAKE, None) == ar.AR_ERR_INVALID_ARG  # K % 128

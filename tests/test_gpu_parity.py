@@ -24,6 +24,10 @@ SIGN_AGREE = 0.999
 CODE_AGREE = 0.995
 MSE_RTOL = 0.01
 W4A16_RTOL = 2e-2
+# tcgen05 W4A16 path: (q - z) and every product are exact, groups are summed in
+# fp32, so the bf16 rounding of the output (relative 2^-9 per element) bounds
+# the relative L2 error, plus a little fp32 summation error.
+W4A16_TC_RTOL = 3e-3
 
 
 @pytest.fixture(scope="module")
@@ -368,7 +372,44 @@ def test_w4a16_matches_oracle(ar, T, N, K, g):
     assert rel_l2(got, ref) <= W4A16_RTOL
 
 
-@pytest.mark.parametrize("T", [1, 16])
+@pytest.mark.parametrize("T", [17, 40, 64, 100, 256])
+@pytest.mark.parametrize("N,K,g", [(320, 1024, 128), (64, 4096, 32), (40, 2048, 1024)])
+def test_w4a16_tensor_core_path_matches_oracle(ar, T, N, K, g):
+    """T > 16 runs the tcgen05 dequant GEMM (one group per TMEM accumulator)."""
+    d = synth.make_linear(N, K, 1, seed=T + N)
+    V, a, b = synth.make_state(N, K, g, seed=2, spread=True)
+    packed, s16, z16 = _packed(ar, d["W"], V, a, b, g)
+    A = synth.make_activations(T, K, seed=T)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_w4a16_gemm(bf16_dev(A), packed, s16, z16, g, out)
+    assert "w4a16_tc_kernel" in ar.ar_last_kernels()
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 4, g)
+    words, s_ref, z_ref = O.pack_int4(st["q"], st["s"], st["zp"])
+    ref = O.w4a16_matmul(synth.bf16_bits_to_f32(A), words, s_ref, z_ref, g)
+    assert rel_l2(out.float().cpu().numpy(), ref) <= W4A16_TC_RTOL
+
+
+def test_w4a16_tensor_core_path_many_tiles(ar):
+    """Enough (row, token) tiles that K is not split; ragged token tail (1000 = 7 x 128 + 104)."""
+    N, K, g, T = 1280, 512, 64, 1000
+    d = synth.make_linear(N, K, 1, seed=11)
+    V, a, b = synth.make_state(N, K, g, seed=3, spread=True)
+    packed, s16, z16 = _packed(ar, d["W"], V, a, b, g)
+    A = synth.make_activations(T, K, seed=12)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_w4a16_gemm(bf16_dev(A), packed, s16, z16, g, out)
+    assert "w4a16_tc_kernel<TN=128>" in ar.ar_last_kernels()
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 4, g)
+    words, s_ref, z_ref = O.pack_int4(st["q"], st["s"], st["zp"])
+    ref = O.w4a16_matmul(synth.bf16_bits_to_f32(A), words, s_ref, z_ref, g)
+    got = out.float().cpu().numpy()
+    assert rel_l2(got, ref) <= W4A16_TC_RTOL
+    # every token row on its own (a wrong tile origin would show in one row only)
+    for t in (0, 127, 128, 895, 896, 999):
+        assert rel_l2(got[t], ref[t]) <= W4A16_TC_RTOL
+
+
+@pytest.mark.parametrize("T", [1, 16, 64, 256])
 def test_w4a16_full_size_sampled_rows(ar, T):
     """8192 x 28672 down projection, sampled output rows against the oracle."""
     wl = synth.WORKLOADS["down_8192_28672"]
