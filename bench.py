@@ -257,7 +257,7 @@ def w4a16_bench(ar, torch, peaks, reps=20):
     # competes with the measured kernel)
     flush = torch.ones(64 * 1024 * 1024, dtype=torch.int32, device="cuda")
     out = {}
-    for T in (1, 4, 16):
+    for T in (1, 4, 16, 256):
         A = to_dev_bf16(synth.make_activations(T, K, seed=T), torch)
         y = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
         for _ in range(3):
@@ -272,7 +272,14 @@ def w4a16_bench(ar, torch, peaks, reps=20):
         ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
         nbytes = packed.numel() * 4 + s16.numel() * 2 + z16.numel() * 2 + A.numel() * 2 + y.numel() * 2
         gbs = nbytes / (ms * 1e-3) / 1e9
-        out[f"T{T}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+        flops = 2.0 * T * N * K
+        tfs = flops / (ms * 1e-3) / 1e12
+        peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        # roofline: the slower of the HBM time of the bytes and the tensor time of the FLOPs
+        t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peak_tf * 1e12))
+        out[f"T{T}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "TFLOP/s": tfs,
+                        "bound": "hbm" if nbytes / peaks["hbm_gbs"] / 1e9 >= flops / peak_tf / 1e12 else "tensor",
+                        "roofline_frac": t_roof / (ms * 1e-3),
                         "algorithmic_bytes": nbytes, "kernel": ar.ar_last_kernels()}
     out["shape"] = f"{N}x{K} int4 g{g}, fp16 scale/zero, bf16 activations; L2 flushed before each launch"
     return out

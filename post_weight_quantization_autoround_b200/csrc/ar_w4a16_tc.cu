@@ -61,15 +61,18 @@ constexpr int kACol0 = 256;   // TMEM column of A stage 0; stage s at kACol0 + k
 constexpr int kTmemCols = 512;
 // Warp roles: 0 activation TMA, 1 TMEM owner + MMA issuer, 2 code TMA, then the
 // dequantization warps, then the epilogue warps.
-constexpr int kDqWarps = 4;   // a multiple of 4: 32 rows each, stages round robin
 constexpr int kEpWarps = 8;   // a multiple of 4: kEpWarps / 4 per TMEM lane quarter
 constexpr int kEpQ = kEpWarps / 4;
 constexpr int kDqWarp0 = 3;
-constexpr int kEpWarp0 = kDqWarp0 + kDqWarps;
-constexpr int kTcThreads = (kEpWarp0 + kEpWarps) * 32;
 
 template <int TN>
 struct TcCfg {
+  // One dequantization warp per TMEM lane quarter is latency bound (its nibble
+  // and permute chains), so narrow tiles, whose epilogue needs few registers,
+  // run two per quarter on alternating stages.
+  static constexpr int kDqWarps = TN >= 128 ? 4 : 8;
+  static constexpr int kEpWarp0 = kDqWarp0 + kDqWarps;
+  static constexpr int kThreads = (kEpWarp0 + kEpWarps) * 32;
   static constexpr int kActBytes = TN * 128 * kSub;    // TN tokens x kTcK k bf16, kSub sub-tiles
   static constexpr int kStageBytes = kActBytes;
   static constexpr int kStages = kAStages;
@@ -243,7 +246,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // Grid: one CTA per (128-row tile, token tile, K half when split); the CTAs of
 // a weight tile are adjacent so that its codes come from HBM once.
 template <int TN, int KSPLIT>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const TcParams p) {
   using Cfg = TcCfg<TN>;
@@ -305,9 +308,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float acc[Cfg::kCols];
 #pragma unroll
   for (int i = 0; i < Cfg::kCols; ++i) acc[i] = 0.f;
-  const bool is_epi = warp >= kEpWarp0;
+  const bool is_epi = warp >= Cfg::kEpWarp0;
   const int quarter = warp & 3;                      // TMEM lane quarter of an epilogue warp
-  const int esub = (warp - kEpWarp0) >> 2;           // 0..kEpQ-1 among the warps of a lane quarter
+  const int esub = (warp - Cfg::kEpWarp0) >> 2;           // 0..kEpQ-1 among the warps of a lane quarter
   const int ecol = esub % Cfg::kColSplit;            // column part
   const int egrp = esub / Cfg::kColSplit;            // group residue
 
@@ -440,7 +443,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     zrow.start(p.z16 + static_cast<size_t>(n < p.N ? n : 0) * p.G, g_begin, p.G, p.vec_meta != 0, n < p.N);
     const uint32_t sw = static_cast<uint32_t>(r & 7);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0;
-    for (int i = dw >> 2; i < c_end - c_begin; i += kDqWarps / 4) {
+    for (int i = dw >> 2; i < c_end - c_begin; i += Cfg::kDqWarps / 4) {
       const int c = c_begin + i;
       const uint32_t stage = static_cast<uint32_t>(i % Cfg::kStages);
       const uint32_t phase = static_cast<uint32_t>((i / Cfg::kStages) & 1);
@@ -530,7 +533,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = 0; i < Cfg::kCols; ++i) dst[i] = acc[i];
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kTcRows * TN; e += kTcThreads) {
+  for (int e = threadIdx.x; e < kTcRows * TN; e += Cfg::kThreads) {
     const int r = e % kTcRows;
     const int c = e / kTcRows;
     float v = red[r * Cfg::kRedStride + c];
@@ -547,7 +550,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     cluster_sync_all();
     if (rank == 0) {
       const float* peer = cg::this_cluster().map_shared_rank(fin, 1);
-      for (int e = threadIdx.x; e < kTcRows * TN; e += kTcThreads) {
+      for (int e = threadIdx.x; e < kTcRows * TN; e += Cfg::kThreads) {
         const int r = e % kTcRows;
         const int c = e / kTcRows;
         const float v = fin[r * Cfg::kRedStride + c] + peer[r * Cfg::kRedStride + c];
@@ -583,7 +586,7 @@ cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(n_tiles * p.t_tiles * KSPLIT));
-  cfg.blockDim = dim3(kTcThreads);
+  cfg.blockDim = dim3(Cfg::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
