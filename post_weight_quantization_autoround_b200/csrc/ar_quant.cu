@@ -102,13 +102,23 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ W
   const bool active = grp < n_groups;
   const int64_t gbase = (active ? grp : 0) * static_cast<int64_t>(G);  // element offset of the group
 
+  // Every load is issued before the group reduction, so the V, alpha and beta
+  // round trips overlap the W one instead of following it.
   uint4 wv[CHUNKS];
+  float4 v0[CHUNKS], v1[CHUNKS];
+#pragma unroll
+  for (int c = 0; c < CHUNKS; ++c) {
+    const int64_t e = gbase + (static_cast<int64_t>(c) * TPG + li) * 8;
+    wv[c] = active ? __ldcs(reinterpret_cast<const uint4*>(W + e)) : make_uint4(0, 0, 0, 0);
+    v0[c] = active ? __ldcs(reinterpret_cast<const float4*>(V + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    v1[c] = active ? __ldcs(reinterpret_cast<const float4*>(V + e + 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float ga = active ? alpha[grp] : 1.0f;
+  const float gb = active ? beta[grp] : 1.0f;
   float lmax = -INFINITY, lmin = INFINITY;
   bool bad = false;
 #pragma unroll
   for (int c = 0; c < CHUNKS; ++c) {
-    const int64_t e = gbase + (static_cast<int64_t>(c) * TPG + li) * 8;
-    wv[c] = active ? *reinterpret_cast<const uint4*>(W + e) : make_uint4(0, 0, 0, 0);
     const uint32_t wr[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -128,15 +138,13 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ W
 
   const float mx = fmaxf(lmax, 0.0f);
   const float mn = fminf(lmin, 0.0f);
-  const QParams p = group_qparams(mx, mn, alpha[grp], beta[grp], bits, symmetric);
+  const QParams p = group_qparams(mx, mn, ga, gb, bits, symmetric);
   const float Q = static_cast<float>((1 << bits) - 1);
 
 #pragma unroll
   for (int c = 0; c < CHUNKS; ++c) {
     const int64_t e = gbase + (static_cast<int64_t>(c) * TPG + li) * 8;
-    const float4 v0 = *reinterpret_cast<const float4*>(V + e);
-    const float4 v1 = *reinterpret_cast<const float4*>(V + e + 4);
-    const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const float vv[8] = {v0[c].x, v0[c].y, v0[c].z, v0[c].w, v1[c].x, v1[c].y, v1[c].z, v1[c].w};
     const uint32_t wr[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
     float wh[8];
     uint32_t qb[2] = {0, 0};
