@@ -277,12 +277,14 @@ cudaError_t launch_qdq(const uint16_t* W, const float* V, const float* alpha, co
   const int64_t n_groups = N * (K / group_size);
   const int groups_per_row = static_cast<int>(K / group_size);
   switch (group_size) {
+    // two 8-element chunks per thread from g = 16 up: twice the loads in flight
+    // per thread at the same occupancy (HBM latency needs ~44 KB in flight per SM)
     AR_QDQ_CASE(1, 1)
-    AR_QDQ_CASE(2, 1)
-    AR_QDQ_CASE(4, 1)
-    AR_QDQ_CASE(8, 1)
-    AR_QDQ_CASE(16, 1)
-    AR_QDQ_CASE(32, 1)
+    AR_QDQ_CASE(1, 2)
+    AR_QDQ_CASE(2, 2)
+    AR_QDQ_CASE(4, 2)
+    AR_QDQ_CASE(8, 2)
+    AR_QDQ_CASE(16, 2)
     AR_QDQ_CASE(32, 2)
     AR_QDQ_CASE(32, 4)
     default:
