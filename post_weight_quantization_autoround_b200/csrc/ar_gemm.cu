@@ -42,22 +42,33 @@
 namespace ar {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;   // A rows per CTA (MMA M of one CTA)
+constexpr int BN = 256;   // output columns per tile
 constexpr int BK = 64;
-constexpr int STAGES = 4;
+constexpr int kMaxStages = 6;
 constexpr int kEpiWarps = 8;                       // two per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;     // TMA warp, MMA warp, epilogue warps
 constexpr int kAStage = BM * BK * 2;  // 16 KiB
-constexpr int kBStage = BN * BK * 2;  // 32 KiB
 constexpr int kTmemCols = 2 * BN;     // double-buffered accumulator
-constexpr int kSmemBytes = STAGES * (kAStage + kBStage) + 1024 + 24576;
+
+// CG = 1: one CTA per 128 x 256 tile.  CG = 2: a CTA pair per 256 x 256 tile
+// (tcgen05 .cta_group::2): each CTA loads its 128 A rows and half of the B
+// columns, so per SM the operand traffic from L2 falls from 48 to 32 KiB per
+// 64-k block of the same MMA work.
+template <int CG>
+struct GemmCfg {
+  static constexpr int kBStage = (BN / CG) * BK * 2;  // 32 or 16 KiB
+  static constexpr int kStages = CG == 2 ? 6 : 4;
+  static constexpr int kSmemBytes = kStages * (kAStage + kBStage) + 1024 + 24576;
+  static_assert(kStages <= kMaxStages, "barrier arrays");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
 
 enum { EPI_STORE = 0, EPI_RESID = 1, EPI_FOLD = 2, EPI_SWIGLU_FWD = 3, EPI_SWIGLU_BWD = 4 };
 
 struct Ctl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t mma_done;
@@ -509,10 +520,18 @@ __device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, 
 // ---------------------------------------------------------------------------
 // KSPLIT = 2 (weight-gradient GEMM only): the two CTAs of a cluster share each
 // tile, rank 0 reducing the first half of the k-blocks and rank 1 the second.
-template <bool A_MN, bool B_MN, int EPI, int KSPLIT>
+// CG = 2: the two CTAs of a cluster compute one 256 x 256 tile as a tcgen05
+// pair; rank 0 issues the MMAs, each rank drains its own 128 rows.
+template <bool A_MN, bool B_MN, int EPI, int KSPLIT, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmB2, const Params p) {
+  static_assert(!(KSPLIT == 2 && CG == 2), "a cluster is either a split pair or a tcgen05 pair");
+  static_assert(CG == 1 || (EPI != EPI_SWIGLU_FWD && EPI != EPI_SWIGLU_BWD), "SwiGLU tiles pair gate and up rows");
+  constexpr int STAGES = GemmCfg<CG>::kStages;
+  constexpr int kBStage = GemmCfg<CG>::kBStage;
+  constexpr bool kPair = CG == 2;
+  constexpr bool kCluster = KSPLIT == 2 || kPair;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smA = base;
@@ -522,11 +541,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_tiles = p.tiles_m * p.tiles_n;
-  const int rank = KSPLIT == 2 ? static_cast<int>(cluster_ctarank()) : 0;
-  const int tile0 = KSPLIT == 2 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
-  const int tile_step = KSPLIT == 2 ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+  const int rank = kCluster ? static_cast<int>(cluster_ctarank()) : 0;
+  const int tile0 = kCluster ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int tile_step = kCluster ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
   const int kb_begin = (KSPLIT == 2 && rank == 1) ? p.num_kb / 2 : 0;
   const int kb_end = (KSPLIT == 2 && rank == 0) ? p.num_kb / 2 : p.num_kb;
+  const bool leader = !kPair || rank == 0;  // issues the MMAs (always, unless a pair's odd CTA)
 
   if (threadIdx.x == 0) {
     for (int w = 0; w < kEpiWarps; ++w) {
@@ -539,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ctl->tmem_full[a], 1);
-      mbar_init(&ctl->tmem_empty[a], kEpiWarps);
+      mbar_init(&ctl->tmem_empty[a], kEpiWarps * CG);  // a pair's accumulator is drained by both CTAs
     }
     mbar_init(&ctl->mma_done, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&ctl->xbar[q], 2);
@@ -552,13 +572,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (EPI == EPI_SWIGLU_FWD) tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, kTmemCols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&ctl->tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (KSPLIT == 2) cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
+  if (kCluster) cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == 0) {
@@ -570,29 +595,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = tile0; ok && t < num_tiles; t += tile_step) {
         const int tm = t / p.tiles_n;
         const int tn = t - tm * p.tiles_n;
+        // this CTA's A rows and B columns
+        const int m0 = tm * (BM * CG) + rank * (kPair ? BM : 0);
+        const int n0 = tn * BN + rank * (kPair ? BN / 2 : 0);
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&ctl->full[stage], kAStage + kBStage);
           uint8_t* a_dst = smA + stage * kAStage;
           uint8_t* b_dst = smB + stage * kBStage;
-          if (A_MN) {
+          if (kPair) {
+            // both CTAs' bytes complete on the even CTA's barrier, which expects them all
+            const uint32_t bar0 = mapa_shared(smem_u32(&ctl->full[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], CG * (kAStage + kBStage));
+            if (A_MN) {
 #pragma unroll
-            for (int i = 0; i < BM / 64; ++i) tma_load_2d(a_dst + i * 8192, &tmA, &ctl->full[stage], tm * BM + 64 * i, kb * BK);
-          } else {
-            tma_load_2d(a_dst, &tmA, &ctl->full[stage], kb * BK, tm * BM);
-          }
-          if (EPI == EPI_SWIGLU_FWD) {
-            // 128 gate rows then the same 128 up rows
-            tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, tn * (BN / 2));
-            tma_load_2d(b_dst + kBStage / 2, &tmB2, &ctl->full[stage], kb * BK, tn * (BN / 2));
-          } else if (B_MN) {
+              for (int i = 0; i < BM / 64; ++i) tma_load_2d_pair(a_dst + i * 8192, &tmA, bar0, m0 + 64 * i, kb * BK);
+            } else {
+              tma_load_2d_pair(a_dst, &tmA, bar0, kb * BK, m0);
+            }
+            if (B_MN) {
 #pragma unroll
-            for (int i = 0; i < BN / 64; ++i) tma_load_2d(b_dst + i * 8192, &tmB, &ctl->full[stage], tn * BN + 64 * i, kb * BK);
+              for (int i = 0; i < BN / 2 / 64; ++i) tma_load_2d_pair(b_dst + i * 8192, &tmB, bar0, n0 + 64 * i, kb * BK);
+            } else {
+              tma_load_2d_pair(b_dst, &tmB, bar0, kb * BK, n0);
+            }
           } else {
-            tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, tn * BN);
+            mbar_arrive_expect_tx(&ctl->full[stage], kAStage + kBStage);
+            if (A_MN) {
+#pragma unroll
+              for (int i = 0; i < BM / 64; ++i) tma_load_2d(a_dst + i * 8192, &tmA, &ctl->full[stage], m0 + 64 * i, kb * BK);
+            } else {
+              tma_load_2d(a_dst, &tmA, &ctl->full[stage], kb * BK, m0);
+            }
+            if (EPI == EPI_SWIGLU_FWD) {
+              // 128 gate rows then the same 128 up rows
+              tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, tn * (BN / 2));
+              tma_load_2d(b_dst + kBStage / 2, &tmB2, &ctl->full[stage], kb * BK, tn * (BN / 2));
+            } else if (B_MN) {
+#pragma unroll
+              for (int i = 0; i < BN / 64; ++i) tma_load_2d(b_dst + i * 8192, &tmB, &ctl->full[stage], n0 + 64 * i, kb * BK);
+            } else {
+              tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, n0);
+            }
           }
           ++issued;
           if (++stage == STAGES) {
@@ -601,18 +647,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // Drain: every issued copy must have landed before the CTA may exit.
-      const uint32_t first = issued > STAGES ? issued - STAGES : 0;
-      for (uint32_t i = first; i < issued; ++i) mbar_wait_drain(&ctl->full[i % STAGES], (i / STAGES) & 1u);
+      // Drain: every issued copy must have landed before the CTA may exit (a
+      // pair's odd CTA signals the even CTA's barriers, which that CTA drains;
+      // the closing cluster barrier keeps the odd CTA alive until then).
+      if (leader) {
+        const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+        for (uint32_t i = first; i < issued; ++i) mbar_wait_drain(&ctl->full[i % STAGES], (i / STAGES) & 1u);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, BN, A_MN, B_MN);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int t = tile0; ok && t < num_tiles; t += tile_step) {
-        if (!mbar_wait(&ctl->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) break;
+        // a pair's accumulator is free once both CTAs' epilogues have drained it
+        const bool got = kPair ? mbar_wait_cluster(&ctl->tmem_empty[acc], acc_phase ^ 1u, abort_flag)
+                               : mbar_wait(&ctl->tmem_empty[acc], acc_phase ^ 1u, abort_flag);
+        if (!got) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
         for (int kb = kb_begin; kb < kb_end; ++kb) {
@@ -625,22 +678,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_base = smem_u32(smB + stage * kBStage);
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
-            umma_bf16(d, operand_desc<A_MN>(a_base, j), operand_desc<B_MN>(b_base, j), idesc,
-                      (kb != kb_begin || j != 0) ? 1u : 0u);
+            if (kPair)
+              umma_bf16_pair(d, operand_desc<A_MN>(a_base, j), operand_desc<B_MN>(b_base, j), idesc,
+                             (kb != kb_begin || j != 0) ? 1u : 0u);
+            else
+              umma_bf16(d, operand_desc<A_MN>(a_base, j), operand_desc<B_MN>(b_base, j), idesc,
+                        (kb != kb_begin || j != 0) ? 1u : 0u);
           }
-          umma_commit(&ctl->empty[stage]);
+          if (kPair) umma_commit_pair(&ctl->empty[stage]);
+          else umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&ctl->tmem_full[acc]);
+        if (kPair) umma_commit_pair(&ctl->tmem_full[acc]);
+        else umma_commit(&ctl->tmem_full[acc]);
         acc ^= 1u;
         if (acc == 0) acc_phase ^= 1u;
       }
       // All issued MMAs must be complete before TMEM is released.
-      umma_commit(&ctl->mma_done);
+      if (kPair) umma_commit_pair(&ctl->mma_done);
+      else umma_commit(&ctl->mma_done);
+      mbar_wait_drain(&ctl->mma_done, 0);
+    } else if (lane == 0) {
+      // a pair's odd CTA: its TMEM is written by the even CTA's MMAs
       mbar_wait_drain(&ctl->mma_done, 0);
     }
   } else {
@@ -665,7 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = tile0; t < num_tiles; t += tile_step) {
       const int tm = t / p.tiles_n;
       const int tn = t - tm * p.tiles_n;
-      const int row = tm * BM + quarter * 32 + lane;
+      const int row = tm * (BM * CG) + rank * (kPair ? BM : 0) + quarter * 32 + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       auto wait_acc = [&]() {
         const bool got = mbar_wait(&ctl->tmem_full[acc], acc_phase, abort_flag);
@@ -708,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           double part = epi_resid(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
-          if (lane == 0) p.partial[static_cast<size_t>(t) * kEpiWarps + half * 4 + quarter] = part;
+          if (lane == 0) p.partial[(static_cast<size_t>(t) * CG + (kPair ? rank : 0)) * kEpiWarps + half * 4 + quarter] = part;
         } else if (EPI == EPI_SWIGLU_FWD) {
           epi_swiglu_fwd(p, taddr, row, tn * (BN / 2), 2 * half, 2 * half + 2);
         } else {
@@ -717,7 +780,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->tmem_empty[acc]);
+      if (lane == 0) {
+        if (kPair) mbar_arrive_remote(mapa_shared(smem_u32(&ctl->tmem_empty[acc]), 0));
+        else mbar_arrive(&ctl->tmem_empty[acc]);
+      }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -726,10 +792,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (KSPLIT == 2) cluster_sync_all();  // the peer may still read or write this CTA's shared memory
+  if (kCluster) cluster_sync_all();  // the peer may still read or write this CTA's shared memory or barriers
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    if (kPair) tmem_dealloc_pair(tmem, kTmemCols);
+    else tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -742,7 +809,7 @@ cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t 
                       CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <bool A_MN, bool B_MN, int EPI, int KSPLIT = 1>
+template <bool A_MN, bool B_MN, int EPI, int KSPLIT = 1, int CG = 1>
 cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t stream, const char* name,
                 const uint16_t* B2 = nullptr) {
   CUtensorMap tmA, tmB, tmB2;
@@ -755,18 +822,20 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
     if (e != cudaSuccess) return e;
     e = make_tmap(&tmB2, B2, p.N, p.K, BN / 2);
   } else {
-    e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64) : make_tmap(&tmB, B, p.N, p.K, BN);
+    // a pair's CTA loads half of the tile's B columns
+    e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64) : make_tmap(&tmB, B, p.N, p.K, BN / CG);
     tmB2 = tmB;
   }
   if (e != cudaSuccess) return e;
-  p.tiles_m = (p.M + BM - 1) / BM;
+  p.tiles_m = (p.M + BM * CG - 1) / (BM * CG);
   p.tiles_n = EPI == EPI_SWIGLU_FWD ? (p.N + BN / 2 - 1) / (BN / 2) : (p.N + BN - 1) / BN;
   p.num_kb = (p.K + BK - 1) / BK;
-  auto kern = umma_gemm_kernel<A_MN, B_MN, EPI, KSPLIT>;
+  auto kern = umma_gemm_kernel<A_MN, B_MN, EPI, KSPLIT, CG>;
+  constexpr int kSmemBytes = GemmCfg<CG>::kSmemBytes;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
-  if (KSPLIT == 1) {
+  if (KSPLIT == 1 && CG == 1) {
     const int grid = tiles < num_sms() ? tiles : num_sms();
     LaunchScope scope(stream, name);
     kern<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, tmB2, p);
@@ -845,7 +914,13 @@ cudaError_t make_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, uint32_t el
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-int resid_partials(int M, int N) { return ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * kEpiWarps; }
+// The residual, reference-forward, plain and (unsplit) weight-gradient GEMMs run
+// as CTA pairs on 256 x 256 tiles; each CTA's eight epilogue warps write one
+// loss partial per tile.
+constexpr int kPairCG = 2;
+int resid_partials(int M, int N) {
+  return ((M + BM * kPairCG - 1) / (BM * kPairCG)) * ((N + BN - 1) / BN) * kPairCG * kEpiWarps;
+}
 
 cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,
                               cudaStream_t stream) {
@@ -854,7 +929,7 @@ cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, in
   p.N = N;
   p.K = K;
   p.D = Y;
-  return run<false, false, EPI_STORE>(X, W, p, stream, "umma_gemm<K,K,store>");
+  return run<false, false, EPI_STORE, 1, kPairCG>(X, W, p, stream, "umma_gemm<K,K,store,pair>");
 }
 
 cudaError_t launch_gemm_resid(const uint16_t* X, const uint16_t* W_hat, const float* Y, uint16_t* G, float gscale,
@@ -867,7 +942,7 @@ cudaError_t launch_gemm_resid(const uint16_t* X, const uint16_t* W_hat, const fl
   p.G = G;
   p.gscale = gscale;
   p.partial = loss_partial;
-  return run<false, false, EPI_RESID>(X, W_hat, p, stream, "umma_gemm<K,K,resid>");
+  return run<false, false, EPI_RESID, 1, kPairCG>(X, W_hat, p, stream, "umma_gemm<K,K,resid,pair>");
 }
 
 cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArgs& fa, int M, int N, int K,
@@ -883,14 +958,16 @@ cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArg
   // a tile (~60 us, compute bound), i.e. from 32768 tokens on; below that the
   // epilogue paces the pair and the unsplit kernel is faster (measured on
   // 16384 tokens: 533 us split vs 511 us unsplit for a 4096 x 4096 layer).
-  const int tiles = ((N + BM - 1) / BM) * ((K + BN - 1) / BN);
-  const int sms = num_sms();
-  const double eff1 = static_cast<double>(tiles) / (((tiles + sms - 1) / sms) * sms);
-  const int pairs = sms / 2;
-  const double eff2 = static_cast<double>(tiles) / (((tiles + pairs - 1) / pairs) * pairs);
+  // Both variants run one cluster of two CTAs per work unit: a 256 x 256 tcgen05
+  // pair tile, or a 128 x 256 tile whose reduction is split in halves.
+  const int pairs = num_sms() / 2;
+  const int tiles_pair = ((N + 2 * BM - 1) / (2 * BM)) * ((K + BN - 1) / BN);
+  const int tiles_split = ((N + BM - 1) / BM) * ((K + BN - 1) / BN);
+  const double eff1 = static_cast<double>(tiles_pair) / (((tiles_pair + pairs - 1) / pairs) * pairs);
+  const double eff2 = static_cast<double>(tiles_split) / (((tiles_split + pairs - 1) / pairs) * pairs);
   if (M >= 32768 && eff2 > eff1 + 0.02)
     return run<true, true, EPI_FOLD, 2>(G, X, p, stream, "umma_gemm<MN,MN,fold,split2>");
-  return run<true, true, EPI_FOLD>(G, X, p, stream, "umma_gemm<MN,MN,fold>");
+  return run<true, true, EPI_FOLD, 1, kPairCG>(G, X, p, stream, "umma_gemm<MN,MN,fold,pair>");
 }
 
 cudaError_t launch_gemm_swiglu_fwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* Wu, uint16_t* A_out,
@@ -927,10 +1004,10 @@ cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, b
   p.N = N;
   p.K = K;
   p.D = D;
-  if (!a_mn && !b_mn) return run<false, false, EPI_STORE>(A, B, p, stream, "umma_gemm<K,K,store>");
-  if (!a_mn && b_mn) return run<false, true, EPI_STORE>(A, B, p, stream, "umma_gemm<K,MN,store>");
-  if (a_mn && !b_mn) return run<true, false, EPI_STORE>(A, B, p, stream, "umma_gemm<MN,K,store>");
-  return run<true, true, EPI_STORE>(A, B, p, stream, "umma_gemm<MN,MN,store>");
+  if (!a_mn && !b_mn) return run<false, false, EPI_STORE, 1, kPairCG>(A, B, p, stream, "umma_gemm<K,K,store,pair>");
+  if (!a_mn && b_mn) return run<false, true, EPI_STORE, 1, kPairCG>(A, B, p, stream, "umma_gemm<K,MN,store,pair>");
+  if (a_mn && !b_mn) return run<true, false, EPI_STORE, 1, kPairCG>(A, B, p, stream, "umma_gemm<MN,K,store,pair>");
+  return run<true, true, EPI_STORE, 1, kPairCG>(A, B, p, stream, "umma_gemm<MN,MN,store,pair>");
 }
 
 cudaError_t launch_loss_reduce(const double* partials, int n, int steps, double inv_count, float* loss,
