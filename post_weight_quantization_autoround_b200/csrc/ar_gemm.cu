@@ -54,7 +54,9 @@ constexpr int kTmemCols = 2 * BN;     // double-buffered accumulator
 // CG = 1: one CTA per 128 x 256 tile.  CG = 2: a CTA pair per 256 x 256 tile
 // (tcgen05 .cta_group::2): each CTA loads its 128 A rows and half of the B
 // columns, so per SM the operand traffic from L2 falls from 48 to 32 KiB per
-// 64-k block of the same MMA work.
+// 64-k block of the same MMA work.  Every CTA's accumulator still holds all
+// 256 columns of its rows, so the epilogues are unchanged (the SwiGLU forward
+// tile's gate half comes from the even CTA, its up half from the odd one).
 template <int CG>
 struct GemmCfg {
   static constexpr int kBStage = (BN / CG) * BK * 2;  // 32 or 16 KiB
@@ -527,7 +529,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmB2, const Params p) {
   static_assert(!(KSPLIT == 2 && CG == 2), "a cluster is either a split pair or a tcgen05 pair");
-  static_assert(CG == 1 || (EPI != EPI_SWIGLU_FWD && EPI != EPI_SWIGLU_BWD), "SwiGLU tiles pair gate and up rows");
   constexpr int STAGES = GemmCfg<CG>::kStages;
   constexpr int kBStage = GemmCfg<CG>::kBStage;
   constexpr bool kPair = CG == 2;
@@ -615,7 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               tma_load_2d_pair(a_dst, &tmA, bar0, kb * BK, m0);
             }
-            if (B_MN) {
+            if (EPI == EPI_SWIGLU_FWD) {
+              // the tile's B columns are 128 gate rows then the same 128 up rows: one half each
+              tma_load_2d_pair(b_dst, rank == 0 ? &tmB : &tmB2, bar0, kb * BK, tn * (BN / 2));
+            } else if (B_MN) {
 #pragma unroll
               for (int i = 0; i < BN / 2 / 64; ++i) tma_load_2d_pair(b_dst + i * 8192, &tmB, bar0, n0 + 64 * i, kb * BK);
             } else {
@@ -979,7 +983,7 @@ cudaError_t launch_gemm_swiglu_fwd(const uint16_t* X, const uint16_t* Wg, const 
   p.act_a = A_out;
   p.act_b = B_out;
   p.act_h = H_out;
-  return run<false, false, EPI_SWIGLU_FWD>(X, Wg, p, stream, "umma_gemm<K,K,swiglu_fwd>", Wu);
+  return run<false, false, EPI_SWIGLU_FWD, 1, kPairCG>(X, Wg, p, stream, "umma_gemm<K,K,swiglu_fwd,pair>", Wu);
 }
 
 cudaError_t launch_gemm_swiglu_bwd(const uint16_t* G, const uint16_t* Wd_hat, const uint16_t* A_in,
@@ -994,7 +998,7 @@ cudaError_t launch_gemm_swiglu_bwd(const uint16_t* G, const uint16_t* Wd_hat, co
   p.act_b = const_cast<uint16_t*>(B_in);
   p.grad_a = dA;
   p.grad_b = dB;
-  return run<false, true, EPI_SWIGLU_BWD>(G, Wd_hat, p, stream, "umma_gemm<K,MN,swiglu_bwd>");
+  return run<false, true, EPI_SWIGLU_BWD, 1, kPairCG>(G, Wd_hat, p, stream, "umma_gemm<K,MN,swiglu_bwd,pair>");
 }
 
 cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, bool b_mn, float* D, int M, int N,
