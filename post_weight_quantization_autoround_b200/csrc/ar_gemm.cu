@@ -20,15 +20,21 @@
 // ([AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
 // Architectural Optimizations of AutoRound"; [IA] = "Intel AutoRound 高级量化".)
 //
-// Block: 320 threads.  Warp 0 lane 0 issues TMA loads into a 4-stage ring
-// (128x64 A tile, 256x64 B tile, 128-byte swizzle); warp 1 allocates 512 TMEM
-// columns (two 128x256 fp32 accumulators) and lane 0 issues
-// tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16); warps 2-9 drain
-// an accumulator with tcgen05.ld while the MMA warp fills the other one: warp
-// w reads TMEM lanes 32*(w%4)..+31 (one output row per thread) and one half
-// of the 256 columns, so two warps share each lane quarter.  The
-// grid is persistent: one CTA per SM, tiles strided by gridDim.x with the
-// N index fastest so that concurrently running CTAs share the A panel.
+// Launch: persistent clusters of two CTAs (320 threads each, one CTA per SM).
+// For the residual, reference-forward, plain, SwiGLU and (unsplit) weight-
+// gradient GEMMs the pair computes one 256x256 output tile as a tcgen05 CTA
+// pair: in each CTA warp 0 lane 0 issues TMA loads of its 128 A rows and its
+// 128 of the tile's 256 B columns into a 6-stage ring (128-byte swizzle),
+// completing on the even CTA's barrier; warp 1 allocates 512 TMEM columns
+// together with the peer (two 128x256 fp32 accumulators) and, in the even CTA,
+// lane 0 issues tcgen05.mma.cta_group::2.kind::f16 (M=256, N=256, K=16) and
+// commits to both CTAs' barriers; warps 2-9 drain this CTA's accumulator rows
+// with tcgen05.ld while the MMAs fill the other accumulator: warp w reads TMEM
+// lanes 32*(w%4)..+31 (one output row per thread) and one half of the 256
+// columns, so two warps share each lane quarter.  Tiles are strided over the
+// clusters with the N index fastest so that concurrently running pairs share
+// the A panel.  The weight-gradient GEMM from 32768 tokens on instead runs
+// 128x256 one-CTA tiles whose reduction the two CTAs of a cluster split.
 //
 // Operands: A is [M][K] (K-major) or [K][M] (MN-major); B is [N][K] or [K][N].
 // The weight-gradient GEMM reads G [tokens][N_w] and X [tokens][K_w] directly

@@ -137,8 +137,11 @@ def test_f32_to_bf16_matches_oracle_rounding(ar):
 # ----------------------------------------------------------------------------
 
 @pytest.mark.parametrize("a_mn,b_mn", [(False, False), (False, True), (True, False), (True, True)])
-@pytest.mark.parametrize("M,N,K", [(200, 320, 192), (128, 256, 64), (512, 512, 1024), (8, 8, 8)])
+@pytest.mark.parametrize("M,N,K", [(200, 320, 192), (128, 256, 64), (512, 512, 1024), (8, 8, 8), (130, 136, 72),
+                                   (1000, 776, 136)])
 def test_gemm_all_operand_layouts(ar, a_mn, b_mn, M, N, K):
+    """256 x 256 tiles on tcgen05 CTA pairs; ragged M, N, K leave the odd CTA's rows or B half
+    partly or wholly outside the matrices."""
     rng = np.random.default_rng(M + N + K)
     A = synth.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
     B = synth.to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32))
@@ -148,6 +151,7 @@ def test_gemm_all_operand_layouts(ar, a_mn, b_mn, M, N, K):
     Bd = bf16_dev(np.ascontiguousarray(B.T) if b_mn else B)
     D = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
     ar.ar_gemm_bf16(Ad, a_mn, Bd, b_mn, D, M, N, K)
+    assert ",pair>" in ar.ar_last_kernels()
     got = D.cpu().numpy()
     assert np.isfinite(got).all()
     tol = 1e-5 * np.sqrt(K) * 4
@@ -232,6 +236,7 @@ def test_single_step_matches_oracle(ar, N, K, M, bits, g, sym, spread):
     cfg, ocfg = cfg_pair(ar, bits, g, sym)
     gl = GpuLinear(ar, d["W"], d["X"], V, a, b, cfg)
     out = gl.step(1, grads=True)
+    assert "resid,pair>" in ar.ar_last_kernels() and "fold,pair>" in ar.ar_last_kernels()
     Wf, Xf = synth.bf16_bits_to_f32(d["W"]), synth.bf16_bits_to_f32(d["X"])
     L, (V1, a1, b1), gr, _ = O.tune_step_linear(Wf, Xf, O.reference_forward(Xf, Wf), V, a, b, ocfg)
     assert out["loss"][0] == pytest.approx(L, rel=1e-4)
