@@ -137,7 +137,7 @@ def test_f32_to_bf16_matches_oracle_rounding(ar):
 # ----------------------------------------------------------------------------
 
 @pytest.mark.parametrize("a_mn,b_mn", [(False, False), (False, True), (True, False), (True, True)])
-@pytest.mark.parametrize("M,N,K", [(200, 320, 192), (128, 256, 64), (512, 512, 1024), (8, 8, 8), (130, 136, 72),
+@pytest.mark.parametrize("M,N,K", [(200, 320, 192), (128, 256, 64), (512, 512, 1024), (8, 8, 8), (120, 136, 72),
                                    (1000, 776, 136)])
 def test_gemm_all_operand_layouts(ar, a_mn, b_mn, M, N, K):
     """256 x 256 tiles on tcgen05 CTA pairs; ragged M, N, K leave the odd CTA's rows or B half
