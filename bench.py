@@ -377,6 +377,29 @@ def other_workloads(ar, torch, peaks, steps=10):
                      "final_loss": float(loss[-1].item())}
         del W, X, V, a, b, Y, ws
         torch.cuda.empty_cache()
+    # block-by-block tuning of two SwiGLU blocks with the "light" preset: every step of the
+    # method (reference forwards over all samples, gathered minibatch steps, quantized forwards)
+    from post_weight_quantization_autoround_b200 import driver
+
+    pre = driver.PRESETS["light"]
+    Hd, F = 4096, 11008
+    S, Lq, Bq, iters = pre["samples"], pre["seqlen"], pre["batch"], pre["iters"]
+    raw = [synth.make_mlp(Hd, F, 1, seed=40 + b) for b in range(2)]
+    blocks = [[to_dev_bf16(d[k], torch) for k in ("Wg", "Wu", "Wd")] for d in raw]
+    del raw
+    X0 = to_dev_bf16(synth.make_activations(S * Lq, Hd, seed=41), torch).view(S, Lq, Hd)
+    sched = synth.make_schedule(S, Bq, iters, seed=0)
+    cfg = ar.ar_qconfig_default(bits=4, group_size=128, lr=driver.LR)
+    driver.tune_mlp_blocks(blocks[:1], X0, cfg, sched[:2])  # allocations and first launches
+    ms = _time_call(torch, lambda: driver.tune_mlp_blocks(blocks, X0, cfg, sched), warmup=0)
+    flops = 2 * (2 * 6.0 * S * Lq * Hd * F + iters * 14.0 * Bq * Lq * Hd * F)
+    out["driver_light_2x_mlp_4096_11008"] = {
+        "blocks": 2, "preset": "light", "samples": S, "seqlen": Lq, "batch": Bq, "iters": iters,
+        "s_per_block": ms / 2e3, "steps_per_s": 2 * iters / (ms * 1e-3),
+        "tflops": flops / (ms * 1e-3) / 1e12, "frac_sustained_bf16": flops / (ms * 1e-3) / 1e12 / peak,
+        "note": "per block: reference forward on all samples, 50 gathered-minibatch joint steps, quantized forward"}
+    del blocks, X0
+    torch.cuda.empty_cache()
     if ar.ar_get_device_status() != 0:
         out["device_status"] = ar.ar_last_error()
     return out

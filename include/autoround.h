@@ -239,6 +239,19 @@ AR_API ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* pac
                         const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, uint16_t* out,
                         ar_stream_t stream);
 
+/* Minibatch assembly for block-by-block tuning ([AR] §8 preset table: each
+ * iteration works on a batch of 8 -- 4 in the "fast" preset -- of the 128
+ * calibration samples; [AR] §3 "Algorithm Flow" steps 3-6 iterate on such
+ * batches).  Copies samples idx[0..n_idx-1] of src (n_src_samples samples of
+ * sample_bytes each, contiguous) to dst in that order:
+ *   dst[i*sample_bytes .. +sample_bytes) = src[idx[i]*sample_bytes .. ).
+ * idx is a HOST array, read before the call returns.  Needs 1 <= n_idx <= 64,
+ * every idx in [0, n_src_samples), sample_bytes a positive multiple of 16,
+ * 16-byte aligned device pointers, dst not overlapping src; otherwise
+ * AR_ERR_INVALID_ARG before any launch. */
+AR_API ar_status ar_gather_samples(const void* src, int64_t n_src_samples, int64_t sample_bytes, const int32_t* idx,
+                                   int n_idx, void* dst, ar_stream_t stream);
+
 /* Plain tensor-core GEMM, fp32 out: D[M][N] = sum_k A(m,k) B(n,k).
  * A is [M][K] (a_mn_major = 0) or [K][M] (a_mn_major = 1); B is [N][K]
  * (b_mn_major = 0) or [K][N] (b_mn_major = 1); all bf16.  The same

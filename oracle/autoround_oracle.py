@@ -534,3 +534,46 @@ def smooth_loss_mlp(Ws, X, Y, states, bits, group_size, symmetric=False):
     fw = mlp_forward(X, sts[0]["What"], sts[1]["What"], sts[2]["What"], dtype=f64)
     R = fw["y"] - np.asarray(Y, f64)
     return float(np.sum(R ** 2) / R.size)
+
+
+# ----------------------------------------------------------------------------
+# Block-by-block tuning of a stack of SwiGLU blocks ([AR] §3 "Algorithm Flow")
+# ----------------------------------------------------------------------------
+
+def tune_blocks_mlp(blocks, X0, cfg: QConfig, schedule):
+    """The blocks in order ([AR] §3 "Algorithm Flow"):
+
+    * step 2: the block's reference output, its forward with the original
+      weights on the block's input (all calibration samples);
+    * steps 3-6: one joint SignSGD step (``tune_step_mlp``) per row of
+      ``schedule`` on the samples the row names, their tokens in that order
+      (the minibatch of [AR] §8's preset table);
+    * step 7: the block's parameters are frozen and the output of the
+      quantized block, rounded to bf16, is the next block's input.
+
+    ``blocks``: list of (Wg, Wu, Wd) bf16 values in float32; ``X0``:
+    [samples][tokens][H] bf16 values in float32; ``schedule``: int
+    [steps][batch] (the random draws, passed in).  Returns one dict per block:
+    ``states`` (three (V, alpha, beta)), ``losses`` [steps] and ``x_out``
+    ([samples][tokens][H], the next block's input).
+    """
+    X = np.asarray(X0, f32)
+    S, L, H = X.shape
+    out = []
+    for Ws in blocks:
+        Xf = X.reshape(S * L, H)
+        Y = mlp_reference(Xf, *Ws).reshape(S, L, H)
+        states = [(np.zeros(W.shape, f32), np.ones((W.shape[0], W.shape[1] // cfg.group_size), f32),
+                   np.ones((W.shape[0], W.shape[1] // cfg.group_size), f32)) for W in Ws]
+        losses = []
+        for idx in np.asarray(schedule):
+            Xb = X[idx].reshape(-1, H)
+            Yb = Y[idx].reshape(-1, H)
+            loss, states, _, _, _ = tune_step_mlp(Ws, Xb, Yb, states, cfg)
+            losses.append(loss)
+        sts = [qdq(W, *st, cfg.bits, cfg.group_size, cfg.symmetric) for W, st in zip(Ws, states)]
+        y = mlp_forward(Xf, sts[0]["What_bf16"], sts[1]["What_bf16"], sts[2]["What_bf16"])["y"]
+        X = bf16_rne(y).reshape(S, L, H)
+        out.append({"states": states, "losses": np.asarray(losses, f64), "x_out": X})
+    return out
+

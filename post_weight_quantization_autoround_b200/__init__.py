@@ -84,6 +84,7 @@ _SIGNATURES = {
     "ar_debug_wait_timeout": (_INT, [ctypes.c_uint64, _P, _P]),
     "ar_profile_start": (_INT, []),
     "ar_profile_stop": (_INT, [ctypes.c_char_p, ctypes.c_size_t]),
+    "ar_gather_samples": (_INT, [_P, _I64, _I64, ctypes.POINTER(ctypes.c_int32), _INT, _P, _P]),
 }
 
 
@@ -262,6 +263,16 @@ def ar_w4a16_gemm(A, packed, scale16, zero16, group_size: int, out, stream=None)
     N = packed.shape[0]
     _check(lib().ar_w4a16_gemm(_ptr(A), T, _ptr(packed), _ptr(scale16), _ptr(zero16), N, K, group_size, _ptr(out),
                                _stream(stream)))
+
+
+def ar_gather_samples(src, idx, dst, stream=None) -> None:
+    """dst[i] = src[idx[i]] for whole samples (first dimension); idx: host sequence of ints."""
+    n_src = src.shape[0]
+    sample_bytes = src[0].numel() * src.element_size() if n_src else 0
+    arr = (ctypes.c_int32 * len(idx))(*[int(i) for i in idx])
+    if dst.shape[0] != len(idx) or dst[0].numel() * dst.element_size() != sample_bytes:
+        raise ARError(AR_ERR_INVALID_ARG, "dst must hold len(idx) samples of src's size")
+    _check(lib().ar_gather_samples(_ptr(src), n_src, sample_bytes, arr, len(idx), _ptr(dst), _stream(stream)))
 
 
 def ar_gemm_bf16(A, a_mn_major: bool, B, b_mn_major: bool, D, M: int, N: int, K: int, stream=None) -> None:

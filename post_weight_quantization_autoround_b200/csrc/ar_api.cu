@@ -586,6 +586,24 @@ ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
   return end_call();
 }
 
+ar_status ar_gather_samples(const void* src, int64_t n_src_samples, int64_t sample_bytes, const int32_t* idx,
+                            int n_idx, void* dst, ar_stream_t stream) {
+  begin_call();
+  if (!src || !dst || !idx) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  if (n_idx < 1 || n_idx > kMaxGatherSamples) return fail(AR_ERR_INVALID_ARG, "n_idx must be in 1..%d", kMaxGatherSamples);
+  if (sample_bytes <= 0 || sample_bytes % 16 != 0) return fail(AR_ERR_INVALID_ARG, "sample_bytes must be a positive multiple of 16");
+  if (n_src_samples <= 0) return fail(AR_ERR_INVALID_ARG, "n_src_samples must be positive");
+  if (!aligned16(src) || !aligned16(dst)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  for (int i = 0; i < n_idx; ++i)
+    if (idx[i] < 0 || idx[i] >= n_src_samples) return fail(AR_ERR_INVALID_ARG, "idx[%d] = %d out of range", i, idx[i]);
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), s1 = s0 + static_cast<uintptr_t>(n_src_samples * sample_bytes);
+  const uintptr_t d0 = reinterpret_cast<uintptr_t>(dst), d1 = d0 + static_cast<uintptr_t>(n_idx * sample_bytes);
+  if (d0 < s1 && s0 < d1) return fail(AR_ERR_INVALID_ARG, "dst overlaps src");
+  cudaError_t e = launch_gather_samples(src, sample_bytes, idx, n_idx, dst, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  return end_call();
+}
+
 ar_status ar_gemm_bf16(const uint16_t* A, int a_mn_major, const uint16_t* B, int b_mn_major, float* D, int64_t M,
                        int64_t N, int64_t K, ar_stream_t stream) {
   begin_call();

@@ -1,0 +1,112 @@
+"""Block-by-block tuning of a stack of SwiGLU MLP blocks on the GPU.
+
+[AR] §3 "Algorithm Flow" (the blocks are tuned one after another):
+
+* step 2: the block's reference output, its forward with the original bf16
+  weights on the block's input (all calibration samples), ``ar_block_forward``;
+* steps 3-6: ``iters`` joint SignSGD steps, each on the minibatch of
+  calibration samples its row of the schedule names (``ar_gather_samples``
+  assembles the tokens and their reference outputs, ``ar_tune_step`` runs the
+  step);
+* step 7: the block's parameters are frozen; ``ar_qdq`` gives its quantized
+  weights, and the quantized block's output (``ar_block_forward`` on them,
+  rounded to bf16 by ``ar_f32_to_bf16``) is the next block's input.
+
+``PRESETS`` are the four modes of [AR] §8's preset table (batch size,
+iterations, sequence length, calibration samples; lr 5e-3 in all).  The
+minibatch draws are data (``synth.make_schedule`` or the caller's own), so a
+run is reproducible and checkable against the oracle.
+
+Every step of the method runs in the library's kernels; this module only
+allocates buffers and orders the calls.  ([AR] = "Low-Bit Quantization in
+Practice with vLLM: Core Mechanisms and Architectural Optimizations of
+AutoRound".)
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Sequence
+
+import numpy as np
+import torch
+
+from . import (AR_BLOCK_SWIGLU_MLP, QConfig, ar_block_forward, ar_block_forward_workspace, ar_f32_to_bf16,
+               ar_gather_samples, ar_pack_int4, ar_qdq, ar_tune_block, ar_tune_block_workspace)
+
+PRESETS: Dict[str, Dict[str, int]] = {
+    "default": {"batch": 8, "iters": 200, "seqlen": 2048, "samples": 128},
+    "best": {"batch": 8, "iters": 1000, "seqlen": 2048, "samples": 128},
+    "light": {"batch": 8, "iters": 50, "seqlen": 512, "samples": 128},
+    "fast": {"batch": 4, "iters": 200, "seqlen": 2048, "samples": 128},
+}
+LR = 0.005
+
+
+def tune_mlp_blocks(blocks: Sequence[Sequence[torch.Tensor]], X0: torch.Tensor, cfg: QConfig,
+                    schedule: np.ndarray, export_int4: bool = False, stream=None) -> List[dict]:
+    """Tunes ``blocks`` (list of (Wg [F][H], Wu [F][H], Wd [H][F]) bf16 device
+    tensors) in order on the calibration tokens ``X0`` (bf16 device tensor
+    [samples][tokens][H]); ``schedule``: int [steps][batch] sample indices per
+    step (host array).
+
+    Returns one dict per block: ``states`` (three (V, alpha, beta) device
+    tensors), ``losses`` (host float32 [steps], the MSE of each step's
+    minibatch before its update), ``x_out`` (bf16 [samples][tokens][H], the
+    next block's input) and, with ``export_int4`` (4-bit configs), ``int4``:
+    three (packed, scale16, zero16) as ``ar_pack_int4`` writes them.
+    """
+    schedule = np.asarray(schedule, dtype=np.int32)
+    if schedule.ndim != 2 or schedule.shape[0] < 1:
+        raise ValueError("schedule must be [steps][batch]")
+    S, L, H = X0.shape
+    dev = X0.device
+    batch = schedule.shape[1]
+    X = X0
+    results = []
+    for Wg, Wu, Wd in blocks:
+        Ws = [Wg, Wu, Wd]
+        g = cfg.group_size
+        # step 2: reference output of the block on its input
+        fws = torch.empty(ar_block_forward_workspace(AR_BLOCK_SWIGLU_MLP, Ws, S * L), dtype=torch.uint8, device=dev)
+        Y = torch.empty((S, L, H), dtype=torch.float32, device=dev)
+        ar_block_forward(AR_BLOCK_SWIGLU_MLP, Ws, X.view(S * L, H), Y.view(S * L, H), fws, stream=stream)
+        states = [(torch.zeros(W.shape, dtype=torch.float32, device=dev),
+                   torch.ones((W.shape[0], W.shape[1] // g), dtype=torch.float32, device=dev),
+                   torch.ones((W.shape[0], W.shape[1] // g), dtype=torch.float32, device=dev)) for W in Ws]
+        layers = [(W, V, a, b) for W, (V, a, b) in zip(Ws, states)]
+        # steps 3-6 on the drawn minibatches
+        Mb = batch * L
+        Xb = torch.empty((batch, L, H), dtype=torch.bfloat16, device=dev)
+        Yb = torch.empty((batch, L, H), dtype=torch.float32, device=dev)
+        ws = torch.empty(ar_tune_block_workspace(AR_BLOCK_SWIGLU_MLP, layers, Mb, cfg, 1), dtype=torch.uint8,
+                         device=dev)
+        losses = torch.empty(schedule.shape[0], dtype=torch.float32, device=dev)
+        for t, idx in enumerate(schedule):
+            ar_gather_samples(X, idx, Xb, stream=stream)
+            ar_gather_samples(Y, idx, Yb, stream=stream)
+            ar_tune_block(AR_BLOCK_SWIGLU_MLP, layers, Xb.view(Mb, H), Yb.view(Mb, H), cfg, 1, losses[t:t + 1], ws,
+                          stream=stream)
+        del ws, Xb, Yb
+        # step 7: frozen parameters; the quantized block's output is the next input
+        What = [torch.empty_like(W) for W in Ws]
+        for W, (V, a, b), Wh in zip(Ws, states, What):
+            ar_qdq(W, V, a, b, cfg, W_hat=Wh, stream=stream)
+        ar_block_forward(AR_BLOCK_SWIGLU_MLP, What, X.view(S * L, H), Y.view(S * L, H), fws, stream=stream)
+        Xn = torch.empty((S, L, H), dtype=torch.bfloat16, device=dev)
+        ar_f32_to_bf16(Y.view(-1), Xn.view(-1), stream=stream)
+        res = {"states": states, "losses": losses, "x_out": Xn}
+        if export_int4:
+            packs = []
+            for W, (V, a, b) in zip(Ws, states):
+                N, K = W.shape
+                packed = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+                s16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+                z16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+                ar_pack_int4(W, V, a, b, cfg, packed, s16, z16, stream=stream)
+                packs.append((packed, s16, z16))
+            res["int4"] = packs
+        del Y, fws, What
+        results.append(res)
+        X = Xn
+    for r in results:
+        r["losses"] = r["losses"].cpu().numpy()
+    return results

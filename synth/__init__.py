@@ -185,3 +185,15 @@ WORKLOADS: Dict[str, Workload] = {
     # Llama-70B-shaped down projection 8192x28672.
     "down_8192_28672": Workload("down_8192_28672", "linear", 8192, 28672, 16384),
 }
+
+
+def make_schedule(n_samples: int, batch: int, steps: int, seed: int = 0) -> np.ndarray:
+    """Calibration samples each tuning step draws: int32 [steps][batch], ``batch``
+    distinct indices in [0, n_samples) per step, uniformly at random (PCG64,
+    seeded).  The draws are data: the GPU driver and the oracle take the same
+    array."""
+    if not (0 < batch <= n_samples):
+        raise ValueError("need 0 < batch <= n_samples")
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 0x5A3D])))
+    return np.stack([rng.choice(n_samples, size=batch, replace=False) for _ in range(steps)]).astype(np.int32)
+

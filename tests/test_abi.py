@@ -133,3 +133,16 @@ def test_binding_refuses_host_tensors():
 
     with pytest.raises(ar.ARError):
         ar.ar_f32_to_bf16(torch.zeros(8), torch.zeros(8, dtype=torch.bfloat16))
+
+
+def test_gather_samples_validation():
+    g = ar.lib().ar_gather_samples
+    idx = (ctypes.c_int32 * 3)(0, 2, 1)
+    assert g(FAKE, 4, 64, idx, 0, 0x20000, None) == ar.AR_ERR_INVALID_ARG           # no samples
+    assert g(FAKE, 4, 64, idx, 65, 0x20000, None) == ar.AR_ERR_INVALID_ARG          # more than 64
+    assert g(FAKE, 4, 60, idx, 3, 0x20000, None) == ar.AR_ERR_INVALID_ARG           # not a multiple of 16 bytes
+    assert g(FAKE, 2, 64, idx, 3, 0x20000, None) == ar.AR_ERR_INVALID_ARG           # index 2 out of range
+    assert g(FAKE, 4, 64, idx, 3, FAKE + 64, None) == ar.AR_ERR_INVALID_ARG         # dst overlaps src
+    assert g(FAKE + 8, 4, 64, idx, 3, 0x20000, None) == ar.AR_ERR_INVALID_ARG       # misaligned
+    assert g(FAKE, 4, 64, None, 3, 0x20000, None) == ar.AR_ERR_INVALID_ARG          # no index array
+
