@@ -41,6 +41,59 @@ PRESETS: Dict[str, Dict[str, int]] = {
 LR = 0.005
 
 
+def tune_mlp_block(Ws: Sequence[torch.Tensor], X: torch.Tensor, cfg: QConfig, schedule: np.ndarray,
+                   export_int4: bool = False, stream=None) -> dict:
+    """One block of ``tune_mlp_blocks``: Ws = (Wg [F][H], Wu [F][H], Wd [H][F]) bf16 device tensors, X the
+    block's input (bf16 [samples][tokens][H]).  Returns the dict described there."""
+    schedule = np.asarray(schedule, dtype=np.int32)
+    if schedule.ndim != 2 or schedule.shape[0] < 1:
+        raise ValueError("schedule must be [steps][batch]")
+    S, L, H = X.shape
+    dev = X.device
+    batch = schedule.shape[1]
+    Ws = list(Ws)
+    g = cfg.group_size
+    # step 2: reference output of the block on its input
+    fws = torch.empty(ar_block_forward_workspace(AR_BLOCK_SWIGLU_MLP, Ws, S * L), dtype=torch.uint8, device=dev)
+    Y = torch.empty((S, L, H), dtype=torch.float32, device=dev)
+    ar_block_forward(AR_BLOCK_SWIGLU_MLP, Ws, X.view(S * L, H), Y.view(S * L, H), fws, stream=stream)
+    states = [(torch.zeros(W.shape, dtype=torch.float32, device=dev),
+               torch.ones((W.shape[0], W.shape[1] // g), dtype=torch.float32, device=dev),
+               torch.ones((W.shape[0], W.shape[1] // g), dtype=torch.float32, device=dev)) for W in Ws]
+    layers = [(W, V, a, b) for W, (V, a, b) in zip(Ws, states)]
+    # steps 3-6 on the drawn minibatches
+    Mb = batch * L
+    Xb = torch.empty((batch, L, H), dtype=torch.bfloat16, device=dev)
+    Yb = torch.empty((batch, L, H), dtype=torch.float32, device=dev)
+    ws = torch.empty(ar_tune_block_workspace(AR_BLOCK_SWIGLU_MLP, layers, Mb, cfg, 1), dtype=torch.uint8, device=dev)
+    losses = torch.empty(schedule.shape[0], dtype=torch.float32, device=dev)
+    for t, idx in enumerate(schedule):
+        ar_gather_samples(X, idx, Xb, stream=stream)
+        ar_gather_samples(Y, idx, Yb, stream=stream)
+        ar_tune_block(AR_BLOCK_SWIGLU_MLP, layers, Xb.view(Mb, H), Yb.view(Mb, H), cfg, 1, losses[t:t + 1], ws,
+                      stream=stream)
+    del ws, Xb, Yb
+    # step 7: frozen parameters; the quantized block's output is the next input
+    What = [torch.empty_like(W) for W in Ws]
+    for W, (V, a, b), Wh in zip(Ws, states, What):
+        ar_qdq(W, V, a, b, cfg, W_hat=Wh, stream=stream)
+    ar_block_forward(AR_BLOCK_SWIGLU_MLP, What, X.view(S * L, H), Y.view(S * L, H), fws, stream=stream)
+    Xn = torch.empty((S, L, H), dtype=torch.bfloat16, device=dev)
+    ar_f32_to_bf16(Y.view(-1), Xn.view(-1), stream=stream)
+    res = {"states": states, "losses": losses, "x_out": Xn}
+    if export_int4:
+        packs = []
+        for W, (V, a, b) in zip(Ws, states):
+            N, K = W.shape
+            packed = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+            s16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+            z16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+            ar_pack_int4(W, V, a, b, cfg, packed, s16, z16, stream=stream)
+            packs.append((packed, s16, z16))
+        res["int4"] = packs
+    return res
+
+
 def tune_mlp_blocks(blocks: Sequence[Sequence[torch.Tensor]], X0: torch.Tensor, cfg: QConfig,
                     schedule: np.ndarray, export_int4: bool = False, stream=None) -> List[dict]:
     """Tunes ``blocks`` (list of (Wg [F][H], Wu [F][H], Wd [H][F]) bf16 device
@@ -54,59 +107,84 @@ def tune_mlp_blocks(blocks: Sequence[Sequence[torch.Tensor]], X0: torch.Tensor, 
     next block's input) and, with ``export_int4`` (4-bit configs), ``int4``:
     three (packed, scale16, zero16) as ``ar_pack_int4`` writes them.
     """
-    schedule = np.asarray(schedule, dtype=np.int32)
-    if schedule.ndim != 2 or schedule.shape[0] < 1:
-        raise ValueError("schedule must be [steps][batch]")
-    S, L, H = X0.shape
-    dev = X0.device
-    batch = schedule.shape[1]
     X = X0
     results = []
-    for Wg, Wu, Wd in blocks:
-        Ws = [Wg, Wu, Wd]
-        g = cfg.group_size
-        # step 2: reference output of the block on its input
-        fws = torch.empty(ar_block_forward_workspace(AR_BLOCK_SWIGLU_MLP, Ws, S * L), dtype=torch.uint8, device=dev)
-        Y = torch.empty((S, L, H), dtype=torch.float32, device=dev)
-        ar_block_forward(AR_BLOCK_SWIGLU_MLP, Ws, X.view(S * L, H), Y.view(S * L, H), fws, stream=stream)
-        states = [(torch.zeros(W.shape, dtype=torch.float32, device=dev),
-                   torch.ones((W.shape[0], W.shape[1] // g), dtype=torch.float32, device=dev),
-                   torch.ones((W.shape[0], W.shape[1] // g), dtype=torch.float32, device=dev)) for W in Ws]
-        layers = [(W, V, a, b) for W, (V, a, b) in zip(Ws, states)]
-        # steps 3-6 on the drawn minibatches
-        Mb = batch * L
-        Xb = torch.empty((batch, L, H), dtype=torch.bfloat16, device=dev)
-        Yb = torch.empty((batch, L, H), dtype=torch.float32, device=dev)
-        ws = torch.empty(ar_tune_block_workspace(AR_BLOCK_SWIGLU_MLP, layers, Mb, cfg, 1), dtype=torch.uint8,
-                         device=dev)
-        losses = torch.empty(schedule.shape[0], dtype=torch.float32, device=dev)
-        for t, idx in enumerate(schedule):
-            ar_gather_samples(X, idx, Xb, stream=stream)
-            ar_gather_samples(Y, idx, Yb, stream=stream)
-            ar_tune_block(AR_BLOCK_SWIGLU_MLP, layers, Xb.view(Mb, H), Yb.view(Mb, H), cfg, 1, losses[t:t + 1], ws,
-                          stream=stream)
-        del ws, Xb, Yb
-        # step 7: frozen parameters; the quantized block's output is the next input
-        What = [torch.empty_like(W) for W in Ws]
-        for W, (V, a, b), Wh in zip(Ws, states, What):
-            ar_qdq(W, V, a, b, cfg, W_hat=Wh, stream=stream)
-        ar_block_forward(AR_BLOCK_SWIGLU_MLP, What, X.view(S * L, H), Y.view(S * L, H), fws, stream=stream)
-        Xn = torch.empty((S, L, H), dtype=torch.bfloat16, device=dev)
-        ar_f32_to_bf16(Y.view(-1), Xn.view(-1), stream=stream)
-        res = {"states": states, "losses": losses, "x_out": Xn}
-        if export_int4:
-            packs = []
-            for W, (V, a, b) in zip(Ws, states):
-                N, K = W.shape
-                packed = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
-                s16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
-                z16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
-                ar_pack_int4(W, V, a, b, cfg, packed, s16, z16, stream=stream)
-                packs.append((packed, s16, z16))
-            res["int4"] = packs
-        del Y, fws, What
+    for Ws in blocks:
+        res = tune_mlp_block(Ws, X, cfg, schedule, export_int4, stream)
         results.append(res)
-        X = Xn
+        X = res["x_out"]
     for r in results:
         r["losses"] = r["losses"].cpu().numpy()
     return results
+
+
+def tune_mlp_blocks_streamed(host_blocks: Sequence[Sequence[torch.Tensor]], X0: torch.Tensor, cfg: QConfig,
+                             schedule: np.ndarray) -> List[dict]:
+    """``tune_mlp_blocks`` for models whose weights live in host memory: each
+    block's weights (pinned host bf16 tensors) are copied to the device on a
+    side stream while the previous block is tuned, and only what a block
+    exports (INT4 words, fp16 scale/zero, the losses) comes back to host
+    memory, so the device holds at most two blocks' weights at a time.  The
+    calibration tokens ``X0`` stay on the device.  Returns per block
+    ``losses`` and ``int4`` (host tensors) and, for the last block, ``x_out``.
+    """
+    dev = X0.device
+    main = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+
+    def upload(Ws):
+        with torch.cuda.stream(copy):
+            d = [W.to(dev, non_blocking=True) for W in Ws]
+            ev = torch.cuda.Event()
+            ev.record(copy)
+        return d, ev
+
+    results = []
+    X = X0
+    nxt = upload(host_blocks[0]) if host_blocks else None
+    for b in range(len(host_blocks)):
+        Wd, ev = nxt
+        main.wait_event(ev)
+        for W in Wd:
+            W.record_stream(main)
+        if b + 1 < len(host_blocks):
+            nxt = upload(host_blocks[b + 1])  # overlaps this block's tuning
+        res = tune_mlp_block(Wd, X, cfg, schedule, export_int4=True)
+        out = {"losses": res["losses"].cpu(), "int4": [tuple(t.cpu() for t in p) for p in res["int4"]]}
+        X = res["x_out"]
+        del res, Wd
+        results.append(out)
+    if results:
+        results[-1]["x_out"] = X
+    for r in results:
+        r["losses"] = r["losses"].numpy()
+    return results
+
+
+def save_int4_checkpoint(path: str, results: Sequence[dict], cfg: QConfig) -> None:
+    """Writes the INT4 export of every layer of every block to one ``.npz``
+    file: arrays ``b{block}.{gate|up|down}.{packed|scale|zero}`` (uint32
+    [N][K/8] with element k at bits 4(k mod 8) of word k/8; fp16 [N][K/g]) and
+    a ``meta`` JSON string (bits, group_size, symmetric, layout)."""
+    import json
+
+    arrays = {}
+    for b, r in enumerate(results):
+        for name, (packed, s16, z16) in zip(("gate", "up", "down"), r["int4"]):
+            arrays[f"b{b}.{name}.packed"] = packed.cpu().numpy().view(np.uint32)
+            arrays[f"b{b}.{name}.scale"] = s16.cpu().numpy()
+            arrays[f"b{b}.{name}.zero"] = z16.cpu().numpy()
+    meta = {"bits": 4, "group_size": int(cfg.group_size), "symmetric": int(cfg.symmetric), "blocks": len(results),
+            "layout": "uint32 [N][K/8], element k at bits 4*(k mod 8) of word k/8; fp16 scale/zero [N][K/g]; "
+                      "dequant (q - zero) * scale"}
+    np.savez(path, meta=np.array(json.dumps(meta)), **arrays)
+
+
+def load_int4_checkpoint(path: str):
+    """Reads ``save_int4_checkpoint``'s file: (meta dict, {name: array})."""
+    import json
+
+    with np.load(path) as f:
+        meta = json.loads(str(f["meta"]))
+        arrays = {k: f[k] for k in f.files if k != "meta"}
+    return meta, arrays

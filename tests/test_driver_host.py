@@ -88,3 +88,29 @@ def test_oracle_driver_with_every_sample_each_step_is_the_full_batch_trajectory(
         assert res[0]["losses"][t] == loss
     for (V1, a1, b1), (V2, a2, b2) in zip(res[0]["states"], st):
         assert np.array_equal(V1, V2) and np.array_equal(a1, a2) and np.array_equal(b1, b2)
+
+
+def test_int4_checkpoint_round_trip(tmp_path):
+    import torch
+
+    from post_weight_quantization_autoround_b200 import QConfig, driver
+
+    rng = np.random.default_rng(0)
+    results = []
+    for b in range(2):
+        layers = []
+        for N, K in ((64, 32), (64, 32), (32, 64)):
+            layers.append((torch.from_numpy(rng.integers(0, 2**31, (N, K // 8), dtype=np.int64).astype(np.int32)),
+                           torch.from_numpy(rng.standard_normal((N, K // 32)).astype(np.float16)),
+                           torch.from_numpy(rng.integers(0, 16, (N, K // 32)).astype(np.float16))))
+        results.append({"int4": layers})
+    cfg = QConfig(4, 32, 0, 0.005, 200, -0.5, 0.5, 0.5, 1.0)
+    path = str(tmp_path / "ckpt.npz")
+    driver.save_int4_checkpoint(path, results, cfg)
+    meta, arrays = driver.load_int4_checkpoint(path)
+    assert meta["bits"] == 4 and meta["group_size"] == 32 and meta["blocks"] == 2
+    for b, r in enumerate(results):
+        for name, (p, s, z) in zip(("gate", "up", "down"), r["int4"]):
+            assert np.array_equal(arrays[f"b{b}.{name}.packed"], p.numpy().view(np.uint32))
+            assert np.array_equal(arrays[f"b{b}.{name}.scale"], s.numpy())
+            assert np.array_equal(arrays[f"b{b}.{name}.zero"], z.numpy())

@@ -88,3 +88,32 @@ def test_driver_matches_oracle_on_a_two_block_model(ar):
             assert np.array_equal(z16.cpu().numpy().view(np.uint16), zref)
         # the first step sees the start state: the GPU and the oracle agree closely
         assert got["losses"][0] == pytest.approx(want["losses"][0], rel=1e-4)
+
+
+def test_streamed_driver_equals_the_device_driver_and_writes_a_checkpoint(ar, tmp_path):
+    """Weights streamed from pinned host memory (next block copied while this one is tuned) give
+    the same results as device-resident weights: the same kernels run on the same data."""
+    from post_weight_quantization_autoround_b200 import driver
+
+    H, F, S, L, batch, steps, g = 256, 512, 8, 32, 4, 3, 128
+    raw = [synth.make_mlp(H, F, 1, seed=30 + b) for b in range(3)]
+    X0 = bf16_dev(synth.make_activations(S * L, H, seed=8)).view(S, L, H)
+    sched = synth.make_schedule(S, batch, steps, seed=2)
+    cfg = ar.ar_qconfig_default(bits=4, group_size=g)
+    dev_res = driver.tune_mlp_blocks([[bf16_dev(d[k]) for k in ("Wg", "Wu", "Wd")] for d in raw], X0, cfg, sched,
+                                     export_int4=True)
+    host = [[bf16_dev(d[k]).cpu().pin_memory() for k in ("Wg", "Wu", "Wd")] for d in raw]
+    st_res = driver.tune_mlp_blocks_streamed(host, X0, cfg, sched)
+    assert ar.ar_get_device_status() == 0
+    for a, b in zip(dev_res, st_res):
+        assert np.array_equal(a["losses"], b["losses"])
+        for pa, pb in zip(a["int4"], b["int4"]):
+            for ta, tb in zip(pa, pb):
+                assert torch.equal(ta.cpu(), tb)
+    assert torch.equal(dev_res[-1]["x_out"], st_res[-1]["x_out"])
+    path = str(tmp_path / "model.npz")
+    driver.save_int4_checkpoint(path, st_res, cfg)
+    meta, arrays = driver.load_int4_checkpoint(path)
+    assert meta["blocks"] == 3
+    assert np.array_equal(arrays["b2.down.packed"], st_res[2]["int4"][2][0].numpy().view(np.uint32))
+
