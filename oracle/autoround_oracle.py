@@ -415,6 +415,40 @@ def w4a16_matmul(A, words, scale16, zero16, group_size: int) -> np.ndarray:
     return np.asarray(A, f64) @ deq.reshape(N, K).T
 
 
+def pack_codes(q: np.ndarray, bits: int) -> np.ndarray:
+    """b-bit codes packed little end first along K: 32/b codes per uint32,
+    element k at bits b*(k mod 32/b) of word k/(32/b) (the INT4 layout of
+    ``pack_int4`` for other widths; b in {2, 4, 8})."""
+    assert bits in (2, 4, 8)
+    per = 32 // bits
+    N, K = q.shape
+    assert K % per == 0
+    qi = np.asarray(q).astype(np.uint32).reshape(N, K // per, per)
+    assert qi.max(initial=0) < (1 << bits)
+    shifts = (bits * np.arange(per, dtype=np.uint32))[None, None, :]
+    return np.bitwise_or.reduce(qi << shifts, axis=-1).astype(np.uint32)
+
+
+def unpack_codes(words: np.ndarray, K: int, bits: int) -> np.ndarray:
+    """Inverse of ``pack_codes``."""
+    per = 32 // bits
+    N = words.shape[0]
+    shifts = (bits * np.arange(per, dtype=np.uint32))[None, None, :]
+    q = (words[:, :, None] >> shifts) & np.uint32((1 << bits) - 1)
+    return q.reshape(N, K).astype(np.uint16)
+
+
+def wxa16_matmul(A, words, scale16, zero16, group_size: int, bits: int) -> np.ndarray:
+    """out[t][n] = Σ_k A[t][k]·(q[n][k] - zero[n][k/g])·scale[n][k/g] for b-bit codes, fp64."""
+    N = words.shape[0]
+    K = words.shape[1] * (32 // bits)
+    q = unpack_codes(words, K, bits).astype(f64)
+    s = scale16.view(np.float16).astype(f64)
+    z = zero16.view(np.float16).astype(f64)
+    deq = (q.reshape(N, K // group_size, group_size) - z[:, :, None]) * s[:, :, None]
+    return np.asarray(A, f64) @ deq.reshape(N, K).T
+
+
 # ----------------------------------------------------------------------------
 # SwiGLU MLP block tuned jointly ([AR] §3 "Why Block-Wise Optimization": the
 # error of downstream sub-layers back-propagates to upstream weights)

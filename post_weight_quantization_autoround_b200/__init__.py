@@ -85,6 +85,8 @@ _SIGNATURES = {
     "ar_profile_start": (_INT, []),
     "ar_profile_stop": (_INT, [ctypes.c_char_p, ctypes.c_size_t]),
     "ar_gather_samples": (_INT, [_P, _I64, _I64, ctypes.POINTER(ctypes.c_int32), _INT, _P, _P]),
+    "ar_pack_codes": (_INT, [_P, _P, _P, _P, _I64, _I64, ctypes.POINTER(QConfig), _P, _P, _P, _P]),
+    "ar_wxa16_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P]),
 }
 
 
@@ -263,6 +265,20 @@ def ar_w4a16_gemm(A, packed, scale16, zero16, group_size: int, out, stream=None)
     N = packed.shape[0]
     _check(lib().ar_w4a16_gemm(_ptr(A), T, _ptr(packed), _ptr(scale16), _ptr(zero16), N, K, group_size, _ptr(out),
                                _stream(stream)))
+
+
+def ar_pack_codes(W, V, alpha, beta, cfg: QConfig, packed, scale16, zero16, stream=None) -> None:
+    """cfg.bits in {2, 4, 8}: packed uint32 [N][K*bits/32] (as int32 tensor), fp16 scale/zero [N][K/g]."""
+    N, K = W.shape
+    _check(lib().ar_pack_codes(_ptr(W), _ptr(V), _ptr(alpha), _ptr(beta), N, K, ctypes.byref(cfg), _ptr(packed),
+                               _ptr(scale16), _ptr(zero16), _stream(stream)))
+
+
+def ar_wxa16_gemm(A, packed, scale16, zero16, group_size: int, bits: int, out, stream=None) -> None:
+    T, K = A.shape
+    N = packed.shape[0]
+    _check(lib().ar_wxa16_gemm(_ptr(A), T, _ptr(packed), _ptr(scale16), _ptr(zero16), N, K, group_size, bits,
+                               _ptr(out), _stream(stream)))
 
 
 def ar_gather_samples(src, idx, dst, stream=None) -> None:

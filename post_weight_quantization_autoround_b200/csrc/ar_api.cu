@@ -586,6 +586,52 @@ ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
   return end_call();
 }
 
+ar_status ar_pack_codes(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                        int64_t K, const ar_qconfig* cfg, uint32_t* packed, uint16_t* scale_f16, uint16_t* zero_f16,
+                        ar_stream_t stream) {
+  begin_call();
+  ar_status st = check_cfg(cfg);
+  if (st != AR_OK) return st;
+  const int bits = cfg->bits;
+  if (bits != 2 && bits != 4 && bits != 8)
+    return fail(AR_ERR_UNSUPPORTED, "ar_pack_codes packs 2, 4 or 8-bit codes (got %d)", bits);
+  const int g = cfg->group_size;
+  if (N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "N, K must be positive");
+  if (!pow2(g) || g < 8 || g > 1024) return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 8..1024", g);
+  if (K % g != 0 || K % (32 / bits) != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and of 32/bits");
+  const void* ptrs[] = {W, V, alpha, beta, packed, scale_f16, zero_f16};
+  for (const void* p : ptrs) {
+    if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  cudaError_t e = launch_pack_codes(W, V, alpha, beta, N, K, g, bits, cfg->symmetric, packed, scale_f16, zero_f16,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return end_call();
+}
+
+ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, const uint16_t* scale_f16,
+                        const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, int bits, uint16_t* out,
+                        ar_stream_t stream) {
+  if (bits == 4) return ar_w4a16_gemm(A, T, packed, scale_f16, zero_f16, N, K, group_size, out, stream);
+  begin_call();
+  if (bits != 2 && bits != 8) return fail(AR_ERR_UNSUPPORTED, "bits=%d: needs 2, 4 or 8", bits);
+  if (T < 1 || N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "T, N, K must be positive");
+  if (!pow2(group_size) || group_size < 32 || group_size > 1024)
+    return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 32..1024", group_size);
+  if (K % group_size != 0 || K % 128 != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and 128");
+  if (N > INT32_MAX || K > INT32_MAX || T > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  const void* ptrs[] = {A, packed, scale_f16, zero_f16, out};
+  for (const void* p : ptrs) {
+    if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  cudaError_t e = launch_wxa16_tc(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N),
+                                  static_cast<int>(K), group_size, bits, out, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wxa16 launch");
+  return end_call();
+}
+
 ar_status ar_gather_samples(const void* src, int64_t n_src_samples, int64_t sample_bytes, const int32_t* idx,
                             int n_idx, void* dst, ar_stream_t stream) {
   begin_call();

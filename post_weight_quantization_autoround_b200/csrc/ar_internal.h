@@ -42,6 +42,10 @@ cudaError_t launch_qdq(const uint16_t* W, const float* V, const float* alpha, co
 cudaError_t launch_pack_int4(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
                              int64_t K, int group_size, int symmetric, uint32_t* packed, uint16_t* scale16,
                              uint16_t* zero16, cudaStream_t stream);
+// 2, 4 or 8 bits per code, 32/bits codes per uint32 (ar_quant.cu)
+cudaError_t launch_pack_codes(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                              int64_t K, int group_size, int bits, int symmetric, uint32_t* packed,
+                              uint16_t* scale16, uint16_t* zero16, cudaStream_t stream);
 
 cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t stream);
 
@@ -119,5 +123,9 @@ cudaError_t launch_gather_samples(const void* src, int64_t sample_bytes, const i
 // T > 16: tcgen05 dequant GEMM (ar_w4a16_tc.cu)
 cudaError_t launch_w4a16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream);
+// 2, 4 or 8-bit codes (32/bits per uint32), any T: the same tcgen05 GEMM
+cudaError_t launch_wxa16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                            const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,
+                            cudaStream_t stream);
 
 }  // namespace ar

@@ -176,14 +176,16 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ W
   (void)groups_per_row;
 }
 
-// INT4 export: the same codes as qdq_kernel, written as nibbles (element k at
-// bits 4*(k mod 8) of word k/8) plus fp16 scale / zero per group.
-template <int TPG, int CHUNKS>
-__global__ void __launch_bounds__(256) pack_int4_kernel(const uint16_t* __restrict__ W, const float* __restrict__ V,
-                                                        const float* __restrict__ alpha,
-                                                        const float* __restrict__ beta, int64_t n_groups,
-                                                        int symmetric, uint32_t* __restrict__ packed,
-                                                        __half* __restrict__ scale16, __half* __restrict__ zero16) {
+// Packed export: the same codes as qdq_kernel, BITS (2, 4 or 8) bits each,
+// packed little end first along K (element k at bits BITS*(k mod 32/BITS) of
+// word k/(32/BITS); INT4: nibbles), plus fp16 scale / zero per group.  A
+// thread's 8 codes fill BITS bytes.
+template <int TPG, int CHUNKS, int BITS>
+__global__ void __launch_bounds__(256) pack_codes_kernel(const uint16_t* __restrict__ W, const float* __restrict__ V,
+                                                         const float* __restrict__ alpha,
+                                                         const float* __restrict__ beta, int64_t n_groups,
+                                                         int symmetric, uint8_t* __restrict__ packed,
+                                                         __half* __restrict__ scale16, __half* __restrict__ zero16) {
   constexpr int G = TPG * 8 * CHUNKS;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t grp = tid / TPG;
@@ -214,7 +216,8 @@ __global__ void __launch_bounds__(256) pack_int4_kernel(const uint16_t* __restri
   }
   if (!active) return;
   if (bad) raise_status(kStatusNonFinite);
-  const QParams p = group_qparams(fmaxf(lmax, 0.0f), fminf(lmin, 0.0f), alpha[grp], beta[grp], 4, symmetric);
+  const QParams p = group_qparams(fmaxf(lmax, 0.0f), fminf(lmin, 0.0f), alpha[grp], beta[grp], BITS, symmetric);
+  constexpr float Q = static_cast<float>((1 << BITS) - 1);
 
 #pragma unroll
   for (int c = 0; c < CHUNKS; ++c) {
@@ -223,16 +226,19 @@ __global__ void __launch_bounds__(256) pack_int4_kernel(const uint16_t* __restri
     const float4 v1 = *reinterpret_cast<const float4*>(V + e + 4);
     const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     const uint32_t wr[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
-    uint32_t word = 0;
+    uint64_t bits = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float w = (i & 1) ? bf16_hi(wr[i >> 1]) : bf16_lo(wr[i >> 1]);
       const float u = __fadd_rn(__fdiv_rn(w, p.s), vv[i]);
       const float t = __fadd_rn(roundf(u), p.zp);
-      const float q = fminf(fmaxf(t, 0.0f), 15.0f);
-      word |= static_cast<uint32_t>(q) << (4 * i);
+      const float q = fminf(fmaxf(t, 0.0f), Q);
+      bits |= static_cast<uint64_t>(q) << (BITS * i);
     }
-    packed[e >> 3] = word;
+    uint8_t* dst = packed + (e * BITS) / 8;
+    if (BITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bits);
+    else if (BITS == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(bits);
+    else *reinterpret_cast<uint2*>(dst) = make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
   }
   if (li == 0) {
     scale16[grp] = __float2half_rn(p.s);
@@ -294,21 +300,24 @@ cudaError_t launch_qdq(const uint16_t* W, const float* V, const float* alpha, co
 }
 #undef AR_QDQ_CASE
 
-#define AR_PACK_CASE(TPG_, CH_)                                                                                 \
-  case (TPG_ * 8 * CH_): {                                                                                      \
-    const int64_t threads = n_groups * TPG_;                                                                    \
-    const int blocks = static_cast<int>((threads + 255) / 256);                                                 \
-    LaunchScope scope(stream, "pack_int4_kernel<g=" #TPG_ "x8x" #CH_ ">");                                     \
-    pack_int4_kernel<TPG_, CH_><<<blocks, 256, 0, stream>>>(W, V, alpha, beta, n_groups, symmetric, packed,   \
-                                                            reinterpret_cast<__half*>(scale16),                \
-                                                            reinterpret_cast<__half*>(zero16));                \
-    break;                                                                                                      \
-  }
-
-cudaError_t launch_pack_int4(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
-                             int64_t K, int group_size, int symmetric, uint32_t* packed, uint16_t* scale16,
+template <int BITS>
+cudaError_t launch_pack_bits(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                             int64_t K, int group_size, int symmetric, uint8_t* packed, uint16_t* scale16,
                              uint16_t* zero16, cudaStream_t stream) {
   const int64_t n_groups = N * (K / group_size);
+  __half* s16 = reinterpret_cast<__half*>(scale16);
+  __half* z16 = reinterpret_cast<__half*>(zero16);
+#define AR_PACK_CASE(TPG_, CH_)                                                                               \
+  case (TPG_ * 8 * CH_): {                                                                                    \
+    const int64_t threads = n_groups * TPG_;                                                                  \
+    const int blocks = static_cast<int>((threads + 255) / 256);                                               \
+    LaunchScope scope(stream, BITS == 4 ? "pack_codes_kernel<b=4,g=" #TPG_ "x8x" #CH_ ">"                      \
+                                        : BITS == 2 ? "pack_codes_kernel<b=2,g=" #TPG_ "x8x" #CH_ ">"          \
+                                                    : "pack_codes_kernel<b=8,g=" #TPG_ "x8x" #CH_ ">");        \
+    pack_codes_kernel<TPG_, CH_, BITS><<<blocks, 256, 0, stream>>>(W, V, alpha, beta, n_groups, symmetric,    \
+                                                                   packed, s16, z16);                         \
+    break;                                                                                                    \
+  }
   switch (group_size) {
     AR_PACK_CASE(1, 1)
     AR_PACK_CASE(2, 1)
@@ -321,9 +330,26 @@ cudaError_t launch_pack_int4(const uint16_t* W, const float* V, const float* alp
     default:
       return cudaErrorInvalidValue;
   }
+#undef AR_PACK_CASE
   return cudaGetLastError();
 }
-#undef AR_PACK_CASE
+
+cudaError_t launch_pack_int4(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                             int64_t K, int group_size, int symmetric, uint32_t* packed, uint16_t* scale16,
+                             uint16_t* zero16, cudaStream_t stream) {
+  return launch_pack_bits<4>(W, V, alpha, beta, N, K, group_size, symmetric, reinterpret_cast<uint8_t*>(packed),
+                             scale16, zero16, stream);
+}
+
+cudaError_t launch_pack_codes(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
+                              int64_t K, int group_size, int bits, int symmetric, uint32_t* packed,
+                              uint16_t* scale16, uint16_t* zero16, cudaStream_t stream) {
+  uint8_t* dst = reinterpret_cast<uint8_t*>(packed);
+  if (bits == 2) return launch_pack_bits<2>(W, V, alpha, beta, N, K, group_size, symmetric, dst, scale16, zero16, stream);
+  if (bits == 4) return launch_pack_bits<4>(W, V, alpha, beta, N, K, group_size, symmetric, dst, scale16, zero16, stream);
+  if (bits == 8) return launch_pack_bits<8>(W, V, alpha, beta, N, K, group_size, symmetric, dst, scale16, zero16, stream);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t stream) {
   const int64_t vec = (n + 3) / 4;

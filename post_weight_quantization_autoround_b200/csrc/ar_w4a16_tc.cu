@@ -50,10 +50,15 @@ namespace {
 constexpr int kTcRows = 128;  // weight rows per CTA (MMA M, TMEM lanes)
 constexpr int kTcK = 128;     // k per stage: 8 MMAs per barrier hand-off
 constexpr int kSub = kTcK / 64;  // 64-k sub-tiles (one 128-byte swizzle row of bf16 each)
-constexpr int kCodeK = 256;   // k per code slot: one 128-byte row of packed words
-constexpr int kCodeBytes = kTcRows * 128;  // 16 KiB per code slot
+constexpr int kCodeBytes = kTcRows * 128;  // 16 KiB per code slot: one 128-byte row of packed words per weight row
+// k per code slot and stages per slot for BITS-bit codes (32/BITS codes per word)
+template <int BITS>
+struct CodeCfg {
+  static constexpr int kCodeK = 1024 / BITS;          // 512, 256 or 128
+  static constexpr int kChunksPerSlot = kCodeK / 128;  // 4, 2 or 1 stages of 128 k
+  static constexpr int kVecPerStage = BITS;            // 16-byte vectors of one row per stage
+};
 constexpr int kCodeSlots = 4;
-constexpr int kChunksPerSlot = kCodeK / kTcK;
 constexpr int kNBufMax = 4;   // TMEM accumulators, one group each
 constexpr int kAStages = 4;   // A operand stages in TMEM (and activation stages in shared memory)
 constexpr int kACols = kTcK / 2;  // TMEM columns per A stage (two bf16 per column)
@@ -180,6 +185,30 @@ __device__ __forceinline__ uint4 dequant8(uint32_t x, uint32_t zz) {
 
 // bf16 pair (128 + z, 128 + z) from the fp16 bits of an integer zero-point 0..15
 // (128 + z is exact in bf16: its ulp is 1 in [128, 256)).
+// 16 two-bit codes of one word -> 16 bf16 values (q - z) in k order (8 words);
+// zz = (128 + z) in both halves.
+__device__ __forceinline__ void dequant16(uint32_t x, uint32_t zz, uint32_t* o) {
+  uint32_t e[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) e[i] = bf16x2_sub(((x >> (2 * i)) & 0x00030003u) | 0x43004300u, zz);  // (k_i, k_{i+8})
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    o[j] = __byte_perm(e[2 * j], e[2 * j + 1], 0x5410);      // (k_{2j}, k_{2j+1})
+    o[4 + j] = __byte_perm(e[2 * j], e[2 * j + 1], 0x7632);  // (k_{8+2j}, k_{9+2j})
+  }
+}
+
+// 4 eight-bit codes of one word -> 4 bf16 values (q - z) in k order (2 words):
+// the byte under an fp32 exponent of 2^23 is 2^23 + q exactly, one subtraction
+// of zf = 2^23 + z leaves q - z exactly (|q - z| <= 255 is exact in bf16).
+__device__ __forceinline__ void dequant4b(uint32_t x, float zf, uint32_t* o) {
+  float f[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f[i] = __fsub_rn(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7540u | i)), zf);
+  o[0] = pack_bf16x2(f[0], f[1]);
+  o[1] = pack_bf16x2(f[2], f[3]);
+}
+
 __device__ __forceinline__ uint32_t zero_pair(uint16_t z16) {
   const uint32_t z = static_cast<uint32_t>(__half2float(__ushort_as_half(z16)));
   return (0x4300u + z) * 0x00010001u;
@@ -245,7 +274,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // Grid: one CTA per (128-row tile, token tile, K half when split); the CTAs of
 // a weight tile are adjacent so that its codes come from HBM once.
-template <int TN, int KSPLIT>
+template <int TN, int KSPLIT, int BITS>
 __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const TcParams p) {
@@ -282,7 +311,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     }
     for (int s = 0; s < kCodeSlots; ++s) {
       mbar_init(&ctl->code_full[s], 1);
-      mbar_init(&ctl->code_empty[s], 4 * kChunksPerSlot);
+      mbar_init(&ctl->code_empty[s], 4 * CodeCfg<BITS>::kChunksPerSlot);
     }
     for (int b = 0; b < Cfg::kNBuf; ++b) {
       mbar_init(&ctl->tmem_full[b], 1);
@@ -420,13 +449,15 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ code TMA: up to 16 stages ahead
     if (lane == 0) {
+      constexpr int kChunksPerSlot = CodeCfg<BITS>::kChunksPerSlot;
       const int n_slots = (c_end - c_begin + kChunksPerSlot - 1) / kChunksPerSlot;
       uint32_t slots = 0;
       for (int j = 0; j < n_slots; ++j) {
         const uint32_t cs = static_cast<uint32_t>(j % kCodeSlots);
         if (!mbar_wait_sleep(&ctl->code_empty[cs], ((j / kCodeSlots) & 1u) ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&ctl->code_full[cs], kCodeBytes);
-        tma_load_2d(codes + cs * kCodeBytes, &tmW, &ctl->code_full[cs], (c_begin + j * kChunksPerSlot) * (kTcK / 8), n0);
+        tma_load_2d(codes + cs * kCodeBytes, &tmW, &ctl->code_full[cs], (c_begin + j * kChunksPerSlot) * (kTcK * BITS / 32),
+                    n0);
         ++slots;
       }
       const uint32_t first_slot = slots > kCodeSlots ? slots - kCodeSlots : 0;
@@ -447,6 +478,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
       const int c = c_begin + i;
       const uint32_t stage = static_cast<uint32_t>(i % Cfg::kStages);
       const uint32_t phase = static_cast<uint32_t>((i / Cfg::kStages) & 1);
+      constexpr int kChunksPerSlot = CodeCfg<BITS>::kChunksPerSlot;
       const uint32_t j = static_cast<uint32_t>(i / kChunksPerSlot);
       const uint32_t cs = j % kCodeSlots;
       // codes landed, the MMAs of this stage's previous use have released its A
@@ -455,30 +487,61 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
                       mbar_wait_sleep(&ctl->empty[stage], phase ^ 1u, abort_flag);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
-      // this stage's 64 bytes of row r: 16-byte chunks q4..q4+3 of the row, swizzled by r % 8
-      const uint32_t q4 = static_cast<uint32_t>(4 * (i % kChunksPerSlot));
+      // this stage's 16*BITS bytes of row r: 16-byte vectors qv..qv+BITS-1 of the row, swizzled by r % 8
+      const uint32_t qv = static_cast<uint32_t>(BITS * (i % kChunksPerSlot));
       const uint32_t pk = smem_u32(codes + cs * kCodeBytes) + r * 128;
-      uint4 pw[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) pw[h] = ld_shared_v4(pk + (((q4 + h) ^ sw) << 4));
       const int k0 = c * kTcK;
-      // zero-points of the four 32-k quarters (equal when g >= 128)
-      uint32_t zq[4];
+      // the stage's codes: all loads issued before any conversion, except that
+      // 8-bit stages (eight 16-byte vectors a row) load one half at a time
+      constexpr int kPre = BITS == 8 ? BITS / 2 : BITS;
+      uint4 pw[kPre];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) zq[h] = (h == 0 || p.group_shift < 7) ? zero_pair(zrow.get((k0 + 32 * h) >> p.group_shift)) : zq[0];
-      // column 4w + e of the stage holds k = 8w + 2e, 8w + 2e + 1
+      for (int v = 0; v < kPre; ++v) pw[v] = ld_shared_v4(pk + (((qv + v) ^ sw) << 4));
+      // zero-points of the four 32-k quarters (equal when g >= 128), converted once:
+      // (128 + z) bf16 pairs for 2 and 4 bits, 2^23 + z in fp32 for 8 bits
+      uint32_t zz[4];
+      float zf[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        if (h == 0 || p.group_shift < 7) {
+          const uint16_t z = zrow.get((k0 + 32 * h) >> p.group_shift);
+          if (BITS == 8) zf[h] = 8388608.0f + __half2float(__ushort_as_half(z));
+          else zz[h] = zero_pair(z);
+        } else {
+          zz[h] = zz[0];
+          zf[h] = zf[0];
+        }
+      }
+      // column c of the stage holds k = 2c, 2c + 1
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t a[32];
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          const uint4 v = pw[2 * half + (w >> 2)];
-          const uint32_t x = (w & 3) == 0 ? v.x : (w & 3) == 1 ? v.y : (w & 3) == 2 ? v.z : v.w;
-          const uint4 o = dequant8(x, zq[2 * half + (w >> 2)]);
-          a[4 * w + 0] = o.x;
-          a[4 * w + 1] = o.y;
-          a[4 * w + 2] = o.z;
-          a[4 * w + 3] = o.w;
+        if (BITS == 8 && half == 1) {
+#pragma unroll
+          for (int v = 0; v < kPre; ++v) pw[v] = ld_shared_v4(pk + (((qv + kPre + v) ^ sw) << 4));
+        }
+#pragma unroll
+        for (int v = 0; v < BITS / 2; ++v) {
+          const uint4 pv = pw[BITS == 8 ? v : half * (BITS / 2) + v];
+          const uint32_t xs[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int w = half * 2 * BITS + 4 * v + u;  // word of the stage; it covers k 32w/BITS ..
+            const int quarter = w / BITS;
+            const int col = (w - half * 2 * BITS) * (16 / BITS);  // first column of this word in the half
+            if (BITS == 4) {
+              const uint4 o = dequant8(xs[u], zz[quarter]);
+              a[col] = o.x;
+              a[col + 1] = o.y;
+              a[col + 2] = o.z;
+              a[col + 3] = o.w;
+            } else if (BITS == 2) {
+              dequant16(xs[u], zz[quarter], &a[col]);
+            } else {
+              dequant4b(xs[u], zf[quarter], &a[col]);
+            }
+          }
         }
         tmem_st32(lane_base + kACols * stage + 32 * half, a);
       }
@@ -566,7 +629,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
   }
 }
 
-template <int TN, int KSPLIT>
+template <int TN, int KSPLIT, int BITS>
 cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int n_tiles, cudaStream_t stream,
                       const char* name) {
   using Cfg = TcCfg<TN>;
@@ -576,7 +639,7 @@ cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int
   if (e != cudaSuccess) return e;
   constexpr int smem = Cfg::kRingBytes + static_cast<int>(sizeof(TcCtl)) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory per CTA");
-  auto kern = w4a16_tc_kernel<TN, KSPLIT>;
+  auto kern = w4a16_tc_kernel<TN, KSPLIT, BITS>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -597,7 +660,7 @@ cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int
   return cudaGetLastError();
 }
 
-template <int TN>
+template <int TN, int BITS>
 cudaError_t launch_tn(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int n_tiles, cudaStream_t stream,
                       const char* name1, const char* name2) {
   // Split K over a CTA pair when one CTA per tile leaves more than half the SMs idle.
@@ -607,17 +670,42 @@ cudaError_t launch_tn(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int
     p.split_units = (total_units + 1) / 2;
     const int g_split = (p.split_units * p.unit_k) >> p.group_shift;
     p.vec_meta = (p.G % 8 == 0 && g_split % 8 == 0) ? 1 : 0;
-    return launch_tc<TN, 2>(A, tmW, p, n_tiles, stream, name2);
+    return launch_tc<TN, 2, BITS>(A, tmW, p, n_tiles, stream, name2);
   }
   p.split_units = total_units;
   p.vec_meta = p.G % 8 == 0 ? 1 : 0;
-  return launch_tc<TN, 1>(A, tmW, p, n_tiles, stream, name1);
+  return launch_tc<TN, 1, BITS>(A, tmW, p, n_tiles, stream, name1);
 }
 
-}  // namespace
 
-cudaError_t launch_w4a16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
-                            const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream) {
+// profiler / trace names per width: TN = 16, 32, 64, 128, each unsplit and split over a CTA pair
+template <int BITS>
+struct TcNames;
+template <>
+struct TcNames<2> {
+  static constexpr const char* n[8] = {"wxa16_tc_kernel<b=2,TN=16>", "wxa16_tc_kernel<b=2,TN=16,split2>",
+                                       "wxa16_tc_kernel<b=2,TN=32>", "wxa16_tc_kernel<b=2,TN=32,split2>",
+                                       "wxa16_tc_kernel<b=2,TN=64>", "wxa16_tc_kernel<b=2,TN=64,split2>",
+                                       "wxa16_tc_kernel<b=2,TN=128>", "wxa16_tc_kernel<b=2,TN=128,split2>"};
+};
+template <>
+struct TcNames<4> {
+  static constexpr const char* n[8] = {"w4a16_tc_kernel<TN=16>", "w4a16_tc_kernel<TN=16,split2>",
+                                       "w4a16_tc_kernel<TN=32>", "w4a16_tc_kernel<TN=32,split2>",
+                                       "w4a16_tc_kernel<TN=64>", "w4a16_tc_kernel<TN=64,split2>",
+                                       "w4a16_tc_kernel<TN=128>", "w4a16_tc_kernel<TN=128,split2>"};
+};
+template <>
+struct TcNames<8> {
+  static constexpr const char* n[8] = {"wxa16_tc_kernel<b=8,TN=16>", "wxa16_tc_kernel<b=8,TN=16,split2>",
+                                       "wxa16_tc_kernel<b=8,TN=32>", "wxa16_tc_kernel<b=8,TN=32,split2>",
+                                       "wxa16_tc_kernel<b=8,TN=64>", "wxa16_tc_kernel<b=8,TN=64,split2>",
+                                       "wxa16_tc_kernel<b=8,TN=128>", "wxa16_tc_kernel<b=8,TN=128,split2>"};
+};
+
+template <int BITS>
+cudaError_t launch_bits_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                           const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream) {
   TcParams p{};
   p.s16 = scale16;
   p.z16 = zero16;
@@ -630,23 +718,39 @@ cudaError_t launch_w4a16_tc(const uint16_t* A, int T, const uint32_t* packed, co
   p.unit_k = group_size > kTcK ? group_size : kTcK;
   CUtensorMap tmW;
   cudaError_t e = make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, static_cast<uint64_t>(N),
-                               static_cast<uint64_t>(K / 8), kCodeK / 8, kTcRows, CU_TENSOR_MAP_SWIZZLE_128B);
+                               static_cast<uint64_t>(K) * BITS / 32, 32, kTcRows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const int n_tiles = (N + kTcRows - 1) / kTcRows;
   if (T <= 16) {
     p.t_tiles = 1;
-    return launch_tn<16>(A, tmW, p, n_tiles, stream, "w4a16_tc_kernel<TN=16>", "w4a16_tc_kernel<TN=16,split2>");
+    return launch_tn<16, BITS>(A, tmW, p, n_tiles, stream, TcNames<BITS>::n[0], TcNames<BITS>::n[1]);
   }
   if (T <= 32) {
     p.t_tiles = 1;
-    return launch_tn<32>(A, tmW, p, n_tiles, stream, "w4a16_tc_kernel<TN=32>", "w4a16_tc_kernel<TN=32,split2>");
+    return launch_tn<32, BITS>(A, tmW, p, n_tiles, stream, TcNames<BITS>::n[2], TcNames<BITS>::n[3]);
   }
   if (T <= 64) {
     p.t_tiles = 1;
-    return launch_tn<64>(A, tmW, p, n_tiles, stream, "w4a16_tc_kernel<TN=64>", "w4a16_tc_kernel<TN=64,split2>");
+    return launch_tn<64, BITS>(A, tmW, p, n_tiles, stream, TcNames<BITS>::n[4], TcNames<BITS>::n[5]);
   }
   p.t_tiles = (T + 127) / 128;
-  return launch_tn<128>(A, tmW, p, n_tiles, stream, "w4a16_tc_kernel<TN=128>", "w4a16_tc_kernel<TN=128,split2>");
+  return launch_tn<128, BITS>(A, tmW, p, n_tiles, stream, TcNames<BITS>::n[6], TcNames<BITS>::n[7]);
+}
+
+}  // namespace
+
+cudaError_t launch_w4a16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                            const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream) {
+  return launch_bits_tc<4>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+}
+
+cudaError_t launch_wxa16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                            const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,
+                            cudaStream_t stream) {
+  if (bits == 2) return launch_bits_tc<2>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+  if (bits == 4) return launch_bits_tc<4>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+  if (bits == 8) return launch_bits_tc<8>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace ar

@@ -146,3 +146,17 @@ def test_gather_samples_validation():
     assert g(FAKE + 8, 4, 64, idx, 3, 0x20000, None) == ar.AR_ERR_INVALID_ARG       # misaligned
     assert g(FAKE, 4, 64, None, 3, 0x20000, None) == ar.AR_ERR_INVALID_ARG          # no index array
 
+
+def test_pack_codes_and_wxa16_validation():
+    c3 = ar.ar_qconfig_default(bits=3)
+    assert ar.lib().ar_pack_codes(FAKE, FAKE, FAKE, FAKE, 8, 128, ctypes.byref(c3), FAKE, FAKE, FAKE, None) == \
+        ar.AR_ERR_UNSUPPORTED
+    c2 = ar.ar_qconfig_default(bits=2, group_size=8)
+    assert ar.lib().ar_pack_codes(FAKE, FAKE, FAKE, FAKE, 8, 8, ctypes.byref(c2), FAKE, FAKE, FAKE, None) == \
+        ar.AR_ERR_INVALID_ARG  # K % 16 for 2-bit words
+    w = ar.lib().ar_wxa16_gemm
+    assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 128, 3, FAKE, None) == ar.AR_ERR_UNSUPPORTED
+    assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 16, 2, FAKE, None) == ar.AR_ERR_UNSUPPORTED
+    assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 192, 64, 8, FAKE, None) == ar.AR_ERR_INVALID_ARG  # K % 128
+    assert w(FAKE, 0, FAKE, FAKE, FAKE, 64, 256, 128, 2, FAKE, None) == ar.AR_ERR_INVALID_ARG
+

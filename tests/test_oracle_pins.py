@@ -534,3 +534,52 @@ def test_mlp_fp32_instantiation_agrees_with_fp64():
     for gr, g64, W, st in zip(grads, (gWg, gWu, gWd), Ws, sts):
         dV64, da64, db64 = O.ste_fold(g64, W, st, 4)
         assert rel(gr["dV"], dV64) < 5e-2 and rel(gr["dalpha"], da64) < 5e-2
+
+
+# ----------------------------------------------------------------------------
+# packed 2/4/8-bit codes (the INT4 layout generalised; pages silent on other widths)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_pack_codes_round_trips_and_places_each_code_by_hand(bits):
+    rng = np.random.default_rng(bits)
+    per = 32 // bits
+    q = rng.integers(0, 1 << bits, (5, 4 * per)).astype(np.uint8)
+    w = O.pack_codes(q, bits)
+    assert w.shape == (5, 4) and w.dtype == np.uint32
+    assert np.array_equal(O.unpack_codes(w, 4 * per, bits), q)
+    # every code sits at bits b*(k mod per) of word k / per, written out with Python ints
+    for n in range(5):
+        for j in range(4):
+            word = 0
+            for i in range(per):
+                word |= int(q[n, j * per + i]) << (bits * i)
+            assert int(w[n, j]) == word
+
+
+def test_pack_codes_at_four_bits_is_the_int4_packing():
+    rng = np.random.default_rng(1)
+    q = rng.integers(0, 16, (3, 64)).astype(np.uint8)
+    s = rng.random((3, 2)).astype(np.float32)
+    z = rng.integers(0, 16, (3, 2)).astype(np.float32)
+    assert np.array_equal(O.pack_codes(q, 4), O.pack_int4(q, s, z)[0])
+
+
+@pytest.mark.parametrize("bits", [2, 8])
+def test_wxa16_matmul_against_loops(bits):
+    rng = np.random.default_rng(10 + bits)
+    N, K, T, g = 3, 64, 2, 32
+    q = rng.integers(0, 1 << bits, (N, K))
+    w = O.pack_codes(q, bits)
+    s16 = rng.random((N, K // g)).astype(np.float16).view(np.uint16)
+    z16 = rng.integers(0, 1 << bits, (N, K // g)).astype(np.float16).view(np.uint16)
+    A = rng.standard_normal((T, K)).astype(np.float32)
+    got = O.wxa16_matmul(A, w, s16, z16, g, bits)
+    for t in range(T):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                sc = float(s16.view(np.float16)[n, k // g])
+                zz = float(z16.view(np.float16)[n, k // g])
+                acc += float(A[t, k]) * (int(q[n, k]) - zz) * sc
+            assert got[t, n] == pytest.approx(acc, rel=1e-12, abs=1e-12)
