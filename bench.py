@@ -282,6 +282,31 @@ def w4a16_bench(ar, torch, peaks, reps=20):
                         "roofline_frac": t_roof / (ms * 1e-3),
                         "algorithmic_bytes": nbytes, "kernel": ar.ar_last_kernels()}
     out["shape"] = f"{N}x{K} int4 g{g}, fp16 scale/zero, bf16 activations; L2 flushed before each launch"
+    # the same layer packed at 2 and 8 bits (tcgen05 dequant GEMM at every T)
+    W = to_dev_bf16(d["W"], torch)
+    V = torch.zeros((N, K), dtype=torch.float32, device="cuda")
+    for bits in (2, 8):
+        cfgb = ar.ar_qconfig_default(bits=bits, group_size=g)
+        pk = torch.empty((N, K * bits // 32), dtype=torch.int32, device="cuda")
+        ar.ar_pack_codes(W, V, a, b, cfgb, pk, s16, z16)
+        for T in (1, 256):
+            A = to_dev_bf16(synth.make_activations(T, K, seed=T), torch)
+            y = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+            for _ in range(3):
+                ar.ar_wxa16_gemm(A, pk, s16, z16, g, bits, y)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for e0, e1 in ev:
+                flush.sum()
+                e0.record()
+                ar.ar_wxa16_gemm(A, pk, s16, z16, g, bits, y)
+                e1.record()
+            torch.cuda.synchronize()
+            ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+            nbytes = pk.numel() * 4 + s16.numel() * 2 + z16.numel() * 2 + A.numel() * 2 + y.numel() * 2
+            out[f"W{bits}A16_T{T}"] = {"us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9,
+                                      "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                      "TFLOP/s": 2.0 * T * N * K / (ms * 1e-3) / 1e12, "kernel": ar.ar_last_kernels()}
+    del W, V
     return out
 
 
