@@ -116,6 +116,11 @@ cudaError_t read_and_clear_status(unsigned int* out, cudaStream_t stream);
 // ---- W4A16 (ar_w4a16.cu) ----
 cudaError_t launch_w4a16(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                          const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream);
+// decode kernel over per-SM row ranges (ar_w4a16_dec.cu); cudaErrorNotSupported
+// (nothing launched) for shapes whose scale/zero rows are not 16-byte multiples
+cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
+                             cudaStream_t stream);
 // minibatch assembly (ar_gather.cu): n <= kMaxGatherSamples samples of sample_bytes each
 constexpr int kMaxGatherSamples = 64;
 cudaError_t launch_gather_samples(const void* src, int64_t sample_bytes, const int32_t* idx, int n, void* dst,

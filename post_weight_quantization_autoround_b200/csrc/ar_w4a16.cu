@@ -365,11 +365,14 @@ cudaError_t launch_tma(const CUtensorMap& tmW, const uint16_t* A, int T, const _
 
 cudaError_t launch_w4a16(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                          const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream) {
+  cudaError_t e = launch_w4a16_dec(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+  if (e != cudaErrorNotSupported) return e;
+  (void)cudaGetLastError();
   int group_shift = 0;
   while ((1 << group_shift) < group_size) ++group_shift;
   CUtensorMap tmW;
-  cudaError_t e = make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, static_cast<uint64_t>(N),
-                               static_cast<uint64_t>(K / 8), 32, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+  e = make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, static_cast<uint64_t>(N),
+                   static_cast<uint64_t>(K / 8), 32, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const __half* s16 = reinterpret_cast<const __half*>(scale16);
   const __half* z16 = reinterpret_cast<const __half*>(zero16);

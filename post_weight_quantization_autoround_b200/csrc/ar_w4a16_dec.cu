@@ -1,0 +1,522 @@
+// W4A16 matmul for decode batches (T <= 16 tokens), one CTA per SM over a
+// contiguous range of weight rows: out[t][n] = sum_k A[t][k] (q[n][k] - z) s.
+//
+// [AR] §4 (comparison table, "Real INT4 Kernel" column): the weights stay
+// 4-bit in memory and are dequantized inside the kernel, activations are
+// 16-bit ([AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms
+// and Architectural Optimizations of AutoRound").
+//
+// At T <= 16 the kernel moves 0.5 byte per weight from HBM and its cost on the
+// SM is the 4-bit -> bf16 conversion (about 7 integer instructions per eight
+// codes).  The layout is chosen so that nothing else costs per weight:
+//
+//  * The weights are the B operand of mma.sync m16n8k16 (an n8 tile is eight
+//    weight rows) and the activations the A operand (16 token rows, rows past
+//    T repeat the last token and are discarded).  Eight-row tiles let every
+//    SM own the same number of rows (8192 rows -> 147 CTAs of 56 rows), and
+//    up to 16 tokens cost no extra MMAs.
+//  * Codes -> bf16 pairs without arithmetic: (word >> 4i) & 0x000F000F |
+//    0x43004300 is the bf16 pair (128 + q_i, 128 + q_{i+4}).  One more MMA
+//    against a fragment of ones gives O = sum of the activations over the same
+//    k, so a group's contribution is s (D - (128 + z) O), applied once per
+//    group span in fp32.
+//  * The reduction index of the MMA is permuted: lane (g = lane/4, c = lane%4)
+//    feeds k-slots {2c, 2c+1, 2c+8, 2c+9} of two consecutive MMAs from one
+//    32-bit word (eight codes, k = 32j + 8c + 0..7) of its weight row, and the
+//    activations are permuted the same way with byte permutes.
+//  * One producer warp streams 512-k stages with TMA: the codes of the pass's
+//    rows (two 256-k boxes, 128-byte swizzle, so that the fragment reads are
+//    free of bank conflicts), the activations, and the window of fp16
+//    (scale, zero) groups the stage touches.  Consumer warps work in groups of
+//    four (one 128-k chunk each) and the groups take stages in turn, so each
+//    warp owns whole group spans of its chunk.
+//  * A CTA's rows are cut into passes of at most 64; the consumer warps' sums
+//    are added in a fixed order through shared memory at the end of a pass.
+//    For small N the two CTAs of a cluster split K and rank 0 adds the
+//    partial sums in a fixed order through distributed shared memory.
+//    Results are deterministic and no workspace is needed.
+//
+// Packed layout (as ar_pack_int4 writes it): uint32 [N][K/8], element k at
+// bits 4*(k mod 8) of word k/8; scale/zero fp16 [N][K/g].
+#include <cooperative_groups.h>
+
+#include <cstdio>
+
+#include "ar_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace ar {
+namespace {
+
+constexpr int kDecStageK = 512;                 // k per stage
+constexpr int kDecPassRows = 64;                // rows per pass (eight n8 tiles)
+constexpr int kDecCodeBox = kDecPassRows * 128; // one 256-k box of codes: 64 rows x 128 bytes
+constexpr int kDecMaxStages = 8;
+constexpr int kDecSmemLimit = 227 * 1024;
+
+template <bool TBIG>
+struct DecCfg {
+  static constexpr int kWarps = TBIG ? 8 : 12;  // consumer warps
+  static constexpr int kGroups = kWarps / 4;    // stages in consumption at once
+  static constexpr int kThreads = (kWarps + 1) * 32;
+  // registers per thread: the warps are spread over the SM's four 16K-register
+  // partitions, so the partition with the most warps (ceil(warps / 4)) sets the cap
+  static constexpr int kMaxRegs = ((16384 / (32 * ((kWarps + 1 + 3) / 4))) / 8) * 8;
+  static constexpr int kTokPad = TBIG ? 16 : 8;
+  static constexpr int kAcc = TBIG ? 4 : 2;     // accumulators per n8 tile and lane
+  static constexpr int kRedBytes = kWarps * kDecPassRows * kTokPad * 4;
+};
+
+struct DecParams {
+  int N, K, T;
+  int rows_per_cta;  // multiple of 8
+  int passes;        // ceil(rows_per_cta / 64)
+  int last_rows;     // box height of the last pass
+  int n_stages;      // ceil(K / 512)
+  int group_shift;
+  int wg;            // groups per table window (8, or 16 when g = 32)
+  int act_off;       // stage layout: codes at 0, activations, scale table, zero table
+  int tab_off;
+  int stage_bytes;
+  int S;             // ring depth
+};
+
+struct alignas(16) DecTail {
+  float2 sm[12][kDecPassRows];  // per consumer warp: (s, -s (128 + z)) of the pass's rows for one group
+  uint64_t full[kDecMaxStages];
+  uint64_t empty[kDecMaxStages];
+  float part[kDecPassRows][16];
+  int abort_flag;
+};
+
+__host__ __device__ constexpr int dec_tail_offset(int S, int stage_bytes, int red_bytes) {
+  return S * stage_bytes + red_bytes;
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Same with a zero accumulator input (the first MMA of a group span).
+__device__ __forceinline__ void mma16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+
+// TBIG: 9..16 tokens (token rows g and g + 8 of the A fragment both live).
+// SPAN: 32-k slices per group span inside a 128-k chunk (4 for g >= 128, 2 for
+// g = 64, 1 for g = 32).  KS: CTAs of a cluster splitting K (1 or 2).  NT: n8
+// tiles per pass, a compile-time count so that the tile loops are straight-line
+// code (tiles past a pass's rows read rows of the stage buffer that the pass
+// does not own and are computed but never stored).
+template <bool TBIG, int SPAN, int KS, int NT>
+__global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
+    w4a16_dec_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWl,
+                     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmSl,
+                     const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmZl,
+                     const __grid_constant__ CUtensorMap tmA, const DecParams p, uint16_t* __restrict__ out) {
+  using C = DecCfg<TBIG>;
+  extern __shared__ uint8_t dec_smem_raw[];
+  // 1024-byte aligned base by pointer arithmetic on the shared array, so that
+  // every access below stays a shared-memory access (ld.shared)
+  uint8_t* smem = dec_smem_raw + ((1024u - (smem_u32(dec_smem_raw) & 1023u)) & 1023u);
+  float* red = reinterpret_cast<float*>(smem + p.S * p.stage_bytes);  // [warp][row][token]
+  DecTail& tl = *reinterpret_cast<DecTail*>(smem + dec_tail_offset(p.S, p.stage_bytes, C::kRedBytes));
+  volatile int* abort_flag = &tl.abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = KS == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int row_base = (blockIdx.x / KS) * p.rows_per_cta;
+  const int rows_here = min(p.rows_per_cta, p.N - row_base);
+  const int passes_here = (rows_here + kDecPassRows - 1) / kDecPassRows;
+  const int ks0 = (p.n_stages * rank) / KS;
+  const int nks = (p.n_stages * (rank + 1)) / KS - ks0;  // stages of one pass
+  const int total = passes_here * nks;
+  const int S = p.S;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&tl.full[s], 1);
+      mbar_init(&tl.empty[s], 4);
+    }
+    tl.abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == C::kWarps) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmW);
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmS);
+      tma_prefetch_desc(&tmZ);
+      int issued = 0;
+      for (int it = 0; it < total; ++it) {
+        const int s = it % S;
+        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+        if (!mbar_wait_sleep(&tl.empty[s], ph ^ 1u, abort_flag)) break;
+        const int pass = it / nks;
+        const int ks = ks0 + (it - pass * nks);
+        const bool last = pass == p.passes - 1;
+        const int h = last ? p.last_rows : kDecPassRows;
+        const int row0 = row_base + pass * kDecPassRows;
+        uint8_t* st = smem + s * p.stage_bytes;
+        const int gi0 = (ks * kDecStageK) >> p.group_shift;
+        const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
+        mbar_arrive_expect_tx(&tl.full[s], static_cast<uint32_t>(2 * 128 * h + 2 * 512 * p.T + 2 * 2 * p.wg * h));
+        tma_load_2d(st, last ? &tmWl : &tmW, &tl.full[s], ks * 64, row0);
+        tma_load_2d(st + kDecCodeBox, last ? &tmWl : &tmW, &tl.full[s], ks * 64 + 32, row0);
+        tma_load_2d(st + p.act_off, &tmA, &tl.full[s], ks * kDecStageK, 0);
+        tma_load_2d(st + p.act_off + 512 * p.T, &tmA, &tl.full[s], ks * kDecStageK + 256, 0);
+        tma_load_2d(st + p.tab_off, last ? &tmSl : &tmS, &tl.full[s], x0, row0);
+        tma_load_2d(st + p.tab_off + 2 * p.wg * kDecPassRows, last ? &tmZl : &tmZ, &tl.full[s], x0, row0);
+        ++issued;
+      }
+      const int first = issued > S ? issued - S : 0;
+      for (int i = first; i < issued; ++i) mbar_wait_drain(&tl.full[i % S], static_cast<uint32_t>(i / S) & 1u);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int cw = warp & 3;     // 128-k chunk of the stage
+    const int grp = warp >> 2;   // stages it == grp (mod kGroups)
+    const int g = lane >> 2;
+    const int c = lane & 3;
+    const int T = p.T;
+    const int tok_lo = min(g, T - 1);
+    const int tok_hi = min(g + 8, T - 1);
+    const int box = cw >> 1;
+    const uint32_t kOne2 = 0x3F803F80u;  // bf16 pair (1, 1)
+    bool ok = true;
+
+    float2* smw = tl.sm[warp];
+    for (int pass = 0; pass < passes_here; ++pass) {
+      const bool last = pass == p.passes - 1;
+      const int h = min(last ? p.last_rows : kDecPassRows, rows_here - pass * kDecPassRows);
+      float acc[NT][C::kAcc];
+#pragma unroll
+      for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+        for (int i = 0; i < C::kAcc; ++i) acc[jt][i] = 0.0f;
+
+      const int it_begin = pass * nks;
+      const int it_end = it_begin + nks;
+      int it = it_begin + ((grp - it_begin % C::kGroups) + C::kGroups) % C::kGroups;
+      for (; it < it_end; it += C::kGroups) {
+        const int s = it % S;
+        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+        if (ok) ok = mbar_wait_sleep(&tl.full[s], ph, abort_flag);
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+          const int ks = ks0 + (it - it_begin);
+          const uint8_t* st = smem + s * p.stage_bytes;
+          const uint8_t* codes = st + box * kDecCodeBox + g * 128 + 4 * c;
+          const uint8_t* act = st + p.act_off + box * 512 * T + (((cw & 1) * 128 + 8 * c) * 2);
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + p.tab_off);
+          const uint16_t* zr = sc + p.wg * kDecPassRows;
+          const int gi0 = (ks * kDecStageK) >> p.group_shift;
+          const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
+          float d[NT][4], o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // activations of this lane's k-range (eight bf16) for token rows g and g + 8
+            const uint4 v = *reinterpret_cast<const uint4*>(act + tok_lo * 512 + 64 * j);
+            uint32_t A0[4], A1[4];
+            A0[0] = __byte_perm(v.x, v.z, 0x5410);  // (k0, k4)
+            A0[2] = __byte_perm(v.x, v.z, 0x7632);  // (k1, k5)
+            A1[0] = __byte_perm(v.y, v.w, 0x5410);  // (k2, k6)
+            A1[2] = __byte_perm(v.y, v.w, 0x7632);  // (k3, k7)
+            if (TBIG) {
+              const uint4 u = *reinterpret_cast<const uint4*>(act + tok_hi * 512 + 64 * j);
+              A0[1] = __byte_perm(u.x, u.z, 0x5410);
+              A0[3] = __byte_perm(u.x, u.z, 0x7632);
+              A1[1] = __byte_perm(u.y, u.w, 0x5410);
+              A1[3] = __byte_perm(u.y, u.w, 0x7632);
+            } else {
+              A0[1] = A0[3] = A1[1] = A1[3] = 0u;
+            }
+            const bool first = (j % SPAN) == 0;
+            if (first) {
+              mma16816_z(o, A0, kOne2, kOne2);
+            } else {
+              mma16816(o, A0, kOne2, kOne2);
+            }
+            mma16816(o, A1, kOne2, kOne2);
+            // 16-byte chunk q of the 128-byte row, stored at chunk q ^ (row % 8) = q ^ g
+            const int q = (cw & 1) * 4 + j;
+            const uint8_t* cj = codes + ((q ^ g) << 4);
+#pragma unroll
+            for (int jt = 0; jt < NT; ++jt) {
+              {
+                const uint32_t x = *reinterpret_cast<const uint32_t*>(cj + jt * 8 * 128);
+                // MMA 0 slots (2c, 2c+1) <- nibbles (0, 4), (2c+8, 2c+9) <- (1, 5); MMA 1: (2, 6), (3, 7)
+                const uint32_t b00 = (x & 0x000F000Fu) | 0x43004300u;
+                const uint32_t b01 = ((x >> 4) & 0x000F000Fu) | 0x43004300u;
+                const uint32_t b10 = ((x >> 8) & 0x000F000Fu) | 0x43004300u;
+                const uint32_t b11 = ((x >> 12) & 0x000F000Fu) | 0x43004300u;
+                if (first) {
+                  mma16816_z(d[jt], A0, b00, b01);
+                } else {
+                  mma16816(d[jt], A0, b00, b01);
+                }
+                mma16816(d[jt], A1, b10, b11);
+              }
+            }
+            if ((j % SPAN) == SPAN - 1) {
+              // group span done: acc += s D - s (128 + z) O for weight rows 2c, 2c + 1 of each tile.
+              // The warp first converts the group's fp16 (scale, zero) of the pass's rows once
+              // (two rows per lane) into fp32 (s, -s (128 + z)) pairs.
+              const int gl = ((ks * kDecStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
+              __syncwarp();
+#pragma unroll
+              for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
+                const int row = lane + 32 * rr;
+                if (row < 8 * NT) {
+                  const float sv = half_bits_to_float(sc[row * p.wg + gl]);
+                  const float zv = half_bits_to_float(zr[row * p.wg + gl]);
+                  smw[row] = make_float2(sv, -sv * (128.0f + zv));
+                }
+              }
+              __syncwarp();
+#pragma unroll
+              for (int jt = 0; jt < NT; ++jt) {
+                const float4 m4 = *reinterpret_cast<const float4*>(&smw[8 * jt + 2 * c]);
+                acc[jt][0] = fmaf(m4.x, d[jt][0], fmaf(m4.y, o[0], acc[jt][0]));
+                acc[jt][1] = fmaf(m4.z, d[jt][1], fmaf(m4.w, o[1], acc[jt][1]));
+                if (TBIG) {
+                  acc[jt][2 % C::kAcc] = fmaf(m4.x, d[jt][2], fmaf(m4.y, o[2], acc[jt][2 % C::kAcc]));
+                  acc[jt][3 % C::kAcc] = fmaf(m4.z, d[jt][3], fmaf(m4.w, o[3], acc[jt][3 % C::kAcc]));
+                }
+              }
+            }
+          }
+        }
+        // every value read from this stage has been consumed above
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tl.empty[s]);
+      }
+
+      // fixed-order reduction of the consumer warps' sums for this pass
+#pragma unroll
+      for (int jt = 0; jt < NT; ++jt) {
+        {
+          const int r0 = 8 * jt + 2 * c;
+          if (g < T) {
+            red[(warp * kDecPassRows + r0) * C::kTokPad + g] = acc[jt][0];
+            red[(warp * kDecPassRows + r0 + 1) * C::kTokPad + g] = acc[jt][1];
+          }
+          if (TBIG && g + 8 < T) {
+            red[(warp * kDecPassRows + r0) * C::kTokPad + g + 8] = acc[jt][2 % C::kAcc];
+            red[(warp * kDecPassRows + r0 + 1) * C::kTokPad + g + 8] = acc[jt][3 % C::kAcc];
+          }
+        }
+      }
+      named_bar_sync(1, C::kWarps * 32);
+      const int row0 = row_base + pass * kDecPassRows;
+      for (int e = threadIdx.x; e < T * h; e += C::kWarps * 32) {
+        const int t = e / h;
+        const int r = e - t * h;
+        float v = 0.0f;
+#pragma unroll
+        for (int w = 0; w < C::kWarps; ++w) v += red[(w * kDecPassRows + r) * C::kTokPad + t];
+        if (KS == 1) {
+          if (row0 + r < p.N) {
+            const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+            out[static_cast<size_t>(t) * p.N + row0 + r] = *reinterpret_cast<const uint16_t*>(&hv);
+          }
+        } else {
+          tl.part[r][t] = v;
+        }
+      }
+      named_bar_sync(1, C::kWarps * 32);  // red is rewritten by the next pass
+    }
+  }
+
+  if (KS == 2) {
+    // one pass per CTA when K is split: rank 0 adds rank 1's partial sums in a fixed order
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    if (rank == 0 && warp < C::kWarps && passes_here > 0) {
+      const int h = rows_here;
+      const float* peer = cluster.map_shared_rank(&tl.part[0][0], 1);
+      for (int e = threadIdx.x; e < p.T * h; e += C::kWarps * 32) {
+        const int t = e / h;
+        const int r = e - t * h;
+        const float v = tl.part[r][t] + peer[r * 16 + t];
+        const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+        out[static_cast<size_t>(t) * p.N + row_base + r] = *reinterpret_cast<const uint16_t*>(&hv);
+      }
+    }
+    cluster.sync();  // rank 1 keeps its shared memory until rank 0 has read it
+  }
+}
+
+const char* dec_name(bool tbig, int span, int ks, int nt) {
+  // "w4a16_dec_kernel<T<=8,g>=128,nt7>", "...,ksplit2,nt7>"; built once, kept for the process
+  static char names[2][3][2][9][64];
+  static const bool filled = [] {
+    const char* gs[3] = {"g>=128", "g=64", "g=32"};
+    for (int a = 0; a < 2; ++a)
+      for (int b = 0; b < 3; ++b)
+        for (int c = 0; c < 2; ++c)
+          for (int d = 1; d <= 8; ++d)
+            snprintf(names[a][b][c][d], sizeof(names[a][b][c][d]), "w4a16_dec_kernel<T<=%d,%s%s,nt%d>", a ? 16 : 8,
+                     gs[b], c ? ",ksplit2" : "", d);
+    return true;
+  }();
+  (void)filled;
+  return names[tbig ? 1 : 0][span == 4 ? 0 : (span == 2 ? 1 : 2)][ks - 1][nt];
+}
+
+template <bool TBIG, int SPAN, int KS, int NT>
+cudaError_t launch_dec(const CUtensorMap (&maps)[7], const DecParams& p, int grid, int smem, uint16_t* out,
+                       cudaStream_t stream) {
+  auto kern = w4a16_dec_kernel<TBIG, SPAN, KS, NT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(DecCfg<TBIG>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LaunchScope scope(stream, dec_name(TBIG, SPAN, KS, NT));
+  e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p, out);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// g >= 128 (the common case) has a kernel per tile count; g = 32, 64 run eight tiles
+template <bool TBIG, int SPAN, int KS>
+cudaError_t launch_dec_nt(int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid, int smem,
+                          uint16_t* out, cudaStream_t stream) {
+  if constexpr (SPAN == 4) {
+    switch (nt) {
+      case 1: return launch_dec<TBIG, SPAN, KS, 1>(maps, p, grid, smem, out, stream);
+      case 2: return launch_dec<TBIG, SPAN, KS, 2>(maps, p, grid, smem, out, stream);
+      case 3: return launch_dec<TBIG, SPAN, KS, 3>(maps, p, grid, smem, out, stream);
+      case 4: return launch_dec<TBIG, SPAN, KS, 4>(maps, p, grid, smem, out, stream);
+      case 5: return launch_dec<TBIG, SPAN, KS, 5>(maps, p, grid, smem, out, stream);
+      case 6: return launch_dec<TBIG, SPAN, KS, 6>(maps, p, grid, smem, out, stream);
+      case 7: return launch_dec<TBIG, SPAN, KS, 7>(maps, p, grid, smem, out, stream);
+      default: return launch_dec<TBIG, SPAN, KS, 8>(maps, p, grid, smem, out, stream);
+    }
+  } else {
+    (void)nt;
+    return launch_dec<TBIG, SPAN, KS, 8>(maps, p, grid, smem, out, stream);
+  }
+}
+
+template <bool TBIG>
+cudaError_t launch_dec_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
+                            int smem, uint16_t* out, cudaStream_t stream) {
+  if (ks == 2) {
+    if (span == 4) return launch_dec_nt<TBIG, 4, 2>(nt, maps, p, grid, smem, out, stream);
+    if (span == 2) return launch_dec_nt<TBIG, 2, 2>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<TBIG, 1, 2>(nt, maps, p, grid, smem, out, stream);
+  }
+  if (span == 4) return launch_dec_nt<TBIG, 4, 1>(nt, maps, p, grid, smem, out, stream);
+  if (span == 2) return launch_dec_nt<TBIG, 2, 1>(nt, maps, p, grid, smem, out, stream);
+  return launch_dec_nt<TBIG, 1, 1>(nt, maps, p, grid, smem, out, stream);
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+}  // namespace
+
+// Returns cudaErrorNotSupported (nothing launched) when the shape does not fit
+// this kernel's tensor maps: the scale/zero row stride must be a multiple of 16
+// bytes (K/g a multiple of 8) and the scale/zero arrays 16-byte aligned.
+cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
+                             cudaStream_t stream) {
+  if (T < 1 || T > 16 || N < 1 || K < 128 || K % 128 != 0 || group_size < 32) return cudaErrorNotSupported;
+  const int G = K / group_size;
+  if (G % 8 != 0 || (reinterpret_cast<uintptr_t>(scale16) & 15u) || (reinterpret_cast<uintptr_t>(zero16) & 15u))
+    return cudaErrorNotSupported;
+  int dev = 0, num_sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+
+  DecParams p = {};
+  p.N = N;
+  p.K = K;
+  p.T = T;
+  p.n_stages = (K + kDecStageK - 1) / kDecStageK;
+  int gs = 0;
+  while ((1 << gs) < group_size) ++gs;
+  p.group_shift = gs;
+  p.wg = group_size == 32 ? 16 : 8;
+
+  // rows per CTA (multiple of 8) with one CTA per SM; a cluster pair splits K
+  // instead when that halves the rows a CTA streams (small N)
+  const int units = (N + 7) / 8;
+  const int rows1 = 8 * ((units + num_sms - 1) / num_sms);
+  const int rows2 = 8 * ((2 * units + num_sms - 1) / num_sms);
+  int ks = 1, rows = rows1;
+  if (p.n_stages >= 2 && rows2 <= kDecPassRows && 2 * rows1 > rows2 + 4) {
+    ks = 2;
+    rows = rows2;
+  }
+  p.rows_per_cta = rows;
+  p.passes = (rows + kDecPassRows - 1) / kDecPassRows;
+  p.last_rows = rows - (p.passes - 1) * kDecPassRows;
+  const int grid = ks * ((N + rows - 1) / rows);
+
+  const bool tbig = T > 8;
+  const int red_bytes = tbig ? DecCfg<true>::kRedBytes : DecCfg<false>::kRedBytes;
+  p.act_off = 2 * kDecCodeBox;
+  p.tab_off = p.act_off + round_up(2 * 512 * T, 128);
+  p.stage_bytes = round_up(p.tab_off + 2 * 2 * p.wg * kDecPassRows, 1024);
+  const int fixed = red_bytes + static_cast<int>(sizeof(DecTail)) + 1024;
+  p.S = std::min(kDecMaxStages, (kDecSmemLimit - fixed) / p.stage_bytes);
+  const int groups = tbig ? DecCfg<true>::kGroups : DecCfg<false>::kGroups;
+  if (p.S < groups + 1) return cudaErrorNotSupported;
+  const int smem = dec_tail_offset(p.S, p.stage_bytes, red_bytes) + static_cast<int>(sizeof(DecTail)) + 1024;
+
+  CUtensorMap maps[7];
+  const int heights[2] = {std::min(kDecPassRows, rows), p.last_rows};
+  for (int m = 0; m < 2; ++m) {
+    e = make_tmap_2d(&maps[m], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(K / 8), 32, static_cast<uint32_t>(heights[m]), CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d(&maps[2 + m], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scale16, static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(G), static_cast<uint32_t>(p.wg), static_cast<uint32_t>(heights[m]),
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d(&maps[4 + m], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, zero16, static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(G), static_cast<uint32_t>(p.wg), static_cast<uint32_t>(heights[m]),
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+  }
+  e = make_tmap_2d(&maps[6], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, static_cast<uint64_t>(T), static_cast<uint64_t>(K),
+                   256, static_cast<uint32_t>(T), CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (e != cudaSuccess) return e;
+
+  const int span = group_size >= 128 ? 4 : group_size / 32;
+  const int nt = p.passes == 1 ? rows / 8 : 8;  // tiles of a full pass
+  return tbig ? launch_dec_span<true>(span, ks, nt, maps, p, grid, smem, out, stream)
+              : launch_dec_span<false>(span, ks, nt, maps, p, grid, smem, out, stream);
+}
+
+}  // namespace ar

@@ -377,6 +377,55 @@ def test_w4a16_matches_oracle(ar, T, N, K, g):
     assert rel_l2(got, ref) <= W4A16_RTOL
 
 
+@pytest.mark.parametrize("T", [1, 5, 8, 9, 16])
+@pytest.mark.parametrize("N,K,g,tag", [
+    (1000, 1280, 32, "g=32,nt8>"),              # N not a multiple of 8; last 512-k stage half empty
+    (10000, 512, 64, "g=64,nt8>"),              # 72 rows per CTA: two row passes (64 + 8); last CTA one pass
+    (10000, 1024, 128, "g>=128,nt8>"),          # the same passes with one group per 128-k chunk
+    (4096, 2048, 128, "g>=128,ksplit2,nt7>"),   # 56-row CTA pairs splitting K
+    (296, 4096, 256, "g>=128,ksplit2,nt1>"),    # 8-row CTA pairs
+])
+def test_w4a16_decode_row_ranges_match_oracle(ar, T, N, K, g, tag):
+    """T <= 16 on the decode kernel that gives each SM a contiguous range of weight rows."""
+    d = synth.make_linear(N, K, 1, seed=T + N)
+    V, a, b = synth.make_state(N, K, g, seed=2, spread=True)
+    packed, s16, z16 = _packed(ar, d["W"], V, a, b, g)
+    A = synth.make_activations(T, K, seed=T)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_w4a16_gemm(bf16_dev(A), packed, s16, z16, g, out)
+    kern = ar.ar_last_kernels()
+    assert "w4a16_dec_kernel<T<=%d,%s" % (8 if T <= 8 else 16, tag) in kern, kern
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 4, g)
+    words, s_ref, z_ref = O.pack_int4(st["q"], st["s"], st["zp"])
+    ref = O.w4a16_matmul(synth.bf16_bits_to_f32(A), words, s_ref, z_ref, g)
+    got = out.float().cpu().numpy()
+    assert rel_l2(got, ref) <= W4A16_RTOL
+    # each token on its own, and the first and last rows (the ends of the row ranges)
+    for t in range(T):
+        assert rel_l2(got[t], ref[t]) <= W4A16_RTOL
+    assert rel_l2(got[:, :8], ref[:, :8]) <= W4A16_RTOL and rel_l2(got[:, -8:], ref[:, -8:]) <= W4A16_RTOL
+    # on the device's own codes, scales and zeros only the bf16 rounding of the output remains
+    own = O.w4a16_matmul(synth.bf16_bits_to_f32(A), packed.cpu().numpy().view(np.uint32),
+                         s16.cpu().numpy().view(np.uint16), z16.cpu().numpy().view(np.uint16), g)
+    assert rel_l2(got, own) <= W4A16_TC_RTOL
+
+
+def test_w4a16_decode_falls_back_when_scale_rows_are_not_16_byte_multiples(ar):
+    """K/g = 2 groups per row: the scale/zero rows cannot be TMA boxes, the older decode kernel runs."""
+    N, K, g, T = 40, 2048, 1024, 3
+    d = synth.make_linear(N, K, 1, seed=9)
+    V, a, b = synth.make_state(N, K, g, seed=2, spread=True)
+    packed, s16, z16 = _packed(ar, d["W"], V, a, b, g)
+    A = synth.make_activations(T, K, seed=4)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_w4a16_gemm(bf16_dev(A), packed, s16, z16, g, out)
+    assert "w4a16_tma_kernel" in ar.ar_last_kernels()
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 4, g)
+    words, s_ref, z_ref = O.pack_int4(st["q"], st["s"], st["zp"])
+    ref = O.w4a16_matmul(synth.bf16_bits_to_f32(A), words, s_ref, z_ref, g)
+    assert rel_l2(out.float().cpu().numpy(), ref) <= W4A16_RTOL
+
+
 @pytest.mark.parametrize("T", [17, 40, 64, 100, 256])
 @pytest.mark.parametrize("N,K,g", [(320, 1024, 128), (64, 4096, 32), (40, 2048, 1024)])
 def test_w4a16_tensor_core_path_matches_oracle(ar, T, N, K, g):
