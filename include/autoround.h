@@ -229,9 +229,12 @@ AR_API ar_status ar_pack_int4(const uint16_t* W, const float* V, const float* al
  * nearest even of the fp32 accumulation).  (q - zero) is exact in bf16; the
  * products are accumulated in fp32 on the tensor cores, one group (or 32-k
  * slice of a group) at a time, and scaled by the group's scale in fp32.
- * T <= 16 runs a decode kernel (mma.sync fragments built in registers);
- * larger T a tcgen05 GEMM that dequantizes each 128-row x 64-k tile of codes
- * into shared memory.  Results are deterministic for a given T.
+ * T <= 16 runs a decode kernel (mma.sync fragments built in registers, one
+ * range of weight rows per SM; when K/g is not a multiple of 8 or scale/zero
+ * are not 16-byte aligned, an older decode kernel with 64-row tiles); larger
+ * T a tcgen05 GEMM whose dequantization warps write each 128-row tile of
+ * (q - zero) into tensor memory as the MMA's A operand.  Results are
+ * deterministic for a given T.
  * Supported: 1 <= T < 2^31, group_size 32..1024 (power of two) dividing K,
  * K % 128 == 0; anything else returns AR_ERR_UNSUPPORTED or
  * AR_ERR_INVALID_ARG before any launch. */
