@@ -19,7 +19,8 @@ void trace_kernel(const char* name);
 
 // Wraps one kernel launch: traces its name and, while device profiling is on
 // (ar_profile_start), records CUDA events around it on the launch stream.
-// `name` must be a string literal.
+// `name` must have static storage (a string literal or a static table): it is
+// kept after the launch.
 class LaunchScope {
  public:
   LaunchScope(cudaStream_t stream, const char* name);

@@ -583,3 +583,102 @@ def test_wxa16_matmul_against_loops(bits):
                 zz = float(z16.view(np.float16)[n, k // g])
                 acc += float(A[t, k]) * (int(q[n, k]) - zz) * sc
             assert got[t, n] == pytest.approx(acc, rel=1e-12, abs=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# helpers of the quantizer, the loss evaluations and the block-by-block driver
+# ----------------------------------------------------------------------------
+
+def test_group_range_contains_zero_and_the_extremes():
+    """Worked by hand: each group's range is widened to contain 0."""
+    W = np.array([[1.0, 2.0, 3.0, 4.0, -1.0, -2.0, 0.5, 0.0, -3.0, -1.0, -2.0, -0.5]])
+    mx, mn = O.group_range(W, 4)
+    assert mx.tolist() == [[4.0, 0.5, 0.0]]
+    assert mn.tolist() == [[0.0, -2.0, -3.0]]
+
+
+def test_qparams_closed_forms():
+    """s and zp worked by hand from the asymmetric and symmetric definitions."""
+    one = np.ones((1, 1))
+    # [AR] §2: range [0, 8] at 4 bits -> s = 8/15, zp = 0
+    _, _, s, zp, _ = O.qparams(np.array([[8.0]]), np.array([[0.0]]), one, one, 4, dtype=np.float64)
+    assert s[0, 0] == pytest.approx(8 / 15, rel=1e-15) and zp[0, 0] == 0
+    # range [-1.25, 2.5]: s = 3.75/15 = 0.25, zp = 1.25/0.25 = 5
+    _, _, s, zp, _ = O.qparams(np.array([[2.5]]), np.array([[-1.25]]), one, one, 4, dtype=np.float64)
+    assert s[0, 0] == 0.25 and zp[0, 0] == 5
+    # upper clip alpha = 0.5: hi = 1.25, s = 2.5/15 = 1/6, zp = round(7.5) = 8 (half away from zero)
+    hi, lo, s, zp, _ = O.qparams(np.array([[2.5]]), np.array([[-1.25]]), 0.5 * one, one, 4, dtype=np.float64)
+    assert hi[0, 0] == 1.25 and lo[0, 0] == -1.25
+    assert s[0, 0] == pytest.approx(1 / 6, rel=1e-15) and zp[0, 0] == 8
+    # symmetric 4-bit: s = max(hi, -lo)/7, zp = 8
+    _, _, s, zp, _ = O.qparams(np.array([[2.0]]), np.array([[-3.0]]), one, one, 4, symmetric=True, dtype=np.float64)
+    assert s[0, 0] == pytest.approx(3 / 7, rel=1e-15) and zp[0, 0] == 8
+
+
+def test_sign0():
+    x = np.array([-2.0, 0.0, 3.0, -0.0, np.nan, 1e-30], np.float32)
+    assert O.sign0(x).tolist() == [-1.0, 0.0, 1.0, 0.0, 0.0, 1.0]
+
+
+def _grid_weights(rng, n, k, g, s=0.25, zp=5):
+    """Weights on the 4-bit grid with every group spanning codes 0..15 (range [-1.25, 2.5] for s = 0.25,
+    zp = 5): the quantizer reproduces them exactly, and they are exact in bf16."""
+    codes = rng.integers(0, 16, (n, k)).astype(np.float64)
+    codes[:, 0::g] = 0
+    codes[:, 1::g] = 15
+    return (s * (codes - zp)).astype(np.float32)
+
+
+def _bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def test_eval_losses_vanish_on_grid_weights():
+    rng = np.random.default_rng(21)
+    cfg = O.QConfig(bits=4, group_size=16)
+    W = _grid_weights(rng, 24, 32, 16)
+    X = _bf16(rng.standard_normal((8, 32)))
+    G = np.ones((24, 2), np.float32)
+    assert O.eval_loss_linear(W, X, O.reference_forward(X, W), np.zeros_like(W), G, G, cfg) == 0.0
+    H, F = 32, 48
+    Ws = [_grid_weights(rng, F, H, 16), _grid_weights(rng, F, H, 16), _grid_weights(rng, H, F, 16)]
+    states = [(np.zeros(W.shape, np.float32), np.ones((W.shape[0], W.shape[1] // 16), np.float32),
+               np.ones((W.shape[0], W.shape[1] // 16), np.float32)) for W in Ws]
+    X = _bf16(rng.standard_normal((8, H)))
+    Y = O.mlp_reference(X, *Ws)
+    assert O.eval_loss_mlp(Ws, X, Y, states, cfg) == 0.0
+    # gate and up exchanged: a different block, so the loss is no longer 0
+    assert O.eval_loss_mlp([Ws[1], Ws[0], Ws[2]], X, Y, [states[1], states[0], states[2]], cfg) > 0.0
+
+
+def test_tune_blocks_mlp_chains_blocks_and_follows_the_schedule():
+    rng = np.random.default_rng(22)
+    cfg = O.QConfig(bits=4, group_size=16)
+    S, L, H, F = 5, 3, 32, 48
+    X0 = _bf16(rng.standard_normal((S, L, H)))
+    schedule = np.array([[4, 1], [0, 2], [3, 4]], np.int32)
+    # two blocks on the grid: every step's loss is 0, nothing moves, and each block passes on
+    # bf16(its reference output) to the next
+    grid = [[_grid_weights(rng, F, H, 16), _grid_weights(rng, F, H, 16), _grid_weights(rng, H, F, 16)]
+            for _ in range(2)]
+    res = O.tune_blocks_mlp(grid, X0, cfg, schedule)
+    x1 = _bf16(O.mlp_reference(X0.reshape(-1, H), *grid[0])).reshape(S, L, H)
+    x2 = _bf16(O.mlp_reference(x1.reshape(-1, H), *grid[1])).reshape(S, L, H)
+    assert np.array_equal(res[0]["x_out"], x1) and np.array_equal(res[1]["x_out"], x2)
+    for r in res:
+        assert not r["losses"].any()
+        for V, a, b in r["states"]:
+            assert not V.any() and (a == 1).all() and (b == 1).all()
+    # off-grid weights: the first step's loss is the initial state's loss on exactly the samples of
+    # the schedule's first row (their tokens in row order), measured against the reference outputs
+    Ws = [_bf16(rng.standard_normal((F, H)) * 0.1), _bf16(rng.standard_normal((F, H)) * 0.1),
+          _bf16(rng.standard_normal((H, F)) * 0.1)]
+    res = O.tune_blocks_mlp([Ws], X0, cfg, schedule)
+    init = [(np.zeros(W.shape, np.float32), np.ones((W.shape[0], W.shape[1] // 16), np.float32),
+             np.ones((W.shape[0], W.shape[1] // 16), np.float32)) for W in Ws]
+    Y = O.mlp_reference(X0.reshape(-1, H), *Ws).reshape(S, L, H)
+    rows = schedule[0]
+    expect = O.eval_loss_mlp(Ws, X0[rows].reshape(-1, H), Y[rows].reshape(-1, H), init, cfg)
+    assert res[0]["losses"][0] == pytest.approx(expect, rel=1e-12)
+    other = O.eval_loss_mlp(Ws, X0[[0, 1]].reshape(-1, H), Y[[0, 1]].reshape(-1, H), init, cfg)
+    assert other != pytest.approx(expect, rel=1e-6)
