@@ -611,3 +611,135 @@ def tune_blocks_mlp(blocks, X0, cfg: QConfig, schedule):
         out.append({"states": states, "losses": np.asarray(losses, f64), "x_out": X})
     return out
 
+
+
+# ----------------------------------------------------------------------------
+# NVFP4 fake quantization: a QDQ function for a new data type ([AR] §4 "Why the
+# Tuning Stage Must Take the QDQ Path", point 3: a new type needs only a
+# tensor-level QDQ function)
+# ----------------------------------------------------------------------------
+#
+# Format: [QC] §2 table ("FP4 E2M1: 1 sign + 2 exponent + 1 mantissa", "FP8
+# E4M3: 1 sign + 4 exponent + 3 mantissa"); [NQ] "量化" (note.yj-dis.top),
+# section "低比特浮点：FP8 与 NVFP4", table row NVFP4: E2M1 values, one FP8
+# scale per micro-block of 16 values, plus a per-tensor scale; [QC] §5 table
+# row "NVFP4 recipe" (E2M1, 16-element block scale and global scale).
+#
+# Readings (the pages give the layout of the values, not the recipe):
+# * exponent bias 2^(e-1) - 1 (1 for E2M1, 7 for E4M3), subnormals at exponent
+#   field 0; E4M3 has no infinities (its all-ones code is NaN), so its largest
+#   finite value is 448; E2M1's is 6;
+# * both conversions round to nearest, ties to the even code, and saturate at
+#   the largest finite value;
+# * global scale S = amax(|W|) / (6 * 448), so the largest block scale, as a
+#   multiple of S, fits E4M3;
+# * AutoRound's variables act as in the integer quantizer: the learnable clip
+#   factor alpha multiplies each block's range (E2M1 is symmetric, so there is
+#   no separate lower bound), V is added to W / s before rounding; block scale
+#   s = E4M3(alpha * amax_block / 6 / S) * S;
+# * every step in fp32 (the codes are decided in the kernel's precision), in
+#   the order written in ``nvfp4_qdq``; a block whose scale rounds to 0 gives 0.
+
+NVFP4_BLOCK = 16
+E2M1_MAX = 6.0
+E4M3_MAX = 448.0
+
+
+def _minifloat_values(e_bits: int, m_bits: int, nan_codes=()):
+    """Value of every code of a sign/exponent/mantissa format with bias 2^(e-1) - 1 and subnormals."""
+    bias = 2 ** (e_bits - 1) - 1
+    vals = []
+    for code in range(2 ** (1 + e_bits + m_bits)):
+        sgn = -1.0 if code >> (e_bits + m_bits) else 1.0
+        e = (code >> m_bits) & (2 ** e_bits - 1)
+        m = code & (2 ** m_bits - 1)
+        if code in nan_codes:
+            vals.append(np.nan)
+        elif e == 0:
+            vals.append(sgn * (m / 2 ** m_bits) * 2.0 ** (1 - bias))
+        else:
+            vals.append(sgn * (1 + m / 2 ** m_bits) * 2.0 ** (e - bias))
+    return np.array(vals, f64)
+
+
+def e2m1_values() -> np.ndarray:
+    """The 16 E2M1 codes' values (code = sign << 3 | exponent << 1 | mantissa)."""
+    return _minifloat_values(2, 1)
+
+
+def e4m3_values() -> np.ndarray:
+    """The 256 E4M3 codes' values; 0x7F and 0xFF are NaN."""
+    return _minifloat_values(4, 3, nan_codes=(0x7F, 0xFF))
+
+
+def _round_to_codes(x, values, vmax):
+    """Nearest finite code to each x (ties to the even code, i.e. mantissa bit 0), saturating at +-vmax.
+    Returns the codes (as int) of the non-negative magnitudes with the sign bit of x."""
+    x = np.asarray(x, f64)
+    n = values.size // 2
+    mags = values[:n]                      # codes 0 .. n-1: the non-negative values, increasing
+    fin = np.isfinite(mags)
+    a = np.minimum(np.abs(x), vmax)
+    d = np.abs(a[..., None] - np.where(fin, mags, np.inf)[None, :])
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best
+    # among equally near codes take the even one (codes are consecutive, so at most two tie)
+    even = cand & ((np.arange(n) % 2) == 0)[None, :]
+    pick = np.where(even.any(axis=-1), even.argmax(axis=-1), cand.argmax(axis=-1))
+    return np.where(np.signbit(x), pick + n, pick).astype(np.int64)
+
+
+def e2m1_round(x):
+    """(code, value) of round-to-nearest-even E2M1 with saturation at +-6."""
+    vals = e2m1_values()
+    code = _round_to_codes(x, vals, E2M1_MAX)
+    return code, vals[code]
+
+
+def e4m3_round(x):
+    """(code, value) of round-to-nearest-even E4M3 with saturation at +-448 (no NaN produced)."""
+    vals = e4m3_values()
+    code = _round_to_codes(x, vals, E4M3_MAX)
+    return code, vals[code]
+
+
+def nvfp4_qdq(W, V=None, alpha=None):
+    """NVFP4 fake quantization of W [N][K] (K a multiple of 16) in fp32.
+
+    amax_t = max |W|; S = amax_t / 2688; per block b of 16 along K:
+    s_b = E4M3((alpha_b * amax_b) / 6 / S) * S; codes q = E2M1(W / s_b + V),
+    Ŵ = q * s_b (0 where s_b = 0).  V [N][K] defaults to 0, alpha [N][K/16]
+    to 1.  Returns codes (uint8 0..15), scale codes (uint8, E4M3), S, the
+    effective block scales, Ŵ (fp32) and Ŵ rounded to bf16.
+    """
+    W = np.asarray(W, f32)
+    N, K = W.shape
+    assert K % NVFP4_BLOCK == 0
+    nb = K // NVFP4_BLOCK
+    V = np.zeros_like(W) if V is None else np.asarray(V, f32)
+    alpha = np.ones((N, nb), f32) if alpha is None else np.asarray(alpha, f32)
+    amax_t = f32(np.max(np.abs(W))) if W.size else f32(0)
+    S = f32(amax_t / f32(E2M1_MAX * E4M3_MAX))
+    Wb = W.reshape(N, nb, NVFP4_BLOCK)
+    amax_b = np.max(np.abs(Wb), axis=-1).astype(f32)
+    sb_raw = ((alpha * amax_b).astype(f32) / f32(E2M1_MAX)).astype(f32)
+    if S > 0:
+        ratio = (sb_raw / S).astype(f32)
+    else:
+        ratio = np.zeros_like(sb_raw)
+    scode, s8 = e4m3_round(ratio)
+    s_eff = (s8.astype(f32) * S).astype(f32)
+    se = np.repeat(s_eff, NVFP4_BLOCK, axis=1).reshape(N, K)
+    live = se > 0
+    x = np.where(live, (W / np.where(live, se, f32(1))).astype(f32) + V, f32(0)).astype(f32)
+    qcode, qval = e2m1_round(x)
+    qcode = np.where(live, qcode, 0)
+    What = np.where(live, (qval.astype(f32) * se).astype(f32), f32(0)).astype(f32)
+    return {"codes": qcode.astype(np.uint8), "scale_codes": scode.astype(np.uint8), "S": S, "s": s_eff,
+            "What": What, "What_bf16": bf16_rne(What)}
+
+
+def pack_fp4(codes: np.ndarray) -> np.ndarray:
+    """Two E2M1 codes per byte along K, element k in the low nibble when k is even: uint8 [N][K/2]."""
+    c = np.asarray(codes).astype(np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)

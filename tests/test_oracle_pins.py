@@ -682,3 +682,104 @@ def test_tune_blocks_mlp_chains_blocks_and_follows_the_schedule():
     assert res[0]["losses"][0] == pytest.approx(expect, rel=1e-12)
     other = O.eval_loss_mlp(Ws, X0[[0, 1]].reshape(-1, H), Y[[0, 1]].reshape(-1, H), init, cfg)
     assert other != pytest.approx(expect, rel=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# NVFP4 QDQ: E2M1 / E4M3 from their bit layouts, the block scales, the packing
+# ----------------------------------------------------------------------------
+
+def test_e2m1_values_from_the_1_2_1_layout():
+    v = O.e2m1_values()
+    assert v[:8].tolist() == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert (v[8:] == -v[:8]).all() and np.signbit(v[8])
+
+
+def test_e2m1_rounding_ties_saturation_and_midpoints():
+    # ties between neighbours go to the even code (mantissa bit 0)
+    x = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 100.0, -0.75, -5.0])
+    assert O.e2m1_round(x)[1].tolist() == [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 6.0, 6.0, -1.0, -4.0]
+    # away from ties: the nearest value, found here by comparing with the midpoints between neighbours
+    rng = np.random.default_rng(30)
+    x = rng.uniform(-7, 7, 20000)
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    mids = (mags[1:] + mags[:-1]) / 2
+    ref = np.sign(x) * mags[np.searchsorted(mids, np.abs(x))]
+    assert np.array_equal(O.e2m1_round(x)[1], ref)
+
+
+def test_e4m3_rounding_matches_torch_float8_cast():
+    rng = np.random.default_rng(31)
+    x = np.concatenate([rng.uniform(-448, 448, 20000), rng.standard_normal(20000) * 2.0 ** rng.integers(-12, 8, 20000),
+                        # exact ties between neighbouring codes (subnormal and normal range)
+                        (np.arange(1, 200) + 0.5) * 2.0 ** -9, (np.arange(8, 16) + 0.5) * 2.0 ** 4])
+    x = x.astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float32).numpy()
+    code, val = O.e4m3_round(x)
+    assert np.array_equal(val.astype(np.float32), ref)
+    assert np.array_equal(code.astype(np.uint8), torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+    assert O.e4m3_round(np.array([1000.0, -1e9]))[1].tolist() == [448.0, -448.0]  # saturates
+
+
+def test_nvfp4_grid_weights_reconstruct_exactly():
+    """Blocks built as E2M1 values times power-of-two scales that E4M3 holds exactly, with the tensor
+    maximum 2.625 so that S = 2.625 / 2688 = 2^-10: the QDQ returns them unchanged."""
+    rng = np.random.default_rng(32)
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    N, K = 6, 64
+    sb = 2.0 ** -rng.integers(2, 12, (N, K // 16)).astype(np.float64)
+    sb[0, 0] = 0.4375                           # 2.625 / 6: the tensor's largest block, ratio 448
+    q = rng.choice(mags, (N, K)) * np.where(rng.random((N, K)) < 0.5, -1, 1)
+    q[:, 0::16] = 6.0                           # each block's largest magnitude is 6 * s_b
+    W = (q * np.repeat(sb, 16, axis=1)).astype(np.float32)
+    o = O.nvfp4_qdq(W)
+    assert o["S"] == np.float32(2.0 ** -10)
+    assert np.array_equal(o["s"], sb.astype(np.float32))
+    assert np.array_equal(o["What"], W)
+
+
+def test_nvfp4_is_the_nearest_point_of_each_block_grid():
+    rng = np.random.default_rng(33)
+    W = (rng.standard_normal((8, 96)) * np.exp(rng.standard_normal((8, 1)))).astype(np.float32)
+    o = O.nvfp4_qdq(W)
+    grid = np.concatenate([-O.e2m1_values()[:8][::-1], O.e2m1_values()[:8]])
+    se = np.repeat(o["s"], 16, axis=1).astype(np.float64)
+    err = np.abs(W - o["What"])
+    best = np.min(np.abs(W[..., None] - grid[None, None, :] * se[..., None]), axis=-1)
+    assert np.allclose(err, best, rtol=0, atol=1e-6 * np.abs(W).max())
+    # the block scale is E4M3 of (amax_b / 6) / S times S: within E4M3's relative spacing of amax_b / 6
+    amax_b = np.abs(W.reshape(8, 6, 16)).max(-1)
+    assert np.all(np.abs(o["s"] - amax_b / 6) <= amax_b / 6 * 2.0 ** -4 + 2.0 ** -9 * o["S"])
+
+
+def test_nvfp4_power_of_two_scaling_commutes():
+    rng = np.random.default_rng(34)
+    W = (rng.standard_normal((4, 64)) * 0.05).astype(np.float32)
+    V = rng.uniform(-0.5, 0.5, W.shape).astype(np.float32)
+    a = rng.uniform(0.5, 1.0, (4, 4)).astype(np.float32)
+    o1 = O.nvfp4_qdq(W, V, a)
+    o2 = O.nvfp4_qdq(W * np.float32(8.0), V, a)
+    assert np.array_equal(o1["codes"], o2["codes"]) and np.array_equal(o1["scale_codes"], o2["scale_codes"])
+    assert np.array_equal(o1["What"] * np.float32(8.0), o2["What"])
+
+
+def test_nvfp4_offsets_and_clip_factor_act_as_in_the_integer_quantizer():
+    """V = +-0.5 moves a value that sits on a grid point by at most one E2M1 step; alpha = 0.5 halves the
+    block's scale (before the E4M3 rounding) so that the block maximum saturates at 6 * s_b."""
+    W = np.zeros((1, 16), np.float32)
+    W[0, :8] = [6.0, 2.0, 1.0, 0.5, 0.0, -1.0, -3.0, 4.0]
+    up = O.nvfp4_qdq(W, np.full_like(W, 0.49))
+    dn = O.nvfp4_qdq(W, np.full_like(W, -0.49))
+    base = O.nvfp4_qdq(W)
+    s = base["s"][0, 0]
+    assert np.array_equal(base["What"], W * (s / s))  # on the grid
+    steps = np.diff(np.concatenate([-O.e2m1_values()[:8][::-1], O.e2m1_values()[1:8]]))
+    assert np.all(up["What"] >= base["What"]) and np.all(dn["What"] <= base["What"])
+    assert np.max(up["What"] - base["What"]) <= steps.max() * s
+    half = O.nvfp4_qdq(W, alpha=np.full((1, 1), 0.5, np.float32))
+    assert half["s"][0, 0] == pytest.approx(s / 2, rel=2 ** -3)
+    assert half["What"][0, 0] == 6.0 * half["s"][0, 0]
+
+
+def test_pack_fp4_places_each_code_by_hand():
+    codes = np.array([[1, 2, 3, 4, 15, 0, 8, 7]], np.uint8)
+    assert O.pack_fp4(codes).tolist() == [[0x21, 0x43, 0x0F, 0x78]]
