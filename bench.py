@@ -310,6 +310,51 @@ def w4a16_bench(ar, torch, peaks, reps=20):
     return out
 
 
+def nvfp4_bench(ar, torch, peaks, reps=20):
+    """NVFP4 QDQ (E2M1 codes, E4M3 scale per 16 values, per-tensor scale) of the 4096² and 8192x28672
+    layers with offsets V and clip factors alpha; outputs Ŵ, packed codes and scale codes.  L2 flushed
+    before each launch.  HBM bytes per weight: W 2 + V 4 + Ŵ 2 + codes 0.5, plus 4 + 1 per 16 (alpha,
+    scale code); the absmax pass reads W once more (2 B per weight)."""
+    out = {}
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.int32, device="cuda")
+    for name, (N, K) in (("linear_4096", (4096, 4096)), ("down_8192_28672", (8192, 28672))):
+        d = synth.make_linear(N, K, 1, seed=3, x_outlier_channels=0)
+        W = to_dev_bf16(d["W"], torch)
+        del d
+        V = (torch.rand((N, K), device="cuda") - 0.5).float()
+        a = (torch.rand((N, K // 16), device="cuda") * 0.5 + 0.5).float()
+        amax = torch.empty(1, dtype=torch.float32, device="cuda")
+        gs = torch.empty(1, dtype=torch.float32, device="cuda")
+        What = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((N, K // 16), dtype=torch.uint8, device="cuda")
+        ar.ar_absmax_bf16(W, amax)
+        for _ in range(3):
+            ar.ar_qdq_nvfp4(W, V, a, amax, What, codes, scales, gs)
+        res, kern = {}, {}
+        for what, fn in (("qdq", lambda: ar.ar_qdq_nvfp4(W, V, a, amax, What, codes, scales, gs)),
+                         ("absmax", lambda: ar.ar_absmax_bf16(W, amax))):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for e0, e1 in ev:
+                flush.sum()
+                e0.record()
+                fn()
+                e1.record()
+            torch.cuda.synchronize()
+            res[what] = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+            kern[what] = ar.ar_last_kernels()
+        n = N * K
+        qbytes = n * (2 + 4 + 2 + 0.5) + (n // 16) * (4 + 1)
+        out[name] = {"qdq_us": res["qdq"] * 1e3, "qdq_GB/s": qbytes / (res["qdq"] * 1e-3) / 1e9,
+                     "qdq_frac_hbm": qbytes / (res["qdq"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "absmax_us": res["absmax"] * 1e3,
+                     "absmax_frac_hbm": 2.0 * n / (res["absmax"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": qbytes, "kernels": kern}
+        del W, V, a, What, codes, scales
+    out["format"] = "NVFP4: E2M1 codes, E4M3 scale per 16 values, fp32 tensor scale amax/2688; V and alpha applied"
+    return out
+
+
 # ----------------------------------------------------------------------------
 # multi-rank plumbing (independent layers per rank; timing only crosses ranks)
 # ----------------------------------------------------------------------------
@@ -438,6 +483,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w4a16", action="store_true")
+    ap.add_argument("--no-nvfp4", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads (MLP, low-bit, 70B down)")
     args = ap.parse_args()
@@ -570,6 +616,8 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_w4a16:
         result["w4a16"] = w4a16_bench(ar, torch, peaks)
+    if rank == 0 and world == 1 and not args.no_nvfp4:
+        result["nvfp4_qdq"] = nvfp4_bench(ar, torch, peaks)
     if rank == 0 and world == 1 and not args.no_extra:
         del W, X, V, alpha, beta, Y, ws
         torch.cuda.empty_cache()

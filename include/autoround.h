@@ -268,6 +268,41 @@ AR_API ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* pac
                                const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, int bits,
                                uint16_t* out, ar_stream_t stream);
 
+/* Absolute maximum of n bf16 values: *amax = max_i |x[i]| (device fp32
+ * scalar, written; exact, as it is one of the inputs).  The per-tensor
+ * statistic of ar_qdq_nvfp4.  Needs n > 0, n % 8 == 0, x 16-byte aligned,
+ * amax 4-byte aligned; otherwise AR_ERR_INVALID_ARG before any launch.  A NaN
+ * or Inf input raises AR_ERR_NONFINITE in the device status
+ * (ar_get_device_status); *amax is then not meaningful. */
+AR_API ar_status ar_absmax_bf16(const uint16_t* x, int64_t n, float* amax, ar_stream_t stream);
+
+/* NVFP4 fake quantization: a QDQ function for a new data type ([AR] §4 "Why
+ * the Tuning Stage Must Take the QDQ Path", point 3).  Format: E2M1 values (1
+ * sign, 2 exponent, 1 mantissa bits; largest 6) with one E4M3 scale (largest
+ * finite 448) per block of 16 values and a per-tensor scale ([QC] "量化：从
+ * Scale 到 W4A8 的完整坐标" §2 table and §5 row "NVFP4 recipe"; [NQ] "量化",
+ * section "低比特浮点：FP8 与 NVFP4").  In fp32, in this order:
+ *   S = amax / 2688                         (2688 = 6 * 448; amax = max |W|)
+ *   per block b of 16 consecutive values along K:
+ *     s_b = E4M3((alpha_b * max_b |W|) / 6 / S) * S
+ *     q = E2M1(W / s_b + V),  W_hat = q * s_b     (q = 0, W_hat = 0 if s_b = 0)
+ * E4M3 and E2M1 round to nearest, ties to even, and saturate.
+ *   W      bf16 [N][K], K % 16 == 0, 16-byte aligned
+ *   V      fp32 [N][K] offsets, or NULL (0); 16-byte aligned
+ *   alpha  fp32 [N][K/16] clip factors, or NULL (1)
+ *   amax   device fp32 scalar, max |W| (ar_absmax_bf16 of W)
+ * Outputs, each optional (at least one):
+ *   W_hat         bf16 [N][K], round to nearest even; 16-byte aligned
+ *   codes         uint8 [N][K/2]: two E2M1 codes per byte along K, element k
+ *                 in the low nibble when k is even; 16-byte aligned
+ *   scales        uint8 [N][K/16]: the E4M3 codes of s_b / S
+ *   global_scale  device fp32 scalar S
+ * All device memory is the caller's.  Invalid shapes, pointers or alignment
+ * return AR_ERR_INVALID_ARG before any launch. */
+AR_API ar_status ar_qdq_nvfp4(const uint16_t* W, const float* V, const float* alpha, int64_t N, int64_t K,
+                              const float* amax, uint16_t* W_hat, uint8_t* codes, uint8_t* scales,
+                              float* global_scale, ar_stream_t stream);
+
 /* Minibatch assembly for block-by-block tuning ([AR] §8 preset table: each
  * iteration works on a batch of 8 -- 4 in the "fast" preset -- of the 128
  * calibration samples; [AR] §3 "Algorithm Flow" steps 3-6 iterate on such

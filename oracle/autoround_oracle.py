@@ -703,14 +703,15 @@ def e4m3_round(x):
     return code, vals[code]
 
 
-def nvfp4_qdq(W, V=None, alpha=None):
+def nvfp4_qdq(W, V=None, alpha=None, amax=None):
     """NVFP4 fake quantization of W [N][K] (K a multiple of 16) in fp32.
 
     amax_t = max |W|; S = amax_t / 2688; per block b of 16 along K:
     s_b = E4M3((alpha_b * amax_b) / 6 / S) * S; codes q = E2M1(W / s_b + V),
     Ŵ = q * s_b (0 where s_b = 0).  V [N][K] defaults to 0, alpha [N][K/16]
-    to 1.  Returns codes (uint8 0..15), scale codes (uint8, E4M3), S, the
-    effective block scales, Ŵ (fp32) and Ŵ rounded to bf16.
+    to 1.  ``amax`` is max |W| of the whole tensor when W holds only some of its
+    rows (default: W's own).  Returns codes (uint8 0..15), scale codes (uint8,
+    E4M3), S, the effective block scales, Ŵ (fp32) and Ŵ rounded to bf16.
     """
     W = np.asarray(W, f32)
     N, K = W.shape
@@ -718,7 +719,7 @@ def nvfp4_qdq(W, V=None, alpha=None):
     nb = K // NVFP4_BLOCK
     V = np.zeros_like(W) if V is None else np.asarray(V, f32)
     alpha = np.ones((N, nb), f32) if alpha is None else np.asarray(alpha, f32)
-    amax_t = f32(np.max(np.abs(W))) if W.size else f32(0)
+    amax_t = f32(amax) if amax is not None else (f32(np.max(np.abs(W))) if W.size else f32(0))
     S = f32(amax_t / f32(E2M1_MAX * E4M3_MAX))
     Wb = W.reshape(N, nb, NVFP4_BLOCK)
     amax_b = np.max(np.abs(Wb), axis=-1).astype(f32)

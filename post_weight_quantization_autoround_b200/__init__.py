@@ -22,6 +22,7 @@ __all__ = [
     "ar_last_error", "ar_last_kernels", "ar_version", "ar_profile_start", "ar_profile_stop", "AR_BLOCK_LINEAR",
     "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES", "AR_BLOCK_SWIGLU_MLP", "ar_block_forward",
     "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace", "ar_debug_wait_timeout",
+    "ar_absmax_bf16", "ar_qdq_nvfp4",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -87,6 +88,8 @@ _SIGNATURES = {
     "ar_gather_samples": (_INT, [_P, _I64, _I64, ctypes.POINTER(ctypes.c_int32), _INT, _P, _P]),
     "ar_pack_codes": (_INT, [_P, _P, _P, _P, _I64, _I64, ctypes.POINTER(QConfig), _P, _P, _P, _P]),
     "ar_wxa16_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P]),
+    "ar_absmax_bf16": (_INT, [_P, _I64, _P, _P]),
+    "ar_qdq_nvfp4": (_INT, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -289,6 +292,20 @@ def ar_gather_samples(src, idx, dst, stream=None) -> None:
     if dst.shape[0] != len(idx) or dst[0].numel() * dst.element_size() != sample_bytes:
         raise ARError(AR_ERR_INVALID_ARG, "dst must hold len(idx) samples of src's size")
     _check(lib().ar_gather_samples(_ptr(src), n_src, sample_bytes, arr, len(idx), _ptr(dst), _stream(stream)))
+
+
+def ar_absmax_bf16(x, amax, stream=None) -> None:
+    """amax (fp32 device scalar) = max |x| over a bf16 device tensor."""
+    _check(lib().ar_absmax_bf16(_ptr(x), x.numel(), _ptr(amax), _stream(stream)))
+
+
+def ar_qdq_nvfp4(W, V, alpha, amax, W_hat=None, codes=None, scales=None, global_scale=None, stream=None) -> None:
+    """NVFP4 fake quantization of W [N][K] (bf16): V [N][K] fp32 or None, alpha [N][K/16] fp32 or None,
+    amax fp32 device scalar (``ar_absmax_bf16`` of W); outputs W_hat bf16 [N][K], codes uint8 [N][K/2],
+    scales uint8 [N][K/16] (E4M3 codes), global_scale fp32 scalar."""
+    N, K = W.shape
+    _check(lib().ar_qdq_nvfp4(_ptr(W), _ptr(V), _ptr(alpha), N, K, _ptr(amax), _ptr(W_hat), _ptr(codes),
+                              _ptr(scales), _ptr(global_scale), _stream(stream)))
 
 
 def ar_gemm_bf16(A, a_mn_major: bool, B, b_mn_major: bool, D, M: int, N: int, K: int, stream=None) -> None:

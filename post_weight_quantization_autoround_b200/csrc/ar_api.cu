@@ -650,6 +650,37 @@ ar_status ar_gather_samples(const void* src, int64_t n_src_samples, int64_t samp
   return end_call();
 }
 
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+ar_status ar_absmax_bf16(const uint16_t* x, int64_t n, float* amax, ar_stream_t stream) {
+  begin_call();
+  if (!x || !amax) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  if (n <= 0 || n % 8 != 0) return fail(AR_ERR_INVALID_ARG, "n must be a positive multiple of 8");
+  if (!aligned16(x) || !aligned4(amax)) return fail(AR_ERR_INVALID_ARG, "x must be 16-byte and amax 4-byte aligned");
+  cudaError_t e = launch_absmax_bf16(x, n, amax, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "absmax launch");
+  return end_call();
+}
+
+ar_status ar_qdq_nvfp4(const uint16_t* W, const float* V, const float* alpha, int64_t N, int64_t K, const float* amax,
+                       uint16_t* W_hat, uint8_t* codes, uint8_t* scales, float* global_scale, ar_stream_t stream) {
+  begin_call();
+  if (N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "N, K must be positive");
+  if (K % 16 != 0) return fail(AR_ERR_INVALID_ARG, "K=%lld is not a multiple of the 16-value block", (long long)K);
+  if (N > INT64_MAX / K) return fail(AR_ERR_INVALID_ARG, "N*K overflows");
+  if (!W || !amax) return fail(AR_ERR_INVALID_ARG, "NULL input pointer");
+  if (!W_hat && !codes && !scales && !global_scale) return fail(AR_ERR_INVALID_ARG, "no output requested");
+  const void* a16[] = {W, V, W_hat, codes};
+  for (const void* p : a16)
+    if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "W, V, W_hat and codes must be 16-byte aligned");
+  if ((alpha && !aligned4(alpha)) || !aligned4(amax) || (global_scale && !aligned4(global_scale)))
+    return fail(AR_ERR_INVALID_ARG, "alpha, amax and global_scale must be 4-byte aligned");
+  cudaError_t e = launch_qdq_nvfp4(W, V, alpha, N * K, amax, W_hat, codes, scales, global_scale,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qdq_nvfp4 launch");
+  return end_call();
+}
+
 ar_status ar_gemm_bf16(const uint16_t* A, int a_mn_major, const uint16_t* B, int b_mn_major, float* D, int64_t M,
                        int64_t N, int64_t K, ar_stream_t stream) {
   begin_call();

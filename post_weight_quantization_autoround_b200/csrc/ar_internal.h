@@ -122,6 +122,11 @@ cudaError_t launch_w4a16(const uint16_t* A, int T, const uint32_t* packed, const
 cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                              const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
                              cudaStream_t stream);
+// NVFP4 QDQ (ar_nvfp4.cu): absmax into a zeroed device scalar, then the block QDQ
+cudaError_t launch_absmax_bf16(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream);
+cudaError_t launch_qdq_nvfp4(const uint16_t* W, const float* V, const float* alpha, int64_t n, const float* amax,
+                             uint16_t* W_hat, uint8_t* codes, uint8_t* scales, float* global_scale,
+                             cudaStream_t stream);
 // minibatch assembly (ar_gather.cu): n <= kMaxGatherSamples samples of sample_bytes each
 constexpr int kMaxGatherSamples = 64;
 cudaError_t launch_gather_samples(const void* src, int64_t sample_bytes, const int32_t* idx, int n, void* dst,

@@ -160,3 +160,19 @@ def test_pack_codes_and_wxa16_validation():
     assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 192, 64, 8, FAKE, None) == ar.AR_ERR_INVALID_ARG  # K % 128
     assert w(FAKE, 0, FAKE, FAKE, FAKE, 64, 256, 128, 2, FAKE, None) == ar.AR_ERR_INVALID_ARG
 
+
+
+def test_absmax_and_qdq_nvfp4_validation():
+    am = ar.lib().ar_absmax_bf16
+    assert am(FAKE, 12, FAKE, None) == ar.AR_ERR_INVALID_ARG          # n % 8
+    assert am(FAKE, 0, FAKE, None) == ar.AR_ERR_INVALID_ARG
+    assert am(FAKE + 8, 16, FAKE, None) == ar.AR_ERR_INVALID_ARG      # x misaligned
+    assert am(FAKE, 16, None, None) == ar.AR_ERR_INVALID_ARG
+    q = ar.lib().ar_qdq_nvfp4
+    assert q(FAKE, None, None, 4, 40, FAKE, FAKE, None, None, None, None) == ar.AR_ERR_INVALID_ARG   # K % 16
+    assert q(FAKE, None, None, 0, 64, FAKE, FAKE, None, None, None, None) == ar.AR_ERR_INVALID_ARG
+    assert q(FAKE, None, None, 4, 64, FAKE, None, None, None, None, None) == ar.AR_ERR_INVALID_ARG  # no output
+    assert q(FAKE, None, None, 4, 64, None, FAKE, None, None, None, None) == ar.AR_ERR_INVALID_ARG  # no amax
+    assert q(FAKE, FAKE + 4, None, 4, 64, FAKE, FAKE, None, None, None, None) == ar.AR_ERR_INVALID_ARG  # V misaligned
+    assert q(FAKE, None, FAKE + 2, 4, 64, FAKE, FAKE, None, None, None, None) == ar.AR_ERR_INVALID_ARG  # alpha
+    assert q(FAKE, None, None, 4, 64, FAKE, None, FAKE + 8, None, None, None) == ar.AR_ERR_INVALID_ARG  # codes
