@@ -48,7 +48,7 @@ typedef struct CUstream_st* ar_stream_t; /* same handle as cudaStream_t */
 typedef enum {
   AR_OK = 0,
   AR_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape */
-  AR_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  AR_ERR_UNSUPPORTED = 2, /* valid request the library does not implement */
   AR_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
   AR_ERR_NONFINITE = 4,   /* device status: NaN/Inf seen in an input or gradient */
   AR_ERR_TIMEOUT = 5,     /* device status: a pipeline wait gave up */

@@ -20,9 +20,11 @@ and fp64 matrix products.  Sources (page title, then section):
   q = clip(round(x/s)), x̂ = s·q; asymmetric adds a zero-point).
 * [IA] "Intel AutoRound 高级量化" (hotdry blog), section on the sign-gradient
   mechanism: rounding is treated as the identity in the backward pass (STE).
+* [QC] §2 table (E2M1 and E4M3 layouts) and §5 table row "NVFP4 recipe";
+  [NQ] "量化" (note.yj-dis.top), section "低比特浮点：FP8 与 NVFP4": the
+  NVFP4 QDQ function at the end of this module.
 
-Readings where the pages are silent or disagree (all stated once more in
-DESIGN.md):
+Readings where the pages are silent or disagree:
 
 * The group range always contains 0: mx = max(0, max W), mn = min(0, min W).
   [AR] §2 needs this: "no clipping" on [0.1, 0.2, 0.15, 8.0] gives scale 8/15.
