@@ -739,6 +739,7 @@ def nvfp4_qdq(W, V=None, alpha=None, amax=None):
     qcode = np.where(live, qcode, 0)
     What = np.where(live, (qval.astype(f32) * se).astype(f32), f32(0)).astype(f32)
     return {"codes": qcode.astype(np.uint8), "scale_codes": scode.astype(np.uint8), "S": S, "s": s_eff,
+            "x": x, "q": np.where(live, qval, 0.0).astype(f32), "amax_b": amax_b,
             "What": What, "What_bf16": bf16_rne(What)}
 
 
@@ -746,3 +747,66 @@ def pack_fp4(codes: np.ndarray) -> np.ndarray:
     """Two E2M1 codes per byte along K, element k in the low nibble when k is even: uint8 [N][K/2]."""
     c = np.asarray(codes).astype(np.uint8)
     return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+# ----------------------------------------------------------------------------
+# one tuning step on NVFP4: the integer step with the NVFP4 QDQ function in
+# its place ([AR] §4 "Why the Tuning Stage Must Take the QDQ Path", point 3;
+# [AR] §3 "Algorithm Flow" steps 3-5 and "SignSGD")
+# ----------------------------------------------------------------------------
+#
+# Straight-through backward as in the integer quantizer: both roundings (E4M3
+# of the block scale, E2M1 of the codes) count as the identity, the saturation
+# at +-6 passes the gradient where |W/s + V| <= 6 (inclusive), and the products
+# use the forward's values:
+#     dV_i     = g_i s_b m_i
+#     dalpha_b = (amax_b / 6) sum_i g_i (q_i - m_i W_i / s_b)
+# (s_b = alpha_b amax_b / 6 up to the E4M3 rounding, so ds_b/dalpha_b =
+# amax_b / 6); a block whose scale is 0 gets no gradient.
+
+def nvfp4_qdq_smooth(W, V, alpha):
+    """``nvfp4_qdq`` in fp64 with both roundings replaced by the identity (the saturation kept):
+    s_b = alpha_b amax_b / 6, x = W / s_b + V, q = clip(x, -6, 6), Ŵ = q s_b.  Its exact gradient is
+    what ``nvfp4_ste_fold`` computes, so finite differences can check the fold."""
+    W = np.asarray(W, f64)
+    N, K = W.shape
+    nb = K // NVFP4_BLOCK
+    amax_b = np.abs(W.reshape(N, nb, NVFP4_BLOCK)).max(-1)
+    s = np.asarray(alpha, f64) * amax_b / E2M1_MAX
+    se = np.repeat(s, NVFP4_BLOCK, axis=1)
+    live = se > 0
+    x = np.where(live, W / np.where(live, se, 1.0) + np.asarray(V, f64), 0.0)
+    q = np.clip(x, -E2M1_MAX, E2M1_MAX)
+    return {"s": s, "x": x, "q": q, "amax_b": amax_b, "What": q * se}
+
+
+def nvfp4_ste_fold(gW, W, st):
+    """(dV [N][K], dalpha [N][K/16]) in fp64 from dL/dŴ and the forward's values."""
+    N, K = gW.shape
+    nb = K // NVFP4_BLOCK
+    g = np.asarray(gW, f64).reshape(N, nb, NVFP4_BLOCK)
+    Wd = np.asarray(W, f64).reshape(N, nb, NVFP4_BLOCK)
+    s = np.asarray(st["s"], f64)[:, :, None]
+    x = np.asarray(st["x"], f64).reshape(N, nb, NVFP4_BLOCK)
+    q = np.asarray(st["q"], f64).reshape(N, nb, NVFP4_BLOCK)
+    live = np.broadcast_to(s > 0, g.shape)
+    m = live & (np.abs(x) <= E2M1_MAX)
+    sd = np.where(live, s, 1.0)
+    dV = np.where(m, g * s, 0.0)
+    c = np.where(live, g * (q - np.where(m, Wd / sd, 0.0)), 0.0)
+    dalpha = (np.asarray(st["amax_b"], f64) / E2M1_MAX) * c.sum(-1)
+    return dV.reshape(N, K), dalpha
+
+
+def nvfp4_tune_step_linear(Wb, Xb, Y, V, alpha, cfg: QConfig, amax=None, count: int | None = None):
+    """One SignSGD step of one linear layer on NVFP4 (the state is V [N][K] and alpha [N][K/16];
+    ``cfg`` gives lr and the bounds).  Returns (loss, (V', alpha'), grads, qdq dict)."""
+    M, N = Xb.shape[0], Wb.shape[0]
+    count = M * N if count is None else count
+    st = nvfp4_qdq(Wb, V, alpha, amax)
+    fw = forward_loss(Xb, st["What_bf16"], Y, count)
+    gW = weight_grad(fw["G"], Xb)
+    dV, da = nvfp4_ste_fold(gW, Wb, st)
+    V1 = signsgd(V, dV, cfg.lr, cfg.v_min, cfg.v_max)
+    a1 = signsgd(alpha, da, cfg.lr, cfg.clip_min, cfg.clip_max)
+    return fw["loss"], (V1, a1), {"gW": gW, "dV": dV.astype(f32), "dalpha": da.astype(f32), "G": fw["G"]}, st

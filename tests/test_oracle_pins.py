@@ -783,3 +783,70 @@ def test_nvfp4_offsets_and_clip_factor_act_as_in_the_integer_quantizer():
 def test_pack_fp4_places_each_code_by_hand():
     codes = np.array([[1, 2, 3, 4, 15, 0, 8, 7]], np.uint8)
     assert O.pack_fp4(codes).tolist() == [[0x21, 0x43, 0x0F, 0x78]]
+
+
+def _nvfp4_smooth_loss(W, X, Y, V, a):
+    st = O.nvfp4_qdq_smooth(W, V, a)
+    return O.forward_loss(X, st["What"], Y, X.shape[0] * W.shape[0], dtype=np.float64)
+
+
+def test_nvfp4_ste_gradients_match_finite_differences():
+    """On the smooth surrogate (E4M3 and E2M1 as the identity, saturation kept) the STE fold is the exact
+    gradient; alpha < 1 saturates each block's largest values, so both branches of the mask occur."""
+    rng = np.random.default_rng(40)
+    N, K, M = 3, 48, 6
+    W = rng.standard_normal((N, K))
+    X = rng.standard_normal((M, K))
+    Y = X @ W.T + 0.1 * rng.standard_normal((M, N))
+    V = rng.uniform(-0.4, 0.4, (N, K))
+    a = rng.uniform(0.6, 0.9, (N, K // 16))
+    fw = _nvfp4_smooth_loss(W, X, Y, V, a)
+    st = O.nvfp4_qdq_smooth(W, V, a)
+    m = np.abs(st["x"]) <= 6
+    assert 0 < m.mean() < 1
+    dV, da = O.nvfp4_ste_fold(O.weight_grad(fw["G"], X, dtype=np.float64), W, st)
+    h = 1e-7
+
+    def f(V_, a_):
+        return _nvfp4_smooth_loss(W, X, Y, V_, a_)["loss"]
+
+    for (n, k) in [(0, 0), (0, 7), (1, 20), (2, 47), (1, 33)] + list(zip(*np.nonzero(~m)))[:3]:
+        Vp, Vm = V.copy(), V.copy()
+        Vp[n, k] += h
+        Vm[n, k] -= h
+        assert dV[n, k] == pytest.approx((f(Vp, a) - f(Vm, a)) / (2 * h), rel=1e-5, abs=1e-12)
+    for n in range(N):
+        for j in range(K // 16):
+            ap, am = a.copy(), a.copy()
+            ap[n, j] += h
+            am[n, j] -= h
+            assert da[n, j] == pytest.approx((f(V, ap) - f(V, am)) / (2 * h), rel=1e-5, abs=1e-12)
+    assert (dV[~m] == 0).all()
+
+
+def test_nvfp4_tuning_step_on_grid_weights_and_exact_moves():
+    rng = np.random.default_rng(41)
+    cfg = O.QConfig(lr=0.005)
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    N, K, M = 4, 64, 8
+    q = rng.choice(mags, (N, K)) * np.where(rng.random((N, K)) < 0.5, -1, 1)
+    q[:, 0::16] = 6.0
+    sb = 2.0 ** -rng.integers(2, 8, (N, K // 16)).astype(np.float64)
+    sb[0, 0] = 0.4375  # the tensor maximum 2.625: S = 2^-10, every block scale exact in E4M3
+    W = (q * np.repeat(sb, 16, axis=1)).astype(np.float32)
+    X = _bf16(rng.standard_normal((M, K)))
+    Y = O.reference_forward(X, W)
+    V0 = np.zeros((N, K), np.float32)
+    a0 = np.ones((N, K // 16), np.float32)
+    L, (V1, a1), gr, _ = O.nvfp4_tune_step_linear(W, X, Y, V0, a0, cfg)
+    assert L == 0.0 and not gr["dV"].any() and not gr["dalpha"].any()
+    assert np.array_equal(V1, V0) and np.array_equal(a1, a0)
+    # off the grid: every parameter moves by exactly one lr step (or stays), within its bounds
+    Wn = _bf16(rng.standard_normal((N, K)) * 0.05)
+    Yn = O.reference_forward(X, Wn)
+    L, (V1, a1), gr, _ = O.nvfp4_tune_step_linear(Wn, X, Yn, V0, a0, cfg)
+    assert L > 0
+    dv = (V1 - V0).astype(np.float64)
+    assert np.all(np.isin(np.round(np.abs(dv) / 0.005, 6), [0.0, 1.0]))
+    assert np.array_equal(np.sign(dv), -np.sign(gr["dV"]).astype(np.float64))
+    assert np.all((a1 <= 1.0) & (a1 >= 0.5))
