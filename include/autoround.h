@@ -303,6 +303,33 @@ AR_API ar_status ar_qdq_nvfp4(const uint16_t* W, const float* V, const float* al
                               const float* amax, uint16_t* W_hat, uint8_t* codes, uint8_t* scales,
                               float* global_scale, ar_stream_t stream);
 
+/* Tuning steps of one linear layer on NVFP4: the SignSGD step of ar_tune_step
+ * ([AR] §3 "Algorithm Flow" steps 3-5, "SignSGD") with ar_qdq_nvfp4 as its QDQ
+ * function ([AR] §4 "Why the Tuning Stage Must Take the QDQ Path", point 3).
+ * Per step: W_hat = NVFP4 QDQ of W (V, alpha); Y_hat = X W_hat^T; loss = mean
+ * (Y_hat - Y)^2; G = bf16(2 (Y_hat - Y) / (M N)); dW_hat = G^T X; straight-
+ * through fold with both roundings (E4M3, E2M1) as the identity and the
+ * gradient passed where |W/s_b + V| <= 6:
+ *   dV = dW_hat s_b m,   dalpha_b = (amax_b / 6) sum_block dW_hat (q - m W / s_b)
+ * then V <- clamp(V - lr sign(dV), v_min, v_max), alpha <- clamp(alpha -
+ * lr sign(dalpha), clip_min, clip_max) (cfg's lr and bounds; bits, group_size
+ * and symmetric are not used).
+ *   W      bf16 [N][K] (K % 16 == 0, N % 8 == 0)
+ *   V      fp32 [N][K], alpha fp32 [N][K/16]: the state, updated in place
+ *   amax   device fp32 scalar, max |W| (ar_absmax_bf16)
+ *   X      bf16 [M][K] (M % 8 == 0), Y fp32 [M][N] the reference output
+ *   loss_per_step  device fp32 [max(n_steps, 1)]: each step's loss before its
+ *                  update (n_steps = 0: the loss of the current state only)
+ *   dV_out [N][K], dalpha_out [N][K/16]: optional, the last step's gradients
+ *   workspace      device, 256-byte aligned, ar_tune_step_nvfp4_workspace bytes
+ * Errors: AR_ERR_INVALID_ARG / AR_ERR_UNSUPPORTED / AR_ERR_WORKSPACE before any
+ * launch. */
+AR_API size_t ar_tune_step_nvfp4_workspace(int64_t M, int64_t N, int64_t K, int n_steps);
+AR_API ar_status ar_tune_step_nvfp4(const uint16_t* W, float* V, float* alpha, int64_t N, int64_t K, const float* amax,
+                                    const uint16_t* X, int64_t M, const float* Y, const ar_qconfig* cfg, int n_steps,
+                                    float* loss_per_step, float* dV_out, float* dalpha_out, void* workspace,
+                                    size_t workspace_bytes, ar_stream_t stream);
+
 /* Minibatch assembly for block-by-block tuning ([AR] §8 preset table: each
  * iteration works on a batch of 8 -- 4 in the "fast" preset -- of the 128
  * calibration samples; [AR] §3 "Algorithm Flow" steps 3-6 iterate on such

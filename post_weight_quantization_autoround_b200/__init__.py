@@ -22,7 +22,7 @@ __all__ = [
     "ar_last_error", "ar_last_kernels", "ar_version", "ar_profile_start", "ar_profile_stop", "AR_BLOCK_LINEAR",
     "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES", "AR_BLOCK_SWIGLU_MLP", "ar_block_forward",
     "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace", "ar_debug_wait_timeout",
-    "ar_absmax_bf16", "ar_qdq_nvfp4",
+    "ar_absmax_bf16", "ar_qdq_nvfp4", "ar_tune_step_nvfp4_workspace", "ar_tune_step_nvfp4",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -90,6 +90,9 @@ _SIGNATURES = {
     "ar_wxa16_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P]),
     "ar_absmax_bf16": (_INT, [_P, _I64, _P, _P]),
     "ar_qdq_nvfp4": (_INT, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P]),
+    "ar_tune_step_nvfp4_workspace": (ctypes.c_size_t, [_I64, _I64, _I64, _INT]),
+    "ar_tune_step_nvfp4": (_INT, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, ctypes.POINTER(QConfig), _INT, _P, _P, _P,
+                                  _P, ctypes.c_size_t, _P]),
 }
 
 
@@ -306,6 +309,25 @@ def ar_qdq_nvfp4(W, V, alpha, amax, W_hat=None, codes=None, scales=None, global_
     N, K = W.shape
     _check(lib().ar_qdq_nvfp4(_ptr(W), _ptr(V), _ptr(alpha), N, K, _ptr(amax), _ptr(W_hat), _ptr(codes),
                               _ptr(scales), _ptr(global_scale), _stream(stream)))
+
+
+def ar_tune_step_nvfp4_workspace(M: int, N: int, K: int, n_steps: int) -> int:
+    n = lib().ar_tune_step_nvfp4_workspace(M, N, K, n_steps)
+    if n == 0:
+        raise ARError(AR_ERR_INVALID_ARG, ar_last_error())
+    return n
+
+
+def ar_tune_step_nvfp4(W, V, alpha, amax, X, Y, cfg: QConfig, n_steps: int, loss_per_step, workspace,
+                       dV=None, dalpha=None, stream=None) -> None:
+    """``n_steps`` SignSGD steps of one linear layer on NVFP4 (V [N][K], alpha [N][K/16] updated in place);
+    loss_per_step: fp32 device [max(n_steps, 1)]; workspace: uint8 device tensor of
+    ``ar_tune_step_nvfp4_workspace`` bytes."""
+    N, K = W.shape
+    M = X.shape[0]
+    _check(lib().ar_tune_step_nvfp4(_ptr(W), _ptr(V), _ptr(alpha), N, K, _ptr(amax), _ptr(X), M, _ptr(Y),
+                                    ctypes.byref(cfg), n_steps, _ptr(loss_per_step), _ptr(dV), _ptr(dalpha),
+                                    _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def ar_gemm_bf16(A, a_mn_major: bool, B, b_mn_major: bool, D, M: int, N: int, K: int, stream=None) -> None:

@@ -681,6 +681,92 @@ ar_status ar_qdq_nvfp4(const uint16_t* W, const float* V, const float* alpha, in
   return end_call();
 }
 
+struct Nvfp4Ws {
+  size_t what, g, dw, partial, total;
+  int partials_per_step;
+};
+
+Nvfp4Ws nvfp4_ws(int64_t M, int64_t N, int64_t K, int n_steps) {
+  Nvfp4Ws w{};
+  size_t off = 0;
+  w.what = off;
+  off = align_up(off + static_cast<size_t>(N * K) * 2, 256);
+  w.g = off;
+  off = align_up(off + static_cast<size_t>(M * N) * 2, 256);
+  w.dw = off;
+  off = align_up(off + static_cast<size_t>(N * K) * 4, 256);
+  w.partials_per_step = resid_partials(static_cast<int>(M), static_cast<int>(N));
+  w.partial = off;
+  off = align_up(off + static_cast<size_t>(w.partials_per_step) * (n_steps > 0 ? n_steps : 1) * 8, 256);
+  w.total = off;
+  return w;
+}
+
+ar_status check_nvfp4_step(int64_t N, int64_t K, int64_t M, int n_steps) {
+  if (N <= 0 || K <= 0 || M <= 0) return fail(AR_ERR_INVALID_ARG, "sizes must be positive");
+  if (K % 16 != 0) return fail(AR_ERR_INVALID_ARG, "K=%lld is not a multiple of the 16-value block", (long long)K);
+  if (N % 8 != 0 || M % 8 != 0) return fail(AR_ERR_INVALID_ARG, "N and M must be multiples of 8");
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  if (n_steps < 0) return fail(AR_ERR_INVALID_ARG, "n_steps must be >= 0");
+  return AR_OK;
+}
+
+size_t ar_tune_step_nvfp4_workspace(int64_t M, int64_t N, int64_t K, int n_steps) {
+  begin_call();
+  if (check_nvfp4_step(N, K, M, n_steps) != AR_OK) return 0;
+  return nvfp4_ws(M, N, K, n_steps).total;
+}
+
+ar_status ar_tune_step_nvfp4(const uint16_t* W, float* V, float* alpha, int64_t N, int64_t K, const float* amax,
+                             const uint16_t* X, int64_t M, const float* Y, const ar_qconfig* cfg, int n_steps,
+                             float* loss_per_step, float* dV_out, float* dalpha_out, void* workspace,
+                             size_t workspace_bytes, ar_stream_t stream) {
+  begin_call();
+  ar_status st = check_cfg(cfg);
+  if (st != AR_OK) return st;
+  st = check_nvfp4_step(N, K, M, n_steps);
+  if (st != AR_OK) return st;
+  if (!W || !V || !alpha || !amax || !X || !Y || !loss_per_step) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  const void* a16[] = {W, V, alpha, X, Y, dV_out};
+  for (const void* p : a16)
+    if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "W, V, alpha, X, Y and dV_out must be 16-byte aligned");
+  if (!aligned4(amax) || !aligned4(loss_per_step) || (dalpha_out && !aligned4(dalpha_out)))
+    return fail(AR_ERR_INVALID_ARG, "amax, loss_per_step and dalpha_out must be 4-byte aligned");
+  const Nvfp4Ws w = nvfp4_ws(M, N, K, n_steps);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* W_hat = reinterpret_cast<uint16_t*>(ws + w.what);
+  uint16_t* G = reinterpret_cast<uint16_t*>(ws + w.g);
+  float* dW = reinterpret_cast<float*>(ws + w.dw);
+  double* partial = reinterpret_cast<double*>(ws + w.partial);
+  const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
+  const float gscale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(N)));
+  const int steps = n_steps > 0 ? n_steps : 1;
+  cudaError_t e;
+  for (int step = 0; step < steps; ++step) {
+    e = launch_qdq_nvfp4(W, V, alpha, N * K, amax, W_hat, nullptr, nullptr, nullptr, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qdq_nvfp4 launch");
+    e = launch_gemm_resid(X, W_hat, Y, G, gscale, partial + static_cast<size_t>(step) * w.partials_per_step, Mi, Ni,
+                          Ki, s);
+    if (e != cudaSuccess) return cuda_fail(e, "forward GEMM launch");
+    if (n_steps == 0) break;
+    // dL/dW_hat [N][K] = G^T X: both operands as stored, MN-major, reduced over the M tokens
+    e = launch_gemm_plain(G, true, X, true, dW, Ni, Ki, Mi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "weight-gradient GEMM launch");
+    const bool last = step == steps - 1;
+    e = launch_fold_nvfp4(dW, W, V, alpha, N * K, amax, cfg->lr, cfg->v_min, cfg->v_max, cfg->clip_min,
+                          cfg->clip_max, last ? dV_out : nullptr, last ? dalpha_out : nullptr, s);
+    if (e != cudaSuccess) return cuda_fail(e, "fold_nvfp4 launch");
+  }
+  e = launch_loss_reduce(partial, w.partials_per_step, steps, 1.0 / (static_cast<double>(M) * static_cast<double>(N)),
+                         loss_per_step, s);
+  if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
+  return end_call();
+}
+
 ar_status ar_gemm_bf16(const uint16_t* A, int a_mn_major, const uint16_t* B, int b_mn_major, float* D, int64_t M,
                        int64_t N, int64_t K, ar_stream_t stream) {
   begin_call();

@@ -127,6 +127,10 @@ cudaError_t launch_absmax_bf16(const uint16_t* x, int64_t n, float* amax, cudaSt
 cudaError_t launch_qdq_nvfp4(const uint16_t* W, const float* V, const float* alpha, int64_t n, const float* amax,
                              uint16_t* W_hat, uint8_t* codes, uint8_t* scales, float* global_scale,
                              cudaStream_t stream);
+// ... and the straight-through fold + SignSGD update of one NVFP4 tuning step from dL/dW_hat
+cudaError_t launch_fold_nvfp4(const float* dW, const uint16_t* W, float* V, float* alpha, int64_t n, const float* amax,
+                              float lr, float v_min, float v_max, float c_min, float c_max, float* dV_out,
+                              float* da_out, cudaStream_t stream);
 // minibatch assembly (ar_gather.cu): n <= kMaxGatherSamples samples of sample_bytes each
 constexpr int kMaxGatherSamples = 64;
 cudaError_t launch_gather_samples(const void* src, int64_t sample_bytes, const int32_t* idx, int n, void* dst,

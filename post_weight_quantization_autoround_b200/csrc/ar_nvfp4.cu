@@ -130,6 +130,95 @@ __global__ void __launch_bounds__(256) qdq_nvfp4_kernel(const uint16_t* __restri
   }
 }
 
+// Backward and update of one tuning step on NVFP4, from dL/dŴ (fp32 [N][K], the
+// weight-gradient GEMM's output).  The forward's values are recomputed exactly
+// as qdq_nvfp4_kernel computes them; the straight-through fold counts both
+// roundings as the identity and passes the gradient where |W/s + V| <= 6:
+//   dV_i = g_i s_b m_i,   dalpha_b = (amax_b / 6) sum_i g_i (q_i - m_i W_i / s_b)
+// then V <- clamp(V - lr sign(dV)), alpha <- clamp(alpha - lr sign(dalpha))
+// ([AR] §3 "SignSGD"; sign(0) = 0, a NaN gradient counts as 0 and raises the
+// non-finite status).  Same lane layout as the QDQ: the two lanes of a block add
+// their halves of the block sum with one shuffle (a + b on both lanes).
+__device__ __forceinline__ float sign0f(float d) { return d > 0.f ? 1.f : (d < 0.f ? -1.f : 0.f); }
+
+__global__ void __launch_bounds__(256) fold_nvfp4_kernel(const float* __restrict__ dW, const uint16_t* __restrict__ W,
+                                                         float* __restrict__ V, float* __restrict__ alpha, int64_t n,
+                                                         const unsigned int* __restrict__ amax_bits, float lr,
+                                                         float v_min, float v_max, float c_min, float c_max,
+                                                         float* __restrict__ dV_out, float* __restrict__ da_out) {
+  const float S = __fdiv_rn(__uint_as_float(*amax_bits), kE2M1xE4M3Max);
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t base = warp * 512; base < n; base += warps * 512) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int64_t e0 = base + c * 256 + 8 * lane;
+      const bool live = e0 < n;
+      uint4 w = make_uint4(0, 0, 0, 0);
+      float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0, g0 = v0, g1 = v0;
+      float a = 1.0f;
+      const int64_t blk = e0 / kNvBlock;
+      if (live) {
+        w = __ldcs(reinterpret_cast<const uint4*>(W + e0));
+        v0 = __ldcs(reinterpret_cast<const float4*>(V + e0));
+        v1 = __ldcs(reinterpret_cast<const float4*>(V + e0 + 4));
+        g0 = __ldcs(reinterpret_cast<const float4*>(dW + e0));
+        g1 = __ldcs(reinterpret_cast<const float4*>(dW + e0 + 4));
+        a = alpha[blk];
+      }
+      uint32_t m = max_mag8(w);
+      m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      const float amax_b = __uint_as_float(m << 16);
+      const float sb = __fdiv_rn(__fmul_rn(a, amax_b), kE2M1Max);
+      const float ratio = S > 0.0f ? __fdiv_rn(sb, S) : 0.0f;
+      const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(ratio, __NV_SATFINITE, __NV_E4M3);
+      const float s_eff = __fmul_rn(__half2float(__half(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3))), S);
+      const float x[8] = {bf16_lo_f(w.x), bf16_hi_f(w.x), bf16_lo_f(w.y), bf16_hi_f(w.y),
+                          bf16_lo_f(w.z), bf16_hi_f(w.z), bf16_lo_f(w.w), bf16_hi_f(w.w)};
+      const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      float dv[8];
+      float csum = 0.0f;
+      bool bad = false;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        dv[i] = 0.0f;
+        if (s_eff > 0.0f) {
+          const float ws = __fdiv_rn(x[i], s_eff);
+          const float t = __fadd_rn(ws, v[i]);
+          const uint32_t q = static_cast<uint32_t>(__nv_cvt_float_to_fp4(t, __NV_E2M1, cudaRoundNearest)) & 0xFu;
+          const float qf = __half2float(__half(__nv_cvt_fp4_to_halfraw(static_cast<__nv_fp4_storage_t>(q), __NV_E2M1)));
+          const bool mi = fabsf(t) <= kE2M1Max;
+          dv[i] = mi ? __fmul_rn(g[i], s_eff) : 0.0f;
+          csum = __fadd_rn(csum, __fmul_rn(g[i], __fsub_rn(qf, mi ? ws : 0.0f)));
+        }
+        bad |= !(fabsf(g[i]) <= 3.0e38f);
+      }
+      // the block sum: this lane's half plus its partner's (the same sum on both lanes)
+      const float other = __shfl_xor_sync(0xFFFFFFFFu, csum, 1);
+      const float cblk = (lane & 1) ? __fadd_rn(other, csum) : __fadd_rn(csum, other);
+      if (!live) continue;
+      if (bad) raise_status(kStatusNonFinite);
+      const float da = __fmul_rn(__fdiv_rn(amax_b, kE2M1Max), cblk);
+      float vo[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        vo[i] = fminf(fmaxf(__fsub_rn(v[i], lr * sign0f(dv[i])), v_min), v_max);
+      __stcs(reinterpret_cast<float4*>(V + e0), make_float4(vo[0], vo[1], vo[2], vo[3]));
+      __stcs(reinterpret_cast<float4*>(V + e0 + 4), make_float4(vo[4], vo[5], vo[6], vo[7]));
+      if (dV_out) {
+        __stcs(reinterpret_cast<float4*>(dV_out + e0), make_float4(dv[0], dv[1], dv[2], dv[3]));
+        __stcs(reinterpret_cast<float4*>(dV_out + e0 + 4), make_float4(dv[4], dv[5], dv[6], dv[7]));
+      }
+      if ((lane & 1) == 0) {
+        alpha[blk] = fminf(fmaxf(__fsub_rn(a, lr * sign0f(da)), c_min), c_max);
+        if (da_out) da_out[blk] = da;
+      }
+    }
+  }
+}
+
 int grid_for(int64_t units, int per_block) {
   int64_t b = (units + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
@@ -158,6 +247,18 @@ cudaError_t launch_qdq_nvfp4(const uint16_t* W, const float* V, const float* alp
     LaunchScope scope(stream, "qdq_nvfp4_kernel");
     qdq_nvfp4_kernel<<<grid_for((n + 511) / 512, 8), 256, 0, stream>>>(
         W, V, alpha, n, reinterpret_cast<const unsigned int*>(amax), W_hat, codes, scales, global_scale);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold_nvfp4(const float* dW, const uint16_t* W, float* V, float* alpha, int64_t n, const float* amax,
+                              float lr, float v_min, float v_max, float c_min, float c_max, float* dV_out,
+                              float* da_out, cudaStream_t stream) {
+  {
+    LaunchScope scope(stream, "fold_nvfp4_kernel");
+    fold_nvfp4_kernel<<<grid_for((n + 511) / 512, 8), 256, 0, stream>>>(
+        dW, W, V, alpha, n, reinterpret_cast<const unsigned int*>(amax), lr, v_min, v_max, c_min, c_max, dV_out,
+        da_out);
   }
   return cudaGetLastError();
 }

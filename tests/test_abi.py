@@ -176,3 +176,26 @@ def test_absmax_and_qdq_nvfp4_validation():
     assert q(FAKE, FAKE + 4, None, 4, 64, FAKE, FAKE, None, None, None, None) == ar.AR_ERR_INVALID_ARG  # V misaligned
     assert q(FAKE, None, FAKE + 2, 4, 64, FAKE, FAKE, None, None, None, None) == ar.AR_ERR_INVALID_ARG  # alpha
     assert q(FAKE, None, None, 4, 64, FAKE, None, FAKE + 8, None, None, None) == ar.AR_ERR_INVALID_ARG  # codes
+
+
+def test_tune_step_nvfp4_validation():
+    cfg = ar.ar_qconfig_default()
+    f = ar.lib().ar_tune_step_nvfp4
+    ws = ar.lib().ar_tune_step_nvfp4_workspace
+
+    def call(N=64, K=64, M=32, n_steps=1, ws_bytes=1 << 40, V=FAKE, amax=FAKE, wsp=0x100000):
+        return f(FAKE, V, FAKE, N, K, amax, FAKE, M, FAKE, ctypes.byref(cfg), n_steps, FAKE, None, None, wsp,
+                 ws_bytes, None)
+
+    assert call(K=40) == ar.AR_ERR_INVALID_ARG          # K % 16
+    assert call(N=12) == ar.AR_ERR_INVALID_ARG          # N % 8
+    assert call(M=30) == ar.AR_ERR_INVALID_ARG          # M % 8
+    assert call(n_steps=-1) == ar.AR_ERR_INVALID_ARG
+    assert call(V=None) == ar.AR_ERR_INVALID_ARG
+    assert call(amax=None) == ar.AR_ERR_INVALID_ARG
+    assert call(ws_bytes=16) == ar.AR_ERR_WORKSPACE
+    assert call(wsp=0x100010) == ar.AR_ERR_INVALID_ARG  # workspace alignment
+    # W_hat + G + dW_hat + loss partials
+    assert ws(16384, 4096, 4096, 1) >= 4096 * 4096 * (2 + 4) + 16384 * 4096 * 2
+    assert ws(16384, 4096, 4096, 200) > ws(16384, 4096, 4096, 1) > 0
+    assert ws(16384, 4096, 40, 1) == 0

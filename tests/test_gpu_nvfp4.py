@@ -104,3 +104,77 @@ def test_qdq_nvfp4_full_size_sampled_rows(ar):
     assert np.array_equal(scales[rows], ref["scale_codes"])
     assert np.array_equal(codes[rows], O.pack_fp4(ref["codes"]))
     assert np.array_equal(What[rows], ref["What_bf16"].view(np.uint32) >> 16)
+
+
+# ----------------------------------------------------------------------------
+# tuning steps on NVFP4
+# ----------------------------------------------------------------------------
+
+GRAD_RTOL = 1e-3
+
+
+def _dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _rel_l2(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+def _nv_state(N, K, seed, spread):
+    rng = np.random.default_rng(seed)
+    if not spread:
+        return np.zeros((N, K), np.float32), np.ones((N, K // 16), np.float32)
+    return rng.uniform(-0.4, 0.4, (N, K)).astype(np.float32), rng.uniform(0.6, 1.0, (N, K // 16)).astype(np.float32)
+
+
+@pytest.mark.parametrize("N,K,M,spread", [(256, 256, 64, False), (136, 768, 200, True), (512, 512, 1024, True)])
+def test_tune_step_nvfp4_matches_oracle(ar, N, K, M, spread):
+    d = synth.make_linear(N, K, M, seed=N + M)
+    Wf, Xf = synth.bf16_bits_to_f32(d["W"]), synth.bf16_bits_to_f32(d["X"])
+    V0, a0 = _nv_state(N, K, seed=5, spread=spread)
+    Y = O.reference_forward(Xf, Wf)
+    W, X = _dev_bf16(d["W"]), _dev_bf16(d["X"])
+    V, a = torch.from_numpy(V0.copy()).cuda(), torch.from_numpy(a0.copy()).cuda()
+    amax = torch.empty(1, dtype=torch.float32, device="cuda")
+    ar.ar_absmax_bf16(W, amax)
+    cfg = ar.ar_qconfig_default()
+    ws = torch.empty(ar.ar_tune_step_nvfp4_workspace(M, N, K, 1), dtype=torch.uint8, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    dV = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    da = torch.empty((N, K // 16), dtype=torch.float32, device="cuda")
+    ar.ar_tune_step_nvfp4(W, V, a, amax, X, torch.from_numpy(Y).cuda(), cfg, 1, loss, ws, dV, da)
+    kern = ar.ar_last_kernels()
+    assert "qdq_nvfp4_kernel" in kern and "fold_nvfp4_kernel" in kern
+    L, (V1, a1), gr, _ = O.nvfp4_tune_step_linear(Wf, Xf, Y, V0, a0, O.QConfig())
+    assert loss.item() == pytest.approx(L, rel=1e-4)
+    assert _rel_l2(dV.cpu().numpy(), gr["dV"]) <= GRAD_RTOL
+    assert _rel_l2(da.cpu().numpy(), gr["dalpha"]) <= GRAD_RTOL
+    assert np.mean(V.cpu().numpy() == V1) >= 0.999
+    assert np.mean(a.cpu().numpy() == a1) >= 0.99
+
+
+def test_tune_step_nvfp4_steps_in_one_call_equal_single_calls_and_lower_the_loss(ar):
+    N, K, M = 256, 512, 256
+    d = synth.make_linear(N, K, M, seed=17)
+    Wf, Xf = synth.bf16_bits_to_f32(d["W"]), synth.bf16_bits_to_f32(d["X"])
+    Y = torch.from_numpy(O.reference_forward(Xf, Wf)).cuda()
+    W, X = _dev_bf16(d["W"]), _dev_bf16(d["X"])
+    amax = torch.empty(1, dtype=torch.float32, device="cuda")
+    ar.ar_absmax_bf16(W, amax)
+    cfg = ar.ar_qconfig_default()
+    V0, a0 = _nv_state(N, K, 0, False)
+    Va, aa = torch.from_numpy(V0.copy()).cuda(), torch.from_numpy(a0.copy()).cuda()
+    Vb, ab = torch.from_numpy(V0.copy()).cuda(), torch.from_numpy(a0.copy()).cuda()
+    ws = torch.empty(ar.ar_tune_step_nvfp4_workspace(M, N, K, 20), dtype=torch.uint8, device="cuda")
+    la = torch.empty(20, dtype=torch.float32, device="cuda")
+    ar.ar_tune_step_nvfp4(W, Va, aa, amax, X, Y, cfg, 20, la, ws)
+    lb = []
+    one = torch.empty(1, dtype=torch.float32, device="cuda")
+    for _ in range(20):
+        ar.ar_tune_step_nvfp4(W, Vb, ab, amax, X, Y, cfg, 1, one, ws)
+        lb.append(one.item())
+    assert np.array_equal(la.cpu().numpy(), np.array(lb, np.float32))
+    assert torch.equal(Va, Vb) and torch.equal(aa, ab)
+    assert lb[-1] < lb[0]
