@@ -352,6 +352,37 @@ def nvfp4_bench(ar, torch, peaks, reps=20):
                      "algorithmic_bytes": qbytes, "kernels": kern}
         del W, V, a, What, codes, scales
     out["format"] = "NVFP4: E2M1 codes, E4M3 scale per 16 values, fp32 tensor scale amax/2688; V and alpha applied"
+    # tuning steps on NVFP4 on the 4096² layer with 16384 tokens (the integer step's workload)
+    wl = synth.WORKLOADS[WORKLOAD]
+    N, K, M = wl.n_out, wl.n_in, wl.m_tokens
+    d = synth.make_linear(N, K, M, seed=wl.seed)
+    W, X = to_dev_bf16(d["W"], torch), to_dev_bf16(d["X"], torch)
+    del d
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    ar.ar_linear_forward(X, W, Y)
+    V = torch.zeros((N, K), dtype=torch.float32, device="cuda")
+    a = torch.ones((N, K // 16), dtype=torch.float32, device="cuda")
+    amax = torch.empty(1, dtype=torch.float32, device="cuda")
+    ar.ar_absmax_bf16(W, amax)
+    steps = 20
+    ws = torch.empty(ar.ar_tune_step_nvfp4_workspace(M, N, K, steps), dtype=torch.uint8, device="cuda")
+    loss = torch.empty(steps, dtype=torch.float32, device="cuda")
+    cfg = ar.ar_qconfig_default()
+    ar.ar_tune_step_nvfp4(W, V, a, amax, X, Y, cfg, 3, loss, ws)  # warm-up
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    ar.ar_tune_step_nvfp4(W, V, a, amax, X, Y, cfg, steps, loss, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    flops = 4.0 * M * N * K
+    tfs = flops / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops"])
+    lv = loss.cpu().numpy()
+    out["tune_linear_4096"] = {"steps_per_s": 1e3 / ms, "ms_per_step": ms, "tflops": tfs, "frac_sustained_bf16": tfs / peak,
+                               "steps": steps, "first_loss": float(lv[0]), "last_loss": float(lv[-1]),
+                               "kernels": ar.ar_last_kernels()}
+    del W, X, Y, V, a, ws
     return out
 
 
