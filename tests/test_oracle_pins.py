@@ -850,3 +850,44 @@ def test_nvfp4_tuning_step_on_grid_weights_and_exact_moves():
     assert np.all(np.isin(np.round(np.abs(dv) / 0.005, 6), [0.0, 1.0]))
     assert np.array_equal(np.sign(dv), -np.sign(gr["dV"]).astype(np.float64))
     assert np.all((a1 <= 1.0) & (a1 >= 0.5))
+
+
+def _fp16_rne_from_definition(x32: np.ndarray) -> np.ndarray:
+    """IEEE binary32 -> binary16, round to nearest, ties to even, written from the formats' definitions
+    with integer arithmetic on the encodings (finite inputs)."""
+    b = x32.view(np.uint32).astype(np.int64)
+    sign = (b >> 31) << 15
+    e32 = (b >> 23) & 0xFF
+    man = (b & 0x7FFFFF) | np.where(e32 > 0, 0x800000, 0)
+    e = np.where(e32 > 0, e32 - 127, -126)            # unbiased exponent of the value man * 2^(e - 23)
+    # value / 2^-24 = man * 2^(e + 1) for subnormal results; value / 2^(e - 10) = man * 2^-13 for normal ones
+    normal = e >= -14
+    shift = np.where(normal, 13, np.minimum(-(e + 1), 40))
+    q = man >> shift
+    rem = man - (q << shift)
+    half = np.int64(1) << (shift - 1)
+    q = q + ((rem > half) | ((rem == half) & ((q & 1) == 1)))
+    h = np.where(normal, ((e + 15) << 10) + (q - 0x400), q)
+    h = np.minimum(h, 0x7C00)                           # past the largest finite value: infinity
+    return (sign | h).astype(np.uint16)
+
+
+def test_fp16_metadata_rounding_against_the_ieee_definition():
+    """The oracle's fp16 scale/zero (pack_int4) against a bit-level RNE from the definition: 4M random
+    finite fp32 encodings, and every exact tie and its neighbours between consecutive fp16 values,
+    subnormals and the overflow edge included."""
+    rng = np.random.default_rng(50)
+    r = rng.integers(0, 2 ** 32, 1 << 22, dtype=np.uint64).astype(np.uint32)
+    r = r[((r >> 23) & 0xFF) != 0xFF].view(np.float32)  # finite only
+    h16 = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    mids = (h16[:-1] + h16[1:]) / 2                      # exact in fp32 (fp16 spacing >= 2^-24)
+    m32 = mids.astype(np.float32)
+    assert np.array_equal(m32.astype(np.float64), mids)
+    near = np.concatenate([m32, np.nextafter(m32, np.float32(0)), np.nextafter(m32, np.float32(np.inf)),
+                           np.float32([65504.0, 65519.996, 65520.0, 1e6, 2.0 ** -25, 2.0 ** -26, 5.96e-8])])
+    x = np.concatenate([r, near, -near])
+    zero = np.zeros((1, 1), np.float32)
+    for chunk in np.array_split(x, 64):
+        _, s16, _ = O.pack_int4(np.zeros((1, 8 * chunk.size), np.uint8), chunk.reshape(1, -1),
+                                np.zeros((1, chunk.size), np.float32))
+        assert np.array_equal(s16.reshape(-1), _fp16_rne_from_definition(chunk))
