@@ -810,3 +810,178 @@ def nvfp4_tune_step_linear(Wb, Xb, Y, V, alpha, cfg: QConfig, amax=None, count: 
     V1 = signsgd(V, dV, cfg.lr, cfg.v_min, cfg.v_max)
     a1 = signsgd(alpha, da, cfg.lr, cfg.clip_min, cfg.clip_max)
     return fw["loss"], (V1, a1), {"gW": gW, "dV": dV.astype(f32), "dalpha": da.astype(f32), "G": fw["G"]}, st
+
+
+# ----------------------------------------------------------------------------
+# A decoder block tuned jointly ([AR] §3 "Why Block-Wise Optimization": the
+# block's output error reaches every weight of the block; [AR] §3 "Algorithm
+# Flow": the block, not the layer, is the unit of tuning)
+# ----------------------------------------------------------------------------
+#
+# Readings (the pages name the decoder block as the unit, not its layers):
+# * a pre-norm block of the Llama family: r1 = rmsnorm(X) γ1; Q, K, V = r1 Wqᵀ,
+#   r1 Wkᵀ, r1 Wvᵀ (nh heads of d = H / nh each, no shared K/V heads); the
+#   rotary embedding on Q and K (the halves of each head rotate as complex
+#   pairs (x_i, x_{i+d/2}) by the angle t 10000^(-2i/d), t the token's position
+#   in its sample); causal softmax attention per head with scale 1/sqrt(d),
+#   within each sample; A = O Woᵀ; X2 = X + A; r2 = rmsnorm(X2) γ2;
+#   Y = X2 + (silu(r2 Wgᵀ) ⊙ (r2 Wuᵀ)) Wdᵀ;
+# * rmsnorm(x) = x / sqrt(mean(x²) + 1e-6) over the hidden dimension; γ1, γ2 are
+#   neither quantized nor tuned;
+# * the seven linear weights (q, k, v, o, gate, up, down) are fake-quantized with
+#   their own V, alpha, beta and tuned jointly from the MSE of Y.
+# This section is in fp64 after the QDQ (whose codes are decided in fp32 as
+# everywhere in this module); the rounding points a GPU path shares with it are
+# fixed together with that path.
+
+RMS_EPS = 1e-6
+ROPE_BASE = 10000.0
+DECODER_LAYERS = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+def rmsnorm(x, gamma):
+    """(x / sqrt(mean_j x_j² + eps) * gamma, the per-row 1/sqrt(...)) along the last axis."""
+    x = np.asarray(x, f64)
+    inv = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + RMS_EPS)
+    return x * inv * np.asarray(gamma, f64), inv
+
+
+def rmsnorm_backward(x, gamma, inv, dy):
+    """dx of y = x r gamma, r = (mean(x²) + eps)^(-1/2): r gamma dy - x r³ mean(dy gamma x)."""
+    x = np.asarray(x, f64)
+    gdy = np.asarray(dy, f64) * np.asarray(gamma, f64)
+    return inv * gdy - x * inv ** 3 * np.mean(gdy * x, axis=-1, keepdims=True)
+
+
+def rope_angles(L: int, d: int):
+    """cos, sin [L][d/2] of the angles t * base^(-2i/d)."""
+    i = np.arange(d // 2, dtype=f64)
+    ang = np.arange(L, dtype=f64)[:, None] * ROPE_BASE ** (-2.0 * i / d)[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def rope(x, nh: int, sign: float = 1.0):
+    """Rotate each head of x [S][L][H]: (x_i, x_{i+d/2}) -> (x_i cos - x_{i+d/2} sin, x_{i+d/2} cos + x_i sin);
+    ``sign`` = -1 rotates back (the transpose, used by the backward)."""
+    x = np.asarray(x, f64)
+    S, L, H = x.shape
+    d = H // nh
+    c, s = rope_angles(L, d)
+    s = sign * s
+    xh = x.reshape(S, L, nh, d)
+    x1, x2 = xh[..., : d // 2], xh[..., d // 2:]
+    c, s = c[None, :, None, :], s[None, :, None, :]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1).reshape(S, L, H)
+
+
+def attention_forward(Q, K, V, nh: int):
+    """Causal softmax attention per sample and head: P = softmax(Q Kᵀ / sqrt(d) + mask), O = P V."""
+    S, L, H = Q.shape
+    d = H // nh
+    q = Q.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
+    k = K.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
+    v = V.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
+    z = q @ k.transpose(0, 1, 3, 2) / np.sqrt(d)
+    z = np.where(np.tril(np.ones((L, L), bool))[None, None], z, -np.inf)
+    z = z - z.max(axis=-1, keepdims=True)
+    p = np.exp(z)
+    p = p / p.sum(axis=-1, keepdims=True)
+    o = p @ v
+    return o.transpose(0, 2, 1, 3).reshape(S, L, H), p
+
+
+def attention_backward(Q, K, V, P, dO, nh: int):
+    """dQ, dK, dV of attention_forward: dP = dO Vᵀ, dV = Pᵀ dO, dZ = P (dP - rowsum(dP P)),
+    dQ = dZ K / sqrt(d), dK = dZᵀ Q / sqrt(d)."""
+    S, L, H = Q.shape
+    d = H // nh
+    split = lambda t: t.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
+    merge = lambda t: t.transpose(0, 2, 1, 3).reshape(S, L, H)
+    q, k, v, do = split(Q), split(K), split(V), split(dO)
+    dp = do @ v.transpose(0, 1, 3, 2)
+    dv = P.transpose(0, 1, 3, 2) @ do
+    dz = P * (dp - np.sum(dp * P, axis=-1, keepdims=True))
+    dq = dz @ k / np.sqrt(d)
+    dk = dz.transpose(0, 1, 3, 2) @ q / np.sqrt(d)
+    return merge(dq), merge(dk), merge(dv)
+
+
+def decoder_forward(X, Wh, gammas, nh: int):
+    """The block on X [S][L][H] with the seven weights Wh (dict by DECODER_LAYERS; q/k/v/o [H][H],
+    gate/up [F][H], down [H][F]) and gammas (γ1, γ2).  fp64; returns every intermediate."""
+    X = np.asarray(X, f64)
+    S, L, H = X.shape
+    W = {n: np.asarray(Wh[n], f64) for n in DECODER_LAYERS}
+    r1, inv1 = rmsnorm(X, gammas[0])
+    Qp, Kp, Vv = r1 @ W["q"].T, r1 @ W["k"].T, r1 @ W["v"].T
+    Qr, Kr = rope(Qp, nh), rope(Kp, nh)
+    O, P = attention_forward(Qr, Kr, Vv, nh)
+    X2 = X + O @ W["o"].T
+    r2, inv2 = rmsnorm(X2, gammas[1])
+    a, b = r2 @ W["gate"].T, r2 @ W["up"].T
+    h = silu(a) * b
+    Y = X2 + h @ W["down"].T
+    return {"X": X, "r1": r1, "inv1": inv1, "Qr": Qr, "Kr": Kr, "V": Vv, "P": P, "O": O, "X2": X2, "r2": r2,
+            "inv2": inv2, "a": a, "b": b, "h": h, "Y": Y}
+
+
+def decoder_backward(fw, dY, Wh, gammas, nh: int):
+    """dL/dŴ for the seven weights from dY = dL/dY [S][L][H] (fp64)."""
+    W = {n: np.asarray(Wh[n], f64) for n in DECODER_LAYERS}
+    S, L, H = fw["X"].shape
+    flat = lambda t: t.reshape(S * L, -1)
+    dY = np.asarray(dY, f64)
+    g = {}
+    # MLP and its norm: Y = X2 + h Wdᵀ
+    g["down"] = flat(dY).T @ flat(fw["h"])
+    dh = dY @ W["down"]
+    da = dh * fw["b"] * silu_grad(fw["a"])
+    db = dh * silu(fw["a"])
+    g["gate"] = flat(da).T @ flat(fw["r2"])
+    g["up"] = flat(db).T @ flat(fw["r2"])
+    dr2 = da @ W["gate"] + db @ W["up"]
+    dX2 = dY + rmsnorm_backward(fw["X2"], gammas[1], fw["inv2"], dr2)
+    # attention: X2 = X + O Woᵀ
+    g["o"] = flat(dX2).T @ flat(fw["O"])
+    dO = dX2 @ W["o"]
+    dQr, dKr, dV = attention_backward(fw["Qr"], fw["Kr"], fw["V"], fw["P"], dO, nh)
+    dQ, dK = rope(dQr, nh, -1.0), rope(dKr, nh, -1.0)
+    g["q"] = flat(dQ).T @ flat(fw["r1"])
+    g["k"] = flat(dK).T @ flat(fw["r1"])
+    g["v"] = flat(dV).T @ flat(fw["r1"])
+    return g
+
+
+def decoder_smooth_loss(Ws, X, Y, states, gammas, nh, bits, group_size):
+    """fp64 block loss with every rounding replaced by the identity (the smooth surrogate whose exact
+    gradient the STE fold gives), its QDQ states and its forward."""
+    sts = {n: qdq(Ws[n], *states[n], bits, group_size, dtype=f64, rnd=round_identity) for n in DECODER_LAYERS}
+    fw = decoder_forward(X, {n: sts[n]["What"] for n in DECODER_LAYERS}, gammas, nh)
+    R = fw["Y"] - np.asarray(Y, f64)
+    return float(np.sum(R ** 2) / R.size), sts, fw, 2.0 * R / R.size
+
+
+def decoder_smooth_grads(Ws, X, Y, states, gammas, nh, bits, group_size):
+    """Loss and the STE-fold gradients (dV, dalpha, dbeta per layer) of ``decoder_smooth_loss``."""
+    L, sts, fw, dY = decoder_smooth_loss(Ws, X, Y, states, gammas, nh, bits, group_size)
+    gW = decoder_backward(fw, dY, {n: sts[n]["What"] for n in DECODER_LAYERS}, gammas, nh)
+    return L, {n: ste_fold(gW[n], Ws[n], sts[n], bits) for n in DECODER_LAYERS}
+
+
+def tune_step_decoder(Ws, X, Y, states, gammas, nh: int, cfg: QConfig):
+    """One joint SignSGD step on the seven weights of the block (QDQ in fp32 deciding the codes, the
+    block in fp64).  Returns (loss, new states, grads per layer)."""
+    sts = {n: qdq(Ws[n], *states[n], cfg.bits, cfg.group_size, cfg.symmetric) for n in DECODER_LAYERS}
+    Wh = {n: np.asarray(sts[n]["What_bf16"], f64) for n in DECODER_LAYERS}
+    fw = decoder_forward(X, Wh, gammas, nh)
+    R = fw["Y"] - np.asarray(Y, f64)
+    loss = float(np.sum(R ** 2) / R.size)
+    gW = decoder_backward(fw, 2.0 * R / R.size, Wh, gammas, nh)
+    new, grads = {}, {}
+    for n in DECODER_LAYERS:
+        dV, da, db = ste_fold(gW[n], Ws[n], sts[n], cfg.bits, cfg.symmetric)
+        V, a, b = states[n]
+        new[n] = (signsgd(V, dV, cfg.lr, cfg.v_min, cfg.v_max), signsgd(a, da, cfg.lr, cfg.clip_min, cfg.clip_max),
+                  signsgd(b, db, cfg.lr, cfg.clip_min, cfg.clip_max))
+        grads[n] = (dV, da, db)
+    return loss, new, grads

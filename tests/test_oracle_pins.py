@@ -891,3 +891,140 @@ def test_fp16_metadata_rounding_against_the_ieee_definition():
         _, s16, _ = O.pack_int4(np.zeros((1, 8 * chunk.size), np.uint8), chunk.reshape(1, -1),
                                 np.zeros((1, chunk.size), np.float32))
         assert np.array_equal(s16.reshape(-1), _fp16_rne_from_definition(chunk))
+
+
+# ----------------------------------------------------------------------------
+# decoder block: forward against loops, RoPE and RMSNorm properties, STE
+# gradients by finite differences, grid weights
+# ----------------------------------------------------------------------------
+
+def _decoder_case(rng, S=2, L=5, H=32, F=48, scale=0.2):
+    Ws = {n: rng.standard_normal((H, H)) * scale for n in ("q", "k", "v", "o")}
+    Ws["gate"] = rng.standard_normal((F, H)) * scale
+    Ws["up"] = rng.standard_normal((F, H)) * scale
+    Ws["down"] = rng.standard_normal((H, F)) * scale
+    X = rng.standard_normal((S, L, H))
+    gammas = (1.0 + 0.1 * rng.standard_normal(H), 1.0 + 0.1 * rng.standard_normal(H))
+    return Ws, X, gammas
+
+
+def _decoder_by_loops(X, Ws, gammas, nh):
+    S, L, H = X.shape
+    d = H // nh
+    Y = np.zeros_like(X)
+    for s in range(S):
+        def norm(x, gam):
+            return [x[j] / np.sqrt(sum(v * v for v in x) / len(x) + 1e-6) * gam[j] for j in range(len(x))]
+        r1 = [norm(X[s, t], gammas[0]) for t in range(L)]
+        proj = {n: [[sum(Ws[n][o, j] * r1[t][j] for j in range(H)) for o in range(H)] for t in range(L)]
+                for n in ("q", "k", "v")}
+        for n in ("q", "k"):                       # rotate the halves of each head
+            for t in range(L):
+                for hh in range(nh):
+                    for i in range(d // 2):
+                        ang = t * 10000.0 ** (-2.0 * i / d)
+                        a_, b_ = proj[n][t][hh * d + i], proj[n][t][hh * d + i + d // 2]
+                        proj[n][t][hh * d + i] = a_ * np.cos(ang) - b_ * np.sin(ang)
+                        proj[n][t][hh * d + i + d // 2] = b_ * np.cos(ang) + a_ * np.sin(ang)
+        for t in range(L):
+            o_vec = [0.0] * H
+            for hh in range(nh):
+                sc = [sum(proj["q"][t][hh * d + i] * proj["k"][u][hh * d + i] for i in range(d)) / np.sqrt(d)
+                      for u in range(t + 1)]
+                mx = max(sc)
+                e = [np.exp(v - mx) for v in sc]
+                z = sum(e)
+                for i in range(d):
+                    o_vec[hh * d + i] = sum(e[u] / z * proj["v"][u][hh * d + i] for u in range(t + 1))
+            x2 = [X[s, t, j] + sum(Ws["o"][j, i] * o_vec[i] for i in range(H)) for j in range(H)]
+            r2 = norm(x2, gammas[1])
+            F = Ws["gate"].shape[0]
+            hv = []
+            for f in range(F):
+                av = sum(Ws["gate"][f, j] * r2[j] for j in range(H))
+                bv = sum(Ws["up"][f, j] * r2[j] for j in range(H))
+                hv.append(av / (1.0 + np.exp(-av)) * bv)
+            for j in range(H):
+                Y[s, t, j] = x2[j] + sum(Ws["down"][j, f] * hv[f] for f in range(F))
+    return Y
+
+
+def test_decoder_forward_against_loops():
+    rng = np.random.default_rng(60)
+    Ws, X, gammas = _decoder_case(rng, S=2, L=4, H=16, F=24)
+    got = O.decoder_forward(X, Ws, gammas, nh=2)["Y"]
+    assert np.allclose(got, _decoder_by_loops(X, Ws, gammas, 2), rtol=1e-12, atol=1e-12)
+
+
+def test_rope_rotates_and_depends_only_on_relative_positions():
+    rng = np.random.default_rng(61)
+    S, L, H, nh = 1, 9, 16, 2
+    q = np.tile(rng.standard_normal(H), (S, L, 1))
+    k = np.tile(rng.standard_normal(H), (S, L, 1))
+    rq, rk = O.rope(q, nh), O.rope(k, nh)
+    assert np.allclose(np.linalg.norm(rq.reshape(L, nh, -1), axis=-1), np.linalg.norm(q.reshape(L, nh, -1), axis=-1))
+    assert np.allclose(rq[0, 0], q[0, 0])                                       # position 0: no rotation
+    sc = rq[0].reshape(L, nh, -1)[:, 0] @ rk[0].reshape(L, nh, -1)[:, 0].T      # head 0 scores
+    for off in range(-L + 1, L):
+        diag = np.diagonal(sc, offset=off)
+        assert np.allclose(diag, diag[0])                                      # Toeplitz: t1 - t2 only
+    assert np.allclose(O.rope(rq, nh, -1.0), q)                                 # the inverse rotation
+
+
+def test_rmsnorm_unit_rms_and_backward_by_finite_differences():
+    rng = np.random.default_rng(62)
+    x = rng.standard_normal((3, 20)) * 5
+    y, inv = O.rmsnorm(x, np.ones(20))
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, rtol=1e-6)
+    gam = rng.standard_normal(20)
+    dy = rng.standard_normal((3, 20))
+    y, inv = O.rmsnorm(x, gam)
+    dx = O.rmsnorm_backward(x, gam, inv, dy)
+    h = 1e-6
+    for (r, c) in [(0, 0), (1, 7), (2, 19)]:
+        xp, xm = x.copy(), x.copy()
+        xp[r, c] += h
+        xm[r, c] -= h
+        fd = (np.sum(O.rmsnorm(xp, gam)[0] * dy) - np.sum(O.rmsnorm(xm, gam)[0] * dy)) / (2 * h)
+        assert dx[r, c] == pytest.approx(fd, rel=1e-6, abs=1e-10)
+
+
+def test_decoder_ste_gradients_match_finite_differences():
+    """Smooth surrogate of the whole block (every rounding the identity): the STE fold of each of the
+    seven weights is the exact gradient."""
+    rng = np.random.default_rng(63)
+    Ws, X, gammas = _decoder_case(rng, S=2, L=4, H=16, F=32)
+    g, bits, nh = 8, 3, 2
+    states = {n: (rng.uniform(-0.4, 0.4, W.shape), rng.uniform(0.6, 1.0, (W.shape[0], W.shape[1] // g)),
+                  rng.uniform(0.6, 1.0, (W.shape[0], W.shape[1] // g))) for n, W in Ws.items()}
+    Y = O.decoder_forward(X, Ws, gammas, nh)["Y"] + 0.05 * rng.standard_normal(X.shape)
+    L, grads = O.decoder_smooth_grads(Ws, X, Y, states, gammas, nh, bits, g)
+    h = 1e-7
+
+    def f(name, which, idx, delta):
+        st = {n: tuple(np.array(p, copy=True) for p in states[n]) for n in states}
+        st[name][which][idx] += delta
+        return O.decoder_smooth_loss(Ws, X, Y, st, gammas, nh, bits, g)[0]
+
+    for name in O.DECODER_LAYERS:
+        for which, idx in ((0, (1, 3)), (0, (2, 9)), (1, (0, 1)), (2, (3, 0))):
+            fd = (f(name, which, idx, h) - f(name, which, idx, -h)) / (2 * h)
+            assert grads[name][which][idx] == pytest.approx(fd, rel=1e-5, abs=1e-11), (name, which, idx)
+
+
+def test_decoder_step_on_grid_weights_is_stationary():
+    rng = np.random.default_rng(64)
+    S, L, H, F, nh, g = 2, 3, 32, 48, 4, 16
+    Ws = {n: _grid_weights(rng, H, H, g) for n in ("q", "k", "v", "o")}
+    Ws["gate"], Ws["up"] = _grid_weights(rng, F, H, g) * 0.25, _grid_weights(rng, F, H, g) * 0.25
+    Ws["down"] = _grid_weights(rng, H, F, g) * 0.25
+    X = _bf16(rng.standard_normal((S, L, H)))
+    gammas = (np.ones(H), np.ones(H))
+    Y = O.decoder_forward(X, Ws, gammas, nh)["Y"]
+    states = {n: (np.zeros(W.shape, np.float32), np.ones((W.shape[0], W.shape[1] // g), np.float32),
+                  np.ones((W.shape[0], W.shape[1] // g), np.float32)) for n, W in Ws.items()}
+    loss, new, grads = O.tune_step_decoder(Ws, X, Y, states, gammas, nh, O.QConfig(group_size=g))
+    assert loss == 0.0
+    for n in O.DECODER_LAYERS:
+        assert all(not np.any(d) for d in grads[n])
+        assert all(np.array_equal(a, b) for a, b in zip(new[n], states[n]))
