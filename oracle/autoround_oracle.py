@@ -417,6 +417,29 @@ def w4a16_matmul(A, words, scale16, zero16, group_size: int) -> np.ndarray:
     return np.asarray(A, f64) @ deq.reshape(N, K).T
 
 
+def pack_bitstream(q: np.ndarray, bits: int) -> np.ndarray:
+    """b-bit codes as a little-endian bit stream per row: element k occupies bits
+    [b k, b k + b) of its row, stream bit i in uint32 word i / 32 at position
+    i mod 32; K b must be a multiple of 32.  For b in {2, 4, 8} this is the
+    per-word layout of ``pack_codes``; for b = 3 it puts 32 codes in 3 words,
+    codes 10 and 21 of each 32 straddling two words (the pages define no
+    packing at any width but 4)."""
+    N, K = q.shape
+    assert (K * bits) % 32 == 0
+    qi = np.asarray(q).astype(np.uint32)
+    assert qi.max(initial=0) < (1 << bits)
+    stream = ((qi[:, :, None] >> np.arange(bits, dtype=np.uint32)) & 1).astype(np.uint8).reshape(N, K * bits)
+    return np.ascontiguousarray(np.packbits(stream, axis=-1, bitorder="little")).view("<u4").astype(np.uint32)
+
+
+def unpack_bitstream(words: np.ndarray, K: int, bits: int) -> np.ndarray:
+    """Inverse of ``pack_bitstream``."""
+    N = words.shape[0]
+    stream = np.unpackbits(np.ascontiguousarray(words.astype("<u4")).view(np.uint8), axis=-1, bitorder="little")
+    b = stream[:, : K * bits].reshape(N, K, bits).astype(np.uint16)
+    return np.sum(b << np.arange(bits, dtype=np.uint16), axis=-1).astype(np.uint16)
+
+
 def pack_codes(q: np.ndarray, bits: int) -> np.ndarray:
     """b-bit codes packed little end first along K: 32/b codes per uint32,
     element k at bits b*(k mod 32/b) of word k/(32/b) (the INT4 layout of

@@ -1028,3 +1028,27 @@ def test_decoder_step_on_grid_weights_is_stationary():
     for n in O.DECODER_LAYERS:
         assert all(not np.any(d) for d in grads[n])
         assert all(np.array_equal(a, b) for a, b in zip(new[n], states[n]))
+
+
+def test_bitstream_packing_is_the_per_word_layout_and_places_3_bit_codes_by_hand():
+    rng = np.random.default_rng(70)
+    for bits in (2, 4, 8):
+        q = rng.integers(0, 1 << bits, (5, 96))
+        assert np.array_equal(O.pack_bitstream(q, bits), O.pack_codes(q, bits))
+    # 3 bits: 32 codes in 3 words; code k at stream bits [3k, 3k + 3)
+    q = rng.integers(0, 8, (4, 64))
+    w = O.pack_bitstream(q, 3)
+    assert w.shape == (4, 6)
+    for n in range(4):
+        stream = 0
+        for j in range(6):
+            stream |= int(w[n, j]) << (32 * j)
+        for k in range(64):
+            assert (stream >> (3 * k)) & 7 == q[n, k]
+    assert np.array_equal(O.unpack_bitstream(w, 64, 3), q.astype(np.uint16))
+    # the straddling codes: code 10 is bits 30-31 of word 0 and bit 0 of word 1
+    q1 = np.zeros((1, 32), np.int64)
+    q1[0, 10] = 0b101
+    q1[0, 21] = 0b011
+    w1 = O.pack_bitstream(q1, 3)
+    assert int(w1[0, 0]) == (0b01 << 30) and int(w1[0, 1]) == (0b1 | (0b1 << 31)) and int(w1[0, 2]) == 0b1
