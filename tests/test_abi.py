@@ -199,3 +199,30 @@ def test_tune_step_nvfp4_validation():
     assert ws(16384, 4096, 4096, 1) >= 4096 * 4096 * (2 + 4) + 16384 * 4096 * 2
     assert ws(16384, 4096, 4096, 200) > ws(16384, 4096, 4096, 1) > 0
     assert ws(16384, 4096, 40, 1) == 0
+
+
+def test_header_is_plain_c_and_a_c_program_links_against_the_library(tmp_path):
+    """The boundary is a C ABI: a C99 program (no C++ compiler involved) includes the header, links
+    against the library and calls two host-only entry points."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_ar.c"
+    src.write_text(
+        '#include "autoround.h"\n'
+        "int main(void) {\n"
+        "  ar_qconfig c;\n"
+        "  ar_qconfig_default(&c);\n"
+        "  if (c.bits != 4 || c.group_size != 128) return 1;\n"
+        "  if (ar_tune_step_nvfp4_workspace(4096, 4096, 4096, 1) == 0) return 2;\n"
+        "  if (ar_tune_step_nvfp4_workspace(4096, 4096, 40, 1) != 0) return 3;\n"
+        "  return 0;\n"
+        "}\n")
+    libdir = os.path.dirname(ar.library_path)
+    exe = tmp_path / "use_ar"
+    subprocess.run([gcc, "-std=c99", "-pedantic-errors", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lautoround", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
