@@ -56,7 +56,6 @@ template <int BITS>
 struct CodeCfg {
   static constexpr int kCodeK = 1024 / BITS;          // 512, 256 or 128
   static constexpr int kChunksPerSlot = kCodeK / 128;  // 4, 2 or 1 stages of 128 k
-  static constexpr int kVecPerStage = BITS;            // 16-byte vectors of one row per stage
 };
 constexpr int kCodeSlots = 4;
 constexpr int kNBufMax = 4;   // TMEM accumulators, one group each
@@ -516,7 +515,6 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t a[32];
-#pragma unroll
         if (BITS == 8 && half == 1) {
 #pragma unroll
           for (int v = 0; v < kPre; ++v) pw[v] = ld_shared_v4(pk + (((qv + kPre + v) ^ sw) << 4));
