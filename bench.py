@@ -21,6 +21,15 @@ and ``w4a16`` (the INT4 decode matmul on the 8192x28672 down projection).
 
 ``--impl reference`` times the CPU oracle itself on the host cores (rank 0
 only), on row samples of the same workload.
+
+``--case NAME`` runs one small invocation of one kernel family (three
+launches, no timing, no JSON line) for an ncu capture of that kernel; see
+``CASES`` below.
+
+Peaks: a kernel's bf16 fraction is taken against the measured burst peak when
+its timed region is shorter than a second and against the sustained peak for a
+seconds-long loop; both fractions are reported, and the ``sustained`` object
+holds the same step loop kept busy for a few seconds.
 """
 from __future__ import annotations
 
@@ -55,6 +64,25 @@ def load_peaks():
             p = json.load(f)
         return p, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+SUSTAINED_FROM_S = 1.0  # timed regions shorter than this run at the burst clock
+
+
+def tensor_peak(peaks, seconds):
+    """The bf16 peak that applies to a kernel timed over ``seconds``: the burst
+    figure for a short region (the clock has not yet settled under the power
+    cap), the sustained one for a seconds-long loop.  Returns (TFLOP/s, label)."""
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if seconds < SUSTAINED_FROM_S:
+        return burst, f"bf16_tflops (burst): timed region {seconds:.3f} s < {SUSTAINED_FROM_S:g} s"
+    return sus, f"bf16_tflops_sustained: timed region {seconds:.2f} s >= {SUSTAINED_FROM_S:g} s"
+
+
+def both_fracs(peaks, tflops):
+    return {"frac_burst": tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+            "frac_sustained": tflops / peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])}
 
 
 def workload_config(wl, n_gpus):
@@ -188,20 +216,31 @@ class OracleSample:
                                                                     self.cfg, count=self.count)
 
 
-def cpu_baseline(wl, d, budget_s=12.0):
+def cpu_baseline(wl, d, budget_s=10.0):
+    """The oracle on a bounded row sample, on one host thread (the plain baseline) and on all BLAS threads."""
+    from threadpoolctl import threadpool_limits
+
     s = OracleSample(wl, d, SAMPLE_ROWS_CPU)
-    s.step()  # warm
-    n, t0 = 0, time.perf_counter()
-    while True:
-        s.step()
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
-    per_layer_step = el / n * s.scale
-    return {"value": 1.0 / per_layer_step, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} oracle steps on {SAMPLE_ROWS_CPU} of {wl.n_out} output rows (rows are independent), "
-                      f"{el:.1f} s, scaled x{s.scale:g} to the full layer"}
+    out = {}
+    for label, limit in (("single", 1), ("multi", None)):
+        with threadpool_limits(limits=limit):
+            cores = blas_threads()
+            s.step()  # warm
+            n, t0 = 0, time.perf_counter()
+            while True:
+                s.step()
+                n += 1
+                el = time.perf_counter() - t0
+                if el >= budget_s / 2:
+                    break
+        per_layer_step = el / n * s.scale
+        out[label] = {"value": 1.0 / per_layer_step, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                      "extrapolated": True,
+                      "sample": f"{n} oracle steps on {SAMPLE_ROWS_CPU} of {wl.n_out} output rows (rows are "
+                                f"independent), {el:.1f} s, time scaled x{s.scale:g} to the full layer"}
+    res = dict(out["single"])
+    res["multi_thread"] = out["multi"]
+    return res
 
 
 def run_reference(args, wl):
@@ -218,14 +257,15 @@ def run_reference(args, wl):
     el = time.perf_counter() - t0
     value = args.steps / (el * s.scale)
     sample = (f"each step: the oracle's SignSGD step on {SAMPLE_ROWS_REF} of {wl.n_out} output rows "
-              f"(exact, rows are independent), time scaled x{s.scale:g} to the full layer")
+              f"(exact, rows are independent); value extrapolated: time scaled x{s.scale:g} to the full layer")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl, 1),
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": sample},
+                         "extrapolated": True, "sample": sample},
+        "timed_s": el, "extrapolated": f"x{s.scale:g} from a {SAMPLE_ROWS_REF}-row sample",
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
     return 0
@@ -377,9 +417,10 @@ def nvfp4_bench(ar, torch, peaks, reps=20):
     ms = e0.elapsed_time(e1) / steps
     flops = 4.0 * M * N * K
     tfs = flops / (ms * 1e-3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops"])
+    peak, plabel = tensor_peak(peaks, ms * steps * 1e-3)
     lv = loss.cpu().numpy()
-    out["tune_linear_4096"] = {"steps_per_s": 1e3 / ms, "ms_per_step": ms, "tflops": tfs, "frac_sustained_bf16": tfs / peak,
+    out["tune_linear_4096"] = {"steps_per_s": 1e3 / ms, "ms_per_step": ms, "tflops": tfs, "frac": tfs / peak,
+                               "peak": plabel, **both_fracs(peaks, tfs),
                                "steps": steps, "first_loss": float(lv[0]), "last_loss": float(lv[-1]),
                                "kernels": ar.ar_last_kernels()}
     del W, X, Y, V, a, ws
@@ -426,7 +467,11 @@ def _time_call(torch, fn, warmup=1):
 def other_workloads(ar, torch, peaks, steps=10):
     """Tuning throughput on the remaining workloads (one call of ``steps`` steps each)."""
     out = {}
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+
+    def fracs(tfs, seconds):
+        peak, label = tensor_peak(peaks, seconds)
+        return {"frac": tfs / peak, "peak": label, **both_fracs(peaks, tfs)}
+
     # SwiGLU MLP block, tuned jointly
     wl = synth.WORKLOADS["mlp_4096_11008"]
     M, Hd, F = wl.m_tokens, wl.n_in, wl.inter
@@ -450,7 +495,7 @@ def other_workloads(ar, torch, peaks, steps=10):
     flops = 14.0 * M * Hd * F
     out[wl.name] = {"steps_per_s": steps / (ms * 1e-3), "ms_per_step": ms / steps,
                     "tflops": flops * steps / (ms * 1e-3) / 1e12,
-                    "frac_sustained_bf16": flops * steps / (ms * 1e-3) / 1e12 / peak,
+                    **fracs(flops * steps / (ms * 1e-3) / 1e12, ms * 1e-3),
                     "kernels": ar.ar_last_kernels().count(";") + 1, "steps": steps,
                     "final_loss": float(loss[-1].item())}
     del Ws, X, Y, st, layers, ws
@@ -474,7 +519,7 @@ def other_workloads(ar, torch, peaks, steps=10):
         ms = _time_call(torch, lambda: ar.ar_tune_step(W, V, a, b, X, Y, cfg, n, loss, ws))
         flops = 4.0 * M * N * K
         out[name] = {"steps_per_s": n / (ms * 1e-3), "ms_per_step": ms / n, "tflops": flops * n / (ms * 1e-3) / 1e12,
-                     "frac_sustained_bf16": flops * n / (ms * 1e-3) / 1e12 / peak, "steps": n,
+                     **fracs(flops * n / (ms * 1e-3) / 1e12, ms * 1e-3), "steps": n,
                      "final_loss": float(loss[-1].item())}
         del W, X, V, a, b, Y, ws
         torch.cuda.empty_cache()
@@ -497,13 +542,94 @@ def other_workloads(ar, torch, peaks, steps=10):
     out["driver_light_2x_mlp_4096_11008"] = {
         "blocks": 2, "preset": "light", "samples": S, "seqlen": Lq, "batch": Bq, "iters": iters,
         "s_per_block": ms / 2e3, "steps_per_s": 2 * iters / (ms * 1e-3),
-        "tflops": flops / (ms * 1e-3) / 1e12, "frac_sustained_bf16": flops / (ms * 1e-3) / 1e12 / peak,
+        "tflops": flops / (ms * 1e-3) / 1e12, **fracs(flops / (ms * 1e-3) / 1e12, ms * 1e-3),
         "note": "per block: reference forward on all samples, 50 gathered-minibatch joint steps, quantized forward"}
     del blocks, X0
     torch.cuda.empty_cache()
     if ar.ar_get_device_status() != 0:
         out["device_status"] = ar.ar_last_error()
     return out
+
+
+# ----------------------------------------------------------------------------
+# single-kernel cases for ncu captures (inputs larger than L2, a few GB at most)
+# ----------------------------------------------------------------------------
+
+def run_case(name, ar, torch):
+    """Three launches of one kernel family on a small case (for ``ncu -k <kernel> -s 2 -c 1``)."""
+    dev = "cuda"
+    if name in ("qdq", "pack_int4", "qdq_nvfp4", "absmax"):
+        N, K, g = 8192, 8192, 128  # W 134 MB + V 268 MB: beyond the 126 MB L2
+        d = synth.make_linear(N, K, 1, seed=5, x_outlier_channels=0)
+        W = to_dev_bf16(d["W"], torch)
+        V = (torch.rand((N, K), device=dev) - 0.5).float()
+        if name in ("qdq", "pack_int4"):
+            a = (torch.rand((N, K // g), device=dev) * 0.5 + 0.5).float()
+            b = (torch.rand((N, K // g), device=dev) * 0.5 + 0.5).float()
+            cfg = ar.ar_qconfig_default(bits=4, group_size=g)
+            if name == "qdq":  # as in the tuning step: W_hat, scale, zero
+                What = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+                sc = torch.empty((N, K // g), device=dev)
+                zp = torch.empty((N, K // g), device=dev)
+                fn = lambda: ar.ar_qdq(W, V, a, b, cfg, What, None, sc, zp)
+            else:
+                pk = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+                s16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+                z16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+                fn = lambda: ar.ar_pack_int4(W, V, a, b, cfg, pk, s16, z16)
+        else:
+            a = (torch.rand((N, K // 16), device=dev) * 0.5 + 0.5).float()
+            amax = torch.empty(1, device=dev)
+            ar.ar_absmax_bf16(W, amax)
+            if name == "absmax":
+                fn = lambda: ar.ar_absmax_bf16(W, amax)
+            else:
+                What = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+                codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+                scales = torch.empty((N, K // 16), dtype=torch.uint8, device=dev)
+                gs = torch.empty(1, device=dev)
+                fn = lambda: ar.ar_qdq_nvfp4(W, V, a, amax, What, codes, scales, gs)
+    elif name == "tune_nvfp4":  # one NVFP4 tuning step per launch set: qdq_nvfp4, GEMMs, fold_nvfp4
+        N, K, M = 4096, 4096, 4096
+        d = synth.make_linear(N, K, M, seed=5)
+        W, X = to_dev_bf16(d["W"], torch), to_dev_bf16(d["X"], torch)
+        Y = torch.empty((M, N), device=dev)
+        ar.ar_linear_forward(X, W, Y)
+        V = torch.zeros((N, K), device=dev)
+        a = torch.ones((N, K // 16), device=dev)
+        amax = torch.empty(1, device=dev)
+        ar.ar_absmax_bf16(W, amax)
+        ws = torch.empty(ar.ar_tune_step_nvfp4_workspace(M, N, K, 1), dtype=torch.uint8, device=dev)
+        loss = torch.empty(1, device=dev)
+        cfg = ar.ar_qconfig_default()
+        fn = lambda: ar.ar_tune_step_nvfp4(W, V, a, amax, X, Y, cfg, 1, loss, ws)
+    elif name == "mlp":  # one joint SwiGLU step: swiglu_fwd, resid, fold x3, swiglu_bwd GEMMs
+        Hd, F, M = 4096, 11008, 2048
+        d = synth.make_mlp(Hd, F, M, seed=5)
+        Ws = [to_dev_bf16(d[k], torch) for k in ("Wg", "Wu", "Wd")]
+        X = to_dev_bf16(d["X"], torch)
+        st = [(torch.zeros(W.shape, device=dev), torch.ones((W.shape[0], W.shape[1] // 128), device=dev),
+               torch.ones((W.shape[0], W.shape[1] // 128), device=dev)) for W in Ws]
+        Y = torch.empty((M, Hd), device=dev)
+        fws = torch.empty(ar.ar_block_forward_workspace(ar.AR_BLOCK_SWIGLU_MLP, Ws, M), dtype=torch.uint8, device=dev)
+        ar.ar_block_forward(ar.AR_BLOCK_SWIGLU_MLP, Ws, X, Y, fws)
+        layers = [(W, *t) for W, t in zip(Ws, st)]
+        cfg = ar.ar_qconfig_default()
+        ws = torch.empty(ar.ar_tune_block_workspace(ar.AR_BLOCK_SWIGLU_MLP, layers, M, cfg, 1), dtype=torch.uint8,
+                         device=dev)
+        loss = torch.empty(1, device=dev)
+        fn = lambda: ar.ar_tune_block(ar.AR_BLOCK_SWIGLU_MLP, layers, X, Y, cfg, 1, loss, ws)
+    else:
+        raise SystemExit(f"unknown case {name}; one of {', '.join(CASES)}")
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    st = ar.ar_get_device_status()
+    print(f"case {name}: kernels {ar.ar_last_kernels()} status {st}", flush=True)
+    return 0 if st == 0 else 1
+
+
+CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp")
 
 
 def main():
@@ -517,6 +643,9 @@ def main():
     ap.add_argument("--no-nvfp4", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads (MLP, low-bit, 70B down)")
+    ap.add_argument("--no-sustained", action="store_true", help="skip the seconds-long sustained loop")
+    ap.add_argument("--case", choices=CASES, help="run one small kernel case for an ncu capture and exit")
+    ap.add_argument("--sustained-s", type=float, default=3.0, help="length of the sustained loop (wall seconds)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -528,6 +657,9 @@ def main():
     import torch.distributed as dist
 
     import post_weight_quantization_autoround_b200 as ar
+
+    if args.case:
+        return run_case(args.case, ar, torch)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -552,7 +684,7 @@ def main():
     beta = torch.ones((N, K // g), dtype=torch.float32, device="cuda")
     Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     ar.ar_linear_forward(X, W, Y)
-    n_max = max(args.steps, args.warmup)
+    n_max = max(args.steps, args.warmup, 200)
     ws = torch.empty(ar.ar_tune_step_workspace(W, V, alpha, beta, M, cfg, n_max), dtype=torch.uint8, device="cuda")
     loss = torch.empty(n_max, dtype=torch.float32, device="cuda")
 
@@ -595,19 +727,21 @@ def main():
     dom = max(gemm_names, key=lambda k: prof[k][1])
     dom_us = kernels[dom]["us_per_launch"]
     achieved = flops_gemm / (dom_us * 1e-6) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # the peak that applies to this timed region: burst for a short one, sustained for a seconds-long one
+    peak, peak_label = tensor_peak(peaks, ms * 1e-3)
     tag = "fwd_gemm" if "resid" in dom else "wgrad_fold_gemm"
     traffic = profiled_traffic(tag)
+    step_tflops = flops_step * steps_s_rank / 1e12
     result = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; Llama-7B-shaped layer and calibration stand-ins)",
         "config": workload_config(wl, world),
-        "tflops": flops_step * steps_s_rank / 1e12 * world,
-        "step_roofline_frac": (max(flops_step / (peak * 1e12), 0.0) * 1e3) / (ms / args.steps),
+        "tflops": step_tflops * world,
+        "step_roofline_frac": step_tflops / peak,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{peaks_src} bf16_tflops_sustained (kernel timed inside a long step loop)",
+                     "frac": achieved / peak, "traffic": traffic, **both_fracs(peaks, achieved),
+                     "peak_source": f"{peaks_src} {peak_label}",
                      "algorithmic_flops_per_launch": flops_gemm},
         "gpu_launches": launches,
         "kernels": kernels,
@@ -615,6 +749,37 @@ def main():
         "device_status": status,
         "final_loss": final_loss,
     }
+
+    # --- the same step loop held for seconds (the clock settles under the power cap): sustained figures
+    if not args.no_sustained:
+        calls, chunk = 0, min(n_max, 200)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as sclk:
+            torch.cuda.synchronize()
+            ar.ar_profile_start()
+            s0.record(stream)
+            t_wall = time.perf_counter()
+            while time.perf_counter() - t_wall < args.sustained_s:
+                steps(chunk)
+                calls += 1
+                if calls % 4 == 0:
+                    torch.cuda.synchronize()
+            s1.record(stream)
+            torch.cuda.synchronize()
+            sprof = ar.ar_profile_stop()
+        sms = s0.elapsed_time(s1)
+        n_sus = calls * chunk
+        sdom_us = 1e3 * sprof[dom][1] / max(sprof[dom][0], 1)
+        sach = flops_gemm / (sdom_us * 1e-6) / 1e12
+        speak, slabel = tensor_peak(peaks, sms * 1e-3)
+        result["sustained"] = {
+            "steps": n_sus, "seconds": sms * 1e-3, "steps_per_s": n_sus / (sms * 1e-3),
+            "ms_per_step": sms / n_sus, "tflops": flops_step * n_sus / (sms * 1e-3) / 1e12,
+            "step_roofline_frac": flops_step * n_sus / (sms * 1e-3) / 1e12 / speak,
+            "kernel": dom, "kernel_us_per_launch": sdom_us, "kernel_tflops": sach, "kernel_frac": sach / speak,
+            **{f"kernel_{k}": v for k, v in both_fracs(peaks, sach).items()},
+            "peak_source": f"{peaks_src} {slabel}", "clocks": sclk.summary(),
+            "note": f"{calls} back-to-back calls of {chunk} steps; device time over the whole loop"}
 
     # --- end to end through the host-buffer API (pinned host tensors, copies timed)
     if not args.no_e2e:

@@ -184,6 +184,26 @@ AR_API ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_laye
                        const float* Y, const ar_qconfig* cfg, int n_steps, float* loss_per_step,
                        const ar_grads* grads, void* workspace, size_t workspace_bytes, ar_stream_t stream);
 
+/* ar_tune_step for a shard of one linear layer's output rows (AR_BLOCK_LINEAR;
+ * [AR] §3 "Algorithm Flow" steps 3-5).  Output rows of a linear layer are
+ * independent: row n of W, V, alpha, beta only meets column n of Y and of G.
+ * So a layer of N_total rows splits over GPUs by rows with no exchange on the
+ * data path; each GPU passes its rows (*layer: W, V, alpha, beta [N][K], N
+ * rows of the N_total), the full X [M][K] and its columns of the reference
+ * output Y [M][N] (ar_linear_forward of its rows).  The only difference from
+ * ar_tune_step is the loss normaliser: M * n_total instead of M * N, so
+ *   G = bf16(2 R / (M n_total))
+ * is bit for bit the whole layer's G on these rows, and every update matches
+ * the unsharded call's rows exactly.  loss_per_step[i] is this shard's part of
+ * the layer's loss, sum_shard R^2 / (M n_total): the shards' values add up to
+ * the layer's loss (a one-float all-reduce, for reporting only).
+ * Workspace: ar_tune_step_workspace of the shard (AR_BLOCK_LINEAR, *layer).
+ * Errors: as ar_tune_step; AR_ERR_INVALID_ARG if n_total < layer->N. */
+AR_API ar_status ar_tune_step_shard(const ar_layer* layer, const uint16_t* X, int64_t M, const float* Y,
+                                    int64_t n_total, const ar_qconfig* cfg, int n_steps, float* loss_per_step,
+                                    const ar_grads* grads, void* workspace, size_t workspace_bytes,
+                                    ar_stream_t stream);
+
 /* Fixed scratch size of ar_tune_step_noalloc, in bytes (16 MiB per GPU). */
 #define AR_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
 
@@ -201,8 +221,10 @@ AR_API ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_laye
  *    this admits e.g. a 1024x1024 layer with 2048 tokens, not a 4096x4096
  *    layer with 16384 tokens.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress, with that device current) and keeps it for later
+ *    calls; make that first call before any stream capture.  The address is
+ *    not looked up again, so do not call this entry point on a device after
+ *    cudaDeviceReset() on it in the same process.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; nothing in it needs to start at zero (each step writes every
  *    scratch byte it later reads).  Calls that overlap on the GPU (other

@@ -23,6 +23,7 @@ __all__ = [
     "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES", "AR_BLOCK_SWIGLU_MLP", "ar_block_forward",
     "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace", "ar_debug_wait_timeout",
     "ar_absmax_bf16", "ar_qdq_nvfp4", "ar_tune_step_nvfp4_workspace", "ar_tune_step_nvfp4",
+    "ar_tune_step_shard",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -71,6 +72,8 @@ _SIGNATURES = {
     "ar_tune_step_workspace": (ctypes.c_size_t, [_INT, ctypes.POINTER(Layer), _INT, _I64, ctypes.POINTER(QConfig), _INT]),
     "ar_tune_step": (_INT, [_INT, ctypes.POINTER(Layer), _INT, _P, _I64, _P, ctypes.POINTER(QConfig), _INT, _P,
                             ctypes.POINTER(Grads), _P, ctypes.c_size_t, _P]),
+    "ar_tune_step_shard": (_INT, [ctypes.POINTER(Layer), _P, _I64, _P, _I64, ctypes.POINTER(QConfig), _INT, _P,
+                                  ctypes.POINTER(Grads), _P, ctypes.c_size_t, _P]),
     "ar_pack_int4": (_INT, [_P, _P, _P, _P, _I64, _I64, ctypes.POINTER(QConfig), _P, _P, _P, _P]),
     "ar_w4a16_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "ar_gemm_bf16": (_INT, [_P, _INT, _P, _INT, _P, _I64, _I64, _I64, _P]),
@@ -192,6 +195,18 @@ def ar_tune_step(W, V, alpha, beta, X, Y, cfg: QConfig, n_steps: int, loss, work
     _check(lib().ar_tune_step(block_kind, ctypes.byref(layer), 1, _ptr(X), X.shape[0], _ptr(Y), ctypes.byref(cfg),
                               n_steps, _ptr(loss), gp, _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)))
+
+
+def ar_tune_step_shard(W, V, alpha, beta, X, Y, n_total: int, cfg: QConfig, n_steps: int, loss, workspace,
+                       dV=None, dalpha=None, dbeta=None, stream=None) -> None:
+    """``ar_tune_step`` on a shard of a layer's output rows (W, V, alpha, beta hold this shard's rows, Y its
+    columns); ``n_total`` is the whole layer's row count, which sets the loss normaliser."""
+    layer = _layer(W, V, alpha, beta)
+    grads = Grads(_ptr(dV), _ptr(dalpha), _ptr(dbeta))
+    gp = ctypes.byref(grads) if (dV is not None or dalpha is not None or dbeta is not None) else None
+    _check(lib().ar_tune_step_shard(ctypes.byref(layer), _ptr(X), X.shape[0], _ptr(Y), n_total, ctypes.byref(cfg),
+                                    n_steps, _ptr(loss), gp, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def _layers(ws):

@@ -3,7 +3,8 @@
     python -m post_weight_quantization_autoround_b200.build [--verbose-ptxas]
 
 Compiles every ``csrc/*.cu`` with relocatable device code (one status word is
-shared by all translation units) and links a shared library next to this file.
+shared by all translation units) into ``_build/obj`` and links a shared library
+next to this file.
 """
 from __future__ import annotations
 
@@ -30,29 +31,46 @@ def sources():
     return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
 
 
-def build(verbose_ptxas: bool = False, extra=None, out: str = LIB) -> str:
-    srcs = sources()
-    cmd = [
-        nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-shared",
-        "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-        "-I", os.path.join(ROOT, "include"),
-        "-o", out, *srcs,
-    ]
-    if verbose_ptxas:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    if extra:
-        cmd[1:1] = list(extra)
+def _compile(args):
+    cmd, = args
     subprocess.run(cmd, check=True)
+
+
+def build(verbose_ptxas: bool = False, extra=None, out: str = LIB, jobs: int | None = None) -> str:
+    """Compiles each source to a relocatable object (in parallel, only those
+    older than a source or header), then device-links them into ``out``."""
+    srcs = sources()
+    obj_dir = os.path.join(ROOT, "_build", "obj")
+    os.makedirs(obj_dir, exist_ok=True)
+    common = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-Xcompiler", "-fPIC",
+              "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]
+    if verbose_ptxas:
+        common = ["-Xptxas", "-v", *common]
+    if extra:
+        common = [*extra, *common]
+    headers = glob.glob(os.path.join(HERE, "csrc", "*.h")) + glob.glob(os.path.join(HERE, "csrc", "*.cuh"))
+    headers += glob.glob(os.path.join(ROOT, "include", "*.h"))
+    newest_header = max((os.path.getmtime(h) for h in headers), default=0.0)
+    stamp = os.path.join(obj_dir, "flags.txt")
+    flags = " ".join(common)
+    same_flags = os.path.exists(stamp) and open(stamp).read() == flags
+    objs, todo = [], []
+    for src in srcs:
+        obj = os.path.join(obj_dir, os.path.basename(src)[:-3] + ".o")
+        objs.append(obj)
+        fresh = (same_flags and os.path.exists(obj)
+                 and os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_header))
+        if not fresh or verbose_ptxas:
+            todo.append(([nvcc_path(), *common, "-dc", "-o", obj, src],))
+    if todo:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(max_workers=jobs or os.cpu_count() or 4) as ex:
+            list(ex.map(_compile, todo))
+        with open(stamp, "w") as f:
+            f.write(flags)
+    subprocess.run([nvcc_path(), *ARCH, "-shared", "-rdc=true", "-Xcompiler", "-fPIC", "-o", out, *objs], check=True)
     return out
-
-
-def up_to_date(out: str = LIB) -> bool:
-    if not os.path.exists(out):
-        return False
-    t = os.path.getmtime(out)
-    deps = sources() + glob.glob(os.path.join(HERE, "csrc", "*.h")) + glob.glob(os.path.join(HERE, "csrc", "*.cuh"))
-    deps += glob.glob(os.path.join(ROOT, "include", "*.h"))
-    return all(os.path.getmtime(d) <= t for d in deps)
 
 
 if __name__ == "__main__":

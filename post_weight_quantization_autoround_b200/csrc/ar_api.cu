@@ -10,6 +10,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/autoround.h"
 #include "ar_internal.h"
 
@@ -258,6 +260,58 @@ ar_status tune_mlp(const ar_layer* L, const uint16_t* X, int64_t M, const float*
   if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
   return end_call();
 }
+
+// n_steps tuning steps of one linear layer (or of a shard of its output rows:
+// n_total > 0 is the whole layer's row count, which sets the loss normaliser).
+ar_status tune_linear(const ar_layer* layers, int n_layers, const uint16_t* X, int64_t M, const float* Y,
+                      const ar_qconfig* cfg, int n_steps, float* loss_per_step, const ar_grads* grads,
+                      void* workspace, size_t workspace_bytes, int64_t n_total, cudaStream_t s) {
+  ar_status st = check_linear(layers, n_layers, M, cfg, true);
+  if (st != AR_OK) return st;
+  if (n_steps < 0) return fail(AR_ERR_INVALID_ARG, "n_steps must be >= 0");
+  if (!X || !Y || !loss_per_step) return fail(AR_ERR_INVALID_ARG, "X, Y and loss_per_step are required");
+  if (!aligned16(X) || !aligned16(Y)) return fail(AR_ERR_INVALID_ARG, "X and Y must be 16-byte aligned");
+  const ar_layer& L = layers[0];
+  const LinearWs w = linear_ws(M, L.N, L.K, cfg->group_size, n_steps);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (grads) {
+    const void* gp[] = {grads->dV, grads->dalpha, grads->dbeta};
+    for (const void* p : gp)
+      if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "gradient outputs must be 16-byte aligned");
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* W_hat = reinterpret_cast<uint16_t*>(ws + w.what);
+  uint16_t* G = reinterpret_cast<uint16_t*>(ws + w.g);
+  float* sc = reinterpret_cast<float*>(ws + w.s);
+  float* zp = reinterpret_cast<float*>(ws + w.zp);
+  float* mx = reinterpret_cast<float*>(ws + w.mx);
+  float* mn = reinterpret_cast<float*>(ws + w.mn);
+  double* partial = reinterpret_cast<double*>(ws + w.partial);
+  const int Mi = static_cast<int>(M), Ni = static_cast<int>(L.N), Ki = static_cast<int>(L.K);
+  // loss normaliser M * N_total: the whole layer's output count (N_total = N unless this is a row shard)
+  const double count = static_cast<double>(M) * static_cast<double>(n_total > 0 ? n_total : L.N);
+  const float gscale = static_cast<float>(2.0 / count);
+  const int steps = n_steps > 0 ? n_steps : 1;
+  cudaError_t e;
+  for (int step = 0; step < steps; ++step) {
+    e = launch_qdq(L.W, L.V, L.alpha, L.beta, L.N, L.K, cfg->group_size, cfg->bits, cfg->symmetric, W_hat, nullptr,
+                   sc, zp, mx, mn, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+    e = launch_gemm_resid(X, W_hat, Y, G, gscale, partial + static_cast<size_t>(step) * w.partials_per_step, Mi, Ni,
+                          Ki, s);
+    if (e != cudaSuccess) return cuda_fail(e, "forward GEMM launch");
+    if (n_steps == 0) break;
+    const bool last = step == steps - 1;
+    const FoldArgs fa = fold_args(L, cfg, sc, zp, mx, mn, (last && grads) ? grads : nullptr);
+    e = launch_gemm_fold(G, X, fa, Mi, Ni, Ki, s);
+    if (e != cudaSuccess) return cuda_fail(e, "weight-gradient GEMM launch");
+  }
+  e = launch_loss_reduce(partial, w.partials_per_step, steps, 1.0 / count, loss_per_step, s);
+  if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
+  return end_call();
+}
 }  // namespace
 
 void set_last_error(const char* msg) { t_error = msg; }
@@ -290,7 +344,10 @@ cudaEvent_t take_event() {
 }
 }  // namespace
 
+// Every launch is also an NVTX range named after the kernel, so a timeline
+// profiler shows which library kernel ran (a no-op without a profiler attached).
 LaunchScope::LaunchScope(cudaStream_t stream, const char* name) : stream_(stream), name_(name), start_(nullptr) {
+  nvtxRangePushA(name);
   if (g_prof_on.load(std::memory_order_relaxed)) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     start_ = take_event();
@@ -299,6 +356,7 @@ LaunchScope::LaunchScope(cudaStream_t stream, const char* name) : stream_(stream
 }
 
 LaunchScope::~LaunchScope() {
+  nvtxRangePop();
   trace_kernel(name_);
   if (start_) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -431,70 +489,20 @@ ar_status ar_tune_step(int block_kind, const ar_layer* layers, int n_layers, con
                     reinterpret_cast<cudaStream_t>(stream));
   }
   if (block_kind != AR_BLOCK_LINEAR) return fail(AR_ERR_UNSUPPORTED, "block_kind %d not supported", block_kind);
-  ar_status st = check_linear(layers, n_layers, M, cfg, true);
-  if (st != AR_OK) return st;
-  if (n_steps < 0) return fail(AR_ERR_INVALID_ARG, "n_steps must be >= 0");
-  if (!X || !Y || !loss_per_step) return fail(AR_ERR_INVALID_ARG, "X, Y and loss_per_step are required");
-  if (!aligned16(X) || !aligned16(Y)) return fail(AR_ERR_INVALID_ARG, "X and Y must be 16-byte aligned");
-  const ar_layer& L = layers[0];
-  const LinearWs w = linear_ws(M, L.N, L.K, cfg->group_size, n_steps);
-  if (!workspace || workspace_bytes < w.total)
-    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  if (grads) {
-    const void* gp[] = {grads->dV, grads->dalpha, grads->dbeta};
-    for (const void* p : gp)
-      if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "gradient outputs must be 16-byte aligned");
-  }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint16_t* W_hat = reinterpret_cast<uint16_t*>(ws + w.what);
-  uint16_t* G = reinterpret_cast<uint16_t*>(ws + w.g);
-  float* sc = reinterpret_cast<float*>(ws + w.s);
-  float* zp = reinterpret_cast<float*>(ws + w.zp);
-  float* mx = reinterpret_cast<float*>(ws + w.mx);
-  float* mn = reinterpret_cast<float*>(ws + w.mn);
-  double* partial = reinterpret_cast<double*>(ws + w.partial);
-  const int Mi = static_cast<int>(M), Ni = static_cast<int>(L.N), Ki = static_cast<int>(L.K);
-  const float gscale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(L.N)));
-  const int steps = n_steps > 0 ? n_steps : 1;
-  cudaError_t e;
-  for (int step = 0; step < steps; ++step) {
-    e = launch_qdq(L.W, L.V, L.alpha, L.beta, L.N, L.K, cfg->group_size, cfg->bits, cfg->symmetric, W_hat, nullptr,
-                   sc, zp, mx, mn, s);
-    if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
-    e = launch_gemm_resid(X, W_hat, Y, G, gscale, partial + static_cast<size_t>(step) * w.partials_per_step, Mi, Ni,
-                          Ki, s);
-    if (e != cudaSuccess) return cuda_fail(e, "forward GEMM launch");
-    if (n_steps == 0) break;
-    FoldArgs fa{};
-    fa.W = L.W;
-    fa.V = L.V;
-    fa.alpha = L.alpha;
-    fa.beta = L.beta;
-    fa.s = sc;
-    fa.zp = zp;
-    fa.mx = mx;
-    fa.mn = mn;
-    const bool last = step == steps - 1;
-    fa.dV_out = (last && grads) ? grads->dV : nullptr;
-    fa.da_out = (last && grads) ? grads->dalpha : nullptr;
-    fa.db_out = (last && grads) ? grads->dbeta : nullptr;
-    fa.group_size = cfg->group_size;
-    fa.bits = cfg->bits;
-    fa.symmetric = cfg->symmetric;
-    fa.lr = cfg->lr;
-    fa.v_min = cfg->v_min;
-    fa.v_max = cfg->v_max;
-    fa.c_min = cfg->clip_min;
-    fa.c_max = cfg->clip_max;
-    e = launch_gemm_fold(G, X, fa, Mi, Ni, Ki, s);
-    if (e != cudaSuccess) return cuda_fail(e, "weight-gradient GEMM launch");
-  }
-  e = launch_loss_reduce(partial, w.partials_per_step, steps, 1.0 / (static_cast<double>(M) * static_cast<double>(L.N)),
-                         loss_per_step, s);
-  if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
-  return end_call();
+  return tune_linear(layers, n_layers, X, M, Y, cfg, n_steps, loss_per_step, grads, workspace, workspace_bytes,
+                     0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ar_status ar_tune_step_shard(const ar_layer* layer, const uint16_t* X, int64_t M, const float* Y, int64_t n_total,
+                             const ar_qconfig* cfg, int n_steps, float* loss_per_step, const ar_grads* grads,
+                             void* workspace, size_t workspace_bytes, ar_stream_t stream) {
+  begin_call();
+  if (!layer) return fail(AR_ERR_INVALID_ARG, "layer is NULL");
+  if (n_total < layer->N || n_total > INT32_MAX)
+    return fail(AR_ERR_INVALID_ARG, "n_total=%lld must be in [N=%lld, 2^31-1]", (long long)n_total,
+                (long long)layer->N);
+  return tune_linear(layer, 1, X, M, Y, cfg, n_steps, loss_per_step, grads, workspace, workspace_bytes, n_total,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t ar_block_forward_workspace(int block_kind, const ar_layer* layers, int n_layers, int64_t M) {

@@ -11,6 +11,8 @@
 // code is loaded and which stays allocated until the process exits.
 #include <stdio.h>
 
+#include <mutex>
+
 #include "../../include/autoround.h"
 #include "ar_internal.h"
 
@@ -23,15 +25,20 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[AR_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
-// Device address of the scratch array for the current device (looked up once
-// per device, with that device current).
+// Device address of the scratch array for the current device.  The first call
+// on a device looks it up (cudaGetSymbolAddress, with that device current) and
+// caches it; the lock makes concurrent first calls from several host threads
+// safe.  A cudaDeviceReset() unloads the library's device code, so the cached
+// address of that device is stale afterwards (documented in autoround.h).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);

@@ -366,8 +366,9 @@ cudaError_t launch_tma(const CUtensorMap& tmW, const uint16_t* A, int T, const _
 cudaError_t launch_w4a16(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                          const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream) {
   cudaError_t e = launch_w4a16_dec(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+  // cudaErrorNotSupported comes from the shape checks before any CUDA call, so
+  // no runtime error state is set and none is cleared here
   if (e != cudaErrorNotSupported) return e;
-  (void)cudaGetLastError();
   int group_shift = 0;
   while ((1 << group_shift) < group_size) ++group_shift;
   CUtensorMap tmW;

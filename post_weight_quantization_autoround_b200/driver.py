@@ -188,3 +188,46 @@ def load_int4_checkpoint(path: str):
         meta = json.loads(str(f["meta"]))
         arrays = {k: f[k] for k in f.files if k != "meta"}
     return meta, arrays
+
+
+_CFG_FIELDS = ("bits", "group_size", "symmetric", "lr", "iters", "v_min", "v_max", "clip_min", "clip_max")
+
+
+def save_tuning_state(path: str, layers: Sequence[Sequence[torch.Tensor]], step: int, cfg: QConfig,
+                      names: Sequence[str] | None = None) -> None:
+    """Writes a resumable tuning state to one ``.npz`` file: each layer's
+    rounding offsets V (fp32 [N][K]) and clip factors alpha, beta (fp32
+    [N][K/g]) as ``{name}.V`` / ``.alpha`` / ``.beta``, the number of steps
+    already taken and the quantizer/optimiser settings (``meta``, JSON).
+    ``layers`` holds (V, alpha, beta) device tensors.  SignSGD keeps no other
+    state (no moments), so these arrays and the step count are everything a
+    later call of ``ar_tune_step`` needs to continue exactly where this one
+    stopped."""
+    import json
+
+    names = list(names) if names is not None else [f"layer{i}" for i in range(len(layers))]
+    if len(names) != len(layers):
+        raise ValueError("one name per layer")
+    arrays = {}
+    for name, (V, a, b) in zip(names, layers):
+        arrays[f"{name}.V"] = V.detach().cpu().numpy()
+        arrays[f"{name}.alpha"] = a.detach().cpu().numpy()
+        arrays[f"{name}.beta"] = b.detach().cpu().numpy()
+    meta = {"step": int(step), "layers": names, "cfg": {k: getattr(cfg, k) for k in _CFG_FIELDS},
+            "content": "AutoRound tuning state: V fp32 [N][K]; alpha, beta fp32 [N][K/group_size]"}
+    np.savez(path, meta=np.array(json.dumps(meta)), **arrays)
+
+
+def load_tuning_state(path: str, device="cuda"):
+    """Reads ``save_tuning_state``'s file: (step, QConfig, [(V, alpha, beta)] device tensors, names)."""
+    import json
+
+    from . import ar_qconfig_default
+
+    with np.load(path) as f:
+        meta = json.loads(str(f["meta"]))
+        names = meta["layers"]
+        layers = [tuple(torch.from_numpy(np.array(f[f"{n}.{k}"])).to(device) for k in ("V", "alpha", "beta"))
+                  for n in names]
+    cfg = ar_qconfig_default(**meta["cfg"])
+    return int(meta["step"]), cfg, layers, names

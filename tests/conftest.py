@@ -8,3 +8,4 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a) and the built library")
+    config.addinivalue_line("markers", "slow: whole tuning runs (minutes of oracle time); part of the gpu set")

@@ -226,3 +226,12 @@ def test_header_is_plain_c_and_a_c_program_links_against_the_library(tmp_path):
     subprocess.run([gcc, "-std=c99", "-pedantic-errors", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
                     str(src), "-L", libdir, "-lautoround", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
     assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_tune_step_shard_rejects_a_total_below_the_shard():
+    cfg = ar.ar_qconfig_default()
+    layer = ar.Layer(FAKE, FAKE, FAKE, FAKE, 256, 256)
+    st = ar.lib().ar_tune_step_shard(ctypes.byref(layer), FAKE, 32, FAKE, 128, ctypes.byref(cfg), 1, FAKE, None,
+                                     0x100000, 1 << 40, None)
+    assert st == ar.AR_ERR_INVALID_ARG
+    assert "n_total" in ar.ar_last_error()

@@ -114,3 +114,28 @@ def test_int4_checkpoint_round_trip(tmp_path):
             assert np.array_equal(arrays[f"b{b}.{name}.packed"], p.numpy().view(np.uint32))
             assert np.array_equal(arrays[f"b{b}.{name}.scale"], s.numpy())
             assert np.array_equal(arrays[f"b{b}.{name}.zero"], z.numpy())
+
+
+def test_tuning_state_file_round_trips(tmp_path):
+    """save_tuning_state / load_tuning_state keep every array bit for bit, the step count and the settings."""
+    import os
+
+    import torch
+
+    import post_weight_quantization_autoround_b200 as ar
+    from post_weight_quantization_autoround_b200 import driver
+
+    if not os.path.exists(ar.library_path):
+        pytest.skip("libautoround.so not built")
+    cfg = ar.ar_qconfig_default(bits=2, group_size=32, lr=0.002)
+    layers = [tuple(torch.from_numpy(x) for x in synth.make_state(n, k, 32, seed=n, spread=True))
+              for n, k in ((64, 128), (128, 64))]
+    path = str(tmp_path / "s.npz")
+    driver.save_tuning_state(path, layers, 37, cfg, names=["gate", "down"])
+    step, cfg2, back, names = driver.load_tuning_state(path, device="cpu")
+    assert step == 37 and names == ["gate", "down"]
+    for f in driver._CFG_FIELDS:
+        assert getattr(cfg2, f) == getattr(cfg, f), f
+    for (V, a, b), (V2, a2, b2) in zip(layers, back):
+        for x, y in ((V, V2), (a, a2), (b, b2)):
+            assert x.dtype == y.dtype and torch.equal(x, y)

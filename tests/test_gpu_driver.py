@@ -117,3 +117,35 @@ def test_streamed_driver_equals_the_device_driver_and_writes_a_checkpoint(ar, tm
     assert meta["blocks"] == 3
     assert np.array_equal(arrays["b2.down.packed"], st_res[2]["int4"][2][0].numpy().view(np.uint32))
 
+
+
+def test_tuning_state_checkpoint_resumes_bit_for_bit(ar, tmp_path):
+    """5 steps, save the state to a file, load it into fresh tensors, 5 more steps == 10 steps in one go."""
+    from post_weight_quantization_autoround_b200 import driver
+
+    N, K, M, g = 256, 512, 320, 128
+    d = synth.make_linear(N, K, M, seed=12)
+    V0, a0, b0 = synth.make_state(N, K, g, seed=3, spread=True)
+    cfg = ar.ar_qconfig_default(bits=3, group_size=g)
+    W, X = bf16_dev(d["W"]), bf16_dev(d["X"])
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    ar.ar_linear_forward(X, W, Y)
+    ref = [torch.from_numpy(x.copy()).cuda() for x in (V0, a0, b0)]
+    ws = torch.empty(ar.ar_tune_step_workspace(W, *ref, M, cfg, 10), dtype=torch.uint8, device="cuda")
+    loss10 = torch.empty(10, device="cuda")
+    ar.ar_tune_step(W, *ref, X, Y, cfg, 10, loss10, ws)
+    st = [torch.from_numpy(x.copy()).cuda() for x in (V0, a0, b0)]
+    loss_a = torch.empty(5, device="cuda")
+    ar.ar_tune_step(W, *st, X, Y, cfg, 5, loss_a, ws)
+    path = str(tmp_path / "state.npz")
+    driver.save_tuning_state(path, [st], 5, cfg, names=["down"])
+    del st
+    step, cfg2, layers, names = driver.load_tuning_state(path)
+    assert step == 5 and names == ["down"]
+    assert (cfg2.bits, cfg2.group_size, cfg2.lr) == (cfg.bits, cfg.group_size, cfg.lr)
+    loss_b = torch.empty(5, device="cuda")
+    ar.ar_tune_step(W, *layers[0], X, Y, cfg2, 5, loss_b, ws)
+    assert ar.ar_get_device_status() == 0
+    assert np.array_equal(np.concatenate([loss_a.cpu().numpy(), loss_b.cpu().numpy()]), loss10.cpu().numpy())
+    for x, y in zip(layers[0], ref):
+        assert np.array_equal(x.cpu().numpy(), y.cpu().numpy())

@@ -334,6 +334,32 @@ def test_full_size_sampled_rows(ar, name, steps):
     assert np.isfinite(rest["loss"]).all()
 
 
+def test_row_shards_reproduce_the_unsharded_step(ar):
+    """ar_tune_step_shard on two row ranges of one layer gives the unsharded call's rows bit for bit."""
+    N, K, M, g, steps, cut = 320, 512, 200, 128, 3, 136  # 136/320: the ratio is not a power of two
+    d = synth.make_linear(N, K, M, seed=31)
+    V, a, b = synth.make_state(N, K, g, seed=6, spread=True)
+    cfg, ocfg = cfg_pair(ar, 4, g)
+    full = GpuLinear(ar, d["W"], d["X"], V, a, b, cfg, n_steps=steps)
+    l_full = full.step(steps)["loss"]
+    shard_losses, shard_states = [], []
+    for lo, hi in ((0, cut), (cut, N)):
+        sh = GpuLinear(ar, d["W"][lo:hi], d["X"], V[lo:hi], a[lo:hi], b[lo:hi], cfg, n_steps=steps)
+        loss = torch.empty(steps, dtype=torch.float32, device="cuda")
+        ar.ar_tune_step_shard(sh.W, sh.V, sh.a, sh.b, sh.X, sh.Y, N, cfg, steps, loss, sh.ws)
+        assert ar.ar_get_device_status() == 0
+        shard_losses.append(loss.cpu().numpy())
+        shard_states.append(sh.state())
+    for i, ref in enumerate(full.state()):
+        assert np.array_equal(np.concatenate([shard_states[0][i], shard_states[1][i]]), ref), i
+    assert np.allclose(shard_losses[0] + shard_losses[1], l_full, rtol=1e-5)
+    # and the oracle on the second shard with the layer's normaliser
+    Wf, Xf = synth.bf16_bits_to_f32(d["W"][cut:]), synth.bf16_bits_to_f32(d["X"])
+    L, _, _, _ = O.tune_step_linear(Wf, Xf, O.reference_forward(Xf, Wf), V[cut:], a[cut:], b[cut:], ocfg,
+                                    count=M * N)
+    assert shard_losses[1][0] == pytest.approx(L, rel=1e-4)
+
+
 def test_steps_are_deterministic_and_resumable(ar):
     d = synth.make_linear(256, 512, 384, seed=9)
     V, a, b = synth.make_state(256, 512, 128, seed=1, spread=True)
