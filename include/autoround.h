@@ -204,6 +204,87 @@ AR_API ar_status ar_tune_step_shard(const ar_layer* layer, const uint16_t* X, in
                                     const ar_grads* grads, void* workspace, size_t workspace_bytes,
                                     ar_stream_t stream);
 
+/* ---- the decoder block ([AR] §3 "Why Block-Wise Optimization", "Algorithm
+ * Flow": the decoder block, not the layer, is the unit of tuning) ----------
+ * The pages name the block but not its layers; this is the Llama family's
+ * pre-norm block on X [M][H] bf16, M = samples * seq_len tokens:
+ *   r1 = bf16(rmsnorm(X) gamma1), rmsnorm(x) = x / sqrt(mean(x^2) + 1e-6)
+ *   Q, K, V = r1 Wq^T, r1 Wk^T, r1 Wv^T  (n_heads heads of d = H / n_heads)
+ *   Qr, Kr = Q, K with the rotary embedding: in every head, (x_i, x_{i+d/2})
+ *            -> (x_i c - x_{i+d/2} s, x_{i+d/2} c + x_i s), c, s = cos, sin of
+ *            t 10000^(-2i/d), t the token's position in its sample
+ *   O      = softmax(Qr Kr^T / sqrt(d) + causal mask) V per sample and head
+ *   X2     = X + O Wo^T;  r2 = bf16(rmsnorm(X2) gamma2)
+ *   Y      = X2 + (silu(r2 Wg^T) * (r2 Wu^T)) Wd^T
+ * Rounding points (each operand of a product is bf16, the rest fp32): r1, Qr,
+ * Kr, V, the attention probabilities P = bf16(exp(z - lse)) (z the scaled
+ * scores, lse the row's log-sum-exp over its keys), O, r2, the MLP's a, b, h;
+ * X2 and Y are fp32.  In the backward: G, dA, dB, dX2 (the gradient at X2),
+ * dO, dS (the softmax gradient times 1/sqrt(d)), dQ, dK (after the inverse
+ * rotation) and dV are bf16.
+ * layers: seven ar_layer in the order q, k, v, o, gate, up, down; q, k, v, o
+ * [H][H], gate, up [F][H], down [H][F]. */
+typedef struct {
+  int64_t hidden;       /* H: a multiple of 128 */
+  int64_t intermediate; /* F: a multiple of 8 */
+  int n_heads;          /* head dim d = H / n_heads, 64 or 128 */
+  int64_t seq_len;      /* L: tokens per sample, a multiple of 64; M % L == 0 */
+  const float* gamma1;  /* device fp32 [H], the two norms' scales (not tuned) */
+  const float* gamma2;
+} ar_decoder_cfg;
+
+/* Bytes of workspace ar_decoder_forward needs (0 on invalid input). */
+AR_API size_t ar_decoder_forward_workspace(const ar_decoder_cfg* dcfg, int64_t M);
+
+/* The block's output with its original weights ([AR] §3 "Algorithm Flow" step
+ * 2): Y fp32 [M][H].  Only layers[i].W are read.  Workspace: device, 256-byte
+ * aligned.  Errors: AR_ERR_INVALID_ARG / AR_ERR_UNSUPPORTED /
+ * AR_ERR_WORKSPACE before any launch. */
+AR_API ar_status ar_decoder_forward(const ar_decoder_cfg* dcfg, const ar_layer* layers, const uint16_t* X, int64_t M,
+                                    float* Y, void* workspace, size_t workspace_bytes, ar_stream_t stream);
+
+/* Bytes of workspace ar_tune_step_decoder needs (0 on invalid input). */
+AR_API size_t ar_tune_step_decoder_workspace(const ar_decoder_cfg* dcfg, const ar_layer* layers, int64_t M,
+                                             const ar_qconfig* cfg, int n_steps);
+
+/* n_steps joint SignSGD steps on the block's seven weights ([AR] §3
+ * "Algorithm Flow" steps 3-5, "SignSGD"; straight-through fold as in
+ * ar_tune_step): QDQ of the seven weights, the block forward above with the
+ * fake-quantized weights, R = Y_hat - Y, loss = sum R^2 / (M H),
+ * G = bf16(2R/(M H)), the block's backward to the seven dW_hat, each folded
+ * into dV, dalpha, dbeta and applied as p <- clamp(p - lr sign(dp)).
+ * Y: fp32 [M][H] from ar_decoder_forward.  loss_per_step, n_steps, grads (an
+ * array of seven, or NULL) and the in-place updates as in ar_tune_step.
+ * Supported: bits 2..8, group_size 32..256 dividing H and F, the shapes of
+ * ar_decoder_cfg.  Errors before any launch as ar_tune_step. */
+AR_API ar_status ar_tune_step_decoder(const ar_decoder_cfg* dcfg, const ar_layer* layers, const uint16_t* X,
+                                      int64_t M, const float* Y, const ar_qconfig* cfg, int n_steps,
+                                      float* loss_per_step, const ar_grads* grads, void* workspace,
+                                      size_t workspace_bytes, ar_stream_t stream);
+
+/* The block's parts on their own (the tuning step runs exactly these kernels):
+ * r [M][H] bf16 = bf16(rmsnorm(x) gamma) and inv [M] fp32 = 1/sqrt(mean(x^2) +
+ * 1e-6) (inv may be NULL); x bf16 (x_is_f32 = 0) or fp32 [M][H]; H % 8 == 0. */
+AR_API ar_status ar_rmsnorm(const void* x, int x_is_f32, const float* gamma, int64_t M, int64_t H, uint16_t* r,
+                            float* inv, ar_stream_t stream);
+
+/* Causal softmax attention per sample and head on qkv [S*L][3H] bf16 (columns
+ * Qr | Kr | V, the rotation already applied): out [S*L][H] bf16 = P V with
+ * P = bf16(exp(z - lse)), z = Qr Kr^T / sqrt(d) (fp32), and lse fp32 [S][nh][L].
+ * Needs L % 64 == 0, d = H / n_heads in {64, 128}. */
+AR_API ar_status ar_attention_forward(const uint16_t* qkv, int64_t S, int64_t L, int64_t H, int n_heads,
+                                      uint16_t* out, float* lse, ar_stream_t stream);
+
+/* Its backward from dO [S*L][H] bf16: dqkv [S*L][3H] bf16 = dQ | dK | dV, with
+ * dQ and dK taken back through the rotation (dQ = R^T dQr).  out and lse are
+ * the forward's.  Workspace: ar_attention_backward_workspace bytes (device,
+ * 256-byte aligned). */
+AR_API size_t ar_attention_backward_workspace(int64_t S, int64_t L, int64_t H, int n_heads);
+AR_API ar_status ar_attention_backward(const uint16_t* qkv, const uint16_t* out, const uint16_t* dout,
+                                       const float* lse, int64_t S, int64_t L, int64_t H, int n_heads,
+                                       uint16_t* dqkv, void* workspace, size_t workspace_bytes,
+                                       ar_stream_t stream);
+
 /* Fixed scratch size of ar_tune_step_noalloc, in bytes (16 MiB per GPU). */
 #define AR_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
 

@@ -854,12 +854,35 @@ def nvfp4_tune_step_linear(Wb, Xb, Y, V, alpha, cfg: QConfig, amax=None, count: 
 # * the seven linear weights (q, k, v, o, gate, up, down) are fake-quantized with
 #   their own V, alpha, beta and tuned jointly from the MSE of Y.
 # This section is in fp64 after the QDQ (whose codes are decided in fp32 as
-# everywhere in this module); the rounding points a GPU path shares with it are
-# fixed together with that path.
+# everywhere in this module).  With ``rounding=True`` it applies the rounding
+# points a GPU path shares with it, in the same order (no page fixes them; the
+# rule is that every operand of a matrix product is bf16 and everything else is
+# fp32):
+# * bf16: r1, r2 (normalised inputs of the projections), Qr, Kr (after the
+#   rotation), V, the attention probabilities P, the attention output O, a, b,
+#   h of the MLP, G, dA, dB, dX2, dO, dS (the softmax gradient times 1/sqrt(d)),
+#   dQ, dK (after the inverse rotation), dV;
+# * fp32: the products' results (Q, K before the rotation, the scores z, Ŷ
+#   parts, dH, dr2, dP, dQr, dKr), the residual stream X2 and Ŷ, R, the row
+#   statistic D = rowsum(dO ⊙ O); the scale 1/sqrt(d) and the rotation's
+#   cos/sin are fp32 constants;
+# * the probabilities come from a two-pass softmax, P = exp(z - lse) with
+#   lse = log sum_j exp(z_j) over the row's keys, so that their rounding to bf16
+#   does not depend on the order in which keys are visited; O = P V is then
+#   the normalised output (no division after the product).
 
 RMS_EPS = 1e-6
 ROPE_BASE = 10000.0
 DECODER_LAYERS = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+def _rounders(rounding: bool):
+    """(to_bf16, to_fp32) as fp64 arrays when rounding, else the identity."""
+    if not rounding:
+        ident = lambda x: np.asarray(x, f64)
+        return ident, ident
+    return (lambda x: bf16_rne(np.asarray(x, f64).astype(f32)).astype(f64),
+            lambda x: np.asarray(x, f64).astype(f32).astype(f64))
 
 
 def rmsnorm(x, gamma):
@@ -876,20 +899,23 @@ def rmsnorm_backward(x, gamma, inv, dy):
     return inv * gdy - x * inv ** 3 * np.mean(gdy * x, axis=-1, keepdims=True)
 
 
-def rope_angles(L: int, d: int):
-    """cos, sin [L][d/2] of the angles t * base^(-2i/d)."""
+def rope_angles(L: int, d: int, rounding: bool = False):
+    """cos, sin [L][d/2] of the angles t * base^(-2i/d) (fp32 constants when rounding)."""
     i = np.arange(d // 2, dtype=f64)
     ang = np.arange(L, dtype=f64)[:, None] * ROPE_BASE ** (-2.0 * i / d)[None, :]
-    return np.cos(ang), np.sin(ang)
+    c, s = np.cos(ang), np.sin(ang)
+    if rounding:
+        c, s = c.astype(f32).astype(f64), s.astype(f32).astype(f64)
+    return c, s
 
 
-def rope(x, nh: int, sign: float = 1.0):
+def rope(x, nh: int, sign: float = 1.0, rounding: bool = False):
     """Rotate each head of x [S][L][H]: (x_i, x_{i+d/2}) -> (x_i cos - x_{i+d/2} sin, x_{i+d/2} cos + x_i sin);
     ``sign`` = -1 rotates back (the transpose, used by the backward)."""
     x = np.asarray(x, f64)
     S, L, H = x.shape
     d = H // nh
-    c, s = rope_angles(L, d)
+    c, s = rope_angles(L, d, rounding)
     s = sign * s
     xh = x.reshape(S, L, nh, d)
     x1, x2 = xh[..., : d // 2], xh[..., d // 2:]
@@ -897,59 +923,78 @@ def rope(x, nh: int, sign: float = 1.0):
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1).reshape(S, L, H)
 
 
-def attention_forward(Q, K, V, nh: int):
-    """Causal softmax attention per sample and head: P = softmax(Q Kᵀ / sqrt(d) + mask), O = P V."""
+def attention_scale(d: int, rounding: bool = False):
+    return float(f32(1.0 / np.sqrt(d))) if rounding else 1.0 / np.sqrt(d)
+
+
+def attention_forward(Q, K, V, nh: int, rounding: bool = False):
+    """Causal softmax attention per sample and head: z = Q Kᵀ / sqrt(d) (keys up to the query's
+    position), lse = log sum exp(z) over those keys, P = exp(z - lse), O = P V.
+    Returns O [S][L][H], P [S][nh][L][L] and lse [S][nh][L]."""
+    rb, rf = _rounders(rounding)
     S, L, H = Q.shape
     d = H // nh
     q = Q.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
     k = K.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
     v = V.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
-    z = q @ k.transpose(0, 1, 3, 2) / np.sqrt(d)
-    z = np.where(np.tril(np.ones((L, L), bool))[None, None], z, -np.inf)
-    z = z - z.max(axis=-1, keepdims=True)
-    p = np.exp(z)
-    p = p / p.sum(axis=-1, keepdims=True)
-    o = p @ v
-    return o.transpose(0, 2, 1, 3).reshape(S, L, H), p
+    z = rf(rf(q @ k.transpose(0, 1, 3, 2)) * attention_scale(d, rounding))
+    causal = np.tril(np.ones((L, L), bool))[None, None]
+    z = np.where(causal, z, -np.inf)
+    m = z.max(axis=-1, keepdims=True)
+    lse = m + np.log(np.sum(np.exp(z - m), axis=-1, keepdims=True))
+    p = rb(np.exp(z - lse))
+    o = rb(p @ v)
+    return o.transpose(0, 2, 1, 3).reshape(S, L, H), p, lse[..., 0]
 
 
-def attention_backward(Q, K, V, P, dO, nh: int):
-    """dQ, dK, dV of attention_forward: dP = dO Vᵀ, dV = Pᵀ dO, dZ = P (dP - rowsum(dP P)),
-    dQ = dZ K / sqrt(d), dK = dZᵀ Q / sqrt(d)."""
+def attention_backward(Q, K, V, P, dO, nh: int, rounding: bool = False, O=None):
+    """dQ, dK, dV of attention_forward: dP = dO Vᵀ, dV = Pᵀ dO, D = rowsum(dO ⊙ O) (= rowsum(dP ⊙ P)),
+    dS = P (dP - D) / sqrt(d), dQ = dS K, dK = dSᵀ Q."""
+    rb, rf = _rounders(rounding)
     S, L, H = Q.shape
     d = H // nh
-    split = lambda t: t.reshape(S, L, nh, d).transpose(0, 2, 1, 3)
+    split = lambda t: np.asarray(t, f64).reshape(S, L, nh, d).transpose(0, 2, 1, 3)
     merge = lambda t: t.transpose(0, 2, 1, 3).reshape(S, L, H)
     q, k, v, do = split(Q), split(K), split(V), split(dO)
-    dp = do @ v.transpose(0, 1, 3, 2)
-    dv = P.transpose(0, 1, 3, 2) @ do
-    dz = P * (dp - np.sum(dp * P, axis=-1, keepdims=True))
-    dq = dz @ k / np.sqrt(d)
-    dk = dz.transpose(0, 1, 3, 2) @ q / np.sqrt(d)
+    dp = rf(do @ v.transpose(0, 1, 3, 2))
+    dv = rb(P.transpose(0, 1, 3, 2) @ do)
+    if O is None:
+        D = np.sum(dp * P, axis=-1, keepdims=True)
+    else:
+        D = rf(np.sum(do * split(O), axis=-1, keepdims=True))
+    ds = rb(P * (dp - D) * attention_scale(d, rounding))
+    dq = rf(ds @ k)
+    dk = rf(ds.transpose(0, 1, 3, 2) @ q)
     return merge(dq), merge(dk), merge(dv)
 
 
-def decoder_forward(X, Wh, gammas, nh: int):
+def decoder_forward(X, Wh, gammas, nh: int, rounding: bool = False):
     """The block on X [S][L][H] with the seven weights Wh (dict by DECODER_LAYERS; q/k/v/o [H][H],
-    gate/up [F][H], down [H][F]) and gammas (γ1, γ2).  fp64; returns every intermediate."""
+    gate/up [F][H], down [H][F]) and gammas (γ1, γ2).  fp64 (with ``rounding``, the shared rounding
+    points); returns every intermediate."""
+    rb, rf = _rounders(rounding)
     X = np.asarray(X, f64)
     S, L, H = X.shape
     W = {n: np.asarray(Wh[n], f64) for n in DECODER_LAYERS}
     r1, inv1 = rmsnorm(X, gammas[0])
-    Qp, Kp, Vv = r1 @ W["q"].T, r1 @ W["k"].T, r1 @ W["v"].T
-    Qr, Kr = rope(Qp, nh), rope(Kp, nh)
-    O, P = attention_forward(Qr, Kr, Vv, nh)
-    X2 = X + O @ W["o"].T
+    r1 = rb(r1)
+    Qp, Kp, Vv = rf(r1 @ W["q"].T), rf(r1 @ W["k"].T), rb(r1 @ W["v"].T)
+    Qr, Kr = rb(rope(Qp, nh, 1.0, rounding)), rb(rope(Kp, nh, 1.0, rounding))
+    O, P, lse = attention_forward(Qr, Kr, Vv, nh, rounding)
+    X2 = rf(X + rf(O @ W["o"].T))
     r2, inv2 = rmsnorm(X2, gammas[1])
-    a, b = r2 @ W["gate"].T, r2 @ W["up"].T
-    h = silu(a) * b
-    Y = X2 + h @ W["down"].T
-    return {"X": X, "r1": r1, "inv1": inv1, "Qr": Qr, "Kr": Kr, "V": Vv, "P": P, "O": O, "X2": X2, "r2": r2,
-            "inv2": inv2, "a": a, "b": b, "h": h, "Y": Y}
+    r2 = rb(r2)
+    a, b = rb(r2 @ W["gate"].T), rb(r2 @ W["up"].T)
+    h = rb(silu(a) * b)
+    Y = rf(X2 + rf(h @ W["down"].T))
+    return {"X": X, "r1": r1, "inv1": inv1, "Qr": Qr, "Kr": Kr, "V": Vv, "P": P, "lse": lse, "O": O, "X2": X2,
+            "r2": r2, "inv2": inv2, "a": a, "b": b, "h": h, "Y": Y}
 
 
-def decoder_backward(fw, dY, Wh, gammas, nh: int):
-    """dL/dŴ for the seven weights from dY = dL/dY [S][L][H] (fp64)."""
+def decoder_backward(fw, dY, Wh, gammas, nh: int, rounding: bool = False):
+    """dL/dŴ for the seven weights from dY = dL/dY [S][L][H] (fp64; with ``rounding``, the shared
+    rounding points, dY being the bf16 G)."""
+    rb, rf = _rounders(rounding)
     W = {n: np.asarray(Wh[n], f64) for n in DECODER_LAYERS}
     S, L, H = fw["X"].shape
     flat = lambda t: t.reshape(S * L, -1)
@@ -957,21 +1002,24 @@ def decoder_backward(fw, dY, Wh, gammas, nh: int):
     g = {}
     # MLP and its norm: Y = X2 + h Wdᵀ
     g["down"] = flat(dY).T @ flat(fw["h"])
-    dh = dY @ W["down"]
-    da = dh * fw["b"] * silu_grad(fw["a"])
-    db = dh * silu(fw["a"])
+    dh = rf(dY @ W["down"])
+    da = rb(dh * fw["b"] * silu_grad(fw["a"]))
+    db = rb(dh * silu(fw["a"]))
     g["gate"] = flat(da).T @ flat(fw["r2"])
     g["up"] = flat(db).T @ flat(fw["r2"])
-    dr2 = da @ W["gate"] + db @ W["up"]
-    dX2 = dY + rmsnorm_backward(fw["X2"], gammas[1], fw["inv2"], dr2)
+    dr2 = rf(da @ W["gate"] + db @ W["up"])
+    dX2 = rb(dY + rmsnorm_backward(fw["X2"], gammas[1], fw["inv2"], dr2))
     # attention: X2 = X + O Woᵀ
     g["o"] = flat(dX2).T @ flat(fw["O"])
-    dO = dX2 @ W["o"]
-    dQr, dKr, dV = attention_backward(fw["Qr"], fw["Kr"], fw["V"], fw["P"], dO, nh)
-    dQ, dK = rope(dQr, nh, -1.0), rope(dKr, nh, -1.0)
+    dO = rb(dX2 @ W["o"])
+    dQr, dKr, dV = attention_backward(fw["Qr"], fw["Kr"], fw["V"], fw["P"], dO, nh, rounding,
+                                      O=fw["O"] if rounding else None)
+    dQ, dK = rb(rope(dQr, nh, -1.0, rounding)), rb(rope(dKr, nh, -1.0, rounding))
     g["q"] = flat(dQ).T @ flat(fw["r1"])
     g["k"] = flat(dK).T @ flat(fw["r1"])
     g["v"] = flat(dV).T @ flat(fw["r1"])
+    if rounding:
+        g = {n: rf(v) for n, v in g.items()}
     return g
 
 
@@ -991,15 +1039,22 @@ def decoder_smooth_grads(Ws, X, Y, states, gammas, nh, bits, group_size):
     return L, {n: ste_fold(gW[n], Ws[n], sts[n], bits) for n in DECODER_LAYERS}
 
 
-def tune_step_decoder(Ws, X, Y, states, gammas, nh: int, cfg: QConfig):
+def tune_step_decoder(Ws, X, Y, states, gammas, nh: int, cfg: QConfig, rounding: bool = False):
     """One joint SignSGD step on the seven weights of the block (QDQ in fp32 deciding the codes, the
-    block in fp64).  Returns (loss, new states, grads per layer)."""
+    block in fp64, or with ``rounding`` at the GPU path's rounding points: then the loss's gradient
+    G = bf16(2R/count) as for a single layer).  Returns (loss, new states, grads per layer)."""
     sts = {n: qdq(Ws[n], *states[n], cfg.bits, cfg.group_size, cfg.symmetric) for n in DECODER_LAYERS}
     Wh = {n: np.asarray(sts[n]["What_bf16"], f64) for n in DECODER_LAYERS}
-    fw = decoder_forward(X, Wh, gammas, nh)
-    R = fw["Y"] - np.asarray(Y, f64)
-    loss = float(np.sum(R ** 2) / R.size)
-    gW = decoder_backward(fw, 2.0 * R / R.size, Wh, gammas, nh)
+    fw = decoder_forward(X, Wh, gammas, nh, rounding)
+    if rounding:
+        R = (fw["Y"] - np.asarray(Y, f32)).astype(f32)
+        loss = float(np.sum(R.astype(f64) ** 2) / R.size)
+        dY = bf16_rne((R * f32(2.0 / float(R.size))).astype(f32)).astype(f64)
+    else:
+        R = fw["Y"] - np.asarray(Y, f64)
+        loss = float(np.sum(R ** 2) / R.size)
+        dY = 2.0 * R / R.size
+    gW = decoder_backward(fw, dY, Wh, gammas, nh, rounding)
     new, grads = {}, {}
     for n in DECODER_LAYERS:
         dV, da, db = ste_fold(gW[n], Ws[n], sts[n], cfg.bits, cfg.symmetric)

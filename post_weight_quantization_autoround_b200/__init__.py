@@ -23,7 +23,9 @@ __all__ = [
     "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES", "AR_BLOCK_SWIGLU_MLP", "ar_block_forward",
     "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace", "ar_debug_wait_timeout",
     "ar_absmax_bf16", "ar_qdq_nvfp4", "ar_tune_step_nvfp4_workspace", "ar_tune_step_nvfp4",
-    "ar_tune_step_shard",
+    "ar_tune_step_shard", "DecoderCfg", "DECODER_LAYERS", "ar_decoder_forward_workspace", "ar_decoder_forward",
+    "ar_tune_step_decoder_workspace", "ar_tune_step_decoder", "ar_rmsnorm", "ar_attention_forward",
+    "ar_attention_backward_workspace", "ar_attention_backward",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libautoround.so")
@@ -59,6 +61,13 @@ class Grads(ctypes.Structure):
     _fields_ = [("dV", ctypes.c_void_p), ("dalpha", ctypes.c_void_p), ("dbeta", ctypes.c_void_p)]
 
 
+class DecoderCfg(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int64), ("intermediate", ctypes.c_int64), ("n_heads", ctypes.c_int),
+                ("seq_len", ctypes.c_int64), ("gamma1", ctypes.c_void_p), ("gamma2", ctypes.c_void_p)]
+
+
+DECODER_LAYERS = ("q", "k", "v", "o", "gate", "up", "down")
+
 _lib = None
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -74,6 +83,18 @@ _SIGNATURES = {
                             ctypes.POINTER(Grads), _P, ctypes.c_size_t, _P]),
     "ar_tune_step_shard": (_INT, [ctypes.POINTER(Layer), _P, _I64, _P, _I64, ctypes.POINTER(QConfig), _INT, _P,
                                   ctypes.POINTER(Grads), _P, ctypes.c_size_t, _P]),
+    "ar_decoder_forward_workspace": (ctypes.c_size_t, [ctypes.POINTER(DecoderCfg), _I64]),
+    "ar_decoder_forward": (_INT, [ctypes.POINTER(DecoderCfg), ctypes.POINTER(Layer), _P, _I64, _P, _P, ctypes.c_size_t,
+                                  _P]),
+    "ar_tune_step_decoder_workspace": (ctypes.c_size_t, [ctypes.POINTER(DecoderCfg), ctypes.POINTER(Layer), _I64,
+                                                         ctypes.POINTER(QConfig), _INT]),
+    "ar_tune_step_decoder": (_INT, [ctypes.POINTER(DecoderCfg), ctypes.POINTER(Layer), _P, _I64, _P,
+                                    ctypes.POINTER(QConfig), _INT, _P, ctypes.POINTER(Grads), _P, ctypes.c_size_t,
+                                    _P]),
+    "ar_rmsnorm": (_INT, [_P, _INT, _P, _I64, _I64, _P, _P, _P]),
+    "ar_attention_forward": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "ar_attention_backward_workspace": (ctypes.c_size_t, [_I64, _I64, _I64, _INT]),
+    "ar_attention_backward": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _INT, _P, _P, ctypes.c_size_t, _P]),
     "ar_pack_int4": (_INT, [_P, _P, _P, _P, _I64, _I64, ctypes.POINTER(QConfig), _P, _P, _P, _P]),
     "ar_w4a16_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _P, _P]),
     "ar_gemm_bf16": (_INT, [_P, _INT, _P, _INT, _P, _I64, _I64, _I64, _P]),
@@ -413,3 +434,77 @@ class LinearTuner:
                      self.workspace, stream=stream)
         for dst, src in ((V, self.V), (alpha, self.alpha), (beta, self.beta), (loss, self.loss)):
             dst.copy_(src, non_blocking=True)
+
+
+# ---- decoder block ----------------------------------------------------------
+
+def _decoder_cfg(H: int, F: int, n_heads: int, seq_len: int, gamma1, gamma2) -> DecoderCfg:
+    return DecoderCfg(H, F, n_heads, seq_len, _ptr(gamma1), _ptr(gamma2))
+
+
+def ar_decoder_forward_workspace(H: int, F: int, n_heads: int, seq_len: int, M: int) -> int:
+    d = DecoderCfg(H, F, n_heads, seq_len, None, None)
+    n = lib().ar_decoder_forward_workspace(ctypes.byref(d), M)
+    if n == 0:
+        raise ARError(AR_ERR_INVALID_ARG, ar_last_error())
+    return int(n)
+
+
+def ar_decoder_forward(weights, gamma1, gamma2, n_heads: int, seq_len: int, X, Y, workspace, stream=None) -> None:
+    """Block output with the original weights; ``weights``: seven W tensors in DECODER_LAYERS order."""
+    H, F = weights[0].shape[0], weights[4].shape[0]
+    d = _decoder_cfg(H, F, n_heads, seq_len, gamma1, gamma2)
+    arr = _layers([(W, None, None, None) for W in weights])
+    _check(lib().ar_decoder_forward(ctypes.byref(d), arr, _ptr(X), X.shape[0], _ptr(Y), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def ar_tune_step_decoder_workspace(layers, gamma1, gamma2, n_heads: int, seq_len: int, M: int, cfg: QConfig,
+                                   n_steps: int) -> int:
+    H, F = layers[0][0].shape[0], layers[4][0].shape[0]
+    d = _decoder_cfg(H, F, n_heads, seq_len, gamma1, gamma2)
+    n = lib().ar_tune_step_decoder_workspace(ctypes.byref(d), _layers(layers), M, ctypes.byref(cfg), n_steps)
+    if n == 0:
+        raise ARError(AR_ERR_INVALID_ARG, ar_last_error())
+    return int(n)
+
+
+def ar_tune_step_decoder(layers, gamma1, gamma2, n_heads: int, seq_len: int, X, Y, cfg: QConfig, n_steps: int, loss,
+                         workspace, grads=None, stream=None) -> None:
+    """Joint steps on the decoder block; ``layers``: seven (W, V, alpha, beta) in DECODER_LAYERS order."""
+    H, F = layers[0][0].shape[0], layers[4][0].shape[0]
+    d = _decoder_cfg(H, F, n_heads, seq_len, gamma1, gamma2)
+    gp = None
+    if grads is not None:
+        g = (Grads * len(layers))()
+        for i, (dv, da, db) in enumerate(grads):
+            g[i] = Grads(_ptr(dv), _ptr(da), _ptr(db))
+        gp = g
+    _check(lib().ar_tune_step_decoder(ctypes.byref(d), _layers(layers), _ptr(X), X.shape[0], _ptr(Y),
+                                      ctypes.byref(cfg), n_steps, _ptr(loss), gp, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def ar_rmsnorm(x, gamma, r, inv=None, stream=None) -> None:
+    M, H = x.shape
+    _check(lib().ar_rmsnorm(_ptr(x), int(x.dtype == torch.float32), _ptr(gamma), M, H, _ptr(r), _ptr(inv),
+                            _stream(stream)))
+
+
+def ar_attention_forward(qkv, S: int, L: int, n_heads: int, out, lse, stream=None) -> None:
+    H = qkv.shape[1] // 3
+    _check(lib().ar_attention_forward(_ptr(qkv), S, L, H, n_heads, _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def ar_attention_backward_workspace(S: int, L: int, H: int, n_heads: int) -> int:
+    n = lib().ar_attention_backward_workspace(S, L, H, n_heads)
+    if n == 0:
+        raise ARError(AR_ERR_INVALID_ARG, ar_last_error())
+    return int(n)
+
+
+def ar_attention_backward(qkv, out, dout, lse, S: int, L: int, n_heads: int, dqkv, workspace, stream=None) -> None:
+    H = qkv.shape[1] // 3
+    _check(lib().ar_attention_backward(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), S, L, H, n_heads, _ptr(dqkv),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))

@@ -312,6 +312,250 @@ ar_status tune_linear(const ar_layer* layers, int n_layers, const uint16_t* X, i
   if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
   return end_call();
 }
+
+// ---- decoder block ----------------------------------------------------------
+// Workspace of the decoder block (H hidden, F intermediate, M tokens, L per sample).
+struct DecWs {
+  size_t wqkv, wo, wgu, wd;             // bf16 fake-quantized (or original) weights, stacked where one GEMM reads them
+  size_t sc[7], zp[7], mx[7], mn[7];    // per-layer group parameters
+  size_t rope, r1, qkv, o, lse, x2, inv2, r2, a, b, h, g, dab, dr2, dx2, dout, dsum, dqkv, partial, total;
+  int partials_per_step;
+};
+
+constexpr int kDecLayers = 7;  // q, k, v, o, gate, up, down
+
+DecWs dec_ws(int64_t M, int64_t H, int64_t F, int64_t L, int head_dim, int g, int n_steps, bool tune) {
+  DecWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  w.wqkv = take(static_cast<size_t>(3 * H * H) * 2);
+  w.wo = take(static_cast<size_t>(H * H) * 2);
+  w.wgu = take(static_cast<size_t>(2 * F * H) * 2);
+  w.wd = take(static_cast<size_t>(H * F) * 2);
+  if (tune) {
+    const int64_t NK[kDecLayers] = {H * H, H * H, H * H, H * H, F * H, F * H, H * F};
+    for (int i = 0; i < kDecLayers; ++i) {
+      const size_t groups = static_cast<size_t>(NK[i] / g) * 4;
+      w.sc[i] = take(groups);
+      w.zp[i] = take(groups);
+      w.mx[i] = take(groups);
+      w.mn[i] = take(groups);
+    }
+  }
+  const size_t MH = static_cast<size_t>(M * H), MF = static_cast<size_t>(M * F);
+  const size_t rows = static_cast<size_t>(M / L) * static_cast<size_t>(H / head_dim) * static_cast<size_t>(L);
+  w.rope = take(static_cast<size_t>(L) * head_dim / 2 * 8);
+  w.r1 = take(MH * 2);
+  w.qkv = take(3 * MH * 2);
+  w.o = take(MH * 2);
+  w.lse = take(rows * 4);
+  w.x2 = take(MH * 4);
+  w.inv2 = take(static_cast<size_t>(M) * 4);
+  w.r2 = take(MH * 2);
+  w.a = take(MF * 2);
+  w.b = take(MF * 2);
+  w.h = take(MF * 2);
+  if (tune) {
+    w.g = take(MH * 2);
+    w.dab = take(2 * MF * 2);
+    w.dr2 = take(MH * 4);
+    w.dx2 = take(MH * 2);
+    w.dout = take(MH * 2);
+    w.dsum = take(rows * 4);
+    w.dqkv = take(3 * MH * 2);
+    w.partials_per_step = resid_partials(static_cast<int>(M), static_cast<int>(H));
+    w.partial = take(static_cast<size_t>(w.partials_per_step) * (n_steps > 0 ? n_steps : 1) * 8);
+  }
+  w.total = off;
+  return w;
+}
+
+ar_status check_decoder(const ar_decoder_cfg* d, const ar_layer* L, int64_t M, const ar_qconfig* cfg, bool tune) {
+  if (!d) return fail(AR_ERR_INVALID_ARG, "decoder config is NULL");
+  const int64_t H = d->hidden, F = d->intermediate, Ls = d->seq_len;
+  if (H <= 0 || F <= 0 || Ls <= 0 || M <= 0 || d->n_heads <= 0)
+    return fail(AR_ERR_INVALID_ARG, "sizes must be positive");
+  if (H % d->n_heads != 0) return fail(AR_ERR_INVALID_ARG, "H=%lld is not a multiple of n_heads", (long long)H);
+  const int64_t hd = H / d->n_heads;
+  if (hd != 64 && hd != 128) return fail(AR_ERR_UNSUPPORTED, "head dim %lld: needs 64 or 128", (long long)hd);
+  if (H % 128 != 0 || F % 8 != 0) return fail(AR_ERR_INVALID_ARG, "H must be a multiple of 128 and F of 8");
+  if (Ls % 64 != 0 || M % Ls != 0) return fail(AR_ERR_INVALID_ARG, "seq_len must be a multiple of 64 dividing M");
+  if (3 * H * M > INT32_MAX * 8ll || 3 * H > INT32_MAX || M > INT32_MAX || F > INT32_MAX)
+    return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  if (!d->gamma1 || !d->gamma2 || !aligned16(d->gamma1) || !aligned16(d->gamma2))
+    return fail(AR_ERR_INVALID_ARG, "gamma1, gamma2 must be 16-byte aligned device pointers");
+  if (!L) return fail(AR_ERR_INVALID_ARG, "layers is NULL");
+  const int64_t shp[kDecLayers][2] = {{H, H}, {H, H}, {H, H}, {H, H}, {F, H}, {F, H}, {H, F}};
+  for (int i = 0; i < kDecLayers; ++i) {
+    if (L[i].N != shp[i][0] || L[i].K != shp[i][1])
+      return fail(AR_ERR_INVALID_ARG, "layer %d: shape [%lld][%lld], expected [%lld][%lld] (q, k, v, o, gate, up, down)",
+                  i, (long long)L[i].N, (long long)L[i].K, (long long)shp[i][0], (long long)shp[i][1]);
+    if (!L[i].W || !aligned16(L[i].W)) return fail(AR_ERR_INVALID_ARG, "layer %d: W must be 16-byte aligned", i);
+    if (tune && (!L[i].V || !L[i].alpha || !L[i].beta || !aligned16(L[i].V) || !aligned16(L[i].alpha) ||
+                 !aligned16(L[i].beta)))
+      return fail(AR_ERR_INVALID_ARG, "layer %d: V, alpha, beta must be 16-byte aligned", i);
+  }
+  if (tune) {
+    ar_status st = check_cfg(cfg);
+    if (st != AR_OK) return st;
+    const int g = cfg->group_size;
+    if (g != 32 && g != 64 && g != 128 && g != 256)
+      return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs 32, 64, 128 or 256", g);
+    if (H % g != 0 || F % g != 0) return fail(AR_ERR_INVALID_ARG, "H and F must be multiples of group_size");
+  }
+  return AR_OK;
+}
+
+// The block forward from r1 on (the QKV, attention, residual, norm and MLP launches);
+// with G != nullptr the last GEMM is the loss epilogue, else Y = X2 + h Wd^T.
+ar_status decoder_forward_launches(const ar_decoder_cfg* d, const DecWs& w, uint8_t* ws, const uint16_t* X, int64_t M,
+                                   float* Y_out, const float* Y_ref, uint16_t* G, float gscale, double* partial,
+                                   cudaStream_t s) {
+  auto bf = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
+  auto f32p = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  const int Mi = static_cast<int>(M), Hi = static_cast<int>(d->hidden), Fi = static_cast<int>(d->intermediate);
+  const int Li = static_cast<int>(d->seq_len), hd = static_cast<int>(d->hidden / d->n_heads);
+  const int S = Mi / Li;
+  cudaError_t e = launch_gemm_qkv(bf(w.r1), bf(w.wqkv), bf(w.qkv), f32p(w.rope), Mi, Hi, Li, hd, s);
+  if (e != cudaSuccess) return cuda_fail(e, "QKV GEMM launch");
+  e = launch_attn_fwd(bf(w.qkv), S, Li, Hi, hd, bf(w.o), f32p(w.lse), s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  e = launch_gemm_resadd(bf(w.o), bf(w.wo), X, nullptr, f32p(w.x2), Mi, Hi, Hi, s);
+  if (e != cudaSuccess) return cuda_fail(e, "output projection GEMM launch");
+  e = launch_rmsnorm_fwd(f32p(w.x2), true, d->gamma2, M, Hi, bf(w.r2), f32p(w.inv2), s);
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+  e = launch_gemm_swiglu_fwd(bf(w.r2), bf(w.wgu), bf(w.wgu) + static_cast<size_t>(Fi) * Hi, bf(w.a), bf(w.b),
+                             bf(w.h), Mi, Fi, Hi, s);
+  if (e != cudaSuccess) return cuda_fail(e, "SwiGLU forward GEMM launch");
+  if (G) e = launch_gemm_resid(bf(w.h), bf(w.wd), Y_ref, G, gscale, partial, Mi, Hi, Fi, s, f32p(w.x2));
+  else e = launch_gemm_resadd(bf(w.h), bf(w.wd), nullptr, f32p(w.x2), Y_out, Mi, Hi, Fi, s);
+  if (e != cudaSuccess) return cuda_fail(e, "down-projection GEMM launch");
+  return AR_OK;
+}
+
+ar_status decoder_tune(const ar_decoder_cfg* d, const ar_layer* L, const uint16_t* X, int64_t M, const float* Y,
+                       const ar_qconfig* cfg, int n_steps, float* loss_per_step, const ar_grads* grads,
+                       void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  ar_status st = check_decoder(d, L, M, cfg, true);
+  if (st != AR_OK) return st;
+  if (n_steps < 0) return fail(AR_ERR_INVALID_ARG, "n_steps must be >= 0");
+  if (!X || !Y || !loss_per_step || !aligned16(X) || !aligned16(Y))
+    return fail(AR_ERR_INVALID_ARG, "X, Y (16-byte aligned) and loss_per_step are required");
+  const int64_t H = d->hidden, F = d->intermediate;
+  const int hd = static_cast<int>(H / d->n_heads);
+  const DecWs w = dec_ws(M, H, F, d->seq_len, hd, cfg->group_size, n_steps, true);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (grads) {
+    for (int i = 0; i < kDecLayers; ++i) {
+      const void* gp[] = {grads[i].dV, grads[i].dalpha, grads[i].dbeta};
+      for (const void* p : gp)
+        if (p && !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "gradient outputs must be 16-byte aligned");
+    }
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto bf = [&](size_t off) { return reinterpret_cast<uint16_t*>(ws + off); };
+  auto f32p = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  const int Mi = static_cast<int>(M), Hi = static_cast<int>(H), Fi = static_cast<int>(F);
+  const int Li = static_cast<int>(d->seq_len), S = Mi / Li;
+  // Where each layer's W_hat goes: q, k, v stacked, gate and up stacked.
+  uint16_t* what[kDecLayers] = {bf(w.wqkv), bf(w.wqkv) + static_cast<size_t>(H) * H,
+                                bf(w.wqkv) + 2 * static_cast<size_t>(H) * H, bf(w.wo), bf(w.wgu),
+                                bf(w.wgu) + static_cast<size_t>(F) * H, bf(w.wd)};
+  const double count = static_cast<double>(M) * static_cast<double>(H);
+  const float gscale = static_cast<float>(2.0 / count);
+  double* partial = reinterpret_cast<double*>(ws + w.partial);
+  cudaError_t e = launch_rope_table(Li, hd, f32p(w.rope), s);
+  if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  // r1 = rmsnorm(X) gamma1 does not depend on the tuned parameters: once per call
+  e = launch_rmsnorm_fwd(X, false, d->gamma1, M, Hi, bf(w.r1), nullptr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+  const int steps = n_steps > 0 ? n_steps : 1;
+  for (int step = 0; step < steps; ++step) {
+    for (int i = 0; i < kDecLayers; ++i) {
+      e = launch_qdq(L[i].W, L[i].V, L[i].alpha, L[i].beta, L[i].N, L[i].K, cfg->group_size, cfg->bits,
+                     cfg->symmetric, what[i], nullptr, f32p(w.sc[i]), f32p(w.zp[i]), f32p(w.mx[i]), f32p(w.mn[i]), s);
+      if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+    }
+    st = decoder_forward_launches(d, w, ws, X, M, nullptr, Y, bf(w.g), gscale,
+                                  partial + static_cast<size_t>(step) * w.partials_per_step, s);
+    if (st != AR_OK) return st;
+    if (n_steps == 0) break;
+    const bool last = step == steps - 1;
+    auto fa = [&](int i) {
+      return fold_args(L[i], cfg, f32p(w.sc[i]), f32p(w.zp[i]), f32p(w.mx[i]), f32p(w.mn[i]),
+                       (last && grads) ? &grads[i] : nullptr);
+    };
+    // MLP: dWd = G^T h; dH = G Wd -> dA, dB (one [M][2F] buffer); dWg = dA^T r2, dWu = dB^T r2
+    e = launch_gemm_fold(bf(w.g), bf(w.h), fa(6), Mi, Hi, Fi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "down weight-gradient GEMM launch");
+    e = launch_gemm_swiglu_bwd(bf(w.g), bf(w.wd), bf(w.a), bf(w.b), bf(w.dab), bf(w.dab) + Fi, Mi, Fi, Hi, s, 2 * Fi);
+    if (e != cudaSuccess) return cuda_fail(e, "SwiGLU backward GEMM launch");
+    e = launch_gemm_fold(bf(w.dab), bf(w.r2), fa(4), Mi, Fi, Hi, s, 2 * F, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "gate weight-gradient GEMM launch");
+    e = launch_gemm_fold(bf(w.dab) + Fi, bf(w.r2), fa(5), Mi, Fi, Hi, s, 2 * F, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "up weight-gradient GEMM launch");
+    // dr2 = [dA | dB] [Wg ; Wu] (fp32), then the norm's backward plus the residual path: dX2 (bf16)
+    e = launch_gemm_plain(bf(w.dab), false, bf(w.wgu), true, f32p(w.dr2), Mi, Hi, 2 * Fi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "norm-input gradient GEMM launch");
+    e = launch_rmsnorm_bwd(f32p(w.x2), f32p(w.inv2), d->gamma2, f32p(w.dr2), bf(w.g), M, Hi, bf(w.dx2), s);
+    if (e != cudaSuccess) return cuda_fail(e, "rmsnorm backward launch");
+    // attention output projection: dWo = dX2^T O; dO = dX2 Wo
+    e = launch_gemm_fold(bf(w.dx2), bf(w.o), fa(3), Mi, Hi, Hi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "o weight-gradient GEMM launch");
+    e = launch_gemm_store_bf16_kmn(bf(w.dx2), bf(w.wo), bf(w.dout), Mi, Hi, Hi, s);
+    if (e != cudaSuccess) return cuda_fail(e, "attention-output gradient GEMM launch");
+    // attention backward -> dQ | dK | dV, then dWq, dWk, dWv = d(.)^T r1
+    e = launch_attn_bwd(bf(w.qkv), bf(w.o), bf(w.dout), f32p(w.lse), f32p(w.dsum), f32p(w.rope), S, Li, Hi, hd,
+                        bf(w.dqkv), s);
+    if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");
+    for (int i = 0; i < 3; ++i) {
+      e = launch_gemm_fold(bf(w.dqkv) + static_cast<size_t>(i) * Hi, bf(w.r1), fa(i), Mi, Hi, Hi, s, 3 * H, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "q/k/v weight-gradient GEMM launch");
+    }
+  }
+  e = launch_loss_reduce(partial, w.partials_per_step, steps, 1.0 / count, loss_per_step, s);
+  if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");
+  return end_call();
+}
+
+ar_status decoder_reference(const ar_decoder_cfg* d, const ar_layer* L, const uint16_t* X, int64_t M, float* Y,
+                            void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  ar_status st = check_decoder(d, L, M, nullptr, false);
+  if (st != AR_OK) return st;
+  if (!X || !Y || !aligned16(X) || !aligned16(Y)) return fail(AR_ERR_INVALID_ARG, "X, Y must be 16-byte aligned");
+  const int64_t H = d->hidden, F = d->intermediate;
+  const int hd = static_cast<int>(H / d->n_heads);
+  const DecWs w = dec_ws(M, H, F, d->seq_len, hd, 32, 0, false);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t HH = static_cast<size_t>(H) * H * 2, FH = static_cast<size_t>(F) * H * 2;
+  // the original weights, stacked where one GEMM reads them
+  const struct {
+    size_t dst;
+    int layer;
+    size_t bytes;
+  } copies[] = {{w.wqkv, 0, HH}, {w.wqkv + HH, 1, HH}, {w.wqkv + 2 * HH, 2, HH}, {w.wo, 3, HH},
+                {w.wgu, 4, FH},  {w.wgu + FH, 5, FH},  {w.wd, 6, FH}};
+  for (const auto& c : copies) {
+    cudaError_t e = cudaMemcpyAsync(ws + c.dst, L[c.layer].W, c.bytes, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "weight copy");
+  }
+  cudaError_t e = launch_rope_table(static_cast<int>(d->seq_len), hd, reinterpret_cast<float*>(ws + w.rope), s);
+  if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  e = launch_rmsnorm_fwd(X, false, d->gamma1, M, static_cast<int>(H), reinterpret_cast<uint16_t*>(ws + w.r1), nullptr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+  st = decoder_forward_launches(d, w, ws, X, M, Y, nullptr, nullptr, 0.f, nullptr, s);
+  if (st != AR_OK) return st;
+  return end_call();
+}
 }  // namespace
 
 void set_last_error(const char* msg) { t_error = msg; }
@@ -851,6 +1095,111 @@ ar_status ar_profile_stop(char* buf, size_t buf_len) {
     buf[n] = 0;
   }
   return st;
+}
+
+size_t ar_decoder_forward_workspace(const ar_decoder_cfg* dcfg, int64_t M) {
+  begin_call();
+  if (!dcfg || dcfg->n_heads <= 0 || dcfg->hidden <= 0 || dcfg->hidden % dcfg->n_heads != 0 || dcfg->seq_len <= 0 ||
+      M <= 0 || M % dcfg->seq_len != 0) {
+    fail(AR_ERR_INVALID_ARG, "invalid decoder shapes");
+    return 0;
+  }
+  return dec_ws(M, dcfg->hidden, dcfg->intermediate, dcfg->seq_len, static_cast<int>(dcfg->hidden / dcfg->n_heads),
+                32, 0, false)
+      .total;
+}
+
+ar_status ar_decoder_forward(const ar_decoder_cfg* dcfg, const ar_layer* layers, const uint16_t* X, int64_t M,
+                             float* Y, void* workspace, size_t workspace_bytes, ar_stream_t stream) {
+  begin_call();
+  return decoder_reference(dcfg, layers, X, M, Y, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ar_tune_step_decoder_workspace(const ar_decoder_cfg* dcfg, const ar_layer* layers, int64_t M,
+                                      const ar_qconfig* cfg, int n_steps) {
+  begin_call();
+  if (n_steps < 0 || check_decoder(dcfg, layers, M, cfg, true) != AR_OK) {
+    if (t_error.empty()) fail(AR_ERR_INVALID_ARG, "invalid decoder block");
+    return 0;
+  }
+  return dec_ws(M, dcfg->hidden, dcfg->intermediate, dcfg->seq_len, static_cast<int>(dcfg->hidden / dcfg->n_heads),
+                cfg->group_size, n_steps, true)
+      .total;
+}
+
+ar_status ar_tune_step_decoder(const ar_decoder_cfg* dcfg, const ar_layer* layers, const uint16_t* X, int64_t M,
+                               const float* Y, const ar_qconfig* cfg, int n_steps, float* loss_per_step,
+                               const ar_grads* grads, void* workspace, size_t workspace_bytes, ar_stream_t stream) {
+  begin_call();
+  return decoder_tune(dcfg, layers, X, M, Y, cfg, n_steps, loss_per_step, grads, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+ar_status ar_rmsnorm(const void* x, int x_is_f32, const float* gamma, int64_t M, int64_t H, uint16_t* r, float* inv,
+                     ar_stream_t stream) {
+  begin_call();
+  if (M <= 0 || H <= 0 || H % 8 != 0 || H > INT32_MAX) return fail(AR_ERR_INVALID_ARG, "M > 0 and H a positive multiple of 8");
+  if (!x || !gamma || !r || !aligned16(x) || !aligned16(gamma) || !aligned16(r) || (inv && !aligned4(inv)))
+    return fail(AR_ERR_INVALID_ARG, "x, gamma, r must be 16-byte aligned device pointers");
+  cudaError_t e = launch_rmsnorm_fwd(x, x_is_f32 != 0, gamma, M, static_cast<int>(H), r, inv,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+  return end_call();
+}
+
+static ar_status check_attention(int64_t S, int64_t L, int64_t H, int n_heads) {
+  if (S <= 0 || L <= 0 || H <= 0 || n_heads <= 0) return fail(AR_ERR_INVALID_ARG, "sizes must be positive");
+  if (L % 64 != 0) return fail(AR_ERR_INVALID_ARG, "L=%lld must be a multiple of 64", (long long)L);
+  if (H % n_heads != 0 || (H / n_heads != 64 && H / n_heads != 128))
+    return fail(AR_ERR_UNSUPPORTED, "head dim H/n_heads must be 64 or 128");
+  if (S > 65535 || n_heads > 65535 || S * L * 3 * H > (int64_t(1) << 40)) return fail(AR_ERR_UNSUPPORTED, "too large");
+  return AR_OK;
+}
+
+ar_status ar_attention_forward(const uint16_t* qkv, int64_t S, int64_t L, int64_t H, int n_heads, uint16_t* out,
+                               float* lse, ar_stream_t stream) {
+  begin_call();
+  ar_status st = check_attention(S, L, H, n_heads);
+  if (st != AR_OK) return st;
+  if (!qkv || !out || !lse || !aligned16(qkv) || !aligned16(out) || !aligned16(lse))
+    return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  cudaError_t e = launch_attn_fwd(qkv, static_cast<int>(S), static_cast<int>(L), static_cast<int>(H),
+                                  static_cast<int>(H / n_heads), out, lse, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return end_call();
+}
+
+size_t ar_attention_backward_workspace(int64_t S, int64_t L, int64_t H, int n_heads) {
+  begin_call();
+  if (check_attention(S, L, H, n_heads) != AR_OK) return 0;
+  const int64_t hd = H / n_heads;
+  return align_up(static_cast<size_t>(L * hd / 2) * 8, 256) + align_up(static_cast<size_t>(S * n_heads * L) * 4, 256);
+}
+
+ar_status ar_attention_backward(const uint16_t* qkv, const uint16_t* out, const uint16_t* dout, const float* lse,
+                                int64_t S, int64_t L, int64_t H, int n_heads, uint16_t* dqkv, void* workspace,
+                                size_t workspace_bytes, ar_stream_t stream) {
+  begin_call();
+  ar_status st = check_attention(S, L, H, n_heads);
+  if (st != AR_OK) return st;
+  const void* ptrs[] = {qkv, out, dout, lse, dqkv};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const int64_t hd = H / n_heads;
+  const size_t rope_bytes = align_up(static_cast<size_t>(L * hd / 2) * 8, 256);
+  const size_t need = rope_bytes + align_up(static_cast<size_t>(S * n_heads * L) * 4, 256);
+  if (!workspace || workspace_bytes < need)
+    return fail(AR_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(AR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* cs = static_cast<float*>(workspace);
+  float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rope_bytes);
+  cudaError_t e = launch_rope_table(static_cast<int>(L), static_cast<int>(hd), cs, s);
+  if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  e = launch_attn_bwd(qkv, out, dout, lse, dsum, cs, static_cast<int>(S), static_cast<int>(L), static_cast<int>(H),
+                      static_cast<int>(hd), dqkv, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");
+  return end_call();
 }
 
 const char* ar_last_error(void) { return t_error.c_str(); }

@@ -16,6 +16,13 @@
 //              h = bf16(silu(a) b)  ([AR] §3 "Why Block-Wise Optimization")
 //   EPI_SWIGLU_BWD  dH = G W_down; SiLU backward: dA = bf16(dH b silu'(a)),
 //              dB = bf16(dH silu(a))
+//   EPI_QKV    the decoder block's stacked Q, K, V projection: bf16 out, with the
+//              rotary embedding applied to the Q and K columns (head halves
+//              (x_i, x_{i+d/2}) rotated by the position's angle, from a table)
+//   EPI_RESADD fp32 out = accumulator + a bf16 residual (X2 = X + O Wo^T)
+//   EPI_STORE_BF16  bf16 out (the attention output's gradient dO = dX2 Wo)
+// EPI_RESID optionally adds an fp32 residual before the difference: R = (acc +
+// X2) - Y, the decoder block's output Y_hat = X2 + h Wd^T.
 //
 // ([AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
 // Architectural Optimizations of AutoRound"; [IA] = "Intel AutoRound 高级量化".)
@@ -72,7 +79,16 @@ struct GemmCfg {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
-enum { EPI_STORE = 0, EPI_RESID = 1, EPI_FOLD = 2, EPI_SWIGLU_FWD = 3, EPI_SWIGLU_BWD = 4 };
+enum {
+  EPI_STORE = 0,
+  EPI_RESID = 1,
+  EPI_FOLD = 2,
+  EPI_SWIGLU_FWD = 3,
+  EPI_SWIGLU_BWD = 4,
+  EPI_QKV = 5,
+  EPI_RESADD = 6,
+  EPI_STORE_BF16 = 7
+};
 
 struct Ctl {
   uint64_t full[kMaxStages];
@@ -104,8 +120,14 @@ struct Params {
   uint16_t* act_a;   // EPI_SWIGLU_FWD outputs / EPI_SWIGLU_BWD inputs: a, b, h [M][N] bf16
   uint16_t* act_b;
   uint16_t* act_h;
-  uint16_t* grad_a;  // EPI_SWIGLU_BWD outputs: dA, dB [M][N] bf16
+  uint16_t* grad_a;  // EPI_SWIGLU_BWD outputs: dA, dB [M][ld_grad] bf16
   uint16_t* grad_b;
+  int ld_grad;
+  const float* Yadd;          // EPI_RESID: optional fp32 residual added before the difference
+  const uint16_t* res;        // EPI_RESADD: bf16 residual [M][N]
+  uint16_t* Dbf;              // EPI_QKV / EPI_STORE_BF16: bf16 out [M][N]
+  const float2* rope;         // EPI_QKV: (cos, sin) [rope_L][head_dim / 2]
+  int rope_cols, rope_L, head_dim;  // columns below rope_cols are rotated; position = row % rope_L
 };
 
 // Byte offsets of the MN-major canonical layout: the leading-dimension offset
@@ -158,6 +180,10 @@ __device__ __forceinline__ double epi_resid(const Params& p, uint32_t taddr, int
     if (row >= p.M || col0 >= p.N) continue;
     const float* y = p.Y + static_cast<size_t>(row) * p.N + col0;
     uint16_t* g = p.G + static_cast<size_t>(row) * p.N + col0;
+    if (p.Yadd) {
+      const float* ya = p.Yadd + static_cast<size_t>(row) * p.N + col0;
+      for (int i = 0; i < 32 && col0 + i < p.N; ++i) v[i] = __fadd_rn(v[i], ya[i]);
+    }
     float part = 0.0f;
     if (col0 + 32 <= p.N) {
       uint32_t gp[16];
@@ -415,6 +441,82 @@ __device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n,
   return bad;
 }
 
+// out = acc + residual (bf16 res or fp32 Yadd), fp32 out.
+__device__ __forceinline__ void epi_resadd(const Params& p, uint32_t taddr, int row, int col_base, int c0, int c1) {
+#pragma unroll 1
+  for (int c = c0; c < c1; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    const int col0 = col_base + c * 32;
+    if (row >= p.M || col0 >= p.N) continue;
+    const size_t e = static_cast<size_t>(row) * p.N + col0;
+    for (int i = 0; i < 32 && col0 + i < p.N; ++i) {
+      const float x = p.res ? __uint_as_float(static_cast<uint32_t>(p.res[e + i]) << 16) : p.Yadd[e + i];
+      p.D[e + i] = __fadd_rn(v[i], x);
+    }
+  }
+}
+
+// bf16 out of 32 accumulator columns (round to nearest even).
+__device__ __forceinline__ void store_bf16_32(uint16_t* dst, const float (&v)[32], int n) {
+  if (n == 32) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  } else {
+    for (int i = 0; i < n; ++i) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v[i]);
+      dst[i] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_store_bf16(const Params& p, uint32_t taddr, int row, int col_base, int c0,
+                                               int c1) {
+#pragma unroll 1
+  for (int c = c0; c < c1; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    const int col0 = col_base + c * 32;
+    if (row >= p.M || col0 >= p.N) continue;
+    store_bf16_32(p.Dbf + static_cast<size_t>(row) * p.N + col0, v, min(32, p.N - col0));
+  }
+}
+
+// Stacked Q, K, V projection with the rotary embedding on the Q and K columns.
+// This thread's 128 columns (chunks c0..c0+3) start on a head boundary, so the
+// head halves it rotates together, columns i and i + d/2, are both its own:
+// chunk pairs (c0, c0+2), (c0+1, c0+3) for d = 128 and (c0, c0+1), (c0+2, c0+3)
+// for d = 64.  (x1, x2) -> (x1 cos - x2 sin, x2 cos + x1 sin) in fp32, then bf16.
+__device__ __forceinline__ void epi_qkv(const Params& p, uint32_t taddr, int row, int col_base, int c0) {
+  const int dist = p.head_dim / 64;  // chunks between the two halves of a head
+#pragma unroll 1
+  for (int pr = 0; pr < 2; ++pr) {
+    const int ca = c0 + (dist == 2 ? pr : 2 * pr);
+    const int cb = ca + dist;
+    float va[32], vb[32];
+    tmem_ld32(taddr + ca * 32, va);
+    tmem_ld32(taddr + cb * 32, vb);
+    const int cola = col_base + ca * 32, colb = col_base + cb * 32;
+    if (row >= p.M || cola >= p.N) continue;
+    if (cola < p.rope_cols) {
+      const int t = row % p.rope_L;
+      const float2* cs = p.rope + static_cast<size_t>(t) * (p.head_dim / 2) + (cola % p.head_dim);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float2 r = cs[i];
+        const float x1 = va[i], x2 = vb[i];
+        va[i] = __fsub_rn(__fmul_rn(x1, r.x), __fmul_rn(x2, r.y));
+        vb[i] = __fadd_rn(__fmul_rn(x2, r.x), __fmul_rn(x1, r.y));
+      }
+    }
+    store_bf16_32(p.Dbf + static_cast<size_t>(row) * p.N + cola, va, 32);
+    store_bf16_32(p.Dbf + static_cast<size_t>(row) * p.N + colb, vb, 32);
+  }
+}
+
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 __device__ __forceinline__ float sigmoidf(float x) { return __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-x))); }
 
@@ -506,17 +608,18 @@ __device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, 
       ga[i / 2] = pack_bf16x2(da[0], da[1]);
       gb[i / 2] = pack_bf16x2(db[0], db[1]);
     }
+    const size_t eo = static_cast<size_t>(row) * p.ld_grad + col0;
     if (n == 32) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        *reinterpret_cast<uint4*>(p.grad_a + e + 8 * i) = make_uint4(ga[4 * i], ga[4 * i + 1], ga[4 * i + 2], ga[4 * i + 3]);
-        *reinterpret_cast<uint4*>(p.grad_b + e + 8 * i) = make_uint4(gb[4 * i], gb[4 * i + 1], gb[4 * i + 2], gb[4 * i + 3]);
+        *reinterpret_cast<uint4*>(p.grad_a + eo + 8 * i) = make_uint4(ga[4 * i], ga[4 * i + 1], ga[4 * i + 2], ga[4 * i + 3]);
+        *reinterpret_cast<uint4*>(p.grad_b + eo + 8 * i) = make_uint4(gb[4 * i], gb[4 * i + 1], gb[4 * i + 2], gb[4 * i + 3]);
       }
     } else {
       for (int i = 0; i < n; ++i) {
         const int sh = (i & 1) ? 16 : 0;
-        p.grad_a[e + i] = static_cast<uint16_t>(ga[i / 2] >> sh);
-        p.grad_b[e + i] = static_cast<uint16_t>(gb[i / 2] >> sh);
+        p.grad_a[eo + i] = static_cast<uint16_t>(ga[i / 2] >> sh);
+        p.grad_b[eo + i] = static_cast<uint16_t>(gb[i / 2] >> sh);
       }
     }
   }
@@ -784,8 +887,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) p.partial[(static_cast<size_t>(t) * CG + (kPair ? rank : 0)) * kEpiWarps + half * 4 + quarter] = part;
         } else if (EPI == EPI_SWIGLU_FWD) {
           epi_swiglu_fwd(p, taddr, row, tn * (BN / 2), 2 * half, 2 * half + 2);
-        } else {
+        } else if (EPI == EPI_SWIGLU_BWD) {
           bad |= epi_swiglu_bwd(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
+        } else if (EPI == EPI_QKV) {
+          epi_qkv(p, taddr, row, tn * BN, 4 * half);
+        } else if (EPI == EPI_RESADD) {
+          epi_resadd(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
+        } else {
+          epi_store_bf16(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
         }
       }
       tc_fence_before();
@@ -813,18 +922,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-// bf16 matrix [rows][cols] (cols contiguous), box of box_rows x 64 columns, 128-byte swizzle.
-cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// bf16 matrix [rows][cols] (cols contiguous, rows ld elements apart; ld = 0: cols), box of
+// box_rows x 64 columns, 128-byte swizzle.
+cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                      uint64_t ld = 0) {
   return make_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, rows, cols, 64, box_rows,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
+                      CU_TENSOR_MAP_SWIZZLE_128B, ld);
 }
 
+// lda, ldb: row strides (elements) of A and B as stored, 0 for dense.
 template <bool A_MN, bool B_MN, int EPI, int KSPLIT = 1, int CG = 1>
 cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t stream, const char* name,
-                const uint16_t* B2 = nullptr) {
+                const uint16_t* B2 = nullptr, uint64_t lda = 0, uint64_t ldb = 0) {
   CUtensorMap tmA, tmB, tmB2;
   // A: K-major [M][K] with 128-row boxes, or MN-major [K][M] with 64-row boxes.
-  cudaError_t e = A_MN ? make_tmap(&tmA, A, p.K, p.M, 64) : make_tmap(&tmA, A, p.M, p.K, BM);
+  cudaError_t e = A_MN ? make_tmap(&tmA, A, p.K, p.M, 64, lda) : make_tmap(&tmA, A, p.M, p.K, BM, lda);
   if (e != cudaSuccess) return e;
   if (EPI == EPI_SWIGLU_FWD) {
     // gate and up weights [N][K], 128-row boxes each
@@ -833,7 +945,7 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
     e = make_tmap(&tmB2, B2, p.N, p.K, BN / 2);
   } else {
     // a pair's CTA loads half of the tile's B columns
-    e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64) : make_tmap(&tmB, B, p.N, p.K, BN / CG);
+    e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64, ldb) : make_tmap(&tmB, B, p.N, p.K, BN / CG, ldb);
     tmB2 = tmB;
   }
   if (e != cudaSuccess) return e;
@@ -912,11 +1024,11 @@ static EncodeTiledFn encode_fn() {
 
 cudaError_t make_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, uint32_t elem_bytes, const void* ptr,
                          uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows,
-                         CUtensorMapSwizzle swizzle) {
+                         CUtensorMapSwizzle swizzle, uint64_t ld) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * elem_bytes};
+  const cuuint64_t strides[1] = {(ld ? ld : cols) * elem_bytes};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(tm, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -943,8 +1055,9 @@ cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, in
 }
 
 cudaError_t launch_gemm_resid(const uint16_t* X, const uint16_t* W_hat, const float* Y, uint16_t* G, float gscale,
-                              double* loss_partial, int M, int N, int K, cudaStream_t stream) {
+                              double* loss_partial, int M, int N, int K, cudaStream_t stream, const float* Yadd) {
   Params p{};
+  p.Yadd = Yadd;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -956,7 +1069,7 @@ cudaError_t launch_gemm_resid(const uint16_t* X, const uint16_t* W_hat, const fl
 }
 
 cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArgs& fa, int M, int N, int K,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, int64_t ldg, int64_t ldx) {
   // dW_hat[N_w][K_w] = G[tokens][N_w]^T X[tokens][K_w]: GEMM M = N_w, N = K_w, reduction = tokens.
   Params p{};
   p.M = N;
@@ -976,8 +1089,8 @@ cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArg
   const double eff1 = static_cast<double>(tiles_pair) / (((tiles_pair + pairs - 1) / pairs) * pairs);
   const double eff2 = static_cast<double>(tiles_split) / (((tiles_split + pairs - 1) / pairs) * pairs);
   if (M >= 32768 && eff2 > eff1 + 0.02)
-    return run<true, true, EPI_FOLD, 2>(G, X, p, stream, "umma_gemm<MN,MN,fold,split2>");
-  return run<true, true, EPI_FOLD, 1, kPairCG>(G, X, p, stream, "umma_gemm<MN,MN,fold,pair>");
+    return run<true, true, EPI_FOLD, 2>(G, X, p, stream, "umma_gemm<MN,MN,fold,split2>", nullptr, ldg, ldx);
+  return run<true, true, EPI_FOLD, 1, kPairCG>(G, X, p, stream, "umma_gemm<MN,MN,fold,pair>", nullptr, ldg, ldx);
 }
 
 cudaError_t launch_gemm_swiglu_fwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* Wu, uint16_t* A_out,
@@ -994,7 +1107,7 @@ cudaError_t launch_gemm_swiglu_fwd(const uint16_t* X, const uint16_t* Wg, const 
 
 cudaError_t launch_gemm_swiglu_bwd(const uint16_t* G, const uint16_t* Wd_hat, const uint16_t* A_in,
                                    const uint16_t* B_in, uint16_t* dA, uint16_t* dB, int M, int F, int Hd,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, int ld_grad) {
   // dH[M][F] = G[M][Hd] W_down[Hd][F]: A = G (K-major over Hd), B = W_down as [K=Hd][N=F] (MN-major)
   Params p{};
   p.M = M;
@@ -1004,6 +1117,7 @@ cudaError_t launch_gemm_swiglu_bwd(const uint16_t* G, const uint16_t* Wd_hat, co
   p.act_b = const_cast<uint16_t*>(B_in);
   p.grad_a = dA;
   p.grad_b = dB;
+  p.ld_grad = ld_grad > 0 ? ld_grad : F;
   return run<false, true, EPI_SWIGLU_BWD, 1, kPairCG>(G, Wd_hat, p, stream, "umma_gemm<K,MN,swiglu_bwd,pair>");
 }
 
@@ -1018,6 +1132,45 @@ cudaError_t launch_gemm_plain(const uint16_t* A, bool a_mn, const uint16_t* B, b
   if (!a_mn && b_mn) return run<false, true, EPI_STORE, 1, kPairCG>(A, B, p, stream, "umma_gemm<K,MN,store,pair>");
   if (a_mn && !b_mn) return run<true, false, EPI_STORE, 1, kPairCG>(A, B, p, stream, "umma_gemm<MN,K,store,pair>");
   return run<true, true, EPI_STORE, 1, kPairCG>(A, B, p, stream, "umma_gemm<MN,MN,store,pair>");
+}
+
+cudaError_t launch_gemm_qkv(const uint16_t* X, const uint16_t* Wqkv, uint16_t* out, const float* rope_cs, int M,
+                            int H, int L, int head_dim, cudaStream_t stream) {
+  // out [M][3H] = X [M][H] Wqkv [3H][H]^T, the first 2H columns rotated
+  Params p{};
+  p.M = M;
+  p.N = 3 * H;
+  p.K = H;
+  p.Dbf = out;
+  p.rope = reinterpret_cast<const float2*>(rope_cs);
+  p.rope_cols = 2 * H;
+  p.rope_L = L;
+  p.head_dim = head_dim;
+  return run<false, false, EPI_QKV, 1, kPairCG>(X, Wqkv, p, stream, "umma_gemm<K,K,qkv_rope,pair>");
+}
+
+cudaError_t launch_gemm_resadd(const uint16_t* A, const uint16_t* W, const uint16_t* res, const float* res_f32,
+                               float* out, int M, int N, int K, cudaStream_t stream) {
+  // out [M][N] fp32 = residual (bf16 res, else fp32 res_f32) + A [M][K] W [N][K]^T
+  Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.res = res;
+  p.Yadd = res_f32;
+  p.D = out;
+  return run<false, false, EPI_RESADD, 1, kPairCG>(A, W, p, stream, "umma_gemm<K,K,resadd,pair>");
+}
+
+cudaError_t launch_gemm_store_bf16_kmn(const uint16_t* A, const uint16_t* B_kn, uint16_t* out, int M, int N, int K,
+                                       cudaStream_t stream) {
+  // out [M][N] bf16 = A [M][K] B with B stored [K][N] (MN-major)
+  Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.Dbf = out;
+  return run<false, true, EPI_STORE_BF16, 1, kPairCG>(A, B_kn, p, stream, "umma_gemm<K,MN,store_bf16,pair>");
 }
 
 cudaError_t launch_loss_reduce(const double* partials, int n, int steps, double inv_count, float* loss,

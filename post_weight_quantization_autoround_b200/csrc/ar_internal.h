@@ -54,7 +54,7 @@ cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaS
 // box of box_rows x box_cols elements; zero fill out of bounds.
 cudaError_t make_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, uint32_t elem_bytes, const void* ptr,
                          uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows,
-                         CUtensorMapSwizzle swizzle);
+                         CUtensorMapSwizzle swizzle, uint64_t ld = 0);
 
 // ---- tensor-core GEMMs (ar_gemm.cu) ----
 struct FoldArgs {
@@ -79,24 +79,55 @@ cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, in
 
 // Forward of the tuning step with the residual epilogue:
 //   R = X W_hat^T - Y, G = bf16(R * gscale), partial[tile*4+warp] = sum R^2 (fp64).
+// With Yadd (fp32 [M][N]), R = (X W_hat^T + Yadd) - Y.
 cudaError_t launch_gemm_resid(const uint16_t* X, const uint16_t* W_hat, const float* Y, uint16_t* G, float gscale,
-                              double* loss_partial, int M, int N, int K, cudaStream_t stream);
+                              double* loss_partial, int M, int N, int K, cudaStream_t stream,
+                              const float* Yadd = nullptr);
 int resid_partials(int M, int N);
 
 // Backward of the tuning step: dW_hat = G^T X (reduction over the M tokens),
 // folded through the straight-through estimator and applied as a SignSGD step.
+// ldg, ldx: row strides of G and X when they are column slices of wider matrices (0: dense).
 cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArgs& fa, int M, int N, int K,
-                             cudaStream_t stream);
+                             cudaStream_t stream, int64_t ldg = 0, int64_t ldx = 0);
 
 // SwiGLU forward of X[M][Hd] with gate/up weights [F][Hd]: a, b, h [M][F]
 // bf16 (a, b nullable).
 cudaError_t launch_gemm_swiglu_fwd(const uint16_t* X, const uint16_t* Wg, const uint16_t* Wu, uint16_t* A_out,
                                    uint16_t* B_out, uint16_t* H_out, int M, int F, int Hd, cudaStream_t stream);
 
-// dH = G[M][Hd] W_down[Hd][F] with the SiLU backward epilogue -> dA, dB [M][F] bf16.
+// dH = G[M][Hd] W_down[Hd][F] with the SiLU backward epilogue -> dA, dB [M][F] bf16
+// (rows ld_grad elements apart; 0: F).
 cudaError_t launch_gemm_swiglu_bwd(const uint16_t* G, const uint16_t* Wd_hat, const uint16_t* A_in,
                                    const uint16_t* B_in, uint16_t* dA, uint16_t* dB, int M, int F, int Hd,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, int ld_grad = 0);
+
+// ---- decoder block (ar_gemm.cu epilogues, ar_decoder.cu kernels) ----
+// out [M][3H] bf16 = X [M][H] Wqkv [3H][H]^T, the Q and K columns (the first 2H)
+// rotated by the position (row % L) angles of rope_cs ((cos, sin) [L][head_dim/2]).
+cudaError_t launch_gemm_qkv(const uint16_t* X, const uint16_t* Wqkv, uint16_t* out, const float* rope_cs, int M,
+                            int H, int L, int head_dim, cudaStream_t stream);
+// out [M][N] fp32 = residual (bf16 res [M][N], else fp32 res_f32) + A [M][K] W [N][K]^T
+cudaError_t launch_gemm_resadd(const uint16_t* A, const uint16_t* W, const uint16_t* res, const float* res_f32,
+                               float* out, int M, int N, int K, cudaStream_t stream);
+// out [M][N] bf16 = A [M][K] B, B stored [K][N]
+cudaError_t launch_gemm_store_bf16_kmn(const uint16_t* A, const uint16_t* B_kn, uint16_t* out, int M, int N, int K,
+                                       cudaStream_t stream);
+// causal attention per sample and head over qkv [S*L][3H] (Q, K rotated; V): O [S*L][H] bf16, lse [S][nh][L]
+cudaError_t launch_attn_fwd(const uint16_t* qkv, int S, int L, int H, int head_dim, uint16_t* out, float* lse,
+                            cudaStream_t st);
+// its backward from dO: dqkv [S*L][3H] bf16 (dQ, dK with the inverse rotation applied; dV); Dsum [S][nh][L] scratch
+cudaError_t launch_attn_bwd(const uint16_t* qkv, const uint16_t* O, const uint16_t* dO, const float* lse,
+                            float* Dsum, const float* rope_cs, int S, int L, int H, int head_dim, uint16_t* dqkv,
+                            cudaStream_t st);
+// r [M][H] bf16 = x inv gamma, inv [M] = 1/sqrt(mean(x^2) + 1e-6) (x bf16 or fp32)
+cudaError_t launch_rmsnorm_fwd(const void* x, bool x_f32, const float* gamma, int64_t M, int H, uint16_t* r,
+                               float* inv, cudaStream_t st);
+// dx [M][H] bf16 = G + RMSNorm backward of dr (fp32) at x (fp32) with inv, gamma
+cudaError_t launch_rmsnorm_bwd(const float* x, const float* inv, const float* gamma, const float* dr,
+                               const uint16_t* G, int64_t M, int H, uint16_t* dx, cudaStream_t st);
+// (cos, sin) [L][head_dim/2] fp32 of t 10000^(-2i/head_dim)
+cudaError_t launch_rope_table(int L, int head_dim, float* cs, cudaStream_t st);
 
 // Plain D[M][N] fp32 = op(A) op(B)^T, with A given K-major ([M][K]) or
 // MN-major ([K][M]) and B given K-major ([N][K]) or MN-major ([K][N]).

@@ -27,6 +27,7 @@ __all__ = [
     "bf16_bits_to_f32",
     "make_linear",
     "make_mlp",
+    "make_decoder",
     "make_activations",
     "Workload",
     "WORKLOADS",
@@ -127,6 +128,36 @@ def make_mlp(
     wd = _weights(r[_S_MLP_D], r[_S_W_OUT], hidden, inter, w_std, outlier_frac, outlier_scale)
     x = _acts(r[_S_X], r[_S_X_OUT], m_tokens, hidden, x_outlier_channels, x_outlier_scale)
     return {"Wg": to_bf16_bits(wg), "Wu": to_bf16_bits(wu), "Wd": to_bf16_bits(wd), "X": to_bf16_bits(x)}
+
+
+def make_decoder(
+    hidden: int,
+    inter: int,
+    m_tokens: int,
+    *,
+    seed: int = 0,
+    w_std: float = 0.02,
+    outlier_frac: float = 0.001,
+    outlier_scale: float = 20.0,
+    x_outlier_channels: int = 8,
+    x_outlier_scale: float = 50.0,
+    gamma_std: float = 0.1,
+) -> Dict[str, np.ndarray]:
+    """Decoder block: q, k, v, o ``[hidden][hidden]``, gate/up ``[inter][hidden]``, down ``[hidden][inter]``
+    (bf16 bits, the linear layers' distribution), input ``X [m_tokens][hidden]`` (bf16 bits) and the two
+    norm scales ``gamma1, gamma2 [hidden]`` ~ 1 + N(0, gamma_std), float32 values that bf16 holds exactly."""
+    root = np.random.SeedSequence(seed).spawn(17)  # 0-13: the seven weights, 14: gammas, 15-16: X
+    rng = lambda i: np.random.Generator(np.random.PCG64(root[i]))
+    shapes = {"q": (hidden, hidden), "k": (hidden, hidden), "v": (hidden, hidden), "o": (hidden, hidden),
+              "gate": (inter, hidden), "up": (inter, hidden), "down": (hidden, inter)}
+    out = {}
+    for i, (name, (n, k)) in enumerate(shapes.items()):
+        out[name] = to_bf16_bits(_weights(rng(2 * i), rng(2 * i + 1), n, k, w_std, outlier_frac, outlier_scale))
+    out["X"] = to_bf16_bits(_acts(rng(15), rng(16), m_tokens, hidden, x_outlier_channels, x_outlier_scale))
+    g = rng(14)
+    for name in ("gamma1", "gamma2"):
+        out[name] = bf16_bits_to_f32(to_bf16_bits(1.0 + _normal(g, (hidden,), gamma_std)))
+    return out
 
 
 def make_activations(t: int, k: int, *, seed: int = 0) -> np.ndarray:

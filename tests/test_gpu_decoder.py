@@ -1,0 +1,247 @@
+"""The decoder block on the GPU against the oracle's block with the same rounding points (needs a B200).
+
+[AR] §3 "Why Block-Wise Optimization" / "Algorithm Flow": the block is the unit
+of tuning.  The oracle's ``rounding=True`` mode rounds at the points the GPU
+path rounds (every operand of a product bf16, the rest fp32; see the oracle's
+decoder section), so the two differ only in summation order:
+  * RMSNorm: r bit-equal on >= 99.9 % of entries and within one bf16 step
+    elsewhere; inv within 1e-6;
+  * attention: O and the gradients within 3e-3 relative L2 (bf16 outputs:
+    2^-9 relative per entry, plus probabilities whose rounding flips between
+    summation orders), lse within 1e-5;
+  * the block forward: Y within 1e-4 relative L2;
+  * one joint tuning step: loss within 1e-3, every layer's dV, dalpha, dbeta
+    within 1e-3 relative L2 with >= 99.9 % sign agreement where |g| > 1e-3 RMS,
+    and the update equal on >= 99.9 % (V) / 99 % (alpha, beta) of entries.
+
+[AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
+Architectural Optimizations of AutoRound".
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import autoround_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+GRAD_RTOL = 1e-3
+SIGN_AGREE = 0.999
+CLIP_AGREE = 0.99
+ATTN_RTOL = 3e-3
+
+
+@pytest.fixture(scope="module")
+def ar():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import post_weight_quantization_autoround_b200 as m
+
+    m.lib()
+    return m
+
+
+def bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def f32_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def bits16(t):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def as_f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def rel_l2(x, y):
+    x, y = np.asarray(x, np.float64), np.asarray(y, np.float64)
+    return float(np.linalg.norm(x - y) / max(np.linalg.norm(y), 1e-300))
+
+
+def rb(x):
+    return O.bf16_rne(np.asarray(x, np.float64).astype(np.float32)).astype(np.float64)
+
+
+@pytest.mark.parametrize("in_f32", [False, True])
+def test_rmsnorm_matches_oracle(ar, in_f32):
+    M, H = 200, 768
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((M, H)).astype(np.float32) * 3
+    gam = synth.bf16_bits_to_f32(synth.to_bf16_bits(1 + 0.1 * rng.standard_normal(H)))
+    if not in_f32:
+        x = synth.bf16_bits_to_f32(synth.to_bf16_bits(x))
+    xd = f32_dev(x) if in_f32 else bf16_dev(synth.to_bf16_bits(x))
+    r = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
+    inv = torch.empty(M, device="cuda")
+    ar.ar_rmsnorm(xd, f32_dev(gam), r, inv)
+    assert ar.ar_get_device_status() == 0
+    ref, ref_inv = O.rmsnorm(x, gam)
+    ref_bits = synth.to_bf16_bits(ref.astype(np.float32))
+    got = bits16(r)
+    assert np.mean(got == ref_bits) >= 0.999
+    assert np.max(np.abs(got.astype(np.int32) - ref_bits.astype(np.int32))) <= 1
+    assert np.allclose(inv.cpu().numpy(), ref_inv[:, 0], rtol=1e-6)
+
+
+def _qkv_problem(S, L, H, seed):
+    rng = np.random.default_rng(seed)
+    qkv = rb(rng.standard_normal((S * L, 3 * H)) * 1.5)
+    return qkv
+
+
+@pytest.mark.parametrize("S,L,H,nh", [(2, 128, 256, 2), (1, 192, 128, 2), (1, 64, 256, 4)])
+def test_attention_forward_and_backward_match_oracle(ar, S, L, H, nh):
+    qkv = _qkv_problem(S, L, H, seed=S + L + H)
+    d = H // nh
+    qd = bf16_dev(synth.to_bf16_bits(qkv.astype(np.float32)))
+    out = torch.empty((S * L, H), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((S, nh, L), device="cuda")
+    ar.ar_attention_forward(qd, S, L, nh, out, lse)
+    assert ar.ar_get_device_status() == 0
+    assert ("attn_fwd_kernel<d%d>" % d) in ar.ar_last_kernels()
+    Qr, Kr, V = (qkv[:, i * H:(i + 1) * H].reshape(S, L, H) for i in range(3))
+    O_ref, P, lse_ref = O.attention_forward(Qr, Kr, V, nh, rounding=True)
+    assert rel_l2(as_f64(out), O_ref.reshape(S * L, H)) <= ATTN_RTOL
+    assert np.allclose(lse.cpu().numpy(), lse_ref, rtol=1e-5, atol=1e-5)
+    # backward from a random dO, with the forward's own O
+    rng = np.random.default_rng(7)
+    dO = rb(rng.standard_normal((S * L, H)) * 0.1)
+    dOd = bf16_dev(synth.to_bf16_bits(dO.astype(np.float32)))
+    ws = torch.empty(ar.ar_attention_backward_workspace(S, L, H, nh), dtype=torch.uint8, device="cuda")
+    dqkv = torch.full((S * L, 3 * H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_attention_backward(qd, out, dOd, lse, S, L, nh, dqkv, ws)
+    assert ar.ar_get_device_status() == 0
+    O_gpu = as_f64(out).reshape(S, L, H)
+    dQr, dKr, dV = O.attention_backward(Qr, Kr, V, P, dO.reshape(S, L, H), nh, rounding=True, O=O_gpu)
+    dQ = rb(O.rope(dQr, nh, -1.0, rounding=True))
+    dK = rb(O.rope(dKr, nh, -1.0, rounding=True))
+    got = as_f64(dqkv)
+    for i, ref in enumerate((dQ, dK, dV)):
+        assert rel_l2(got[:, i * H:(i + 1) * H], ref.reshape(S * L, H)) <= ATTN_RTOL, i
+
+
+def _block(d_np, H, F):
+    Ws = {n: synth.bf16_bits_to_f32(d_np[n]).astype(np.float64) for n in O.DECODER_LAYERS}
+    X = synth.bf16_bits_to_f32(d_np["X"]).astype(np.float64)
+    gammas = (d_np["gamma1"].astype(np.float64), d_np["gamma2"].astype(np.float64))
+    return Ws, X, gammas
+
+
+class GpuDecoder:
+    def __init__(self, ar, d_np, S, L, nh, states, cfg, n_steps):
+        self.ar, self.cfg, self.nh, self.L = ar, cfg, nh, L
+        self.W = [bf16_dev(d_np[n]) for n in O.DECODER_LAYERS]
+        self.X = bf16_dev(d_np["X"])
+        self.g1, self.g2 = f32_dev(d_np["gamma1"]), f32_dev(d_np["gamma2"])
+        self.st = [tuple(f32_dev(x) for x in states[n]) for n in O.DECODER_LAYERS]
+        M, H = d_np["X"].shape
+        F = d_np["gate"].shape[0]
+        self.Y = torch.empty((M, H), device="cuda")
+        fws = torch.empty(ar.ar_decoder_forward_workspace(H, F, nh, L, M), dtype=torch.uint8, device="cuda")
+        ar.ar_decoder_forward(self.W, self.g1, self.g2, nh, L, self.X, self.Y, fws)
+        assert ar.ar_get_device_status() == 0
+        n = ar.ar_tune_step_decoder_workspace(self.layers(), self.g1, self.g2, nh, L, M, cfg, n_steps)
+        self.ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+
+    def layers(self):
+        return [(W, *s) for W, s in zip(self.W, self.st)]
+
+    def step(self, n_steps, grads=False):
+        loss = torch.empty(max(n_steps, 1), device="cuda")
+        gr = None
+        if grads:
+            gr = [(torch.full(W.shape, float("nan"), device="cuda"),
+                   torch.full((W.shape[0], W.shape[1] // self.cfg.group_size), float("nan"), device="cuda"),
+                   torch.full((W.shape[0], W.shape[1] // self.cfg.group_size), float("nan"), device="cuda"))
+                  for W in self.W]
+        self.ar.ar_tune_step_decoder(self.layers(), self.g1, self.g2, self.nh, self.L, self.X, self.Y, self.cfg,
+                                     n_steps, loss, self.ws, grads=gr)
+        assert self.ar.ar_get_device_status() == 0, self.ar.ar_last_error()
+        out = {"loss": loss.cpu().numpy()}
+        if grads:
+            out["grads"] = [tuple(t.cpu().numpy() for t in g) for g in gr]
+        return out
+
+    def state(self):
+        return {n: tuple(t.cpu().numpy() for t in s) for n, s in zip(O.DECODER_LAYERS, self.st)}
+
+
+def test_decoder_forward_matches_oracle(ar):
+    S, L, H, F, nh = 2, 128, 256, 512, 2
+    d = synth.make_decoder(H, F, S * L, seed=4)
+    Ws, X, gammas = _block(d, H, F)
+    Wd = [bf16_dev(d[n]) for n in O.DECODER_LAYERS]
+    Y = torch.empty((S * L, H), device="cuda")
+    ws = torch.empty(ar.ar_decoder_forward_workspace(H, F, nh, L, S * L), dtype=torch.uint8, device="cuda")
+    ar.ar_decoder_forward(Wd, f32_dev(d["gamma1"]), f32_dev(d["gamma2"]), nh, L, bf16_dev(d["X"]), Y, ws)
+    assert ar.ar_get_device_status() == 0
+    ref = O.decoder_forward(X.reshape(S, L, H), Ws, gammas, nh, rounding=True)["Y"].reshape(S * L, H)
+    assert rel_l2(Y.cpu().numpy(), ref) <= 1e-4
+
+
+def _check_step(out, st_gpu, ref_loss, ref_new, ref_grads):
+    assert out["loss"][0] == pytest.approx(ref_loss, rel=1e-3)
+    for li, n in enumerate(O.DECODER_LAYERS):
+        for k in range(3):
+            got, ref = out["grads"][li][k], ref_grads[n][k]
+            assert rel_l2(got, ref) <= GRAD_RTOL, (n, k, rel_l2(got, ref))
+            rms = np.sqrt(np.mean(np.asarray(ref, np.float64) ** 2))
+            mask = np.abs(ref) > 1e-3 * rms
+            assert np.mean(np.sign(got[mask]) == np.sign(ref[mask])) >= SIGN_AGREE, (n, k)
+        assert np.mean(st_gpu[n][0] == ref_new[n][0]) >= SIGN_AGREE, n
+        for k in (1, 2):
+            assert np.mean(st_gpu[n][k] == ref_new[n][k]) >= CLIP_AGREE, (n, k)
+
+
+@pytest.mark.parametrize("S,L,H,F,nh,g,bits,spread", [
+    (2, 128, 256, 512, 2, 128, 4, False),   # head dim 128, the initial state
+    (1, 192, 256, 384, 4, 64, 3, True),     # head dim 64, a spread state, 3 bits
+])
+def test_decoder_step_matches_oracle(ar, S, L, H, F, nh, g, bits, spread):
+    d = synth.make_decoder(H, F, S * L, seed=S * 10 + nh)
+    Ws, X, gammas = _block(d, H, F)
+    states = {n: synth.make_state(*Ws[n].shape, g, seed=i, spread=spread) for i, n in enumerate(O.DECODER_LAYERS)}
+    cfg = ar.ar_qconfig_default(bits=bits, group_size=g)
+    ocfg = O.QConfig(bits=bits, group_size=g)
+    gd = GpuDecoder(ar, d, S, L, nh, states, cfg, 1)
+    out = gd.step(1, grads=True)
+    assert "attn_bwd_dkdv_kernel" in ar.ar_last_kernels() and "qkv_rope" in ar.ar_last_kernels()
+    Xs = X.reshape(S, L, H)
+    Y = O.decoder_forward(Xs, Ws, gammas, nh, rounding=True)["Y"].astype(np.float32)  # the oracle's own reference
+    L_ref, new, grads = O.tune_step_decoder(Ws, Xs, Y, states, gammas, nh, ocfg, rounding=True)
+    _check_step(out, gd.state(), L_ref, new, grads)
+
+
+def test_decoder_steps_are_deterministic_and_resumable(ar):
+    S, L, H, F, nh, g = 1, 128, 256, 512, 2, 128
+    d = synth.make_decoder(H, F, S * L, seed=9)
+    states = {n: synth.make_state(*d[n].shape, g, seed=i, spread=True) for i, n in enumerate(O.DECODER_LAYERS)}
+    cfg = ar.ar_qconfig_default(group_size=g)
+    a = GpuDecoder(ar, d, S, L, nh, states, cfg, 4)
+    la = a.step(4)["loss"]
+    b = GpuDecoder(ar, d, S, L, nh, states, cfg, 2)
+    lb = np.concatenate([b.step(2)["loss"], b.step(2)["loss"]])
+    assert np.array_equal(la, lb)
+    for n in O.DECODER_LAYERS:
+        for x, y in zip(a.state()[n], b.state()[n]):
+            assert np.array_equal(x, y), n
+
+
+def test_decoder_llama7b_shapes_token_sample(ar):
+    """The Llama-7B block's shapes (H 4096, F 11008, 32 heads of 128), 128 tokens: one joint step."""
+    S, L, H, F, nh, g = 1, 128, 4096, 11008, 32, 128
+    d = synth.make_decoder(H, F, S * L, seed=11)
+    Ws, X, gammas = _block(d, H, F)
+    states = {n: synth.make_state(*Ws[n].shape, g) for n in O.DECODER_LAYERS}
+    cfg = ar.ar_qconfig_default(group_size=g)
+    gd = GpuDecoder(ar, d, S, L, nh, states, cfg, 1)
+    out = gd.step(1, grads=True)
+    Xs = X.reshape(S, L, H)
+    Y = O.decoder_forward(Xs, Ws, gammas, nh, rounding=True)["Y"].astype(np.float32)
+    L_ref, new, grads = O.tune_step_decoder(Ws, Xs, Y, states, gammas, nh, O.QConfig(group_size=g), rounding=True)
+    _check_step(out, gd.state(), L_ref, new, grads)

@@ -295,45 +295,6 @@ def test_small_workload_full_trajectory(ar):
     assert final_gpu == pytest.approx(final, rel=MSE_RTOL)
 
 
-@pytest.mark.parametrize("name,steps", [("linear_4096", 20), ("lowbit_b2g32", 20), ("lowbit_b8g256", 10)])
-def test_full_size_sampled_rows(ar, name, steps):
-    """Full-size layer on the GPU; the oracle follows 64 sampled rows exactly (rows are independent).
-
-    Step-1 gradients on the sampled rows, then after ``steps`` steps the codes
-    and the sampled rows' MSE (evaluated on the GPU on the same rows).
-    """
-    wl = synth.WORKLOADS[name]
-    N, K, M, g = wl.n_out, wl.n_in, wl.m_tokens, wl.group_size
-    d = synth.make_linear(N, K, M, seed=wl.seed)
-    V, a, b = synth.make_state(N, K, g)
-    cfg, ocfg = cfg_pair(ar, wl.bits, g, lr=wl.lr)
-    gl = GpuLinear(ar, d["W"], d["X"], V, a, b, cfg, n_steps=steps)
-    first = gl.step(1, grads=True)
-    rest = gl.step(steps - 1)
-    rows = np.sort(np.random.default_rng(123).choice(N, 64, replace=False))
-    Wf = synth.bf16_bits_to_f32(d["W"][rows])
-    Xf = synth.bf16_bits_to_f32(d["X"])
-    Y = O.reference_forward(Xf, Wf)
-    count = M * N
-    L, (Vo, ao, bo), gr, _ = O.tune_step_linear(Wf, Xf, Y, V[rows], a[rows], b[rows], ocfg, count=count)
-    for k in ("dV", "dalpha", "dbeta"):
-        assert rel_l2(first[k][rows], gr[k]) <= GRAD_RTOL, (k, rel_l2(first[k][rows], gr[k]))
-        rms = np.sqrt(np.mean(gr[k].astype(np.float64) ** 2))
-        agree, n = sign_agreement(first[k][rows], gr[k], 1e-3 * rms)
-        assert agree >= SIGN_AGREE, (k, agree, n)
-    for _ in range(steps - 1):
-        _, (Vo, ao, bo), _, _ = O.tune_step_linear(Wf, Xf, Y, Vo, ao, bo, ocfg, count=count)
-    Vg, ag, bg = gl.state()
-    st = O.qdq(Wf, Vo, ao, bo, wl.bits, g)
-    assert np.mean(gl.codes()[rows] == st["q"]) >= CODE_AGREE
-    # sampled rows' MSE: the GPU evaluates its own state on the same rows
-    sub = GpuLinear(ar, d["W"][rows], d["X"], Vg[rows], ag[rows], bg[rows], cfg, n_steps=0)
-    mse_gpu = sub.step(0)["loss"][0]
-    mse_ref = O.eval_loss_linear(Wf, Xf, Y, Vo, ao, bo, ocfg)
-    assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
-    assert np.isfinite(rest["loss"]).all()
-
-
 def test_row_shards_reproduce_the_unsharded_step(ar):
     """ar_tune_step_shard on two row ranges of one layer gives the unsharded call's rows bit for bit."""
     N, K, M, g, steps, cut = 320, 512, 200, 128, 3, 136  # 136/320: the ratio is not a power of two

@@ -18,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import synth
 from oracle import autoround_oracle as O
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -1030,6 +1031,49 @@ def test_decoder_step_on_grid_weights_is_stationary():
         assert all(np.array_equal(a, b) for a, b in zip(new[n], states[n]))
 
 
+def test_attention_row_term_from_the_output_equals_the_one_from_the_probabilities():
+    """D = rowsum(dO ⊙ O) (what a fused backward reads) is rowsum(dP ⊙ P) exactly in fp64, since O = P V."""
+    rng = np.random.default_rng(65)
+    S, L, H, nh = 2, 7, 16, 2
+    Q, K, V, dO = (rng.standard_normal((S, L, H)) for _ in range(4))
+    Ov, P, lse = O.attention_forward(Q, K, V, nh)
+    assert np.allclose(P.sum(axis=-1), 1.0, rtol=1e-13)
+    assert np.all(np.triu(P, 1) == 0)
+    a = O.attention_backward(Q, K, V, P, dO, nh)
+    b = O.attention_backward(Q, K, V, P, dO, nh, O=Ov)
+    for x, y in zip(a, b):
+        assert np.allclose(x, y, rtol=1e-12, atol=1e-13)
+
+
+def test_decoder_rounding_points_stay_within_bf16_noise_of_fp64():
+    """The shared rounding points only round: the step with them is within bf16 noise of the fp64 step
+    (a dropped term or a wrong sign in either would be off by far more)."""
+    rng = np.random.default_rng(66)
+    S, L, H, F, nh, g = 2, 16, 64, 128, 2, 32
+    Ws = {n: _bf16(rng.standard_normal((H, H)) * 0.1) for n in ("q", "k", "v", "o")}
+    Ws["gate"], Ws["up"] = _bf16(rng.standard_normal((F, H)) * 0.1), _bf16(rng.standard_normal((F, H)) * 0.1)
+    Ws["down"] = _bf16(rng.standard_normal((H, F)) * 0.1)
+    X = _bf16(rng.standard_normal((S, L, H)))
+    gammas = (_bf16(1.0 + 0.1 * rng.standard_normal(H)), _bf16(1.0 + 0.1 * rng.standard_normal(H)))
+    Y = O.decoder_forward(X, Ws, gammas, nh)["Y"].astype(np.float32)
+    states = {n: synth.make_state(W.shape[0], W.shape[1], g, seed=3, spread=True) for n, W in Ws.items()}
+    cfg = O.QConfig(group_size=g)
+    sts = {n: O.qdq(Ws[n], *states[n], 4, g) for n in O.DECODER_LAYERS}
+    Wh = {n: sts[n]["What_bf16"] for n in O.DECODER_LAYERS}
+    f64 = O.decoder_forward(X, Wh, gammas, nh)
+    f32 = O.decoder_forward(X, Wh, gammas, nh, rounding=True)
+    for k in ("Qr", "O", "X2", "h", "Y"):
+        assert np.linalg.norm(f32[k] - f64[k]) <= 1e-2 * np.linalg.norm(f64[k]), k
+    R64, R32 = f64["Y"] - Y, f32["Y"] - Y
+    g64 = O.decoder_backward(f64, 2 * R64 / R64.size, Wh, gammas, nh)
+    g32 = O.decoder_backward(f32, O.bf16_rne((2 * R32 / R32.size).astype(np.float32)), Wh, gammas, nh, rounding=True)
+    for n in O.DECODER_LAYERS:
+        assert np.linalg.norm(g32[n] - g64[n]) <= 3e-2 * np.linalg.norm(g64[n]), n
+    L64, _, _ = O.tune_step_decoder(Ws, X, Y, states, gammas, nh, cfg)
+    L32, _, _ = O.tune_step_decoder(Ws, X, Y, states, gammas, nh, cfg, rounding=True)
+    assert L32 == pytest.approx(L64, rel=2e-2)
+
+
 def test_bitstream_packing_is_the_per_word_layout_and_places_3_bit_codes_by_hand():
     rng = np.random.default_rng(70)
     for bits in (2, 4, 8):
@@ -1052,3 +1096,36 @@ def test_bitstream_packing_is_the_per_word_layout_and_places_3_bit_codes_by_hand
     q1[0, 21] = 0b011
     w1 = O.pack_bitstream(q1, 3)
     assert int(w1[0, 0]) == (0b01 << 30) and int(w1[0, 1]) == (0b1 | (0b1 << 31)) and int(w1[0, 2]) == 0b1
+
+
+def test_free_running_runs_agree_over_a_horizon_then_depend_on_summation_order():
+    """SignSGD moves every parameter by exactly lr, so parameters with near-zero gradients follow
+    rounding noise: the oracle with fp64 products and the same step with fp32 products (the only
+    difference) agree code for code over the first tens of steps and drift apart over hundreds.
+    This is why a whole run is compared with the GPU only over its first steps, and at later steps
+    from the GPU's own state."""
+    N, K, M, g, bits = 16, 2048, 2048, 128, 4
+    d = synth.make_linear(N, K, M, seed=0)
+    W = synth.bf16_bits_to_f32(d["W"])
+    X64 = synth.bf16_bits_to_f32(d["X"]).astype(np.float64)
+    X32 = X64.astype(np.float32)
+    Y = O.reference_forward(X64, W)
+    cfg = O.QConfig(bits=bits, group_size=g)
+
+    def step_f32_products(V, a, b):
+        st = O.qdq(W, V, a, b, bits, g)
+        R = ((X32 @ st["What_bf16"].T).astype(np.float32) - Y).astype(np.float32)
+        G = O.bf16_rne((R * np.float32(2.0 / (M * N))).astype(np.float32))
+        dV, da, db = O.ste_fold((G.T @ X32).astype(np.float32), W, st, bits)
+        return (O.signsgd(V, dV, cfg.lr, -0.5, 0.5), O.signsgd(a, da, cfg.lr, 0.5, 1.0),
+                O.signsgd(b, db, cfg.lr, 0.5, 1.0))
+
+    A = B = synth.make_state(N, K, g)
+    same = {}
+    for i in range(1, 201):
+        _, A, _, _ = O.tune_step_linear(W, X64, Y, *A, cfg)
+        B = step_f32_products(*B)
+        if i in (20, 200):
+            same[i] = np.mean(O.qdq(W, *A, bits, g)["q"] == O.qdq(W, *B, bits, g)["q"])
+    assert same[20] >= 0.995
+    assert same[200] < 0.95
