@@ -322,10 +322,11 @@ def w4a16_bench(ar, torch, peaks, reps=20):
                         "roofline_frac": t_roof / (ms * 1e-3),
                         "algorithmic_bytes": nbytes, "kernel": ar.ar_last_kernels()}
     out["shape"] = f"{N}x{K} int4 g{g}, fp16 scale/zero, bf16 activations; L2 flushed before each launch"
-    # the same layer packed at 2 and 8 bits (tcgen05 dequant GEMM at every T)
+    # the same layer packed at 2, 3 and 8 bits (decode kernel at T = 1; T = 256: tcgen05 dequant GEMM for 2
+    # and 8 bits, the decode kernel 16 tokens at a time for 3 bits)
     W = to_dev_bf16(d["W"], torch)
     V = torch.zeros((N, K), dtype=torch.float32, device="cuda")
-    for bits in (2, 8):
+    for bits in (2, 3, 8):
         cfgb = ar.ar_qconfig_default(bits=bits, group_size=g)
         pk = torch.empty((N, K * bits // 32), dtype=torch.int32, device="cuda")
         ar.ar_pack_codes(W, V, a, b, cfgb, pk, s16, z16)
@@ -343,7 +344,7 @@ def w4a16_bench(ar, torch, peaks, reps=20):
             torch.cuda.synchronize()
             ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
             nbytes = pk.numel() * 4 + s16.numel() * 2 + z16.numel() * 2 + A.numel() * 2 + y.numel() * 2
-            out[f"W{bits}A16_T{T}"] = {"us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9,
+            out[f"W{bits}A16_T{T}"] = {"us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9, "algorithmic_bytes": nbytes,
                                       "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                       "TFLOP/s": 2.0 * T * N * K / (ms * 1e-3) / 1e12, "kernel": ar.ar_last_kernels()}
     del W, V
@@ -452,7 +453,12 @@ def job_throughput(world: int, steps: int, max_ms: float) -> float:
     return world * steps / (max_ms * 1e-3)
 
 
-def _time_call(torch, fn, warmup=1):
+_LAST_PROFILE = {}
+
+
+def _time_call(torch, fn, warmup=1, ar=None):
+    """Device time (ms) of one call of fn; with ``ar`` the per-kernel device times of that call are kept in
+    _LAST_PROFILE (the library's event profiler; it adds two events per launch)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -461,7 +467,19 @@ def _time_call(torch, fn, warmup=1):
     fn()
     e1.record()
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1)
+    ms = e0.elapsed_time(e1)
+    _LAST_PROFILE.clear()
+    if ar is not None:
+        ar.ar_profile_start()
+        fn()
+        torch.cuda.synchronize()
+        _LAST_PROFILE.update(ar.ar_profile_stop())
+    return ms
+
+
+def _kernel_split(n_steps):
+    """Per-kernel share of the last profiled call: {name: [launches, us per step]}."""
+    return {k: [n, round(1e3 * t / n_steps, 2)] for k, (n, t) in sorted(_LAST_PROFILE.items(), key=lambda kv: -kv[1][1])}
 
 
 def other_workloads(ar, torch, peaks, steps=10):
@@ -516,13 +534,28 @@ def other_workloads(ar, torch, peaks, steps=10):
         n = steps if name.startswith("down") else 5 * steps
         ws = torch.empty(ar.ar_tune_step_workspace(W, V, a, b, M, cfg, n), dtype=torch.uint8, device="cuda")
         loss = torch.empty(n, device="cuda")
-        ms = _time_call(torch, lambda: ar.ar_tune_step(W, V, a, b, X, Y, cfg, n, loss, ws))
+        ms = _time_call(torch, lambda: ar.ar_tune_step(W, V, a, b, X, Y, cfg, n, loss, ws), ar=ar)
         flops = 4.0 * M * N * K
         out[name] = {"steps_per_s": n / (ms * 1e-3), "ms_per_step": ms / n, "tflops": flops * n / (ms * 1e-3) / 1e12,
                      **fracs(flops * n / (ms * 1e-3) / 1e12, ms * 1e-3), "steps": n,
+                     "kernels_us_per_step": _kernel_split(n),
                      "final_loss": float(loss[-1].item())}
         del W, X, V, a, b, Y, ws
         torch.cuda.empty_cache()
+    # the decoder block (attention + MLP, seven tuned weights) at the Llama-7B shapes, 8 x 2048 tokens
+    steps_d = 5
+    fn, flops_d, loss_d = decoder_step_fn(ar, torch, 8, 2048, steps_d)
+    ms = _time_call(torch, fn, ar=ar)
+    out["decoder_llama7b_16384"] = {
+        "kernels_us_per_step": _kernel_split(steps_d),
+        "steps_per_s": steps_d / (ms * 1e-3), "ms_per_step": ms / steps_d,
+        "tflops": flops_d * steps_d / (ms * 1e-3) / 1e12, **fracs(flops_d * steps_d / (ms * 1e-3) / 1e12, ms * 1e-3),
+        "steps": steps_d, "first_loss": float(loss_d[0].item()), "last_loss": float(loss_d[-1].item()),
+        "kernels": ar.ar_last_kernels().count(";") + 1,
+        "note": "H 4096, F 11008, 32 heads of 128, 8 samples x 2048 tokens, W4 g128; FLOPs: the seven tuned GEMMs "
+                "(x3 for forward and backward) plus causal attention's six products"}
+    del fn, loss_d
+    torch.cuda.empty_cache()
     # block-by-block tuning of two SwiGLU blocks with the "light" preset: every step of the
     # method (reference forwards over all samples, gathered minibatch steps, quantized forwards)
     from post_weight_quantization_autoround_b200 import driver
@@ -554,6 +587,36 @@ def other_workloads(ar, torch, peaks, steps=10):
 # ----------------------------------------------------------------------------
 # single-kernel cases for ncu captures (inputs larger than L2, a few GB at most)
 # ----------------------------------------------------------------------------
+
+def decoder_step_fn(ar, torch, samples, seqlen, steps, H=4096, F=11008, nh=32, g=128):
+    """A Llama-7B-shaped decoder block (H 4096, F 11008, 32 heads) on ``samples`` x ``seqlen`` tokens: returns
+    (a call running ``steps`` joint tuning steps, FLOPs per step).  Synthetic weights and activations."""
+    M = samples * seqlen
+    d = synth.make_decoder(H, F, M, seed=7)
+    names = ar.DECODER_LAYERS
+    Ws = [to_dev_bf16(d[n], torch) for n in names]
+    X = to_dev_bf16(d["X"], torch)
+    g1 = torch.from_numpy(d["gamma1"]).cuda()
+    g2 = torch.from_numpy(d["gamma2"]).cuda()
+    del d
+    layers = [(W, torch.zeros(W.shape, device="cuda"), torch.ones((W.shape[0], W.shape[1] // g), device="cuda"),
+               torch.ones((W.shape[0], W.shape[1] // g), device="cuda")) for W in Ws]
+    Y = torch.empty((M, H), device="cuda")
+    fws = torch.empty(ar.ar_decoder_forward_workspace(H, F, nh, seqlen, M), dtype=torch.uint8, device="cuda")
+    ar.ar_decoder_forward(Ws, g1, g2, nh, seqlen, X, Y, fws)
+    del fws
+    cfg = ar.ar_qconfig_default(group_size=g)
+    ws = torch.empty(ar.ar_tune_step_decoder_workspace(layers, g1, g2, nh, seqlen, M, cfg, steps), dtype=torch.uint8,
+                     device="cuda")
+    loss = torch.empty(steps, device="cuda")
+    fn = lambda: ar.ar_tune_step_decoder(layers, g1, g2, nh, seqlen, X, Y, cfg, steps, loss, ws)
+    # the seven tuned GEMMs, forward and backward (2 MNK each, x3), plus causal attention
+    # (Q K^T and P V forward; dO V^T, P^T dO, dS K, dS^T Q backward; half the keys each; the scores the
+    # two-pass softmax and the backward recompute are not counted)
+    gemm = 2.0 * M * (4 * H * H + 3 * H * F) * 3
+    attn = 2.0 * samples * nh * seqlen * seqlen * (H // nh) * 6 / 2
+    return fn, gemm + attn, loss
+
 
 def run_case(name, ar, torch):
     """Three launches of one kernel family on a small case (for ``ncu -k <kernel> -s 2 -c 1``)."""
@@ -619,6 +682,8 @@ def run_case(name, ar, torch):
                          device=dev)
         loss = torch.empty(1, device=dev)
         fn = lambda: ar.ar_tune_block(ar.AR_BLOCK_SWIGLU_MLP, layers, X, Y, cfg, 1, loss, ws)
+    elif name == "decoder":  # one joint step of a Llama-7B-shaped decoder block on one 2048-token sample
+        fn = decoder_step_fn(ar, torch, 1, 2048, 1)[0]
     else:
         raise SystemExit(f"unknown case {name}; one of {', '.join(CASES)}")
     for _ in range(3):
@@ -629,7 +694,7 @@ def run_case(name, ar, torch):
     return 0 if st == 0 else 1
 
 
-CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp")
+CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp", "decoder")
 
 
 def main():

@@ -345,28 +345,33 @@ AR_API ar_status ar_w4a16_gemm(const uint16_t* A, int64_t T, const uint32_t* pac
                         const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, uint16_t* out,
                         ar_stream_t stream);
 
-/* Packed export of the tuned codes at 2, 4 or 8 bits (cfg->bits): the INT4
+/* Packed export of the tuned codes at 2, 3, 4 or 8 bits (cfg->bits): the INT4
  * layout of ar_pack_int4 for other widths (the pages define no packing for
- * them; config 4's b2/b8 tunings need one):
- *   packed  uint32 [N][K*bits/32]: element k at bits bits*(k mod 32/bits) of
- *           word k/(32/bits), little end first along K
+ * them; the low-bit tunings need one).  Each row is one little-endian bit
+ * stream: element k at stream bits [bits*k, bits*k + bits), stream bit i in
+ * bit i mod 32 of the row's word i/32.
+ *   packed  uint32 [N][K*bits/32]: for 2, 4, 8 bits element k at bits
+ *           bits*(k mod 32/bits) of word k/(32/bits); for 3 bits 32 codes in
+ *           3 words, codes 10 and 21 of every 32 straddling two words
  *   scale   fp16  [N][K/g]: fp16(s), round to nearest even
  *   zero    fp16  [N][K/g]: fp16(zp) (exact: integer < 2^bits)
- * Same codes as ar_qdq.  Needs K % (32/bits) == 0 and group_size 8..1024
- * (power of two) dividing K; 3-bit codes do not tile a 32-bit word and
- * return AR_ERR_UNSUPPORTED, as do other widths. */
+ * Same codes as ar_qdq.  Needs K % (32/bits) == 0 (3 bits: K % 32 == 0) and
+ * group_size 8..1024 (power of two) dividing K; other widths return
+ * AR_ERR_UNSUPPORTED. */
 AR_API ar_status ar_pack_codes(const uint16_t* W, const float* V, const float* alpha, const float* beta, int64_t N,
                                int64_t K, const ar_qconfig* cfg, uint32_t* packed, uint16_t* scale_f16,
                                uint16_t* zero_f16, ar_stream_t stream);
 
-/* WbA16 matmul for codes packed by ar_pack_codes (bits 2, 4 or 8):
+/* WbA16 matmul for codes packed by ar_pack_codes (bits 2, 3, 4 or 8):
  *   out[t][n] = sum_k A[t][k] (q[n][k] - zero[n][k/g]) scale[n][k/g]
  * A bf16 [T][K]; zero must hold integers 0..2^bits-1; out bf16 [T][N].  bits 4
- * is ar_w4a16_gemm; 2 and 8 run the tcgen05 dequant GEMM for every T ((q - z)
- * is exact in bf16 for all three widths; each group's sum is scaled once in
- * fp32).  Needs 1 <= T < 2^31, group_size 32..1024 (power of two) dividing K,
- * K % 128 == 0; otherwise AR_ERR_UNSUPPORTED or AR_ERR_INVALID_ARG before any
- * launch. */
+ * is ar_w4a16_gemm.  2 and 8 bits at T <= 16, and 3 bits at every T (16 tokens
+ * per launch), run a decode kernel (mma.sync, one range of weight rows per SM,
+ * the codes read straight from the bit stream); 2 and 8 bits from 17 tokens
+ * run the tcgen05 dequant GEMM.  (q - z) is exact in bf16 for every width and
+ * each group's sum is scaled once in fp32.  Needs 1 <= T < 2^31, group_size
+ * 32..1024 (power of two) dividing K, K % 128 == 0; otherwise
+ * AR_ERR_UNSUPPORTED or AR_ERR_INVALID_ARG before any launch. */
 AR_API ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, const uint16_t* scale_f16,
                                const uint16_t* zero_f16, int64_t N, int64_t K, int group_size, int bits,
                                uint16_t* out, ar_stream_t stream);

@@ -464,10 +464,13 @@ def unpack_codes(words: np.ndarray, K: int, bits: int) -> np.ndarray:
 
 
 def wxa16_matmul(A, words, scale16, zero16, group_size: int, bits: int) -> np.ndarray:
-    """out[t][n] = Σ_k A[t][k]·(q[n][k] - zero[n][k/g])·scale[n][k/g] for b-bit codes, fp64."""
+    """out[t][n] = Σ_k A[t][k]·(q[n][k] - zero[n][k/g])·scale[n][k/g] for b-bit codes, fp64.
+
+    ``words`` is the per-row bit stream of ``pack_bitstream`` (at 2, 4 and 8 bits
+    the per-word layout of ``pack_codes``; 3 bits: 32 codes in 3 words)."""
     N = words.shape[0]
-    K = words.shape[1] * (32 // bits)
-    q = unpack_codes(words, K, bits).astype(f64)
+    K = words.shape[1] * 32 // bits
+    q = unpack_bitstream(words, K, bits).astype(f64)
     s = scale16.view(np.float16).astype(f64)
     z = zero16.view(np.float16).astype(f64)
     deq = (q.reshape(N, K // group_size, group_size) - z[:, :, None]) * s[:, :, None]

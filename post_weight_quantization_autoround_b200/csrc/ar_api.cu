@@ -845,12 +845,14 @@ ar_status ar_pack_codes(const uint16_t* W, const float* V, const float* alpha, c
   ar_status st = check_cfg(cfg);
   if (st != AR_OK) return st;
   const int bits = cfg->bits;
-  if (bits != 2 && bits != 4 && bits != 8)
-    return fail(AR_ERR_UNSUPPORTED, "ar_pack_codes packs 2, 4 or 8-bit codes (got %d)", bits);
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
+    return fail(AR_ERR_UNSUPPORTED, "ar_pack_codes packs 2, 3, 4 or 8-bit codes (got %d)", bits);
   const int g = cfg->group_size;
   if (N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "N, K must be positive");
   if (!pow2(g) || g < 8 || g > 1024) return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 8..1024", g);
-  if (K % g != 0 || K % (32 / bits) != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and of 32/bits");
+  // every row holds a whole number of 32-bit words: K bits / 32
+  const int kmul = bits == 3 ? 32 : 32 / bits;
+  if (K % g != 0 || K % kmul != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of group_size and of %d", kmul);
   const void* ptrs[] = {W, V, alpha, beta, packed, scale_f16, zero_f16};
   for (const void* p : ptrs) {
     if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
@@ -867,7 +869,7 @@ ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
                         ar_stream_t stream) {
   if (bits == 4) return ar_w4a16_gemm(A, T, packed, scale_f16, zero_f16, N, K, group_size, out, stream);
   begin_call();
-  if (bits != 2 && bits != 8) return fail(AR_ERR_UNSUPPORTED, "bits=%d: needs 2, 4 or 8", bits);
+  if (bits != 2 && bits != 3 && bits != 8) return fail(AR_ERR_UNSUPPORTED, "bits=%d: needs 2, 3, 4 or 8", bits);
   if (T < 1 || N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "T, N, K must be positive");
   if (!pow2(group_size) || group_size < 32 || group_size > 1024)
     return fail(AR_ERR_UNSUPPORTED, "group_size %d: needs a power of two in 32..1024", group_size);
@@ -878,8 +880,15 @@ ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
     if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   }
-  cudaError_t e = launch_wxa16_tc(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N),
-                                  static_cast<int>(K), group_size, bits, out, reinterpret_cast<cudaStream_t>(stream));
+  // decode batches and every 3-bit call: the mma.sync decode kernel (16 tokens at a time);
+  // 2 and 8 bits from 17 tokens: the tcgen05 dequant GEMM
+  cudaError_t e = (bits == 3 || T <= 16)
+                      ? launch_wbx_dec(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N),
+                                       static_cast<int>(K), group_size, bits, out,
+                                       reinterpret_cast<cudaStream_t>(stream))
+                      : launch_wxa16_tc(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N),
+                                        static_cast<int>(K), group_size, bits, out,
+                                        reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "wxa16 launch");
   return end_call();
 }

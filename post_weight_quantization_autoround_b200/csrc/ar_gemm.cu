@@ -111,6 +111,8 @@ static_assert(sizeof(Ctl) <= 24576, "control block too large");
 struct Params {
   int M, N, K;  // D is M x N, reduction over K
   int tiles_m, tiles_n, num_kb;
+  int num_units;   // work units of this launch (tiles, or half tiles of a pair grid's tail)
+  int tail_pair0;  // >= 0: unit u is half u % 2 of tile tail_pair0 + u / 2 of the 256-row pair grid
   float* D;          // EPI_STORE
   const float* Y;    // EPI_RESID
   uint16_t* G;
@@ -626,6 +628,18 @@ __device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, 
   return bad;
 }
 
+// Output tile (tm, tn) of work unit t, in this launch's BM * CG-row tiles.
+__device__ __forceinline__ void unit_coords(const Params& p, int t, int& tm, int& tn) {
+  if (p.tail_pair0 >= 0) {
+    const int tp = p.tail_pair0 + (t >> 1);
+    tm = 2 * (tp / p.tiles_n) + (t & 1);
+    tn = tp % p.tiles_n;
+  } else {
+    tm = t / p.tiles_n;
+    tn = t - tm * p.tiles_n;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
@@ -650,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &ctl->abort_flag;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int num_tiles = p.num_units;
   const int rank = kCluster ? static_cast<int>(cluster_ctarank()) : 0;
   const int tile0 = kCluster ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
   const int tile_step = kCluster ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
@@ -703,8 +717,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued = 0;
       bool ok = true;
       for (int t = tile0; ok && t < num_tiles; t += tile_step) {
-        const int tm = t / p.tiles_n;
-        const int tn = t - tm * p.tiles_n;
+        int tm, tn;
+        unit_coords(p, t, tm, tn);
         // this CTA's A rows and B columns
         const int m0 = tm * (BM * CG) + rank * (kPair ? BM : 0);
         const int n0 = tn * BN + rank * (kPair ? BN / 2 : 0);
@@ -839,8 +853,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t peer_slot = KSPLIT == 2 ? mapa_shared(smem_u32(&ctl->slot[ew][lane][0]), 0) : 0;
     const uint32_t peer_full = KSPLIT == 2 ? mapa_shared(smem_u32(&ctl->full_x[ew]), 0) : 0;
     for (int t = tile0; t < num_tiles; t += tile_step) {
-      const int tm = t / p.tiles_n;
-      const int tn = t - tm * p.tiles_n;
+      int tm, tn;
+      unit_coords(p, t, tm, tn);
       const int row = tm * (BM * CG) + rank * (kPair ? BM : 0) + quarter * 32 + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       auto wait_acc = [&]() {
@@ -952,11 +966,15 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
   p.tiles_m = (p.M + BM * CG - 1) / (BM * CG);
   p.tiles_n = EPI == EPI_SWIGLU_FWD ? (p.N + BN / 2 - 1) / (BN / 2) : (p.N + BN - 1) / BN;
   p.num_kb = (p.K + BK - 1) / BK;
+  if (p.num_units <= 0) {
+    p.num_units = p.tiles_m * p.tiles_n;
+    p.tail_pair0 = -1;
+  }
   auto kern = umma_gemm_kernel<A_MN, B_MN, EPI, KSPLIT, CG>;
   constexpr int kSmemBytes = GemmCfg<CG>::kSmemBytes;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int tiles = p.tiles_m * p.tiles_n;
+  const int tiles = p.num_units;
   if (KSPLIT == 1 && CG == 1) {
     const int grid = tiles < num_sms() ? tiles : num_sms();
     LaunchScope scope(stream, name);
@@ -1090,6 +1108,23 @@ cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArg
   const double eff2 = static_cast<double>(tiles_split) / (((tiles_split + pairs - 1) / pairs) * pairs);
   if (M >= 32768 && eff2 > eff1 + 0.02)
     return run<true, true, EPI_FOLD, 2>(G, X, p, stream, "umma_gemm<MN,MN,fold,split2>", nullptr, ldg, ldx);
+  // A last wave that leaves many pairs idle: the full waves run as pair tiles,
+  // then the tail's tiles as 128-row halves whose reduction the two CTAs of a
+  // cluster split, so the tail's work spreads over every pair (each half tile
+  // is a quarter of a pair tile's MMA work per cluster).
+  const int rem = tiles_pair % pairs;
+  if (tiles_pair > pairs && rem > 0 && 2 * rem <= pairs) {
+    Params pp = p;
+    pp.num_units = tiles_pair - rem;
+    pp.tail_pair0 = -1;
+    cudaError_t e = run<true, true, EPI_FOLD, 1, kPairCG>(G, X, pp, stream, "umma_gemm<MN,MN,fold,pair>", nullptr,
+                                                          ldg, ldx);
+    if (e != cudaSuccess) return e;
+    Params pt = p;
+    pt.num_units = 2 * rem;
+    pt.tail_pair0 = tiles_pair - rem;
+    return run<true, true, EPI_FOLD, 2>(G, X, pt, stream, "umma_gemm<MN,MN,fold,split2_tail>", nullptr, ldg, ldx);
+  }
   return run<true, true, EPI_FOLD, 1, kPairCG>(G, X, p, stream, "umma_gemm<MN,MN,fold,pair>", nullptr, ldg, ldx);
 }
 

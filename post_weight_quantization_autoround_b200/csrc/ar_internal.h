@@ -169,6 +169,10 @@ cudaError_t launch_gather_samples(const void* src, int64_t sample_bytes, const i
 // T > 16: tcgen05 dequant GEMM (ar_w4a16_tc.cu)
 cudaError_t launch_w4a16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream);
+// 2, 3 or 8-bit codes (ar_wbx_dec.cu): mma.sync decode kernel, 16 tokens at a time
+cudaError_t launch_wbx_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                           const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,
+                           cudaStream_t stream);
 // 2, 4 or 8-bit codes (32/bits per uint32), any T: the same tcgen05 GEMM
 cudaError_t launch_wxa16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                             const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,

@@ -176,10 +176,12 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ W
   (void)groups_per_row;
 }
 
-// Packed export: the same codes as qdq_kernel, BITS (2, 4 or 8) bits each,
-// packed little end first along K (element k at bits BITS*(k mod 32/BITS) of
-// word k/(32/BITS); INT4: nibbles), plus fp16 scale / zero per group.  A
-// thread's 8 codes fill BITS bytes.
+// Packed export: the same codes as qdq_kernel, BITS (2, 3, 4 or 8) bits each, as
+// one little-endian bit stream per row: element k at stream bits [BITS k,
+// BITS k + BITS), stream bit i in bit i mod 32 of word i / 32 (2, 4, 8 bits:
+// element k at bits BITS*(k mod 32/BITS) of word k/(32/BITS); INT4: nibbles;
+// 3 bits: 32 codes in 3 words, codes 10 and 21 straddling two), plus fp16
+// scale / zero per group.  A thread's 8 codes fill BITS whole bytes.
 template <int TPG, int CHUNKS, int BITS>
 __global__ void __launch_bounds__(256) pack_codes_kernel(const uint16_t* __restrict__ W, const float* __restrict__ V,
                                                          const float* __restrict__ alpha,
@@ -236,9 +238,17 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(const uint16_t* __restr
       bits |= static_cast<uint64_t>(q) << (BITS * i);
     }
     uint8_t* dst = packed + (e * BITS) / 8;
-    if (BITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bits);
-    else if (BITS == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(bits);
-    else *reinterpret_cast<uint2*>(dst) = make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
+    if (BITS == 2) {
+      *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bits);
+    } else if (BITS == 3) {  // 24 bits at byte offset 3 (e / 8): three byte stores
+      dst[0] = static_cast<uint8_t>(bits);
+      dst[1] = static_cast<uint8_t>(bits >> 8);
+      dst[2] = static_cast<uint8_t>(bits >> 16);
+    } else if (BITS == 4) {
+      *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(bits);
+    } else {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
+    }
   }
   if (li == 0) {
     scale16[grp] = __float2half_rn(p.s);
@@ -311,9 +321,10 @@ cudaError_t launch_pack_bits(const uint16_t* W, const float* V, const float* alp
   case (TPG_ * 8 * CH_): {                                                                                    \
     const int64_t threads = n_groups * TPG_;                                                                  \
     const int blocks = static_cast<int>((threads + 255) / 256);                                               \
-    LaunchScope scope(stream, BITS == 4 ? "pack_codes_kernel<b=4,g=" #TPG_ "x8x" #CH_ ">"                      \
-                                        : BITS == 2 ? "pack_codes_kernel<b=2,g=" #TPG_ "x8x" #CH_ ">"          \
-                                                    : "pack_codes_kernel<b=8,g=" #TPG_ "x8x" #CH_ ">");        \
+    LaunchScope scope(stream, BITS == 4   ? "pack_codes_kernel<b=4,g=" #TPG_ "x8x" #CH_ ">"                    \
+                              : BITS == 2 ? "pack_codes_kernel<b=2,g=" #TPG_ "x8x" #CH_ ">"                    \
+                              : BITS == 3 ? "pack_codes_kernel<b=3,g=" #TPG_ "x8x" #CH_ ">"                    \
+                                          : "pack_codes_kernel<b=8,g=" #TPG_ "x8x" #CH_ ">");                  \
     pack_codes_kernel<TPG_, CH_, BITS><<<blocks, 256, 0, stream>>>(W, V, alpha, beta, n_groups, symmetric,    \
                                                                    packed, s16, z16);                         \
     break;                                                                                                    \
@@ -346,6 +357,7 @@ cudaError_t launch_pack_codes(const uint16_t* W, const float* V, const float* al
                               uint16_t* scale16, uint16_t* zero16, cudaStream_t stream) {
   uint8_t* dst = reinterpret_cast<uint8_t*>(packed);
   if (bits == 2) return launch_pack_bits<2>(W, V, alpha, beta, N, K, group_size, symmetric, dst, scale16, zero16, stream);
+  if (bits == 3) return launch_pack_bits<3>(W, V, alpha, beta, N, K, group_size, symmetric, dst, scale16, zero16, stream);
   if (bits == 4) return launch_pack_bits<4>(W, V, alpha, beta, N, K, group_size, symmetric, dst, scale16, zero16, stream);
   if (bits == 8) return launch_pack_bits<8>(W, V, alpha, beta, N, K, group_size, symmetric, dst, scale16, zero16, stream);
   return cudaErrorInvalidValue;

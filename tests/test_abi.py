@@ -148,14 +148,17 @@ def test_gather_samples_validation():
 
 
 def test_pack_codes_and_wxa16_validation():
-    c3 = ar.ar_qconfig_default(bits=3)
-    assert ar.lib().ar_pack_codes(FAKE, FAKE, FAKE, FAKE, 8, 128, ctypes.byref(c3), FAKE, FAKE, FAKE, None) == \
+    c5 = ar.ar_qconfig_default(bits=5)
+    assert ar.lib().ar_pack_codes(FAKE, FAKE, FAKE, FAKE, 8, 128, ctypes.byref(c5), FAKE, FAKE, FAKE, None) == \
         ar.AR_ERR_UNSUPPORTED
+    c3 = ar.ar_qconfig_default(bits=3, group_size=16)
+    assert ar.lib().ar_pack_codes(FAKE, FAKE, FAKE, FAKE, 8, 48, ctypes.byref(c3), FAKE, FAKE, FAKE, None) == \
+        ar.AR_ERR_INVALID_ARG  # 3-bit rows fill whole words: K % 32
     c2 = ar.ar_qconfig_default(bits=2, group_size=8)
     assert ar.lib().ar_pack_codes(FAKE, FAKE, FAKE, FAKE, 8, 8, ctypes.byref(c2), FAKE, FAKE, FAKE, None) == \
         ar.AR_ERR_INVALID_ARG  # K % 16 for 2-bit words
     w = ar.lib().ar_wxa16_gemm
-    assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 128, 3, FAKE, None) == ar.AR_ERR_UNSUPPORTED
+    assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 128, 5, FAKE, None) == ar.AR_ERR_UNSUPPORTED
     assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 256, 16, 2, FAKE, None) == ar.AR_ERR_UNSUPPORTED
     assert w(FAKE, 1, FAKE, FAKE, FAKE, 64, 192, 64, 8, FAKE, None) == ar.AR_ERR_INVALID_ARG  # K % 128
     assert w(FAKE, 0, FAKE, FAKE, FAKE, 64, 256, 128, 2, FAKE, None) == ar.AR_ERR_INVALID_ARG

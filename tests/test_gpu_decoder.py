@@ -10,9 +10,14 @@ decoder section), so the two differ only in summation order:
     2^-9 relative per entry, plus probabilities whose rounding flips between
     summation orders), lse within 1e-5;
   * the block forward: Y within 1e-4 relative L2;
-  * one joint tuning step: loss within 1e-3, every layer's dV, dalpha, dbeta
-    within 1e-3 relative L2 with >= 99.9 % sign agreement where |g| > 1e-3 RMS,
-    and the update equal on >= 99.9 % (V) / 99 % (alpha, beta) of entries.
+  * one joint tuning step: loss within 1e-3; dV, dalpha, dbeta of o, gate, up,
+    down within 1e-3 relative L2 and of q, k, v within 2.5e-3 (their gradients
+    pass through every rounding point of the block: perturbing each rounding
+    point's input by 2^-24 relative, the size of one fp32 rounding, already moves
+    them by ~6e-4 in the oracle itself, see test_oracle_pins.py), >= 99.9 % sign
+    agreement where |g| > 1e-3 RMS, and the update equal on >= 99 % of alpha,
+    beta and on >= 99.9 % of V (q, k, v: >= 99.7 %; the same perturbation
+    already flips the sign of 0.06 % of their near-zero dV).
 
 [AR] = "Low-Bit Quantization in Practice with vLLM: Core Mechanisms and
 Architectural Optimizations of AutoRound".
@@ -27,7 +32,9 @@ from oracle import autoround_oracle as O
 pytestmark = pytest.mark.gpu
 
 GRAD_RTOL = 1e-3
+QKV_GRAD_RTOL = 2.5e-3
 SIGN_AGREE = 0.999
+QKV_UPDATE_AGREE = 0.997
 CLIP_AGREE = 0.99
 ATTN_RTOL = 3e-3
 
@@ -189,11 +196,13 @@ def _check_step(out, st_gpu, ref_loss, ref_new, ref_grads):
     for li, n in enumerate(O.DECODER_LAYERS):
         for k in range(3):
             got, ref = out["grads"][li][k], ref_grads[n][k]
-            assert rel_l2(got, ref) <= GRAD_RTOL, (n, k, rel_l2(got, ref))
+            tol = QKV_GRAD_RTOL if n in ("q", "k", "v") else GRAD_RTOL
+            assert rel_l2(got, ref) <= tol, (n, k, rel_l2(got, ref))
             rms = np.sqrt(np.mean(np.asarray(ref, np.float64) ** 2))
             mask = np.abs(ref) > 1e-3 * rms
             assert np.mean(np.sign(got[mask]) == np.sign(ref[mask])) >= SIGN_AGREE, (n, k)
-        assert np.mean(st_gpu[n][0] == ref_new[n][0]) >= SIGN_AGREE, n
+        agree = QKV_UPDATE_AGREE if n in ("q", "k", "v") else SIGN_AGREE
+        assert np.mean(st_gpu[n][0] == ref_new[n][0]) >= agree, (n, np.mean(st_gpu[n][0] == ref_new[n][0]))
         for k in (1, 2):
             assert np.mean(st_gpu[n][k] == ref_new[n][k]) >= CLIP_AGREE, (n, k)
 

@@ -255,6 +255,26 @@ def test_single_step_matches_oracle(ar, N, K, M, bits, g, sym, spread):
     assert np.mean(Vg == V1) >= SIGN_AGREE and np.mean(ag == a1) >= 0.99 and np.mean(bg == b1) >= 0.99
 
 
+def test_weight_gradient_tail_runs_split_half_tiles(ar):
+    """80 pair tiles on 74 CTA pairs: the full wave on pairs, the 6-tile tail as 12 half tiles whose reduction
+    two CTAs split; the step still matches the oracle."""
+    N, K, M, g = 1280, 4096, 256, 128
+    d = synth.make_linear(N, K, M, seed=77, x_outlier_channels=4)
+    V, a, b = synth.make_state(N, K, g, seed=5, spread=True)
+    cfg, ocfg = cfg_pair(ar)
+    gl = GpuLinear(ar, d["W"], d["X"], V, a, b, cfg)
+    out = gl.step(1, grads=True)
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert "split2_tail" in ar.ar_last_kernels(), ar.ar_last_kernels()
+    Wf, Xf = synth.bf16_bits_to_f32(d["W"]), synth.bf16_bits_to_f32(d["X"])
+    L, (V1, a1, b1), gr, _ = O.tune_step_linear(Wf, Xf, O.reference_forward(Xf, Wf), V, a, b, ocfg)
+    assert out["loss"][0] == pytest.approx(L, rel=1e-4)
+    for k in ("dV", "dalpha", "dbeta"):
+        assert rel_l2(out[k], gr[k]) <= GRAD_RTOL, (k, rel_l2(out[k], gr[k]))
+    Vg, ag, bg = gl.state()
+    assert np.mean(Vg == V1) >= SIGN_AGREE and np.mean(ag == a1) >= 0.99 and np.mean(bg == b1) >= 0.99
+
+
 def test_eval_only_call_updates_nothing(ar):
     d = synth.make_linear(64, 256, 96, seed=5)
     V, a, b = synth.make_state(64, 256, 128, seed=5, spread=True)

@@ -1,6 +1,7 @@
-"""2- and 8-bit packed export and the WbA16 matmul (the INT4 layout and the
+"""2-, 3- and 8-bit packed export and the WbA16 matmul (the INT4 layout and the
 tcgen05 dequant GEMM generalised; the pages define no packing for these
-widths) against the oracle."""
+widths) against the oracle.  Packing follows the oracle's per-row bit stream
+(``pack_bitstream``), which at 2, 4 and 8 bits is the per-word layout."""
 import numpy as np
 import pytest
 import torch
@@ -47,7 +48,7 @@ def pack_gpu(ar, Wbits, V, a, b, bits, g, sym=False):
     return packed, s16, z16
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
 @pytest.mark.parametrize("g,sym", [(32, False), (128, False), (128, True), (256, False)])
 def test_pack_codes_bit_exact(ar, bits, g, sym):
     N, K = 136, 1024
@@ -56,24 +57,28 @@ def test_pack_codes_bit_exact(ar, bits, g, sym):
     packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, bits, g, sym)
     assert "pack_codes_kernel<b=%d" % bits in ar.ar_last_kernels()
     st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, bits, g, sym)
-    assert np.array_equal(packed.cpu().numpy().view(np.uint32), O.pack_codes(st["q"], bits))
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), O.pack_bitstream(st["q"], bits))
     assert np.array_equal(s16.cpu().numpy(), np.asarray(st["s"], np.float32).astype(np.float16))
     assert np.array_equal(z16.cpu().numpy(), np.asarray(st["zp"], np.float32).astype(np.float16))
 
 
-@pytest.mark.parametrize("bits", [2, 8])
-@pytest.mark.parametrize("T", [1, 16, 40, 256])
-@pytest.mark.parametrize("N,K,g", [(320, 1024, 128), (64, 4096, 32), (200, 2048, 256)])
+@pytest.mark.parametrize("bits", [2, 3, 8])
+@pytest.mark.parametrize("T", [1, 5, 16, 40, 256])
+@pytest.mark.parametrize("N,K,g", [(320, 1024, 128), (64, 4096, 32), (200, 2048, 256), (1000, 768, 64)])
 def test_wxa16_matches_oracle(ar, bits, T, N, K, g):
     d = synth.make_linear(N, K, 1, seed=T + N + bits)
     V, a, b = synth.make_state(N, K, g, seed=2, spread=True)
     packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, bits, g)
     A = synth.make_activations(T, K, seed=T)
-    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, bits, out)
-    assert "wxa16_tc_kernel<b=%d" % bits in ar.ar_last_kernels()
+    assert ar.ar_get_device_status() == 0
+    if bits == 3 or T <= 16:
+        assert "wbx_dec_kernel<b=%d" % bits in ar.ar_last_kernels()
+    else:
+        assert "wxa16_tc_kernel<b=%d" % bits in ar.ar_last_kernels()
     st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, bits, g)
-    words = O.pack_codes(st["q"], bits)
+    words = O.pack_bitstream(st["q"], bits)
     ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16),
                          z16.cpu().numpy().view(np.uint16), g, bits)
     assert rel_l2(out.float().cpu().numpy(), ref) <= TC_RTOL
