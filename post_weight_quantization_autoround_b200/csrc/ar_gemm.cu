@@ -50,6 +50,8 @@
 // Every mbarrier wait is bounded (ar_device.cuh): on a timeout the kernel
 // raises a block abort flag and the sticky device status, all roles leave
 // their loops, in-flight TMA copies and MMAs are drained, TMEM is freed.
+#include <algorithm>
+
 #include "ar_internal.h"
 
 namespace ar {
@@ -111,8 +113,8 @@ static_assert(sizeof(Ctl) <= 24576, "control block too large");
 struct Params {
   int M, N, K;  // D is M x N, reduction over K
   int tiles_m, tiles_n, num_kb;
-  int num_units;   // work units of this launch (tiles, or half tiles of a pair grid's tail)
-  int tail_pair0;  // >= 0: unit u is half u % 2 of tile tail_pair0 + u / 2 of the 256-row pair grid
+  int num_units;   // work units (tiles) of this launch
+  int group_m;     // tile rows per raster group (columns swept inside a group, rows fastest)
   float* D;          // EPI_STORE
   const float* Y;    // EPI_RESID
   uint16_t* G;
@@ -628,16 +630,35 @@ __device__ __forceinline__ bool epi_swiglu_bwd(const Params& p, uint32_t taddr, 
   return bad;
 }
 
+// Tile (tm, tn) of unit t of a grid of tiles_m x tiles_n tiles in raster order:
+// groups of group_m tile rows, and inside a group the row index fastest (group_m
+// = 1: rows one after another, columns fastest).
+__host__ __device__ __forceinline__ void raster(int t, int tiles_m, int tiles_n, int group_m, int& tm, int& tn) {
+  if (group_m <= 1) {
+    tm = t / tiles_n;
+    tn = t - tm * tiles_n;
+    return;
+  }
+  const int per_group = group_m * tiles_n;
+  const int grp = t / per_group;
+  const int in = t - grp * per_group;
+  const int rows = min(group_m, tiles_m - grp * group_m);
+  tn = in / rows;
+  tm = grp * group_m + (in - tn * rows);
+}
+
 // Output tile (tm, tn) of work unit t, in this launch's BM * CG-row tiles.
 __device__ __forceinline__ void unit_coords(const Params& p, int t, int& tm, int& tn) {
-  if (p.tail_pair0 >= 0) {
-    const int tp = p.tail_pair0 + (t >> 1);
-    tm = 2 * (tp / p.tiles_n) + (t & 1);
-    tn = tp % p.tiles_n;
-  } else {
-    tm = t / p.tiles_n;
-    tn = t - tm * p.tiles_n;
-  }
+  raster(t, p.tiles_m, p.tiles_n, p.group_m, tm, tn);
+}
+
+// Raster group for a grid whose B operand has b_bytes: 1 while B fits in a share of
+// L2 (B stays resident, A streams once), else as many tile rows as that share holds
+// A panels of (A streams once, B once per group).
+int raster_group(double b_bytes, double a_panel_bytes, int tiles_m) {
+  constexpr double kL2Share = 64.0 * 1024 * 1024;
+  if (b_bytes <= kL2Share) return 1;
+  return std::max(1, std::min(tiles_m, static_cast<int>(kL2Share / a_panel_bytes)));
 }
 
 // ---------------------------------------------------------------------------
@@ -966,9 +987,11 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
   p.tiles_m = (p.M + BM * CG - 1) / (BM * CG);
   p.tiles_n = EPI == EPI_SWIGLU_FWD ? (p.N + BN / 2 - 1) / (BN / 2) : (p.N + BN - 1) / BN;
   p.num_kb = (p.K + BK - 1) / BK;
-  if (p.num_units <= 0) {
-    p.num_units = p.tiles_m * p.tiles_n;
-    p.tail_pair0 = -1;
+  p.num_units = p.tiles_m * p.tiles_n;
+  // raster order
+  {
+    const double b_bytes = static_cast<double>(p.N) * p.K * 2 * (EPI == EPI_SWIGLU_FWD ? 2 : 1);
+    p.group_m = raster_group(b_bytes, static_cast<double>(BM * CG) * p.K * 2, p.tiles_m);
   }
   auto kern = umma_gemm_kernel<A_MN, B_MN, EPI, KSPLIT, CG>;
   constexpr int kSmemBytes = GemmCfg<CG>::kSmemBytes;
@@ -1108,23 +1131,6 @@ cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArg
   const double eff2 = static_cast<double>(tiles_split) / (((tiles_split + pairs - 1) / pairs) * pairs);
   if (M >= 32768 && eff2 > eff1 + 0.02)
     return run<true, true, EPI_FOLD, 2>(G, X, p, stream, "umma_gemm<MN,MN,fold,split2>", nullptr, ldg, ldx);
-  // A last wave that leaves many pairs idle: the full waves run as pair tiles,
-  // then the tail's tiles as 128-row halves whose reduction the two CTAs of a
-  // cluster split, so the tail's work spreads over every pair (each half tile
-  // is a quarter of a pair tile's MMA work per cluster).
-  const int rem = tiles_pair % pairs;
-  if (tiles_pair > pairs && rem > 0 && 2 * rem <= pairs) {
-    Params pp = p;
-    pp.num_units = tiles_pair - rem;
-    pp.tail_pair0 = -1;
-    cudaError_t e = run<true, true, EPI_FOLD, 1, kPairCG>(G, X, pp, stream, "umma_gemm<MN,MN,fold,pair>", nullptr,
-                                                          ldg, ldx);
-    if (e != cudaSuccess) return e;
-    Params pt = p;
-    pt.num_units = 2 * rem;
-    pt.tail_pair0 = tiles_pair - rem;
-    return run<true, true, EPI_FOLD, 2>(G, X, pt, stream, "umma_gemm<MN,MN,fold,split2_tail>", nullptr, ldg, ldx);
-  }
   return run<true, true, EPI_FOLD, 1, kPairCG>(G, X, p, stream, "umma_gemm<MN,MN,fold,pair>", nullptr, ldg, ldx);
 }
 

@@ -1075,11 +1075,12 @@ def test_decoder_rounding_points_stay_within_bf16_noise_of_fp64():
 
 
 def test_decoder_attention_weight_gradients_sit_at_a_rounding_noise_floor(monkeypatch):
-    """The GPU tolerance for q, k, v (2.5e-3, against 1e-3 for the other weights) comes from this floor:
-    perturbing the input of every rounding point by 2^-24 relative (one fp32 rounding) moves the attention
-    weights' gradients by several 1e-4, several times more than the MLP weights' (bf16 rounding flips
-    upstream of the loss, amplified through the chain); an implementation summing in another order in fp32
-    differs by more."""
+    """The decoder block's GPU tolerances are measured against this floor: perturbing the input of every
+    rounding point by 2^-24 relative (one fp32 rounding) moves the attention weights' gradients by several
+    1e-4, several times more than the down projection's (bf16 rounding flips upstream of the loss,
+    amplified through the chain), and flips the update of a few near-zero dV; an implementation summing in
+    another order in fp32 differs by more.  (The GPU test measures the same floor at 2^-22 on each of its
+    own problems and allows 3x it.)"""
     rng = np.random.default_rng(0)
     S, L, H, F, nh, g = 2, 128, 256, 512, 2, 128
     d = synth.make_decoder(H, F, S * L, seed=22)
@@ -1106,7 +1107,7 @@ def test_decoder_attention_weight_gradients_sit_at_a_rounding_noise_floor(monkey
     assert max(rel[n] for n in ("q", "k", "v")) > 2e-4                        # a real floor, not zero
     assert max(rel[n] for n in ("q", "k", "v")) > 2 * max(rel["o"], rel["down"])  # largest far from the loss
     assert max(rel.values()) < 2.5e-3 / 2                                     # the tolerance has room above it
-    # and the V updates: near-zero dV of q, k, v flip sign at this floor, well above the GPU bar of 99.7 %
+    # and the V updates: near-zero dV of q, k, v flip sign at this floor
     same_v = {n: np.mean(new0[n][0] == new1[n][0]) for n in ("q", "k", "v")}
     assert min(same_v.values()) < 1.0 and min(same_v.values()) > 0.9985, same_v
 
