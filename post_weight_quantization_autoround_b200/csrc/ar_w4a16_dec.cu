@@ -109,6 +109,20 @@ __device__ __forceinline__ void mma16816_z(float (&d)[4], const uint32_t (&a)[4]
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// (x & 0x000F000F) | 0x43004300 as one three-input logic op: the bf16 pair
+// (128 + nibble 0, 128 + nibble 4) of x.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t x) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(x), "r"(0x000F000Fu), "r"(0x43004300u));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t shr(uint32_t x, uint32_t n) {
+  uint32_t d;
+  asm("shf.r.clamp.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(x), "r"(0u), "r"(n));
+  return d;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -262,10 +276,10 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               {
                 const uint32_t x = *reinterpret_cast<const uint32_t*>(cj + jt * 8 * 128);
                 // MMA 0 slots (2c, 2c+1) <- nibbles (0, 4), (2c+8, 2c+9) <- (1, 5); MMA 1: (2, 6), (3, 7)
-                const uint32_t b00 = (x & 0x000F000Fu) | 0x43004300u;
-                const uint32_t b01 = ((x >> 4) & 0x000F000Fu) | 0x43004300u;
-                const uint32_t b10 = ((x >> 8) & 0x000F000Fu) | 0x43004300u;
-                const uint32_t b11 = ((x >> 12) & 0x000F000Fu) | 0x43004300u;
+                const uint32_t b00 = nib_pair(x);
+                const uint32_t b01 = nib_pair(shr(x, 4));
+                const uint32_t b10 = nib_pair(shr(x, 8));
+                const uint32_t b11 = nib_pair(shr(x, 12));
                 if (first) {
                   mma16816_z(d[jt], A0, b00, b01);
                 } else {
