@@ -10,11 +10,15 @@
 // SM is the 4-bit -> bf16 conversion (about 7 integer instructions per eight
 // codes).  The layout is chosen so that nothing else costs per weight:
 //
-//  * The weights are the B operand of mma.sync m16n8k16 (an n8 tile is eight
-//    weight rows) and the activations the A operand (16 token rows, rows past
-//    T repeat the last token and are discarded).  Eight-row tiles let every
-//    SM own the same number of rows (8192 rows -> 147 CTAs of 56 rows), and
-//    up to 16 tokens cost no extra MMAs.
+//  * Rows are handed out in groups of eight, so every SM owns the same number
+//    of rows (8192 rows -> 147 CTAs of 56 rows).  Up to 8 tokens, the weights
+//    are the A operand of mma.sync m16n8k16 (a 16-row tile is two row groups;
+//    each lane converts one word of row g and one of row g + 8, so a word
+//    costs one MMA) and the activations the B operand (8 token columns,
+//    columns past T repeat the last token and are discarded).  From 9 to 16
+//    tokens the roles swap: the weights are the B operand (an n8 tile is one
+//    row group, two MMAs a word) and the activations the A operand (16 token
+//    rows).
 //  * Codes -> bf16 pairs without arithmetic: (word >> 4i) & 0x000F000F |
 //    0x43004300 is the bf16 pair (128 + q_i, 128 + q_{i+4}).  One more MMA
 //    against a fragment of ones gives O = sum of the activations over the same
@@ -22,14 +26,20 @@
 //    group span in fp32.
 //  * The reduction index of the MMA is permuted: lane (g = lane/4, c = lane%4)
 //    feeds k-slots {2c, 2c+1, 2c+8, 2c+9} of two consecutive MMAs from one
-//    32-bit word (eight codes, k = 32j + 8c + 0..7) of its weight row, and the
-//    activations are permuted the same way with byte permutes.
+//    32-bit word (eight codes, k = 32j + 8c + 0..7) of a weight row, and the
+//    activations are permuted the same way with byte permutes.  Both operand
+//    arrangements use the same k-slots, so they give bit-identical sums.
 //  * One producer warp streams 512-k stages with TMA: the codes of the pass's
 //    rows (two 256-k boxes, 128-byte swizzle, so that the fragment reads are
 //    free of bank conflicts), the activations, and the window of fp16
 //    (scale, zero) groups the stage touches.  Consumer warps work in groups of
 //    four (one 128-k chunk each) and the groups take stages in turn, so each
-//    warp owns whole group spans of its chunk.
+//    warp owns whole group spans of its chunk.  The ring depth is a multiple
+//    of the number of groups, so a slot is always taken by the same group and
+//    its waits on the slot's barrier follow the barrier's phases in order (a
+//    parity wait cannot tell a phase from the one two before it: were two
+//    groups to share a slot, one could pass its wait on a fill that another
+//    group's previous phase completed).
 //  * A CTA's rows are cut into passes of at most 64; the consumer warps' sums
 //    are added in a fixed order through shared memory at the end of a pass.
 //    For small N the two CTAs of a cluster split K and rank 0 adds the
@@ -57,7 +67,7 @@ constexpr int kDecSmemLimit = 227 * 1024;
 
 template <bool TBIG>
 struct DecCfg {
-  static constexpr int kWarps = TBIG ? 8 : 12;  // consumer warps
+  static constexpr int kWarps = 8;              // consumer warps
   static constexpr int kGroups = kWarps / 4;    // stages in consumption at once
   static constexpr int kThreads = (kWarps + 1) * 32;
   // registers per thread: the warps are spread over the SM's four 16K-register
@@ -83,7 +93,7 @@ struct DecParams {
 };
 
 struct alignas(16) DecTail {
-  float2 sm[12][kDecPassRows];  // per consumer warp: (s, -s (128 + z)) of the pass's rows for one group
+  float2 sm[8][kDecPassRows];   // per consumer warp: (s, -s (128 + z)) of the pass's rows for one group
   uint64_t full[kDecMaxStages];
   uint64_t empty[kDecMaxStages];
   float part[kDecPassRows][16];
@@ -220,11 +230,15 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
     for (int pass = 0; pass < passes_here; ++pass) {
       const bool last = pass == p.passes - 1;
       const int h = min(last ? p.last_rows : kDecPassRows, rows_here - pass * kDecPassRows);
-      float acc[NT][C::kAcc];
+      // T <= 8: MT 16-row tiles x (row g, g + 8) x (token 2c, 2c + 1); else NT row groups x kAcc
+      constexpr int MT = (NT + 1) / 2;
+      constexpr int kTiles = TBIG ? NT : MT;
+      constexpr int kAccN = TBIG ? C::kAcc : 4;
+      float acc[kTiles][kAccN];
 #pragma unroll
-      for (int jt = 0; jt < NT; ++jt)
+      for (int jt = 0; jt < kTiles; ++jt)
 #pragma unroll
-        for (int i = 0; i < C::kAcc; ++i) acc[jt][i] = 0.0f;
+        for (int i = 0; i < kAccN; ++i) acc[jt][i] = 0.0f;
 
       const int it_begin = pass * nks;
       const int it_end = it_begin + nks;
@@ -242,6 +256,80 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
           const uint16_t* zr = sc + p.wg * kDecPassRows;
           const int gi0 = (ks * kDecStageK) >> p.group_shift;
           const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
+          if constexpr (!TBIG) {
+            // weights as the A operand: tile mt holds row groups 2 mt and 2 mt + 1 (rows g and g + 8
+            // of the lane); an odd last row group leaves the tile's lower half zero
+            float d[MT][4], o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              // activations of this lane's k-range (eight bf16) for token column g
+              const uint4 v = *reinterpret_cast<const uint4*>(act + tok_lo * 512 + 64 * j);
+              const uint32_t b0[2] = {__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632)};  // (k0,k4) (k1,k5)
+              const uint32_t b1[2] = {__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632)};  // (k2,k6) (k3,k7)
+              const uint32_t ones[4] = {kOne2, kOne2, kOne2, kOne2};
+              const bool first = (j % SPAN) == 0;
+              if (first) {
+                mma16816_z(o, ones, b0[0], b0[1]);
+              } else {
+                mma16816(o, ones, b0[0], b0[1]);
+              }
+              mma16816(o, ones, b1[0], b1[1]);
+              const int q = (cw & 1) * 4 + j;
+              const uint8_t* cj = codes + ((q ^ g) << 4);
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                const bool pair = 2 * mt + 1 < NT;
+                const uint32_t xg = *reinterpret_cast<const uint32_t*>(cj + (2 * mt) * 8 * 128);
+                const uint32_t xh = pair ? *reinterpret_cast<const uint32_t*>(cj + (2 * mt + 1) * 8 * 128) : 0u;
+                // MMA 0: k-slots (2c, 2c+1) <- nibbles (0, 4), (2c+8, 2c+9) <- (1, 5); MMA 1: (2, 6), (3, 7)
+                uint32_t a0[4], a1[4];
+                a0[0] = nib_pair(xg);
+                a0[2] = nib_pair(shr(xg, 4));
+                a1[0] = nib_pair(shr(xg, 8));
+                a1[2] = nib_pair(shr(xg, 12));
+                if (pair) {
+                  a0[1] = nib_pair(xh);
+                  a0[3] = nib_pair(shr(xh, 4));
+                  a1[1] = nib_pair(shr(xh, 8));
+                  a1[3] = nib_pair(shr(xh, 12));
+                } else {
+                  a0[1] = a0[3] = a1[1] = a1[3] = 0u;
+                }
+                if (first) {
+                  mma16816_z(d[mt], a0, b0[0], b0[1]);
+                } else {
+                  mma16816(d[mt], a0, b0[0], b0[1]);
+                }
+                mma16816(d[mt], a1, b1[0], b1[1]);
+              }
+              if ((j % SPAN) == SPAN - 1) {
+                // group span done: acc += s D - s (128 + z) O for rows g, g + 8 of each tile
+                const int gl = ((ks * kDecStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                __syncwarp();
+#pragma unroll
+                for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
+                  const int row = lane + 32 * rr;
+                  if (row < 8 * NT) {
+                    const float sv = half_bits_to_float(sc[row * p.wg + gl]);
+                    const float zv = half_bits_to_float(zr[row * p.wg + gl]);
+                    smw[row] = make_float2(sv, -sv * (128.0f + zv));
+                  }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                  const float2 mg = smw[16 * mt + g];
+                  acc[mt][0] = fmaf(mg.x, d[mt][0], fmaf(mg.y, o[0], acc[mt][0]));
+                  acc[mt][1] = fmaf(mg.x, d[mt][1], fmaf(mg.y, o[1], acc[mt][1]));
+                  if (2 * mt + 1 < NT) {
+                    const float2 mh = smw[16 * mt + 8 + g];
+                    acc[mt][2] = fmaf(mh.x, d[mt][2], fmaf(mh.y, o[2], acc[mt][2]));
+                    acc[mt][3] = fmaf(mh.x, d[mt][3], fmaf(mh.y, o[3], acc[mt][3]));
+                  }
+                }
+              }
+            }
+          } else {
           float d[NT][4], o[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -316,6 +404,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               }
             }
           }
+          }
         }
         // every value read from this stage has been consumed above
         __syncwarp();
@@ -323,6 +412,18 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
       }
 
       // fixed-order reduction of the consumer warps' sums for this pass
+      if constexpr (!TBIG) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          float* rw = red + (warp * kDecPassRows + 16 * mt + g) * C::kTokPad + 2 * c;
+          if (2 * c < T) rw[0] = acc[mt][0];
+          if (2 * c + 1 < T) rw[1] = acc[mt][1];
+          if (2 * mt + 1 < NT) {
+            if (2 * c < T) rw[8 * C::kTokPad] = acc[mt][2];
+            if (2 * c + 1 < T) rw[8 * C::kTokPad + 1] = acc[mt][3];
+          }
+        }
+      } else
 #pragma unroll
       for (int jt = 0; jt < NT; ++jt) {
         {
@@ -503,9 +604,10 @@ cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, c
   p.tab_off = p.act_off + round_up(2 * 512 * T, 128);
   p.stage_bytes = round_up(p.tab_off + 2 * 2 * p.wg * kDecPassRows, 1024);
   const int fixed = red_bytes + static_cast<int>(sizeof(DecTail)) + 1024;
-  p.S = std::min(kDecMaxStages, (kDecSmemLimit - fixed) / p.stage_bytes);
+  // ring depth: a multiple of the consumer groups (each slot always taken by the same group)
   const int groups = tbig ? DecCfg<true>::kGroups : DecCfg<false>::kGroups;
-  if (p.S < groups + 1) return cudaErrorNotSupported;
+  p.S = std::min(kDecMaxStages, (kDecSmemLimit - fixed) / p.stage_bytes) / groups * groups;
+  if (p.S < 2 * groups) return cudaErrorNotSupported;
   const int smem = dec_tail_offset(p.S, p.stage_bytes, red_bytes) + static_cast<int>(sizeof(DecTail)) + 1024;
 
   CUtensorMap maps[7];

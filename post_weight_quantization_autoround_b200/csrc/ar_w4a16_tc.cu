@@ -69,6 +69,13 @@ constexpr int kEpWarps = 8;   // a multiple of 4: kEpWarps / 4 per TMEM lane qua
 constexpr int kEpQ = kEpWarps / 4;
 constexpr int kDqWarp0 = 3;
 
+// True when sets of warps that take a ring's stages in turn (set i takes stages
+// i, i + sets, ...), with `per_slot` consecutive stages sharing one slot of a
+// `slots`-slot ring, each wait on a slot's phases in order.
+__host__ __device__ constexpr bool slot_phases_in_order(int per_slot, int sets, int slots) {
+  return per_slot % sets == 0 || (sets % per_slot == 0 && slots % (sets / per_slot) == 0);
+}
+
 template <int TN>
 struct TcCfg {
   // One dequantization warp per TMEM lane quarter is latency bound (its nibble
@@ -95,6 +102,12 @@ struct TcCfg {
   static constexpr int kFinBytes = kTcRows * kRedStride * 4;
   static_assert(kActBytes % 1024 == 0, "stage parts must keep 1024-byte alignment");
   static_assert(kRedBytes + kFinBytes <= kRingBytes, "reduction buffers reuse the rings");
+  // Every waiter on a ring barrier must see the barrier's phases in order: a
+  // parity wait cannot tell a phase from the one two before it.  So when
+  // several warp sets take a ring's entries in turn, each entry is always
+  // taken by the same set (the set count divides the entry count).
+  static_assert(kStages % (kDqWarps / 4) == 0, "A stages: one dequantization set per stage");
+  static_assert(kNBuf % kGrpSplit == 0, "accumulators: one epilogue set per accumulator");
 };
 
 struct TcCtl {
@@ -473,6 +486,11 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     zrow.start(p.z16 + static_cast<size_t>(n < p.N ? n : 0) * p.G, g_begin, p.G, p.vec_meta != 0, n < p.N);
     const uint32_t sw = static_cast<uint32_t>(r & 7);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0;
+    // code slots: every dequantization set reads every phase of a slot (stages per slot a multiple
+    // of the sets), or each slot is always read by the same set (the sets a multiple of the stages
+    // per slot and their ratio dividing the slot count), so each set waits on a slot's phases in order
+    static_assert(slot_phases_in_order(CodeCfg<BITS>::kChunksPerSlot, Cfg::kDqWarps / 4, kCodeSlots),
+                  "code slots: phases waited in order by every dequantization set");
     for (int i = dw >> 2; i < c_end - c_begin; i += Cfg::kDqWarps / 4) {
       const int c = c_begin + i;
       const uint32_t stage = static_cast<uint32_t>(i % Cfg::kStages);
