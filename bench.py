@@ -347,7 +347,36 @@ def w4a16_bench(ar, torch, peaks, reps=20):
             out[f"W{bits}A16_T{T}"] = {"us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9, "algorithmic_bytes": nbytes,
                                       "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                       "TFLOP/s": 2.0 * T * N * K / (ms * 1e-3) / 1e12, "kernel": ar.ar_last_kernels()}
-    del W, V
+    # the same layer exported as NVFP4 (E2M1 codes, E4M3 scale per 16 values, per-tensor scale) through
+    # the tcgen05 dequant GEMM: 0.5 B per weight + 1 B per 16 weights
+    amax = torch.empty(1, dtype=torch.float32, device="cuda")
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((N, K // 16), dtype=torch.uint8, device="cuda")
+    ar.ar_absmax_bf16(W, amax)
+    ar.ar_qdq_nvfp4(W, None, None, amax, None, codes, scales, gs)
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    for T in (1, 16, 256):
+        A = to_dev_bf16(synth.make_activations(T, K, seed=T), torch)
+        y = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            ar.ar_nvfp4_gemm(A, codes, scales, gs, y)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in ev:
+            flush.sum()
+            e0.record()
+            ar.ar_nvfp4_gemm(A, codes, scales, gs, y)
+            e1.record()
+        torch.cuda.synchronize()
+        ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+        nbytes = codes.numel() + scales.numel() + A.numel() * 2 + y.numel() * 2
+        flops = 2.0 * T * N * K
+        out[f"NVFP4A16_T{T}"] = {"us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9, "algorithmic_bytes": nbytes,
+                                 "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                 "TFLOP/s": flops / (ms * 1e-3) / 1e12,
+                                 "frac_bf16_burst": flops / (ms * 1e-3) / 1e12 / peak_tf,
+                                 "kernel": ar.ar_last_kernels()}
+    del W, V, codes, scales
     return out
 
 

@@ -411,6 +411,29 @@ AR_API ar_status ar_qdq_nvfp4(const uint16_t* W, const float* V, const float* al
                               const float* amax, uint16_t* W_hat, uint8_t* codes, uint8_t* scales,
                               float* global_scale, ar_stream_t stream);
 
+/* Matmul with NVFP4 weights as ar_qdq_nvfp4 exports them, for bf16 activations:
+ *   out[t][n] = S * sum_k A[t][k] * E4M3(scales[n][k/16]) * E2M1(codes[n][k])
+ * the real-kernel side of the NVFP4 format ([QC] "量化：从 Scale 到 W4A8 的完整坐标"
+ * §2 table and §5 row "NVFP4 recipe"; [NQ] "量化", section "低比特浮点：FP8 与
+ * NVFP4": E2M1 values, an E4M3 scale per 16-value block, a per-tensor scale, on
+ * Blackwell).  Reading: the pages list the format for weights and activations;
+ * this call keeps the activations in bf16 (weight-only NVFP4, like W4A16), so that
+ * it consumes exactly what the tuning exports.  Each E2M1 value times its block
+ * scale is exact in bf16; the tensor cores (tcgen05) accumulate in fp32 and S
+ * scales the fp32 sums; out is rounded to bf16 (nearest even).
+ *   A       bf16 [T][K], 16-byte aligned
+ *   codes   uint8 [N][K/2]: two E2M1 codes per byte along K, element k in the
+ *           low nibble when k is even (ar_qdq_nvfp4's codes); 16-byte aligned
+ *   scales  uint8 [N][K/16]: E4M3 codes of the block scales (ar_qdq_nvfp4's
+ *           scales); 16-byte aligned
+ *   global_scale  device fp32 scalar S (ar_qdq_nvfp4's global_scale)
+ *   out     bf16 [T][N], 16-byte aligned
+ * Needs 1 <= T < 2^31, N >= 1, K % 128 == 0; otherwise AR_ERR_INVALID_ARG or
+ * AR_ERR_UNSUPPORTED before any launch.  All memory is the caller's. */
+AR_API ar_status ar_nvfp4_gemm(const uint16_t* A, int64_t T, const uint8_t* codes, const uint8_t* scales,
+                               const float* global_scale, int64_t N, int64_t K, uint16_t* out,
+                               ar_stream_t stream);
+
 /* Tuning steps of one linear layer on NVFP4: the SignSGD step of ar_tune_step
  * ([AR] §3 "Algorithm Flow" steps 3-5, "SignSGD") with ar_qdq_nvfp4 as its QDQ
  * function ([AR] §4 "Why the Tuning Stage Must Take the QDQ Path", point 3).

@@ -22,7 +22,8 @@ and fp64 matrix products.  Sources (page title, then section):
   mechanism: rounding is treated as the identity in the backward pass (STE).
 * [QC] §2 table (E2M1 and E4M3 layouts) and §5 table row "NVFP4 recipe";
   [NQ] "量化" (note.yj-dis.top), section "低比特浮点：FP8 与 NVFP4": the
-  NVFP4 QDQ function at the end of this module.
+  NVFP4 QDQ function and the NVFP4 weights' matmul (``nvfp4_matmul``) at the
+  end of this module.
 
 Readings where the pages are silent or disagree:
 
@@ -773,6 +774,30 @@ def pack_fp4(codes: np.ndarray) -> np.ndarray:
     """Two E2M1 codes per byte along K, element k in the low nibble when k is even: uint8 [N][K/2]."""
     c = np.asarray(codes).astype(np.uint8)
     return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_fp4(packed: np.ndarray) -> np.ndarray:
+    """Inverse of ``pack_fp4``: uint8 [N][K/2] -> codes uint8 [N][K]."""
+    b = np.asarray(packed).astype(np.uint8)
+    out = np.empty((b.shape[0], 2 * b.shape[1]), np.uint8)
+    out[:, 0::2] = b & 0x0F
+    out[:, 1::2] = b >> 4
+    return out
+
+
+def nvfp4_matmul(A, packed_codes, scale_codes, S) -> np.ndarray:
+    """The NVFP4 weights' matmul with bf16-valued activations, in fp64:
+    out[t][n] = S * sum_k A[t][k] * E4M3(scale_codes[n][k/16]) * E2M1(code[n][k])
+    ([QC] §2 table and §5 row "NVFP4 recipe"; [NQ] "量化", section "低比特浮点：FP8 与
+    NVFP4": E2M1 values, one E4M3 scale per 16-value block, a per-tensor scale).
+    A [T][K] (values), packed_codes uint8 [N][K/2] (``pack_fp4``), scale_codes uint8
+    [N][K/16], S the per-tensor scale.  Returns fp64 [T][N]."""
+    codes = unpack_fp4(packed_codes)
+    N, K = codes.shape
+    q = e2m1_values()[codes.astype(np.int64)]
+    sb = np.repeat(e4m3_values()[np.asarray(scale_codes).astype(np.int64)], NVFP4_BLOCK, axis=1).reshape(N, K)
+    W = f64(S) * sb * q
+    return np.asarray(A, f64) @ W.T
 
 
 # ----------------------------------------------------------------------------

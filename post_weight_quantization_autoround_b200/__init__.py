@@ -22,7 +22,7 @@ __all__ = [
     "ar_last_error", "ar_last_kernels", "ar_version", "ar_profile_start", "ar_profile_stop", "AR_BLOCK_LINEAR",
     "ar_tune_step_noalloc", "AR_NOALLOC_SCRATCH_BYTES", "AR_BLOCK_SWIGLU_MLP", "ar_block_forward",
     "ar_block_forward_workspace", "ar_tune_block", "ar_tune_block_workspace", "ar_debug_wait_timeout",
-    "ar_absmax_bf16", "ar_qdq_nvfp4", "ar_tune_step_nvfp4_workspace", "ar_tune_step_nvfp4",
+    "ar_absmax_bf16", "ar_qdq_nvfp4", "ar_nvfp4_gemm", "ar_tune_step_nvfp4_workspace", "ar_tune_step_nvfp4",
     "ar_tune_step_shard", "DecoderCfg", "DECODER_LAYERS", "ar_decoder_forward_workspace", "ar_decoder_forward",
     "ar_tune_step_decoder_workspace", "ar_tune_step_decoder", "ar_rmsnorm", "ar_attention_forward",
     "ar_attention_backward_workspace", "ar_attention_backward",
@@ -114,6 +114,7 @@ _SIGNATURES = {
     "ar_wxa16_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P]),
     "ar_absmax_bf16": (_INT, [_P, _I64, _P, _P]),
     "ar_qdq_nvfp4": (_INT, [_P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P]),
+    "ar_nvfp4_gemm": (_INT, [_P, _I64, _P, _P, _P, _I64, _I64, _P, _P]),
     "ar_tune_step_nvfp4_workspace": (ctypes.c_size_t, [_I64, _I64, _I64, _INT]),
     "ar_tune_step_nvfp4": (_INT, [_P, _P, _P, _I64, _I64, _P, _P, _I64, _P, ctypes.POINTER(QConfig), _INT, _P, _P, _P,
                                   _P, ctypes.c_size_t, _P]),
@@ -345,6 +346,15 @@ def ar_qdq_nvfp4(W, V, alpha, amax, W_hat=None, codes=None, scales=None, global_
     N, K = W.shape
     _check(lib().ar_qdq_nvfp4(_ptr(W), _ptr(V), _ptr(alpha), N, K, _ptr(amax), _ptr(W_hat), _ptr(codes),
                               _ptr(scales), _ptr(global_scale), _stream(stream)))
+
+
+def ar_nvfp4_gemm(A, codes, scales, global_scale, out, stream=None) -> None:
+    """out [T][N] bf16 = A [T][K] bf16 times the NVFP4 weights: codes uint8 [N][K/2], scales uint8
+    [N][K/16] (E4M3 codes), global_scale fp32 device scalar (as ``ar_qdq_nvfp4`` writes them)."""
+    T, K = A.shape
+    N = codes.shape[0]
+    _check(lib().ar_nvfp4_gemm(_ptr(A), T, _ptr(codes), _ptr(scales), _ptr(global_scale), N, K, _ptr(out),
+                               _stream(stream)))
 
 
 def ar_tune_step_nvfp4_workspace(M: int, N: int, K: int, n_steps: int) -> int:

@@ -894,6 +894,24 @@ ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
   return end_call();
 }
 
+ar_status ar_nvfp4_gemm(const uint16_t* A, int64_t T, const uint8_t* codes, const uint8_t* scales,
+                        const float* global_scale, int64_t N, int64_t K, uint16_t* out, ar_stream_t stream) {
+  begin_call();
+  if (T < 1 || N <= 0 || K <= 0) return fail(AR_ERR_INVALID_ARG, "T, N, K must be positive");
+  if (K % 128 != 0) return fail(AR_ERR_INVALID_ARG, "K must be a multiple of 128");
+  if (N > INT32_MAX || K > INT32_MAX || T > INT32_MAX) return fail(AR_ERR_UNSUPPORTED, "dimension exceeds 2^31-1");
+  const void* ptrs[] = {A, codes, scales, out};
+  for (const void* p : ptrs) {
+    if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  if (!global_scale) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
+  cudaError_t e = launch_nvfp4_tc(A, static_cast<int>(T), codes, scales, global_scale, static_cast<int>(N),
+                                  static_cast<int>(K), out, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm launch");
+  return end_call();
+}
+
 ar_status ar_gather_samples(const void* src, int64_t n_src_samples, int64_t sample_bytes, const int32_t* idx,
                             int n_idx, void* dst, ar_stream_t stream) {
   begin_call();

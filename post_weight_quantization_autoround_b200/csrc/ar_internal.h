@@ -173,6 +173,10 @@ cudaError_t launch_w4a16_tc(const uint16_t* A, int T, const uint32_t* packed, co
 cudaError_t launch_wbx_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                            const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,
                            cudaStream_t stream);
+// NVFP4 weights (E2M1 codes uint8 [N][K/2], E4M3 block scales uint8 [N][K/16],
+// device per-tensor scale), any T: the same tcgen05 GEMM (ar_w4a16_tc.cu)
+cudaError_t launch_nvfp4_tc(const uint16_t* A, int T, const uint8_t* codes, const uint8_t* scales, const float* gscale,
+                            int N, int K, uint16_t* out, cudaStream_t stream);
 // 2, 4 or 8-bit codes (32/bits per uint32), any T: the same tcgen05 GEMM
 cudaError_t launch_wxa16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                             const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,

@@ -40,6 +40,8 @@
 // bits 4*(k mod 8) of word k/8; scale/zero fp16 [N][K/g].
 #include <cooperative_groups.h>
 
+#include <cuda_fp8.h>
+
 #include "ar_internal.h"
 
 namespace cg = cooperative_groups;
@@ -126,6 +128,8 @@ struct TcCtl {
 struct TcParams {
   const uint16_t* s16;  // fp16 bits [N][G]
   const uint16_t* z16;
+  const uint8_t* sc8;   // NVFP4: E4M3 block-scale codes [N][K/16]
+  const float* gscale;  // NVFP4: device per-tensor scale S
   uint16_t* out;        // bf16 bits [T][N]
   int N, K, T, G;
   int group_shift;
@@ -221,6 +225,55 @@ __device__ __forceinline__ void dequant4b(uint32_t x, float zf, uint32_t* o) {
   o[1] = pack_bf16x2(f[2], f[3]);
 }
 
+// 8 E2M1 codes of one word (element k in bits 4k..4k+3; code = sign << 3 |
+// magnitude index) -> 8 bf16 values in k order, each times the bf16 pair sc2 (the
+// block scale in both halves).  The magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 are
+// bf16 0x0000, 0x3F00, 0x3F80, 0x3FC0, 0x4000, 0x4040, 0x4080, 0x40C0: byte
+// tables of their low and high bytes, indexed by the 3-bit magnitude index
+// through byte permutes, give four values per permute; the sign bit of each
+// code moves to bit 15 or 31 of its pair.  An E2M1 value times an E4M3 scale
+// has at most 6 significant bits and stays in bf16's normal range, so every
+// product is exact.
+__device__ __forceinline__ uint4 dequant_e2m1x8(uint32_t x, uint32_t sc2) {
+  constexpr uint32_t kL0 = 0xC0800000u, kL1 = 0xC0804000u;  // low bytes for magnitudes 0..3, 4..7
+  constexpr uint32_t kH0 = 0x3F3F3F00u, kH1 = 0x40404040u;  // high bytes
+  const uint32_t y = x & 0x77777777u;                       // magnitude indices (selector bit 3 cleared)
+  const uint32_t y2 = y >> 16;
+  const uint32_t l03 = __byte_perm(kL0, kL1, y), h03 = __byte_perm(kH0, kH1, y);
+  const uint32_t l47 = __byte_perm(kL0, kL1, y2), h47 = __byte_perm(kH0, kH1, y2);
+  // sign of code 2j: bit 7 of byte j of sx4; of code 2j + 1: bit 7 of byte j of sx
+  const uint32_t sx = x & 0x88888888u;
+  const uint32_t sx4 = (x << 4) & 0x88888888u;
+  uint32_t m[4];
+  m[0] = __byte_perm(l03, h03, 0x5140) | (__byte_perm(sx4, sx, 0x4000) & 0x80008000u);  // (k0, k1)
+  m[1] = __byte_perm(l03, h03, 0x7362) | (__byte_perm(sx4, sx, 0x5111) & 0x80008000u);  // (k2, k3)
+  m[2] = __byte_perm(l47, h47, 0x5140) | (__byte_perm(sx4, sx, 0x6222) & 0x80008000u);  // (k4, k5)
+  m[3] = __byte_perm(l47, h47, 0x7362) | (__byte_perm(sx4, sx, 0x7333) & 0x80008000u);  // (k6, k7)
+  uint4 o;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o.x) : "r"(m[0]), "r"(sc2));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o.y) : "r"(m[1]), "r"(sc2));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o.z) : "r"(m[2]), "r"(sc2));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o.w) : "r"(m[3]), "r"(sc2));
+  return o;
+}
+
+// The 8 E4M3 block-scale codes of one row's 128-k stage -> 8 bf16 pairs (each
+// scale in both halves); E4M3 values are exact in bf16.
+__device__ __forceinline__ void e4m3x8_to_bf16_pairs(uint2 c, uint32_t (&sc2)[8]) {
+  const uint32_t w[2] = {c.x, c.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[h] >> (16 * i)), __NV_E4M3);
+      const float f0 = __half2float(__half(__half_raw{hr.x}));
+      const float f1 = __half2float(__half(__half_raw{hr.y}));
+      sc2[4 * h + 2 * i] = pack_bf16x2(f0, f0);
+      sc2[4 * h + 2 * i + 1] = pack_bf16x2(f1, f1);
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t zero_pair(uint16_t z16) {
   const uint32_t z = static_cast<uint32_t>(__half2float(__ushort_as_half(z16)));
   return (0x4300u + z) * 0x00010001u;
@@ -286,7 +339,10 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // Grid: one CTA per (128-row tile, token tile, K half when split); the CTAs of
 // a weight tile are adjacent so that its codes come from HBM once.
-template <int TN, int KSPLIT, int BITS>
+// FP4: NVFP4 weights (E2M1 codes in the 4-bit layout, E4M3 block scales folded
+// into the dequantized operand, the per-tensor scale applied per group in the
+// epilogue); BITS is then 4.
+template <int TN, int KSPLIT, int BITS, bool FP4>
 __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const TcParams p) {
@@ -483,7 +539,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     const int r = (warp & 3) * 32 + lane;  // weight row within the tile = TMEM lane
     const int n = n0 + r;
     MetaRow zrow;
-    zrow.start(p.z16 + static_cast<size_t>(n < p.N ? n : 0) * p.G, g_begin, p.G, p.vec_meta != 0, n < p.N);
+    if (!FP4) zrow.start(p.z16 + static_cast<size_t>(n < p.N ? n : 0) * p.G, g_begin, p.G, p.vec_meta != 0, n < p.N);
     const uint32_t sw = static_cast<uint32_t>(r & 7);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0;
     // code slots: every dequantization set reads every phase of a slot (stages per slot a multiple
@@ -514,13 +570,23 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
       uint4 pw[kPre];
 #pragma unroll
       for (int v = 0; v < kPre; ++v) pw[v] = ld_shared_v4(pk + (((qv + v) ^ sw) << 4));
+      // NVFP4: the row's 8 block scales of this stage (one per two words)
+      uint32_t sc2[8];
+      if (FP4) {
+        uint2 c8 = make_uint2(0u, 0u);
+        if (n < p.N) c8 = __ldg(reinterpret_cast<const uint2*>(p.sc8 + static_cast<size_t>(n) * (p.K / 16) + k0 / 16));
+        e4m3x8_to_bf16_pairs(c8, sc2);
+      }
       // zero-points of the four 32-k quarters (equal when g >= 128), converted once:
       // (128 + z) bf16 pairs for 2 and 4 bits, 2^23 + z in fp32 for 8 bits
       uint32_t zz[4];
       float zf[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        if (h == 0 || p.group_shift < 7) {
+        if (FP4) {
+          zz[h] = 0u;
+          zf[h] = 0.f;
+        } else if (h == 0 || p.group_shift < 7) {
           const uint16_t z = zrow.get((k0 + 32 * h) >> p.group_shift);
           if (BITS == 8) zf[h] = 8388608.0f + __half2float(__ushort_as_half(z));
           else zz[h] = zero_pair(z);
@@ -546,7 +612,13 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
             const int w = half * 2 * BITS + 4 * v + u;  // word of the stage; it covers k 32w/BITS ..
             const int quarter = w / BITS;
             const int col = (w - half * 2 * BITS) * (16 / BITS);  // first column of this word in the half
-            if (BITS == 4) {
+            if (FP4) {
+              const uint4 o = dequant_e2m1x8(xs[u], sc2[w >> 1]);  // word w holds k 8w .. 8w + 7: block w / 2
+              a[col] = o.x;
+              a[col + 1] = o.y;
+              a[col + 2] = o.z;
+              a[col + 3] = o.w;
+            } else if (BITS == 4) {
               const uint4 o = dequant8(xs[u], zz[quarter]);
               a[col] = o.x;
               a[col + 1] = o.y;
@@ -579,14 +651,15 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     const int gfirst = egrp;
     constexpr int gstep = Cfg::kGrpSplit;
     MetaRow srow;
-    srow.start(p.s16 + static_cast<size_t>(n < p.N ? n : 0) * p.G, g_begin + gfirst, p.G, p.vec_meta != 0, n < p.N);
+    if (!FP4) srow.start(p.s16 + static_cast<size_t>(n < p.N ? n : 0) * p.G, g_begin + gfirst, p.G, p.vec_meta != 0, n < p.N);
+    const float S = FP4 ? __ldg(p.gscale) : 0.f;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
     for (int li = gfirst; li < n_groups; li += gstep) {
       const uint32_t buf = static_cast<uint32_t>(li % Cfg::kNBuf);
       const uint32_t par = static_cast<uint32_t>((li / Cfg::kNBuf) & 1);
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_sleep(&ctl->tmem_full[buf], par, abort_flag))) break;
       tc_fence_after();
-      const float s = __half2float(__ushort_as_half(srow.get(g_begin + li)));
+      const float s = FP4 ? S : __half2float(__ushort_as_half(srow.get(g_begin + li)));
 #pragma unroll
       for (int c = 0; c < Cfg::kCols; c += 16) {
         float v[16];
@@ -645,7 +718,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
   }
 }
 
-template <int TN, int KSPLIT, int BITS>
+template <int TN, int KSPLIT, int BITS, bool FP4>
 cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int n_tiles, cudaStream_t stream,
                       const char* name) {
   using Cfg = TcCfg<TN>;
@@ -655,7 +728,7 @@ cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int
   if (e != cudaSuccess) return e;
   constexpr int smem = Cfg::kRingBytes + static_cast<int>(sizeof(TcCtl)) + 1024;
   static_assert(smem <= 227 * 1024, "shared memory per CTA");
-  auto kern = w4a16_tc_kernel<TN, KSPLIT, BITS>;
+  auto kern = w4a16_tc_kernel<TN, KSPLIT, BITS, FP4>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -676,7 +749,7 @@ cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int
   return cudaGetLastError();
 }
 
-template <int TN, int BITS>
+template <int TN, int BITS, bool FP4 = false>
 cudaError_t launch_tn(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int n_tiles, cudaStream_t stream,
                       const char* name1, const char* name2) {
   // Split K over a CTA pair when one CTA per tile leaves more than half the SMs idle.
@@ -686,11 +759,11 @@ cudaError_t launch_tn(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int
     p.split_units = (total_units + 1) / 2;
     const int g_split = (p.split_units * p.unit_k) >> p.group_shift;
     p.vec_meta = (p.G % 8 == 0 && g_split % 8 == 0) ? 1 : 0;
-    return launch_tc<TN, 2, BITS>(A, tmW, p, n_tiles, stream, name2);
+    return launch_tc<TN, 2, BITS, FP4>(A, tmW, p, n_tiles, stream, name2);
   }
   p.split_units = total_units;
   p.vec_meta = p.G % 8 == 0 ? 1 : 0;
-  return launch_tc<TN, 1, BITS>(A, tmW, p, n_tiles, stream, name1);
+  return launch_tc<TN, 1, BITS, FP4>(A, tmW, p, n_tiles, stream, name1);
 }
 
 
@@ -718,6 +791,12 @@ struct TcNames<8> {
                                        "wxa16_tc_kernel<b=8,TN=64>", "wxa16_tc_kernel<b=8,TN=64,split2>",
                                        "wxa16_tc_kernel<b=8,TN=128>", "wxa16_tc_kernel<b=8,TN=128,split2>"};
 };
+
+// NVFP4 names (TN = 16, 32, 64, 128, each unsplit and split over a CTA pair)
+constexpr const char* kFp4Names[8] = {"nvfp4_tc_kernel<TN=16>", "nvfp4_tc_kernel<TN=16,split2>",
+                                      "nvfp4_tc_kernel<TN=32>", "nvfp4_tc_kernel<TN=32,split2>",
+                                      "nvfp4_tc_kernel<TN=64>", "nvfp4_tc_kernel<TN=64,split2>",
+                                      "nvfp4_tc_kernel<TN=128>", "nvfp4_tc_kernel<TN=128,split2>"};
 
 template <int BITS>
 cudaError_t launch_bits_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
@@ -758,6 +837,43 @@ cudaError_t launch_bits_tc(const uint16_t* A, int T, const uint32_t* packed, con
 cudaError_t launch_w4a16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out, cudaStream_t stream) {
   return launch_bits_tc<4>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+}
+
+cudaError_t launch_nvfp4_tc(const uint16_t* A, int T, const uint8_t* codes, const uint8_t* scales, const float* gscale,
+                            int N, int K, uint16_t* out, cudaStream_t stream) {
+  if (T < 1 || N < 1 || K < kTcK || K % kTcK != 0) return cudaErrorInvalidValue;
+  TcParams p{};
+  p.sc8 = scales;
+  p.gscale = gscale;
+  p.out = out;
+  p.N = N;
+  p.K = K;
+  p.T = T;
+  // accumulation groups: the largest power of two up to 1024 that divides K (the per-tensor
+  // scale is the same for all of them, so fewer groups mean fewer epilogue passes)
+  p.group_shift = 7;
+  while (p.group_shift < 10 && K % (1 << (p.group_shift + 1)) == 0) ++p.group_shift;
+  p.G = K >> p.group_shift;
+  p.unit_k = 1 << p.group_shift;
+  CUtensorMap tmW;
+  cudaError_t e = make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, codes, static_cast<uint64_t>(N),
+                               static_cast<uint64_t>(K) / 8, 32, kTcRows, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  const int n_tiles = (N + kTcRows - 1) / kTcRows;
+  if (T <= 16) {
+    p.t_tiles = 1;
+    return launch_tn<16, 4, true>(A, tmW, p, n_tiles, stream, kFp4Names[0], kFp4Names[1]);
+  }
+  if (T <= 32) {
+    p.t_tiles = 1;
+    return launch_tn<32, 4, true>(A, tmW, p, n_tiles, stream, kFp4Names[2], kFp4Names[3]);
+  }
+  if (T <= 64) {
+    p.t_tiles = 1;
+    return launch_tn<64, 4, true>(A, tmW, p, n_tiles, stream, kFp4Names[4], kFp4Names[5]);
+  }
+  p.t_tiles = (T + 127) / 128;
+  return launch_tn<128, 4, true>(A, tmW, p, n_tiles, stream, kFp4Names[6], kFp4Names[7]);
 }
 
 cudaError_t launch_wxa16_tc(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,

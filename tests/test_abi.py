@@ -181,6 +181,16 @@ def test_absmax_and_qdq_nvfp4_validation():
     assert q(FAKE, None, None, 4, 64, FAKE, None, FAKE + 8, None, None, None) == ar.AR_ERR_INVALID_ARG  # codes
 
 
+def test_nvfp4_gemm_validation():
+    g = ar.lib().ar_nvfp4_gemm
+    assert g(FAKE, 1, FAKE, FAKE, FAKE, 64, 192, FAKE, None) == ar.AR_ERR_INVALID_ARG       # K % 128
+    assert g(FAKE, 0, FAKE, FAKE, FAKE, 64, 256, FAKE, None) == ar.AR_ERR_INVALID_ARG       # T
+    assert g(FAKE, 1, FAKE, FAKE, FAKE, 0, 256, FAKE, None) == ar.AR_ERR_INVALID_ARG        # N
+    assert g(FAKE, 1, FAKE, FAKE + 8, FAKE, 64, 256, FAKE, None) == ar.AR_ERR_INVALID_ARG   # scales misaligned
+    assert g(FAKE, 1, FAKE, FAKE, None, 64, 256, FAKE, None) == ar.AR_ERR_INVALID_ARG       # no global scale
+    assert g(FAKE, 1, None, FAKE, FAKE, 64, 256, FAKE, None) == ar.AR_ERR_INVALID_ARG       # no codes
+
+
 def test_tune_step_nvfp4_validation():
     cfg = ar.ar_qconfig_default()
     f = ar.lib().ar_tune_step_nvfp4

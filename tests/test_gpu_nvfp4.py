@@ -1,6 +1,9 @@
 """NVFP4 QDQ on the GPU against the oracle: codes, E4M3 block scales, the per-tensor scale and Ŵ,
 all bit-exact (both sides take every step in fp32 in the same order, and the roundings to E4M3 and
-E2M1 are round-to-nearest-even with saturation on both)."""
+E2M1 are round-to-nearest-even with saturation on both).  The NVFP4 weights' matmul against the
+oracle's fp64 matmul on the same codes, scales and S: every E2M1 value times its E4M3 block scale is
+exact in bf16 and every product in the tensor cores is exact, so only the fp32 accumulation and the
+bf16 rounding of the output (2^-9 relative) remain; bar 3e-3 relative L2."""
 import numpy as np
 import pytest
 import torch
@@ -178,3 +181,81 @@ def test_tune_step_nvfp4_steps_in_one_call_equal_single_calls_and_lower_the_loss
     assert np.array_equal(la.cpu().numpy(), np.array(lb, np.float32))
     assert torch.equal(Va, Vb) and torch.equal(aa, ab)
     assert lb[-1] < lb[0]
+
+
+NVFP4_GEMM_RTOL = 3e-3
+
+
+def _rel_l2(x, y):
+    x = np.asarray(x, np.float64)
+    y = np.asarray(y, np.float64)
+    return float(np.linalg.norm(x - y) / max(np.linalg.norm(y), 1e-300))
+
+
+def _nvfp4_weights(ar, Wb, V, a):
+    """The GPU QDQ's exports (device tensors) of bf16 bits Wb."""
+    N, K = Wb.shape
+    dev = "cuda"
+    W = torch.from_numpy(Wb.view(np.int16)).to(dev).view(torch.bfloat16)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // 16), dtype=torch.uint8, device=dev)
+    gs = torch.empty(1, dtype=torch.float32, device=dev)
+    ar.ar_absmax_bf16(W, amax)
+    ar.ar_qdq_nvfp4(W, None if V is None else torch.from_numpy(V).to(dev),
+                    None if a is None else torch.from_numpy(a).to(dev), amax, None, codes, scales, gs)
+    return codes, scales, gs
+
+
+def _gemm(ar, A_bits, codes, scales, gs):
+    T = A_bits.shape[0]
+    N = codes.shape[0]
+    A = torch.from_numpy(A_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_nvfp4_gemm(A, codes, scales, gs, out)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("N,K,T", [(136, 256, 1), (200, 768, 5), (1000, 1024, 16), (320, 2048, 40),
+                                   (256, 384, 64), (130, 640, 129), (40, 4096, 3)])
+def test_nvfp4_gemm_matches_oracle(ar, N, K, T):
+    """Ragged N (not a multiple of 128 rows), K with 1-8 accumulation groups, every token-tile width
+    (16, 32, 64, 128 tokens, two 128-token tiles at T = 129) and the CTA pair splitting K (small N)."""
+    Wb, V, a = _inputs(N, K, seed=3 * N + K)
+    codes, scales, gs = _nvfp4_weights(ar, Wb, V, a)
+    A_bits = synth.make_activations(T, K, seed=T + 7)
+    got = _gemm(ar, A_bits, codes, scales, gs)
+    assert "nvfp4_tc_kernel" in ar.ar_last_kernels()
+    ref = O.nvfp4_matmul(synth.bf16_bits_to_f32(A_bits), codes.cpu().numpy(), scales.cpu().numpy(), gs.item())
+    assert _rel_l2(got, ref) <= NVFP4_GEMM_RTOL
+    for t in range(T):
+        assert _rel_l2(got[t], ref[t]) <= NVFP4_GEMM_RTOL
+    # the same against the oracle's own QDQ of the weights (the GPU QDQ is bit-exact, so its codes are these)
+    st = O.nvfp4_qdq(synth.bf16_bits_to_f32(Wb), V, a)
+    ref2 = O.nvfp4_matmul(synth.bf16_bits_to_f32(A_bits), O.pack_fp4(st["codes"]), st["scale_codes"], st["S"])
+    assert _rel_l2(got, ref2) <= NVFP4_GEMM_RTOL
+
+
+def test_nvfp4_gemm_zero_weights(ar):
+    """An all-zero matrix: S = 0, every code and scale 0, the product exactly 0."""
+    N, K, T = 64, 256, 4
+    Wb = np.zeros((N, K), np.uint16)
+    codes, scales, gs = _nvfp4_weights(ar, Wb, None, None)
+    got = _gemm(ar, synth.make_activations(T, K, seed=1), codes, scales, gs)
+    assert np.all(got == 0.0)
+
+
+@pytest.mark.parametrize("T", [1, 16, 256])
+def test_nvfp4_gemm_full_size_sampled_rows(ar, T):
+    """The 8192 x 28672 layer, checked on 64 sampled output rows (the rows of a linear layer are
+    independent): the oracle recomputes them from the GPU's codes, scales and S of those rows."""
+    N, K = 8192, 28672
+    d = synth.make_linear(N, K, 1, seed=5, x_outlier_channels=0)
+    codes, scales, gs = _nvfp4_weights(ar, d["W"], None, None)
+    A_bits = synth.make_activations(T, K, seed=11)
+    got = _gemm(ar, A_bits, codes, scales, gs)
+    rows = np.sort(np.random.default_rng(2).choice(N, 64, replace=False))
+    ref = O.nvfp4_matmul(synth.bf16_bits_to_f32(A_bits), codes.cpu().numpy()[rows], scales.cpu().numpy()[rows],
+                         gs.item())
+    assert _rel_l2(got[:, rows], ref) <= NVFP4_GEMM_RTOL

@@ -786,6 +786,37 @@ def test_pack_fp4_places_each_code_by_hand():
     assert O.pack_fp4(codes).tolist() == [[0x21, 0x43, 0x0F, 0x78]]
 
 
+def test_unpack_fp4_inverts_pack_fp4():
+    codes = np.random.default_rng(3).integers(0, 16, size=(5, 48)).astype(np.uint8)
+    assert np.array_equal(O.unpack_fp4(O.pack_fp4(codes)), codes)
+
+
+def test_nvfp4_matmul_by_hand():
+    """One row, one block: codes 7 (6.0), 9 (-0.5), 3 (1.5), 0 and the rest 0; block scale code
+    0x40 (E4M3 2.0); S = 0.25; A = 1, 2, 3 on the first three k."""
+    codes = np.zeros((1, 16), np.uint8)
+    codes[0, :3] = [7, 9, 3]
+    A = np.zeros((1, 16))
+    A[0, :3] = [1.0, 2.0, 3.0]
+    out = O.nvfp4_matmul(A, O.pack_fp4(codes), np.array([[0x40]], np.uint8), 0.25)
+    assert out.shape == (1, 1)
+    assert out[0, 0] == 0.25 * 2.0 * (1.0 * 6.0 + 2.0 * -0.5 + 3.0 * 1.5)
+
+
+def test_nvfp4_matmul_reproduces_the_qdq_weights():
+    """The matmul of the QDQ's own codes, scale codes and S equals A @ Ŵᵀ of the same QDQ up to
+    the fp32 rounding of the QDQ's block scale s_b = E4M3(...) * S and of Ŵ = q * s_b (a
+    dropped block scale, a wrong nibble order or a missing S would be off by far more)."""
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((24, 64)) * np.exp(rng.standard_normal((24, 1)))).astype(np.float32)
+    V = rng.uniform(-0.5, 0.5, W.shape).astype(np.float32)
+    st = O.nvfp4_qdq(W, V)
+    A = rng.standard_normal((3, 64))
+    got = O.nvfp4_matmul(A, O.pack_fp4(st["codes"]), st["scale_codes"], st["S"])
+    ref = A @ st["What"].astype(np.float64).T
+    assert np.max(np.abs(got - ref)) <= 1e-6 * np.max(np.abs(A) @ np.abs(st["What"].astype(np.float64)).T)
+
+
 def _nvfp4_smooth_loss(W, X, Y, V, a):
     st = O.nvfp4_qdq_smooth(W, V, a)
     return O.forward_loss(X, st["What"], Y, X.shape[0] * W.shape[0], dtype=np.float64)
