@@ -713,6 +713,34 @@ def run_case(name, ar, torch):
         fn = lambda: ar.ar_tune_block(ar.AR_BLOCK_SWIGLU_MLP, layers, X, Y, cfg, 1, loss, ws)
     elif name == "decoder":  # one joint step of a Llama-7B-shaped decoder block on one 2048-token sample
         fn = decoder_step_fn(ar, torch, 1, 2048, 1)[0]
+    elif name in ("w4a16_t1", "nvfp4_gemm_t1", "nvfp4_gemm_t256"):  # the 8192 x 28672 layer's exports
+        N, K, g = 8192, 28672, 128
+        d = synth.make_linear(N, K, 1, seed=5, x_outlier_channels=0)
+        W = to_dev_bf16(d["W"], torch)
+        del d
+        T = 256 if name.endswith("t256") else 1
+        A = to_dev_bf16(synth.make_activations(T, K, seed=T), torch)
+        y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+        if name == "w4a16_t1":
+            V = torch.zeros((N, K), device=dev)
+            a = torch.ones((N, K // g), device=dev)
+            pk = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+            s16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+            z16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+            ar.ar_pack_int4(W, V, a, a, ar.ar_qconfig_default(bits=4, group_size=g), pk, s16, z16)
+            del V, a
+            fn = lambda: ar.ar_w4a16_gemm(A, pk, s16, z16, g, y)
+        else:
+            amax = torch.empty(1, device=dev)
+            gs = torch.empty(1, device=dev)
+            codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+            scales = torch.empty((N, K // 16), dtype=torch.uint8, device=dev)
+            ar.ar_absmax_bf16(W, amax)
+            ar.ar_qdq_nvfp4(W, None, None, amax, None, codes, scales, gs)
+            fn = lambda: ar.ar_nvfp4_gemm(A, codes, scales, gs, y)
+        del W
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()  # only the exports, activations and output stay on the device
     else:
         raise SystemExit(f"unknown case {name}; one of {', '.join(CASES)}")
     for _ in range(3):
@@ -723,7 +751,8 @@ def run_case(name, ar, torch):
     return 0 if st == 0 else 1
 
 
-CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp", "decoder")
+CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp", "decoder", "w4a16_t1", "nvfp4_gemm_t1",
+         "nvfp4_gemm_t256")
 
 
 def main():
