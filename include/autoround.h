@@ -176,6 +176,12 @@ AR_API size_t ar_tune_step_workspace(int block_kind, const ar_layer* layers, int
  *   dB = bf16(dH silu(a)); dWg = dA^T X, dWu = dB^T X; each folded and
  *   updated as above.  X [M][H] bf16, Y [M][H] fp32 from ar_block_forward.
  * workspace: device buffer of at least ar_tune_step_workspace() bytes.
+ * Where the fold runs (the same values either way, up to the order of a
+ * group's sums): from 8192 tokens the weight-gradient GEMM folds and updates
+ * in its epilogue (dW_hat never leaves the SM); an AR_BLOCK_LINEAR step with
+ * fewer tokens and group_size <= 128 writes dW_hat (fp32 [N][K]) to the
+ * workspace and a separate kernel folds, updates and takes the next step's QDQ,
+ * so that only the first step runs the QDQ kernel.
  * Supported: AR_BLOCK_LINEAR with n_layers = 1 and AR_BLOCK_SWIGLU_MLP with
  * n_layers = 3; bits 2..8; group_size 32, 64, 128, 256 dividing every K;
  * N % 8 == 0 (H, F % 8 == 0 for the MLP).

@@ -63,8 +63,9 @@ ar_status check_cfg(const ar_qconfig* cfg) {
 
 // Layout of the tuning workspace for one linear layer.
 struct LinearWs {
-  size_t what, g, s, zp, mx, mn, partial, total;
+  size_t what, g, s, zp, mx, mn, dw, partial, total;
   int partials_per_step;
+  bool split_fold;  // dL/dW_hat materialised in dw and folded by the standalone kernel
 };
 
 LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int g, int n_steps) {
@@ -83,6 +84,9 @@ LinearWs linear_ws(int64_t M, int64_t N, int64_t K, int g, int n_steps) {
   off = align_up(off + static_cast<size_t>(groups) * 4, 256);
   w.mn = off;
   off = align_up(off + static_cast<size_t>(groups) * 4, 256);
+  w.split_fold = use_split_fold(M, g);
+  w.dw = off;
+  if (w.split_fold) off = align_up(off + static_cast<size_t>(N * K) * 4, 256);
   w.partials_per_step = resid_partials(static_cast<int>(M), static_cast<int>(N));
   w.partial = off;
   off = align_up(off + static_cast<size_t>(w.partials_per_step) * (n_steps > 0 ? n_steps : 1) * 8, 256);
@@ -296,17 +300,29 @@ ar_status tune_linear(const ar_layer* layers, int n_layers, const uint16_t* X, i
   const int steps = n_steps > 0 ? n_steps : 1;
   cudaError_t e;
   for (int step = 0; step < steps; ++step) {
-    e = launch_qdq(L.W, L.V, L.alpha, L.beta, L.N, L.K, cfg->group_size, cfg->bits, cfg->symmetric, W_hat, nullptr,
-                   sc, zp, mx, mn, s);
-    if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+    // on the split-fold path the previous step's fold kernel already took this step's QDQ
+    if (step == 0 || !w.split_fold) {
+      e = launch_qdq(L.W, L.V, L.alpha, L.beta, L.N, L.K, cfg->group_size, cfg->bits, cfg->symmetric, W_hat, nullptr,
+                     sc, zp, mx, mn, s);
+      if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+    }
     e = launch_gemm_resid(X, W_hat, Y, G, gscale, partial + static_cast<size_t>(step) * w.partials_per_step, Mi, Ni,
                           Ki, s);
     if (e != cudaSuccess) return cuda_fail(e, "forward GEMM launch");
     if (n_steps == 0) break;
     const bool last = step == steps - 1;
     const FoldArgs fa = fold_args(L, cfg, sc, zp, mx, mn, (last && grads) ? grads : nullptr);
-    e = launch_gemm_fold(G, X, fa, Mi, Ni, Ki, s);
-    if (e != cudaSuccess) return cuda_fail(e, "weight-gradient GEMM launch");
+    if (w.split_fold) {
+      // short token reduction: dL/dW_hat = G^T X to the workspace, then the fold at full occupancy
+      float* dW = reinterpret_cast<float*>(ws + w.dw);
+      e = launch_gemm_plain(G, true, X, true, dW, Ni, Ki, Mi, s);
+      if (e != cudaSuccess) return cuda_fail(e, "weight-gradient GEMM launch");
+      e = launch_fold_int(dW, fa, L.N, L.K, last ? nullptr : W_hat, s);
+      if (e != cudaSuccess) return cuda_fail(e, "fold launch");
+    } else {
+      e = launch_gemm_fold(G, X, fa, Mi, Ni, Ki, s);
+      if (e != cudaSuccess) return cuda_fail(e, "weight-gradient GEMM launch");
+    }
   }
   e = launch_loss_reduce(partial, w.partials_per_step, steps, 1.0 / count, loss_per_step, s);
   if (e != cudaSuccess) return cuda_fail(e, "loss reduction launch");

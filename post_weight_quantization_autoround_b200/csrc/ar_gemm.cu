@@ -52,6 +52,7 @@
 // their loops, in-flight TMA copies and MMAs are drained, TMEM is freed.
 #include <algorithm>
 
+#include "ar_fold.cuh"
 #include "ar_internal.h"
 
 namespace ar {
@@ -218,13 +219,6 @@ __device__ __forceinline__ double epi_resid(const Params& p, uint32_t taddr, int
   return acc;
 }
 
-// p - lr*sign(d), clamped; sign(0) = sign(NaN) = 0.  p - (-lr) is the same
-// IEEE result as p + lr.
-__device__ __forceinline__ float sign_step(float p, float d, float lr, float lo, float hi) {
-  const float step = d > 0.0f ? lr : (d < 0.0f ? -lr : 0.0f);
-  return fminf(fmaxf(__fsub_rn(p, step), lo), hi);
-}
-
 // Straight-through fold + SignSGD.  GEMM rows are weight rows n (M = N_w),
 // GEMM columns are weight columns k (N = K_w).  Each epilogue warp owns 32
 // rows and half of the tile's 256 columns (chunks c0..c0+3 of 32).  Groups of
@@ -245,61 +239,6 @@ __device__ __forceinline__ void fold_load(const FoldArgs& f, size_t e, FoldChunk
   for (int i = 0; i < 4; ++i) ch.w[i] = *reinterpret_cast<const uint4*>(f.W + e + 8 * i);
 #pragma unroll
   for (int i = 0; i < 8; ++i) ch.v[i] = *reinterpret_cast<const float4*>(f.V + e + 4 * i);
-}
-
-struct GroupParams {
-  float s, zp, lo_s, mx, mn, al, be;
-  bool guarded, take_hi;
-  size_t gidx;
-};
-
-__device__ __forceinline__ void group_load(const FoldArgs& f, size_t gidx, GroupParams& gp) {
-  gp.gidx = gidx;
-  gp.s = f.s[gidx];
-  gp.zp = f.zp[gidx];
-  gp.mx = f.mx[gidx];
-  gp.mn = f.mn[gidx];
-  gp.al = f.alpha[gidx];
-  gp.be = f.beta[gidx];
-}
-
-__device__ __forceinline__ void group_prepare(const FoldArgs& f, GroupParams& gp) {
-  const float Q = static_cast<float>((1 << f.bits) - 1);
-  const float Qs = static_cast<float>((1 << (f.bits - 1)) - 1);
-  const float hi = __fmul_rn(gp.al, gp.mx);
-  const float lo = __fmul_rn(gp.be, gp.mn);
-  const float s_raw = f.symmetric ? __fdiv_rn(fmaxf(hi, -lo), Qs) : __fdiv_rn(__fsub_rn(hi, lo), Q);
-  gp.guarded = s_raw < kScaleGuard;
-  gp.take_hi = hi >= -lo;
-  gp.lo_s = __fdiv_rn(lo, gp.s);
-}
-
-// Finishes a group: dalpha, dbeta from the (full) sums and the SignSGD step of alpha, beta.
-__device__ __forceinline__ bool group_finish(const FoldArgs& f, const GroupParams& gp, float csum, float osum,
-                                             bool write) {
-  const float Q = static_cast<float>((1 << f.bits) - 1);
-  const float Qs = static_cast<float>((1 << (f.bits - 1)) - 1);
-  if (gp.guarded) csum = 0.0f;
-  float dhi, dlo;
-  if (f.symmetric) {
-    const float ds = __fdiv_rn(csum, Qs);
-    dhi = gp.take_hi ? ds : 0.0f;
-    dlo = gp.take_hi ? 0.0f : -ds;
-  } else {
-    const float cq = __fdiv_rn(csum, Q);
-    dhi = cq;
-    dlo = __fsub_rn(osum, cq);
-  }
-  const bool sums_bad = !isfinite(csum) || !isfinite(osum);
-  const float da = __fmul_rn(gp.mx, dhi);
-  const float db = __fmul_rn(gp.mn, dlo);
-  if (write) {
-    f.alpha[gp.gidx] = sign_step(gp.al, da, f.lr, f.c_min, f.c_max);
-    f.beta[gp.gidx] = sign_step(gp.be, db, f.lr, f.c_min, f.c_max);
-    if (f.da_out) f.da_out[gp.gidx] = da;
-    if (f.db_out) f.db_out[gp.gidx] = db;
-  }
-  return sums_bad || !isfinite(da) || !isfinite(db);
 }
 
 // `wait_acc` waits for the accumulator (returns false on abort); `xch` is this

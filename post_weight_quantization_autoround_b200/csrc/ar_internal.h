@@ -88,6 +88,18 @@ int resid_partials(int M, int N);
 // Backward of the tuning step: dW_hat = G^T X (reduction over the M tokens),
 // folded through the straight-through estimator and applied as a SignSGD step.
 // ldg, ldx: row strides of G and X when they are column slices of wider matrices (0: dense).
+// Standalone fold + SignSGD from a materialised dL/dW_hat (fp32 [N][K]) (ar_fold.cu),
+// group sizes 32, 64, 128, 256; used for short token counts instead of the
+// weight-gradient GEMM's fold epilogue.  With W_hat_next it also writes the next
+// step's QDQ (W_hat_next bf16, and the new scale / zero-point into fa.s, fa.zp).
+bool fold_int_supported(int group_size);
+// The linear step's choice: the split fold below kFoldSplitTokens tokens for g <= 128.
+bool use_split_fold(int64_t M, int group_size);
+cudaError_t launch_fold_int(const float* dW, const FoldArgs& fa, int64_t N, int64_t K, uint16_t* W_hat_next,
+                            cudaStream_t stream);
+// Below this many tokens a linear layer's step writes dL/dW_hat and folds in a
+// separate kernel (the fold epilogue would pace the weight-gradient GEMM).
+constexpr int64_t kFoldSplitTokens = 8192;
 cudaError_t launch_gemm_fold(const uint16_t* G, const uint16_t* X, const FoldArgs& fa, int M, int N, int K,
                              cudaStream_t stream, int64_t ldg = 0, int64_t ldx = 0);
 

@@ -15,6 +15,7 @@
 // a warp; each thread owns 8 consecutive weights per chunk (one 16-byte load
 // of bf16 W, two 16-byte loads of fp32 V) and g/(8*TPG) chunks.  The group's
 // min/max are reduced with xor-shuffles inside the TPG lanes.
+#include "ar_fold.cuh"
 #include "ar_internal.h"
 
 namespace ar {
@@ -59,33 +60,6 @@ cudaError_t launch_wait_timeout(uint64_t limit_ns, int* gave_up, cudaStream_t st
   LaunchScope scope(stream, "wait_timeout_kernel");
   wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_ns, gave_up);
   return cudaGetLastError();
-}
-
-struct QParams {
-  float s, zp, lo, mx, mn;
-  bool guarded;
-};
-
-// Scale / zero-point of a group; identical arithmetic in every kernel that needs it.
-__device__ __forceinline__ QParams group_qparams(float mx, float mn, float alpha, float beta, int bits,
-                                                 int symmetric) {
-  QParams p;
-  p.mx = mx;
-  p.mn = mn;
-  const float hi = __fmul_rn(alpha, mx);
-  const float lo = __fmul_rn(beta, mn);
-  float s;
-  if (!symmetric) {
-    s = __fdiv_rn(__fsub_rn(hi, lo), static_cast<float>((1 << bits) - 1));
-  } else {
-    s = __fdiv_rn(fmaxf(hi, -lo), static_cast<float>((1 << (bits - 1)) - 1));
-  }
-  p.guarded = s < kScaleGuard;
-  if (p.guarded) s = kScaleGuard;
-  p.s = s;
-  p.lo = lo;
-  p.zp = symmetric ? static_cast<float>(1 << (bits - 1)) : roundf(__fdiv_rn(-lo, s));
-  return p;
 }
 
 template <int TPG, int CHUNKS>
@@ -151,10 +125,8 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ W
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float w = (i & 1) ? bf16_hi(wr[i >> 1]) : bf16_lo(wr[i >> 1]);
-      const float u = __fadd_rn(__fdiv_rn(w, p.s), vv[i]);
-      const float t = __fadd_rn(roundf(u), p.zp);
-      const float q = fminf(fmaxf(t, 0.0f), Q);
-      wh[i] = __fmul_rn(p.s, __fsub_rn(q, p.zp));
+      float q;
+      wh[i] = qdq_elem(w, vv[i], p, Q, q);
       qb[i >> 2] |= static_cast<uint32_t>(q) << (8 * (i & 3));
     }
     if (W_hat) {
@@ -232,9 +204,8 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(const uint16_t* __restr
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float w = (i & 1) ? bf16_hi(wr[i >> 1]) : bf16_lo(wr[i >> 1]);
-      const float u = __fadd_rn(__fdiv_rn(w, p.s), vv[i]);
-      const float t = __fadd_rn(roundf(u), p.zp);
-      const float q = fminf(fmaxf(t, 0.0f), Q);
+      float q;
+      (void)qdq_elem(w, vv[i], p, Q, q);
       bits |= static_cast<uint64_t>(q) << (BITS * i);
     }
     uint8_t* dst = packed + (e * BITS) / 8;
