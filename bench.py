@@ -322,8 +322,8 @@ def w4a16_bench(ar, torch, peaks, reps=20):
                         "roofline_frac": t_roof / (ms * 1e-3),
                         "algorithmic_bytes": nbytes, "kernel": ar.ar_last_kernels()}
     out["shape"] = f"{N}x{K} int4 g{g}, fp16 scale/zero, bf16 activations; L2 flushed before each launch"
-    # the same layer packed at 2, 3 and 8 bits (decode kernel at T = 1; T = 256: tcgen05 dequant GEMM for 2
-    # and 8 bits, the decode kernel 16 tokens at a time for 3 bits)
+    # the same layer packed at 2, 3 and 8 bits (T = 1: the decode kernel at 2 and 3 bits, the tcgen05
+    # dequant GEMM at 8 bits; T = 256: the tcgen05 dequant GEMM)
     W = to_dev_bf16(d["W"], torch)
     V = torch.zeros((N, K), dtype=torch.float32, device="cuda")
     for bits in (2, 3, 8):
@@ -713,7 +713,22 @@ def run_case(name, ar, torch):
         fn = lambda: ar.ar_tune_block(ar.AR_BLOCK_SWIGLU_MLP, layers, X, Y, cfg, 1, loss, ws)
     elif name == "decoder":  # one joint step of a Llama-7B-shaped decoder block on one 2048-token sample
         fn = decoder_step_fn(ar, torch, 1, 2048, 1)[0]
-    elif name in ("w4a16_t1", "nvfp4_gemm_t1", "nvfp4_gemm_t256"):  # the 8192 x 28672 layer's exports
+    elif name == "lowbit_b2g32":  # two tuning steps per call of the W2 g32 4096 x 4096 layer, 2048 tokens
+        wl = synth.WORKLOADS[name]
+        N, K, M, g = wl.n_out, wl.n_in, wl.m_tokens, wl.group_size
+        d = synth.make_linear(N, K, M, seed=wl.seed)
+        W, X = to_dev_bf16(d["W"], torch), to_dev_bf16(d["X"], torch)
+        del d
+        V = torch.zeros((N, K), device=dev)
+        a = torch.ones((N, K // g), device=dev)
+        b = torch.ones((N, K // g), device=dev)
+        cfg = ar.ar_qconfig_default(bits=wl.bits, group_size=g, lr=wl.lr)
+        Y = torch.empty((M, N), device=dev)
+        ar.ar_linear_forward(X, W, Y)
+        ws = torch.empty(ar.ar_tune_step_workspace(W, V, a, b, M, cfg, 2), dtype=torch.uint8, device=dev)
+        loss = torch.empty(2, device=dev)
+        fn = lambda: ar.ar_tune_step(W, V, a, b, X, Y, cfg, 2, loss, ws)
+    elif name in ("w4a16_t1", "w3a16_t256", "nvfp4_gemm_t1", "nvfp4_gemm_t256"):  # the 8192 x 28672 layer's exports
         N, K, g = 8192, 28672, 128
         d = synth.make_linear(N, K, 1, seed=5, x_outlier_channels=0)
         W = to_dev_bf16(d["W"], torch)
@@ -721,7 +736,16 @@ def run_case(name, ar, torch):
         T = 256 if name.endswith("t256") else 1
         A = to_dev_bf16(synth.make_activations(T, K, seed=T), torch)
         y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
-        if name == "w4a16_t1":
+        if name == "w3a16_t256":
+            V = torch.zeros((N, K), device=dev)
+            a = torch.ones((N, K // g), device=dev)
+            pk = torch.empty((N, K * 3 // 32), dtype=torch.int32, device=dev)
+            s16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+            z16 = torch.empty((N, K // g), dtype=torch.float16, device=dev)
+            ar.ar_pack_codes(W, V, a, a, ar.ar_qconfig_default(bits=3, group_size=g), pk, s16, z16)
+            del V, a
+            fn = lambda: ar.ar_wxa16_gemm(A, pk, s16, z16, g, 3, y)
+        elif name == "w4a16_t1":
             V = torch.zeros((N, K), device=dev)
             a = torch.ones((N, K // g), device=dev)
             pk = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
@@ -751,8 +775,8 @@ def run_case(name, ar, torch):
     return 0 if st == 0 else 1
 
 
-CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp", "decoder", "w4a16_t1", "nvfp4_gemm_t1",
-         "nvfp4_gemm_t256")
+CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp", "decoder", "lowbit_b2g32", "w4a16_t1",
+         "w3a16_t256", "nvfp4_gemm_t1", "nvfp4_gemm_t256")
 
 
 def main():

@@ -371,10 +371,11 @@ AR_API ar_status ar_pack_codes(const uint16_t* W, const float* V, const float* a
 /* WbA16 matmul for codes packed by ar_pack_codes (bits 2, 3, 4 or 8):
  *   out[t][n] = sum_k A[t][k] (q[n][k] - zero[n][k/g]) scale[n][k/g]
  * A bf16 [T][K]; zero must hold integers 0..2^bits-1; out bf16 [T][N].  bits 4
- * is ar_w4a16_gemm.  3 bits at every T (16 tokens per launch) and 2 bits at
- * T <= 16 run a decode kernel (mma.sync, one range of weight rows per SM, the
- * codes read straight from the bit stream); 8 bits, and 2 bits from 17 tokens,
- * run the tcgen05 dequant GEMM.  (q - z) is exact in bf16 for every width and
+ * is ar_w4a16_gemm.  2 and 3 bits at T <= 8 run a decode kernel (mma.sync,
+ * one range of weight rows per SM, the codes read straight from the bit
+ * stream); 8 bits, and 2 and 3 bits from 9 tokens, run the tcgen05 dequant
+ * GEMM (a 3-bit stage of 128 k is 48 bytes of a row: its code slots hold
+ * three 128-byte boxes, eight stages).  (q - z) is exact in bf16 for every width and
  * each group's sum is scaled once in fp32.  Needs 1 <= T < 2^31, group_size
  * 32..1024 (power of two) dividing K, K % 128 == 0; otherwise
  * AR_ERR_UNSUPPORTED or AR_ERR_INVALID_ARG before any launch. */

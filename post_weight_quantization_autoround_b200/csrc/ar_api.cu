@@ -896,10 +896,11 @@ ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
     if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   }
-  // every 3-bit call and 2-bit decode batches: the mma.sync decode kernel (16 tokens at a
-  // time); 8 bits, and 2 bits from 17 tokens: the tcgen05 dequant GEMM (at 8 bits it is the
-  // faster of the two for decode batches too)
-  cudaError_t e = (bits == 3 || (bits == 2 && T <= 16))
+  // 2 and 3 bits up to 8 tokens: the mma.sync decode kernel; 8 bits, and 2 and 3 bits from
+  // 9 tokens: the tcgen05 dequant GEMM (measured on 8192 x 28672: the decode kernel 80 us
+  // at T <= 8 against 88-90 us, but 90-96 us at T = 16 against 88-90 us; at 8 bits the
+  // GEMM is the faster at every T)
+  cudaError_t e = ((bits == 2 || bits == 3) && T <= 8)
                       ? launch_wbx_dec(A, static_cast<int>(T), packed, scale_f16, zero_f16, static_cast<int>(N),
                                        static_cast<int>(K), group_size, bits, out,
                                        reinterpret_cast<cudaStream_t>(stream))

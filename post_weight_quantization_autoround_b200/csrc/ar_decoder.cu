@@ -19,6 +19,11 @@
 // over its keys, so that their rounding does not depend on the order in which
 // keys are visited; O = P V needs no division afterwards.
 //
+// The exponentials are CUDA's fast exponential intrinsic (__expf, accurate to
+// a few fp32 ulp), much cheaper per score than the accurate expf; a
+// probability's bf16 rounding changes only within ~1e-7 of a rounding midpoint,
+// the size of a summation-order difference.
+//
 // Attention runs on mma.sync m16n8k16 (bf16, fp32 accumulation) over 64-row
 // tiles staged in shared memory with cp.async (double-buffered, 16-byte row
 // padding so that ldmatrix reads are free of bank conflicts).  It is ~5 % of the
@@ -175,10 +180,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float mn = fmaxf(m[hr], mx);
       float t = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) t += expf(z[i] - mn);
+      for (int i = 0; i < 16; ++i) t += __expf(z[i] - mn);
       t += __shfl_xor_sync(0xFFFFFFFFu, t, 1);
       t += __shfl_xor_sync(0xFFFFFFFFu, t, 2);
-      lsum[hr] = lsum[hr] * expf(m[hr] - mn) + t;
+      lsum[hr] = lsum[hr] * __expf(m[hr] - mn) + t;
       m[hr] = mn;
     }
     __syncthreads();  // the next iteration refills the buffer read here
@@ -227,7 +232,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int qi = r0 + g + 8 * (i >> 1);
         const int kj = 8 * nt + 2 * c + (i & 1);
         const float z = __fmul_rn(acc[nt][i], scale);
-        acc[nt][i] = (kb == qb && kj > qi) ? 0.f : expf(z - lse[i >> 1]);
+        acc[nt][i] = (kb == qb && kj > qi) ? 0.f : __expf(z - lse[i >> 1]);
       }
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {  // keys 16 kk .. 16 kk + 15
@@ -384,7 +389,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int qi = r0 + g + 8 * hr;
         const int kj = 8 * nt + 2 * c + (i & 1);
         const float z = __fmul_rn(sc[nt][i], scale);
-        const float p = (kb == qb && kj > qi) ? 0.f : round_bf16(expf(z - lr[hr]));
+        const float p = (kb == qb && kj > qi) ? 0.f : round_bf16(__expf(z - lr[hr]));
         sc[nt][i] = __fmul_rn(__fmul_rn(p, __fsub_rn(dp[nt][i], dr[hr])), scale);
       }
 #pragma unroll
@@ -503,7 +508,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int kj = r0 + g + 8 * (i >> 1);                  // key within the block
           const int qi = 32 * half + 8 * nt + 2 * c + (i & 1);   // query within its block
           const float z = __fmul_rn(st[nt][i], scale);
-          const float p = (qb == kb && qi < kj) ? 0.f : round_bf16(expf(z - lq[qi]));
+          const float p = (qb == kb && qi < kj) ? 0.f : round_bf16(__expf(z - lq[qi]));
           st[nt][i] = p;
           dpt[nt][i] = __fmul_rn(__fmul_rn(p, __fsub_rn(dpt[nt][i], dq[qi])), scale);
         }

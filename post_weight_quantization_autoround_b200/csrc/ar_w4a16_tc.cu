@@ -37,7 +37,9 @@
 //    in a fixed order: no workspace, deterministic results.
 //
 // Packed layout (as ar_pack_int4 writes it): uint32 [N][K/8], element k at
-// bits 4*(k mod 8) of word k/8; scale/zero fp16 [N][K/g].
+// bits 4*(k mod 8) of word k/8; scale/zero fp16 [N][K/g].  Other widths (2, 3,
+// 8 bits, as ar_pack_codes writes them): each row a little-endian bit stream,
+// element k at stream bits BITS k .. BITS k + BITS - 1.
 #include <cooperative_groups.h>
 
 #include <cuda_fp8.h>
@@ -52,14 +54,19 @@ namespace {
 constexpr int kTcRows = 128;  // weight rows per CTA (MMA M, TMEM lanes)
 constexpr int kTcK = 128;     // k per stage: 8 MMAs per barrier hand-off
 constexpr int kSub = kTcK / 64;  // 64-k sub-tiles (one 128-byte swizzle row of bf16 each)
-constexpr int kCodeBytes = kTcRows * 128;  // 16 KiB per code slot: one 128-byte row of packed words per weight row
-// k per code slot and stages per slot for BITS-bit codes (32/BITS codes per word)
+constexpr int kCodeBytes = kTcRows * 128;  // 16 KiB per TMA box of codes: a 128-byte row of packed words per weight row
+// Code slots per width.  A 128-k stage takes 16 BITS bytes of a row.  At 2, 4 and 8
+// bits a slot is one box (4, 2 or 1 stages); a 3-bit stage (48 bytes) does not divide
+// a box, so a 3-bit slot is three boxes side by side, 384 bytes a row: eight stages.
 template <int BITS>
 struct CodeCfg {
-  static constexpr int kCodeK = 1024 / BITS;          // 512, 256 or 128
-  static constexpr int kChunksPerSlot = kCodeK / 128;  // 4, 2 or 1 stages of 128 k
+  static constexpr int kBoxes = BITS == 3 ? 3 : 1;
+  static constexpr int kChunksPerSlot = BITS == 3 ? 8 : 8 / BITS;  // stages of 128 k per slot
+  static constexpr int kSlots = BITS == 3 ? 2 : 4;
+  static constexpr int kSlotBytes = kBoxes * kCodeBytes;
+  static_assert(kChunksPerSlot * 16 * BITS == kBoxes * 128, "a slot holds whole stages");
 };
-constexpr int kCodeSlots = 4;
+constexpr int kCodeSlotsMax = 4;
 constexpr int kNBufMax = 4;   // TMEM accumulators, one group each
 constexpr int kAStages = 4;   // A operand stages in TMEM (and activation stages in shared memory)
 constexpr int kACols = kTcK / 2;  // TMEM columns per A stage (two bf16 per column)
@@ -78,7 +85,7 @@ __host__ __device__ constexpr bool slot_phases_in_order(int per_slot, int sets, 
   return per_slot % sets == 0 || (sets % per_slot == 0 && slots % (sets / per_slot) == 0);
 }
 
-template <int TN>
+template <int TN, int BITS>
 struct TcCfg {
   // One dequantization warp per TMEM lane quarter is latency bound (its nibble
   // and permute chains), so narrow tiles, whose epilogue needs few registers,
@@ -89,7 +96,7 @@ struct TcCfg {
   static constexpr int kActBytes = TN * 128 * kSub;    // TN tokens x kTcK k bf16, kSub sub-tiles
   static constexpr int kStageBytes = kActBytes;
   static constexpr int kStages = kAStages;
-  static constexpr int kRingBytes = kStages * kStageBytes + kCodeSlots * kCodeBytes;
+  static constexpr int kRingBytes = kStages * kStageBytes + CodeCfg<BITS>::kSlots * CodeCfg<BITS>::kSlotBytes;
   static constexpr int kNBuf = TN >= 128 ? 2 : kNBufMax;  // accumulators fit below kACol0
   static_assert(kNBuf * TN <= kACol0, "accumulators and A stages share the 512 TMEM columns");
   static_assert(kACol0 + kACols * kAStages <= kTmemCols, "A stages fit in TMEM");
@@ -116,8 +123,8 @@ struct TcCtl {
   uint64_t full[kAStages];      // TMA: activations of the stage landed
   uint64_t dq_full[kAStages];   // A operand written and activations landed (one arrival per row quarter)
   uint64_t empty[kAStages];     // MMAs of the stage done (tcgen05.commit)
-  uint64_t code_full[kCodeSlots];   // TMA: codes of the slot landed
-  uint64_t code_empty[kCodeSlots];  // codes of the slot read (one arrival per row quarter and stage)
+  uint64_t code_full[kCodeSlotsMax];   // TMA: codes of the slot landed
+  uint64_t code_empty[kCodeSlotsMax];  // codes of the slot read (one arrival per row quarter and stage)
   uint64_t tmem_full[kNBufMax];
   uint64_t tmem_empty[kNBufMax];
   uint64_t mma_done;
@@ -211,6 +218,34 @@ __device__ __forceinline__ void dequant16(uint32_t x, uint32_t zz, uint32_t* o) 
   for (int j = 0; j < 4; ++j) {
     o[j] = __byte_perm(e[2 * j], e[2 * j + 1], 0x5410);      // (k_{2j}, k_{2j+1})
     o[4 + j] = __byte_perm(e[2 * j], e[2 * j + 1], 0x7632);  // (k_{8+2j}, k_{9+2j})
+  }
+}
+
+// Component c (0..3, known at compile time) of a 16-byte vector.
+__device__ __forceinline__ uint32_t vec_word(const uint4& v, int c) {
+  return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
+}
+
+// 32 three-bit codes of three consecutive words (the row's bit stream: code m at
+// bits 3m .. 3m + 2 of the 96 bits, words little-endian) -> 32 bf16 values (q - z)
+// in k order (16 words); zz = (128 + z) in both halves.  For each four codes y (12
+// bits), y (1 + 2^13) = y | y << 13 (the two do not overlap, so nothing carries)
+// holds q0 at bit 0, q1 at bit 16, q2 at bit 6 and q3 at bit 22: one mask gives
+// the pair (q0, q1) and, after a 6-bit shift, (q2, q3).
+__device__ __forceinline__ void dequant3x32(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t zz, uint32_t* o) {
+  constexpr uint32_t kMask = 0x00070007u, kBias = 0x43004300u;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {  // codes 4j .. 4j + 3: stream bits 12j .. 12j + 11
+    const int b = 12 * j;
+    uint32_t y;
+    if (b + 12 <= 32) y = w0 >> b;
+    else if (b < 32) y = __funnelshift_r(w0, w1, b);
+    else if (b + 12 <= 64) y = w1 >> (b - 32);
+    else if (b < 64) y = __funnelshift_r(w1, w2, b - 32);
+    else y = w2 >> (b - 64);
+    const uint32_t m = (y & 0xFFFu) * 0x2001u;
+    o[2 * j] = bf16x2_sub((m & kMask) | kBias, zz);             // (k 4j, 4j + 1)
+    o[2 * j + 1] = bf16x2_sub(((m >> 6) & kMask) | kBias, zz);  // (k 4j + 2, 4j + 3)
   }
 }
 
@@ -343,10 +378,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // into the dequantized operand, the per-tensor scale applied per group in the
 // epilogue); BITS is then 4.
 template <int TN, int KSPLIT, int BITS, bool FP4>
-__global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
+__global__ void __launch_bounds__(TcCfg<TN, BITS>::kThreads, 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const TcParams p) {
-  using Cfg = TcCfg<TN>;
+  using Cfg = TcCfg<TN, BITS>;
+  using Code = CodeCfg<BITS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* codes = ring + Cfg::kStages * Cfg::kStageBytes;
@@ -377,9 +413,9 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
       mbar_init(&ctl->dq_full[s], 4);  // the four warps that cover one stage's 128 rows
       mbar_init(&ctl->empty[s], 1);
     }
-    for (int s = 0; s < kCodeSlots; ++s) {
+    for (int s = 0; s < Code::kSlots; ++s) {
       mbar_init(&ctl->code_full[s], 1);
-      mbar_init(&ctl->code_empty[s], 4 * CodeCfg<BITS>::kChunksPerSlot);
+      mbar_init(&ctl->code_empty[s], 4 * Code::kChunksPerSlot);
     }
     for (int b = 0; b < Cfg::kNBuf; ++b) {
       mbar_init(&ctl->tmem_full[b], 1);
@@ -517,19 +553,26 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ code TMA: up to 16 stages ahead
     if (lane == 0) {
-      constexpr int kChunksPerSlot = CodeCfg<BITS>::kChunksPerSlot;
+      constexpr int kChunksPerSlot = Code::kChunksPerSlot;
+      constexpr int kStageWords = kTcK * BITS / 32;  // 32-bit words of a row per stage
       const int n_slots = (c_end - c_begin + kChunksPerSlot - 1) / kChunksPerSlot;
       uint32_t slots = 0;
       for (int j = 0; j < n_slots; ++j) {
-        const uint32_t cs = static_cast<uint32_t>(j % kCodeSlots);
-        if (!mbar_wait_sleep(&ctl->code_empty[cs], ((j / kCodeSlots) & 1u) ^ 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(&ctl->code_full[cs], kCodeBytes);
-        tma_load_2d(codes + cs * kCodeBytes, &tmW, &ctl->code_full[cs], (c_begin + j * kChunksPerSlot) * (kTcK * BITS / 32),
-                    n0);
+        const uint32_t cs = static_cast<uint32_t>(j % Code::kSlots);
+        if (!mbar_wait_sleep(&ctl->code_empty[cs], ((j / Code::kSlots) & 1u) ^ 1u, abort_flag)) break;
+        // a slot's boxes are consecutive 32-word spans of the rows; boxes that start past this
+        // CTA's last stage hold nothing it reads and are not loaded (the first always is)
+        const int x0 = (c_begin + j * kChunksPerSlot) * kStageWords;
+        int boxes = 1;
+        while (boxes < Code::kBoxes && x0 + 32 * boxes < c_end * kStageWords) ++boxes;
+        mbar_arrive_expect_tx(&ctl->code_full[cs], boxes * kCodeBytes);
+        for (int b = 0; b < boxes; ++b)
+          tma_load_2d(codes + cs * Code::kSlotBytes + b * kCodeBytes, &tmW, &ctl->code_full[cs], x0 + 32 * b, n0);
         ++slots;
       }
-      const uint32_t first_slot = slots > kCodeSlots ? slots - kCodeSlots : 0;
-      for (uint32_t j = first_slot; j < slots; ++j) mbar_wait_drain(&ctl->code_full[j % kCodeSlots], (j / kCodeSlots) & 1u);
+      const uint32_t first_slot = slots > Code::kSlots ? slots - Code::kSlots : 0;
+      for (uint32_t j = first_slot; j < slots; ++j)
+        mbar_wait_drain(&ctl->code_full[j % Code::kSlots], (j / Code::kSlots) & 1u);
     }
   } else if (!is_epi) {
     // ------------------------------------------------------------ dequantization
@@ -545,31 +588,35 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
     // code slots: every dequantization set reads every phase of a slot (stages per slot a multiple
     // of the sets), or each slot is always read by the same set (the sets a multiple of the stages
     // per slot and their ratio dividing the slot count), so each set waits on a slot's phases in order
-    static_assert(slot_phases_in_order(CodeCfg<BITS>::kChunksPerSlot, Cfg::kDqWarps / 4, kCodeSlots),
+    static_assert(slot_phases_in_order(Code::kChunksPerSlot, Cfg::kDqWarps / 4, Code::kSlots),
                   "code slots: phases waited in order by every dequantization set");
     for (int i = dw >> 2; i < c_end - c_begin; i += Cfg::kDqWarps / 4) {
       const int c = c_begin + i;
       const uint32_t stage = static_cast<uint32_t>(i % Cfg::kStages);
       const uint32_t phase = static_cast<uint32_t>((i / Cfg::kStages) & 1);
-      constexpr int kChunksPerSlot = CodeCfg<BITS>::kChunksPerSlot;
+      constexpr int kChunksPerSlot = Code::kChunksPerSlot;
       const uint32_t j = static_cast<uint32_t>(i / kChunksPerSlot);
-      const uint32_t cs = j % kCodeSlots;
+      const uint32_t cs = j % Code::kSlots;
       // codes landed, the MMAs of this stage's previous use have released its A
       // operand, and the stage's activations landed (so the MMA thread waits once)
-      const bool ok = mbar_wait_sleep(&ctl->code_full[cs], (j / kCodeSlots) & 1u, abort_flag) &&
+      const bool ok = mbar_wait_sleep(&ctl->code_full[cs], (j / Code::kSlots) & 1u, abort_flag) &&
                       mbar_wait_sleep(&ctl->empty[stage], phase ^ 1u, abort_flag);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
-      // this stage's 16*BITS bytes of row r: 16-byte vectors qv..qv+BITS-1 of the row, swizzled by r % 8
+      // this stage's 16*BITS bytes of row r: 16-byte vectors qv..qv+BITS-1 of the slot's
+      // row (vector v in box v / 8 at position v % 8), each box swizzled by r % 8
       const uint32_t qv = static_cast<uint32_t>(BITS * (i % kChunksPerSlot));
-      const uint32_t pk = smem_u32(codes + cs * kCodeBytes) + r * 128;
+      const uint32_t pk = smem_u32(codes + cs * Code::kSlotBytes) + r * 128;
       const int k0 = c * kTcK;
       // the stage's codes: all loads issued before any conversion, except that
       // 8-bit stages (eight 16-byte vectors a row) load one half at a time
       constexpr int kPre = BITS == 8 ? BITS / 2 : BITS;
       uint4 pw[kPre];
 #pragma unroll
-      for (int v = 0; v < kPre; ++v) pw[v] = ld_shared_v4(pk + (((qv + v) ^ sw) << 4));
+      for (int v = 0; v < kPre; ++v) {
+        const uint32_t qvv = qv + v;
+        pw[v] = ld_shared_v4(pk + (qvv >> 3) * kCodeBytes + (((qvv & 7) ^ sw) << 4));
+      }
       // NVFP4: the row's 8 block scales of this stage (one per two words)
       uint32_t sc2[8];
       if (FP4) {
@@ -603,6 +650,15 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
 #pragma unroll
           for (int v = 0; v < kPre; ++v) pw[v] = ld_shared_v4(pk + (((qv + kPre + v) ^ sw) << 4));
         }
+        if constexpr (BITS == 3) {
+          // the half's two 32-code units: words 3u .. 3u + 2 of the stage for unit u = 2 half, 2 half + 1
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int w = 3 * (2 * half + u);
+            dequant3x32(vec_word(pw[w >> 2], w & 3), vec_word(pw[(w + 1) >> 2], (w + 1) & 3),
+                        vec_word(pw[(w + 2) >> 2], (w + 2) & 3), zz[2 * half + u], &a[16 * u]);
+          }
+        } else {
 #pragma unroll
         for (int v = 0; v < BITS / 2; ++v) {
           const uint4 pv = pw[BITS == 8 ? v : half * (BITS / 2) + v];
@@ -630,6 +686,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
               dequant4b(xs[u], zf[quarter], &a[col]);
             }
           }
+        }
         }
         tmem_st32(lane_base + kACols * stage + 32 * half, a);
       }
@@ -721,7 +778,7 @@ __global__ void __launch_bounds__(TcCfg<TN>::kThreads, 1)
 template <int TN, int KSPLIT, int BITS, bool FP4>
 cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int n_tiles, cudaStream_t stream,
                       const char* name) {
-  using Cfg = TcCfg<TN>;
+  using Cfg = TcCfg<TN, BITS>;
   CUtensorMap tmA;
   cudaError_t e = make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, static_cast<uint64_t>(p.T),
                                static_cast<uint64_t>(p.K), 64, TN, CU_TENSOR_MAP_SWIZZLE_128B);  // kSub boxes per stage
@@ -776,6 +833,13 @@ struct TcNames<2> {
                                        "wxa16_tc_kernel<b=2,TN=32>", "wxa16_tc_kernel<b=2,TN=32,split2>",
                                        "wxa16_tc_kernel<b=2,TN=64>", "wxa16_tc_kernel<b=2,TN=64,split2>",
                                        "wxa16_tc_kernel<b=2,TN=128>", "wxa16_tc_kernel<b=2,TN=128,split2>"};
+};
+template <>
+struct TcNames<3> {
+  static constexpr const char* n[8] = {"wxa16_tc_kernel<b=3,TN=16>", "wxa16_tc_kernel<b=3,TN=16,split2>",
+                                       "wxa16_tc_kernel<b=3,TN=32>", "wxa16_tc_kernel<b=3,TN=32,split2>",
+                                       "wxa16_tc_kernel<b=3,TN=64>", "wxa16_tc_kernel<b=3,TN=64,split2>",
+                                       "wxa16_tc_kernel<b=3,TN=128>", "wxa16_tc_kernel<b=3,TN=128,split2>"};
 };
 template <>
 struct TcNames<4> {
@@ -880,6 +944,7 @@ cudaError_t launch_wxa16_tc(const uint16_t* A, int T, const uint32_t* packed, co
                             const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,
                             cudaStream_t stream) {
   if (bits == 2) return launch_bits_tc<2>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
+  if (bits == 3) return launch_bits_tc<3>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
   if (bits == 4) return launch_bits_tc<4>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
   if (bits == 8) return launch_bits_tc<8>(A, T, packed, scale16, zero16, N, K, group_size, out, stream);
   return cudaErrorInvalidValue;

@@ -1,6 +1,6 @@
 // WbA16 matmul at decode batches (T <= 16 tokens) for codes packed at 2, 3 or 8
-// bits (the per-row little-endian bit stream of ar_pack_codes), and the 3-bit
-// matmul at any T (16 tokens at a time):
+// bits (the per-row little-endian bit stream of ar_pack_codes); the launcher
+// takes any T, 16 tokens at a time:
 //   out[t][n] = sum_k A[t][k] (q[n][k] - zero[n][k/g]) scale[n][k/g].
 //
 // [AR] §4 (comparison table, "Real INT4 Kernel" column): the weights stay

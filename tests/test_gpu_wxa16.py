@@ -73,7 +73,7 @@ def test_wxa16_matches_oracle(ar, bits, T, N, K, g):
     out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, bits, out)
     assert ar.ar_get_device_status() == 0
-    if bits == 3 or (bits == 2 and T <= 16):
+    if bits in (2, 3) and T <= 8:
         assert "wbx_dec_kernel<b=%d" % bits in ar.ar_last_kernels()
     else:
         assert "wxa16_tc_kernel<b=%d" % bits in ar.ar_last_kernels()
@@ -95,3 +95,48 @@ def test_wxa16_four_bits_is_w4a16(ar):
     ar.ar_wxa16_gemm(A, packed, s16, z16, g, 4, o1)
     ar.ar_w4a16_gemm(A, packed, s16, z16, g, o2)
     assert torch.equal(o1, o2)
+
+
+def test_wxa16_three_bit_tensor_core_many_tiles(ar):
+    """3-bit codes on the tcgen05 dequant GEMM: K = 4096 is 32 stages of 128 k, four
+    three-box code slots of eight stages each; eight row tiles with a ragged last one
+    (1000 rows) and a ragged token tail (300 = 2 x 128 + 44)."""
+    N, K, g, T = 1000, 4096, 64, 300
+    d = synth.make_linear(N, K, 1, seed=31)
+    V, a, b = synth.make_state(N, K, g, seed=3, spread=True)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 3, g)
+    A = synth.make_activations(T, K, seed=32)
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 3, out)
+    assert ar.ar_get_device_status() == 0
+    assert "wxa16_tc_kernel<b=3,TN=128" in ar.ar_last_kernels()
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 3, g)
+    words = O.pack_bitstream(st["q"], 3)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16),
+                         z16.cpu().numpy().view(np.uint16), g, 3)
+    got = out.float().cpu().numpy()
+    for t in range(T):  # every token row, the ragged tail included
+        assert rel_l2(got[t], ref[t]) <= TC_RTOL
+
+
+@pytest.mark.parametrize("T", [17, 256])
+def test_wxa16_three_bit_full_size_sampled_rows(ar, T):
+    """8192 x 28672 down projection at 3 bits (g 128) on the tensor-core path, sampled
+    output rows against the oracle."""
+    wl = synth.WORKLOADS["down_8192_28672"]
+    N, K, g = wl.n_out, wl.n_in, wl.group_size
+    d = synth.make_linear(N, K, 1, seed=wl.seed, x_outlier_channels=0)
+    V, a, b = synth.make_state(N, K, g)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 3, g)
+    A = synth.make_activations(T, K, seed=1)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 3, out)
+    assert ar.ar_get_device_status() == 0
+    assert "wxa16_tc_kernel<b=3" in ar.ar_last_kernels()
+    rows = np.sort(np.random.default_rng(7).choice(N, 64, replace=False))
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"][rows]), V[rows], a[rows], b[rows], 3, g)
+    words = O.pack_bitstream(st["q"], 3)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32)[rows], words)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16)[rows],
+                         z16.cpu().numpy().view(np.uint16)[rows], g, 3)
+    assert rel_l2(out.float().cpu().numpy()[:, rows], ref) <= TC_RTOL
