@@ -24,11 +24,12 @@
 // probability's bf16 rounding changes only within ~1e-7 of a rounding midpoint,
 // the size of a summation-order difference.
 //
-// Attention runs on mma.sync m16n8k16 (bf16, fp32 accumulation) over 64-row
-// tiles staged in shared memory with cp.async (double-buffered, 16-byte row
-// padding so that ldmatrix reads are free of bank conflicts).  It is ~5 % of the
-// block step's FLOPs at the Llama-7B shapes.  No kernel here waits on another
-// CTA: every wait is a cp.async group wait or a CTA barrier.
+// The attention kernels here run on mma.sync m16n8k16 (bf16, fp32 accumulation)
+// over 64-row tiles staged in shared memory with cp.async (double-buffered,
+// 16-byte row padding so that ldmatrix reads are free of bank conflicts); the
+// forward at head dimension 128 on whole 128-row blocks runs on tcgen05 instead
+// (ar_attn_tc.cu).  No kernel here waits on another CTA: every wait is a
+// cp.async group wait or a CTA barrier.
 #include "ar_internal.h"
 
 namespace ar {
@@ -713,6 +714,8 @@ cudaError_t attn_bwd_launch(const uint16_t* qkv, const uint16_t* O, const uint16
 
 cudaError_t launch_attn_fwd(const uint16_t* qkv, int S, int L, int H, int head_dim, uint16_t* out, float* lse,
                             cudaStream_t st) {
+  // head dimension 128 and whole 128-row blocks: the tcgen05 kernel (ar_attn_tc.cu)
+  if (head_dim == 128 && L % 128 == 0) return launch_attn_fwd_tc(qkv, S, L, H, out, lse, st);
   if (head_dim == 128) return attn_fwd_launch<128>(qkv, S, L, H, out, lse, st);
   if (head_dim == 64) return attn_fwd_launch<64>(qkv, S, L, H, out, lse, st);
   return cudaErrorInvalidValue;

@@ -114,7 +114,8 @@ static_assert(sizeof(Ctl) <= 24576, "control block too large");
 struct Params {
   int M, N, K;  // D is M x N, reduction over K
   int tiles_m, tiles_n, num_kb;
-  int num_units;   // work units (tiles) of this launch
+  int num_units;   // work units of this launch
+  int full_units;  // units below this are whole tiles; from it on, two half-width units per tile
   int group_m;     // tile rows per raster group (columns swept inside a group, rows fastest)
   float* D;          // EPI_STORE
   const float* Y;    // EPI_RESID
@@ -221,10 +222,11 @@ __device__ __forceinline__ double epi_resid(const Params& p, uint32_t taddr, int
 
 // Straight-through fold + SignSGD.  GEMM rows are weight rows n (M = N_w),
 // GEMM columns are weight columns k (N = K_w).  Each epilogue warp owns 32
-// rows and half of the tile's 256 columns (chunks c0..c0+3 of 32).  Groups of
-// g <= 128 columns lie inside one half, so their sums stay in the thread; a
-// group of 256 spans both halves and the two warps of a lane quarter add
-// their partial sums through shared memory (fixed order: half 0 + half 1).
+// rows and half of the unit's columns (chunks of 32: four of a whole 256-column
+// tile, two of a half-width unit).  A group that fits in a warp's half keeps
+// its sums in the thread; a group as wide as the unit (256 of a whole tile, 128
+// of a half-width unit) spans both halves and the two warps of a lane quarter
+// add their partial sums through shared memory (fixed order: half 0 + half 1).
 //
 // All global loads of the tile (group parameters, W and V of the first chunk)
 // are issued before waiting for the accumulator, and each next chunk's W and
@@ -254,8 +256,11 @@ struct SplitRecv {
   uint32_t* msg;          // messages received so far by this warp
 };
 
+// `nch`: 32-column chunks per warp, 4 for a whole tile and 2 for a half-width unit;
+// a group of 2 nch chunks spans both warps of the lane quarter (the host never
+// gives a half-width unit groups wider than the unit).
 template <class WaitAcc>
-__device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n, int col_base, int half,
+__device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n, int col_base, int half, int nch,
                                          float2* xch, uint64_t* xbar, volatile int* abort_flag, WaitAcc wait_acc,
                                          bool* aborted, const SplitRecv& rx) {
   const FoldArgs& f = p.fold;
@@ -263,7 +268,7 @@ __device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n,
   const int cpg = g >> 5;  // chunks per group: 1, 2, 4 or 8
   const int groups_per_row = p.N / g;
   const float Q = static_cast<float>((1 << f.bits) - 1);
-  const int c0 = 4 * half;
+  const int c0 = nch * half;
   const bool row_ok = n < p.M;
   bool bad = false;
 
@@ -281,11 +286,11 @@ __device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n,
   }
   float csum = 0.f, osum = 0.f;
 #pragma unroll 1
-  for (int c = c0; c < c0 + 4; ++c) {
+  for (int c = c0; c < c0 + nch; ++c) {
     const int col0 = col_base + c * 32;
     const bool ok = row_ok && col0 < p.N;
     cur = nxt;
-    if (ok && c + 1 < c0 + 4 && col0 + 32 < p.N) fold_load(f, static_cast<size_t>(n) * p.N + col0 + 32, nxt);
+    if (ok && c + 1 < c0 + nch && col0 + 32 < p.N) fold_load(f, static_cast<size_t>(n) * p.N + col0 + 32, nxt);
     if (ok && ((c % cpg) == 0 || c == c0)) {
       if (c != c0) group_load(f, static_cast<size_t>(n) * groups_per_row + col0 / g, gp);
       group_prepare(f, gp);
@@ -358,10 +363,10 @@ __device__ __forceinline__ bool epi_fold(const Params& p, uint32_t taddr, int n,
       }
     }
     if (!ok) continue;
-    if (cpg <= 4 && (c % cpg) == cpg - 1) bad |= group_finish(f, gp, csum, osum, true);
+    if (cpg <= nch && (c % cpg) == cpg - 1) bad |= group_finish(f, gp, csum, osum, true);
   }
-  if (cpg == 8) {
-    // a 256-wide group: add the two halves' sums (the same order in both warps);
+  if (cpg > nch) {
+    // a group as wide as the unit: add the two halves' sums (the same order in both warps);
     // phase 0 publishes both halves, phase 1 frees the slot for the next tile
     const int lane = threadIdx.x & 31;
     xch[half * 32 + lane] = make_float2(csum, osum);
@@ -586,9 +591,31 @@ __host__ __device__ __forceinline__ void raster(int t, int tiles_m, int tiles_n,
   tm = grp * group_m + (in - tn * rows);
 }
 
-// Output tile (tm, tn) of work unit t, in this launch's BM * CG-row tiles.
-__device__ __forceinline__ void unit_coords(const Params& p, int t, int& tm, int& tn) {
-  raster(t, p.tiles_m, p.tiles_n, p.group_m, tm, tn);
+// Work unit t: output tile (tm, tn) of this launch's BM * CG-row tiles, its first
+// column and width.  Units below full_units are whole tiles in raster order; the
+// tiles after them (the last wave's, when it would leave clusters idle) are run
+// as two units of BN / 2 columns each, which other clusters take at the same time.
+struct Unit {
+  int tm, tn, col0;
+  int tile;   // tile index in raster order
+  int part;   // 0, or 1 for the right half of a split tile
+  bool wide;  // BN columns (else BN / 2)
+};
+
+__device__ __forceinline__ Unit unit_of(const Params& p, int t) {
+  Unit u;
+  if (t < p.full_units) {
+    u.tile = t;
+    u.part = 0;
+    u.wide = true;
+  } else {
+    u.tile = p.full_units + ((t - p.full_units) >> 1);
+    u.part = (t - p.full_units) & 1;
+    u.wide = false;
+  }
+  raster(u.tile, p.tiles_m, p.tiles_n, p.group_m, u.tm, u.tn);
+  u.col0 = u.tn * BN + u.part * (BN / 2);
+  return u;
 }
 
 // Raster group for a grid whose B operand has b_bytes: 1 while B fits in a share of
@@ -677,11 +704,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued = 0;
       bool ok = true;
       for (int t = tile0; ok && t < num_tiles; t += tile_step) {
-        int tm, tn;
-        unit_coords(p, t, tm, tn);
-        // this CTA's A rows and B columns
+        const Unit u = unit_of(p, t);
+        const int tm = u.tm, tn = u.tn;
+        // this CTA's A rows and B columns (a pair's CTA loads half of the unit's columns)
+        const int b_cols = u.wide ? BN / CG : BN / (2 * CG);
         const int m0 = tm * (BM * CG) + rank * (kPair ? BM : 0);
-        const int n0 = tn * BN + rank * (kPair ? BN / 2 : 0);
+        const int n0 = u.col0 + rank * (kPair ? b_cols : 0);
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -692,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kPair) {
             // both CTAs' bytes complete on the even CTA's barrier, which expects them all
             const uint32_t bar0 = mapa_shared(smem_u32(&ctl->full[stage]), 0);
-            if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], CG * (kAStage + kBStage));
+            if (rank == 0) mbar_arrive_expect_tx(&ctl->full[stage], CG * (kAStage + b_cols * BK * 2));
             if (A_MN) {
 #pragma unroll
               for (int i = 0; i < BM / 64; ++i) tma_load_2d_pair(a_dst + i * 8192, &tmA, bar0, m0 + 64 * i, kb * BK);
@@ -703,10 +731,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               // the tile's B columns are 128 gate rows then the same 128 up rows: one half each
               tma_load_2d_pair(b_dst, rank == 0 ? &tmB : &tmB2, bar0, kb * BK, tn * (BN / 2));
             } else if (B_MN) {
-#pragma unroll
-              for (int i = 0; i < BN / 2 / 64; ++i) tma_load_2d_pair(b_dst + i * 8192, &tmB, bar0, n0 + 64 * i, kb * BK);
+              // 64-column boxes: two for a whole tile's half, one for a half-width unit's
+              for (int i = 0; i < b_cols / 64; ++i) tma_load_2d_pair(b_dst + i * 8192, &tmB, bar0, n0 + 64 * i, kb * BK);
             } else {
-              tma_load_2d_pair(b_dst, &tmB, bar0, kb * BK, n0);
+              // tmB: boxes of BN / 2 rows; tmB2: boxes of BN / 4 rows (half-width units)
+              tma_load_2d_pair(b_dst, u.wide ? &tmB : &tmB2, bar0, kb * BK, n0);
             }
           } else {
             mbar_arrive_expect_tx(&ctl->full[stage], kAStage + kBStage);
@@ -745,10 +774,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, BN, A_MN, B_MN);
+      constexpr uint32_t idesc_wide = idesc_bf16_f32(BM * CG, BN, A_MN, B_MN);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(BM * CG, BN / 2, A_MN, B_MN);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int t = tile0; ok && t < num_tiles; t += tile_step) {
+        const uint32_t idesc = t < p.full_units ? idesc_wide : idesc_half;
         // a pair's accumulator is free once both CTAs' epilogues have drained it
         const bool got = kPair ? mbar_wait_cluster(&ctl->tmem_empty[acc], acc_phase ^ 1u, abort_flag)
                                : mbar_wait(&ctl->tmem_empty[acc], acc_phase ^ 1u, abort_flag);
@@ -813,8 +844,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t peer_slot = KSPLIT == 2 ? mapa_shared(smem_u32(&ctl->slot[ew][lane][0]), 0) : 0;
     const uint32_t peer_full = KSPLIT == 2 ? mapa_shared(smem_u32(&ctl->full_x[ew]), 0) : 0;
     for (int t = tile0; t < num_tiles; t += tile_step) {
-      int tm, tn;
-      unit_coords(p, t, tm, tn);
+      const Unit u = unit_of(p, t);
+      const int tm = u.tm, tn = u.tn;
+      const int nch = u.wide ? 4 : 2;  // 32-column chunks per warp: half of the unit's columns
       const int row = tm * (BM * CG) + rank * (kPair ? BM : 0) + quarter * 32 + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       auto wait_acc = [&]() {
@@ -847,18 +879,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (aborted) break;
       } else if (EPI == EPI_FOLD) {
         bool aborted = false;
-        bad |= epi_fold(p, taddr, row, tn * BN, half, &ctl->xch[quarter][0][0], &ctl->xbar[quarter], abort_flag,
+        bad |= epi_fold(p, taddr, row, u.col0, half, nch, &ctl->xch[quarter][0][0], &ctl->xbar[quarter], abort_flag,
                         wait_acc, &aborted, rx);
         if (aborted) break;
       } else {
         if (!wait_acc()) break;
         if (EPI == EPI_STORE) {
-          epi_store(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
+          epi_store(p, taddr, row, u.col0, nch * half, nch * half + nch);
         } else if (EPI == EPI_RESID) {
-          double part = epi_resid(p, taddr, row, tn * BN, 4 * half, 4 * half + 4);
+          double part = epi_resid(p, taddr, row, u.col0, nch * half, nch * half + nch);
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, off);
-          if (lane == 0) p.partial[(static_cast<size_t>(t) * CG + (kPair ? rank : 0)) * kEpiWarps + half * 4 + quarter] = part;
+          // two partial slots per tile and warp, one per half: a whole tile fills the first
+          // and zeroes the second, so every slot is written once whatever the split
+          if (lane == 0) {
+            const size_t slot = ((static_cast<size_t>(u.tile) * 2 + u.part) * CG + (kPair ? rank : 0)) * kEpiWarps +
+                                half * 4 + quarter;
+            p.partial[slot] = part;
+            if (u.wide) p.partial[slot + static_cast<size_t>(CG) * kEpiWarps] = 0.0;
+          }
         } else if (EPI == EPI_SWIGLU_FWD) {
           epi_swiglu_fwd(p, taddr, row, tn * (BN / 2), 2 * half, 2 * half + 2);
         } else if (EPI == EPI_SWIGLU_BWD) {
@@ -918,15 +957,18 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
     if (e != cudaSuccess) return e;
     e = make_tmap(&tmB2, B2, p.N, p.K, BN / 2);
   } else {
-    // a pair's CTA loads half of the tile's B columns
+    // a pair's CTA loads half of the unit's B columns: BN / CG rows of a K-major B for a
+    // whole tile (tmB), half of that for a half-width unit (tmB2); MN-major B in 64-column boxes
     e = B_MN ? make_tmap(&tmB, B, p.K, p.N, 64, ldb) : make_tmap(&tmB, B, p.N, p.K, BN / CG, ldb);
     tmB2 = tmB;
+    if (e == cudaSuccess && !B_MN && CG == 2) e = make_tmap(&tmB2, B, p.N, p.K, BN / (2 * CG), ldb);
   }
   if (e != cudaSuccess) return e;
   p.tiles_m = (p.M + BM * CG - 1) / (BM * CG);
   p.tiles_n = EPI == EPI_SWIGLU_FWD ? (p.N + BN / 2 - 1) / (BN / 2) : (p.N + BN - 1) / BN;
   p.num_kb = (p.K + BK - 1) / BK;
   p.num_units = p.tiles_m * p.tiles_n;
+  p.full_units = p.num_units;
   // raster order
   {
     const double b_bytes = static_cast<double>(p.N) * p.K * 2 * (EPI == EPI_SWIGLU_FWD ? 2 : 1);
@@ -960,7 +1002,20 @@ cudaError_t run(const uint16_t* A, const uint16_t* B, Params p, cudaStream_t str
   e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
   if (e != cudaSuccess) return e;
   if (max_clusters < 1) return cudaErrorInvalidConfiguration;
-  const int clusters = tiles < max_clusters ? tiles : max_clusters;
+  // A last wave of rem < clusters whole tiles leaves clusters idle while it runs: when its
+  // tiles split in two fit one wave (2 rem <= clusters), they run as half-width units (same
+  // rows, BN / 2 columns each), so that wave takes about half a tile's time.  Tcgen05 pair
+  // tiles of the store, residual and fold epilogues only, with whole column tiles, and for
+  // the fold groups no wider than the half unit.
+  if (CG == 2 && KSPLIT == 1 && p.N % BN == 0 &&
+      (EPI == EPI_STORE || EPI == EPI_RESID || (EPI == EPI_FOLD && p.fold.group_size <= BN / 2))) {
+    const int rem = tiles % max_clusters;
+    if (rem > 0 && 2 * rem <= max_clusters) {
+      p.full_units = tiles - rem;
+      p.num_units = tiles + rem;
+    }
+  }
+  const int clusters = p.num_units < max_clusters ? p.num_units : max_clusters;
   cfg.gridDim = dim3(2 * clusters);
   LaunchScope scope(stream, name);
   e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmB2, p);
@@ -1017,11 +1072,11 @@ cudaError_t make_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, uint32_t el
 }
 
 // The residual, reference-forward, plain and (unsplit) weight-gradient GEMMs run
-// as CTA pairs on 256 x 256 tiles; each CTA's eight epilogue warps write one
-// loss partial per tile.
+// as CTA pairs on 256 x 256 tiles; each CTA's eight epilogue warps write two
+// loss partials per tile (one per half-width unit; a whole tile zeroes the second).
 constexpr int kPairCG = 2;
 int resid_partials(int M, int N) {
-  return ((M + BM * kPairCG - 1) / (BM * kPairCG)) * ((N + BN - 1) / BN) * kPairCG * kEpiWarps;
+  return ((M + BM * kPairCG - 1) / (BM * kPairCG)) * ((N + BN - 1) / BN) * 2 * kPairCG * kEpiWarps;
 }
 
 cudaError_t launch_gemm_store(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,

@@ -128,6 +128,8 @@ cudaError_t launch_gemm_store_bf16_kmn(const uint16_t* A, const uint16_t* B_kn, 
 // causal attention per sample and head over qkv [S*L][3H] (Q, K rotated; V): O [S*L][H] bf16, lse [S][nh][L]
 cudaError_t launch_attn_fwd(const uint16_t* qkv, int S, int L, int H, int head_dim, uint16_t* out, float* lse,
                             cudaStream_t st);
+// the same on tcgen05 for head dimension 128 and L % 128 == 0 (cudaErrorNotSupported otherwise)
+cudaError_t launch_attn_fwd_tc(const uint16_t* qkv, int S, int L, int H, uint16_t* out, float* lse, cudaStream_t st);
 // its backward from dO: dqkv [S*L][3H] bf16 (dQ, dK with the inverse rotation applied; dV); Dsum [S][nh][L] scratch
 cudaError_t launch_attn_bwd(const uint16_t* qkv, const uint16_t* O, const uint16_t* dO, const float* lse,
                             float* Dsum, const float* rope_cs, int S, int L, int H, int head_dim, uint16_t* dqkv,

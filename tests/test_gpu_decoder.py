@@ -105,7 +105,8 @@ def _qkv_problem(S, L, H, seed):
     return qkv
 
 
-@pytest.mark.parametrize("S,L,H,nh", [(2, 128, 256, 2), (1, 192, 128, 2), (1, 64, 256, 4)])
+@pytest.mark.parametrize("S,L,H,nh", [(2, 128, 256, 2), (1, 192, 128, 2), (1, 64, 256, 4), (2, 384, 256, 2),
+                                      (1, 512, 512, 4)])
 def test_attention_forward_and_backward_match_oracle(ar, S, L, H, nh):
     qkv = _qkv_problem(S, L, H, seed=S + L + H)
     d = H // nh
@@ -114,7 +115,9 @@ def test_attention_forward_and_backward_match_oracle(ar, S, L, H, nh):
     lse = torch.empty((S, nh, L), device="cuda")
     ar.ar_attention_forward(qd, S, L, nh, out, lse)
     assert ar.ar_get_device_status() == 0
-    assert ("attn_fwd_kernel<d%d>" % d) in ar.ar_last_kernels()
+    # head dimension 128 on whole 128-row blocks: the tcgen05 forward; else mma.sync
+    fwd = "attn_fwd_tc_kernel<d128>" if d == 128 and L % 128 == 0 else "attn_fwd_kernel<d%d>" % d
+    assert fwd in ar.ar_last_kernels()
     Qr, Kr, V = (qkv[:, i * H:(i + 1) * H].reshape(S, L, H) for i in range(3))
     O_ref, P, lse_ref = O.attention_forward(Qr, Kr, V, nh, rounding=True)
     assert rel_l2(as_f64(out), O_ref.reshape(S * L, H)) <= ATTN_RTOL
