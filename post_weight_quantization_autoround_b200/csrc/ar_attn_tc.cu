@@ -1,10 +1,12 @@
 // Causal softmax attention forward of the decoder block on the fifth-generation
 // tensor cores (tcgen05 + TMEM + TMA), head dimension 128, sample lengths a
-// multiple of 128.  Same arithmetic as the mma.sync kernel of ar_decoder.cu:
-// z = fl(s * scale) with s = q . k (fp32 accumulation of bf16 products), lse the
-// row's log-sum-exp over its keys (pass 1), then P = bf16(exp(z - lse)) and
-// O = P V (pass 2), so a probability's rounding does not depend on the order in
-// which keys are visited.
+// multiple of 128.  The mma.sync kernel's method (ar_decoder.cu): z = s * scale
+// with s = q . k (fp32 accumulation of bf16 products), lse the row's log-sum-exp
+// over its keys (pass 1), then P = bf16(exp(z - lse)) and O = P V (pass 2), so a
+// probability's rounding does not depend on the order in which keys are
+// visited.  Here every exp(z - a) is 2^(s scale log2 e - a log2 e) by the
+// hardware's base-2 exponential after one fused multiply-add: a few fp32 ulp
+// from the exact value, far below the bf16 rounding of P.
 //
 // [AR] §3 "Why Block-Wise Optimization" and "Algorithm Flow": the decoder block
 // is the unit of tuning, its output's error reaches every weight through
@@ -35,7 +37,7 @@
 // Every mbarrier wait is bounded (ar_device.cuh): on a timeout the kernel
 // raises the abort flag and the sticky device status, every role leaves its
 // loop, in-flight copies and MMAs are drained and TMEM is freed.
-#include "ar_internal.h"
+#include "ar_attn_tc.cuh"
 
 namespace ar {
 namespace {
@@ -72,37 +74,6 @@ struct AtCtl {
 
 constexpr int kAtSmem = kAtTile * (1 + kAtKStages + kAtVStages) + static_cast<int>(sizeof(AtCtl)) + 1024;
 static_assert(kAtSmem <= 227 * 1024, "shared memory per CTA");
-
-// D[tmem] (+)= A[tmem] x B[smem]^T (kind::f16, bf16 in, fp32 accumulate); A is
-// 128 lanes x 8 columns of bf16 pairs per K = 16 step.
-__device__ __forceinline__ void at_mma_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// 32 lanes x 32 columns of 32-bit values into TMEM (this warp's lane quarter).
-__device__ __forceinline__ void at_tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-__device__ __forceinline__ void at_tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ void at_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
 
 // K-major operand of 128 rows x 128 columns (two 64-column swizzled boxes): the
 // descriptor of K = 16 step kk (32 bytes inside a swizzle row, box kk / 4).
@@ -259,33 +230,43 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     const int k0 = hh * 64;               // first key column of this warp's half
     uint32_t ns = 0;
     bool ok = true;
-    // pass 1: running (max, sum of exp(z - max)) over this half's keys
+    // Exponentials as 2^x with the hardware ex2: exp(z - a) = 2^(s c2 - a log2 e),
+    // c2 = scale log2 e, one fused multiply-add per score (a few fp32 ulp from
+    // exp(fl(s scale) - a), far below the bf16 rounding of P).  The row maximum is
+    // taken over the raw scores (scale > 0).  Only the diagonal block is masked.
+    const float c2 = scale * 1.4426950408889634f;
+    // pass 1: running (max, sum of exp(scale (s - max))) over this half's keys
     float m = -INFINITY, l = 0.f;
     for (int j = 0; ok && j < n_kb; ++j, ++ns) {
       const uint32_t buf = ns & 1u;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->s_full[buf], (ns >> 1) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float v0[32], v1[32];
-      tmem_ld32(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v0);
-      tmem_ld32(tmem + lane_off + kAtColS + buf * kAtBlk + k0 + 32, v1);
+      float v[64];
+      at_ld64(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->s_empty[buf]);
-      const bool diag = j == qb;
-      float mx = -INFINITY;
+      if (j == qb) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        v0[i] = (diag && k0 + i > r) ? -INFINITY : __fmul_rn(v0[i], scale);
-        v1[i] = (diag && k0 + 32 + i > r) ? -INFINITY : __fmul_rn(v1[i], scale);
-        mx = fmaxf(mx, fmaxf(v0[i], v1[i]));
+        for (int i = 0; i < 64; ++i) v[i] = k0 + i > r ? -INFINITY : v[i];
       }
-      const float mn = fmaxf(m, mx);
-      if (mn != -INFINITY) {  // else every key of the half so far is masked: nothing to add
-        float t = 0.f;
+      float mx0 = v[0], mx1 = v[1];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) t += __expf(v0[i] - mn) + __expf(v1[i] - mn);
-        l = l * __expf(m - mn) + t;
+      for (int i = 2; i < 64; i += 2) {
+        mx0 = fmaxf(mx0, v[i]);
+        mx1 = fmaxf(mx1, v[i + 1]);
+      }
+      const float mn = fmaxf(m, fmaxf(mx0, mx1));
+      if (mn != -INFINITY) {  // else every key of the half so far is masked: nothing to add
+        const float off = mn * c2;
+        float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          t0 += at_ex2(fmaf(v[i], c2, -off));
+          t1 += at_ex2(fmaf(v[i + 1], c2, -off));
+        }
+        l = l * at_ex2((m - mn) * c2) + (t0 + t1);
         m = mn;
       }
     }
@@ -296,7 +277,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     const float2 a0 = ctl->ml[quarter][0][lane];
     const float2 a1 = ctl->ml[quarter][1][lane];
     const float mm = fmaxf(a0.x, a1.x);
-    const float lse = mm + logf(a0.y * __expf(a0.x - mm) + a1.y * __expf(a1.x - mm));
+    const float lsum = a0.y * at_ex2((a0.x - mm) * c2) + a1.y * at_ex2((a1.x - mm) * c2);
+    const float lse = __fmul_rn(mm, scale) + logf(lsum);
+    const float lse2 = lse * 1.4426950408889634f;
     ok = ok && *abort_flag == 0;
     // pass 2: P = bf16(exp(z - lse)) into a P buffer, read there by the P V MMAs
     for (int j = 0; ok && j < n_kb; ++j, ++ns) {
@@ -304,23 +287,23 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->s_full[buf], (ns >> 1) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float v0[32], v1[32];
-      tmem_ld32(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v0);
-      tmem_ld32(tmem + lane_off + kAtColS + buf * kAtBlk + k0 + 32, v1);
+      float v[64];
+      at_ld64(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->s_empty[buf]);
-      const bool diag = j == qb;
       uint32_t pk[32];
+      if (j == qb) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int ka = k0 + 2 * i;
-        const float p0 = (diag && ka > r) ? 0.f : __expf(__fmul_rn(v0[2 * i], scale) - lse);
-        const float p1 = (diag && ka + 1 > r) ? 0.f : __expf(__fmul_rn(v0[2 * i + 1], scale) - lse);
-        const float p2 = (diag && ka + 32 > r) ? 0.f : __expf(__fmul_rn(v1[2 * i], scale) - lse);
-        const float p3 = (diag && ka + 33 > r) ? 0.f : __expf(__fmul_rn(v1[2 * i + 1], scale) - lse);
-        pk[i] = pack_bf16x2(p0, p1);
-        pk[16 + i] = pack_bf16x2(p2, p3);
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = k0 + 2 * i > r ? 0.f : at_ex2(fmaf(v[2 * i], c2, -lse2));
+          const float p1 = k0 + 2 * i + 1 > r ? 0.f : at_ex2(fmaf(v[2 * i + 1], c2, -lse2));
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          pk[i] = pack_bf16x2(at_ex2(fmaf(v[2 * i], c2, -lse2)), at_ex2(fmaf(v[2 * i + 1], c2, -lse2)));
       }
       const uint32_t pbuf = static_cast<uint32_t>(j) & 1u;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->p_empty[pbuf], ((static_cast<uint32_t>(j) >> 1) & 1u) ^ 1u,

@@ -27,9 +27,9 @@
 // The attention kernels here run on mma.sync m16n8k16 (bf16, fp32 accumulation)
 // over 64-row tiles staged in shared memory with cp.async (double-buffered,
 // 16-byte row padding so that ldmatrix reads are free of bank conflicts); the
-// forward at head dimension 128 on whole 128-row blocks runs on tcgen05 instead
-// (ar_attn_tc.cu).  No kernel here waits on another CTA: every wait is a
-// cp.async group wait or a CTA barrier.
+// forward and backward at head dimension 128 on whole 128-row blocks run on
+// tcgen05 instead (ar_attn_tc.cu, ar_attn_bwd_tc.cu).  No kernel here waits on
+// another CTA: every wait is a cp.async group wait or a CTA barrier.
 #include "ar_internal.h"
 
 namespace ar {
@@ -675,19 +675,23 @@ cudaError_t attn_fwd_launch(const uint16_t* qkv, int S, int L, int H, uint16_t* 
   return cudaGetLastError();
 }
 
+// D[s][h][t] = rowsum(dO * O) over each head's columns
+cudaError_t attn_bwd_prep(const uint16_t* O, const uint16_t* dO, int S, int L, int H, int D, float* Dsum,
+                          cudaStream_t st) {
+  const int nh = H / D;
+  const int64_t M = static_cast<int64_t>(S) * L;
+  const int64_t warps = M * nh;
+  LaunchScope scope(st, "attn_bwd_prep_kernel");
+  attn_bwd_prep_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(dO, O, M, H, L, nh, D, Dsum);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t attn_bwd_launch(const uint16_t* qkv, const uint16_t* O, const uint16_t* dO, const float* lse,
                             float* Dsum, const float2* cs, int S, int L, int H, uint16_t* dqkv, cudaStream_t st) {
   const int nh = H / D;
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
-  const int64_t M = static_cast<int64_t>(S) * L;
-  {
-    const int64_t warps = M * nh;
-    LaunchScope scope(st, "attn_bwd_prep_kernel");
-    attn_bwd_prep_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(dO, O, M, H, L, nh, D,
-                                                                                          Dsum);
-  }
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = attn_bwd_prep(O, dO, S, L, H, D, Dsum, st);
   if (e != cudaSuccess) return e;
   const int smem_dq = 6 * Tile<D>::kBytes;
   e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq);
@@ -725,6 +729,11 @@ cudaError_t launch_attn_bwd(const uint16_t* qkv, const uint16_t* O, const uint16
                             float* Dsum, const float* rope_cs, int S, int L, int H, int head_dim, uint16_t* dqkv,
                             cudaStream_t st) {
   const float2* cs = reinterpret_cast<const float2*>(rope_cs);
+  if (head_dim == 128 && L % 128 == 0) {  // the tcgen05 kernels (ar_attn_bwd_tc.cu)
+    const cudaError_t e = attn_bwd_prep(O, dO, S, L, H, head_dim, Dsum, st);
+    if (e != cudaSuccess) return e;
+    return launch_attn_bwd_tc(qkv, dO, lse, Dsum, rope_cs, S, L, H, dqkv, st);
+  }
   if (head_dim == 128) return attn_bwd_launch<128>(qkv, O, dO, lse, Dsum, cs, S, L, H, dqkv, st);
   if (head_dim == 64) return attn_bwd_launch<64>(qkv, O, dO, lse, Dsum, cs, S, L, H, dqkv, st);
   return cudaErrorInvalidValue;

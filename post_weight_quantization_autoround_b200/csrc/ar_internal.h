@@ -130,6 +130,9 @@ cudaError_t launch_attn_fwd(const uint16_t* qkv, int S, int L, int H, int head_d
                             cudaStream_t st);
 // the same on tcgen05 for head dimension 128 and L % 128 == 0 (cudaErrorNotSupported otherwise)
 cudaError_t launch_attn_fwd_tc(const uint16_t* qkv, int S, int L, int H, uint16_t* out, float* lse, cudaStream_t st);
+// the dQ, dK, dV kernels on tcgen05 for head dimension 128 and L % 128 == 0, Dsum already = rowsum(dO O)
+cudaError_t launch_attn_bwd_tc(const uint16_t* qkv, const uint16_t* dO, const float* lse, const float* Dsum,
+                               const float* rope_cs, int S, int L, int H, uint16_t* dqkv, cudaStream_t st);
 // its backward from dO: dqkv [S*L][3H] bf16 (dQ, dK with the inverse rotation applied; dV); Dsum [S][nh][L] scratch
 cudaError_t launch_attn_bwd(const uint16_t* qkv, const uint16_t* O, const uint16_t* dO, const float* lse,
                             float* Dsum, const float* rope_cs, int S, int L, int H, int head_dim, uint16_t* dqkv,

@@ -130,6 +130,8 @@ def test_attention_forward_and_backward_match_oracle(ar, S, L, H, nh):
     dqkv = torch.full((S * L, 3 * H), float("nan"), dtype=torch.bfloat16, device="cuda")
     ar.ar_attention_backward(qd, out, dOd, lse, S, L, nh, dqkv, ws)
     assert ar.ar_get_device_status() == 0
+    bwd = "attn_bwd_dkdv_tc_kernel<d128>" if d == 128 and L % 128 == 0 else "attn_bwd_dkdv_kernel<d%d>" % d
+    assert bwd in ar.ar_last_kernels()
     O_gpu = as_f64(out).reshape(S, L, H)
     dQr, dKr, dV = O.attention_backward(Qr, Kr, V, P, dO.reshape(S, L, H), nh, rounding=True, O=O_gpu)
     dQ = rb(O.rope(dQr, nh, -1.0, rounding=True))
@@ -257,7 +259,8 @@ def test_decoder_step_matches_oracle(ar, S, L, H, F, nh, g, bits, spread):
     ocfg = O.QConfig(bits=bits, group_size=g)
     gd = GpuDecoder(ar, d, S, L, nh, states, cfg, 1)
     out = gd.step(1, grads=True)
-    assert "attn_bwd_dkdv_kernel" in ar.ar_last_kernels() and "qkv_rope" in ar.ar_last_kernels()
+    bwd = "attn_bwd_dkdv_tc_kernel" if H // nh == 128 and L % 128 == 0 else "attn_bwd_dkdv_kernel"
+    assert bwd in ar.ar_last_kernels() and "qkv_rope" in ar.ar_last_kernels()
     Xs = X.reshape(S, L, H)
     Y = O.decoder_forward(Xs, Ws, gammas, nh, rounding=True)["Y"].astype(np.float32)  # the oracle's own reference
     L_ref, new, grads = O.tune_step_decoder(Ws, Xs, Y, states, gammas, nh, ocfg, rounding=True)
