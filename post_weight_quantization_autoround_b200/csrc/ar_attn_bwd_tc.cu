@@ -119,7 +119,8 @@ __device__ __forceinline__ void bw_mma(BwCtl* ctl, uint32_t tmem, const uint8_t*
                                        const uint8_t* ring, int n, volatile int* abort_flag) {
   constexpr uint32_t idesc_st = idesc_bf16_f32(kBwRows, kBwCols, false, false);
   constexpr uint32_t idesc_acc = idesc_bf16_f32(kBwRows, kBwD, false, true);
-  const uint32_t a1 = smem_u32(resA), a2 = smem_u32(resB);
+  // descriptors built once per tile; each K = 16 step adds a compile-time offset
+  const uint64_t a1 = sdesc_sw128(smem_u32(resA), 16, 1024), a2 = sdesc_sw128(smem_u32(resB), 16, 1024);
   bool ok = mbar_wait(&ctl->res_full, 0, abort_flag);
   tc_fence_after();
   for (int it = 0; ok && it <= n; ++it) {
@@ -132,16 +133,19 @@ __device__ __forceinline__ void bw_mma(BwCtl* ctl, uint32_t tmem, const uint8_t*
         break;
       }
       tc_fence_after();
-      const uint32_t x = smem_u32(ring + slot * 2 * kBwSmall);
-      const uint32_t y = x + kBwSmall;
+      const uint32_t xs = smem_u32(ring + slot * 2 * kBwSmall);
+      const uint64_t x = sdesc_sw128(xs, 16, 1024), y = sdesc_sw128(xs + kBwSmall, 16, 1024);
+      // K-major steps: 32 bytes inside a 128-byte swizzle row, the second 64-column box from kk = 4
+      // on; the S and dP accumulations alternate step by step (two independent chains)
 #pragma unroll
-      for (int kk = 0; kk < kBwD / 16; ++kk)
-        umma_bf16(tmem + kBwColS + buf * kBwCols, at_desc_kmaj(a1, kBwRows, kk), at_desc_kmaj(x, kBwCols, kk),
-                  idesc_st, kk > 0 ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < kBwD / 16; ++kk)
-        umma_bf16(tmem + kBwColDP + buf * kBwCols, at_desc_kmaj(a2, kBwRows, kk), at_desc_kmaj(y, kBwCols, kk),
-                  idesc_st, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < kBwD / 16; ++kk) {
+        const uint32_t oa = (kk >> 2) * kBwRows * 128 + (kk & 3) * 32;
+        const uint32_t ob = (kk >> 2) * kBwCols * 128 + (kk & 3) * 32;
+        umma_bf16(tmem + kBwColS + buf * kBwCols, at_desc_add(a1, oa), at_desc_add(x, ob), idesc_st,
+                  kk > 0 ? 1u : 0u);
+        umma_bf16(tmem + kBwColDP + buf * kBwCols, at_desc_add(a2, oa), at_desc_add(y, ob), idesc_st,
+                  kk > 0 ? 1u : 0u);
+      }
       umma_commit(&ctl->st_full[buf]);
     }
     if (it > 0) {
@@ -153,18 +157,20 @@ __device__ __forceinline__ void bw_mma(BwCtl* ctl, uint32_t tmem, const uint8_t*
         break;
       }
       tc_fence_after();
-      const uint32_t x = smem_u32(ring + pslot * 2 * kBwSmall);
-      const uint32_t y = x + kBwSmall;
+      // MN-major views of the streamed tiles (64 rows x 128 columns as two 64-column boxes):
+      // 64-column chunks one box apart, 8-row groups 1 KiB apart, a K = 16 step 2 KiB
+      const uint32_t xs = smem_u32(ring + pslot * 2 * kBwSmall);
+      const uint64_t x = sdesc_sw128(xs, kBwCols * 128, 1024), y = sdesc_sw128(xs + kBwSmall, kBwCols * 128, 1024);
 #pragma unroll
       for (int kk = 0; kk < kBwCols / 16; ++kk) {
         // streamed rows 16 kk .. 16 kk + 15: written by warp half kk / 2, pair columns 8 (kk % 2) on
         const uint32_t col = pbuf * kBwCols + 32 * (kk >> 1) + 8 * (kk & 1);
         const uint32_t acc = (p > 0 || kk > 0) ? 1u : 0u;
         if (DKDV) {
-          at_mma_ta(tmem + kBwColAcc, tmem + kBwColS + col, at_desc_mnmaj(y, kBwCols, kk), idesc_acc, acc);
-          at_mma_ta(tmem + kBwColAcc + kBwD, tmem + kBwColDP + col, at_desc_mnmaj(x, kBwCols, kk), idesc_acc, acc);
+          at_mma_ta(tmem + kBwColAcc, tmem + kBwColS + col, at_desc_add(y, kk * 2048), idesc_acc, acc);
+          at_mma_ta(tmem + kBwColAcc + kBwD, tmem + kBwColDP + col, at_desc_add(x, kk * 2048), idesc_acc, acc);
         } else {
-          at_mma_ta(tmem + kBwColAcc, tmem + kBwColDP + col, at_desc_mnmaj(x, kBwCols, kk), idesc_acc, acc);
+          at_mma_ta(tmem + kBwColAcc, tmem + kBwColDP + col, at_desc_add(x, kk * 2048), idesc_acc, acc);
         }
       }
       umma_commit(&ctl->st_empty[pbuf]);
@@ -198,8 +204,7 @@ __device__ __forceinline__ bool bw_store32(uint16_t* dst, const float (&v)[32]) 
 __device__ __forceinline__ bool bw_store_rope(uint32_t taddr, int half, int t, const float2* __restrict__ cs,
                                               uint16_t* dst) {
   float x1[32], x2[32];
-  tmem_ld32(taddr + 32 * half, x1);
-  tmem_ld32(taddr + 64 + 32 * half, x2);
+  at_ld32x2(taddr + 32 * half, x1, taddr + 64 + 32 * half, x2);
   const float4* c4 = reinterpret_cast<const float4*>(cs + static_cast<size_t>(t) * (kBwD / 2) + 32 * half);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -260,8 +265,7 @@ __device__ __forceinline__ bool bw_elementwise(BwCtl* ctl, uint32_t tmem, uint32
     const uint32_t cs = kBwColS + buf * kBwCols + 32 * half;
     const uint32_t cd = kBwColDP + buf * kBwCols + 32 * half;
     float sv[32], dpv[32];
-    tmem_ld32(tmem + lane_off + cs, sv);
-    tmem_ld32(tmem + lane_off + cd, dpv);
+    at_ld32x2(tmem + lane_off + cs, sv, tmem + lane_off + cd, dpv);
     uint32_t pp[16], dd[16];
     // causal: a query sees the keys at or before its position; only the two blocks
     // that overlap the diagonal hold masked entries

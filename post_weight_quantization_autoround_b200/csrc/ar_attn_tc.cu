@@ -75,18 +75,13 @@ struct AtCtl {
 constexpr int kAtSmem = kAtTile * (1 + kAtKStages + kAtVStages) + static_cast<int>(sizeof(AtCtl)) + 1024;
 static_assert(kAtSmem <= 227 * 1024, "shared memory per CTA");
 
-// K-major operand of 128 rows x 128 columns (two 64-column swizzled boxes): the
-// descriptor of K = 16 step kk (32 bytes inside a swizzle row, box kk / 4).
-__device__ __forceinline__ uint64_t at_desc_k(uint32_t tile, int kk) {
-  return sdesc_sw128(tile + (kk >> 2) * kAtBox + (kk & 3) * 32, 16, 1024);
-}
-
-// V as the MN-major B operand (N = head columns, K = keys): 64-column chunks are
-// the two boxes (16 KiB apart), 8-key row groups 1 KiB apart, K = 16 step kk
-// 16 rows = 2 KiB further.
-__device__ __forceinline__ uint64_t at_desc_v(uint32_t tile, int kk) {
-  return sdesc_sw128(tile + kk * 2048, kAtBox, 1024);
-}
+// Operand layouts (descriptor offsets per K = 16 step kk, added to a descriptor
+// built once per tile with at_desc_add):
+//  * Q and K, K-major 128 rows x 128 columns as two 64-column swizzled boxes:
+//    32 bytes inside a 128-byte swizzle row, box kk / 4 (16 KiB further);
+//  * V as the MN-major B operand (N = head columns, K = keys): 64-column chunks
+//    are the two boxes (leading offset 16 KiB), 8-key row groups 1 KiB apart,
+//    step kk 16 rows = 2 KiB further.
 
 __global__ void __launch_bounds__(kAtThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, int H, int L, int nh, float scale,
@@ -174,7 +169,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kAtBlk, kAtBlk, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kAtBlk, kAtD, false, true);
-      const uint32_t q_base = smem_u32(sQ);
+      const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);  // K = 16 steps: compile-time offsets
       uint32_t ki = 0, ns = 0;
       bool ok = mbar_wait(&ctl->q_full, 0, abort_flag);
       tc_fence_after();
@@ -185,11 +180,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (!mbar_wait(&ctl->k_full[slot], (ki / kAtKStages) & 1u, abort_flag)) return false;
         if (!mbar_wait(&ctl->s_empty[buf], ((ns >> 1) & 1u) ^ 1u, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + slot * kAtTile);
+        const uint64_t k_desc = sdesc_sw128(smem_u32(sK + slot * kAtTile), 16, 1024);
         const uint32_t d = tmem + kAtColS + buf * kAtBlk;
 #pragma unroll
-        for (int kk = 0; kk < kAtD / 16; ++kk)
-          umma_bf16(d, at_desc_k(q_base, kk), at_desc_k(k_base, kk), idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kAtD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kAtBox + (kk & 3) * 32;
+          umma_bf16(d, at_desc_add(q_desc, off), at_desc_add(k_desc, off), idesc_s, kk > 0 ? 1u : 0u);
+        }
         umma_commit(&ctl->s_full[buf]);
         umma_commit(&ctl->k_empty[slot]);
         ++ki;
@@ -208,10 +205,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t v_base = smem_u32(sV + vslot * kAtTile);
+        const uint64_t v_desc = sdesc_sw128(smem_u32(sV + vslot * kAtTile), kAtBox, 1024);
 #pragma unroll
         for (int kk = 0; kk < kAtBlk / 16; ++kk)
-          at_mma_ta(tmem + kAtColO, tmem + kAtColP + pbuf * 64 + 8 * kk, at_desc_v(v_base, kk), idesc_o,
+          at_mma_ta(tmem + kAtColO, tmem + kAtColP + pbuf * 64 + 8 * kk, at_desc_add(v_desc, kk * 2048), idesc_o,
                     (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&ctl->p_empty[pbuf]);
         umma_commit(&ctl->v_empty[vslot]);

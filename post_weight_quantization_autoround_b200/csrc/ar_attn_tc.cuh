@@ -48,19 +48,6 @@ static __device__ __forceinline__ void at_tmem_st16(uint32_t taddr, const uint32
       : "memory");
 }
 
-// Operand descriptors of a tile of `rows` rows x 128 bf16 columns stored as two
-// 64-column boxes (rows x 128 bytes each, 128-byte swizzle), K = 16 step kk.
-// K-major (the 128 columns are the reduction): 32 bytes inside a swizzle row,
-// the second box from kk = 4 on.
-static __device__ __forceinline__ uint64_t at_desc_kmaj(uint32_t tile, int rows, int kk) {
-  return sdesc_sw128(tile + (kk >> 2) * rows * 128 + (kk & 3) * 32, 16, 1024);
-}
-// MN-major (the rows are the reduction, the 128 columns the MMA's N): 64-column
-// chunks one box apart, 8-row groups 1 KiB apart, a K = 16 step 16 rows further.
-static __device__ __forceinline__ uint64_t at_desc_mnmaj(uint32_t tile, int rows, int kk) {
-  return sdesc_sw128(tile + kk * 2048, rows * 128, 1024);
-}
-
 // 32 lanes x 64 columns of fp32 from TMEM (this warp's lane quarter), waited.
 static __device__ __forceinline__ void at_ld64(uint32_t taddr, float (&v)[64]) {
   uint32_t r[64];
@@ -74,12 +61,35 @@ static __device__ __forceinline__ void at_ld64(uint32_t taddr, float (&v)[64]) {
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two 32-column slices of fp32 from TMEM (this warp's lane quarter) with one wait
+// for both loads.
+static __device__ __forceinline__ void at_ld32x2(uint32_t ta, float (&va)[32], uint32_t tb, float (&vb)[32]) {
+  uint32_t a[32], b[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]), "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]), "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
+      : "r"(ta), "r"(tb)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    va[i] = __uint_as_float(a[i]);
+    vb[i] = __uint_as_float(b[i]);
+  }
+}
+
 // 2^x by the hardware's approximate base-2 exponential (2^-inf = +0).
 static __device__ __forceinline__ float at_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// A shared-memory descriptor moved by `off` bytes (a multiple of 16): the start
+// address sits in the low 14 bits as address / 16, and shared memory lies below
+// 256 KiB, so the move is one add that never carries out of the field.
+static __device__ __forceinline__ uint64_t at_desc_add(uint64_t d, uint32_t off) { return d + (off >> 4); }
 
 static __device__ __forceinline__ float at_round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
