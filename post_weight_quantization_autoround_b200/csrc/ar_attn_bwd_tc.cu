@@ -43,19 +43,21 @@ constexpr int kBwBig = kBwRows * kBwD * 2;  // 32 KiB: a resident 128 x 128 tile
 constexpr int kBwSmall = kBwCols * kBwD * 2;  // 16 KiB: a streamed 64 x 128 tile
 constexpr int kBwStages = 3;
 constexpr int kBwSmWarps = 8;
-constexpr int kBwThreads = (2 + kBwSmWarps) * 32;
+constexpr int kBwDpWarp = 2 + kBwSmWarps;          // the second MMA-issuing warp (the dP chain)
+constexpr int kBwThreads = (3 + kBwSmWarps) * 32;
 constexpr uint32_t kBwColS = 0, kBwColDP = 128, kBwColAcc = 256;
 constexpr uint32_t kBwTmemCols = 512;
 
 struct BwCtl {
   uint64_t res_full;              // resident tiles landed
   uint64_t full[kBwStages];       // streamed pair landed
-  uint64_t empty[kBwStages];      // streamed pair no longer read
-  uint64_t st_full[2];            // MMA: S and dP of the buffer pair written
+  uint64_t empty[kBwStages];      // streamed pair no longer read (one commit from each issuer)
+  uint64_t st_full[2];            // MMA: S and dP of the buffer pair written (one commit from each issuer)
   uint64_t ds_full[2];            // elementwise warps: their bf16 operands written (8 arrivals)
   uint64_t st_empty[2];           // MMA: the accumulating products of the pair done
   uint64_t acc_full;
   uint64_t mma_done;
+  uint64_t mma_done_dp;           // the dP issuer's MMAs all complete
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -67,15 +69,16 @@ __device__ __forceinline__ void bw_init(BwCtl* ctl) {
   mbar_init(&ctl->res_full, 1);
   for (int i = 0; i < kBwStages; ++i) {
     mbar_init(&ctl->full[i], 1);
-    mbar_init(&ctl->empty[i], 1);
+    mbar_init(&ctl->empty[i], 2);
   }
   for (int i = 0; i < 2; ++i) {
-    mbar_init(&ctl->st_full[i], 1);
+    mbar_init(&ctl->st_full[i], 2);
     mbar_init(&ctl->ds_full[i], kBwSmWarps);
     mbar_init(&ctl->st_empty[i], 1);
   }
   mbar_init(&ctl->acc_full, 1);
   mbar_init(&ctl->mma_done, 1);
+  mbar_init(&ctl->mma_done_dp, 1);
   ctl->abort_flag = 0;
   fence_barrier_init();
 }
@@ -120,7 +123,7 @@ __device__ __forceinline__ void bw_mma(BwCtl* ctl, uint32_t tmem, const uint8_t*
   constexpr uint32_t idesc_st = idesc_bf16_f32(kBwRows, kBwCols, false, false);
   constexpr uint32_t idesc_acc = idesc_bf16_f32(kBwRows, kBwD, false, true);
   // descriptors built once per tile; each K = 16 step adds a compile-time offset
-  const uint64_t a1 = sdesc_sw128(smem_u32(resA), 16, 1024), a2 = sdesc_sw128(smem_u32(resB), 16, 1024);
+  const uint64_t a1 = sdesc_sw128(smem_u32(resA), 16, 1024);
   bool ok = mbar_wait(&ctl->res_full, 0, abort_flag);
   tc_fence_after();
   for (int it = 0; ok && it <= n; ++it) {
@@ -134,16 +137,14 @@ __device__ __forceinline__ void bw_mma(BwCtl* ctl, uint32_t tmem, const uint8_t*
       }
       tc_fence_after();
       const uint32_t xs = smem_u32(ring + slot * 2 * kBwSmall);
-      const uint64_t x = sdesc_sw128(xs, 16, 1024), y = sdesc_sw128(xs + kBwSmall, 16, 1024);
+      const uint64_t x = sdesc_sw128(xs, 16, 1024);
       // K-major steps: 32 bytes inside a 128-byte swizzle row, the second 64-column box from kk = 4
-      // on; the S and dP accumulations alternate step by step (two independent chains)
+      // on (dP's chain is issued by the other MMA thread, bw_mma_dp)
 #pragma unroll
       for (int kk = 0; kk < kBwD / 16; ++kk) {
         const uint32_t oa = (kk >> 2) * kBwRows * 128 + (kk & 3) * 32;
         const uint32_t ob = (kk >> 2) * kBwCols * 128 + (kk & 3) * 32;
         umma_bf16(tmem + kBwColS + buf * kBwCols, at_desc_add(a1, oa), at_desc_add(x, ob), idesc_st,
-                  kk > 0 ? 1u : 0u);
-        umma_bf16(tmem + kBwColDP + buf * kBwCols, at_desc_add(a2, oa), at_desc_add(y, ob), idesc_st,
                   kk > 0 ? 1u : 0u);
       }
       umma_commit(&ctl->st_full[buf]);
@@ -180,6 +181,39 @@ __device__ __forceinline__ void bw_mma(BwCtl* ctl, uint32_t tmem, const uint8_t*
   if (ok) umma_commit(&ctl->acc_full);
   umma_commit(&ctl->mma_done);  // every issued MMA completes before TMEM is released
   mbar_wait_drain(&ctl->mma_done, 0);
+}
+
+// The second MMA thread: dP = A2 Y^T of every block into its buffer, so that the
+// S and dP chains are issued by two threads on two sub-partitions (one thread
+// issuing all of a block's MMAs was the kernel's limit: ~80 cycles per MMA
+// against 48 of tensor work at N = 64).  Commits to st_full and to the ring
+// slot's empty barrier, both of which count one commit from each issuer.
+__device__ __forceinline__ void bw_mma_dp(BwCtl* ctl, uint32_t tmem, const uint8_t* resB, const uint8_t* ring, int n,
+                                          volatile int* abort_flag) {
+  constexpr uint32_t idesc_st = idesc_bf16_f32(kBwRows, kBwCols, false, false);
+  const uint64_t a2 = sdesc_sw128(smem_u32(resB), 16, 1024);
+  bool ok = mbar_wait(&ctl->res_full, 0, abort_flag);
+  tc_fence_after();
+  for (int it = 0; ok && it < n; ++it) {
+    const uint32_t slot = static_cast<uint32_t>(it) % kBwStages;
+    const uint32_t buf = static_cast<uint32_t>(it) & 1u;
+    if (!mbar_wait(&ctl->full[slot], (static_cast<uint32_t>(it) / kBwStages) & 1u, abort_flag) ||
+        !mbar_wait(&ctl->st_empty[buf], ((static_cast<uint32_t>(it) >> 1) & 1u) ^ 1u, abort_flag))
+      break;
+    tc_fence_after();
+    const uint64_t y = sdesc_sw128(smem_u32(ring + slot * 2 * kBwSmall) + kBwSmall, 16, 1024);
+#pragma unroll
+    for (int kk = 0; kk < kBwD / 16; ++kk) {
+      const uint32_t oa = (kk >> 2) * kBwRows * 128 + (kk & 3) * 32;
+      const uint32_t ob = (kk >> 2) * kBwCols * 128 + (kk & 3) * 32;
+      umma_bf16(tmem + kBwColDP + buf * kBwCols, at_desc_add(a2, oa), at_desc_add(y, ob), idesc_st,
+                kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&ctl->st_full[buf]);
+    umma_commit(&ctl->empty[slot]);  // this issuer's reads of the slot (Y) are done with its dP
+  }
+  umma_commit(&ctl->mma_done_dp);  // every issued MMA completes before TMEM is released
+  mbar_wait_drain(&ctl->mma_done_dp, 0);
 }
 
 // 32 fp32 accumulator values of a row -> 32 bf16 at dst (16-byte aligned); returns
@@ -343,6 +377,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                  &tmDO64, h * kBwD, row0 + q0 * kBwCols, n, abort_flag);
   } else if (warp == 1) {
     if (lane == 0) bw_mma<true>(ctl, tmem, sK, sV, ring, n, abort_flag);
+  } else if (warp == kBwDpWarp) {
+    if (lane == 0) bw_mma_dp(ctl, tmem, sV, ring, n, abort_flag);
   } else {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
@@ -434,6 +470,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) bw_mma<false>(ctl, tmem, sQ, sDO, ring, n, abort_flag);
+  } else if (warp == kBwDpWarp) {
+    if (lane == 0) bw_mma_dp(ctl, tmem, sDO, ring, n, abort_flag);
   } else {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
