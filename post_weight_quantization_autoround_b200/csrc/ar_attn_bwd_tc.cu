@@ -19,14 +19,17 @@
 //    S^T = K Q^T and dP^T = V dO^T (N = 64 queries) into one of two buffer
 //    pairs; the softmax warps write P^T and dS^T as bf16 pairs back over the
 //    columns they read; then dV += P^T dO and dK += dS^T Q with those as the A
-//    operand from tensor memory and dO, Q as MN-major B operands.  The MMAs of
-//    the next block's S^T, dP^T are issued before this block's dV, dK.
+//    operand from tensor memory and dO, Q as MN-major B operands.  The next
+//    block's S^T, dP^T run while this block's elementwise work does.
 //  * dQ: one CTA per 128 queries, over the 64-key blocks up to the diagonal:
 //    S = Q K^T, dP = dO V^T, dS written back over dP, dQ += dS K.
-// Warp roles as in the forward: warp 0 TMA producer (the resident operands
-// once, then a 3-deep ring of the streamed pair), warp 1 TMEM owner and MMA
-// issuer, warps 2-9 the elementwise work (two per TMEM lane quarter, one half
-// of each block's 64 columns each) and the epilogue.
+// Warp roles: warp 0 TMA producer (the resident operands once, then a 3-deep
+// ring of the streamed pair); warp 1 TMEM owner and issuer of the S chain;
+// warps 2-17 the elementwise work (four per TMEM lane quarter, 16 of each
+// block's 64 columns each) and the epilogue; warp 18 issuer of the dP chain;
+// warp 19 issuer of the accumulating products.  Three issuing threads on three
+// sub-partitions, because one thread issuing every MMA of a block (20-24 per
+// 64-column block) was the limit.
 // TMEM columns: S buffers 0 and 64, dP buffers 128 and 192, then the fp32
 // accumulators (dV at 256 and dK at 384; dQ at 256).
 #include <type_traits>
@@ -42,22 +45,26 @@ constexpr int kBwCols = 64;                 // streamed queries (dK, dV) or keys
 constexpr int kBwBig = kBwRows * kBwD * 2;  // 32 KiB: a resident 128 x 128 tile
 constexpr int kBwSmall = kBwCols * kBwD * 2;  // 16 KiB: a streamed 64 x 128 tile
 constexpr int kBwStages = 3;
-constexpr int kBwSmWarps = 8;
-constexpr int kBwDpWarp = 2 + kBwSmWarps;          // the second MMA-issuing warp (the dP chain)
-constexpr int kBwThreads = (3 + kBwSmWarps) * 32;
+constexpr int kBwSmWarps = 16;                     // four per TMEM lane quarter
+constexpr int kBwWCols = kBwCols / (kBwSmWarps / 4);  // streamed columns per elementwise warp
+static_assert(kBwWCols == 16, "the elementwise role loads and stores 16-column slices");
+constexpr int kBwDpWarp = 2 + kBwSmWarps;          // MMA issuer of the dP chain
+constexpr int kBwAccWarp = 3 + kBwSmWarps;         // MMA issuer of the accumulating products
+constexpr int kBwThreads = (4 + kBwSmWarps) * 32;
 constexpr uint32_t kBwColS = 0, kBwColDP = 128, kBwColAcc = 256;
 constexpr uint32_t kBwTmemCols = 512;
 
 struct BwCtl {
   uint64_t res_full;              // resident tiles landed
   uint64_t full[kBwStages];       // streamed pair landed
-  uint64_t empty[kBwStages];      // streamed pair no longer read (one commit from each issuer)
+  uint64_t empty[kBwStages];      // streamed pair no longer read (one commit from each of three issuers)
   uint64_t st_full[2];            // MMA: S and dP of the buffer pair written (one commit from each issuer)
   uint64_t ds_full[2];            // elementwise warps: their bf16 operands written (8 arrivals)
   uint64_t st_empty[2];           // MMA: the accumulating products of the pair done
   uint64_t acc_full;
   uint64_t mma_done;
   uint64_t mma_done_dp;           // the dP issuer's MMAs all complete
+  uint64_t mma_done_acc;          // the accumulating issuer's MMAs all complete
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -69,7 +76,7 @@ __device__ __forceinline__ void bw_init(BwCtl* ctl) {
   mbar_init(&ctl->res_full, 1);
   for (int i = 0; i < kBwStages; ++i) {
     mbar_init(&ctl->full[i], 1);
-    mbar_init(&ctl->empty[i], 2);
+    mbar_init(&ctl->empty[i], 3);
   }
   for (int i = 0; i < 2; ++i) {
     mbar_init(&ctl->st_full[i], 2);
@@ -79,6 +86,7 @@ __device__ __forceinline__ void bw_init(BwCtl* ctl) {
   mbar_init(&ctl->acc_full, 1);
   mbar_init(&ctl->mma_done, 1);
   mbar_init(&ctl->mma_done_dp, 1);
+  mbar_init(&ctl->mma_done_acc, 1);
   ctl->abort_flag = 0;
   fence_barrier_init();
 }
@@ -113,85 +121,22 @@ __device__ __forceinline__ void bw_produce(BwCtl* ctl, uint8_t* resA, uint8_t* r
     mbar_wait_drain(&ctl->full[i % kBwStages], (i / kBwStages) & 1u);
 }
 
-// MMA issuer.  Resident A1 (K, or Q for dQ) and A2 (V, or dO); streamed X (Q, or
-// K) and Y (dO, or V) per block.  S = A1 X^T and dP = A2 Y^T into buffer pair
-// it % 2; after the elementwise warps have written their bf16 operands over the
-// pair: DKDV: dV += P^T Y and dK += dS^T X; else dQ += dS X.
-template <bool DKDV>
-__device__ __forceinline__ void bw_mma(BwCtl* ctl, uint32_t tmem, const uint8_t* resA, const uint8_t* resB,
-                                       const uint8_t* ring, int n, volatile int* abort_flag) {
+// Three MMA-issuing threads on three sub-partitions (one thread issuing all of a
+// block's MMAs was the kernel's limit: ~80 cycles per N = 64 MMA against 48 of
+// tensor work).  Resident A1 (K, or Q for dQ) and A2 (V, or dO); streamed X (Q,
+// or K) and Y (dO, or V) per block, in ring slot it % 3; buffer pair it % 2.
+//  * bw_mma_st<false>: S = A1 X^T;  bw_mma_st<true>: dP = A2 Y^T (each commits to
+//    st_full, which counts both, and to the slot's empty barrier);
+//  * bw_mma_acc: after the elementwise warps have written their bf16 operands over
+//    the pair, DKDV: dV += P^T Y and dK += dS^T X; else dQ += dS X; commits
+//    st_empty (the pair may be overwritten) and the slot's empty barrier.
+// Every issuer waits on each phase of its barriers in order.
+template <bool DP>
+__device__ __forceinline__ void bw_mma_st(BwCtl* ctl, uint32_t tmem, const uint8_t* res, const uint8_t* ring, int n,
+                                          uint64_t* done, volatile int* abort_flag) {
   constexpr uint32_t idesc_st = idesc_bf16_f32(kBwRows, kBwCols, false, false);
-  constexpr uint32_t idesc_acc = idesc_bf16_f32(kBwRows, kBwD, false, true);
-  // descriptors built once per tile; each K = 16 step adds a compile-time offset
-  const uint64_t a1 = sdesc_sw128(smem_u32(resA), 16, 1024);
-  bool ok = mbar_wait(&ctl->res_full, 0, abort_flag);
-  tc_fence_after();
-  for (int it = 0; ok && it <= n; ++it) {
-    if (it < n) {
-      const uint32_t slot = static_cast<uint32_t>(it) % kBwStages;
-      const uint32_t buf = static_cast<uint32_t>(it) & 1u;
-      if (!mbar_wait(&ctl->full[slot], (static_cast<uint32_t>(it) / kBwStages) & 1u, abort_flag) ||
-          !mbar_wait(&ctl->st_empty[buf], ((static_cast<uint32_t>(it) >> 1) & 1u) ^ 1u, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t xs = smem_u32(ring + slot * 2 * kBwSmall);
-      const uint64_t x = sdesc_sw128(xs, 16, 1024);
-      // K-major steps: 32 bytes inside a 128-byte swizzle row, the second 64-column box from kk = 4
-      // on (dP's chain is issued by the other MMA thread, bw_mma_dp)
-#pragma unroll
-      for (int kk = 0; kk < kBwD / 16; ++kk) {
-        const uint32_t oa = (kk >> 2) * kBwRows * 128 + (kk & 3) * 32;
-        const uint32_t ob = (kk >> 2) * kBwCols * 128 + (kk & 3) * 32;
-        umma_bf16(tmem + kBwColS + buf * kBwCols, at_desc_add(a1, oa), at_desc_add(x, ob), idesc_st,
-                  kk > 0 ? 1u : 0u);
-      }
-      umma_commit(&ctl->st_full[buf]);
-    }
-    if (it > 0) {
-      const uint32_t p = static_cast<uint32_t>(it - 1);
-      const uint32_t pbuf = p & 1u;
-      const uint32_t pslot = p % kBwStages;
-      if (!mbar_wait(&ctl->ds_full[pbuf], (p >> 1) & 1u, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // MN-major views of the streamed tiles (64 rows x 128 columns as two 64-column boxes):
-      // 64-column chunks one box apart, 8-row groups 1 KiB apart, a K = 16 step 2 KiB
-      const uint32_t xs = smem_u32(ring + pslot * 2 * kBwSmall);
-      const uint64_t x = sdesc_sw128(xs, kBwCols * 128, 1024), y = sdesc_sw128(xs + kBwSmall, kBwCols * 128, 1024);
-#pragma unroll
-      for (int kk = 0; kk < kBwCols / 16; ++kk) {
-        // streamed rows 16 kk .. 16 kk + 15: written by warp half kk / 2, pair columns 8 (kk % 2) on
-        const uint32_t col = pbuf * kBwCols + 32 * (kk >> 1) + 8 * (kk & 1);
-        const uint32_t acc = (p > 0 || kk > 0) ? 1u : 0u;
-        if (DKDV) {
-          at_mma_ta(tmem + kBwColAcc, tmem + kBwColS + col, at_desc_add(y, kk * 2048), idesc_acc, acc);
-          at_mma_ta(tmem + kBwColAcc + kBwD, tmem + kBwColDP + col, at_desc_add(x, kk * 2048), idesc_acc, acc);
-        } else {
-          at_mma_ta(tmem + kBwColAcc, tmem + kBwColDP + col, at_desc_add(x, kk * 2048), idesc_acc, acc);
-        }
-      }
-      umma_commit(&ctl->st_empty[pbuf]);
-      umma_commit(&ctl->empty[pslot]);
-    }
-  }
-  if (ok) umma_commit(&ctl->acc_full);
-  umma_commit(&ctl->mma_done);  // every issued MMA completes before TMEM is released
-  mbar_wait_drain(&ctl->mma_done, 0);
-}
-
-// The second MMA thread: dP = A2 Y^T of every block into its buffer, so that the
-// S and dP chains are issued by two threads on two sub-partitions (one thread
-// issuing all of a block's MMAs was the kernel's limit: ~80 cycles per MMA
-// against 48 of tensor work at N = 64).  Commits to st_full and to the ring
-// slot's empty barrier, both of which count one commit from each issuer.
-__device__ __forceinline__ void bw_mma_dp(BwCtl* ctl, uint32_t tmem, const uint8_t* resB, const uint8_t* ring, int n,
-                                          volatile int* abort_flag) {
-  constexpr uint32_t idesc_st = idesc_bf16_f32(kBwRows, kBwCols, false, false);
-  const uint64_t a2 = sdesc_sw128(smem_u32(resB), 16, 1024);
+  const uint64_t a = sdesc_sw128(smem_u32(res), 16, 1024);  // K = 16 steps add compile-time offsets
+  const uint32_t col = DP ? kBwColDP : kBwColS;
   bool ok = mbar_wait(&ctl->res_full, 0, abort_flag);
   tc_fence_after();
   for (int it = 0; ok && it < n; ++it) {
@@ -201,19 +146,56 @@ __device__ __forceinline__ void bw_mma_dp(BwCtl* ctl, uint32_t tmem, const uint8
         !mbar_wait(&ctl->st_empty[buf], ((static_cast<uint32_t>(it) >> 1) & 1u) ^ 1u, abort_flag))
       break;
     tc_fence_after();
-    const uint64_t y = sdesc_sw128(smem_u32(ring + slot * 2 * kBwSmall) + kBwSmall, 16, 1024);
+    const uint64_t b = sdesc_sw128(smem_u32(ring + slot * 2 * kBwSmall) + (DP ? kBwSmall : 0), 16, 1024);
+    // K-major steps: 32 bytes inside a 128-byte swizzle row, the second 64-column box from kk = 4 on
 #pragma unroll
     for (int kk = 0; kk < kBwD / 16; ++kk) {
       const uint32_t oa = (kk >> 2) * kBwRows * 128 + (kk & 3) * 32;
       const uint32_t ob = (kk >> 2) * kBwCols * 128 + (kk & 3) * 32;
-      umma_bf16(tmem + kBwColDP + buf * kBwCols, at_desc_add(a2, oa), at_desc_add(y, ob), idesc_st,
-                kk > 0 ? 1u : 0u);
+      umma_bf16(tmem + col + buf * kBwCols, at_desc_add(a, oa), at_desc_add(b, ob), idesc_st, kk > 0 ? 1u : 0u);
     }
     umma_commit(&ctl->st_full[buf]);
-    umma_commit(&ctl->empty[slot]);  // this issuer's reads of the slot (Y) are done with its dP
+    umma_commit(&ctl->empty[slot]);
   }
-  umma_commit(&ctl->mma_done_dp);  // every issued MMA completes before TMEM is released
-  mbar_wait_drain(&ctl->mma_done_dp, 0);
+  umma_commit(done);  // every issued MMA completes before TMEM is released
+  mbar_wait_drain(done, 0);
+}
+
+template <bool DKDV>
+__device__ __forceinline__ void bw_mma_acc(BwCtl* ctl, uint32_t tmem, const uint8_t* ring, int n,
+                                           volatile int* abort_flag) {
+  constexpr uint32_t idesc_acc = idesc_bf16_f32(kBwRows, kBwD, false, true);
+  bool ok = true;
+  for (int p = 0; p < n; ++p) {
+    const uint32_t pbuf = static_cast<uint32_t>(p) & 1u;
+    const uint32_t pslot = static_cast<uint32_t>(p) % kBwStages;
+    if (!mbar_wait(&ctl->ds_full[pbuf], (static_cast<uint32_t>(p) >> 1) & 1u, abort_flag)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    // MN-major views of the streamed tiles (64 rows x 128 columns as two 64-column boxes):
+    // 64-column chunks one box apart, 8-row groups 1 KiB apart, a K = 16 step 2 KiB
+    const uint32_t xs = smem_u32(ring + pslot * 2 * kBwSmall);
+    const uint64_t x = sdesc_sw128(xs, kBwCols * 128, 1024), y = sdesc_sw128(xs + kBwSmall, kBwCols * 128, 1024);
+#pragma unroll
+    for (int kk = 0; kk < kBwCols / 16; ++kk) {
+      // streamed rows 16 kk .. 16 kk + 15: written by the lane quarter's warp kk over its own first 8 columns
+      const uint32_t c = pbuf * kBwCols + kBwWCols * kk;
+      const uint32_t acc = (p > 0 || kk > 0) ? 1u : 0u;
+      if (DKDV) {
+        at_mma_ta(tmem + kBwColAcc, tmem + kBwColS + c, at_desc_add(y, kk * 2048), idesc_acc, acc);
+        at_mma_ta(tmem + kBwColAcc + kBwD, tmem + kBwColDP + c, at_desc_add(x, kk * 2048), idesc_acc, acc);
+      } else {
+        at_mma_ta(tmem + kBwColAcc, tmem + kBwColDP + c, at_desc_add(x, kk * 2048), idesc_acc, acc);
+      }
+    }
+    umma_commit(&ctl->st_empty[pbuf]);
+    umma_commit(&ctl->empty[pslot]);
+  }
+  if (ok) umma_commit(&ctl->acc_full);
+  umma_commit(&ctl->mma_done_acc);
+  mbar_wait_drain(&ctl->mma_done_acc, 0);
 }
 
 // 32 fp32 accumulator values of a row -> 32 bf16 at dst (16-byte aligned); returns
@@ -232,16 +214,31 @@ __device__ __forceinline__ bool bw_store32(uint16_t* dst, const float (&v)[32]) 
   return bad;
 }
 
-// A head row's accumulator columns c and c + 64 (c = 32 half .. + 31) through the
+// 16 fp32 accumulator values of a row -> 16 bf16 at dst (16-byte aligned); returns
+// true when one is not finite.
+__device__ __forceinline__ bool bw_store16(uint16_t* dst, const float (&v)[16]) {
+  bool bad = false;
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    bad |= !isfinite(v[2 * i]) || !isfinite(v[2 * i + 1]);
+    w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  }
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(dst + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+  return bad;
+}
+
+// A head row's accumulator columns c and c + 64 (c = 16 sub .. + 15) through the
 // inverse rotary rotation at position t (cs = (cos, sin) [L][64]), to dst and
 // dst + 64.
-__device__ __forceinline__ bool bw_store_rope(uint32_t taddr, int half, int t, const float2* __restrict__ cs,
+__device__ __forceinline__ bool bw_store_rope(uint32_t taddr, int sub, int t, const float2* __restrict__ cs,
                                               uint16_t* dst) {
-  float x1[32], x2[32];
-  at_ld32x2(taddr + 32 * half, x1, taddr + 64 + 32 * half, x2);
-  const float4* c4 = reinterpret_cast<const float4*>(cs + static_cast<size_t>(t) * (kBwD / 2) + 32 * half);
+  float x1[16], x2[16];
+  at_ld16x2(taddr + 16 * sub, x1, taddr + 64 + 16 * sub, x2);
+  const float4* c4 = reinterpret_cast<const float4*>(cs + static_cast<size_t>(t) * (kBwD / 2) + 16 * sub);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const float4 r = __ldg(c4 + i);  // (cos, sin) of columns 2i, 2i + 1
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -252,20 +249,20 @@ __device__ __forceinline__ bool bw_store_rope(uint32_t taddr, int half, int t, c
       x2[2 * i + e] = __fsub_rn(__fmul_rn(b, cv), __fmul_rn(a, sv));
     }
   }
-  bool bad = bw_store32(dst + 32 * half, x1);
-  bad |= bw_store32(dst + 64 + 32 * half, x2);
+  bool bad = bw_store16(dst + 16 * sub, x1);
+  bad |= bw_store16(dst + 64 + 16 * sub, x2);
   return bad;
 }
 
 // Elementwise warps: per block, P = bf16(exp(fl(s scale) - lse)) and
-// dS = bf16(P (dP - D) scale) for this warp's 32 of the block's 64 streamed
+// dS = bf16(P (dP - D) scale) for this warp's 16 of the block's 64 streamed
 // columns, written as bf16 pairs over the columns read (P over S only for DKDV,
 // where dV needs it).  DKDV: the rows are keys, the columns queries (lse and D
 // per column); else the rows are queries (lse and D per row), the columns keys.
 // `row_pos` is the row's position in the sample, `col_pos0` the position of the
 // first streamed column of block 0.
 template <bool DKDV>
-__device__ __forceinline__ bool bw_elementwise(BwCtl* ctl, uint32_t tmem, uint32_t lane_off, int half, int n,
+__device__ __forceinline__ bool bw_elementwise(BwCtl* ctl, uint32_t tmem, uint32_t lane_off, int sub, int n,
                                                int row_pos, int col_pos0, const float* __restrict__ lse_row,
                                                const float* __restrict__ D_row, float scale,
                                                volatile int* abort_flag) {
@@ -281,13 +278,13 @@ __device__ __forceinline__ bool bw_elementwise(BwCtl* ctl, uint32_t tmem, uint32
   }
   for (int it = 0; it < n; ++it) {
     const uint32_t buf = static_cast<uint32_t>(it) & 1u;
-    const int c0 = col_pos0 + kBwCols * it + 32 * half;  // position of this warp's first column
-    float lc[32], dc[32];
+    const int c0 = col_pos0 + kBwCols * it + kBwWCols * sub;  // position of this warp's first column
+    float lc[kBwWCols], dc[kBwWCols];
     if (DKDV) {  // the columns' lse and D (the same addresses in every lane: broadcast loads)
       const float4* l4 = reinterpret_cast<const float4*>(lse_row + c0);
       const float4* d4 = reinterpret_cast<const float4*>(D_row + c0);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kBwWCols / 4; ++i) {
         const float4 a = __ldg(l4 + i), b = __ldg(d4 + i);
         lc[4 * i] = a.x, lc[4 * i + 1] = a.y, lc[4 * i + 2] = a.z, lc[4 * i + 3] = a.w;
         dc[4 * i] = b.x, dc[4 * i + 1] = b.y, dc[4 * i + 2] = b.z, dc[4 * i + 3] = b.w;
@@ -296,18 +293,18 @@ __device__ __forceinline__ bool bw_elementwise(BwCtl* ctl, uint32_t tmem, uint32
     if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->st_full[buf], (static_cast<uint32_t>(it) >> 1) & 1u, abort_flag)))
       return false;
     tc_fence_after();
-    const uint32_t cs = kBwColS + buf * kBwCols + 32 * half;
-    const uint32_t cd = kBwColDP + buf * kBwCols + 32 * half;
-    float sv[32], dpv[32];
-    at_ld32x2(tmem + lane_off + cs, sv, tmem + lane_off + cd, dpv);
-    uint32_t pp[16], dd[16];
+    const uint32_t cs = kBwColS + buf * kBwCols + kBwWCols * sub;
+    const uint32_t cd = kBwColDP + buf * kBwCols + kBwWCols * sub;
+    float sv[kBwWCols], dpv[kBwWCols];
+    at_ld16x2(tmem + lane_off + cs, sv, tmem + lane_off + cd, dpv);
+    uint32_t pp[kBwWCols / 2], dd[kBwWCols / 2];
     // causal: a query sees the keys at or before its position; only the two blocks
     // that overlap the diagonal hold masked entries
     const bool near_diag = DKDV ? it < 2 : it >= n - 2;
     auto body = [&](auto masked_tag) {
       constexpr bool kMask = decltype(masked_tag)::value;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < kBwWCols / 2; ++i) {
         float pe[2], de[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -328,8 +325,9 @@ __device__ __forceinline__ bool bw_elementwise(BwCtl* ctl, uint32_t tmem, uint32
     };
     if (near_diag) body(std::true_type{});
     else body(std::false_type{});
-    if (DKDV) at_tmem_st16(tmem + lane_off + cs, pp);
-    at_tmem_st16(tmem + lane_off + cd, dd);
+    // pair column j of the slice holds streamed columns 2j, 2j + 1 (over the slice's first 8 columns)
+    if (DKDV) at_tmem_st8(tmem + lane_off + cs, pp);
+    at_tmem_st8(tmem + lane_off + cd, dd);
     at_tmem_st_wait();
     tc_fence_before();
     __syncwarp();
@@ -376,30 +374,29 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       bw_produce(ctl, sK, sV, ring, &tmBig, H + h * kBwD, 2 * H + h * kBwD, row0 + kb * kBwRows, &tmQ64, h * kBwD,
                  &tmDO64, h * kBwD, row0 + q0 * kBwCols, n, abort_flag);
   } else if (warp == 1) {
-    if (lane == 0) bw_mma<true>(ctl, tmem, sK, sV, ring, n, abort_flag);
+    if (lane == 0) bw_mma_st<false>(ctl, tmem, sK, ring, n, &ctl->mma_done, abort_flag);
   } else if (warp == kBwDpWarp) {
-    if (lane == 0) bw_mma_dp(ctl, tmem, sV, ring, n, abort_flag);
+    if (lane == 0) bw_mma_st<true>(ctl, tmem, sV, ring, n, &ctl->mma_done_dp, abort_flag);
+  } else if (warp == kBwAccWarp) {
+    if (lane == 0) bw_mma_acc<true>(ctl, tmem, ring, n, abort_flag);
   } else {
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int sub = (warp - 2) >> 2;  // the warp's part of its lane quarter's columns
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int t = kb * kBwRows + r;  // key position in the sample
     const size_t lrow = (static_cast<size_t>(s) * nh + h) * L;
-    bool ok = bw_elementwise<true>(ctl, tmem, lane_off, half, n, t, q0 * kBwCols, lse + lrow, Dsum + lrow, scale,
+    bool ok = bw_elementwise<true>(ctl, tmem, lane_off, sub, n, t, q0 * kBwCols, lse + lrow, Dsum + lrow, scale,
                                    abort_flag);
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->acc_full, 0, abort_flag));
     bool bad = false;
     if (ok) {
       tc_fence_after();
       uint16_t* row = dqkv + static_cast<size_t>(row0 + t) * (3 * H);
-      bad |= bw_store_rope(tmem + lane_off + kBwColAcc + kBwD, half, t, cs, row + H + h * kBwD);  // dK
-      float v[32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {  // dV: this warp's 64 head columns
-        tmem_ld32(tmem + lane_off + kBwColAcc + 64 * half + 32 * c, v);
-        bad |= bw_store32(row + 2 * H + h * kBwD + 64 * half + 32 * c, v);
-      }
+      bad |= bw_store_rope(tmem + lane_off + kBwColAcc + kBwD, sub, t, cs, row + H + h * kBwD);  // dK
+      float v[32];  // dV: this warp's 32 head columns
+      tmem_ld32(tmem + lane_off + kBwColAcc + 32 * sub, v);
+      bad |= bw_store32(row + 2 * H + h * kBwD + 32 * sub, v);
       tc_fence_before();
     }
     if (bad) raise_status(kStatusNonFinite);
@@ -469,23 +466,25 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         mbar_wait_drain(&ctl->full[i % kBwStages], (i / kBwStages) & 1u);
     }
   } else if (warp == 1) {
-    if (lane == 0) bw_mma<false>(ctl, tmem, sQ, sDO, ring, n, abort_flag);
+    if (lane == 0) bw_mma_st<false>(ctl, tmem, sQ, ring, n, &ctl->mma_done, abort_flag);
   } else if (warp == kBwDpWarp) {
-    if (lane == 0) bw_mma_dp(ctl, tmem, sDO, ring, n, abort_flag);
+    if (lane == 0) bw_mma_st<true>(ctl, tmem, sDO, ring, n, &ctl->mma_done_dp, abort_flag);
+  } else if (warp == kBwAccWarp) {
+    if (lane == 0) bw_mma_acc<false>(ctl, tmem, ring, n, abort_flag);
   } else {
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int sub = (warp - 2) >> 2;  // the warp's part of its lane quarter's columns
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int t = qb * kBwRows + r;  // query position in the sample
     const size_t lrow = (static_cast<size_t>(s) * nh + h) * L;
-    bool ok = bw_elementwise<false>(ctl, tmem, lane_off, half, n, t, 0, lse + lrow, Dsum + lrow, scale, abort_flag);
+    bool ok = bw_elementwise<false>(ctl, tmem, lane_off, sub, n, t, 0, lse + lrow, Dsum + lrow, scale, abort_flag);
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->acc_full, 0, abort_flag));
     bool bad = false;
     if (ok) {
       tc_fence_after();
       uint16_t* row = dqkv + static_cast<size_t>(row0 + t) * (3 * H);
-      bad |= bw_store_rope(tmem + lane_off + kBwColAcc, half, t, cs, row + h * kBwD);  // dQ
+      bad |= bw_store_rope(tmem + lane_off + kBwColAcc, sub, t, cs, row + h * kBwD);  // dQ
       tc_fence_before();
     }
     if (bad) raise_status(kStatusNonFinite);
