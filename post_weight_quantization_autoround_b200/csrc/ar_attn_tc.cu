@@ -18,20 +18,22 @@
 //  * warp 0: TMA producer.  Q once (two 64-column boxes of 128 rows, 128-byte
 //    swizzle), then the K blocks of pass 1 and the K and V blocks of pass 2 in
 //    the order the MMAs consume them, into a 3-deep K ring and a 2-deep V ring.
-//  * warp 1: TMEM owner (512 columns) and, in lane 0, the MMA issuer.
-//    S = Q K^T (M = 128 queries, N = 128 keys, K = 128, A and B K-major from
-//    shared memory) into one of two fp32 S buffers; O += P V (A = P as bf16
-//    pairs in tensor memory, B = V as an MN-major operand from shared memory)
-//    into the fp32 O accumulator.  In pass 2 the next block's S is issued
-//    before this block's P V, so the softmax of one block overlaps the MMAs of
-//    the other.
-//  * warps 2-9: softmax and epilogue.  Warp w reads TMEM lanes 32 (w % 4) ..
-//    + 31 (one query row per thread, hardware rule) and one half of the 128 key
-//    columns.  Pass 1 keeps a running (max, sum) per thread over its half; the
-//    two warps of a lane quarter combine them once at the end through shared
-//    memory.  Pass 2 writes P = bf16(exp(z - lse)) into one of two P buffers in
-//    tensor memory (column c holds keys 2c, 2c + 1).  At the end each warp
-//    drains its half of O's 128 columns and stores bf16, and the lse.
+//  * warp 1: TMEM owner (512 columns) and, in lane 0, the S issuer: S = Q K^T
+//    (M = 128 queries, N = 128 keys, K = 128, A and B K-major from shared
+//    memory) into one of two fp32 S buffers, for pass 1 and then pass 2.
+//  * warp 18, lane 0: the P V issuer: O += P V (A = P as bf16 pairs in tensor
+//    memory, B = V as an MN-major operand from shared memory) into the fp32 O
+//    accumulator.  Two issuing threads on two sub-partitions, so that neither
+//    chain waits on the other's issue; the softmax of one block overlaps the
+//    MMAs of the next.
+//  * warps 2-17: softmax and epilogue.  Warp w reads TMEM lanes 32 (w % 4) ..
+//    + 31 (one query row per thread, hardware rule) and 32 of the 128 key
+//    columns (four warps per lane quarter).  Pass 1 keeps a running (max, sum)
+//    per thread over its 32 keys; the four warps of a lane quarter combine them
+//    once at the end through shared memory, in a fixed order.  Pass 2 writes
+//    P = bf16(exp(z - lse)) into one of two P buffers in tensor memory (column
+//    c holds keys 2c, 2c + 1).  At the end each warp drains 32 of O's 128
+//    columns and stores bf16, and the lse.
 //
 // TMEM columns: S buffers [0, 256), P buffers [256, 384), O [384, 512).
 // Every mbarrier wait is bounded (ar_device.cuh): on a timeout the kernel
@@ -48,8 +50,12 @@ constexpr int kAtBox = kAtBlk * 128;       // 16 KiB: 128 rows x 64 bf16 columns
 constexpr int kAtTile = 2 * kAtBox;        // 32 KiB: 128 rows x 128 columns
 constexpr int kAtKStages = 3;
 constexpr int kAtVStages = 2;
-constexpr int kAtSmWarps = 8;              // two per TMEM lane quarter
-constexpr int kAtThreads = (2 + kAtSmWarps) * 32;
+constexpr int kAtSmWarps = 16;             // four per TMEM lane quarter
+constexpr int kAtPerQ = kAtSmWarps / 4;
+constexpr int kAtWCols = kAtBlk / kAtPerQ;  // key columns of a block (and head columns of O) per warp
+static_assert(kAtWCols == 32, "the softmax role loads and stores 32-column slices");
+constexpr int kAtPvWarp = 2 + kAtSmWarps;   // issuer of the P V products
+constexpr int kAtThreads = (3 + kAtSmWarps) * 32;
 constexpr uint32_t kAtColS = 0;            // two S buffers of 128 fp32 columns
 constexpr uint32_t kAtColP = 256;          // two P buffers of 64 columns (bf16 pairs)
 constexpr uint32_t kAtColO = 384;          // O: 128 fp32 columns
@@ -67,9 +73,10 @@ struct AtCtl {
   uint64_t p_empty[2];  // MMA: P V of the buffer done
   uint64_t o_full;
   uint64_t mma_done;
+  uint64_t mma_done_pv;
   uint32_t tmem_base;
   int abort_flag;
-  float2 ml[4][2][32];  // pass 1: (max, sum) per lane quarter, column half and row
+  float2 ml[4][kAtPerQ][32];  // pass 1: (max, sum) per lane quarter, column part and row
 };
 
 constexpr int kAtSmem = kAtTile * (1 + kAtKStages + kAtVStages) + static_cast<int>(sizeof(AtCtl)) + 1024;
@@ -120,6 +127,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     mbar_init(&ctl->o_full, 1);
     mbar_init(&ctl->mma_done, 1);
+    mbar_init(&ctl->mma_done_pv, 1);
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
@@ -165,20 +173,23 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         mbar_wait_drain(&ctl->v_full[i % kAtVStages], (i / kAtVStages) & 1u);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
+    // (two issuing threads on two sub-partitions: one thread issuing both the
+    // S and the P V products of a block was a limit)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kAtBlk, kAtBlk, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kAtBlk, kAtD, false, true);
       const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);  // K = 16 steps: compile-time offsets
-      uint32_t ki = 0, ns = 0;
       bool ok = mbar_wait(&ctl->q_full, 0, abort_flag);
       tc_fence_after();
-      // S buffer ns % 2 = Q K^T of the next K block in the ring
-      auto issue_s = [&]() -> bool {
-        const uint32_t slot = ki % kAtKStages;
+      // S buffer ns % 2 = Q K^T of the next K block in the ring: pass 1, then pass 2
+      for (uint32_t ns = 0; ok && ns < static_cast<uint32_t>(2 * n_kb); ++ns) {
+        const uint32_t slot = ns % kAtKStages;
         const uint32_t buf = ns & 1u;
-        if (!mbar_wait(&ctl->k_full[slot], (ki / kAtKStages) & 1u, abort_flag)) return false;
-        if (!mbar_wait(&ctl->s_empty[buf], ((ns >> 1) & 1u) ^ 1u, abort_flag)) return false;
+        if (!mbar_wait(&ctl->k_full[slot], (ns / kAtKStages) & 1u, abort_flag) ||
+            !mbar_wait(&ctl->s_empty[buf], ((ns >> 1) & 1u) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint64_t k_desc = sdesc_sw128(smem_u32(sK + slot * kAtTile), 16, 1024);
         const uint32_t d = tmem + kAtColS + buf * kAtBlk;
@@ -189,14 +200,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         }
         umma_commit(&ctl->s_full[buf]);
         umma_commit(&ctl->k_empty[slot]);
-        ++ki;
-        ++ns;
-        return true;
-      };
-      for (int j = 0; ok && j < n_kb; ++j) ok = issue_s();  // pass 1
-      if (ok) ok = issue_s();                                // pass 2: block 0
-      for (int j = 0; ok && j < n_kb; ++j) {
-        if (j + 1 < n_kb && !(ok = issue_s())) break;  // the next block's S before this block's P V
+      }
+      // every issued MMA completes before TMEM is released
+      umma_commit(&ctl->mma_done);
+      mbar_wait_drain(&ctl->mma_done, 0);
+    }
+  } else if (warp == kAtPvWarp) {
+    // ------------------------------------------------------------ P V issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kAtBlk, kAtD, false, true);
+      bool ok = true;
+      for (int j = 0; j < n_kb; ++j) {
         const uint32_t pbuf = static_cast<uint32_t>(j) & 1u;
         const uint32_t vslot = static_cast<uint32_t>(j) % kAtVStages;
         if (!mbar_wait(&ctl->p_full[pbuf], (static_cast<uint32_t>(j) >> 1) & 1u, abort_flag) ||
@@ -214,17 +228,16 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         umma_commit(&ctl->v_empty[vslot]);
       }
       if (ok) umma_commit(&ctl->o_full);
-      // every issued MMA completes before TMEM is released
-      umma_commit(&ctl->mma_done);
-      mbar_wait_drain(&ctl->mma_done, 0);
+      umma_commit(&ctl->mma_done_pv);
+      mbar_wait_drain(&ctl->mma_done_pv, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax and epilogue
     const int quarter = warp & 3;         // TMEM lane quarter (hardware rule: warp % 4)
-    const int hh = (warp - 2) >> 2;       // key-column half of each block, head-column half of O
+    const int sub = (warp - 2) >> 2;      // 32-column part: keys of each block, head columns of O
     const int r = quarter * 32 + lane;    // query row within the block
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int k0 = hh * 64;               // first key column of this warp's half
+    const int k0 = sub * kAtWCols;        // first key column of this warp's part
     uint32_t ns = 0;
     bool ok = true;
     // Exponentials as 2^x with the hardware ex2: exp(z - a) = 2^(s c2 - a log2 e),
@@ -232,34 +245,34 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // exp(fl(s scale) - a), far below the bf16 rounding of P).  The row maximum is
     // taken over the raw scores (scale > 0).  Only the diagonal block is masked.
     const float c2 = scale * 1.4426950408889634f;
-    // pass 1: running (max, sum of exp(scale (s - max))) over this half's keys
+    // pass 1: running (max, sum of exp(scale (s - max))) over this part's keys
     float m = -INFINITY, l = 0.f;
     for (int j = 0; ok && j < n_kb; ++j, ++ns) {
       const uint32_t buf = ns & 1u;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->s_full[buf], (ns >> 1) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float v[64];
-      at_ld64(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v);
+      float v[kAtWCols];
+      tmem_ld32(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->s_empty[buf]);
       if (j == qb) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) v[i] = k0 + i > r ? -INFINITY : v[i];
+        for (int i = 0; i < kAtWCols; ++i) v[i] = k0 + i > r ? -INFINITY : v[i];
       }
       float mx0 = v[0], mx1 = v[1];
 #pragma unroll
-      for (int i = 2; i < 64; i += 2) {
+      for (int i = 2; i < kAtWCols; i += 2) {
         mx0 = fmaxf(mx0, v[i]);
         mx1 = fmaxf(mx1, v[i + 1]);
       }
       const float mn = fmaxf(m, fmaxf(mx0, mx1));
-      if (mn != -INFINITY) {  // else every key of the half so far is masked: nothing to add
+      if (mn != -INFINITY) {  // else every key of the part so far is masked: nothing to add
         const float off = mn * c2;
         float t0 = 0.f, t1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
+        for (int i = 0; i < kAtWCols; i += 2) {
           t0 += at_ex2(fmaf(v[i], c2, -off));
           t1 += at_ex2(fmaf(v[i + 1], c2, -off));
         }
@@ -267,14 +280,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         m = mn;
       }
     }
-    // the row's lse from the two halves (half 0 always holds key 0, so its max is finite);
-    // both warps add in the same order and reach this barrier exactly once
-    ctl->ml[quarter][hh][lane] = make_float2(m, l);
-    at_bar_sync(1 + quarter, 64);
-    const float2 a0 = ctl->ml[quarter][0][lane];
-    const float2 a1 = ctl->ml[quarter][1][lane];
-    const float mm = fmaxf(a0.x, a1.x);
-    const float lsum = a0.y * at_ex2((a0.x - mm) * c2) + a1.y * at_ex2((a1.x - mm) * c2);
+    // the row's lse from the parts (part 0 always holds key 0, so its max is finite);
+    // every warp of the quarter adds in the same order and reaches this barrier once
+    ctl->ml[quarter][sub][lane] = make_float2(m, l);
+    at_bar_sync(1 + quarter, 32 * kAtPerQ);
+    float mm = ctl->ml[quarter][0][lane].x;
+#pragma unroll
+    for (int q = 1; q < kAtPerQ; ++q) mm = fmaxf(mm, ctl->ml[quarter][q][lane].x);
+    float lsum = 0.f;
+#pragma unroll
+    for (int q = 0; q < kAtPerQ; ++q) {
+      const float2 a = ctl->ml[quarter][q][lane];
+      lsum += a.y * at_ex2((a.x - mm) * c2);
+    }
     const float lse = __fmul_rn(mm, scale) + logf(lsum);
     const float lse2 = lse * 1.4426950408889634f;
     ok = ok && *abort_flag == 0;
@@ -284,22 +302,22 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->s_full[buf], (ns >> 1) & 1u, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float v[64];
-      at_ld64(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v);
+      float v[kAtWCols];
+      tmem_ld32(tmem + lane_off + kAtColS + buf * kAtBlk + k0, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->s_empty[buf]);
-      uint32_t pk[32];
+      uint32_t pk[kAtWCols / 2];
       if (j == qb) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < kAtWCols / 2; ++i) {
           const float p0 = k0 + 2 * i > r ? 0.f : at_ex2(fmaf(v[2 * i], c2, -lse2));
           const float p1 = k0 + 2 * i + 1 > r ? 0.f : at_ex2(fmaf(v[2 * i + 1], c2, -lse2));
           pk[i] = pack_bf16x2(p0, p1);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < kAtWCols / 2; ++i)
           pk[i] = pack_bf16x2(at_ex2(fmaf(v[2 * i], c2, -lse2)), at_ex2(fmaf(v[2 * i + 1], c2, -lse2)));
       }
       const uint32_t pbuf = static_cast<uint32_t>(j) & 1u;
@@ -307,34 +325,32 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                                              abort_flag));
       if (!ok) break;
       tc_fence_after();
-      at_tmem_st32(tmem + lane_off + kAtColP + pbuf * 64 + hh * 32, pk);
+      // pair column c of a P buffer holds keys 2c, 2c + 1
+      at_tmem_st16(tmem + lane_off + kAtColP + pbuf * 64 + k0 / 2, pk);
       at_tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[pbuf]);
     }
-    // epilogue: O (bf16) for this warp's 64 head columns, and the lse
+    // epilogue: O (bf16) for this warp's 32 head columns, and the lse
     bool bad = false;
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&ctl->o_full, 0, abort_flag));
     if (ok) {
       tc_fence_after();
       const int qi = qb * kAtBlk + r;
       uint16_t* orow = out + static_cast<size_t>(row0 + qi) * H + h * kAtD + k0;
+      float o[kAtWCols];
+      tmem_ld32(tmem + lane_off + kAtColO + k0, o);
+      uint32_t w[kAtWCols / 2];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float o[32];
-        tmem_ld32(tmem + lane_off + kAtColO + k0 + 32 * c, o);
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          bad |= !isfinite(o[2 * i]) || !isfinite(o[2 * i + 1]);
-          w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<uint4*>(orow + 32 * c + 8 * i) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      for (int i = 0; i < kAtWCols / 2; ++i) {
+        bad |= !isfinite(o[2 * i]) || !isfinite(o[2 * i + 1]);
+        w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
       }
-      if (hh == 0) lse_out[(static_cast<size_t>(s) * nh + h) * L + qi] = lse;
+#pragma unroll
+      for (int i = 0; i < kAtWCols / 8; ++i)
+        *reinterpret_cast<uint4*>(orow + 8 * i) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      if (sub == 0) lse_out[(static_cast<size_t>(s) * nh + h) * L + qi] = lse;
       tc_fence_before();
     }
     if (bad) raise_status(kStatusNonFinite);
