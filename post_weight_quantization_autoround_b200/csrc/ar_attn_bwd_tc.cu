@@ -59,7 +59,7 @@ struct BwCtl {
   uint64_t full[kBwStages];       // streamed pair landed
   uint64_t empty[kBwStages];      // streamed pair no longer read (one commit from each of three issuers)
   uint64_t st_full[2];            // MMA: S and dP of the buffer pair written (one commit from each issuer)
-  uint64_t ds_full[2];            // elementwise warps: their bf16 operands written (8 arrivals)
+  uint64_t ds_full[2];            // elementwise warps: their bf16 operands written (one arrival per warp)
   uint64_t st_empty[2];           // MMA: the accumulating products of the pair done
   uint64_t acc_full;
   uint64_t mma_done;

@@ -68,9 +68,9 @@ struct AtCtl {
   uint64_t v_full[kAtVStages];
   uint64_t v_empty[kAtVStages];
   uint64_t s_full[2];   // MMA: S buffer written
-  uint64_t s_empty[2];  // softmax warps: S buffer read (8 arrivals)
-  uint64_t p_full[2];   // softmax warps: P buffer written (8 arrivals)
-  uint64_t p_empty[2];  // MMA: P V of the buffer done
+  uint64_t s_empty[2];  // softmax warps: S buffer read (one arrival per softmax warp)
+  uint64_t p_full[2];   // softmax warps: P buffer written (one arrival per softmax warp)
+  uint64_t p_empty[2];  // P V issuer: P V of the buffer done
   uint64_t o_full;
   uint64_t mma_done;
   uint64_t mma_done_pv;
