@@ -85,12 +85,16 @@ __host__ __device__ constexpr bool slot_phases_in_order(int per_slot, int sets, 
   return per_slot % sets == 0 || (sets % per_slot == 0 && slots % (sets / per_slot) == 0);
 }
 
-template <int TN, int BITS>
+template <int TN, int BITS, bool FP4 = false>
 struct TcCfg {
   // One dequantization warp per TMEM lane quarter is latency bound (its nibble
   // and permute chains), so narrow tiles, whose epilogue needs few registers,
-  // run two per quarter on alternating stages.
-  static constexpr int kDqWarps = TN >= 128 ? 4 : 8;
+  // run two per quarter on alternating stages.  At TN = 128 a second set costs
+  // epilogue spills (the 608 threads leave ~104 registers), which pays only where
+  // the dequantization is long enough: measured on 8192 x 28672 at 256 tokens,
+  // NVFP4 219 -> 176 us and 2 bits 221 -> 212 us, but 4 bits 227 -> 239 us,
+  // 3 bits 223 -> 270 us, 8 bits unchanged.
+  static constexpr int kDqWarps = (TN < 128 || FP4 || BITS == 2) ? 8 : 4;
   static constexpr int kEpWarp0 = kDqWarp0 + kDqWarps;
   static constexpr int kThreads = (kEpWarp0 + kEpWarps) * 32;
   static constexpr int kActBytes = TN * 128 * kSub;    // TN tokens x kTcK k bf16, kSub sub-tiles
@@ -378,10 +382,10 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // into the dequantized operand, the per-tensor scale applied per group in the
 // epilogue); BITS is then 4.
 template <int TN, int KSPLIT, int BITS, bool FP4>
-__global__ void __launch_bounds__(TcCfg<TN, BITS>::kThreads, 1)
+__global__ void __launch_bounds__(TcCfg<TN, BITS, FP4>::kThreads, 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const TcParams p) {
-  using Cfg = TcCfg<TN, BITS>;
+  using Cfg = TcCfg<TN, BITS, FP4>;
   using Code = CodeCfg<BITS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -778,7 +782,7 @@ __global__ void __launch_bounds__(TcCfg<TN, BITS>::kThreads, 1)
 template <int TN, int KSPLIT, int BITS, bool FP4>
 cudaError_t launch_tc(const uint16_t* A, const CUtensorMap& tmW, TcParams p, int n_tiles, cudaStream_t stream,
                       const char* name) {
-  using Cfg = TcCfg<TN, BITS>;
+  using Cfg = TcCfg<TN, BITS, FP4>;
   CUtensorMap tmA;
   cudaError_t e = make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, static_cast<uint64_t>(p.T),
                                static_cast<uint64_t>(p.K), 64, TN, CU_TENSOR_MAP_SWIZZLE_128B);  // kSub boxes per stage
