@@ -159,6 +159,25 @@ def test_gemm_all_operand_layouts(ar, a_mn, b_mn, M, N, K):
 
 
 @pytest.mark.parametrize("a_mn,b_mn", [(False, False), (True, True)])
+def test_gemm_last_wave_half_width_units(ar, a_mn, b_mn):
+    """2048 x 2560 output = 8 x 10 pair tiles of 256 x 256: on a 148-SM B200 (74 clusters) one wave of
+    74 whole tiles, then the last 6 tiles as 12 units of 256 x 128; every output element is checked."""
+    M, N, K = 2048, 2560, 128
+    rng = np.random.default_rng(21)
+    A = synth.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    B = synth.to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32))
+    ref = O.reference_forward(synth.bf16_bits_to_f32(A), synth.bf16_bits_to_f32(B)).astype(np.float64)
+    Ad = bf16_dev(np.ascontiguousarray(A.T) if a_mn else A)
+    Bd = bf16_dev(np.ascontiguousarray(B.T) if b_mn else B)
+    D = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    ar.ar_gemm_bf16(Ad, a_mn, Bd, b_mn, D, M, N, K)
+    assert ar.ar_get_device_status() == 0
+    got = D.cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.max(np.abs(got - ref)) <= 1e-5 * np.sqrt(K) * 4
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(False, False), (True, True)])
 def test_gemm_grouped_raster_covers_every_tile(ar, a_mn, b_mn):
     """B of 4608 x 8192 bf16 (75 MB) does not stay resident in L2, so the tiles run in groups of
     16 tile rows (20 rows: a full and a partial group); every output tile is computed once, checked on
