@@ -277,13 +277,18 @@ AR_API ar_status ar_rmsnorm(const void* x, int x_is_f32, const float* gamma, int
 /* Causal softmax attention per sample and head on qkv [S*L][3H] bf16 (columns
  * Qr | Kr | V, the rotation already applied): out [S*L][H] bf16 = P V with
  * P = bf16(exp(z - lse)), z = Qr Kr^T / sqrt(d) (fp32), and lse fp32 [S][nh][L].
- * Needs L % 64 == 0, d = H / n_heads in {64, 128}. */
+ * Needs L % 64 == 0, d = H / n_heads in {64, 128}.  d = 128 with L % 128 == 0
+ * runs on tcgen05 (128-query CTAs, S and O in tensor memory, the exponential
+ * as 2^x by the hardware after one fused multiply-add); other shapes on
+ * mma.sync.  Both compute the two passes the same way (lse, then P). */
 AR_API ar_status ar_attention_forward(const uint16_t* qkv, int64_t S, int64_t L, int64_t H, int n_heads,
                                       uint16_t* out, float* lse, ar_stream_t stream);
 
 /* Its backward from dO [S*L][H] bf16: dqkv [S*L][3H] bf16 = dQ | dK | dV, with
  * dQ and dK taken back through the rotation (dQ = R^T dQr).  out and lse are
- * the forward's.  Workspace: ar_attention_backward_workspace bytes (device,
+ * the forward's.  d = 128 with L % 128 == 0 runs two tcgen05 kernels (dQ per
+ * 128 queries, dK and dV per 128 keys; no atomics, deterministic); other
+ * shapes mma.sync.  Workspace: ar_attention_backward_workspace bytes (device,
  * 256-byte aligned). */
 AR_API size_t ar_attention_backward_workspace(int64_t S, int64_t L, int64_t H, int n_heads);
 AR_API ar_status ar_attention_backward(const uint16_t* qkv, const uint16_t* out, const uint16_t* dout,
