@@ -48,6 +48,20 @@
 //
 // Packed layout (as ar_pack_int4 writes it): uint32 [N][K/8], element k at
 // bits 4*(k mod 8) of word k/8; scale/zero fp16 [N][K/g].
+//
+// The same kernel takes 2-bit codes (ar_pack_codes' stream: element k at bits
+// 2*(k mod 16) of word k/16) up to 8 tokens for g >= 64.  A 512-k stage is one
+// 128-byte box per row, and a lane's 32-bit word holds 16 codes, so a 128-k
+// chunk is two 64-k slices of four MMAs each (weights as the A operand).  The
+// codes are not shifted down one by one: (x & (3 << 2m)) | 0x4300 for
+// m = 0, 1, 2 is the bf16 128 + 4^m q, since bits 0..6 are the mantissa of a
+// bf16 in [128, 256), so one word needs two shifts (by 6 and 12) and eight
+// logic ops to give its eight pairs (q_i, q_{i+8}).  The activation paired
+// with a code at scale 4^m is multiplied by 4^-m (exact in bf16), so each
+// product is (128 / 4^m) a + q a.  One MMA of the scaled activations against a
+// constant fragment gives both corrections: rows 0..7 hold the class weights
+// 4^m (Oa = sum of a), rows 8..15 ones (Ob = sum of a / 4^m), and a group adds
+// s (D - 128 Ob) - s z Oa.
 #include <cooperative_groups.h>
 
 #include <cstdio>
@@ -62,7 +76,8 @@ namespace {
 constexpr int kDecStageK = 512;                 // k per stage
 constexpr int kDecPassRows = 64;                // rows per pass (eight n8 tiles)
 constexpr int kDecCodeBox = kDecPassRows * 128; // one 256-k box of codes: 64 rows x 128 bytes
-constexpr int kDecMaxStages = 8;
+constexpr int kDecMaxStages = 8;               // ring depth cap, 4-bit codes (two boxes per stage)
+constexpr int kDecMaxStages2 = 16;             // ... 2-bit codes (one box per stage)
 constexpr int kDecSmemLimit = 227 * 1024;
 
 template <bool TBIG>
@@ -94,8 +109,8 @@ struct DecParams {
 
 struct alignas(16) DecTail {
   float2 sm[8][kDecPassRows];   // per consumer warp: (s, -s (128 + z)) of the pass's rows for one group
-  uint64_t full[kDecMaxStages];
-  uint64_t empty[kDecMaxStages];
+  uint64_t full[kDecMaxStages2];
+  uint64_t empty[kDecMaxStages2];
   float part[kDecPassRows][16];
   int abort_flag;
 };
@@ -133,6 +148,36 @@ __device__ __forceinline__ uint32_t shr(uint32_t x, uint32_t n) {
   return d;
 }
 
+// (x & m) | 0x43004300 for a mask m inside bits 0..5 of each half: the bf16
+// pair (128 + code, 128 + code') scaled by the mask's position.
+template <uint32_t M>
+__device__ __forceinline__ uint32_t mask_pair(uint32_t x) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(x), "r"(M), "r"(0x43004300u));
+  return d;
+}
+
+// The eight bf16 pairs of one word of 2-bit codes: r[i] = (128 + s_i q_i,
+// 128 + s_i q_{i+8}) with s = (1, 4, 16, 1, 4, 16, 1, 4).
+__device__ __forceinline__ void two_bit_pairs(uint32_t x, uint32_t (&r)[8]) {
+  const uint32_t y = shr(x, 6);
+  const uint32_t z = shr(x, 12);
+  r[0] = mask_pair<0x00030003u>(x);
+  r[1] = mask_pair<0x000C000Cu>(x);
+  r[2] = mask_pair<0x00300030u>(x);
+  r[3] = mask_pair<0x00030003u>(y);
+  r[4] = mask_pair<0x000C000Cu>(y);
+  r[5] = mask_pair<0x00300030u>(y);
+  r[6] = mask_pair<0x00030003u>(z);
+  r[7] = mask_pair<0x000C000Cu>(z);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -140,18 +185,21 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 __device__ __forceinline__ float half_bits_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 
 // TBIG: 9..16 tokens (token rows g and g + 8 of the A fragment both live).
-// SPAN: 32-k slices per group span inside a 128-k chunk (4 for g >= 128, 2 for
-// g = 64, 1 for g = 32).  KS: CTAs of a cluster splitting K (1 or 2).  NT: n8
+// SPAN: slices per group span inside a 128-k chunk; 4-bit codes: 32-k slices (4
+// for g >= 128, 2 for g = 64, 1 for g = 32), 2-bit codes: 64-k slices (2 for
+// g >= 128, 1 for g = 64).  KS: CTAs of a cluster splitting K (1 or 2).  NT: n8
 // tiles per pass, a compile-time count so that the tile loops are straight-line
 // code (tiles past a pass's rows read rows of the stage buffer that the pass
-// does not own and are computed but never stored).
-template <bool TBIG, int SPAN, int KS, int NT>
+// does not own and are computed but never stored).  BITS: 4, or 2 (T <= 8 only).
+template <bool TBIG, int SPAN, int KS, int NT, int BITS>
 __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
     w4a16_dec_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWl,
                      const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmSl,
                      const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmZl,
                      const __grid_constant__ CUtensorMap tmA, const DecParams p, uint16_t* __restrict__ out) {
   using C = DecCfg<TBIG>;
+  static_assert(BITS == 4 || (BITS == 2 && !TBIG), "4-bit codes, or 2-bit codes up to 8 tokens");
+  constexpr int kCodeBoxes = BITS / 2;  // 128-byte boxes of codes per row and stage
   extern __shared__ uint8_t dec_smem_raw[];
   // 1024-byte aligned base by pointer arithmetic on the shared array, so that
   // every access below stays a shared-memory access (ld.shared)
@@ -201,9 +249,12 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
         uint8_t* st = smem + s * p.stage_bytes;
         const int gi0 = (ks * kDecStageK) >> p.group_shift;
         const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
-        mbar_arrive_expect_tx(&tl.full[s], static_cast<uint32_t>(2 * 128 * h + 2 * 512 * p.T + 2 * 2 * p.wg * h));
-        tma_load_2d(st, last ? &tmWl : &tmW, &tl.full[s], ks * 64, row0);
-        tma_load_2d(st + kDecCodeBox, last ? &tmWl : &tmW, &tl.full[s], ks * 64 + 32, row0);
+        mbar_arrive_expect_tx(&tl.full[s],
+                              static_cast<uint32_t>(kCodeBoxes * 128 * h + 2 * 512 * p.T + 2 * 2 * p.wg * h));
+        // 16 BITS words of codes per row and stage, in boxes of 32
+#pragma unroll
+        for (int b = 0; b < kCodeBoxes; ++b)
+          tma_load_2d(st + b * kDecCodeBox, last ? &tmWl : &tmW, &tl.full[s], ks * 16 * BITS + 32 * b, row0);
         tma_load_2d(st + p.act_off, &tmA, &tl.full[s], ks * kDecStageK, 0);
         tma_load_2d(st + p.act_off + 512 * p.T, &tmA, &tl.full[s], ks * kDecStageK + 256, 0);
         tma_load_2d(st + p.tab_off, last ? &tmSl : &tmS, &tl.full[s], x0, row0);
@@ -256,7 +307,104 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
           const uint16_t* zr = sc + p.wg * kDecPassRows;
           const int gi0 = (ks * kDecStageK) >> p.group_shift;
           const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
-          if constexpr (!TBIG) {
+          if constexpr (BITS == 2) {
+            // weights as the A operand as below; per 64-k slice j a lane takes word c of the
+            // slice's 16-byte chunk of its rows (codes k = 64 j + 16 c + 0..15 of the chunk) and
+            // feeds pair i of the word (codes i, i + 8) to k-slots (2c, 2c+1) of MMA i/2 when i is
+            // even, (2c+8, 2c+9) when odd
+            float d[MT][4], o[4];
+            const uint8_t* codes2 = st + g * 128 + 4 * c;
+            const uint8_t* act2 = st + p.act_off + box * 512 * T + ((cw & 1) * 128 + 16 * c) * 2;
+            constexpr uint32_t kQuarter2 = 0x3E803E80u;    // bf16 pair (1/4, 1/4)
+            constexpr uint32_t kSixteenth2 = 0x3D803D80u;  // (1/16, 1/16)
+            constexpr uint32_t kFour2 = 0x40804080u;       // (4, 4)
+            constexpr uint32_t kSixteen2 = 0x41804180u;    // (16, 16)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              // the lane's 16 activations of token column g, paired (k_i, k_{i+8}) and divided by
+              // the scale of code pair i
+              const uint8_t* aj = act2 + tok_lo * 512 + 128 * j;
+              const uint4 v = *reinterpret_cast<const uint4*>(aj);
+              const uint4 u = *reinterpret_cast<const uint4*>(aj + 16);
+              uint32_t b[8];
+              b[0] = __byte_perm(v.x, u.x, 0x5410);
+              b[1] = bf16x2_mul(__byte_perm(v.x, u.x, 0x7632), kQuarter2);
+              b[2] = bf16x2_mul(__byte_perm(v.y, u.y, 0x5410), kSixteenth2);
+              b[3] = __byte_perm(v.y, u.y, 0x7632);
+              b[4] = bf16x2_mul(__byte_perm(v.z, u.z, 0x5410), kQuarter2);
+              b[5] = bf16x2_mul(__byte_perm(v.z, u.z, 0x7632), kSixteenth2);
+              b[6] = __byte_perm(v.w, u.w, 0x5410);
+              b[7] = bf16x2_mul(__byte_perm(v.w, u.w, 0x7632), kQuarter2);
+              const bool first = (j % SPAN) == 0;
+              {
+                // rows 0..7: Oa = sum of the activations (the scale of each pair against its scaled
+                // activations); rows 8..15: Ob = sum of the scaled activations (ones)
+                const uint32_t c0[4] = {kOne2, kOne2, kFour2, kOne2};
+                const uint32_t c1[4] = {kSixteen2, kOne2, kOne2, kOne2};
+                const uint32_t c2[4] = {kFour2, kOne2, kSixteen2, kOne2};
+                if (first) {
+                  mma16816_z(o, c0, b[0], b[1]);
+                } else {
+                  mma16816(o, c0, b[0], b[1]);
+                }
+                mma16816(o, c1, b[2], b[3]);
+                mma16816(o, c2, b[4], b[5]);
+                mma16816(o, c0, b[6], b[7]);
+              }
+              const int q = 2 * cw + j;
+              const uint8_t* cj = codes2 + ((q ^ g) << 4);
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                const bool pair = 2 * mt + 1 < NT;
+                uint32_t rg[8], rh[8];
+                two_bit_pairs(*reinterpret_cast<const uint32_t*>(cj + (2 * mt) * 8 * 128), rg);
+                if (pair) {
+                  two_bit_pairs(*reinterpret_cast<const uint32_t*>(cj + (2 * mt + 1) * 8 * 128), rh);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) rh[i] = 0u;
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                  const uint32_t a[4] = {rg[2 * m], rh[2 * m], rg[2 * m + 1], rh[2 * m + 1]};
+                  if (first && m == 0) {
+                    mma16816_z(d[mt], a, b[0], b[1]);
+                  } else {
+                    mma16816(d[mt], a, b[2 * m], b[2 * m + 1]);
+                  }
+                }
+              }
+              if ((j % SPAN) == SPAN - 1) {
+                // group span done: D = sum (128 / s_k) a_k + sum q a, so acc += s D - s z Oa -
+                // 128 s Ob for rows g, g + 8 of each tile (o[0..1]: Oa, o[2..3]: Ob of tokens 2c, 2c+1)
+                const int gl = ((ks * kDecStageK + cw * 128 + 64 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                __syncwarp();
+#pragma unroll
+                for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
+                  const int row = lane + 32 * rr;
+                  if (row < 8 * NT) {
+                    const float sv = half_bits_to_float(sc[row * p.wg + gl]);
+                    const float zv = half_bits_to_float(zr[row * p.wg + gl]);
+                    smw[row] = make_float2(sv, -sv * zv);
+                  }
+                }
+                __syncwarp();
+                const float ob0 = -128.0f * o[2];
+                const float ob1 = -128.0f * o[3];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                  const float2 mg = smw[16 * mt + g];
+                  acc[mt][0] = fmaf(mg.x, d[mt][0] + ob0, fmaf(mg.y, o[0], acc[mt][0]));
+                  acc[mt][1] = fmaf(mg.x, d[mt][1] + ob1, fmaf(mg.y, o[1], acc[mt][1]));
+                  if (2 * mt + 1 < NT) {
+                    const float2 mh = smw[16 * mt + 8 + g];
+                    acc[mt][2] = fmaf(mh.x, d[mt][2] + ob0, fmaf(mh.y, o[0], acc[mt][2]));
+                    acc[mt][3] = fmaf(mh.x, d[mt][3] + ob1, fmaf(mh.y, o[1], acc[mt][3]));
+                  }
+                }
+              }
+            }
+          } else if constexpr (!TBIG) {
             // weights as the A operand: tile mt holds row groups 2 mt and 2 mt + 1 (rows g and g + 8
             // of the lane); an odd last row group leaves the tile's lower half zero
             float d[MT][4], o[4];
@@ -478,27 +626,35 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
   }
 }
 
-const char* dec_name(bool tbig, int span, int ks, int nt) {
-  // "w4a16_dec_kernel<T<=8,g>=128,nt7>", "...,ksplit2,nt7>"; built once, kept for the process
-  static char names[2][3][2][9][64];
+// group-size class: 0 for g >= 128, 1 for g = 64, 2 for g = 32
+template <int BITS, int SPAN>
+constexpr int dec_gclass() {
+  return BITS == 4 ? (SPAN == 4 ? 0 : (SPAN == 2 ? 1 : 2)) : (SPAN == 2 ? 0 : 1);
+}
+
+const char* dec_name(int bits, bool tbig, int gclass, int ks, int nt) {
+  // "w4a16_dec_kernel<T<=8,g>=128,nt7>", "...,ksplit2,nt7>", "w2a16_dec_kernel<T<=8,g=64,nt8>";
+  // built once, kept for the process
+  static char names[2][2][3][2][9][64];
   static const bool filled = [] {
     const char* gs[3] = {"g>=128", "g=64", "g=32"};
-    for (int a = 0; a < 2; ++a)
-      for (int b = 0; b < 3; ++b)
-        for (int c = 0; c < 2; ++c)
-          for (int d = 1; d <= 8; ++d)
-            snprintf(names[a][b][c][d], sizeof(names[a][b][c][d]), "w4a16_dec_kernel<T<=%d,%s%s,nt%d>", a ? 16 : 8,
-                     gs[b], c ? ",ksplit2" : "", d);
+    for (int w = 0; w < 2; ++w)
+      for (int a = 0; a < 2; ++a)
+        for (int b = 0; b < 3; ++b)
+          for (int c = 0; c < 2; ++c)
+            for (int d = 1; d <= 8; ++d)
+              snprintf(names[w][a][b][c][d], sizeof(names[w][a][b][c][d]), "w%da16_dec_kernel<T<=%d,%s%s,nt%d>",
+                       w ? 2 : 4, a ? 16 : 8, gs[b], c ? ",ksplit2" : "", d);
     return true;
   }();
   (void)filled;
-  return names[tbig ? 1 : 0][span == 4 ? 0 : (span == 2 ? 1 : 2)][ks - 1][nt];
+  return names[bits == 2 ? 1 : 0][tbig ? 1 : 0][gclass][ks - 1][nt];
 }
 
-template <bool TBIG, int SPAN, int KS, int NT>
+template <bool TBIG, int SPAN, int KS, int NT, int BITS>
 cudaError_t launch_dec(const CUtensorMap (&maps)[7], const DecParams& p, int grid, int smem, uint16_t* out,
                        cudaStream_t stream) {
-  auto kern = w4a16_dec_kernel<TBIG, SPAN, KS, NT>;
+  auto kern = w4a16_dec_kernel<TBIG, SPAN, KS, NT, BITS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -513,30 +669,30 @@ cudaError_t launch_dec(const CUtensorMap (&maps)[7], const DecParams& p, int gri
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  LaunchScope scope(stream, dec_name(TBIG, SPAN, KS, NT));
+  LaunchScope scope(stream, dec_name(BITS, TBIG, dec_gclass<BITS, SPAN>(), KS, NT));
   e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], p, out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 // g >= 128 (the common case) has a kernel per tile count; g = 32, 64 run eight tiles
-template <bool TBIG, int SPAN, int KS>
+template <bool TBIG, int SPAN, int KS, int BITS>
 cudaError_t launch_dec_nt(int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid, int smem,
                           uint16_t* out, cudaStream_t stream) {
-  if constexpr (SPAN == 4) {
+  if constexpr (dec_gclass<BITS, SPAN>() == 0) {
     switch (nt) {
-      case 1: return launch_dec<TBIG, SPAN, KS, 1>(maps, p, grid, smem, out, stream);
-      case 2: return launch_dec<TBIG, SPAN, KS, 2>(maps, p, grid, smem, out, stream);
-      case 3: return launch_dec<TBIG, SPAN, KS, 3>(maps, p, grid, smem, out, stream);
-      case 4: return launch_dec<TBIG, SPAN, KS, 4>(maps, p, grid, smem, out, stream);
-      case 5: return launch_dec<TBIG, SPAN, KS, 5>(maps, p, grid, smem, out, stream);
-      case 6: return launch_dec<TBIG, SPAN, KS, 6>(maps, p, grid, smem, out, stream);
-      case 7: return launch_dec<TBIG, SPAN, KS, 7>(maps, p, grid, smem, out, stream);
-      default: return launch_dec<TBIG, SPAN, KS, 8>(maps, p, grid, smem, out, stream);
+      case 1: return launch_dec<TBIG, SPAN, KS, 1, BITS>(maps, p, grid, smem, out, stream);
+      case 2: return launch_dec<TBIG, SPAN, KS, 2, BITS>(maps, p, grid, smem, out, stream);
+      case 3: return launch_dec<TBIG, SPAN, KS, 3, BITS>(maps, p, grid, smem, out, stream);
+      case 4: return launch_dec<TBIG, SPAN, KS, 4, BITS>(maps, p, grid, smem, out, stream);
+      case 5: return launch_dec<TBIG, SPAN, KS, 5, BITS>(maps, p, grid, smem, out, stream);
+      case 6: return launch_dec<TBIG, SPAN, KS, 6, BITS>(maps, p, grid, smem, out, stream);
+      case 7: return launch_dec<TBIG, SPAN, KS, 7, BITS>(maps, p, grid, smem, out, stream);
+      default: return launch_dec<TBIG, SPAN, KS, 8, BITS>(maps, p, grid, smem, out, stream);
     }
   } else {
     (void)nt;
-    return launch_dec<TBIG, SPAN, KS, 8>(maps, p, grid, smem, out, stream);
+    return launch_dec<TBIG, SPAN, KS, 8, BITS>(maps, p, grid, smem, out, stream);
   }
 }
 
@@ -544,26 +700,38 @@ template <bool TBIG>
 cudaError_t launch_dec_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
                             int smem, uint16_t* out, cudaStream_t stream) {
   if (ks == 2) {
-    if (span == 4) return launch_dec_nt<TBIG, 4, 2>(nt, maps, p, grid, smem, out, stream);
-    if (span == 2) return launch_dec_nt<TBIG, 2, 2>(nt, maps, p, grid, smem, out, stream);
-    return launch_dec_nt<TBIG, 1, 2>(nt, maps, p, grid, smem, out, stream);
+    if (span == 4) return launch_dec_nt<TBIG, 4, 2, 4>(nt, maps, p, grid, smem, out, stream);
+    if (span == 2) return launch_dec_nt<TBIG, 2, 2, 4>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<TBIG, 1, 2, 4>(nt, maps, p, grid, smem, out, stream);
   }
-  if (span == 4) return launch_dec_nt<TBIG, 4, 1>(nt, maps, p, grid, smem, out, stream);
-  if (span == 2) return launch_dec_nt<TBIG, 2, 1>(nt, maps, p, grid, smem, out, stream);
-  return launch_dec_nt<TBIG, 1, 1>(nt, maps, p, grid, smem, out, stream);
+  if (span == 4) return launch_dec_nt<TBIG, 4, 1, 4>(nt, maps, p, grid, smem, out, stream);
+  if (span == 2) return launch_dec_nt<TBIG, 2, 1, 4>(nt, maps, p, grid, smem, out, stream);
+  return launch_dec_nt<TBIG, 1, 1, 4>(nt, maps, p, grid, smem, out, stream);
+}
+
+// 2-bit codes, T <= 8: span 2 (g >= 128) or 1 (g = 64)
+cudaError_t launch_dec2_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
+                             int smem, uint16_t* out, cudaStream_t stream) {
+  if (ks == 2) {
+    if (span == 2) return launch_dec_nt<false, 2, 2, 2>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<false, 1, 2, 2>(nt, maps, p, grid, smem, out, stream);
+  }
+  if (span == 2) return launch_dec_nt<false, 2, 1, 2>(nt, maps, p, grid, smem, out, stream);
+  return launch_dec_nt<false, 1, 1, 2>(nt, maps, p, grid, smem, out, stream);
 }
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-}  // namespace
-
 // Returns cudaErrorNotSupported (nothing launched) when the shape does not fit
 // this kernel's tensor maps: the scale/zero row stride must be a multiple of 16
-// bytes (K/g a multiple of 8) and the scale/zero arrays 16-byte aligned.
-cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
-                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
-                             cudaStream_t stream) {
+// bytes (K/g a multiple of 8) and the scale/zero arrays 16-byte aligned; 2-bit
+// codes also need T <= 8, g >= 64 (a 64-k slice inside one group) and K >= 512
+// (a row of codes at least one box wide).
+cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                            const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,
+                            cudaStream_t stream) {
   if (T < 1 || T > 16 || N < 1 || K < 128 || K % 128 != 0 || group_size < 32) return cudaErrorNotSupported;
+  if (bits != 4 && (bits != 2 || T > 8 || group_size < 64 || K < kDecStageK)) return cudaErrorNotSupported;
   const int G = K / group_size;
   if (G % 8 != 0 || (reinterpret_cast<uintptr_t>(scale16) & 15u) || (reinterpret_cast<uintptr_t>(zero16) & 15u))
     return cudaErrorNotSupported;
@@ -600,13 +768,13 @@ cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, c
 
   const bool tbig = T > 8;
   const int red_bytes = tbig ? DecCfg<true>::kRedBytes : DecCfg<false>::kRedBytes;
-  p.act_off = 2 * kDecCodeBox;
+  p.act_off = (bits / 2) * kDecCodeBox;
   p.tab_off = p.act_off + round_up(2 * 512 * T, 128);
   p.stage_bytes = round_up(p.tab_off + 2 * 2 * p.wg * kDecPassRows, 1024);
   const int fixed = red_bytes + static_cast<int>(sizeof(DecTail)) + 1024;
   // ring depth: a multiple of the consumer groups (each slot always taken by the same group)
   const int groups = tbig ? DecCfg<true>::kGroups : DecCfg<false>::kGroups;
-  p.S = std::min(kDecMaxStages, (kDecSmemLimit - fixed) / p.stage_bytes) / groups * groups;
+  p.S = std::min(bits == 4 ? kDecMaxStages : kDecMaxStages2, (kDecSmemLimit - fixed) / p.stage_bytes) / groups * groups;
   if (p.S < 2 * groups) return cudaErrorNotSupported;
   const int smem = dec_tail_offset(p.S, p.stage_bytes, red_bytes) + static_cast<int>(sizeof(DecTail)) + 1024;
 
@@ -614,7 +782,8 @@ cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, c
   const int heights[2] = {std::min(kDecPassRows, rows), p.last_rows};
   for (int m = 0; m < 2; ++m) {
     e = make_tmap_2d(&maps[m], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, static_cast<uint64_t>(N),
-                     static_cast<uint64_t>(K / 8), 32, static_cast<uint32_t>(heights[m]), CU_TENSOR_MAP_SWIZZLE_128B);
+                     static_cast<uint64_t>(K / (32 / bits)), 32, static_cast<uint32_t>(heights[m]),
+                     CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     e = make_tmap_2d(&maps[2 + m], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scale16, static_cast<uint64_t>(N),
                      static_cast<uint64_t>(G), static_cast<uint32_t>(p.wg), static_cast<uint32_t>(heights[m]),
@@ -629,10 +798,25 @@ cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, c
                    256, static_cast<uint32_t>(T), CU_TENSOR_MAP_SWIZZLE_NONE);
   if (e != cudaSuccess) return e;
 
-  const int span = group_size >= 128 ? 4 : group_size / 32;
   const int nt = p.passes == 1 ? rows / 8 : 8;  // tiles of a full pass
+  if (bits == 2) return launch_dec2_span(group_size >= 128 ? 2 : 1, ks, nt, maps, p, grid, smem, out, stream);
+  const int span = group_size >= 128 ? 4 : group_size / 32;
   return tbig ? launch_dec_span<true>(span, ks, nt, maps, p, grid, smem, out, stream)
               : launch_dec_span<false>(span, ks, nt, maps, p, grid, smem, out, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_w4a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
+                             cudaStream_t stream) {
+  return launch_dec_bits(A, T, packed, scale16, zero16, N, K, group_size, 4, out, stream);
+}
+
+cudaError_t launch_w2a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
+                             cudaStream_t stream) {
+  return launch_dec_bits(A, T, packed, scale16, zero16, N, K, group_size, 2, out, stream);
 }
 
 }  // namespace ar

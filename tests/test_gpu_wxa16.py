@@ -73,7 +73,9 @@ def test_wxa16_matches_oracle(ar, bits, T, N, K, g):
     out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, bits, out)
     assert ar.ar_get_device_status() == 0
-    if bits in (2, 3) and T <= 8:
+    if bits == 2 and T <= 8 and g >= 64 and (K // g) % 8 == 0:
+        assert "w2a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    elif bits in (2, 3) and T <= 8:
         assert "wbx_dec_kernel<b=%d" % bits in ar.ar_last_kernels()
     else:
         assert "wxa16_tc_kernel<b=%d" % bits in ar.ar_last_kernels()
@@ -139,4 +141,77 @@ def test_wxa16_three_bit_full_size_sampled_rows(ar, T):
     assert np.array_equal(packed.cpu().numpy().view(np.uint32)[rows], words)
     ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16)[rows],
                          z16.cpu().numpy().view(np.uint16)[rows], g, 3)
+    assert rel_l2(out.float().cpu().numpy()[:, rows], ref) <= TC_RTOL
+
+
+@pytest.mark.parametrize("T", [1, 5, 8])
+@pytest.mark.parametrize("N,K,g,tag", [
+    (10000, 512, 64, "g=64,nt8>"),              # 72 rows per CTA: two row passes (64 + 8); last CTA one pass
+    (10000, 1024, 128, "g>=128,nt8>"),          # the same passes with one group per 128-k chunk
+    (4096, 2048, 128, "g>=128,ksplit2,nt7>"),   # 56-row CTA pairs splitting K
+    (296, 4096, 256, "g>=128,ksplit2,nt1>"),    # 8-row CTA pairs
+    (1001, 1024, 128, "g>=128,nt1>"),           # the last CTA holds one row
+])
+def test_w2a16_decode_row_ranges_match_oracle(ar, T, N, K, g, tag):
+    """2-bit codes up to 8 tokens on the W4A16 decode kernel's 2-bit form (16 codes a word,
+    codes taken at three mantissa positions, activations scaled to match)."""
+    d = synth.make_linear(N, K, 1, seed=T + N + 2)
+    V, a, b = synth.make_state(N, K, g, seed=2, spread=True)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 2, g)
+    A = synth.make_activations(T, K, seed=T)
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 2, out)
+    assert ar.ar_get_device_status() == 0
+    kern = ar.ar_last_kernels()
+    assert "w2a16_dec_kernel<T<=8,%s" % tag in kern, kern
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 2, g)
+    words = O.pack_bitstream(st["q"], 2)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16),
+                         z16.cpu().numpy().view(np.uint16), g, 2)
+    got = out.float().cpu().numpy()
+    assert rel_l2(got, ref) <= TC_RTOL
+    # each token on its own, and the first and last rows (the ends of the row ranges)
+    for t in range(T):
+        assert rel_l2(got[t], ref[t]) <= TC_RTOL
+    assert rel_l2(got[:, :8], ref[:, :8]) <= TC_RTOL and rel_l2(got[:, -8:], ref[:, -8:]) <= TC_RTOL
+
+
+def test_w2a16_decode_extreme_codes(ar):
+    """All-zero and all-three code rows (every code at each of the three mantissa positions at
+    its extreme) against the oracle: rows alternate between q = 0 and q = 3 words."""
+    N, K, g, T = 64, 1024, 128, 3
+    words = np.zeros((N, K // 16), np.uint32)
+    words[1::2] = 0xFFFFFFFF
+    s16 = np.full((N, K // g), 0.0123, np.float16)
+    z16 = np.tile(np.array([0.0, 1.0, 2.0, 3.0], np.float16), (N, K // g // 4))
+    A = synth.make_activations(T, K, seed=5)
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), torch.from_numpy(words.view(np.int32)).cuda(), torch.from_numpy(s16).cuda(),
+                     torch.from_numpy(z16).cuda(), g, 2, out)
+    assert ar.ar_get_device_status() == 0
+    assert "w2a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.view(np.uint16), z16.view(np.uint16), g, 2)
+    assert rel_l2(out.float().cpu().numpy(), ref) <= TC_RTOL
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_w2a16_decode_full_size_sampled_rows(ar, T):
+    """8192 x 28672 down projection at 2 bits (g 128) on the decode kernel, sampled output rows
+    against the oracle."""
+    wl = synth.WORKLOADS["down_8192_28672"]
+    N, K, g = wl.n_out, wl.n_in, wl.group_size
+    d = synth.make_linear(N, K, 1, seed=wl.seed, x_outlier_channels=0)
+    V, a, b = synth.make_state(N, K, g)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 2, g)
+    A = synth.make_activations(T, K, seed=1)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 2, out)
+    assert ar.ar_get_device_status() == 0
+    assert "w2a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    rows = np.sort(np.random.default_rng(7).choice(N, 64, replace=False))
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"][rows]), V[rows], a[rows], b[rows], 2, g)
+    words = O.pack_bitstream(st["q"], 2)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32)[rows], words)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16)[rows],
+                         z16.cpu().numpy().view(np.uint16)[rows], g, 2)
     assert rel_l2(out.float().cpu().numpy()[:, rows], ref) <= TC_RTOL
