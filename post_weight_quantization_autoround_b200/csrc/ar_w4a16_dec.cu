@@ -199,7 +199,11 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                      const __grid_constant__ CUtensorMap tmA, const DecParams p, uint16_t* __restrict__ out) {
   using C = DecCfg<TBIG>;
   static_assert(BITS == 4 || (BITS == 2 && !TBIG), "4-bit codes, or 2-bit codes up to 8 tokens");
-  constexpr int kCodeBoxes = BITS / 2;  // 128-byte boxes of codes per row and stage
+  // k per stage: 512 for 4-bit codes, 1024 for 2-bit codes, so that a stage is two 128-byte
+  // boxes of codes per row either way (256 contiguous bytes of each row)
+  constexpr int kStageK = BITS == 2 ? 2 * kDecStageK : kDecStageK;
+  constexpr int kCodeBoxes = 2;
+  constexpr int kActBoxes = kStageK / 256;  // 256-k boxes of activations per stage
   extern __shared__ uint8_t dec_smem_raw[];
   // 1024-byte aligned base by pointer arithmetic on the shared array, so that
   // every access below stays a shared-memory access (ld.shared)
@@ -247,16 +251,17 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
         const int h = last ? p.last_rows : kDecPassRows;
         const int row0 = row_base + pass * kDecPassRows;
         uint8_t* st = smem + s * p.stage_bytes;
-        const int gi0 = (ks * kDecStageK) >> p.group_shift;
+        const int gi0 = (ks * kStageK) >> p.group_shift;
         const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
-        mbar_arrive_expect_tx(&tl.full[s],
-                              static_cast<uint32_t>(kCodeBoxes * 128 * h + 2 * 512 * p.T + 2 * 2 * p.wg * h));
-        // 16 BITS words of codes per row and stage, in boxes of 32
+        mbar_arrive_expect_tx(&tl.full[s], static_cast<uint32_t>(kCodeBoxes * 128 * h + kActBoxes * 512 * p.T +
+                                                                 2 * 2 * p.wg * h));
+        // 64 words of codes per row and stage, in boxes of 32
 #pragma unroll
         for (int b = 0; b < kCodeBoxes; ++b)
-          tma_load_2d(st + b * kDecCodeBox, last ? &tmWl : &tmW, &tl.full[s], ks * 16 * BITS + 32 * b, row0);
-        tma_load_2d(st + p.act_off, &tmA, &tl.full[s], ks * kDecStageK, 0);
-        tma_load_2d(st + p.act_off + 512 * p.T, &tmA, &tl.full[s], ks * kDecStageK + 256, 0);
+          tma_load_2d(st + b * kDecCodeBox, last ? &tmWl : &tmW, &tl.full[s], ks * 64 + 32 * b, row0);
+#pragma unroll
+        for (int b = 0; b < kActBoxes; ++b)
+          tma_load_2d(st + p.act_off + b * 512 * p.T, &tmA, &tl.full[s], ks * kStageK + 256 * b, 0);
         tma_load_2d(st + p.tab_off, last ? &tmSl : &tmS, &tl.full[s], x0, row0);
         tma_load_2d(st + p.tab_off + 2 * p.wg * kDecPassRows, last ? &tmZl : &tmZ, &tl.full[s], x0, row0);
         ++issued;
@@ -305,22 +310,23 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
           const uint8_t* act = st + p.act_off + box * 512 * T + (((cw & 1) * 128 + 8 * c) * 2);
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + p.tab_off);
           const uint16_t* zr = sc + p.wg * kDecPassRows;
-          const int gi0 = (ks * kDecStageK) >> p.group_shift;
+          const int gi0 = (ks * kStageK) >> p.group_shift;
           const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
           if constexpr (BITS == 2) {
-            // weights as the A operand as below; per 64-k slice j a lane takes word c of the
-            // slice's 16-byte chunk of its rows (codes k = 64 j + 16 c + 0..15 of the chunk) and
-            // feeds pair i of the word (codes i, i + 8) to k-slots (2c, 2c+1) of MMA i/2 when i is
-            // even, (2c+8, 2c+9) when odd
+            // weights as the A operand as below; warp cw takes k 256 cw .. 256 cw + 255 of the
+            // stage (half of code box cw / 2, all of activation box cw).  Per 64-k slice j a lane
+            // takes word c of the slice's 16-byte chunk of its rows (codes k = 64 j + 16 c + 0..15
+            // of the warp's range) and feeds pair i of the word (codes i, i + 8) to k-slots
+            // (2c, 2c+1) of MMA i/2 when i is even, (2c+8, 2c+9) when odd
             float d[MT][4], o[4];
-            const uint8_t* codes2 = st + g * 128 + 4 * c;
-            const uint8_t* act2 = st + p.act_off + box * 512 * T + ((cw & 1) * 128 + 16 * c) * 2;
+            const uint8_t* codes2 = st + box * kDecCodeBox + g * 128 + 4 * c;
+            const uint8_t* act2 = st + p.act_off + cw * 512 * T + 16 * c * 2;
             constexpr uint32_t kQuarter2 = 0x3E803E80u;    // bf16 pair (1/4, 1/4)
             constexpr uint32_t kSixteenth2 = 0x3D803D80u;  // (1/16, 1/16)
             constexpr uint32_t kFour2 = 0x40804080u;       // (4, 4)
             constexpr uint32_t kSixteen2 = 0x41804180u;    // (16, 16)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
+            for (int j = 0; j < 4; ++j) {
               // the lane's 16 activations of token column g, paired (k_i, k_{i+8}) and divided by
               // the scale of code pair i
               const uint8_t* aj = act2 + tok_lo * 512 + 128 * j;
@@ -351,7 +357,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                 mma16816(o, c2, b[4], b[5]);
                 mma16816(o, c0, b[6], b[7]);
               }
-              const int q = 2 * cw + j;
+              const int q = (cw & 1) * 4 + j;
               const uint8_t* cj = codes2 + ((q ^ g) << 4);
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) {
@@ -377,7 +383,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               if ((j % SPAN) == SPAN - 1) {
                 // group span done: D = sum (128 / s_k) a_k + sum q a, so acc += s D - s z Oa -
                 // 128 s Ob for rows g, g + 8 of each tile (o[0..1]: Oa, o[2..3]: Ob of tokens 2c, 2c+1)
-                const int gl = ((ks * kDecStageK + cw * 128 + 64 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                const int gl = ((ks * kStageK + cw * 256 + 64 * (j - SPAN + 1)) >> p.group_shift) - x0;
                 __syncwarp();
 #pragma unroll
                 for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
@@ -452,7 +458,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               }
               if ((j % SPAN) == SPAN - 1) {
                 // group span done: acc += s D - s (128 + z) O for rows g, g + 8 of each tile
-                const int gl = ((ks * kDecStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                const int gl = ((ks * kStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
                 __syncwarp();
 #pragma unroll
                 for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
@@ -528,7 +534,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               // group span done: acc += s D - s (128 + z) O for weight rows 2c, 2c + 1 of each tile.
               // The warp first converts the group's fp16 (scale, zero) of the pass's rows once
               // (two rows per lane) into fp32 (s, -s (128 + z)) pairs.
-              const int gl = ((ks * kDecStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
+              const int gl = ((ks * kStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
               __syncwarp();
 #pragma unroll
               for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
@@ -745,11 +751,12 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   p.N = N;
   p.K = K;
   p.T = T;
-  p.n_stages = (K + kDecStageK - 1) / kDecStageK;
+  const int stage_k = bits == 2 ? 2 * kDecStageK : kDecStageK;
+  p.n_stages = (K + stage_k - 1) / stage_k;
   int gs = 0;
   while ((1 << gs) < group_size) ++gs;
   p.group_shift = gs;
-  p.wg = group_size == 32 ? 16 : 8;
+  p.wg = stage_k / group_size >= 16 ? 16 : 8;  // a window of the groups a stage touches
 
   // rows per CTA (multiple of 8) with one CTA per SM; a cluster pair splits K
   // instead when that halves the rows a CTA streams (small N)
@@ -768,8 +775,8 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
 
   const bool tbig = T > 8;
   const int red_bytes = tbig ? DecCfg<true>::kRedBytes : DecCfg<false>::kRedBytes;
-  p.act_off = (bits / 2) * kDecCodeBox;
-  p.tab_off = p.act_off + round_up(2 * 512 * T, 128);
+  p.act_off = 2 * kDecCodeBox;
+  p.tab_off = p.act_off + round_up(2 * stage_k * T, 128);
   p.stage_bytes = round_up(p.tab_off + 2 * 2 * p.wg * kDecPassRows, 1024);
   const int fixed = red_bytes + static_cast<int>(sizeof(DecTail)) + 1024;
   // ring depth: a multiple of the consumer groups (each slot always taken by the same group)
