@@ -191,7 +191,7 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t h) { return __half2
 // tiles per pass, a compile-time count so that the tile loops are straight-line
 // code (tiles past a pass's rows read rows of the stage buffer that the pass
 // does not own and are computed but never stored).  BITS: 4, or 2 (T <= 8 only).
-template <bool TBIG, int SPAN, int KS, int NT, int BITS>
+template <bool TBIG, int SPAN, int KS, int NT, int BITS, int STAGEK>
 __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
     w4a16_dec_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWl,
                      const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmSl,
@@ -199,10 +199,11 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                      const __grid_constant__ CUtensorMap tmA, const DecParams p, uint16_t* __restrict__ out) {
   using C = DecCfg<TBIG>;
   static_assert(BITS == 4 || (BITS == 2 && !TBIG), "4-bit codes, or 2-bit codes up to 8 tokens");
-  // k per stage: 512 for 4-bit codes, 1024 for 2-bit codes, so that a stage is two 128-byte
-  // boxes of codes per row either way (256 contiguous bytes of each row)
-  constexpr int kStageK = BITS == 2 ? 2 * kDecStageK : kDecStageK;
-  constexpr int kCodeBoxes = 2;
+  // k per stage (512 or 1024; 2-bit codes: 1024); a stage holds kStageK * BITS / 1024 128-byte
+  // boxes of codes per row, contiguous in the row
+  constexpr int kStageK = STAGEK;
+  static_assert((kStageK == 512 || kStageK == 1024) && (BITS == 4 || kStageK == 1024), "stage size");
+  constexpr int kCodeBoxes = kStageK * BITS / 1024;
   constexpr int kActBoxes = kStageK / 256;  // 256-k boxes of activations per stage
   extern __shared__ uint8_t dec_smem_raw[];
   // 1024-byte aligned base by pointer arithmetic on the shared array, so that
@@ -252,13 +253,13 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
         const int row0 = row_base + pass * kDecPassRows;
         uint8_t* st = smem + s * p.stage_bytes;
         const int gi0 = (ks * kStageK) >> p.group_shift;
-        const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
+        const int x0 = p.wg >= 16 ? gi0 : (gi0 & ~7);
         mbar_arrive_expect_tx(&tl.full[s], static_cast<uint32_t>(kCodeBoxes * 128 * h + kActBoxes * 512 * p.T +
                                                                  2 * 2 * p.wg * h));
-        // 64 words of codes per row and stage, in boxes of 32
+        // kStageK * BITS / 32 words of codes per row and stage, in boxes of 32
 #pragma unroll
         for (int b = 0; b < kCodeBoxes; ++b)
-          tma_load_2d(st + b * kDecCodeBox, last ? &tmWl : &tmW, &tl.full[s], ks * 64 + 32 * b, row0);
+          tma_load_2d(st + b * kDecCodeBox, last ? &tmWl : &tmW, &tl.full[s], ks * 32 * kCodeBoxes + 32 * b, row0);
 #pragma unroll
         for (int b = 0; b < kActBoxes; ++b)
           tma_load_2d(st + p.act_off + b * 512 * p.T, &tmA, &tl.full[s], ks * kStageK + 256 * b, 0);
@@ -278,7 +279,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
     const int T = p.T;
     const int tok_lo = min(g, T - 1);
     const int tok_hi = min(g + 8, T - 1);
-    const int box = cw >> 1;
+    const int kw0 = cw * (kStageK / 4);  // k offset of the warp's quarter of a stage
     const uint32_t kOne2 = 0x3F803F80u;  // bf16 pair (1, 1)
     bool ok = true;
 
@@ -306,27 +307,28 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
         if (__all_sync(0xFFFFFFFFu, ok)) {
           const int ks = ks0 + (it - it_begin);
           const uint8_t* st = smem + s * p.stage_bytes;
-          const uint8_t* codes = st + box * kDecCodeBox + g * 128 + 4 * c;
-          const uint8_t* act = st + p.act_off + box * 512 * T + (((cw & 1) * 128 + 8 * c) * 2);
+          // 4-bit codes: a box is 256 k of a row; activations: a box is 256 k of each token
+          const uint8_t* codes = st + (kw0 >> 8) * kDecCodeBox + g * 128 + 4 * c;
+          const uint8_t* act = st + p.act_off + (kw0 >> 8) * 512 * T + (((kw0 & 255) + 8 * c) * 2);
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + p.tab_off);
           const uint16_t* zr = sc + p.wg * kDecPassRows;
           const int gi0 = (ks * kStageK) >> p.group_shift;
-          const int x0 = p.wg == 16 ? gi0 : (gi0 & ~7);
+          const int x0 = p.wg >= 16 ? gi0 : (gi0 & ~7);
           if constexpr (BITS == 2) {
             // weights as the A operand as below; warp cw takes k 256 cw .. 256 cw + 255 of the
-            // stage (half of code box cw / 2, all of activation box cw).  Per 64-k slice j a lane
+            // stage (half of code box cw / 2 of 512 k, all of activation box cw).  Per 64-k slice j a lane
             // takes word c of the slice's 16-byte chunk of its rows (codes k = 64 j + 16 c + 0..15
             // of the warp's range) and feeds pair i of the word (codes i, i + 8) to k-slots
             // (2c, 2c+1) of MMA i/2 when i is even, (2c+8, 2c+9) when odd
             float d[MT][4], o[4];
-            const uint8_t* codes2 = st + box * kDecCodeBox + g * 128 + 4 * c;
-            const uint8_t* act2 = st + p.act_off + cw * 512 * T + 16 * c * 2;
+            const uint8_t* codes2 = st + (kw0 >> 9) * kDecCodeBox + g * 128 + 4 * c;
+            const uint8_t* act2 = st + p.act_off + (kw0 >> 8) * 512 * T + ((kw0 & 255) + 16 * c) * 2;
             constexpr uint32_t kQuarter2 = 0x3E803E80u;    // bf16 pair (1/4, 1/4)
             constexpr uint32_t kSixteenth2 = 0x3D803D80u;  // (1/16, 1/16)
             constexpr uint32_t kFour2 = 0x40804080u;       // (4, 4)
             constexpr uint32_t kSixteen2 = 0x41804180u;    // (16, 16)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < kStageK / 256; ++j) {
               // the lane's 16 activations of token column g, paired (k_i, k_{i+8}) and divided by
               // the scale of code pair i
               const uint8_t* aj = act2 + tok_lo * 512 + 128 * j;
@@ -357,7 +359,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                 mma16816(o, c2, b[4], b[5]);
                 mma16816(o, c0, b[6], b[7]);
               }
-              const int q = (cw & 1) * 4 + j;
+              const int q = ((kw0 & 511) >> 6) + j;
               const uint8_t* cj = codes2 + ((q ^ g) << 4);
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) {
@@ -383,7 +385,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               if ((j % SPAN) == SPAN - 1) {
                 // group span done: D = sum (128 / s_k) a_k + sum q a, so acc += s D - s z Oa -
                 // 128 s Ob for rows g, g + 8 of each tile (o[0..1]: Oa, o[2..3]: Ob of tokens 2c, 2c+1)
-                const int gl = ((ks * kStageK + cw * 256 + 64 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                const int gl = ((ks * kStageK + kw0 + 64 * (j - SPAN + 1)) >> p.group_shift) - x0;
                 __syncwarp();
 #pragma unroll
                 for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
@@ -415,7 +417,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
             // of the lane); an odd last row group leaves the tile's lower half zero
             float d[MT][4], o[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < kStageK / 128; ++j) {
               // activations of this lane's k-range (eight bf16) for token column g
               const uint4 v = *reinterpret_cast<const uint4*>(act + tok_lo * 512 + 64 * j);
               const uint32_t b0[2] = {__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632)};  // (k0,k4) (k1,k5)
@@ -428,7 +430,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                 mma16816(o, ones, b0[0], b0[1]);
               }
               mma16816(o, ones, b1[0], b1[1]);
-              const int q = (cw & 1) * 4 + j;
+              const int q = ((kw0 & 255) >> 5) + j;
               const uint8_t* cj = codes + ((q ^ g) << 4);
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) {
@@ -458,7 +460,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               }
               if ((j % SPAN) == SPAN - 1) {
                 // group span done: acc += s D - s (128 + z) O for rows g, g + 8 of each tile
-                const int gl = ((ks * kStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                const int gl = ((ks * kStageK + kw0 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
                 __syncwarp();
 #pragma unroll
                 for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
@@ -486,7 +488,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
           } else {
           float d[NT][4], o[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < kStageK / 128; ++j) {
             // activations of this lane's k-range (eight bf16) for token rows g and g + 8
             const uint4 v = *reinterpret_cast<const uint4*>(act + tok_lo * 512 + 64 * j);
             uint32_t A0[4], A1[4];
@@ -511,7 +513,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
             }
             mma16816(o, A1, kOne2, kOne2);
             // 16-byte chunk q of the 128-byte row, stored at chunk q ^ (row % 8) = q ^ g
-            const int q = (cw & 1) * 4 + j;
+            const int q = ((kw0 & 255) >> 5) + j;
             const uint8_t* cj = codes + ((q ^ g) << 4);
 #pragma unroll
             for (int jt = 0; jt < NT; ++jt) {
@@ -534,7 +536,7 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
               // group span done: acc += s D - s (128 + z) O for weight rows 2c, 2c + 1 of each tile.
               // The warp first converts the group's fp16 (scale, zero) of the pass's rows once
               // (two rows per lane) into fp32 (s, -s (128 + z)) pairs.
-              const int gl = ((ks * kStageK + cw * 128 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
+              const int gl = ((ks * kStageK + kw0 + 32 * (j - SPAN + 1)) >> p.group_shift) - x0;
               __syncwarp();
 #pragma unroll
               for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
@@ -657,10 +659,10 @@ const char* dec_name(int bits, bool tbig, int gclass, int ks, int nt) {
   return names[bits == 2 ? 1 : 0][tbig ? 1 : 0][gclass][ks - 1][nt];
 }
 
-template <bool TBIG, int SPAN, int KS, int NT, int BITS>
+template <bool TBIG, int SPAN, int KS, int NT, int BITS, int STAGEK>
 cudaError_t launch_dec(const CUtensorMap (&maps)[7], const DecParams& p, int grid, int smem, uint16_t* out,
                        cudaStream_t stream) {
-  auto kern = w4a16_dec_kernel<TBIG, SPAN, KS, NT, BITS>;
+  auto kern = w4a16_dec_kernel<TBIG, SPAN, KS, NT, BITS, STAGEK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -682,48 +684,49 @@ cudaError_t launch_dec(const CUtensorMap (&maps)[7], const DecParams& p, int gri
 }
 
 // g >= 128 (the common case) has a kernel per tile count; g = 32, 64 run eight tiles
-template <bool TBIG, int SPAN, int KS, int BITS>
+template <bool TBIG, int SPAN, int KS, int BITS, int STAGEK>
 cudaError_t launch_dec_nt(int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid, int smem,
                           uint16_t* out, cudaStream_t stream) {
   if constexpr (dec_gclass<BITS, SPAN>() == 0) {
     switch (nt) {
-      case 1: return launch_dec<TBIG, SPAN, KS, 1, BITS>(maps, p, grid, smem, out, stream);
-      case 2: return launch_dec<TBIG, SPAN, KS, 2, BITS>(maps, p, grid, smem, out, stream);
-      case 3: return launch_dec<TBIG, SPAN, KS, 3, BITS>(maps, p, grid, smem, out, stream);
-      case 4: return launch_dec<TBIG, SPAN, KS, 4, BITS>(maps, p, grid, smem, out, stream);
-      case 5: return launch_dec<TBIG, SPAN, KS, 5, BITS>(maps, p, grid, smem, out, stream);
-      case 6: return launch_dec<TBIG, SPAN, KS, 6, BITS>(maps, p, grid, smem, out, stream);
-      case 7: return launch_dec<TBIG, SPAN, KS, 7, BITS>(maps, p, grid, smem, out, stream);
-      default: return launch_dec<TBIG, SPAN, KS, 8, BITS>(maps, p, grid, smem, out, stream);
+      case 1: return launch_dec<TBIG, SPAN, KS, 1, BITS, STAGEK>(maps, p, grid, smem, out, stream);
+      case 2: return launch_dec<TBIG, SPAN, KS, 2, BITS, STAGEK>(maps, p, grid, smem, out, stream);
+      case 3: return launch_dec<TBIG, SPAN, KS, 3, BITS, STAGEK>(maps, p, grid, smem, out, stream);
+      case 4: return launch_dec<TBIG, SPAN, KS, 4, BITS, STAGEK>(maps, p, grid, smem, out, stream);
+      case 5: return launch_dec<TBIG, SPAN, KS, 5, BITS, STAGEK>(maps, p, grid, smem, out, stream);
+      case 6: return launch_dec<TBIG, SPAN, KS, 6, BITS, STAGEK>(maps, p, grid, smem, out, stream);
+      case 7: return launch_dec<TBIG, SPAN, KS, 7, BITS, STAGEK>(maps, p, grid, smem, out, stream);
+      default: return launch_dec<TBIG, SPAN, KS, 8, BITS, STAGEK>(maps, p, grid, smem, out, stream);
     }
   } else {
     (void)nt;
-    return launch_dec<TBIG, SPAN, KS, 8, BITS>(maps, p, grid, smem, out, stream);
+    return launch_dec<TBIG, SPAN, KS, 8, BITS, STAGEK>(maps, p, grid, smem, out, stream);
   }
 }
 
-template <bool TBIG>
+// 4-bit codes
+template <bool TBIG, int STAGEK>
 cudaError_t launch_dec_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
                             int smem, uint16_t* out, cudaStream_t stream) {
   if (ks == 2) {
-    if (span == 4) return launch_dec_nt<TBIG, 4, 2, 4>(nt, maps, p, grid, smem, out, stream);
-    if (span == 2) return launch_dec_nt<TBIG, 2, 2, 4>(nt, maps, p, grid, smem, out, stream);
-    return launch_dec_nt<TBIG, 1, 2, 4>(nt, maps, p, grid, smem, out, stream);
+    if (span == 4) return launch_dec_nt<TBIG, 4, 2, 4, STAGEK>(nt, maps, p, grid, smem, out, stream);
+    if (span == 2) return launch_dec_nt<TBIG, 2, 2, 4, STAGEK>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<TBIG, 1, 2, 4, STAGEK>(nt, maps, p, grid, smem, out, stream);
   }
-  if (span == 4) return launch_dec_nt<TBIG, 4, 1, 4>(nt, maps, p, grid, smem, out, stream);
-  if (span == 2) return launch_dec_nt<TBIG, 2, 1, 4>(nt, maps, p, grid, smem, out, stream);
-  return launch_dec_nt<TBIG, 1, 1, 4>(nt, maps, p, grid, smem, out, stream);
+  if (span == 4) return launch_dec_nt<TBIG, 4, 1, 4, STAGEK>(nt, maps, p, grid, smem, out, stream);
+  if (span == 2) return launch_dec_nt<TBIG, 2, 1, 4, STAGEK>(nt, maps, p, grid, smem, out, stream);
+  return launch_dec_nt<TBIG, 1, 1, 4, STAGEK>(nt, maps, p, grid, smem, out, stream);
 }
 
-// 2-bit codes, T <= 8: span 2 (g >= 128) or 1 (g = 64)
+// 2-bit codes, T <= 8, 1024-k stages: span 2 (g >= 128) or 1 (g = 64)
 cudaError_t launch_dec2_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
                              int smem, uint16_t* out, cudaStream_t stream) {
   if (ks == 2) {
-    if (span == 2) return launch_dec_nt<false, 2, 2, 2>(nt, maps, p, grid, smem, out, stream);
-    return launch_dec_nt<false, 1, 2, 2>(nt, maps, p, grid, smem, out, stream);
+    if (span == 2) return launch_dec_nt<false, 2, 2, 2, 1024>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<false, 1, 2, 2, 1024>(nt, maps, p, grid, smem, out, stream);
   }
-  if (span == 2) return launch_dec_nt<false, 2, 1, 2>(nt, maps, p, grid, smem, out, stream);
-  return launch_dec_nt<false, 1, 1, 2>(nt, maps, p, grid, smem, out, stream);
+  if (span == 2) return launch_dec_nt<false, 2, 1, 2, 1024>(nt, maps, p, grid, smem, out, stream);
+  return launch_dec_nt<false, 1, 1, 2, 1024>(nt, maps, p, grid, smem, out, stream);
 }
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
@@ -751,12 +754,32 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   p.N = N;
   p.K = K;
   p.T = T;
-  const int stage_k = bits == 2 ? 2 * kDecStageK : kDecStageK;
-  p.n_stages = (K + stage_k - 1) / stage_k;
   int gs = 0;
   while ((1 << gs) < group_size) ++gs;
   p.group_shift = gs;
-  p.wg = stage_k / group_size >= 16 ? 16 : 8;  // a window of the groups a stage touches
+
+  const bool tbig = T > 8;
+  const int red_bytes = tbig ? DecCfg<true>::kRedBytes : DecCfg<false>::kRedBytes;
+  const int fixed = red_bytes + static_cast<int>(sizeof(DecTail)) + 1024;
+  // ring depth: a multiple of the consumer groups (each slot always taken by the same group)
+  const int groups = tbig ? DecCfg<true>::kGroups : DecCfg<false>::kGroups;
+  // stage layout for stage_k k per stage: codes, activations, scale table, zero table; false
+  // when fewer than two stages per consumer group fit
+  auto layout = [&](int stage_k) {
+    p.n_stages = (K + stage_k - 1) / stage_k;
+    p.wg = std::max(8, stage_k / group_size);  // a window of the groups a stage touches
+    p.act_off = (stage_k * bits / 1024) * kDecCodeBox;
+    p.tab_off = p.act_off + round_up(2 * stage_k * T, 128);
+    p.stage_bytes = round_up(p.tab_off + 2 * 2 * p.wg * kDecPassRows, 1024);
+    p.S = std::min(bits == 4 ? kDecMaxStages : kDecMaxStages2, (kDecSmemLimit - fixed) / p.stage_bytes) / groups *
+          groups;
+    return p.S >= 2 * groups;
+  };
+  // 1024-k stages (half the per-stage costs) unless the ring would be too shallow; 9..16 tokens
+  // keep 512-k stages
+  int stage_k = 1024;
+  if (bits == 4 && (tbig || !layout(1024))) stage_k = 512;
+  if (!layout(stage_k)) return cudaErrorNotSupported;
 
   // rows per CTA (multiple of 8) with one CTA per SM; a cluster pair splits K
   // instead when that halves the rows a CTA streams (small N)
@@ -772,17 +795,6 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   p.passes = (rows + kDecPassRows - 1) / kDecPassRows;
   p.last_rows = rows - (p.passes - 1) * kDecPassRows;
   const int grid = ks * ((N + rows - 1) / rows);
-
-  const bool tbig = T > 8;
-  const int red_bytes = tbig ? DecCfg<true>::kRedBytes : DecCfg<false>::kRedBytes;
-  p.act_off = 2 * kDecCodeBox;
-  p.tab_off = p.act_off + round_up(2 * stage_k * T, 128);
-  p.stage_bytes = round_up(p.tab_off + 2 * 2 * p.wg * kDecPassRows, 1024);
-  const int fixed = red_bytes + static_cast<int>(sizeof(DecTail)) + 1024;
-  // ring depth: a multiple of the consumer groups (each slot always taken by the same group)
-  const int groups = tbig ? DecCfg<true>::kGroups : DecCfg<false>::kGroups;
-  p.S = std::min(bits == 4 ? kDecMaxStages : kDecMaxStages2, (kDecSmemLimit - fixed) / p.stage_bytes) / groups * groups;
-  if (p.S < 2 * groups) return cudaErrorNotSupported;
   const int smem = dec_tail_offset(p.S, p.stage_bytes, red_bytes) + static_cast<int>(sizeof(DecTail)) + 1024;
 
   CUtensorMap maps[7];
@@ -808,8 +820,9 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   const int nt = p.passes == 1 ? rows / 8 : 8;  // tiles of a full pass
   if (bits == 2) return launch_dec2_span(group_size >= 128 ? 2 : 1, ks, nt, maps, p, grid, smem, out, stream);
   const int span = group_size >= 128 ? 4 : group_size / 32;
-  return tbig ? launch_dec_span<true>(span, ks, nt, maps, p, grid, smem, out, stream)
-              : launch_dec_span<false>(span, ks, nt, maps, p, grid, smem, out, stream);
+  if (tbig) return launch_dec_span<true, 512>(span, ks, nt, maps, p, grid, smem, out, stream);
+  return stage_k == 1024 ? launch_dec_span<false, 1024>(span, ks, nt, maps, p, grid, smem, out, stream)
+                         : launch_dec_span<false, 512>(span, ks, nt, maps, p, grid, smem, out, stream);
 }
 
 }  // namespace
