@@ -29,12 +29,15 @@
 //    32-bit word (eight codes, k = 32j + 8c + 0..7) of a weight row, and the
 //    activations are permuted the same way with byte permutes.  Both operand
 //    arrangements use the same k-slots, so they give bit-identical sums.
-//  * One producer warp streams 512-k stages with TMA: the codes of the pass's
-//    rows (two 256-k boxes, 128-byte swizzle, so that the fragment reads are
-//    free of bank conflicts), the activations, and the window of fp16
-//    (scale, zero) groups the stage touches.  Consumer warps work in groups of
-//    four (one 128-k chunk each) and the groups take stages in turn, so each
-//    warp owns whole group spans of its chunk.  The ring depth is a multiple
+//  * One producer warp streams stages of 1024 k (up to 8 tokens, where four
+//    stages fit in shared memory) or 512 k with TMA: the codes of the pass's
+//    rows (256-k boxes, 128-byte swizzle, so that the fragment reads are free
+//    of bank conflicts), the activations, and the window of fp16 (scale, zero)
+//    groups the stage touches.  Consumer warps work in groups of four (one
+//    quarter of the stage each) and the groups take stages in turn, so each
+//    warp owns whole group spans of its chunk.  The costs per stage (barrier
+//    waits, the table boxes) are what 1024-k stages halve: 42 -> 36 us for the
+//    8192 x 28672 layer at T = 1.  The ring depth is a multiple
 //    of the number of groups, so a slot is always taken by the same group and
 //    its waits on the slot's barrier follow the barrier's phases in order (a
 //    parity wait cannot tell a phase from the one two before it: were two
@@ -50,9 +53,10 @@
 // bits 4*(k mod 8) of word k/8; scale/zero fp16 [N][K/g].
 //
 // The same kernel takes 2-bit codes (ar_pack_codes' stream: element k at bits
-// 2*(k mod 16) of word k/16) up to 8 tokens for g >= 64.  A 512-k stage is one
-// 128-byte box per row, and a lane's 32-bit word holds 16 codes, so a 128-k
-// chunk is two 64-k slices of four MMAs each (weights as the A operand).  The
+// 2*(k mod 16) of word k/16) up to 8 tokens for g >= 64.  A stage is always
+// 1024 k (two 128-byte boxes per row), and a lane's 32-bit word holds 16 codes,
+// so a warp's 256-k quarter is four 64-k slices of four MMAs each (weights as
+// the A operand).  The
 // codes are not shifted down one by one: (x & (3 << 2m)) | 0x4300 for
 // m = 0, 1, 2 is the bf16 128 + 4^m q, since bits 0..6 are the mantissa of a
 // bf16 in [128, 256), so one word needs two shifts (by 6 and 12) and eight
