@@ -81,7 +81,7 @@ constexpr int kDecStageK = 512;                 // k per stage
 constexpr int kDecPassRows = 64;                // rows per pass (eight n8 tiles)
 constexpr int kDecCodeBox = kDecPassRows * 128; // one 256-k box of codes: 64 rows x 128 bytes
 constexpr int kDecMaxStages = 8;               // ring depth cap, 4-bit codes (two boxes per stage)
-constexpr int kDecMaxStages2 = 16;             // ... 2-bit codes (one box per stage)
+constexpr int kDecMaxStages2 = 16;             // ... 2-bit codes
 constexpr int kDecSmemLimit = 227 * 1024;
 
 template <bool TBIG>
@@ -206,7 +206,8 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
   // k per stage (512 or 1024; 2-bit codes: 1024); a stage holds kStageK * BITS / 1024 128-byte
   // boxes of codes per row, contiguous in the row
   constexpr int kStageK = STAGEK;
-  static_assert((kStageK == 512 || kStageK == 1024) && (BITS == 4 || kStageK == 1024), "stage size");
+  static_assert(BITS == 4 ? (kStageK == 512 || kStageK == 1024) : (kStageK == 1024 || kStageK == 2048),
+                "stage size");
   constexpr int kCodeBoxes = kStageK * BITS / 1024;
   constexpr int kActBoxes = kStageK / 256;  // 256-k boxes of activations per stage
   extern __shared__ uint8_t dec_smem_raw[];
@@ -319,14 +320,14 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
           const int gi0 = (ks * kStageK) >> p.group_shift;
           const int x0 = p.wg >= 16 ? gi0 : (gi0 & ~7);
           if constexpr (BITS == 2) {
-            // weights as the A operand as below; warp cw takes k 256 cw .. 256 cw + 255 of the
-            // stage (half of code box cw / 2 of 512 k, all of activation box cw).  Per 64-k slice j a lane
+            // weights as the A operand as below; warp cw takes the k range kw0 .. kw0 + kStageK / 4 - 1
+            // of the stage (code boxes hold 512 k, activation boxes 256 k).  Per 64-k slice j a lane
             // takes word c of the slice's 16-byte chunk of its rows (codes k = 64 j + 16 c + 0..15
             // of the warp's range) and feeds pair i of the word (codes i, i + 8) to k-slots
             // (2c, 2c+1) of MMA i/2 when i is even, (2c+8, 2c+9) when odd
             float d[MT][4], o[4];
             const uint8_t* codes2 = st + (kw0 >> 9) * kDecCodeBox + g * 128 + 4 * c;
-            const uint8_t* act2 = st + p.act_off + (kw0 >> 8) * 512 * T + ((kw0 & 255) + 16 * c) * 2;
+            const uint8_t* act2 = st + p.act_off + 16 * c * 2;
             constexpr uint32_t kQuarter2 = 0x3E803E80u;    // bf16 pair (1/4, 1/4)
             constexpr uint32_t kSixteenth2 = 0x3D803D80u;  // (1/16, 1/16)
             constexpr uint32_t kFour2 = 0x40804080u;       // (4, 4)
@@ -335,7 +336,8 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
             for (int j = 0; j < kStageK / 256; ++j) {
               // the lane's 16 activations of token column g, paired (k_i, k_{i+8}) and divided by
               // the scale of code pair i
-              const uint8_t* aj = act2 + tok_lo * 512 + 128 * j;
+              const int kj = kw0 + 64 * j;  // k of the slice in the stage: box kj / 256 of each token
+              const uint8_t* aj = act2 + (kj >> 8) * 512 * T + (kj & 255) * 2 + tok_lo * 512;
               const uint4 v = *reinterpret_cast<const uint4*>(aj);
               const uint4 u = *reinterpret_cast<const uint4*>(aj + 16);
               uint32_t b[8];
@@ -722,15 +724,22 @@ cudaError_t launch_dec_span(int span, int ks, int nt, const CUtensorMap (&maps)[
   return launch_dec_nt<TBIG, 1, 1, 4, STAGEK>(nt, maps, p, grid, smem, out, stream);
 }
 
-// 2-bit codes, T <= 8, 1024-k stages: span 2 (g >= 128) or 1 (g = 64)
+// 2-bit codes, T <= 8, 1024-k stages: span 2 (g >= 128) or 1 (g = 64); 2048-k stages: g >= 128
+template <int STAGEK>
 cudaError_t launch_dec2_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
                              int smem, uint16_t* out, cudaStream_t stream) {
-  if (ks == 2) {
-    if (span == 2) return launch_dec_nt<false, 2, 2, 2, 1024>(nt, maps, p, grid, smem, out, stream);
-    return launch_dec_nt<false, 1, 2, 2, 1024>(nt, maps, p, grid, smem, out, stream);
+  if constexpr (STAGEK == 2048) {
+    (void)span;
+    return ks == 2 ? launch_dec_nt<false, 2, 2, 2, STAGEK>(nt, maps, p, grid, smem, out, stream)
+                   : launch_dec_nt<false, 2, 1, 2, STAGEK>(nt, maps, p, grid, smem, out, stream);
+  } else {
+    if (ks == 2) {
+      if (span == 2) return launch_dec_nt<false, 2, 2, 2, STAGEK>(nt, maps, p, grid, smem, out, stream);
+      return launch_dec_nt<false, 1, 2, 2, STAGEK>(nt, maps, p, grid, smem, out, stream);
+    }
+    if (span == 2) return launch_dec_nt<false, 2, 1, 2, STAGEK>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<false, 1, 1, 2, STAGEK>(nt, maps, p, grid, smem, out, stream);
   }
-  if (span == 2) return launch_dec_nt<false, 2, 1, 2, 1024>(nt, maps, p, grid, smem, out, stream);
-  return launch_dec_nt<false, 1, 1, 2, 1024>(nt, maps, p, grid, smem, out, stream);
 }
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
@@ -780,9 +789,13 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
     return p.S >= 2 * groups;
   };
   // 1024-k stages (half the per-stage costs) unless the ring would be too shallow; 9..16 tokens
-  // keep 512-k stages
+  // keep 512-k stages.  2-bit codes: 2048-k stages for one token at g >= 128 where four fit and K
+  // holds two of them (so a small N can still split K over a CTA pair), else 1024 (measured on the
+  // 8192 x 28672 layer: T = 1 g 128 30.8 against 32.8 us; T = 2 the same; g = 64 slower, 38.9
+  // against 34.8 us, from its 32-group table windows and spills)
   int stage_k = 1024;
   if (bits == 4 && (tbig || !layout(1024))) stage_k = 512;
+  if (bits == 2 && T == 1 && group_size >= 128 && K >= 4096 && layout(2048)) stage_k = 2048;
   if (!layout(stage_k)) return cudaErrorNotSupported;
 
   // rows per CTA (multiple of 8) with one CTA per SM; a cluster pair splits K
@@ -822,7 +835,11 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   if (e != cudaSuccess) return e;
 
   const int nt = p.passes == 1 ? rows / 8 : 8;  // tiles of a full pass
-  if (bits == 2) return launch_dec2_span(group_size >= 128 ? 2 : 1, ks, nt, maps, p, grid, smem, out, stream);
+  if (bits == 2) {
+    const int span2 = group_size >= 128 ? 2 : 1;
+    return stage_k == 2048 ? launch_dec2_span<2048>(span2, ks, nt, maps, p, grid, smem, out, stream)
+                           : launch_dec2_span<1024>(span2, ks, nt, maps, p, grid, smem, out, stream);
+  }
   const int span = group_size >= 128 ? 4 : group_size / 32;
   if (tbig) return launch_dec_span<true, 512>(span, ks, nt, maps, p, grid, smem, out, stream);
   return stage_k == 1024 ? launch_dec_span<false, 1024>(span, ks, nt, maps, p, grid, smem, out, stream)

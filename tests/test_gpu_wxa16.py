@@ -151,6 +151,9 @@ def test_wxa16_three_bit_full_size_sampled_rows(ar, T):
     (4096, 2048, 128, "g>=128,ksplit2,nt7>"),   # 56-row CTA pairs splitting K
     (296, 4096, 256, "g>=128,ksplit2,nt1>"),    # 8-row CTA pairs
     (1001, 1024, 128, "g>=128,nt1>"),           # the last CTA holds one row
+    (10000, 4096, 128, "g>=128,nt8>"),          # two row passes; 2048-k stages at T = 1
+    (2000, 8192, 64, "g=64,nt8>"),              # 16-row CTAs, eight 1024-k stages with 16-group windows
+    (296, 8192, 128, "g>=128,ksplit2,nt1>"),    # 8-row CTA pairs, each CTA two 2048-k stages at T = 1
 ])
 def test_w2a16_decode_row_ranges_match_oracle(ar, T, N, K, g, tag):
     """2-bit codes up to 8 tokens on the W4A16 decode kernel's 2-bit form (16 codes a word,
