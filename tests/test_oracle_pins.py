@@ -425,6 +425,57 @@ def test_small_workload_tuning_lowers_the_loss():
     assert final < losses[0]
 
 
+def test_tune_linear_follows_the_closed_form_sign_trajectory():
+    """tune_linear on a case whose trajectory is known without the oracle ([AR] §3 "SignSGD" and the
+    "Minimal State-Evolution Example": each step moves a parameter by lr against its gradient's sign).
+
+    One row, one group of 32 bf16 weights with range [-1.875, 1.875] (s = 0.25, zp = round(7.5) = 8 at
+    4 bits), one token of ones, and a target of 100, above the largest reachable output (32 x 7 x 0.25
+    = 56): the residual, hence dL/dW_hat, is negative at every step, so every weight whose code is in
+    range (0 <= t <= 15) has dV = g s m < 0 and V rises by exactly lr (capped at 0.5), while a weight
+    whose code left the range (m = 0) has dV = 0 and keeps its V.  alpha, beta are held at 1 by
+    clip_min = clip_max = 1, so s and zp stay fixed, and each code flips when 4w + V crosses its
+    rounding point.  Every value is a multiple of 2^-5 (lr = 1/32), so the loss sequence, the final
+    loss and the final V are exact.  A flipped gradient sign, a missing range mask, a step of the
+    wrong size, state not carried between steps or the loss of the wrong state fails here.
+    """
+    x4 = np.array([7.5, -7.5, 7.25, 6.75, 3.15625, -3.15625, 0.46875, -0.46875, 2.5, -2.5, 0.0, 1.03125,
+                   -1.96875, 5.90625, -6.09375, 4.5, -4.5, 0.21875, -0.78125, 3.84375, -3.84375, 6.0, -6.0,
+                   1.5, -1.5, 2.28125, -2.71875, 0.65625, 5.34375, -5.34375, 7.0, -7.0], np.float32)
+    W = (x4 / 4).reshape(1, 32).astype(np.float32)
+    assert np.array_equal(O.bf16_rne(W), W)
+    X = np.ones((1, 32), np.float32)
+    Y = np.array([[100.0]], np.float32)
+    lr, steps = 2.0 ** -5, 24
+    cfg = O.QConfig(bits=4, group_size=32, lr=lr, clip_min=1.0, clip_max=1.0)
+    V0 = np.zeros((1, 32), np.float32)
+    one = np.ones((1, 1), np.float32)
+    losses, (V, a, b), final = O.tune_linear(W, X, V0, one, one, cfg, steps, Y=Y)
+
+    def rha(v):  # round half away from zero, exact for these multiples of 2^-5
+        return np.sign(v) * np.floor(np.abs(v) + 0.5)
+
+    v = np.zeros(32)
+    expect = []
+    for _ in range(steps + 1):
+        t = rha(x4.astype(np.float64) + v) + 8
+        m = (t >= 0) & (t <= 15)
+        expect.append((np.sum((np.clip(t, 0, 15) - 8) * 0.25) - 100.0) ** 2)
+        v = np.where(m, np.minimum(v + lr, 0.5), v)
+    # the trajectory is not trivial: codes flip, some weights freeze at the clamp, some at v_max
+    assert len(set(expect)) > 5
+    assert np.array_equal(np.asarray(losses), np.array(expect[:steps]))
+    assert final == expect[steps]
+    # V after `steps` updates: the loop above ran one update past the last state; redo it exactly
+    v = np.zeros(32)
+    for _ in range(steps):
+        t = rha(x4.astype(np.float64) + v) + 8
+        v = np.where((t >= 0) & (t <= 15), np.minimum(v + lr, 0.5), v)
+    assert np.array_equal(V.astype(np.float64), v.reshape(1, 32))
+    assert np.any(v == 0.5) and np.any((v > 0) & (v < 0.5))  # capped, and frozen mid-way by the range mask
+    assert np.array_equal(a, one) and np.array_equal(b, one)
+
+
 def test_fp32_instantiation_agrees_with_fp64():
     """The fp32 path (the GPU's rounding points) stays within bf16 precision of the fp64 path.
 
@@ -515,8 +566,13 @@ def test_mlp_ste_gradients_match_finite_differences():
                 assert dref[n, j] == pytest.approx((f(sp) - f(sm)) / (2 * h), rel=1e-5, abs=1e-12)
 
 
-def test_mlp_fp32_instantiation_agrees_with_fp64():
-    rng = np.random.default_rng(14)
+@pytest.mark.parametrize("seed", [14, 2, 5])
+def test_mlp_fp32_instantiation_agrees_with_fp64(seed):
+    """The fp32 branch differs from the fp64 one only by its bf16 rounding points (a, b, h, G, dA, dB:
+    relative 2^-9 each, about four in series on a gradient path), so its loss is within 5e-3 and its
+    folded gradients within 2e-2 (about ten such roundings) in relative L2; measured at most 2.4e-3 and
+    9.8e-3 over six seeds."""
+    rng = np.random.default_rng(seed)
     M, H, F, g = 32, 128, 96, 32
     Ws = [O.bf16_rne((rng.standard_normal(s) * 0.05).astype(np.float32)) for s in ((F, H), (F, H), (H, F))]
     X = O.bf16_rne(rng.standard_normal((M, H)).astype(np.float32))
@@ -529,12 +585,12 @@ def test_mlp_fp32_instantiation_agrees_with_fp64():
     # the same step with every rounding point kept in fp64
     fw64 = O.mlp_forward(X, sts[0]["What_bf16"], sts[1]["What_bf16"], sts[2]["What_bf16"], dtype=np.float64)
     R = fw64["y"] - np.asarray(Y, np.float64)
-    assert L == pytest.approx(np.mean(R ** 2), rel=2e-2)
+    assert L == pytest.approx(np.mean(R ** 2), rel=5e-3)
     gWg, gWu, gWd, _ = O.mlp_backward(X, fw64, 2 * R / R.size, sts[2]["What_bf16"], dtype=np.float64)
     rel = lambda x, y: np.linalg.norm(x - y) / np.linalg.norm(y)
     for gr, g64, W, st in zip(grads, (gWg, gWu, gWd), Ws, sts):
         dV64, da64, db64 = O.ste_fold(g64, W, st, 4)
-        assert rel(gr["dV"], dV64) < 5e-2 and rel(gr["dalpha"], da64) < 5e-2
+        assert rel(gr["dV"], dV64) < 2e-2 and rel(gr["dalpha"], da64) < 2e-2 and rel(gr["dbeta"], db64) < 2e-2
 
 
 # ----------------------------------------------------------------------------
