@@ -376,13 +376,13 @@ AR_API ar_status ar_pack_codes(const uint16_t* W, const float* V, const float* a
 /* WbA16 matmul for codes packed by ar_pack_codes (bits 2, 3, 4 or 8):
  *   out[t][n] = sum_k A[t][k] (q[n][k] - zero[n][k/g]) scale[n][k/g]
  * A bf16 [T][K]; zero must hold integers 0..2^bits-1; out bf16 [T][N].  bits 4
- * is ar_w4a16_gemm.  2 bits at T <= 8 with group_size >= 64, K/group_size a
- * multiple of 8 and K >= 512 run the W4A16 decode kernel's 2-bit form (16
- * codes a word, taken at three mantissa positions of a bf16 with the paired
- * activations scaled by 4^-m); other 2 and 3-bit shapes at T <= 8 run a
- * generic decode kernel (mma.sync, one range of weight rows per SM, the codes
- * read straight from the bit stream); 8 bits, and 2 and 3 bits from 9 tokens,
- * run the tcgen05 dequant
+ * is ar_w4a16_gemm.  At T <= 8 with K/group_size a multiple of 8, 2 bits
+ * (group_size >= 64, K >= 512) and 8 bits run the W4A16 decode kernel's 2-bit
+ * and 8-bit forms (codes taken at mantissa positions of a bf16 with the paired
+ * activations scaled to match; an 8-bit code as its two nibbles); other 2 and
+ * 3-bit shapes at T <= 8 run a generic decode kernel (mma.sync, one range of
+ * weight rows per SM, the codes read straight from the bit stream); the rest,
+ * and every width from 9 tokens, run the tcgen05 dequant
  * GEMM (a 3-bit stage of 128 k is 48 bytes of a row: its code slots hold
  * three 128-byte boxes, eight stages).  (q - z) is exact in bf16 for every width and
  * each group's sum is scaled once in fp32.  Needs 1 <= T < 2^31, group_size

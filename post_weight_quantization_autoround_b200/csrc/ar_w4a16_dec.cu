@@ -66,6 +66,12 @@
 // constant fragment gives both corrections: rows 0..7 hold the class weights
 // 4^m (Oa = sum of a), rows 8..15 ones (Ob = sum of a / 4^m), and a group adds
 // s (D - 128 Ob) - s z Oa.
+//
+// 8-bit codes (T <= 8; 512-k stages, four boxes per row) are split into their
+// nibbles: (x & 0x000F000F) | 0x4300 is (128 + lo_0, 128 + lo_2), and
+// ((x >> 1) & 0x00780078) | 0x4300, the high nibbles at mantissa bits 3..6, is
+// (128 + 8 hi_0, 128 + 8 hi_2), paired with doubled activations; a code then
+// contributes 384 a + q a, and a group adds s D - s (384 + z) O.
 #include <cooperative_groups.h>
 
 #include <cstdio>
@@ -202,11 +208,13 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                      const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmZl,
                      const __grid_constant__ CUtensorMap tmA, const DecParams p, uint16_t* __restrict__ out) {
   using C = DecCfg<TBIG>;
-  static_assert(BITS == 4 || (BITS == 2 && !TBIG), "4-bit codes, or 2-bit codes up to 8 tokens");
+  static_assert(BITS == 4 || ((BITS == 2 || BITS == 8) && !TBIG), "4-bit codes, or 2/8-bit codes up to 8 tokens");
   // k per stage (512 or 1024; 2-bit codes: 1024); a stage holds kStageK * BITS / 1024 128-byte
   // boxes of codes per row, contiguous in the row
   constexpr int kStageK = STAGEK;
-  static_assert(BITS == 4 ? (kStageK == 512 || kStageK == 1024) : (kStageK == 1024 || kStageK == 2048),
+  static_assert(BITS == 4   ? (kStageK == 512 || kStageK == 1024)
+                : BITS == 2 ? (kStageK == 1024 || kStageK == 2048)
+                            : kStageK == 512,
                 "stage size");
   constexpr int kCodeBoxes = kStageK * BITS / 1024;
   constexpr int kActBoxes = kStageK / 256;  // 256-k boxes of activations per stage
@@ -319,7 +327,91 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
           const uint16_t* zr = sc + p.wg * kDecPassRows;
           const int gi0 = (ks * kStageK) >> p.group_shift;
           const int x0 = p.wg >= 16 ? gi0 : (gi0 & ~7);
-          if constexpr (BITS == 2) {
+          if constexpr (BITS == 8) {
+            // weights as the A operand as below; warp cw takes k kw0 .. kw0 + 127 (code box cw of
+            // 128 k, half of activation box cw / 2).  Per 16-k chunk j a lane takes word c of the
+            // chunk (codes k = 16 j + 4 c + 0..3) of its rows; each code is split into nibbles:
+            // (x & 0x000F000F) | 0x4300 is the pair (128 + lo_0, 128 + lo_2) and
+            // ((x >> 1) & 0x00780078) | 0x4300 the pair (128 + 8 hi_0, 128 + 8 hi_2), paired with
+            // the activations (a_0, a_2) and (2 a_0, 2 a_2) in k-slots (2c, 2c+1) and (2c+8, 2c+9) of
+            // MMA 0 (codes 1, 3 likewise in MMA 1), so a code contributes 384 a + q a
+            float d[MT][4], o[4];
+            const uint8_t* codes8 = st + (kw0 >> 7) * kDecCodeBox + g * 128 + 4 * c;
+            const uint8_t* act8 = st + p.act_off + (kw0 >> 8) * 512 * T + ((kw0 & 255) + 4 * c) * 2;
+            constexpr uint32_t kTwo2 = 0x40004000u;  // bf16 pair (2, 2)
+#pragma unroll
+            for (int j = 0; j < kStageK / 64; ++j) {
+              const uint2 v = *reinterpret_cast<const uint2*>(act8 + tok_lo * 512 + 32 * j);
+              const uint32_t p02 = __byte_perm(v.x, v.y, 0x5410);  // (a_0, a_2)
+              const uint32_t p13 = __byte_perm(v.x, v.y, 0x7632);  // (a_1, a_3)
+              const uint32_t b0[2] = {p02, bf16x2_mul(p02, kTwo2)};
+              const uint32_t b1[2] = {p13, bf16x2_mul(p13, kTwo2)};
+              const bool first = (j % SPAN) == 0;
+              {
+                // O = sum of the activations: ones against the low-nibble slots, zeros against the high
+                const uint32_t ones[4] = {kOne2, kOne2, 0u, 0u};
+                if (first) {
+                  mma16816_z(o, ones, b0[0], b0[1]);
+                } else {
+                  mma16816(o, ones, b0[0], b0[1]);
+                }
+                mma16816(o, ones, b1[0], b1[1]);
+              }
+              const uint8_t* cj = codes8 + ((((kw0 & 127) >> 4) + j) ^ g) * 16;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                const bool pair = 2 * mt + 1 < NT;
+                const uint32_t xg = *reinterpret_cast<const uint32_t*>(cj + (2 * mt) * 8 * 128);
+                const uint32_t xh = pair ? *reinterpret_cast<const uint32_t*>(cj + (2 * mt + 1) * 8 * 128) : 0u;
+                const uint32_t yg = shr(xg, 8), yh = shr(xh, 8);
+                uint32_t a0[4], a1[4];
+                a0[0] = nib_pair(xg);
+                a0[2] = mask_pair<0x00780078u>(shr(xg, 1));
+                a1[0] = nib_pair(yg);
+                a1[2] = mask_pair<0x00780078u>(shr(xg, 9));
+                if (pair) {
+                  a0[1] = nib_pair(xh);
+                  a0[3] = mask_pair<0x00780078u>(shr(xh, 1));
+                  a1[1] = nib_pair(yh);
+                  a1[3] = mask_pair<0x00780078u>(shr(xh, 9));
+                } else {
+                  a0[1] = a0[3] = a1[1] = a1[3] = 0u;
+                }
+                if (first) {
+                  mma16816_z(d[mt], a0, b0[0], b0[1]);
+                } else {
+                  mma16816(d[mt], a0, b0[0], b0[1]);
+                }
+                mma16816(d[mt], a1, b1[0], b1[1]);
+              }
+              if ((j % SPAN) == SPAN - 1) {
+                // group span done: acc += s D - s (384 + z) O for rows g, g + 8 of each tile
+                const int gl = ((ks * kStageK + kw0 + 16 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                __syncwarp();
+#pragma unroll
+                for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
+                  const int row = lane + 32 * rr;
+                  if (row < 8 * NT) {
+                    const float sv = half_bits_to_float(sc[row * p.wg + gl]);
+                    const float zv = half_bits_to_float(zr[row * p.wg + gl]);
+                    smw[row] = make_float2(sv, -sv * (384.0f + zv));
+                  }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                  const float2 mg = smw[16 * mt + g];
+                  acc[mt][0] = fmaf(mg.x, d[mt][0], fmaf(mg.y, o[0], acc[mt][0]));
+                  acc[mt][1] = fmaf(mg.x, d[mt][1], fmaf(mg.y, o[1], acc[mt][1]));
+                  if (2 * mt + 1 < NT) {
+                    const float2 mh = smw[16 * mt + 8 + g];
+                    acc[mt][2] = fmaf(mh.x, d[mt][2], fmaf(mh.y, o[2], acc[mt][2]));
+                    acc[mt][3] = fmaf(mh.x, d[mt][3], fmaf(mh.y, o[3], acc[mt][3]));
+                  }
+                }
+              }
+            }
+          } else if constexpr (BITS == 2) {
             // weights as the A operand as below; warp cw takes the k range kw0 .. kw0 + kStageK / 4 - 1
             // of the stage (code boxes hold 512 k, activation boxes 256 k).  Per 64-k slice j a lane
             // takes word c of the slice's 16-byte chunk of its rows (codes k = 64 j + 16 c + 0..15
@@ -643,26 +735,29 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
 // group-size class: 0 for g >= 128, 1 for g = 64, 2 for g = 32
 template <int BITS, int SPAN>
 constexpr int dec_gclass() {
-  return BITS == 4 ? (SPAN == 4 ? 0 : (SPAN == 2 ? 1 : 2)) : (SPAN == 2 ? 0 : 1);
+  return BITS == 4   ? (SPAN == 4 ? 0 : (SPAN == 2 ? 1 : 2))
+         : BITS == 2 ? (SPAN == 2 ? 0 : 1)
+                     : (SPAN == 8 ? 0 : (SPAN == 4 ? 1 : 2));
 }
 
 const char* dec_name(int bits, bool tbig, int gclass, int ks, int nt) {
   // "w4a16_dec_kernel<T<=8,g>=128,nt7>", "...,ksplit2,nt7>", "w2a16_dec_kernel<T<=8,g=64,nt8>";
   // built once, kept for the process
-  static char names[2][2][3][2][9][64];
+  static char names[3][2][3][2][9][64];
   static const bool filled = [] {
     const char* gs[3] = {"g>=128", "g=64", "g=32"};
-    for (int w = 0; w < 2; ++w)
+    const int widths[3] = {4, 2, 8};
+    for (int w = 0; w < 3; ++w)
       for (int a = 0; a < 2; ++a)
         for (int b = 0; b < 3; ++b)
           for (int c = 0; c < 2; ++c)
             for (int d = 1; d <= 8; ++d)
               snprintf(names[w][a][b][c][d], sizeof(names[w][a][b][c][d]), "w%da16_dec_kernel<T<=%d,%s%s,nt%d>",
-                       w ? 2 : 4, a ? 16 : 8, gs[b], c ? ",ksplit2" : "", d);
+                       widths[w], a ? 16 : 8, gs[b], c ? ",ksplit2" : "", d);
     return true;
   }();
   (void)filled;
-  return names[bits == 2 ? 1 : 0][tbig ? 1 : 0][gclass][ks - 1][nt];
+  return names[bits == 2 ? 1 : (bits == 8 ? 2 : 0)][tbig ? 1 : 0][gclass][ks - 1][nt];
 }
 
 template <bool TBIG, int SPAN, int KS, int NT, int BITS, int STAGEK>
@@ -742,6 +837,19 @@ cudaError_t launch_dec2_span(int span, int ks, int nt, const CUtensorMap (&maps)
   }
 }
 
+// 8-bit codes, T <= 8, 512-k stages: span 8 (g >= 128), 4 (g = 64) or 2 (g = 32) 16-k chunks
+cudaError_t launch_dec8_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
+                             int smem, uint16_t* out, cudaStream_t stream) {
+  if (ks == 2) {
+    if (span == 8) return launch_dec_nt<false, 8, 2, 8, 512>(nt, maps, p, grid, smem, out, stream);
+    if (span == 4) return launch_dec_nt<false, 4, 2, 8, 512>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<false, 2, 2, 8, 512>(nt, maps, p, grid, smem, out, stream);
+  }
+  if (span == 8) return launch_dec_nt<false, 8, 1, 8, 512>(nt, maps, p, grid, smem, out, stream);
+  if (span == 4) return launch_dec_nt<false, 4, 1, 8, 512>(nt, maps, p, grid, smem, out, stream);
+  return launch_dec_nt<false, 2, 1, 8, 512>(nt, maps, p, grid, smem, out, stream);
+}
+
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Returns cudaErrorNotSupported (nothing launched) when the shape does not fit
@@ -753,7 +861,9 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
                             const uint16_t* zero16, int N, int K, int group_size, int bits, uint16_t* out,
                             cudaStream_t stream) {
   if (T < 1 || T > 16 || N < 1 || K < 128 || K % 128 != 0 || group_size < 32) return cudaErrorNotSupported;
-  if (bits != 4 && (bits != 2 || T > 8 || group_size < 64 || K < kDecStageK)) return cudaErrorNotSupported;
+  if (bits == 2 && (T > 8 || group_size < 64 || K < kDecStageK)) return cudaErrorNotSupported;
+  if (bits == 8 && T > 8) return cudaErrorNotSupported;
+  if (bits != 2 && bits != 4 && bits != 8) return cudaErrorNotSupported;
   const int G = K / group_size;
   if (G % 8 != 0 || (reinterpret_cast<uintptr_t>(scale16) & 15u) || (reinterpret_cast<uintptr_t>(zero16) & 15u))
     return cudaErrorNotSupported;
@@ -793,7 +903,7 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   // holds two of them (so a small N can still split K over a CTA pair), else 1024 (measured on the
   // 8192 x 28672 layer: T = 1 g 128 30.8 against 32.8 us; T = 2 the same; g = 64 slower, 38.9
   // against 34.8 us, from its 32-group table windows and spills)
-  int stage_k = 1024;
+  int stage_k = bits == 8 ? 512 : 1024;
   if (bits == 4 && (tbig || !layout(1024))) stage_k = 512;
   if (bits == 2 && T == 1 && group_size >= 128 && K >= 4096 && layout(2048)) stage_k = 2048;
   if (!layout(stage_k)) return cudaErrorNotSupported;
@@ -835,6 +945,7 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   if (e != cudaSuccess) return e;
 
   const int nt = p.passes == 1 ? rows / 8 : 8;  // tiles of a full pass
+  if (bits == 8) return launch_dec8_span(std::min(8, group_size / 16), ks, nt, maps, p, grid, smem, out, stream);
   if (bits == 2) {
     const int span2 = group_size >= 128 ? 2 : 1;
     return stage_k == 2048 ? launch_dec2_span<2048>(span2, ks, nt, maps, p, grid, smem, out, stream)
@@ -858,6 +969,12 @@ cudaError_t launch_w2a16_dec(const uint16_t* A, int T, const uint32_t* packed, c
                              const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
                              cudaStream_t stream) {
   return launch_dec_bits(A, T, packed, scale16, zero16, N, K, group_size, 2, out, stream);
+}
+
+cudaError_t launch_w8a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
+                             cudaStream_t stream) {
+  return launch_dec_bits(A, T, packed, scale16, zero16, N, K, group_size, 8, out, stream);
 }
 
 }  // namespace ar

@@ -75,6 +75,8 @@ def test_wxa16_matches_oracle(ar, bits, T, N, K, g):
     assert ar.ar_get_device_status() == 0
     if bits == 2 and T <= 8 and g >= 64 and (K // g) % 8 == 0:
         assert "w2a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    elif bits == 8 and T <= 8 and (K // g) % 8 == 0:
+        assert "w8a16_dec_kernel<T<=8" in ar.ar_last_kernels()
     elif bits in (2, 3) and T <= 8:
         assert "wbx_dec_kernel<b=%d" % bits in ar.ar_last_kernels()
     else:
@@ -217,4 +219,78 @@ def test_w2a16_decode_full_size_sampled_rows(ar, T):
     assert np.array_equal(packed.cpu().numpy().view(np.uint32)[rows], words)
     ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16)[rows],
                          z16.cpu().numpy().view(np.uint16)[rows], g, 2)
+    assert rel_l2(out.float().cpu().numpy()[:, rows], ref) <= TC_RTOL
+
+
+@pytest.mark.parametrize("T", [1, 5, 8])
+@pytest.mark.parametrize("N,K,g,tag", [
+    (10000, 512, 64, "g=64,nt8>"),              # 72 rows per CTA: two row passes (64 + 8); last CTA one pass
+    (10000, 1024, 128, "g>=128,nt8>"),          # the same passes with one group per 128-k quarter
+    (4096, 2048, 128, "g>=128,ksplit2,nt7>"),   # 56-row CTA pairs splitting K
+    (296, 4096, 256, "g>=128,ksplit2,nt1>"),    # 8-row CTA pairs
+    (1000, 1280, 32, "g=32,nt8>"),              # the last 512-k stage half empty; 16-group windows
+    (1001, 1024, 128, "g>=128,nt1>"),           # the last CTA holds one row
+])
+def test_w8a16_decode_row_ranges_match_oracle(ar, T, N, K, g, tag):
+    """8-bit codes up to 8 tokens on the W4A16 decode kernel's 8-bit form (each code split into its
+    two nibbles, the high one taken at mantissa bits 3-6 against doubled activations)."""
+    d = synth.make_linear(N, K, 1, seed=T + N + 8)
+    V, a, b = synth.make_state(N, K, g, seed=2, spread=True)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 8, g)
+    A = synth.make_activations(T, K, seed=T)
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 8, out)
+    assert ar.ar_get_device_status() == 0
+    kern = ar.ar_last_kernels()
+    assert "w8a16_dec_kernel<T<=8,%s" % tag in kern, kern
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 8, g)
+    words = O.pack_bitstream(st["q"], 8)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16),
+                         z16.cpu().numpy().view(np.uint16), g, 8)
+    got = out.float().cpu().numpy()
+    assert rel_l2(got, ref) <= TC_RTOL
+    for t in range(T):
+        assert rel_l2(got[t], ref[t]) <= TC_RTOL
+    assert rel_l2(got[:, :8], ref[:, :8]) <= TC_RTOL and rel_l2(got[:, -8:], ref[:, -8:]) <= TC_RTOL
+
+
+def test_w8a16_decode_extreme_codes(ar):
+    """Codes 0, 255, 0x0F and 0xF0 (each nibble at its extremes) against the oracle."""
+    N, K, g, T = 64, 1024, 128, 3
+    words = np.zeros((N, K // 4), np.uint32)
+    words[1::4] = 0xFFFFFFFF
+    words[2::4] = 0x0F0F0F0F
+    words[3::4] = 0xF0F0F0F0
+    s16 = np.full((N, K // g), 0.0123, np.float16)
+    z16 = np.tile(np.array([0.0, 17.0, 128.0, 255.0], np.float16), (N, K // g // 4))
+    A = synth.make_activations(T, K, seed=6)
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), torch.from_numpy(words.view(np.int32)).cuda(), torch.from_numpy(s16).cuda(),
+                     torch.from_numpy(z16).cuda(), g, 8, out)
+    assert ar.ar_get_device_status() == 0
+    assert "w8a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.view(np.uint16), z16.view(np.uint16), g, 8)
+    assert rel_l2(out.float().cpu().numpy(), ref) <= TC_RTOL
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_w8a16_decode_full_size_sampled_rows(ar, T):
+    """8192 x 28672 down projection at 8 bits (g 128) on the decode kernel, sampled output rows
+    against the oracle."""
+    wl = synth.WORKLOADS["down_8192_28672"]
+    N, K, g = wl.n_out, wl.n_in, wl.group_size
+    d = synth.make_linear(N, K, 1, seed=wl.seed, x_outlier_channels=0)
+    V, a, b = synth.make_state(N, K, g)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 8, g)
+    A = synth.make_activations(T, K, seed=1)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 8, out)
+    assert ar.ar_get_device_status() == 0
+    assert "w8a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    rows = np.sort(np.random.default_rng(7).choice(N, 64, replace=False))
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"][rows]), V[rows], a[rows], b[rows], 8, g)
+    words = O.pack_bitstream(st["q"], 8)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32)[rows], words)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16)[rows],
+                         z16.cpu().numpy().view(np.uint16)[rows], g, 8)
     assert rel_l2(out.float().cpu().numpy()[:, rows], ref) <= TC_RTOL
