@@ -728,7 +728,7 @@ def run_case(name, ar, torch):
         ws = torch.empty(ar.ar_tune_step_workspace(W, V, a, b, M, cfg, 2), dtype=torch.uint8, device=dev)
         loss = torch.empty(2, device=dev)
         fn = lambda: ar.ar_tune_step(W, V, a, b, X, Y, cfg, 2, loss, ws)
-    elif name in ("w4a16_t1", "w2a16_t1", "w3a16_t256", "nvfp4_gemm_t1", "nvfp4_gemm_t256"):  # the 8192 x 28672 layer's exports
+    elif name in ("w4a16_t1", "w2a16_t1", "w8a16_t1", "w3a16_t256", "nvfp4_gemm_t1", "nvfp4_gemm_t256"):  # the 8192 x 28672 layer's exports
         N, K, g = 8192, 28672, 128
         d = synth.make_linear(N, K, 1, seed=5, x_outlier_channels=0)
         W = to_dev_bf16(d["W"], torch)
@@ -736,8 +736,8 @@ def run_case(name, ar, torch):
         T = 256 if name.endswith("t256") else 1
         A = to_dev_bf16(synth.make_activations(T, K, seed=T), torch)
         y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
-        if name in ("w3a16_t256", "w2a16_t1"):
-            bits = 3 if name == "w3a16_t256" else 2
+        if name in ("w3a16_t256", "w2a16_t1", "w8a16_t1"):
+            bits = {"w3a16_t256": 3, "w2a16_t1": 2, "w8a16_t1": 8}[name]
             V = torch.zeros((N, K), device=dev)
             a = torch.ones((N, K // g), device=dev)
             pk = torch.empty((N, K * bits // 32), dtype=torch.int32, device=dev)
@@ -777,7 +777,7 @@ def run_case(name, ar, torch):
 
 
 CASES = ("qdq", "pack_int4", "qdq_nvfp4", "absmax", "tune_nvfp4", "mlp", "decoder", "lowbit_b2g32", "w4a16_t1",
-         "w2a16_t1", "w3a16_t256", "nvfp4_gemm_t1", "nvfp4_gemm_t256")
+         "w2a16_t1", "w8a16_t1", "w3a16_t256", "nvfp4_gemm_t1", "nvfp4_gemm_t256")
 
 
 def main():
