@@ -53,11 +53,12 @@
 // bits 4*(k mod 8) of word k/8; scale/zero fp16 [N][K/g].
 //
 // The same kernel takes 2-bit codes (ar_pack_codes' stream: element k at bits
-// 2*(k mod 16) of word k/16) up to 8 tokens for g >= 64.  A stage is always
-// 1024 k (two 128-byte boxes per row), and a lane's 32-bit word holds 16 codes,
-// so a warp's 256-k quarter is four 64-k slices of four MMAs each (weights as
-// the A operand).  The
-// codes are not shifted down one by one: (x & (3 << 2m)) | 0x4300 for
+// 2*(k mod 16) of word k/16) up to 8 tokens for g >= 64.  A stage is 1024 k
+// (two 128-byte boxes per row), or 2048 k for one token at g >= 128 where four
+// such stages fit (30.8 against 32.8 us on the 8192 x 28672 layer), and a
+// lane's 32-bit word holds 16 codes, so a warp's quarter of a stage is 64-k
+// slices of four MMAs each (weights as the A operand).  The codes are not
+// shifted down one by one: (x & (3 << 2m)) | 0x4300 for
 // m = 0, 1, 2 is the bf16 128 + 4^m q, since bits 0..6 are the mantissa of a
 // bf16 in [128, 256), so one word needs two shifts (by 6 and 12) and eight
 // logic ops to give its eight pairs (q_i, q_{i+8}).  The activation paired
