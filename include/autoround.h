@@ -376,10 +376,10 @@ AR_API ar_status ar_pack_codes(const uint16_t* W, const float* V, const float* a
 /* WbA16 matmul for codes packed by ar_pack_codes (bits 2, 3, 4 or 8):
  *   out[t][n] = sum_k A[t][k] (q[n][k] - zero[n][k/g]) scale[n][k/g]
  * A bf16 [T][K]; zero must hold integers 0..2^bits-1; out bf16 [T][N].  bits 4
- * is ar_w4a16_gemm.  At T <= 8 with K/group_size a multiple of 8, 2 bits
- * (group_size >= 64, K >= 512) and 8 bits run the W4A16 decode kernel's 2-bit
- * and 8-bit forms (codes taken at mantissa positions of a bf16 with the paired
- * activations scaled to match; an 8-bit code as its two nibbles); other 2 and
+ * is ar_w4a16_gemm.  At T <= 8 with K/group_size a multiple of 8, 2 and 3
+ * bits (group_size >= 64, K >= 512) and 8 bits run the W4A16 decode kernel's
+ * 2, 3 and 8-bit forms (codes taken at mantissa positions of a bf16 with the
+ * paired activations scaled to match; an 8-bit code as its two nibbles); other 2 and
  * 3-bit shapes at T <= 8 run a generic decode kernel (mma.sync, one range of
  * weight rows per SM, the codes read straight from the bit stream); the rest,
  * and every width from 9 tokens, run the tcgen05 dequant

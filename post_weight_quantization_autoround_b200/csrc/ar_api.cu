@@ -896,9 +896,9 @@ ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
     if (!p) return fail(AR_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned16(p)) return fail(AR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   }
-  // Up to 8 tokens with K/g a multiple of 8: the W4A16 decode kernel's 2-bit (g >= 64) and
-  // 8-bit forms (measured on 8192 x 28672, T = 1: 30.7 and 59.4 us against 79.7 us on the
-  // generic decode kernel and 90 us on the tcgen05 GEMM); other 2 and 3-bit shapes up to 8
+  // Up to 8 tokens with K/g a multiple of 8: the W4A16 decode kernel's 2-bit, 3-bit (g >= 64)
+  // and 8-bit forms (measured on 8192 x 28672, T = 1: 30.7, 38.9 and 59.4 us against 79.7 and
+  // 79.9 us on the generic decode kernel and 90 us on the tcgen05 GEMM); other 2 and 3-bit shapes up to 8
   // tokens: the generic mma.sync decode kernel (80 us at T <= 8 against 88-90 us for the GEMM,
   // but 90-96 us at T = 16); the rest, and everything from 9 tokens: the tcgen05 dequant GEMM
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -907,6 +907,7 @@ ar_status ar_wxa16_gemm(const uint16_t* A, int64_t T, const uint32_t* packed, co
   // cudaErrorNotSupported comes from shape checks before any CUDA call: nothing to clear
   if (bits == 2 && T <= 8) e = launch_w2a16_dec(A, t, packed, scale_f16, zero_f16, n, k, group_size, out, s);
   if (bits == 8 && T <= 8) e = launch_w8a16_dec(A, t, packed, scale_f16, zero_f16, n, k, group_size, out, s);
+  if (bits == 3 && T <= 8) e = launch_w3a16_dec(A, t, packed, scale_f16, zero_f16, n, k, group_size, out, s);
   if (e == cudaErrorNotSupported)
     e = ((bits == 2 || bits == 3) && T <= 8)
             ? launch_wbx_dec(A, t, packed, scale_f16, zero_f16, n, k, group_size, bits, out, s)

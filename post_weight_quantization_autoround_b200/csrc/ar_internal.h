@@ -179,6 +179,10 @@ cudaError_t launch_w2a16_dec(const uint16_t* A, int T, const uint32_t* packed, c
 cudaError_t launch_w8a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
                              const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
                              cudaStream_t stream);
+// ... and on 3-bit codes (ar_pack_codes' 32-codes-in-3-words stream): T <= 8, g >= 64, K >= 512
+cudaError_t launch_w3a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
+                             cudaStream_t stream);
 // NVFP4 QDQ (ar_nvfp4.cu): absmax into a zeroed device scalar, then the block QDQ
 cudaError_t launch_absmax_bf16(const uint16_t* x, int64_t n, float* amax, cudaStream_t stream);
 cudaError_t launch_qdq_nvfp4(const uint16_t* W, const float* V, const float* alpha, int64_t n, const float* amax,

@@ -73,6 +73,12 @@
 // ((x >> 1) & 0x00780078) | 0x4300, the high nibbles at mantissa bits 3..6, is
 // (128 + 8 hi_0, 128 + 8 hi_2), paired with doubled activations; a code then
 // contributes 384 a + q a, and a group adds s D - s (384 + z) O.
+//
+// 3-bit codes (T <= 8, g >= 64; 1024-k stages, three boxes per row): a lane's
+// 16 codes are 6 bytes of the bit stream, read as the two aligned words that
+// hold them and funnel-shifted into place; two byte permutes put codes 0..7
+// and 8..15 side by side, and masks at mantissa bits 0-2 and 3-5 give the
+// pairs at scales 1 and 8, corrected as at 2 bits.
 #include <cooperative_groups.h>
 
 #include <cstdio>
@@ -183,6 +189,26 @@ __device__ __forceinline__ void two_bit_pairs(uint32_t x, uint32_t (&r)[8]) {
   r[7] = mask_pair<0x000C000Cu>(z);
 }
 
+// The eight bf16 pairs of 16 consecutive 3-bit codes that start at bit `sh` (0 or 16) of the
+// 64-bit value (w1:w0): r[i] = (128 + s_i q_i, 128 + s_i q_{i+8}) with s = (1, 8, 1, 8, ...).
+// u holds codes 0..7 at bits 3i, v codes 8..15; a byte permute puts the low 16 bits of each side
+// by side, so each half carries codes at bits 0-2 and 3-5, both inside a bf16 mantissa.
+__device__ __forceinline__ void three_bit_pairs(uint32_t w0, uint32_t w1, uint32_t sh, uint32_t (&r)[8]) {
+  const uint32_t u = __funnelshift_r(w0, w1, sh);
+  const uint32_t v = __funnelshift_r(u, shr(w1, sh), 24);
+  const uint32_t a = __byte_perm(u, v, 0x5410);                    // codes 0, 1 | 8, 9 (+ 2, 3 | 10, 11 above)
+  const uint32_t b = __byte_perm(shr(u, 12), shr(v, 12), 0x5410);  // codes 4, 5 | 12, 13 (+ 6, 7 | 14, 15)
+  const uint32_t a6 = shr(a, 6), b6 = shr(b, 6);
+  r[0] = mask_pair<0x00070007u>(a);
+  r[1] = mask_pair<0x00380038u>(a);
+  r[2] = mask_pair<0x00070007u>(a6);
+  r[3] = mask_pair<0x00380038u>(a6);
+  r[4] = mask_pair<0x00070007u>(b);
+  r[5] = mask_pair<0x00380038u>(b);
+  r[6] = mask_pair<0x00070007u>(b6);
+  r[7] = mask_pair<0x00380038u>(b6);
+}
+
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -209,12 +235,14 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                      const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmZl,
                      const __grid_constant__ CUtensorMap tmA, const DecParams p, uint16_t* __restrict__ out) {
   using C = DecCfg<TBIG>;
-  static_assert(BITS == 4 || ((BITS == 2 || BITS == 8) && !TBIG), "4-bit codes, or 2/8-bit codes up to 8 tokens");
+  static_assert(BITS == 4 || ((BITS == 2 || BITS == 3 || BITS == 8) && !TBIG),
+                "4-bit codes, or 2, 3 or 8-bit codes up to 8 tokens");
   // k per stage (512 or 1024; 2-bit codes: 1024); a stage holds kStageK * BITS / 1024 128-byte
   // boxes of codes per row, contiguous in the row
   constexpr int kStageK = STAGEK;
   static_assert(BITS == 4   ? (kStageK == 512 || kStageK == 1024)
                 : BITS == 2 ? (kStageK == 1024 || kStageK == 2048)
+                : BITS == 3 ? kStageK == 1024
                             : kStageK == 512,
                 "stage size");
   constexpr int kCodeBoxes = kStageK * BITS / 1024;
@@ -408,6 +436,106 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
                     const float2 mh = smw[16 * mt + 8 + g];
                     acc[mt][2] = fmaf(mh.x, d[mt][2], fmaf(mh.y, o[2], acc[mt][2]));
                     acc[mt][3] = fmaf(mh.x, d[mt][3], fmaf(mh.y, o[3], acc[mt][3]));
+                  }
+                }
+              }
+            }
+          } else if constexpr (BITS == 3) {
+            // weights as the A operand as below.  A row's 1024-k stage is 384 bytes (three boxes);
+            // warp cw takes its bytes 96 cw .. 96 cw + 95.  Per 64-k slice j (24 bytes) lane c takes
+            // the 16 codes at bytes 24 j + 6 c .. + 5 of that range (k = 64 j + 16 c + 0..15), read as
+            // the two aligned words that hold them; pair i of the lane (codes i, i + 8) feeds k-slots
+            // (2c, 2c+1) of MMA i/2 when i is even, (2c+8, 2c+9) when odd, as at 2 bits
+            float d[MT][4], o[4];
+            const uint8_t* row3 = st + g * 128;
+            const uint8_t* act3 = st + p.act_off + 16 * c * 2;
+            constexpr uint32_t kEighth2 = 0x3E003E00u;  // bf16 pair (1/8, 1/8)
+            constexpr uint32_t kEight2 = 0x41004100u;   // (8, 8)
+#pragma unroll
+            for (int j = 0; j < kStageK / 256; ++j) {
+              const int kj = kw0 + 64 * j;
+              const uint8_t* aj = act3 + (kj >> 8) * 512 * T + (kj & 255) * 2 + tok_lo * 512;
+              const uint4 v = *reinterpret_cast<const uint4*>(aj);
+              const uint4 u = *reinterpret_cast<const uint4*>(aj + 16);
+              uint32_t b[8];
+              b[0] = __byte_perm(v.x, u.x, 0x5410);
+              b[1] = bf16x2_mul(__byte_perm(v.x, u.x, 0x7632), kEighth2);
+              b[2] = __byte_perm(v.y, u.y, 0x5410);
+              b[3] = bf16x2_mul(__byte_perm(v.y, u.y, 0x7632), kEighth2);
+              b[4] = __byte_perm(v.z, u.z, 0x5410);
+              b[5] = bf16x2_mul(__byte_perm(v.z, u.z, 0x7632), kEighth2);
+              b[6] = __byte_perm(v.w, u.w, 0x5410);
+              b[7] = bf16x2_mul(__byte_perm(v.w, u.w, 0x7632), kEighth2);
+              const bool first = (j % SPAN) == 0;
+              {
+                // rows 0..7: Oa = sum of a (class weights 1, 8); rows 8..15: Ob = sum of the scaled a
+                const uint32_t c0[4] = {kOne2, kOne2, kEight2, kOne2};
+                if (first) {
+                  mma16816_z(o, c0, b[0], b[1]);
+                } else {
+                  mma16816(o, c0, b[0], b[1]);
+                }
+                mma16816(o, c0, b[2], b[3]);
+                mma16816(o, c0, b[4], b[5]);
+                mma16816(o, c0, b[6], b[7]);
+              }
+              // the lane's two aligned words: byte x of the row segment is in box x / 128, 16-byte
+              // chunk (x % 128) / 16 stored at chunk ((x % 128) / 16) ^ (row % 8)
+              const int x = ((kw0 * 3) >> 3) + 24 * j + 6 * c;
+              const int x0w = x & ~3, x1w = x0w + 4;
+              const int off0 = (x0w >> 7) * kDecCodeBox + ((((x0w & 127) >> 4) ^ g) << 4) + (x0w & 15);
+              const int off1 = (x1w >> 7) * kDecCodeBox + ((((x1w & 127) >> 4) ^ g) << 4) + (x1w & 15);
+              const uint32_t sh = static_cast<uint32_t>(x & 3) * 8u;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                const bool pair = 2 * mt + 1 < NT;
+                const uint8_t* rg = row3 + (2 * mt) * 8 * 128;
+                uint32_t qg[8], qh[8];
+                three_bit_pairs(*reinterpret_cast<const uint32_t*>(rg + off0),
+                                *reinterpret_cast<const uint32_t*>(rg + off1), sh, qg);
+                if (pair) {
+                  const uint8_t* rh = rg + 8 * 128;
+                  three_bit_pairs(*reinterpret_cast<const uint32_t*>(rh + off0),
+                                  *reinterpret_cast<const uint32_t*>(rh + off1), sh, qh);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) qh[i] = 0u;
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                  const uint32_t a[4] = {qg[2 * m], qh[2 * m], qg[2 * m + 1], qh[2 * m + 1]};
+                  if (first && m == 0) {
+                    mma16816_z(d[mt], a, b[0], b[1]);
+                  } else {
+                    mma16816(d[mt], a, b[2 * m], b[2 * m + 1]);
+                  }
+                }
+              }
+              if ((j % SPAN) == SPAN - 1) {
+                // group span done: acc += s (D - 128 Ob) - s z Oa, as at 2 bits
+                const int gl = ((ks * kStageK + kw0 + 64 * (j - SPAN + 1)) >> p.group_shift) - x0;
+                __syncwarp();
+#pragma unroll
+                for (int rr = 0; rr < (8 * NT + 31) / 32; ++rr) {
+                  const int row = lane + 32 * rr;
+                  if (row < 8 * NT) {
+                    const float sv = half_bits_to_float(sc[row * p.wg + gl]);
+                    const float zv = half_bits_to_float(zr[row * p.wg + gl]);
+                    smw[row] = make_float2(sv, -sv * zv);
+                  }
+                }
+                __syncwarp();
+                const float ob0 = -128.0f * o[2];
+                const float ob1 = -128.0f * o[3];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                  const float2 mg = smw[16 * mt + g];
+                  acc[mt][0] = fmaf(mg.x, d[mt][0] + ob0, fmaf(mg.y, o[0], acc[mt][0]));
+                  acc[mt][1] = fmaf(mg.x, d[mt][1] + ob1, fmaf(mg.y, o[1], acc[mt][1]));
+                  if (2 * mt + 1 < NT) {
+                    const float2 mh = smw[16 * mt + 8 + g];
+                    acc[mt][2] = fmaf(mh.x, d[mt][2] + ob0, fmaf(mh.y, o[0], acc[mt][2]));
+                    acc[mt][3] = fmaf(mh.x, d[mt][3] + ob1, fmaf(mh.y, o[1], acc[mt][3]));
                   }
                 }
               }
@@ -736,19 +864,19 @@ __global__ void __maxnreg__(DecCfg<TBIG>::kMaxRegs)
 // group-size class: 0 for g >= 128, 1 for g = 64, 2 for g = 32
 template <int BITS, int SPAN>
 constexpr int dec_gclass() {
-  return BITS == 4   ? (SPAN == 4 ? 0 : (SPAN == 2 ? 1 : 2))
-         : BITS == 2 ? (SPAN == 2 ? 0 : 1)
-                     : (SPAN == 8 ? 0 : (SPAN == 4 ? 1 : 2));
+  return BITS == 4                 ? (SPAN == 4 ? 0 : (SPAN == 2 ? 1 : 2))
+         : (BITS == 2 || BITS == 3) ? (SPAN == 2 ? 0 : 1)
+                                    : (SPAN == 8 ? 0 : (SPAN == 4 ? 1 : 2));
 }
 
 const char* dec_name(int bits, bool tbig, int gclass, int ks, int nt) {
   // "w4a16_dec_kernel<T<=8,g>=128,nt7>", "...,ksplit2,nt7>", "w2a16_dec_kernel<T<=8,g=64,nt8>";
   // built once, kept for the process
-  static char names[3][2][3][2][9][64];
+  static char names[4][2][3][2][9][64];
   static const bool filled = [] {
     const char* gs[3] = {"g>=128", "g=64", "g=32"};
-    const int widths[3] = {4, 2, 8};
-    for (int w = 0; w < 3; ++w)
+    const int widths[4] = {4, 2, 8, 3};
+    for (int w = 0; w < 4; ++w)
       for (int a = 0; a < 2; ++a)
         for (int b = 0; b < 3; ++b)
           for (int c = 0; c < 2; ++c)
@@ -758,7 +886,7 @@ const char* dec_name(int bits, bool tbig, int gclass, int ks, int nt) {
     return true;
   }();
   (void)filled;
-  return names[bits == 2 ? 1 : (bits == 8 ? 2 : 0)][tbig ? 1 : 0][gclass][ks - 1][nt];
+  return names[bits == 2 ? 1 : (bits == 8 ? 2 : (bits == 3 ? 3 : 0))][tbig ? 1 : 0][gclass][ks - 1][nt];
 }
 
 template <bool TBIG, int SPAN, int KS, int NT, int BITS, int STAGEK>
@@ -851,6 +979,17 @@ cudaError_t launch_dec8_span(int span, int ks, int nt, const CUtensorMap (&maps)
   return launch_dec_nt<false, 2, 1, 8, 512>(nt, maps, p, grid, smem, out, stream);
 }
 
+// 3-bit codes, T <= 8, 1024-k stages: span 2 (g >= 128) or 1 (g = 64)
+cudaError_t launch_dec3_span(int span, int ks, int nt, const CUtensorMap (&maps)[7], const DecParams& p, int grid,
+                             int smem, uint16_t* out, cudaStream_t stream) {
+  if (ks == 2) {
+    if (span == 2) return launch_dec_nt<false, 2, 2, 3, 1024>(nt, maps, p, grid, smem, out, stream);
+    return launch_dec_nt<false, 1, 2, 3, 1024>(nt, maps, p, grid, smem, out, stream);
+  }
+  if (span == 2) return launch_dec_nt<false, 2, 1, 3, 1024>(nt, maps, p, grid, smem, out, stream);
+  return launch_dec_nt<false, 1, 1, 3, 1024>(nt, maps, p, grid, smem, out, stream);
+}
+
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Returns cudaErrorNotSupported (nothing launched) when the shape does not fit
@@ -863,8 +1002,9 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
                             cudaStream_t stream) {
   if (T < 1 || T > 16 || N < 1 || K < 128 || K % 128 != 0 || group_size < 32) return cudaErrorNotSupported;
   if (bits == 2 && (T > 8 || group_size < 64 || K < kDecStageK)) return cudaErrorNotSupported;
+  if (bits == 3 && (T > 8 || group_size < 64 || K < kDecStageK)) return cudaErrorNotSupported;
   if (bits == 8 && T > 8) return cudaErrorNotSupported;
-  if (bits != 2 && bits != 4 && bits != 8) return cudaErrorNotSupported;
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return cudaErrorNotSupported;
   const int G = K / group_size;
   if (G % 8 != 0 || (reinterpret_cast<uintptr_t>(scale16) & 15u) || (reinterpret_cast<uintptr_t>(zero16) & 15u))
     return cudaErrorNotSupported;
@@ -929,7 +1069,7 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
   const int heights[2] = {std::min(kDecPassRows, rows), p.last_rows};
   for (int m = 0; m < 2; ++m) {
     e = make_tmap_2d(&maps[m], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, static_cast<uint64_t>(N),
-                     static_cast<uint64_t>(K / (32 / bits)), 32, static_cast<uint32_t>(heights[m]),
+                     static_cast<uint64_t>(K) * bits / 32, 32, static_cast<uint32_t>(heights[m]),
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     e = make_tmap_2d(&maps[2 + m], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scale16, static_cast<uint64_t>(N),
@@ -947,6 +1087,7 @@ cudaError_t launch_dec_bits(const uint16_t* A, int T, const uint32_t* packed, co
 
   const int nt = p.passes == 1 ? rows / 8 : 8;  // tiles of a full pass
   if (bits == 8) return launch_dec8_span(std::min(8, group_size / 16), ks, nt, maps, p, grid, smem, out, stream);
+  if (bits == 3) return launch_dec3_span(group_size >= 128 ? 2 : 1, ks, nt, maps, p, grid, smem, out, stream);
   if (bits == 2) {
     const int span2 = group_size >= 128 ? 2 : 1;
     return stage_k == 2048 ? launch_dec2_span<2048>(span2, ks, nt, maps, p, grid, smem, out, stream)
@@ -976,6 +1117,12 @@ cudaError_t launch_w8a16_dec(const uint16_t* A, int T, const uint32_t* packed, c
                              const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
                              cudaStream_t stream) {
   return launch_dec_bits(A, T, packed, scale16, zero16, N, K, group_size, 8, out, stream);
+}
+
+cudaError_t launch_w3a16_dec(const uint16_t* A, int T, const uint32_t* packed, const uint16_t* scale16,
+                             const uint16_t* zero16, int N, int K, int group_size, uint16_t* out,
+                             cudaStream_t stream) {
+  return launch_dec_bits(A, T, packed, scale16, zero16, N, K, group_size, 3, out, stream);
 }
 
 }  // namespace ar

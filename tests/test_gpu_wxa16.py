@@ -73,8 +73,8 @@ def test_wxa16_matches_oracle(ar, bits, T, N, K, g):
     out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, bits, out)
     assert ar.ar_get_device_status() == 0
-    if bits == 2 and T <= 8 and g >= 64 and (K // g) % 8 == 0:
-        assert "w2a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    if bits in (2, 3) and T <= 8 and g >= 64 and (K // g) % 8 == 0:
+        assert "w%da16_dec_kernel<T<=8" % bits in ar.ar_last_kernels()
     elif bits == 8 and T <= 8 and (K // g) % 8 == 0:
         assert "w8a16_dec_kernel<T<=8" in ar.ar_last_kernels()
     elif bits in (2, 3) and T <= 8:
@@ -293,4 +293,75 @@ def test_w8a16_decode_full_size_sampled_rows(ar, T):
     assert np.array_equal(packed.cpu().numpy().view(np.uint32)[rows], words)
     ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16)[rows],
                          z16.cpu().numpy().view(np.uint16)[rows], g, 8)
+    assert rel_l2(out.float().cpu().numpy()[:, rows], ref) <= TC_RTOL
+
+
+@pytest.mark.parametrize("T", [1, 5, 8])
+@pytest.mark.parametrize("N,K,g,tag", [
+    (10000, 512, 64, "g=64,nt8>"),              # 72 rows per CTA: two row passes; one half-empty 1024-k stage
+    (10000, 1024, 128, "g>=128,nt8>"),          # the same passes with one group per 128 k
+    (4096, 2048, 128, "g>=128,ksplit2,nt7>"),   # 56-row CTA pairs splitting K
+    (296, 4096, 256, "g>=128,ksplit2,nt1>"),    # 8-row CTA pairs
+    (1001, 1024, 128, "g>=128,nt1>"),           # the last CTA holds one row
+])
+def test_w3a16_decode_row_ranges_match_oracle(ar, T, N, K, g, tag):
+    """3-bit codes up to 8 tokens on the W4A16 decode kernel's 3-bit form (a lane's 16 codes read as
+    the two aligned words that hold them, codes taken at mantissa bits 0-2 and 3-5)."""
+    d = synth.make_linear(N, K, 1, seed=T + N + 3)
+    V, a, b = synth.make_state(N, K, g, seed=2, spread=True)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 3, g)
+    A = synth.make_activations(T, K, seed=T)
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 3, out)
+    assert ar.ar_get_device_status() == 0
+    kern = ar.ar_last_kernels()
+    assert "w3a16_dec_kernel<T<=8,%s" % tag in kern, kern
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"]), V, a, b, 3, g)
+    words = O.pack_bitstream(st["q"], 3)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16),
+                         z16.cpu().numpy().view(np.uint16), g, 3)
+    got = out.float().cpu().numpy()
+    assert rel_l2(got, ref) <= TC_RTOL
+    for t in range(T):
+        assert rel_l2(got[t], ref[t]) <= TC_RTOL
+    assert rel_l2(got[:, :8], ref[:, :8]) <= TC_RTOL and rel_l2(got[:, -8:], ref[:, -8:]) <= TC_RTOL
+
+
+def test_w3a16_decode_extreme_codes(ar):
+    """All-zero and all-seven code rows (every code, straddling ones included, at its extremes)."""
+    N, K, g, T = 64, 1024, 128, 3
+    words = np.zeros((N, K * 3 // 32), np.uint32)
+    words[1::2] = 0xFFFFFFFF
+    s16 = np.full((N, K // g), 0.0123, np.float16)
+    z16 = np.tile(np.array([0.0, 3.0, 4.0, 7.0], np.float16), (N, K // g // 4))
+    A = synth.make_activations(T, K, seed=7)
+    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), torch.from_numpy(words.view(np.int32)).cuda(), torch.from_numpy(s16).cuda(),
+                     torch.from_numpy(z16).cuda(), g, 3, out)
+    assert ar.ar_get_device_status() == 0
+    assert "w3a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.view(np.uint16), z16.view(np.uint16), g, 3)
+    assert rel_l2(out.float().cpu().numpy(), ref) <= TC_RTOL
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_w3a16_decode_full_size_sampled_rows(ar, T):
+    """8192 x 28672 down projection at 3 bits (g 128) on the decode kernel, sampled output rows
+    against the oracle."""
+    wl = synth.WORKLOADS["down_8192_28672"]
+    N, K, g = wl.n_out, wl.n_in, wl.group_size
+    d = synth.make_linear(N, K, 1, seed=wl.seed, x_outlier_channels=0)
+    V, a, b = synth.make_state(N, K, g)
+    packed, s16, z16 = pack_gpu(ar, d["W"], V, a, b, 3, g)
+    A = synth.make_activations(T, K, seed=1)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    ar.ar_wxa16_gemm(bf16_dev(A), packed, s16, z16, g, 3, out)
+    assert ar.ar_get_device_status() == 0
+    assert "w3a16_dec_kernel<T<=8" in ar.ar_last_kernels()
+    rows = np.sort(np.random.default_rng(7).choice(N, 64, replace=False))
+    st = O.qdq(synth.bf16_bits_to_f32(d["W"][rows]), V[rows], a[rows], b[rows], 3, g)
+    words = O.pack_bitstream(st["q"], 3)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32)[rows], words)
+    ref = O.wxa16_matmul(synth.bf16_bits_to_f32(A), words, s16.cpu().numpy().view(np.uint16)[rows],
+                         z16.cpu().numpy().view(np.uint16)[rows], g, 3)
     assert rel_l2(out.float().cpu().numpy()[:, rows], ref) <= TC_RTOL
